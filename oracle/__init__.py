@@ -1,0 +1,269 @@
+"""fp64 CPU oracle for the SeerAttention prefill path (test infrastructure).
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+may import this package.  The product path (the CUDA library and its Python
+binding) never does, and this package never imports the product.
+
+The arithmetic lives in ``seer_oracle.c`` (plain C, fp64, OpenMP); this module
+compiles it with gcc and marshals numpy arrays.  Every entry point names the
+passage of "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs"
+it follows (paper-graph summary page, section 3.4; OpenReview rebuttal,
+section 3.3).
+
+Parity status: block RoPE's base reading (theta' = theta / B) is "parity
+unpinned"; every other function is pinned by the CPU tests.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "seer_oracle.c")
+_LIB = os.path.join(_HERE, "libseer_oracle.so")
+BLOCK = 64
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into oracle/libseer_oracle.so (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int64
+        D = ctypes.c_double
+        F = ctypes.c_float
+        lib.orc_pool_q.argtypes = [P, I, I, I, I, P]
+        lib.orc_pool_k.argtypes = [P, I, I, I, I, P]
+        lib.orc_project.argtypes = [P, P, I, I, I, I, I, P]
+        lib.orc_block_rope.argtypes = [P, I, I, I, D, I]
+        lib.orc_gate_scores.argtypes = [P, P, I, I, I, I, I, D, P]
+        lib.orc_select_threshold.argtypes = [P, I, I, F, P, P, I]
+        lib.orc_select_threshold.restype = I
+        lib.orc_select_topk.argtypes = [P, I, I, ctypes.c_int, I, F, P, P, I]
+        lib.orc_select_topk.restype = I
+        lib.orc_topk_count.argtypes = [I, ctypes.c_int, I, F]
+        lib.orc_topk_count.restype = I
+        lib.orc_sparse_attn_units.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, D, P, I, P, P]
+        lib.orc_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, I, P, P, I, D, P, P]
+        lib.orc_blockmax_units.argtypes = [P, P, I, I, I, I, I, I, D, P, I, P, P]
+        lib.orc_blockmax.argtypes = [P, P, I, I, I, I, I, I, D, P, P]
+        lib.orc_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f32(x) -> np.ndarray:
+    """Contiguous fp32 numpy view of a tensor/array (bf16 is upcast exactly)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu")
+            if x.dtype != torch.float32:
+                x = x.to(torch.float32)
+            return np.ascontiguousarray(x.numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _f64(x) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu").to(torch.float64)
+            return np.ascontiguousarray(x.numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+# ---------------------------------------------------------------- gate ---
+def pool_q(Q) -> np.ndarray:
+    """Average pooling of Q per 64-token block (summary page, section 3.4,
+    "Input and pooling").  Q [B,H,n,d] -> [B,H,nb,d] fp64."""
+    q = _f32(Q)
+    B, H, n, d = q.shape
+    out = np.empty((B, H, n // BLOCK, d), np.float64)
+    _load().orc_pool_q(_p(q), B * H, n, d, BLOCK, _p(out))
+    return out
+
+
+def pool_k(K) -> np.ndarray:
+    """Max, min and average pooling of K concatenated as [max|min|avg]
+    (summary page, section 3.4, "Pooling Method Selection").
+    K [B,H,n,d] -> [B,H,nb,3d] fp64."""
+    k = _f32(K)
+    B, H, n, d = k.shape
+    out = np.empty((B, H, n // BLOCK, 3 * d), np.float64)
+    _load().orc_pool_k(_p(k), B * H, n, d, BLOCK, _p(out))
+    return out
+
+
+def project(x, W) -> np.ndarray:
+    """Gate linear layer, no bias (summary page, section 3.4, "Linear
+    transformation"): y[b,hh,i] = W[hh] @ x[b,hh,i].  W is [H, h, din]."""
+    xv = _f64(x)
+    w = _f32(W)
+    B, H, nb, din = xv.shape
+    h = w.shape[1]
+    assert w.shape == (H, h, din)
+    out = np.empty((B, H, nb, h), np.float64)
+    _load().orc_project(_p(xv), _p(w), B, H, nb, din, h, _p(out))
+    return out
+
+
+def block_rope(x, theta: float) -> np.ndarray:
+    """Block-level RoPE with base theta / 64 at block positions (summary page,
+    section 3.4, "Block-Level RoPE").  Parity unpinned for the base reading."""
+    xv = _f64(x).copy()
+    B, H, nb, h = xv.shape
+    _load().orc_block_rope(_p(xv), B * H, nb, h, float(theta), BLOCK)
+    return xv
+
+
+def gate_scores(qt, kt, d: int) -> np.ndarray:
+    """Eq. 1 (summary page, section 3.4): causal row softmax of
+    q~ k~^T / sqrt(d) over key blocks j <= i; 0 above the diagonal."""
+    q = _f64(qt)
+    k = _f64(kt)
+    B, Hq, nb, h = q.shape
+    Hkv = k.shape[1]
+    out = np.empty((B, Hq, nb, nb), np.float64)
+    _load().orc_gate_scores(_p(q), _p(k), B, Hq, Hkv, nb, h, 1.0 / math.sqrt(d), _p(out))
+    return out
+
+
+def gate(Q, K, Wq, Wk, rope_theta: float = 0.0) -> np.ndarray:
+    """The whole AttnGate (pool, project, optional block RoPE, Eq. 1)."""
+    d = Q.shape[-1]
+    qt = project(pool_q(Q), Wq)
+    kt = project(pool_k(K), Wk)
+    if rope_theta > 0:
+        qt = block_rope(qt, rope_theta)
+        kt = block_rope(kt, rope_theta)
+    return gate_scores(qt, kt, d)
+
+
+# ----------------------------------------------------------- selection ---
+MODE_THRESHOLD, MODE_TOPK_K, MODE_TOPK_DENSITY = 0, 1, 2
+
+
+def select(scores, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
+           cap: int | None = None):
+    """Binary block mask as ascending index lists (summary page, section 3.4,
+    "Generating the binary block mask"; rebuttal section 3.3).
+    Returns (counts [B,Hq,nb] int32, idx [B,Hq,nb,cap] int32 padded with -1,
+    worst) where worst is the largest per-row count before truncation."""
+    s = _f64(scores)
+    B, Hq, nb, _ = s.shape
+    cap = nb if cap is None else cap
+    rows = B * Hq * nb
+    counts = np.zeros((B, Hq, nb), np.int32)
+    idx = np.full((B, Hq, nb, cap), -1, np.int32)
+    lib = _load()
+    if mode == MODE_THRESHOLD:
+        worst = lib.orc_select_threshold(_p(s), rows, nb, float(T), _p(counts), _p(idx), cap)
+    else:
+        worst = lib.orc_select_topk(_p(s), rows, nb, int(mode), int(k), float(density),
+                                    _p(counts), _p(idx), cap)
+    return counts, idx, int(worst)
+
+
+def topk_count(i: int, mode: int, k: int = 0, density: float = 0.0) -> int:
+    return int(_load().orc_topk_count(i, mode, k, density))
+
+
+# ----------------------------------------------------------- attention ---
+def sparse_attn(Q, K, V, counts, idx, scale: float | None = None):
+    """Block-sparse causal attention (summary page, section 3.4,
+    "Block-sparse FlashAttention kernel").  Returns (O [B,Hq,n,d], lse
+    [B,Hq,n]) in fp64; rows with no admissible key get O = 0, lse = -inf."""
+    q, k, v = _f32(Q), _f32(K), _f32(V)
+    B, Hq, n, d = q.shape
+    Hkv = k.shape[1]
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    ix = np.ascontiguousarray(idx, dtype=np.int32)
+    cap = ix.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    O = np.empty((B, Hq, n, d), np.float64)
+    lse = np.empty((B, Hq, n), np.float64)
+    _load().orc_sparse_attn(_p(q), _p(k), _p(v), B, Hq, Hkv, n, d, BLOCK, _p(c), _p(ix), cap,
+                            scale, _p(O), _p(lse))
+    return O, lse
+
+
+def sparse_attn_units(Q, K, V, counts, idx, units, scale: float | None = None):
+    """As sparse_attn, for the listed units u = (b*Hq + hq)*nb + i only.
+    Returns (O [len(units), 64, d], lse [len(units), 64])."""
+    q, k, v = _f32(Q), _f32(K), _f32(V)
+    B, Hq, n, d = q.shape
+    Hkv = k.shape[1]
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    ix = np.ascontiguousarray(idx, dtype=np.int32)
+    cap = ix.shape[-1]
+    u = np.ascontiguousarray(units, dtype=np.int64)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    O = np.empty((len(u), BLOCK, d), np.float64)
+    lse = np.empty((len(u), BLOCK), np.float64)
+    _load().orc_sparse_attn_units(_p(q), _p(k), _p(v), B, Hq, Hkv, n, d, BLOCK, _p(c), _p(ix),
+                                  cap, scale, _p(u), len(u), _p(O), _p(lse))
+    return O, lse
+
+
+def dense_lists(B: int, Hq: int, nb: int):
+    """All-ones causal mask as lists: row i lists 0..i."""
+    counts = np.broadcast_to(np.arange(1, nb + 1, dtype=np.int32), (B, Hq, nb)).copy()
+    idx = np.broadcast_to(np.arange(nb, dtype=np.int32), (B, Hq, nb, nb)).copy()
+    return counts, idx
+
+
+def blockmax(Q, K, scale: float | None = None):
+    """2D max-pooled causal attention probabilities (summary page, section
+    3.4, "Ground truth generation").  Returns (gt [B,Hq,nb,nb], lse)."""
+    q, k = _f32(Q), _f32(K)
+    B, Hq, n, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    gt = np.empty((B, Hq, n // BLOCK, n // BLOCK), np.float64)
+    lse = np.empty((B, Hq, n), np.float64)
+    _load().orc_blockmax(_p(q), _p(k), B, Hq, Hkv, n, d, BLOCK, scale, _p(gt), _p(lse))
+    return gt, lse
+
+
+def blockmax_units(Q, K, units, scale: float | None = None):
+    """As blockmax for the listed units: (gt rows [len, nb], lse [len, 64])."""
+    q, k = _f32(Q), _f32(K)
+    B, Hq, n, d = q.shape
+    Hkv = k.shape[1]
+    u = np.ascontiguousarray(units, dtype=np.int64)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    gt = np.empty((len(u), n // BLOCK), np.float64)
+    lse = np.empty((len(u), BLOCK), np.float64)
+    _load().orc_blockmax_units(_p(q), _p(k), B, Hq, Hkv, n, d, BLOCK, scale, _p(u), len(u),
+                               _p(gt), _p(lse))
+    return gt, lse

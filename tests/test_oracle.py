@@ -1,0 +1,440 @@
+"""Pins for the fp64 oracle: library routines, closed forms, invariants and the
+values the SeerAttention pages print.  CPU only.
+
+Each test checks the oracle against something other than itself, so that a
+dropped term, wrong sign, wrong index or transposed operand in any oracle
+function fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from learned_block_sparse_seer_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_examples.json")
+BLK = 64
+
+
+def _rand(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * scale).contiguous()
+
+
+# ------------------------------------------------------------------ pooling --
+def test_pool_q_is_avg_pool1d():
+    Q = _rand((2, 3, 256, 16), 1)
+    ref = F.avg_pool1d(Q.double().reshape(-1, 256, 16).transpose(1, 2), BLK, BLK)
+    ref = ref.transpose(1, 2).reshape(2, 3, 4, 16).numpy()
+    np.testing.assert_allclose(oracle.pool_q(Q), ref, rtol=0, atol=1e-14)
+
+
+def test_pool_k_is_max_min_avg_in_that_order():
+    K = _rand((1, 2, 192, 8), 2)
+    x = K.double().reshape(-1, 192, 8).transpose(1, 2)
+    mx = F.max_pool1d(x, BLK, BLK)
+    mn = -F.max_pool1d(-x, BLK, BLK)
+    av = F.avg_pool1d(x, BLK, BLK)
+    ref = torch.cat([mx, mn, av], dim=1).transpose(1, 2).reshape(1, 2, 3, 24).numpy()
+    got = oracle.pool_k(K)
+    np.testing.assert_array_equal(got[..., :16], ref[..., :16])  # max/min exact
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-14)
+
+
+def test_pool_constant_block_and_ordering():
+    K = torch.zeros(1, 1, 128, 4)
+    K[0, 0, :64] = torch.tensor([1.5, -2.0, 0.25, 7.0])
+    kb = oracle.pool_k(K)
+    np.testing.assert_array_equal(kb[0, 0, 0], np.tile([1.5, -2.0, 0.25, 7.0], 3))
+    R = _rand((1, 2, 512, 8), 3)
+    kb = oracle.pool_k(R)
+    d = 8
+    assert np.all(kb[..., :d] >= kb[..., 2 * d:]) and np.all(kb[..., 2 * d:] >= kb[..., d:2 * d])
+
+
+# --------------------------------------------------------------- projection --
+def test_project_matches_matmul_and_selects_rows():
+    x = _rand((2, 3, 5, 12), 4).double()
+    W = _rand((3, 7, 12), 5)
+    ref = torch.einsum("hrc,bhic->bhir", W.double(), x).numpy()
+    np.testing.assert_allclose(oracle.project(x, W), ref, rtol=1e-13, atol=1e-13)
+    # a selector matrix picks the first 4 features (catches transposed W)
+    sel = torch.zeros(3, 4, 12)
+    sel[:, torch.arange(4), torch.arange(4)] = 1.0
+    np.testing.assert_array_equal(oracle.project(x, sel), x[..., :4].numpy())
+
+
+# ---------------------------------------------------------------- gate (Eq.1)
+def _gate_inputs(seed=6, B=2, Hq=4, Hkv=2, nb=9, h=8):
+    qt = _rand((B, Hq, nb, h), seed).double()
+    kt = _rand((B, Hkv, nb, h), seed + 1).double()
+    return qt, kt
+
+
+def test_gate_scores_match_masked_softmax():
+    qt, kt = _gate_inputs()
+    d = 64
+    G = qt.shape[1] // kt.shape[1]
+    z = torch.einsum("bhic,bhjc->bhij", qt, kt.repeat_interleave(G, dim=1)) / math.sqrt(d)
+    nb = qt.shape[2]
+    mask = torch.tril(torch.ones(nb, nb, dtype=torch.bool))
+    ref = torch.softmax(z.masked_fill(~mask, float("-inf")), dim=-1).numpy()
+    got = oracle.gate_scores(qt, kt, d)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_gate_rows_sum_to_one_and_upper_triangle_zero():
+    qt, kt = _gate_inputs(seed=9)
+    s = oracle.gate_scores(qt, kt, 128)
+    np.testing.assert_allclose(s.sum(-1), 1.0, rtol=0, atol=1e-13)
+    nb = s.shape[-1]
+    assert np.all(s[..., np.triu_indices(nb, 1)[0], np.triu_indices(nb, 1)[1]] == 0)
+
+
+def test_gate_uniform_when_query_weights_zero():
+    w = synth.custom("g", 1, 2, 1, 512, 16, 8, "fp32", "tiny", 3)
+    Q, K, _ = synth.make_qkv(w)
+    Wq = torch.zeros(2, 8, 16)
+    _, Wk = synth.make_gate_weights(w)
+    s = oracle.gate(Q, K, Wq, Wk)
+    nb = w.nb
+    ref = np.tril(1.0 / np.arange(1, nb + 1)[:, None] * np.ones((nb, nb)))
+    np.testing.assert_allclose(s[0, 0], ref, rtol=1e-14, atol=0)
+
+
+def test_gate_two_blocks_is_sigmoid():
+    qt, kt = _gate_inputs(seed=12, B=1, Hq=1, Hkv=1, nb=2, h=4)
+    d = 16
+    z10 = float(qt[0, 0, 1] @ kt[0, 0, 0]) / 4.0
+    z11 = float(qt[0, 0, 1] @ kt[0, 0, 1]) / 4.0
+    s = oracle.gate_scores(qt, kt, d)
+    assert s[0, 0, 0, 0] == 1.0 and s[0, 0, 0, 1] == 0.0
+    assert abs(s[0, 0, 1, 0] - 1.0 / (1.0 + math.exp(z11 - z10))) < 1e-15
+    assert abs(s[0, 0, 1, 1] - 1.0 / (1.0 + math.exp(z10 - z11))) < 1e-15
+
+
+def test_gate_gqa_uses_kv_head_of_group():
+    # query heads 0,1 -> kv head 0; 2,3 -> kv head 1.  Swapping kv heads must
+    # swap the score maps of the two groups.
+    qt, kt = _gate_inputs(seed=21)
+    s = oracle.gate_scores(qt, kt, 64)
+    s_sw = oracle.gate_scores(qt[:, [2, 3, 0, 1]], kt[:, [1, 0]], 64)
+    np.testing.assert_array_equal(s[:, [2, 3, 0, 1]], s_sw)
+
+
+def test_gate_end_to_end_against_torch_pipeline():
+    w = synth.custom("g2", 1, 4, 2, 640, 32, 16, "bf16", "layer", 4)
+    Q, K, _ = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    x = Q.double().reshape(-1, w.n, w.d).transpose(1, 2)
+    qb = F.avg_pool1d(x, BLK, BLK).transpose(1, 2).reshape(1, 4, w.nb, w.d)
+    y = K.double().reshape(-1, w.n, w.d).transpose(1, 2)
+    kb = torch.cat([F.max_pool1d(y, BLK, BLK), -F.max_pool1d(-y, BLK, BLK),
+                    F.avg_pool1d(y, BLK, BLK)], 1).transpose(1, 2).reshape(1, 2, w.nb, 3 * w.d)
+    qt = torch.einsum("hrc,bhic->bhir", Wq.double(), qb)
+    kt = torch.einsum("hrc,bhic->bhir", Wk.double(), kb).repeat_interleave(2, dim=1)
+    z = qt @ kt.transpose(-1, -2) / math.sqrt(w.d)
+    mask = torch.tril(torch.ones(w.nb, w.nb, dtype=torch.bool))
+    ref = torch.softmax(z.masked_fill(~mask, float("-inf")), -1).numpy()
+    np.testing.assert_allclose(oracle.gate(Q, K, Wq, Wk), ref, rtol=1e-11, atol=1e-16)
+
+
+# ------------------------------------------------------------- block RoPE --
+def test_block_rope_rotation_structure():
+    """Rotation keeps norms, rotates pair 0 by exactly the block index, and
+    makes the dot product depend only on the block offset.  (The base reading
+    theta/B itself is parity unpinned.)"""
+    nb, h = 12, 8
+    x = _rand((1, 1, nb, h), 30).double()
+    y = oracle.block_rope(x, 10000.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x.numpy(), axis=-1),
+                               rtol=1e-13)
+    for i in range(nb):
+        a, b = x[0, 0, i, 0].item(), x[0, 0, i, h // 2].item()
+        assert abs(y[0, 0, i, 0] - (a * math.cos(i) - b * math.sin(i))) < 1e-12
+    # relative position: same vectors placed at (i, j) and (i+3, j+3)
+    q = _rand((1, 1, 1, h), 31).double()
+    k = _rand((1, 1, 1, h), 32).double()
+    qs = oracle.block_rope(q.expand(1, 1, nb, h).contiguous(), 500000.0)[0, 0]
+    ks = oracle.block_rope(k.expand(1, 1, nb, h).contiguous(), 500000.0)[0, 0]
+    assert abs(qs[7] @ ks[2] - qs[10] @ ks[5]) < 1e-12
+    assert abs(qs[7] @ ks[2] - qs[8] @ ks[2]) > 1e-6
+
+
+# --------------------------------------------------------------- selection --
+def test_threshold_is_strict_and_causal():
+    w = synth.custom("s", 1, 2, 1, 64 * 40, 16, 8, "fp32")
+    s = synth.make_scores_like(w, seed=3)
+    T = 0.03
+    counts, idx, worst = oracle.select(s, oracle.MODE_THRESHOLD, T=T)
+    s64 = s.double().numpy()
+    for h in range(2):
+        for i in range(w.nb):
+            ref = [j for j in range(i + 1) if s64[0, h, i, j] > np.float32(T)]
+            assert counts[0, h, i] == len(ref)
+            assert list(idx[0, h, i, :len(ref)]) == ref
+    # a score exactly equal to T is not selected (strict '>')
+    s2 = torch.zeros(1, 1, 2, 2)
+    s2[0, 0, 0, 0] = 1.0
+    s2[0, 0, 1] = torch.tensor([np.float32(0.25), np.float32(0.75)])
+    c, ix, _ = oracle.select(s2, oracle.MODE_THRESHOLD, T=0.25)
+    assert c[0, 0, 1] == 1 and ix[0, 0, 1, 0] == 1
+
+
+def test_topk_matches_stable_argsort_with_ties():
+    w = synth.custom("s", 1, 3, 1, 64 * 33, 16, 8, "fp32")
+    for ties in (False, True):
+        s = synth.make_scores_like(w, seed=5, ties=ties)
+        s64 = s.double().numpy()
+        for mode, k, rho in ((oracle.MODE_TOPK_K, 5, 0.0), (oracle.MODE_TOPK_DENSITY, 0, 0.3)):
+            counts, idx, _ = oracle.select(s, mode, k=k, density=rho)
+            for h in range(3):
+                for i in range(w.nb):
+                    row = s64[0, h, i, :i + 1]
+                    order = np.argsort(-row, kind="stable")  # ties: lower j first
+                    if mode == oracle.MODE_TOPK_K:
+                        ki = min(k, i + 1)
+                    else:
+                        ki = min(max(math.ceil(float(np.float32(np.float32(rho) * np.float32(i + 1)))), 1), i + 1)
+                    ref = sorted(order[:ki].tolist())
+                    assert counts[0, h, i] == ki
+                    assert idx[0, h, i, :ki].tolist() == ref
+                    sel = set(ref)
+                    if 0 < ki < i + 1:
+                        lo = min(row[j] for j in sel)
+                        hi = max(row[j] for j in range(i + 1) if j not in sel)
+                        assert lo >= hi
+
+
+def test_topk_row_zero_always_selects_block_zero():
+    w = synth.custom("s", 1, 1, 1, 64 * 8, 16, 8, "fp32")
+    s = synth.make_scores_like(w)
+    for mode, k, rho in ((1, 1, 0.0), (2, 0, 0.01)):
+        c, ix, _ = oracle.select(s, mode, k=k, density=rho)
+        assert c[0, 0, 0] == 1 and ix[0, 0, 0, 0] == 0
+
+
+def test_select_capacity_reports_worst_count():
+    w = synth.custom("s", 1, 1, 1, 64 * 16, 16, 8, "fp32")
+    s = synth.make_scores_like(w)
+    c, ix, worst = oracle.select(s, oracle.MODE_TOPK_K, k=10, cap=4)
+    assert worst == 10 and c.max() == 4
+
+
+def test_pages_topk_sparsity_example():
+    g = json.load(open(GOLDEN))["topk_sparsity"]
+    nb, k = g["nb"], g["k"]
+    # the last causal row has all nb blocks as candidates
+    assert oracle.topk_count(nb - 1, oracle.MODE_TOPK_K, k) == k
+    assert abs((1 - k / nb) - g["sparsity"]) < 1e-12
+    # and the density form gives the same count on that row
+    assert oracle.topk_count(nb - 1, oracle.MODE_TOPK_DENSITY, density=1 - g["sparsity"]) == k
+
+
+def test_pages_gate_size_ratio_and_threshold_example():
+    g = json.load(open(GOLDEN))
+    B = g["gate_size_ratio"]["block"]
+    assert (1.0 / B) ** 2 == g["gate_size_ratio"]["ratio"]
+    # a uniform row of length L has scores 1/L; with T = 0.002 rows longer than
+    # 500 blocks select nothing and shorter ones select everything.
+    T = g["threshold_example"]["T_longbench"]
+    nb = 520
+    s = torch.tril(torch.ones(nb, nb, dtype=torch.float64))
+    s = (s / s.sum(-1, keepdim=True)).float()[None, None]
+    c, _, _ = oracle.select(s, oracle.MODE_THRESHOLD, T=T)
+    L = np.arange(1, nb + 1)
+    expect = np.where(np.float32(1.0) / L.astype(np.float32) > np.float32(T), L, 0)
+    # 1/L as fp32 vs T as fp32: the strict comparison of the stored fp32 scores
+    sf = s[0, 0].numpy()
+    expect = np.array([(i + 1) if sf[i, 0] > np.float32(T) else 0 for i in range(nb)])
+    np.testing.assert_array_equal(c[0, 0], expect)
+    assert c[0, 0, 498] == 499 and c[0, 0, 500] == 0
+
+
+# --------------------------------------------------------------- attention --
+def _attn_case(B=1, Hq=4, Hkv=2, n=320, d=32, seed=40):
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(B, Hq, n, d, generator=g)
+    K = torch.randn(B, Hkv, n, d, generator=g)
+    V = torch.randn(B, Hkv, n, d, generator=g)
+    return Q, K, V
+
+
+def _sdpa(Q, K, V, mask=None, causal=False):
+    G = Q.shape[1] // K.shape[1]
+    Kr = K.double().repeat_interleave(G, 1)
+    Vr = V.double().repeat_interleave(G, 1)
+    return F.scaled_dot_product_attention(Q.double(), Kr, Vr, attn_mask=mask, is_causal=causal)
+
+
+def test_all_ones_mask_equals_dense_causal_sdpa():
+    Q, K, V = _attn_case()
+    B, Hq, n, d = Q.shape
+    counts, idx = oracle.dense_lists(B, Hq, n // BLK)
+    O, lse = oracle.sparse_attn(Q, K, V, counts, idx)
+    ref = _sdpa(Q, K, V, causal=True).numpy()
+    np.testing.assert_allclose(O, ref, rtol=0, atol=1e-12)
+    G = Hq // K.shape[1]
+    z = Q.double() @ K.double().repeat_interleave(G, 1).transpose(-1, -2) / math.sqrt(d)
+    z = z.masked_fill(~torch.tril(torch.ones(n, n, dtype=torch.bool)), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(z, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_sparse_mask_equals_sdpa_with_block_mask():
+    Q, K, V = _attn_case(seed=41)
+    B, Hq, n, d = Q.shape
+    nb = n // BLK
+    w = synth.custom("a", B, Hq, 2, n, d, 8, "fp32")
+    s = synth.make_scores_like(w, seed=9)
+    counts, idx, _ = oracle.select(s, oracle.MODE_TOPK_DENSITY, density=0.4)
+    blockmask = torch.zeros(B, Hq, nb, nb, dtype=torch.bool)
+    for h in range(Hq):
+        for i in range(nb):
+            blockmask[0, h, i, idx[0, h, i, :counts[0, h, i]]] = True
+    m = blockmask.repeat_interleave(BLK, 2).repeat_interleave(BLK, 3)
+    m &= torch.tril(torch.ones(n, n, dtype=torch.bool))
+    O, lse = oracle.sparse_attn(Q, K, V, counts, idx)
+    ref = _sdpa(Q, K, V, mask=m).numpy()
+    np.testing.assert_allclose(O, ref, rtol=0, atol=1e-12)
+
+
+def test_dropped_blocks_contribute_nothing():
+    Q, K, V = _attn_case(seed=42)
+    B, Hq, n, d = Q.shape
+    nb = n // BLK
+    counts = np.zeros((B, Hq, nb), np.int32)
+    idx = np.full((B, Hq, nb, nb), -1, np.int32)
+    for i in range(nb):
+        lst = [j for j in range(i + 1) if (i + j) % 2 == 0]  # keeps even blocks of even rows...
+        counts[0, :, i] = len(lst)
+        idx[0, :, i, :len(lst)] = lst
+    O1, l1 = oracle.sparse_attn(Q, K, V, counts, idx)
+    # every query head of kv head 0 only uses blocks listed for it; poison all
+    # blocks of kv heads that no list of that row uses.  Use row 4 only.
+    i = 4
+    used = set(idx[0, 0, i, :counts[0, 0, i]].tolist())
+    K2, V2 = K.clone(), V.clone()
+    for j in range(nb):
+        if j not in used:
+            K2[:, :, j * BLK:(j + 1) * BLK] = float("nan")
+            V2[:, :, j * BLK:(j + 1) * BLK] = 1e30
+    units = [(0 * Hq + h) * nb + i for h in range(Hq)]
+    O2, l2 = oracle.sparse_attn_units(Q, K2, V2, counts, idx, units)
+    for u, h in enumerate(range(Hq)):
+        np.testing.assert_array_equal(O2[u], O1[0, h, i * BLK:(i + 1) * BLK])
+        np.testing.assert_array_equal(l2[u], l1[0, h, i * BLK:(i + 1) * BLK])
+
+
+def test_single_block_list_and_empty_row():
+    Q, K, V = _attn_case(B=1, Hq=1, Hkv=1, n=256, d=16, seed=43)
+    nb = 4
+    counts = np.array([[[0, 1, 1, 1]]], np.int32)
+    idx = np.array([[[[-1], [0], [2], [3]]]], np.int32)
+    O, lse = oracle.sparse_attn(Q, K, V, counts, idx)
+    assert np.all(O[0, 0, :64] == 0) and np.all(np.isneginf(lse[0, 0, :64]))
+    # row 1 attends block 0 only: plain (non-causal) attention over those keys
+    ref = F.scaled_dot_product_attention(Q[:, :, 64:128].double(), K[:, :, :64].double(),
+                                         V[:, :, :64].double())
+    np.testing.assert_allclose(O[0, 0, 64:128], ref[0, 0].numpy(), rtol=0, atol=1e-12)
+    # row 3 attends its own block only: causal attention inside the block
+    ref = F.scaled_dot_product_attention(Q[:, :, 192:].double(), K[:, :, 192:].double(),
+                                         V[:, :, 192:].double(), is_causal=True)
+    np.testing.assert_allclose(O[0, 0, 192:], ref[0, 0].numpy(), rtol=0, atol=1e-12)
+    assert abs(lse[0, 0, 192] - float(Q[0, 0, 192].double() @ K[0, 0, 192].double()) / 4.0) < 1e-12
+
+
+def test_lse_merge_of_split_lists():
+    Q, K, V = _attn_case(seed=44)
+    B, Hq, n, d = Q.shape
+    nb = n // BLK
+    cA, iA = oracle.dense_lists(B, Hq, nb)
+    OA, lA = oracle.sparse_attn(Q, K, V, cA, iA)
+    # split every row's list into even and odd blocks
+    cE = np.zeros_like(cA); iE = np.full_like(iA, -1)
+    cO = np.zeros_like(cA); iO = np.full_like(iA, -1)
+    for i in range(nb):
+        ev = [j for j in range(i + 1) if j % 2 == 0]
+        od = [j for j in range(i + 1) if j % 2 == 1]
+        cE[..., i] = len(ev); iE[..., i, :len(ev)] = ev
+        cO[..., i] = len(od); iO[..., i, :len(od)] = od
+    OE, lE = oracle.sparse_attn(Q, K, V, cE, iE)
+    OO, lO = oracle.sparse_attn(Q, K, V, cO, iO)
+    lm = np.logaddexp(lE, lO)
+    wE = np.exp(lE - lm)[..., None]
+    wO = np.exp(lO - lm)[..., None]
+    np.testing.assert_allclose(lm, lA, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(wE * OE + np.nan_to_num(wO) * OO, OA, rtol=0, atol=1e-12)
+
+
+def test_gqa_head_mapping():
+    Q, K, V = _attn_case(Hq=4, Hkv=2, seed=45)
+    counts, idx = oracle.dense_lists(1, 4, Q.shape[2] // BLK)
+    O, _ = oracle.sparse_attn(Q, K, V, counts, idx)
+    # heads 2,3 must use kv head 1: recompute with kv heads swapped and heads permuted
+    O2, _ = oracle.sparse_attn(Q[:, [2, 3, 0, 1]], K[:, [1, 0]], V[:, [1, 0]], counts, idx)
+    np.testing.assert_array_equal(O[:, [2, 3, 0, 1]], O2)
+
+
+# ----------------------------------------------------------------- blockmax --
+def test_blockmax_is_maxpool2d_of_causal_softmax():
+    Q, K, _ = _attn_case(B=2, Hq=4, Hkv=2, n=320, d=32, seed=50)
+    B, Hq, n, d = Q.shape
+    gt, lse = oracle.blockmax(Q, K)
+    z = Q.double() @ K.double().repeat_interleave(2, 1).transpose(-1, -2) / math.sqrt(d)
+    z = z.masked_fill(~torch.tril(torch.ones(n, n, dtype=torch.bool)), float("-inf"))
+    P = torch.softmax(z, -1)
+    ref = F.max_pool2d(P.reshape(B * Hq, 1, n, n), BLK, BLK).reshape(B, Hq, n // BLK, n // BLK)
+    np.testing.assert_allclose(gt, ref.numpy(), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, torch.logsumexp(z, -1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_blockmax_invariants():
+    w = synth.custom("b", 1, 2, 1, 512, 32, 8, "bf16", "layer", 8)
+    Q, K, _ = synth.make_qkv(w)
+    gt, _ = oracle.blockmax(Q, K)
+    nb = w.nb
+    assert np.all(gt[..., 0, 0] == 1.0)  # token 0 attends only to itself
+    assert np.all(gt <= 1.0 + 1e-15) and np.all(gt >= 0)
+    iu = np.triu_indices(nb, 1)
+    assert np.all(gt[..., iu[0], iu[1]] == 0)
+    rowmax = gt.max(-1)
+    for i in range(nb):
+        assert np.all(rowmax[..., i] >= 1.0 / (64 * i + 1) - 1e-15)
+    # units API agrees with the full map
+    units = [0 * nb + 3, 1 * nb + 7]
+    gu, lu = oracle.blockmax_units(Q, K, units)
+    np.testing.assert_array_equal(gu[0], gt[0, 0, 3])
+    np.testing.assert_array_equal(gu[1], gt[0, 1, 7])
+
+
+def test_blockmax_lse_matches_dense_attention_lse():
+    Q, K, V = _attn_case(B=1, Hq=2, Hkv=1, n=256, d=16, seed=51)
+    _, lse_b = oracle.blockmax(Q, K)
+    c, ix = oracle.dense_lists(1, 2, 4)
+    _, lse_a = oracle.sparse_attn(Q, K, V, c, ix)
+    np.testing.assert_allclose(lse_b, lse_a, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ input recipe --
+def test_synth_is_deterministic_and_shaped():
+    w = synth.WORKLOADS["tiny"]
+    a = synth.make_qkv(w)
+    b = synth.make_qkv(w)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    assert a[0].shape == (1, 2, 512, 64) and a[1].shape == (1, 1, 512, 64)
+    assert a[0].dtype == torch.float32
+    Wq, Wk = synth.make_gate_weights(w)
+    assert Wq.shape == (2, 64, 64) and Wk.shape == (1, 64, 192)
+    assert abs(Wq.std().item() - 0.02) < 0.002
+    w8 = synth.custom("l", 1, 4, 2, 1024, 32, 16, "bf16", "layer", 1)
+    Q, K, V = synth.make_qkv(w8)
+    assert Q.dtype == torch.bfloat16 and K.shape == (1, 2, 1024, 32)
+    # the sink block carries the planted shift: its mean key norm is larger
+    kb = K.float().view(1, 2, 16, 64, 32).mean(3).norm(dim=-1)
+    assert torch.all(kb[:, :, 0] > 2.0)
