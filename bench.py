@@ -1,0 +1,499 @@
+"""Benchmark of the SeerAttention prefill hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one pass of the inference hot path over one synthetic Llama-3.1-8B
+attention layer at 128k tokens: the AttnGate (pooling, projections, block
+scores, top-k at 10% density = 90% block sparsity) and the block-sparse
+causal attention over the selected blocks.  The gate's ground-truth path
+(the max-pooled attention map) is timed in the same run on its own workload
+(B=1, 32k tokens) and reported as an extra object.
+
+value = active-block attention TFLOP/s of the whole step (gate included), all
+ranks together; each rank runs its own independent layer (weak scaling, no
+data-path collective).  Inputs (1.5 GB) are larger than L2, so no flush is
+needed between steps.  With --impl reference the fp64 CPU oracle is timed on
+the host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("sparse prefill attn ms & active-block TFLOP/s (% BF16 peak) at 128k, 90% sparsity")
+WORKLOAD = "layer128k"
+DENSITY = 0.1
+BMAX_WORKLOAD = "bmax32k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="seer", choices=["seer", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--density", type=float, default=DENSITY)
+    ap.add_argument("--no-blockmax", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="also time the 50-95%% sparsity sweep")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def attn_flops(counts, indices, d):
+    """Algorithmic FLOPs of the active blocks: 4*d per (query, key) pair, a
+    diagonal block counts its 64*65/2 causal pairs."""
+    import torch
+    nb = counts.shape[-1]
+    total_blocks = counts.long().sum().item()
+    cap = indices.shape[-1]
+    i = torch.arange(nb, device=counts.device).view(1, 1, nb)
+    pos = torch.arange(cap, device=counts.device).view(1, 1, 1, cap)
+    valid = pos < counts.unsqueeze(-1)
+    diag = ((indices == i.unsqueeze(-1)) & valid).sum().item()
+    pairs = (total_blocks - diag) * 64 * 64 + diag * (64 * 65 // 2)
+    causal = counts.shape[0] * counts.shape[1] * (nb * (nb + 1) // 2)
+    return 4.0 * d * pairs, total_blocks, diag, 1.0 - total_blocks / causal
+
+
+def source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "learned_block_sparse_seer_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload, src):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel, {})
+    except Exception:
+        return None
+    if d.get("source_hash") != src or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ oracle --
+class OracleSampler:
+    """Times the fp64 CPU oracle (as it stands) on a bounded sample of the
+    workload and extrapolates to the whole layer.
+
+    The oracle's work splits into a part per KV head (K max/min/avg pooling
+    and its projection over all blocks) and a part per unit (Q pooling and
+    projection of one block, its Eq. 1 score row, top-k selection, block-sparse
+    attention of its 64 rows).  Full-layer time = (#KV heads) x mean per-head
+    time + (#units) x mean per-unit time; value = the layer's active-block
+    attention FLOPs / that time."""
+
+    def __init__(self, w, Q, K, V, Wq, Wk, density, seed=0):
+        import numpy as np
+
+        import oracle
+        self.np, self.oracle = np, oracle
+        oracle.build()
+        self.w, self.density = w, density
+        # the oracle's input format: fp32 arrays holding the bf16 values exactly
+        self.Qf = Q.float().numpy()
+        self.Kf = K.float().numpy()
+        self.Vf = V.float().numpy()
+        self.Wq = Wq.numpy()
+        self.Wk = Wk.numpy()
+        self.rng = np.random.default_rng(seed)
+        self.t_head, self.t_unit, self.flops = [], [], []
+
+    def _units(self, b, g, hq, blocks, kt):
+        """Gate rows, selection and attention for query blocks `blocks` of
+        head hq, batched into single oracle calls (its OpenMP loops run over
+        the units)."""
+        np, oracle, w = self.np, self.oracle, self.w
+        nb = w.nb
+        cap = int(math.ceil(self.density * nb)) + 1
+        rows = np.concatenate([np.arange(i * 64, (i + 1) * 64) for i in blocks])
+        qb = oracle.pool_q(np.ascontiguousarray(self.Qf[b:b + 1, hq:hq + 1, rows]))
+        qrow = oracle.project(qb, self.Wq[hq:hq + 1])
+        qt = np.zeros((1, 1, nb, w.h))
+        qt[0, 0, blocks] = qrow[0, 0]
+        srows = oracle.gate_scores_units(qt, kt, w.d, blocks)
+        c1, i1 = oracle.select_rows(srows, blocks, oracle.MODE_TOPK_DENSITY, density=self.density,
+                                    cap=cap)
+        counts = np.zeros((1, 1, nb), np.int32)
+        idx = np.full((1, 1, nb, cap), -1, np.int32)
+        counts[0, 0, blocks] = c1
+        idx[0, 0, blocks] = i1
+        oracle.sparse_attn_units(self.Qf[b:b + 1, hq:hq + 1], self.Kf[b:b + 1, g:g + 1],
+                                 self.Vf[b:b + 1, g:g + 1], counts, idx, blocks)
+        return int(c1.sum())
+
+    def step(self, budget_s):
+        """One KV head's fixed part plus a batch of random units of one of its
+        query heads, sized to take about budget_s."""
+        np, oracle, w = self.np, self.oracle, self.w
+        b = int(self.rng.integers(w.B))
+        g = int(self.rng.integers(w.Hkv))
+        hq = g * w.G + int(self.rng.integers(w.G))
+        nb = w.nb
+        t0 = time.perf_counter()
+        kt = oracle.project(oracle.pool_k(self.Kf[b:b + 1, g:g + 1]), self.Wk[g:g + 1])
+        self.t_head.append(time.perf_counter() - t0)
+        n = 8
+        while True:
+            blocks = np.sort(self.rng.choice(nb, size=min(n, nb), replace=False))
+            t0 = time.perf_counter()
+            nblk = self._units(b, g, hq, blocks, kt)
+            dt = time.perf_counter() - t0
+            self.t_unit.extend([dt / len(blocks)] * len(blocks))
+            self.flops.append(4.0 * w.d * 64 * 64 * nblk)
+            budget_s -= dt
+            if budget_s <= 0:
+                break
+            n = int(min(nb, max(n * 2, len(blocks) * budget_s / max(dt, 1e-3))))
+
+    def rate(self, layer_flops):
+        """Extrapolated whole-layer TFLOP/s and layer time (s)."""
+        w = self.w
+        t_layer = (w.B * w.Hkv * (sum(self.t_head) / len(self.t_head))
+                   + w.B * w.Hq * w.nb * (sum(self.t_unit) / len(self.t_unit)))
+        return layer_flops / t_layer / 1e12, t_layer
+
+    def describe(self):
+        return (f"{len(self.t_head)} KV head(s) pooled+projected and {len(self.t_unit)} random units "
+                f"(query head x 64-row block: Q pooling, Eq.1 row, top-k, attention), fp64, "
+                f"{sum(self.t_head) + sum(self.t_unit):.1f} s; extrapolated to the whole layer")
+
+
+def layer_flops_expected(w, density):
+    """Active-block FLOPs of the layer under density top-k (diagonal counted
+    in full), for the reference arm that has no GPU lists."""
+    import oracle
+    tot = 0
+    for i in range(w.nb):
+        tot += oracle.topk_count(i, oracle.MODE_TOPK_DENSITY, density=density)
+    return 4.0 * w.d * 64 * 64 * tot * w.B * w.Hq
+
+
+# -------------------------------------------------------------------- main --
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from learned_block_sparse_seer_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    Q, K, V = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    smp = OracleSampler(w, Q, K, V, Wq, Wk, args.density)
+    lf = layer_flops_expected(w, args.density)
+    per_step = max(3.0, 100.0 / max(1, args.steps + args.warmup))
+    rates, times = [], []
+    for step in range(args.warmup + args.steps):
+        n0h, n0u = len(smp.t_head), len(smp.t_unit)
+        smp.step(per_step)
+        if step >= args.warmup:
+            r, t_layer = smp.rate(lf)
+            rates.append(r)
+            times.append(t_layer)
+    value, t_layer = smp.rate(lf)
+    cores = smp.oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} n={w.n} d={w.d} "
+                               f"gate h={w.h}, top-k density {args.density}"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": smp.describe()},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import learned_block_sparse_seer_b200 as seer
+    from learned_block_sparse_seer_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    seer.lib()
+
+    base = synth.WORKLOADS[args.workload]
+    w = synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.n, base.d, base.h, base.dtype,
+                       base.structure, base.seed + 1000 * rank)
+    Q, K, V = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    Qd, Kd, Vd, Wqd, Wkd = (t.to(dev) for t in (Q, K, V, Wq, Wk))
+    nb = w.nb
+    cap = seer.gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, "density", density=args.density)
+    counts = torch.empty(w.B, w.Hq, nb, dtype=torch.int32, device=dev)
+    indices = torch.empty(w.B, w.Hq, nb, cap, dtype=torch.int32, device=dev)
+    O = torch.empty_like(Qd)
+    lse = torch.empty(w.B, w.Hq, w.n, dtype=torch.float32, device=dev)
+    gws = torch.empty(seer.gate_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d, w.h), dtype=torch.uint8, device=dev)
+    aws = torch.empty(seer.sparse_attn_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def gate():
+        seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=args.density, cap=cap, workspace=gws,
+                       out=(counts, indices, None))
+
+    def attn():
+        seer.seer_sparse_attn(Qd, Kd, Vd, counts, indices, workspace=aws, out=(O, lse))
+
+    for _ in range(args.warmup):
+        gate()
+        attn()
+    torch.cuda.synchronize(dev)
+    assert seer.seer_workspace_status(aws) == 0, "device status after warm-up"
+    flops, nblocks, ndiag, sparsity = attn_flops(counts, indices, w.d)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        gate()
+        ev[s][1].record(stream)
+        attn()
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    gate_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    gate_avg = sum(gate_ms) / len(gate_ms)
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    attn_tflops = flops / (attn_avg * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    gate_bytes = (Q.numel() + K.numel()) * 2 + counts.numel() * 4 + nblocks * 4
+    src = source_hash(["attn.cu", "ptx.cuh"])
+    traffic = profiled_traffic("sparse_attn_kernel", args.workload, src)
+
+    # ------------------------------------------ end to end with host buffers --
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.pin_memory() for t in (Q, K, V))
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(2, min(args.steps, 5))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            Qd.copy_(hQ, non_blocking=True)
+            Kd.copy_(hK, non_blocking=True)
+            Vd.copy_(hV, non_blocking=True)
+            gate()
+            attn()
+            hO.copy_(O, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * 2,
+               "d2h_bytes_per_step": O.numel() * 2}
+
+    # --------------------------------------------------------- blockmax path --
+    bmax = None
+    if not args.no_blockmax and rank == 0:
+        bw = synth.WORKLOADS[BMAX_WORKLOAD]
+        bQ, bK, _ = synth.make_qkv(bw)
+        bQd, bKd = bQ.to(dev), bK.to(dev)
+        bws = torch.empty(seer.blockmax_workspace_size(bw.B, bw.Hq, bw.Hkv, bw.n, bw.d), dtype=torch.uint8,
+                          device=dev)
+        M = torch.empty(bw.B, bw.Hq, bw.nb, bw.nb, dtype=torch.float32, device=dev)
+        bl = torch.empty(bw.B, bw.Hq, bw.n, dtype=torch.float32, device=dev)
+        for _ in range(2):
+            seer.seer_attn_blockmax(bQd, bKd, workspace=bws, out=(M, bl))
+        torch.cuda.synchronize(dev)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nrep = 5
+        b0.record(stream)
+        for _ in range(nrep):
+            seer.seer_attn_blockmax(bQd, bKd, workspace=bws, out=(M, bl))
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = b0.elapsed_time(b1) / nrep
+        pairs = bw.B * bw.Hq * (bw.n * (bw.n + 1) // 2)
+        bflops = 2.0 * bw.d * pairs
+        bmax = {"workload": f"{BMAX_WORKLOAD}: B={bw.B} Hq={bw.Hq} Hkv={bw.Hkv} n={bw.n} d={bw.d}",
+                "ms": bms, "qk_tflops": bflops / (bms * 1e-3) / 1e12,
+                "frac_of_peak": bflops / (bms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                "exp_per_s": pairs / (bms * 1e-3),
+                "status": seer.seer_workspace_status(bws)}
+        del bQd, bKd, bws, M, bl
+
+    # ------------------------------------------------------ density sweep ----
+    sweep = None
+    if args.sweep and rank == 0:
+        sweep = []
+        for rho in (0.5, 0.3, 0.2, 0.1, 0.05):
+            c2 = seer.gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, "density", density=rho)
+            cc = torch.empty(w.B, w.Hq, nb, dtype=torch.int32, device=dev)
+            ii = torch.empty(w.B, w.Hq, nb, c2, dtype=torch.int32, device=dev)
+            seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=rho, cap=c2, workspace=gws, out=(cc, ii, None))
+            for _ in range(2):
+                seer.seer_sparse_attn(Qd, Kd, Vd, cc, ii, workspace=aws, out=(O, lse))
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(3):
+                seer.seer_sparse_attn(Qd, Kd, Vd, cc, ii, workspace=aws, out=(O, lse))
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = a.elapsed_time(b) / 3
+            f, nbk, _, sp = attn_flops(cc, ii, w.d)
+            sweep.append({"density": rho, "sparsity": sp, "active_blocks": nbk, "attn_ms": ms,
+                          "tflops": f / (ms * 1e-3) / 1e12})
+
+    # ------------------------------------------------------ oracle baseline --
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        smp = OracleSampler(w, Q, K, V, Wq, Wk, args.density)
+        for _ in range(3):
+            smp.step(4.0)
+        rate, _ = smp.rate(flops)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": smp.oracle.num_threads(), "kind": "oracle",
+               "sample": smp.describe()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} n={w.n} d={w.d} "
+                                   f"gate h={w.h}, top-k density {args.density}",
+                       "achieved_sparsity": sparsity, "active_blocks": nblocks,
+                       "l2": "inputs larger than L2 (Q+K+V = 1.5 GB), no flush",
+                       "parallelism": f"replica per GPU (independent layer per rank), {world} GPU(s)"},
+            "attn_ms": attn_avg, "gate_ms": gate_avg, "attn_tflops": attn_tflops,
+            "attn_pct_bf16_peak": {"burst": attn_tflops / pk["bf16_tflops"],
+                                   "sustained": attn_tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                                   "peaks": pk_kind},
+            "gate_gbs": gate_bytes / (gate_avg * 1e-3) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "traffic": traffic,
+                         "kernel": "sparse_attn_kernel", "peak_kind": f"bf16 sustained ({pk_kind})",
+                         "algorithmic_flops_per_launch": flops},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": 7 * args.steps,
+            "blockmax": bmax, "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * seer.h -- C ABI of the B200 (sm_100a) SeerAttention prefill library.
+ *
+ * The library implements the prefill hot path of "SeerAttention: Learning
+ * Intrinsic Sparse Attention in Your LLMs" (arXiv 2410.13276):
+ *   seer_gate           AttnGate block scorer + binary block-mask generation
+ *   seer_gate_select    the mask-generation step alone, on supplied scores
+ *   seer_sparse_attn    block-sparse causal attention over the selected blocks
+ *   seer_attn_blockmax  2D max-pooled attention-probability map (the gate's
+ *                       self-distillation target)
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory; scratch comes from the caller's workspace,
+ *    whose size the matching *_workspace_size() call returns.  Workspace
+ *    pointers must be 256-byte aligned.
+ *  - Layout: every tensor is contiguous [B, H, n, d], row-major ("head-major").
+ *    Query head hq uses KV head hq / (Hq / Hkv) (grouped-query attention).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronises.  Arguments are validated on the
+ *    host before anything is launched; on any error nothing is written.
+ *  - Device-side failures (a bounded wait that gave up, an index that failed a
+ *    bounds check) are recorded in a status word at the start of the
+ *    workspace.  seer_workspace_status() synchronises `stream` and reads it.
+ *  - The library keeps no global state and is safe to call from several host
+ *    threads on different streams (each call with its own workspace).
+ *  - The block size is fixed at 64 tokens (the pages fix B = 64 in all
+ *    experiments: summary page, section 3.4, "Key Configuration Summary").
+ */
+#ifndef SEER_H
+#define SEER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SEER_API __attribute__((visibility("default")))
+#else
+#define SEER_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *seer_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  SEER_OK = 0,
+  SEER_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, T <= 0, k < 1, ... */
+  SEER_ERR_UNSUPPORTED = 2,   /* block != 64, d not in {64,128}, dtype, ...    */
+  SEER_ERR_CAPACITY = 3,      /* cap smaller than the largest possible count  */
+  SEER_ERR_CUDA = 4,          /* a CUDA runtime call failed; see
+                                 seer_last_cuda_error()                        */
+  SEER_ERR_TIMEOUT = 5,       /* device status: a bounded wait gave up        */
+  SEER_ERR_DEVICE_CHECK = 6,  /* device status: an index failed its check     */
+  SEER_ERR_WORKSPACE = 7      /* workspace null, misaligned or too small      */
+} seer_status;
+
+typedef enum { SEER_BF16 = 0, SEER_FP32 = 1 } seer_dtype;
+
+typedef enum {
+  /* Thresholding: block j is active iff score[i][j] > T (strict).
+     Summary page, section 3.4, "Method 2: Thresholding"; rebuttal 3.3. */
+  SEER_SELECT_THRESHOLD = 0,
+  /* TopK with a uniform k: the k_i = min(k, i+1) largest scores of row i.
+     Summary page, section 3.4, "Method 1: TopK selection". */
+  SEER_SELECT_TOPK_K = 1,
+  /* TopK with a density rho: k_i = clamp(ceil(rho*(i+1)), 1, i+1), the product
+     rounded in fp32.  Gives block sparsity ~ 1 - rho on every causal row. */
+  SEER_SELECT_TOPK_DENSITY = 2
+} seer_select_mode;
+
+/* Problem shape.  n must be a multiple of `block`; Hq a multiple of Hkv. */
+typedef struct {
+  int32_t B;     /* batch                                   */
+  int32_t Hq;    /* query heads                             */
+  int32_t Hkv;   /* key/value heads                         */
+  int32_t n;     /* sequence length (tokens), multiple of 64 */
+  int32_t d;     /* head dimension: 64 or 128               */
+  int32_t block; /* block size: must be 64                  */
+} seer_dims;
+
+/* ------------------------------------------------------------------------ */
+/* seer_gate -- the AttnGate of SeerAttention plus mask generation.
+ *
+ * Computes, per query head and query block i (summary page, section 3.4,
+ * "AttnGate", Eq. 1; pooling per "Pooling Method Selection"):
+ *   qbar_i = mean of Q over block i                       [d]
+ *   kbar_j = [max | min | mean] of K over block j         [3d]
+ *   q~_i   = Wq[hq] qbar_i,   k~_j = Wk[g] kbar_j        [h]  (no bias)
+ *   optional block RoPE on q~, k~ at block positions with base rope_theta/64
+ *     (summary page, "Block-Level RoPE"; rope_theta <= 0 disables it)
+ *   score[i][j] = softmax_{j <= i}( q~_i . k~_j / sqrt(d) ), 0 for j > i
+ * then the active key blocks of every row as an ascending index list
+ * (rebuttal, section 3.3: "torch.topk ... indices [S/B, k]").
+ *
+ *   Q         [B, Hq, n, d]  bf16 or fp32 (dtype)
+ *   K         [B, Hkv, n, d] same dtype
+ *   Wq        [Hq, h, d]     fp32
+ *   Wk        [Hkv, h, 3d]   fp32, input features ordered [max | min | avg]
+ *   h         gate hidden size, 1..256, multiple of 4
+ *   mode/T/k/density   selection (see seer_select_mode); T > 0 for
+ *             THRESHOLD, k >= 1 for TOPK_K, 0 < density <= 1 for TOPK_DENSITY
+ *   scores_out  optional [B, Hq, nb, nb] fp32 (nb = n/64): the scores the
+ *             selection used; entries j > i are written as 0.  May be NULL.
+ *   counts    [B, Hq, nb] int32: number of active blocks of each row
+ *   indices   [B, Hq, nb, cap] int32: ascending active key blocks of each row;
+ *             entries past counts[row] are left untouched
+ *   cap       row capacity; must be >= seer_gate_required_cap(...)
+ *   ws/ws_bytes  workspace of at least seer_gate_workspace_size(...) bytes
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CAPACITY,
+ *         SEER_ERR_WORKSPACE, SEER_ERR_CUDA.                               */
+SEER_API seer_status seer_gate(const seer_dims *dims, const void *Q, const void *K, seer_dtype dtype,
+                      const float *Wq, const float *Wk, int32_t h, float rope_theta,
+                      seer_select_mode mode, float T, int32_t k, float density,
+                      float *scores_out, int32_t *counts, int32_t *indices, int32_t cap,
+                      void *ws, size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_gate_workspace_size(const seer_dims *dims, int32_t h);
+
+/* Smallest `cap` that can hold every row's list for this selection:
+ * nb for THRESHOLD, min(k, nb) for TOPK_K, the largest k_i for TOPK_DENSITY.
+ * Returns -1 on invalid arguments. */
+SEER_API int32_t seer_gate_required_cap(const seer_dims *dims, seer_select_mode mode, int32_t k,
+                               float density);
+
+/* seer_gate_select -- the mask-generation step alone on caller-supplied fp32
+ * scores [B, Hq, nb, nb] (entries j > i are ignored).  Same selection rules
+ * and outputs as seer_gate; used to check index lists bit-exactly against an
+ * independent implementation fed the same scores.  No workspace. */
+SEER_API seer_status seer_gate_select(const seer_dims *dims, const float *scores, seer_select_mode mode,
+                             float T, int32_t k, float density, int32_t *counts,
+                             int32_t *indices, int32_t cap, seer_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* seer_sparse_attn -- block-sparse causal attention forward (summary page,
+ * section 3.4, "Block-sparse FlashAttention kernel"): for query block i of
+ * head hq, only key blocks j in its list are used -- a skipped block costs no
+ * QK^T, no softmax, no PV and no K/V load.  Inside the diagonal block the
+ * causal rule (key position <= query position) applies.  Per query row t:
+ *   O[t]   = sum_s softmax_s(scale * q_t . k_s) v_s
+ *   lse[t] = ln sum_s exp(scale * q_t . k_s)
+ * over the admissible keys s; a row with none gets O = 0 and lse = -inf.
+ *
+ *   Q [B,Hq,n,d], K/V [B,Hkv,n,d]: bf16 (fp32 is converted to bf16 in the
+ *             workspace before the tensor-core pass)
+ *   counts [B,Hq,nb], indices [B,Hq,nb,cap]: lists as written by seer_gate:
+ *             ascending, unique, every j <= i.  The kernel checks every
+ *             count (0 <= c <= min(cap, i+1)) and entry (in range, strictly
+ *             ascending) before loading; a failing one is clamped into range
+ *             and recorded as SEER_ERR_DEVICE_CHECK in the workspace status.
+ *   scale     softmax scale; 0 means 1/sqrt(d)
+ *   O         [B,Hq,n,d] same dtype as Q;  lse [B,Hq,n] fp32 (may be NULL)
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
+SEER_API seer_status seer_sparse_attn(const seer_dims *dims, const void *Q, const void *K, const void *V,
+                             seer_dtype dtype, const int32_t *counts, const int32_t *indices,
+                             int32_t cap, float scale, void *O, float *lse, void *ws,
+                             size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_sparse_attn_workspace_size(const seer_dims *dims, seer_dtype dtype);
+
+/* ------------------------------------------------------------------------ */
+/* seer_attn_blockmax -- the ground truth of the gate's self-distillation
+ * (summary page, section 3.4, "Ground truth generation" and "The customized
+ * training kernel", Figure 10):
+ *   map[i][j] = max over the 64x64 block (i, j) of softmax(scale * Q K^T)
+ * with the causal softmax of every query row; map[i][j] = 0 for j > i.
+ * Two passes: the first forms every row's log-sum-exp and each row's raw
+ * maximum per key block; the second rescales those maxima into
+ * probabilities and takes the column maximum over the rows of the block.
+ *
+ *   Q [B,Hq,n,d], K [B,Hkv,n,d]  bf16 (fp32 converted in the workspace)
+ *   scale     0 means 1/sqrt(d)
+ *   map_out   [B, Hq, nb, nb] fp32
+ *   lse_out   optional [B, Hq, n] fp32 row log-sum-exp (may be NULL)
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
+SEER_API seer_status seer_attn_blockmax(const seer_dims *dims, const void *Q, const void *K,
+                               seer_dtype dtype, float scale, float *map_out, float *lse_out,
+                               void *ws, size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_blockmax_workspace_size(const seer_dims *dims, seer_dtype dtype);
+
+/* ------------------------------------------------------------------------ */
+/* Synchronises `stream`, reads the device status word at the start of a
+ * workspace that a previous call used, and maps it: SEER_OK,
+ * SEER_ERR_TIMEOUT or SEER_ERR_DEVICE_CHECK (SEER_ERR_CUDA if the read
+ * fails).  Every call clears the word when it starts. */
+SEER_API seer_status seer_workspace_status(const void *ws, seer_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+SEER_API const char *seer_status_string(seer_status s);
+
+/* The cudaError_t of the last SEER_ERR_CUDA returned on this host thread. */
+SEER_API int32_t seer_last_cuda_error(void);
+
+/* Library version, e.g. "0.1.0". */
+SEER_API const char *seer_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SEER_H */

@@ -1,0 +1,249 @@
+"""Thin ctypes binding of libseer.so (include/seer.h): argument marshalling only.
+
+Every computation runs in the CUDA library; this module only checks tensor
+properties, allocates caller-owned outputs and workspaces with torch, and
+passes raw device pointers and the current CUDA stream.  If the library is
+missing it raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libseer.so")
+
+SEER_OK = 0
+STATUS_NAMES = {
+    0: "SEER_OK", 1: "SEER_ERR_INVALID_ARG", 2: "SEER_ERR_UNSUPPORTED", 3: "SEER_ERR_CAPACITY",
+    4: "SEER_ERR_CUDA", 5: "SEER_ERR_TIMEOUT", 6: "SEER_ERR_DEVICE_CHECK", 7: "SEER_ERR_WORKSPACE",
+}
+SEER_BF16, SEER_FP32 = 0, 1
+SELECT_THRESHOLD, SELECT_TOPK_K, SELECT_TOPK_DENSITY = 0, 1, 2
+
+
+class SeerError(RuntimeError):
+    def __init__(self, func: str, status: int, cuda_err: int = 0):
+        name = STATUS_NAMES.get(status, str(status))
+        msg = f"{func} returned {name}"
+        if status == 4:
+            msg += f" (cudaError {cuda_err})"
+        super().__init__(msg)
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("n", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if libseer.so has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m learned_block_sparse_seer_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+        DP = ctypes.POINTER(Dims)
+        L.seer_gate.argtypes = [DP, P, P, I32, P, P, I32, F, I32, F, I32, F, P, P, P, I32, P, SZ, P]
+        L.seer_gate.restype = I32
+        L.seer_gate_workspace_size.argtypes = [DP, I32]
+        L.seer_gate_workspace_size.restype = SZ
+        L.seer_gate_required_cap.argtypes = [DP, I32, I32, F]
+        L.seer_gate_required_cap.restype = I32
+        L.seer_gate_select.argtypes = [DP, P, I32, F, I32, F, P, P, I32, P]
+        L.seer_gate_select.restype = I32
+        L.seer_sparse_attn.argtypes = [DP, P, P, P, I32, P, P, I32, F, P, P, P, SZ, P]
+        L.seer_sparse_attn.restype = I32
+        L.seer_sparse_attn_workspace_size.argtypes = [DP, I32]
+        L.seer_sparse_attn_workspace_size.restype = SZ
+        L.seer_attn_blockmax.argtypes = [DP, P, P, I32, F, P, P, P, SZ, P]
+        L.seer_attn_blockmax.restype = I32
+        L.seer_blockmax_workspace_size.argtypes = [DP, I32]
+        L.seer_blockmax_workspace_size.restype = SZ
+        L.seer_workspace_status.argtypes = [P, P]
+        L.seer_workspace_status.restype = I32
+        L.seer_status_string.argtypes = [I32]
+        L.seer_status_string.restype = ctypes.c_char_p
+        L.seer_last_cuda_error.restype = I32
+        L.seer_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(func: str, status: int):
+    if status != SEER_OK:
+        raise SeerError(func, status, lib().seer_last_cuda_error())
+
+
+def _dims(B, Hq, Hkv, n, d) -> Dims:
+    return Dims(int(B), int(Hq), int(Hkv), int(n), int(d), 64)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SEER_BF16
+    if t.dtype == torch.float32:
+        return SEER_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp32")
+
+
+def _dev(*ts: torch.Tensor):
+    dev = ts[0].device
+    for t in ts:
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, n, d]")
+    return dev
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(dev) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _workspace(nbytes: int, dev, ws: torch.Tensor | None) -> torch.Tensor:
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return ws
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+
+
+def mode_code(mode) -> int:
+    if isinstance(mode, int):
+        return mode
+    return {"threshold": SELECT_THRESHOLD, "topk": SELECT_TOPK_K, "topk_k": SELECT_TOPK_K,
+            "density": SELECT_TOPK_DENSITY, "topk_density": SELECT_TOPK_DENSITY}[mode]
+
+
+# --------------------------------------------------------------------- gate --
+def gate_workspace_size(B, Hq, Hkv, n, d, h) -> int:
+    return int(lib().seer_gate_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)), int(h)))
+
+
+def gate_required_cap(B, Hq, Hkv, n, d, mode, k=0, density=0.0) -> int:
+    return int(lib().seer_gate_required_cap(ctypes.byref(_dims(B, Hq, Hkv, n, d)), mode_code(mode),
+                                            int(k), float(density)))
+
+
+def seer_gate(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, return_scores=False,
+              cap=None, workspace=None, out=None):
+    """AttnGate + mask generation.  Returns (counts, indices[, scores])."""
+    dev = _dev(Q, K, Wq, Wk)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    if Wq.dtype != torch.float32 or Wk.dtype != torch.float32:
+        raise TypeError("gate weights must be fp32")
+    h = Wq.shape[1]
+    nb = n // 64
+    mc = mode_code(mode)
+    dims = _dims(B, Hq, Hkv, n, d)
+    if cap is None:
+        cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
+    if out is None:
+        counts = torch.empty(B, Hq, nb, dtype=torch.int32, device=dev)
+        indices = torch.empty(B, Hq, nb, cap, dtype=torch.int32, device=dev)
+        scores = torch.empty(B, Hq, nb, nb, dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        counts, indices, scores = out
+    ws = _workspace(gate_workspace_size(B, Hq, Hkv, n, d, h), dev, workspace)
+    st = lib().seer_gate(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq), _ptr(Wk),
+                         int(h), float(rope_theta), mc, float(T), int(k), float(density),
+                         _ptr(scores), _ptr(counts), _ptr(indices), int(cap), _ptr(ws),
+                         ws.numel(), _stream(dev))
+    _check("seer_gate", st)
+    return (counts, indices, scores) if return_scores else (counts, indices)
+
+
+def seer_gate_select(scores, mode, T=0.0, k=0, density=0.0, cap=None, out=None):
+    """Mask generation on supplied fp32 scores [B, Hq, nb, nb]."""
+    dev = _dev(scores)
+    if scores.dtype != torch.float32:
+        raise TypeError("scores must be fp32")
+    B, Hq, nb, _ = scores.shape
+    mc = mode_code(mode)
+    dims = _dims(B, Hq, 1, nb * 64, 64)
+    if cap is None:
+        cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
+    if out is None:
+        counts = torch.empty(B, Hq, nb, dtype=torch.int32, device=dev)
+        indices = torch.empty(B, Hq, nb, cap, dtype=torch.int32, device=dev)
+    else:
+        counts, indices = out
+    st = lib().seer_gate_select(ctypes.byref(dims), _ptr(scores), mc, float(T), int(k),
+                                float(density), _ptr(counts), _ptr(indices), int(cap), _stream(dev))
+    _check("seer_gate_select", st)
+    return counts, indices
+
+
+# ---------------------------------------------------------------- attention --
+def sparse_attn_workspace_size(B, Hq, Hkv, n, d, dtype_code=SEER_BF16) -> int:
+    return int(lib().seer_sparse_attn_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)),
+                                                     int(dtype_code)))
+
+
+def seer_sparse_attn(Q, K, V, counts, indices, scale=0.0, workspace=None, out=None,
+                     return_lse=True):
+    """Block-sparse causal attention over the listed key blocks.
+    Returns (O, lse)."""
+    dev = _dev(Q, K, V, counts, indices)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    dt = _dtype_code(Q)
+    if counts.dtype != torch.int32 or indices.dtype != torch.int32:
+        raise TypeError("counts/indices must be int32")
+    cap = indices.shape[-1]
+    if out is None:
+        O = torch.empty_like(Q)
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=dev) if return_lse else None
+    else:
+        O, lse = out
+    ws = _workspace(sparse_attn_workspace_size(B, Hq, Hkv, n, d, dt), dev, workspace)
+    st = lib().seer_sparse_attn(ctypes.byref(_dims(B, Hq, Hkv, n, d)), _ptr(Q), _ptr(K), _ptr(V),
+                                dt, _ptr(counts), _ptr(indices), int(cap), float(scale), _ptr(O),
+                                _ptr(lse), _ptr(ws), ws.numel(), _stream(dev))
+    _check("seer_sparse_attn", st)
+    return O, lse
+
+
+def blockmax_workspace_size(B, Hq, Hkv, n, d, dtype_code=SEER_BF16) -> int:
+    return int(lib().seer_blockmax_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)),
+                                                  int(dtype_code)))
+
+
+def seer_attn_blockmax(Q, K, scale=0.0, workspace=None, out=None, return_lse=True):
+    """2D max-pooled causal attention probabilities.  Returns (map, lse)."""
+    dev = _dev(Q, K)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    dt = _dtype_code(Q)
+    nb = n // 64
+    if out is None:
+        M = torch.empty(B, Hq, nb, nb, dtype=torch.float32, device=dev)
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=dev) if return_lse else None
+    else:
+        M, lse = out
+    ws = _workspace(blockmax_workspace_size(B, Hq, Hkv, n, d, dt), dev, workspace)
+    st = lib().seer_attn_blockmax(ctypes.byref(_dims(B, Hq, Hkv, n, d)), _ptr(Q), _ptr(K), dt,
+                                  float(scale), _ptr(M), _ptr(lse), _ptr(ws), ws.numel(),
+                                  _stream(dev))
+    _check("seer_attn_blockmax", st)
+    return M, lse
+
+
+def seer_workspace_status(workspace: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the device status code."""
+    return int(lib().seer_workspace_status(_ptr(workspace), _stream(workspace.device)))

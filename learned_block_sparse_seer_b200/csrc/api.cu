@@ -1,0 +1,428 @@
+// api.cu -- the C ABI of the library (include/seer.h): argument validation,
+// workspace carving, TMA tensor-map encoding and kernel launches.  Every call
+// is asynchronous on the caller's stream; nothing here allocates device
+// memory.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/seer.h"
+#include "attn.cuh"
+#include "blockmax.cuh"
+#include "common.cuh"
+#include "gate.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+seer_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int32_t)e;
+  return SEER_ERR_CUDA;
+}
+
+#define SEER_CUDA(x)                            \
+  do {                                          \
+    cudaError_t e_ = (x);                       \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+bool dims_ok(const seer_dims* d) {
+  if (!d) return false;
+  if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->n < 1) return false;
+  if (d->Hq % d->Hkv != 0) return false;
+  if (d->n % seer::kBlock != 0) return false;
+  // TMA row coordinates and the persistent work index are 32-bit
+  if ((long long)d->B * d->Hq * d->n >= (1LL << 31)) return false;
+  return true;
+}
+
+seer_status dims_supported(const seer_dims* d) {
+  if (d->block != seer::kBlock) return SEER_ERR_UNSUPPORTED;
+  if (d->d != 64 && d->d != 128) return SEER_ERR_UNSUPPORTED;
+  return SEER_OK;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows, d] with a (64 x box_rows) box, 128-byte swizzle.
+bool make_tmap(CUtensorMap* tm, const void* base, long long rows, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                   long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    y[i] = __float2bfloat16_rn(x[i]);
+}
+
+cudaError_t to_bf16(const void* x, void* y, long long n, cudaStream_t st) {
+  f32_to_bf16_kernel<<<1184, 256, 0, st>>>((const float*)x, (__nv_bfloat16*)y, n);
+  return cudaGetLastError();
+}
+
+struct GateWs {
+  size_t qbar, kbar, qt, kt, logits, total;
+};
+
+GateWs gate_ws(const seer_dims* d, int h) {
+  const long long nb = d->n / seer::kBlock;
+  seer::WsCarver c;
+  GateWs w;
+  w.qbar = c.take(sizeof(float) * d->B * d->Hq * nb * d->d);
+  w.kbar = c.take(sizeof(float) * d->B * d->Hkv * nb * 3 * d->d);
+  w.qt = c.take(sizeof(float) * d->B * d->Hq * nb * h);
+  w.kt = c.take(sizeof(float) * d->B * d->Hkv * nb * h);
+  w.logits = c.take(sizeof(float) * d->B * d->Hq * nb * nb);
+  w.total = c.off;
+  return w;
+}
+
+struct AttnWs {
+  size_t q16, k16, v16, total;
+};
+
+AttnWs attn_ws(const seer_dims* d, seer_dtype dt) {
+  seer::WsCarver c;
+  AttnWs w{0, 0, 0, 0};
+  if (dt == SEER_FP32) {
+    w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
+    w.k16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+    w.v16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+  }
+  w.total = c.off;
+  return w;
+}
+
+struct BmaxWs {
+  size_t q16, k16, r, total;
+  int ctas;
+};
+
+BmaxWs bmax_ws(const seer_dims* d, seer_dtype dt, int sms) {
+  seer::WsCarver c;
+  BmaxWs w{0, 0, 0, 0, 0};
+  if (dt == SEER_FP32) {
+    w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
+    w.k16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+  }
+  const long long nb = d->n / seer::kBlock;
+  w.ctas = sms;
+  w.r = c.take(sizeof(float) * (size_t)sms * 128 * nb);
+  w.total = c.off;
+  return w;
+}
+
+seer_status begin_ws(void* ws, size_t ws_bytes, size_t need, cudaStream_t st) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEER_ERR_WORKSPACE;
+  SEER_CUDA(cudaMemsetAsync(ws, 0, sizeof(seer::WsHeader), st));
+  return SEER_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* seer_version(void) { return "0.1.0"; }
+
+int32_t seer_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* seer_status_string(seer_status s) {
+  switch (s) {
+    case SEER_OK: return "SEER_OK";
+    case SEER_ERR_INVALID_ARG: return "SEER_ERR_INVALID_ARG";
+    case SEER_ERR_UNSUPPORTED: return "SEER_ERR_UNSUPPORTED";
+    case SEER_ERR_CAPACITY: return "SEER_ERR_CAPACITY";
+    case SEER_ERR_CUDA: return "SEER_ERR_CUDA";
+    case SEER_ERR_TIMEOUT: return "SEER_ERR_TIMEOUT";
+    case SEER_ERR_DEVICE_CHECK: return "SEER_ERR_DEVICE_CHECK";
+    case SEER_ERR_WORKSPACE: return "SEER_ERR_WORKSPACE";
+  }
+  return "SEER_ERR_UNKNOWN";
+}
+
+seer_status seer_workspace_status(const void* ws, seer_stream_t stream) {
+  if (!ws) return SEER_ERR_WORKSPACE;
+  uint32_t h[2] = {0, 0};
+  cudaStream_t st = (cudaStream_t)stream;
+  SEER_CUDA(cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, st));
+  SEER_CUDA(cudaStreamSynchronize(st));
+  switch (h[0]) {
+    case seer::kDevOk: return SEER_OK;
+    case seer::kDevTimeout: return SEER_ERR_TIMEOUT;
+    default: return SEER_ERR_DEVICE_CHECK;
+  }
+}
+
+// ------------------------------------------------------------------- gate --
+size_t seer_gate_workspace_size(const seer_dims* dims, int32_t h) {
+  if (!dims_ok(dims) || h < 1) return 0;
+  return gate_ws(dims, h).total;
+}
+
+int32_t seer_gate_required_cap(const seer_dims* dims, seer_select_mode mode, int32_t k,
+                               float density) {
+  if (!dims_ok(dims)) return -1;
+  const int nb = dims->n / seer::kBlock;
+  switch (mode) {
+    case SEER_SELECT_THRESHOLD: return nb;
+    case SEER_SELECT_TOPK_K: return k < 1 ? -1 : (k < nb ? k : nb);
+    case SEER_SELECT_TOPK_DENSITY: {
+      if (!(density > 0.f && density <= 1.f)) return -1;
+      int worst = 0;
+      for (int i = 0; i < nb; ++i) {
+        int ki = (int)std::ceil((double)(density * (float)(i + 1)));
+        if (ki < 1) ki = 1;
+        if (ki > i + 1) ki = i + 1;
+        if (ki > worst) worst = ki;
+      }
+      return worst;
+    }
+  }
+  return -1;
+}
+
+static seer_status check_select(const seer_dims* dims, seer_select_mode mode, float T, int32_t k,
+                                float density, int32_t cap) {
+  switch (mode) {
+    case SEER_SELECT_THRESHOLD:
+      if (!(T > 0.f) || !std::isfinite(T)) return SEER_ERR_INVALID_ARG;
+      break;
+    case SEER_SELECT_TOPK_K:
+      if (k < 1) return SEER_ERR_INVALID_ARG;
+      break;
+    case SEER_SELECT_TOPK_DENSITY:
+      if (!(density > 0.f && density <= 1.f)) return SEER_ERR_INVALID_ARG;
+      break;
+    default:
+      return SEER_ERR_INVALID_ARG;
+  }
+  if (cap < 1) return SEER_ERR_INVALID_ARG;
+  if (cap < seer_gate_required_cap(dims, mode, k, density)) return SEER_ERR_CAPACITY;
+  return SEER_OK;
+}
+
+seer_status seer_gate(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype,
+                      const float* Wq, const float* Wk, int32_t h, float rope_theta,
+                      seer_select_mode mode, float T, int32_t k, float density, float* scores_out,
+                      int32_t* counts, int32_t* indices, int32_t cap, void* ws, size_t ws_bytes,
+                      seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !Wq || !Wk || !counts || !indices) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (h < 1 || h > 256 || (h % 4) != 0) return SEER_ERR_INVALID_ARG;
+  if (!std::isfinite(rope_theta)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16)) return SEER_ERR_INVALID_ARG;
+  s = check_select(dims, mode, T, k, density, cap);
+  if (s != SEER_OK) return s;
+  const GateWs w = gate_ws(dims, h);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+
+  uint8_t* base = (uint8_t*)ws;
+  float* qbar = (float*)(base + w.qbar);
+  float* kbar = (float*)(base + w.kbar);
+  float* qt = (float*)(base + w.qt);
+  float* kt = (float*)(base + w.kt);
+  float* logits = scores_out ? scores_out : (float*)(base + w.logits);
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  const int nb = n / seer::kBlock, G = Hq / Hkv;
+
+  SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st));
+  SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st));
+  // q~ = Wq[hq] qbar, k~ = Wk[g] kbar (batch z = b*H + head; weights by head)
+  SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
+                                 (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
+  SEER_CUDA(seer::launch_gemm_nt(kbar, Wk, kt, nb, h, 3 * d, (long long)nb * 3 * d,
+                                 (long long)h * 3 * d, (long long)nb * h, h, B * Hkv, Hkv, 0, 1,
+                                 1.0f, false, st));
+  if (rope_theta > 0.f) {
+    SEER_CUDA(seer::launch_rope(qt, (long long)B * Hq * nb, nb, h, rope_theta, st));
+    SEER_CUDA(seer::launch_rope(kt, (long long)B * Hkv * nb, nb, h, rope_theta, st));
+  }
+  // causal block logits q~_i . k~_j / sqrt(d), KV head of query head z%Hq
+  SEER_CUDA(seer::launch_gemm_nt(qt, kt, logits, nb, nb, h, (long long)nb * h, (long long)nb * h,
+                                 (long long)nb * nb, nb, B * Hq, Hq, Hkv, G,
+                                 (float)(1.0 / std::sqrt((double)d)), true, st));
+  SEER_CUDA(seer::launch_row_select(logits, scores_out, true, (long long)B * Hq * nb, nb, (int)mode,
+                                    T, k, density, counts, indices, cap, st));
+  return SEER_OK;
+}
+
+seer_status seer_gate_select(const seer_dims* dims, const float* scores, seer_select_mode mode,
+                             float T, int32_t k, float density, int32_t* counts, int32_t* indices,
+                             int32_t cap, seer_stream_t stream) {
+  if (!dims_ok(dims) || !scores || !counts || !indices) return SEER_ERR_INVALID_ARG;
+  if (dims->block != seer::kBlock) return SEER_ERR_UNSUPPORTED;
+  seer_status s = check_select(dims, mode, T, k, density, cap);
+  if (s != SEER_OK) return s;
+  const int nb = dims->n / seer::kBlock;
+  SEER_CUDA(seer::launch_row_select(scores, nullptr, false, (long long)dims->B * dims->Hq * nb, nb,
+                                    (int)mode, T, k, density, counts, indices, cap,
+                                    (cudaStream_t)stream));
+  return SEER_OK;
+}
+
+// ---------------------------------------------------------- sparse attn ---
+size_t seer_sparse_attn_workspace_size(const seer_dims* dims, seer_dtype dtype) {
+  if (!dims_ok(dims)) return 0;
+  return attn_ws(dims, dtype).total;
+}
+
+seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V,
+                             seer_dtype dtype, const int32_t* counts, const int32_t* indices,
+                             int32_t cap, float scale, void* O, float* lse, void* ws,
+                             size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !V || !counts || !indices || !O) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (cap < 1 || !(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return SEER_ERR_INVALID_ARG;
+  const AttnWs w = attn_ws(dims, dtype);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+  uint8_t* base = (uint8_t*)ws;
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  const void *q = Q, *k = K, *v = V;
+  if (dtype == SEER_FP32) {
+    SEER_CUDA(to_bf16(Q, base + w.q16, (long long)B * Hq * n * d, st));
+    SEER_CUDA(to_bf16(K, base + w.k16, (long long)B * Hkv * n * d, st));
+    SEER_CUDA(to_bf16(V, base + w.v16, (long long)B * Hkv * n * d, st));
+    q = base + w.q16;
+    k = base + w.k16;
+    v = base + w.v16;
+  }
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) ||
+      !make_tmap(&tmK, k, (long long)B * Hkv * n, d, 64) ||
+      !make_tmap(&tmV, v, (long long)B * Hkv * n, d, 64))
+    return cuda_fail(cudaErrorInvalidValue);
+  seer::AttnParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.d = d;
+  p.nb = n / seer::kBlock;
+  p.G = Hq / Hkv;
+  p.cap = cap;
+  p.total_units = (long long)B * Hq * p.nb;
+  p.counts = counts;
+  p.indices = indices;
+  p.O = O;
+  p.lse = lse;
+  p.out_fp32 = dtype == SEER_FP32;
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+  p.scale_log2 = (float)(sc * 1.4426950408889634);
+  seer::WsHeader* hdr = (seer::WsHeader*)ws;
+  p.status = &hdr->status;
+  p.work_counter = &hdr->work_counter;
+  p.timeout_ns = kTimeoutNs;
+  SEER_CUDA(seer::launch_sparse_attn(tmQ, tmK, tmV, p, num_sms(), st));
+  return SEER_OK;
+}
+
+// -------------------------------------------------------------- blockmax --
+size_t seer_blockmax_workspace_size(const seer_dims* dims, seer_dtype dtype) {
+  if (!dims_ok(dims)) return 0;
+  return bmax_ws(dims, dtype, num_sms()).total;
+}
+
+seer_status seer_attn_blockmax(const seer_dims* dims, const void* Q, const void* K,
+                               seer_dtype dtype, float scale, float* map_out, float* lse_out,
+                               void* ws, size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !map_out) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16)) return SEER_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  const BmaxWs w = bmax_ws(dims, dtype, sms);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+  uint8_t* base = (uint8_t*)ws;
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  const void *q = Q, *k = K;
+  if (dtype == SEER_FP32) {
+    SEER_CUDA(to_bf16(Q, base + w.q16, (long long)B * Hq * n * d, st));
+    SEER_CUDA(to_bf16(K, base + w.k16, (long long)B * Hkv * n * d, st));
+    q = base + w.q16;
+    k = base + w.k16;
+  }
+  CUtensorMap tmQ, tmK;
+  if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 128) ||
+      !make_tmap(&tmK, k, (long long)B * Hkv * n, d, 128))
+    return cuda_fail(cudaErrorInvalidValue);
+  seer::BmaxParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.d = d;
+  p.nb = n / seer::kBlock;
+  p.G = Hq / Hkv;
+  p.npairs = (p.nb + 1) / 2;
+  p.total_units = (long long)B * Hq * p.npairs;
+  p.map = map_out;
+  p.lse = lse_out;
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+  p.scale_log2 = (float)(sc * 1.4426950408889634);
+  p.r = (float*)(base + w.r);
+  seer::WsHeader* hdr = (seer::WsHeader*)ws;
+  p.status = &hdr->status;
+  p.work_counter = &hdr->work_counter;
+  p.timeout_ns = kTimeoutNs;
+  SEER_CUDA(seer::launch_blockmax(tmQ, tmK, p, w.ctas, st));
+  return SEER_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,396 @@
+// blockmax.cu -- the max-pooled attention-probability map that SeerAttention's
+// gate is distilled against, for sm_100a (B200).
+//
+// Paper: "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs";
+// paper-graph summary page, section 3.4, "Ground truth generation"
+// (gt = MaxPool2D_{BxB}(softmax(Q K^T / sqrt(d)))) and "The customized
+// training kernel" / Figure 10: a first pass over the key blocks forms the
+// online-softmax statistics and keeps each row's raw maximum per key block,
+// r_ij = rowmax(S_ij); a second pass rescales the kept maxima into
+// probabilities a_ij = exp(r_ij - m_i) / l_i and takes the column maximum
+// over the rows of the block.
+//
+// B200 design:
+//  * A unit is one query head and two consecutive 64-row query blocks
+//    (i0 = 2m, i1 = 2m+1): a 128-row tile, so every tcgen05 MMA is
+//    M = 128 x N = 128 (two key blocks per step), both operands from 128-byte
+//    swizzled shared memory loaded by TMA (no multicast), S in TMEM.
+//  * Two softmax warpgroups split the 128 score columns (one key block each);
+//    each thread owns one query row, keeps its own (max, sum) with a lazily
+//    raised running max, and stores its per-key-block raw maxima to a per-CTA
+//    scratch slot (L2-resident, rewritten by every unit).
+//  * The second pass runs in the unit's epilogue: every thread reads back the
+//    maxima it stored, turns them into probabilities with the final
+//    log-sum-exp, and a shuffle reduce-scatter takes the maximum over the 64
+//    rows of each query block.
+//  * Warp roles (384 threads): warp 0 schedules units and loads Q, warp 1
+//    loads K pairs, warp 2 issues the MMAs, warps 4..7 and 8..11 are the two
+//    softmax warpgroups.  All waits are bounded.
+#include <cstdint>
+
+#include "blockmax.cuh"
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace seer {
+
+namespace bmax {
+constexpr int kThreads = 384;
+constexpr int kNK = 4;
+constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 dims x bf16
+constexpr uint32_t kOffQ = 0;           // 2 x 32 KB
+constexpr uint32_t kOffK = 2 * kTileBytes;
+constexpr uint32_t kSmemTiles = kOffK + kNK * kTileBytes;  // 192 KB
+constexpr uint32_t kTmemCols = 256;                        // S x 2 (128 cols each)
+constexpr float kRaise = 8.0f;
+
+struct Ctrl {
+  uint64_t unit_full[2], unit_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kNK], k_empty[kNK];
+  uint64_t s_full[2], s_free[2];
+  uint64_t wg[2], both, fin;
+  int unit_w[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  float m_part[2][128], l_part[2][128];
+  float lse2[128];
+  float red[2][4][32];
+};
+constexpr uint32_t kSmemAlloc = kSmemTiles + (uint32_t)sizeof(Ctrl);
+}  // namespace bmax
+
+namespace {
+
+struct Sync {
+  uint64_t* bar;
+  volatile int* abort;
+  uint32_t* status;
+  uint64_t tmo;
+  uint32_t phase;
+  __device__ __forceinline__ bool sync(int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase & 1, abort, status, tmo);
+    ++phase;
+    return ok;
+  }
+};
+
+struct BUnit {
+  int b, hq, g, m;
+};
+
+__device__ __forceinline__ BUnit decode(const BmaxParams& p, int w) {
+  BUnit u;
+  const int per_bg = p.npairs * p.G;
+  const int bg = w / per_bg, rem = w % per_bg;
+  u.b = bg / p.Hkv;
+  u.g = bg % p.Hkv;
+  u.m = p.npairs - 1 - rem / p.G;
+  u.hq = u.g * p.G + rem % p.G;
+  return u;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(bmax::kThreads, 1)
+    blockmax_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const BmaxParams p) {
+  using namespace bmax;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) record_status(p.status, kDevBadSchedule, smem_u32(smem));
+    return;
+  }
+  Ctrl& C = *reinterpret_cast<Ctrl*>(smem + kSmemTiles);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  volatile int* abort_p = &C.abort_flag;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    C.abort_flag = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&C.unit_full[s], 1);
+      mbar_init(&C.unit_empty[s], 2 + 8);  // K loader, MMA, 8 softmax warps
+      mbar_init(&C.q_full[s], 1);
+      mbar_init(&C.q_empty[s], 1);
+      mbar_init(&C.s_full[s], 1);
+      mbar_init(&C.s_free[s], 8);
+      mbar_init(&C.wg[s], 4);
+    }
+    for (int s = 0; s < kNK; ++s) {
+      mbar_init(&C.k_full[s], 1);
+      mbar_init(&C.k_empty[s], 1);
+    }
+    mbar_init(&C.both, 8);
+    mbar_init(&C.fin, 1);
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&C.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = C.tmem_base;
+  const int dpanels = p.d / 64;
+  const uint32_t tile_bytes = 128u * p.d * 2u;
+
+  if (warp == 0) {
+    // ------------------------------------------------ scheduler + Q loads --
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      int u_idx = 0;
+      for (;;) {
+        const int slot = u_idx & 1;
+        if (u_idx >= 2 && !mbar_wait(&C.unit_empty[slot], ((u_idx >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+        int w = (int)atomicAdd(p.work_counter, 1u);
+        if (w >= p.total_units || *abort_p) w = -1;
+        C.unit_w[slot] = w;
+        mbar_arrive(&C.unit_full[slot]);
+        if (w < 0) break;
+        const BUnit u = decode(p, w);
+        if (u_idx >= 2 && !mbar_wait(&C.q_empty[slot], ((u_idx >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+        mbar_arrive_expect_tx(&C.q_full[slot], tile_bytes);
+        const int row = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.m * 128);
+        for (int pn = 0; pn < dpanels; ++pn)
+          tma_load_2d(smem + kOffQ + slot * kTileBytes + pn * 16384, &tmQ, &C.q_full[slot], pn * 64, row);
+        ++u_idx;
+      }
+      for (int k = 0; k < 2 && k < u_idx; ++k) {
+        const int uu = u_idx - 1 - k;
+        mbar_wait(&C.q_full[uu & 1], (uu >> 1) & 1, abort_p, nullptr, 20000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- K loads ---
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      int u_idx = 0, step = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = u_idx & 1;
+        if (!mbar_wait(&C.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
+        const int w = C.unit_w[slot];
+        mbar_arrive(&C.unit_empty[slot]);
+        if (w < 0) break;
+        ++u_idx;
+        const BUnit u = decode(p, w);
+        const long long row0 = ((long long)u.b * p.Hkv + u.g) * p.n;
+        for (int s = 0; s <= u.m; ++s, ++step) {
+          const int ks = step % kNK;
+          if (step >= kNK && !mbar_wait(&C.k_empty[ks], ((step / kNK) - 1) & 1, abort_p, p.status, tmo)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&C.k_full[ks], tile_bytes);
+          for (int pn = 0; pn < dpanels; ++pn)
+            tma_load_2d(smem + kOffK + ks * kTileBytes + pn * 16384, &tmK, &C.k_full[ks], pn * 64,
+                        (int)(row0 + (long long)s * 128));
+        }
+      }
+      for (int k = 0; k < kNK && k < step; ++k) {
+        const int st = step - 1 - k;
+        mbar_wait(&C.k_full[st % kNK], (st / kNK) & 1, abort_p, nullptr, 20000000ull);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t sbase = smem_u32(smem);
+      const int ksteps = p.d / 16;
+      int u_idx = 0, step = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = u_idx & 1;
+        if (!mbar_wait(&C.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
+        const int w = C.unit_w[slot];
+        mbar_arrive(&C.unit_empty[slot]);
+        if (w < 0) break;
+        const BUnit u = decode(p, w);
+        if (!mbar_wait(&C.q_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
+        const uint32_t qa = sbase + kOffQ + slot * kTileBytes;
+        for (int s = 0; s <= u.m; ++s) {
+          const int g = step + s;
+          const int ks = g % kNK;
+          if (!mbar_wait(&C.k_full[ks], (g / kNK) & 1, abort_p, p.status, tmo)) { ok = false; break; }
+          if (g >= 2 && !mbar_wait(&C.s_free[g & 1], ((g - 2) >> 1) & 1, abort_p, p.status, tmo)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ka = sbase + kOffK + ks * kTileBytes;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + (g & 1) * 128, make_sw128_desc(qa + off, 16, 1024),
+                        make_sw128_desc(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&C.s_full[g & 1]);
+          mma_commit(&C.k_empty[ks]);
+        }
+        if (!ok) break;
+        mma_commit(&C.q_empty[slot]);
+        step += u.m + 1;
+        ++u_idx;
+      }
+      mma_commit(&C.fin);
+      mbar_wait(&C.fin, 0, abort_p, nullptr, 20000000ull);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------ softmax WGs ---
+    const int wgi = (warp - 4) / 4;   // 0: even key block of a step, 1: odd
+    const int ww = (warp - 4) % 4;    // TMEM sub-partition
+    const int row = ww * 32 + lane;   // 0..127
+    const int half = row >> 6, rloc = row & 63;
+    const uint32_t lane_addr = tmem + ((uint32_t)(ww * 32) << 16) + wgi * 64;
+    const float c = p.scale_log2;
+    Sync wgs{&C.wg[wgi], abort_p, p.status, tmo, 0};
+    Sync both{&C.both, abort_p, p.status, tmo, 0};
+    float* rslot = p.r + (long long)blockIdx.x * 128 * p.nb;
+    int u_idx = 0, step = 0;
+    for (;;) {
+      const int slot = u_idx & 1;
+      if (!mbar_wait(&C.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
+      const int w = C.unit_w[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&C.unit_empty[slot]);
+      if (w < 0) break;
+      ++u_idx;
+      const BUnit u = decode(p, w);
+      const int irow = 2 * u.m + half;        // query block of this row
+      const bool row_valid = irow < p.nb;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int s = 0; s <= u.m; ++s) {
+        const int g = step + s;
+        const int j = 2 * s + wgi;           // key block of these columns
+        if (!mbar_wait(&C.s_full[g & 1], (g >> 1) & 1, abort_p, p.status, tmo)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_addr + (g & 1) * 128, r0);
+        tmem_ld32(lane_addr + (g & 1) * 128 + 32, r1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&C.s_free[g & 1]);
+        if (j > irow || !row_valid) continue;  // key block entirely in the future
+        float x[64];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          x[q] = __uint_as_float(r0[q]) * c;
+          x[q + 32] = __uint_as_float(r1[q]) * c;
+        }
+        if (j == irow) {
+#pragma unroll
+          for (int q = 0; q < 64; ++q) x[q] = q > rloc ? -INFINITY : x[q];
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int q = 1; q < 64; ++q) mx = fmaxf(mx, x[q]);
+        rslot[(long long)j * 128 + row] = mx;
+        if (mx > m_run + kRaise) {
+          l_run *= ex2_approx(m_run - mx);
+          m_run = mx;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) sum += ex2_approx(x[q] - m_run);
+        l_run += sum;
+      }
+      if (!ok) break;
+      // ---- combine the two warpgroups' statistics into the row's lse (log2)
+      C.m_part[wgi][row] = m_run;
+      C.l_part[wgi][row] = l_run;
+      if (!both.sync(lane)) break;
+      float lse2 = -INFINITY;
+      {
+        const float m0 = C.m_part[0][row], m1 = C.m_part[1][row];
+        const float mm = fmaxf(m0, m1);
+        const float l = (m0 > -INFINITY ? C.l_part[0][row] * ex2_approx(m0 - mm) : 0.f) +
+                        (m1 > -INFINITY ? C.l_part[1][row] * ex2_approx(m1 - mm) : 0.f);
+        lse2 = mm + log2f(l);
+      }
+      if (wgi == 0 && row_valid && p.lse)
+        p.lse[((long long)u.b * p.Hq + u.hq) * p.n + (long long)irow * 64 + rloc] = lse2 * 0.6931471805599453f;
+      // ---- second pass: probabilities of the kept maxima, max over rows ----
+      // this warpgroup owns the key blocks j = 2s + wgi that it stored itself
+      const int nsj = u.m + 1;
+      for (int s0 = 0; s0 < nsj && ok; s0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int j = 2 * (s0 + k) + wgi;
+          v[k] = (s0 + k < nsj && j <= irow && row_valid) ? ex2_approx(rslot[(long long)j * 128 + row] - lse2) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const bool up = lane & 16;
+          const float send = up ? v[k] : v[k + 16], keep = up ? v[k + 16] : v[k];
+          v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const bool up = lane & 8;
+          const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
+          v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const bool up = lane & 4;
+          const float send = up ? v[k] : v[k + 4], keep = up ? v[k + 4] : v[k];
+          v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const bool up = lane & 2;
+          const float send = up ? v[k] : v[k + 2], keep = up ? v[k + 2] : v[k];
+          v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+        }
+        {
+          const bool up = lane & 1;
+          const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+          v[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+        }
+        // lane holds the max over this warp's 32 rows for s = s0 + lane
+        C.red[wgi][ww][lane] = v[0];
+        if (!wgs.sync(lane)) { ok = false; break; }
+        if (ww == 0 || ww == 2) {
+          const int hb = ww >> 1;  // 0: block i0 (warps 0,1), 1: block i1 (warps 2,3)
+          const int ib = 2 * u.m + hb;
+          const int s = s0 + lane;
+          const int j = 2 * s + wgi;
+          if (ib < p.nb && s < nsj && j <= ib) {
+            const float val = fmaxf(C.red[wgi][ww][lane], C.red[wgi][ww + 1][lane]);
+            p.map[(((long long)u.b * p.Hq + u.hq) * p.nb + ib) * p.nb + j] = val;
+          }
+        }
+        if (!wgs.sync(lane)) { ok = false; break; }
+      }
+      if (!ok) break;
+      // keep the statistics area until both warpgroups have read it
+      if (!both.sync(lane)) break;
+      step += u.m + 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, bmax::kTmemCols);
+}
+
+cudaError_t launch_blockmax(const CUtensorMap& tmQ, const CUtensorMap& tmK, const BmaxParams& p,
+                            int ctas, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(blockmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bmax::kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  // entries above the diagonal are 0; the kernel writes j <= i only
+  e = cudaMemsetAsync(p.map, 0, sizeof(float) * (size_t)p.B * p.Hq * p.nb * p.nb, st);
+  if (e != cudaSuccess) return e;
+  long long grid = p.total_units < ctas ? p.total_units : ctas;
+  if (grid < 1) grid = 1;
+  blockmax_kernel<<<(unsigned)grid, bmax::kThreads, bmax::kSmemAlloc, st>>>(tmQ, tmK, p);
+  return cudaGetLastError();
+}
+
+}  // namespace seer

@@ -54,9 +54,10 @@ def _load():
         lib.orc_project.argtypes = [P, P, I, I, I, I, I, P]
         lib.orc_block_rope.argtypes = [P, I, I, I, D, I]
         lib.orc_gate_scores.argtypes = [P, P, I, I, I, I, I, D, P]
-        lib.orc_select_threshold.argtypes = [P, I, I, F, P, P, I]
+        lib.orc_select_threshold.argtypes = [P, I, I, F, P, P, I, P]
         lib.orc_select_threshold.restype = I
-        lib.orc_select_topk.argtypes = [P, I, I, ctypes.c_int, I, F, P, P, I]
+        lib.orc_select_topk.argtypes = [P, I, I, ctypes.c_int, I, F, P, P, I, P]
+        lib.orc_gate_scores_units.argtypes = [P, P, I, I, I, I, I, D, P, I, P]
         lib.orc_select_topk.restype = I
         lib.orc_topk_count.argtypes = [I, ctypes.c_int, I, F]
         lib.orc_topk_count.restype = I
@@ -187,11 +188,43 @@ def select(scores, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
     idx = np.full((B, Hq, nb, cap), -1, np.int32)
     lib = _load()
     if mode == MODE_THRESHOLD:
-        worst = lib.orc_select_threshold(_p(s), rows, nb, float(T), _p(counts), _p(idx), cap)
+        worst = lib.orc_select_threshold(_p(s), rows, nb, float(T), _p(counts), _p(idx), cap, None)
     else:
         worst = lib.orc_select_topk(_p(s), rows, nb, int(mode), int(k), float(density),
-                                    _p(counts), _p(idx), cap)
+                                    _p(counts), _p(idx), cap, None)
     return counts, idx, int(worst)
+
+
+def select_rows(rows_scores, row_i, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
+                cap: int | None = None):
+    """As select, for a stack of score rows [R, nb] whose query blocks are
+    given by row_i [R].  Returns (counts [R], idx [R, cap])."""
+    s = _f64(rows_scores)
+    R, nb = s.shape
+    ri = np.ascontiguousarray(row_i, dtype=np.int64)
+    cap = nb if cap is None else cap
+    counts = np.zeros(R, np.int32)
+    idx = np.full((R, cap), -1, np.int32)
+    lib = _load()
+    if mode == MODE_THRESHOLD:
+        lib.orc_select_threshold(_p(s), R, nb, float(T), _p(counts), _p(idx), cap, _p(ri))
+    else:
+        lib.orc_select_topk(_p(s), R, nb, int(mode), int(k), float(density), _p(counts), _p(idx),
+                            cap, _p(ri))
+    return counts, idx
+
+
+def gate_scores_units(qt, kt, d: int, units) -> np.ndarray:
+    """Eq. 1 for the listed rows u = (b*Hq + hq)*nb + i: [len(units), nb]."""
+    q = _f64(qt)
+    k = _f64(kt)
+    B, Hq, nb, h = q.shape
+    Hkv = k.shape[1]
+    u = np.ascontiguousarray(units, dtype=np.int64)
+    out = np.empty((len(u), nb), np.float64)
+    _load().orc_gate_scores_units(_p(q), _p(k), B, Hq, Hkv, nb, h, 1.0 / math.sqrt(d), _p(u),
+                                  len(u), _p(out))
+    return out
 
 
 def topk_count(i: int, mode: int, k: int = 0, density: float = 0.0) -> int:

@@ -155,23 +155,60 @@ void orc_gate_scores(const double *qt, const double *kt, i64 B, i64 Hq,
             }
 }
 
+
+/* Eq. 1 for listed rows only: unit u = (b*Hq + hq)*nb + i; out is [nunits, nb]
+ * (entries j > i are 0).  Same arithmetic as orc_gate_scores.              */
+void orc_gate_scores_units(const double *qt, const double *kt, i64 B, i64 Hq,
+                           i64 Hkv, i64 nb, i64 h, double scale,
+                           const i64 *units, i64 nunits, double *out)
+{
+    (void)B;
+    i64 G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i64 u = 0; u < nunits; ++u) {
+        i64 unit = units[u];
+        i64 i = unit % nb, bhq = unit / nb;
+        i64 b = bhq / Hq, hq = bhq % Hq;
+        const double *q = qt + ((b * Hq + hq) * nb + i) * h;
+        const double *kbase = kt + (b * Hkv + hq / G) * nb * h;
+        double *row = out + u * nb;
+        double mx = -INFINITY;
+        for (i64 j = 0; j <= i; ++j) {
+            double z = 0.0;
+            for (i64 c = 0; c < h; ++c) z += q[c] * kbase[j * h + c];
+            z *= scale;
+            row[j] = z;
+            if (z > mx) mx = z;
+        }
+        double sum = 0.0;
+        for (i64 j = 0; j <= i; ++j) {
+            row[j] = exp(row[j] - mx);
+            sum += row[j];
+        }
+        for (i64 j = 0; j <= i; ++j) row[j] /= sum;
+        for (i64 j = i + 1; j < nb; ++j) row[j] = 0.0;
+    }
+}
+
 /* ---------------------------------------------------------------------- */
 /* Binary mask generation (summary page, section 3.4 "Generating the binary
  * block mask"; rebuttal section 3.3).  The mask of row i is returned as the
  * ascending list of active key blocks j <= i.  rows = B*Hq*nb rows of
- * length nb; row r is query block i = r % nb.  idx is [rows, cap].
+ * length nb; row r is query block i = r % nb, or row_i[r] when row_i is
+ * not NULL.  idx is [rows, cap].
  * Return value: the largest count of any row (the caller checks it against
  * cap; rows whose count exceeds cap are truncated to cap entries).         */
 
 /* Method 2, thresholding: active iff score > T (strict).  T is an fp32 value
  * so that supplied fp32 scores are compared exactly as an fp32 kernel does. */
 i64 orc_select_threshold(const double *scores, i64 rows, i64 nb, float T,
-                         int32_t *counts, int32_t *idx, i64 cap)
+                         int32_t *counts, int32_t *idx, i64 cap,
+                         const i64 *row_i)
 {
     i64 worst = 0;
 #pragma omp parallel for schedule(static) reduction(max : worst)
     for (i64 r = 0; r < rows; ++r) {
-        i64 i = r % nb, c = 0;
+        i64 i = row_i ? row_i[r] : r % nb, c = 0;
         const double *s = scores + r * nb;
         for (i64 j = 0; j <= i; ++j)
             if (s[j] > (double)T) {
@@ -221,7 +258,8 @@ static int int_cmp(const void *pa, const void *pb)
 /* Method 1, TopK: the k_i largest scores of row i (ties: lower j first),
  * returned in ascending j.                                                 */
 i64 orc_select_topk(const double *scores, i64 rows, i64 nb, int mode, i64 k,
-                    float density, int32_t *counts, int32_t *idx, i64 cap)
+                    float density, int32_t *counts, int32_t *idx, i64 cap,
+                    const i64 *row_i)
 {
     i64 worst = 0;
 #pragma omp parallel reduction(max : worst)
@@ -229,7 +267,7 @@ i64 orc_select_topk(const double *scores, i64 rows, i64 nb, int mode, i64 k,
         cand_t *buf = (cand_t *)malloc(sizeof(cand_t) * (size_t)nb);
 #pragma omp for schedule(static)
         for (i64 r = 0; r < rows; ++r) {
-            i64 i = r % nb;
+            i64 i = row_i ? row_i[r] : r % nb;
             const double *s = scores + r * nb;
             for (i64 j = 0; j <= i; ++j) { buf[j].s = s[j]; buf[j].j = j; }
             qsort(buf, (size_t)(i + 1), sizeof(cand_t), cand_cmp);

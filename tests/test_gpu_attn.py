@@ -1,0 +1,169 @@
+"""GPU parity of seer_sparse_attn against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import learned_block_sparse_seer_b200 as seer
+import oracle
+from learned_block_sparse_seer_b200 import synth
+
+from gpu_common import (LSE_TOL_FP32_INPUT, check_lse, check_o, inputs, sample_units, to_dev,
+                        unit_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(Q, K, V, counts, idx, **kw):
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    cd = torch.as_tensor(counts, dtype=torch.int32).cuda()
+    idd = torch.as_tensor(idx, dtype=torch.int32).cuda()
+    ws = torch.empty(seer.sparse_attn_workspace_size(*Q.shape[:2], K.shape[1], *Q.shape[2:],
+                                                     0 if Q.dtype == torch.bfloat16 else 1),
+                     dtype=torch.uint8, device="cuda")
+    O, lse = seer.seer_sparse_attn(Qd, Kd, Vd, cd, idd, workspace=ws, **kw)
+    assert seer.seer_workspace_status(ws) == 0
+    return O.cpu(), lse.cpu()
+
+
+def _oracle_lists(w, mode, **sel):
+    _, Q, K, V, Wq, Wk = inputs(w.name)
+    s = oracle.gate(Q, K, Wq, Wk)
+    c, ix, _ = oracle.select(s, mode, **sel)
+    return c, ix
+
+
+def test_tiny_fp32_threshold():
+    w, Q, K, V, Wq, Wk = inputs("tiny")
+    c, ix = _oracle_lists(w, oracle.MODE_THRESHOLD, T=5e-4)
+    O, lse = _run(Q, K, V, c, ix)
+    O_ref, lse_ref = oracle.sparse_attn(Q, K, V, c, ix)
+    check_o(O.double().numpy(), O_ref)
+    check_lse(lse.double().numpy(), lse_ref, LSE_TOL_FP32_INPUT)
+
+
+def test_tiny_bf16_topk():
+    w, Q, K, V, Wq, Wk = inputs("tiny")
+    Qb, Kb, Vb = (t.to(torch.bfloat16) for t in (Q, K, V))
+    s = oracle.gate(Qb, Kb, Wq, Wk)
+    for k in (1, 2, 3, 8):
+        c, ix, _ = oracle.select(s, oracle.MODE_TOPK_K, k=k)
+        O, lse = _run(Qb, Kb, Vb, c, ix)
+        O_ref, lse_ref = oracle.sparse_attn(Qb, Kb, Vb, c, ix)
+        check_o(O.double().numpy(), O_ref)
+        check_lse(lse.double().numpy(), lse_ref)
+
+
+def test_layer8k_threshold_sampled():
+    w, Q, K, V, Wq, Wk = inputs("layer8k")
+    Qd, Kd, Wqd, Wkd = to_dev(Q, K, Wq, Wk)
+    cd, idd = seer.seer_gate(Qd, Kd, Wqd, Wkd, "threshold", T=5e-4)
+    c, ix = cd.cpu().numpy(), idd.cpu().numpy()
+    O, lse = _run(Q, K, V, c, ix)
+    units = sample_units(w.B, w.Hq, w.nb, 40, seed=8)
+    O_ref, lse_ref = oracle.sparse_attn_units(Q, K, V, c, ix, units)
+    check_o(unit_rows(O, units, w.nb).double().numpy(), O_ref)
+    check_lse(unit_rows(lse, units, w.nb).double().numpy(), lse_ref)
+
+
+@pytest.mark.parametrize("name,rho", [("layer32k", 0.1), ("layer128k", 0.1), ("layer128k", 0.5)])
+def test_full_size_density_sampled(name, rho):
+    w, Q, K, V, Wq, Wk = inputs(name)
+    Qd, Kd, Wqd, Wkd = to_dev(Q, K, Wq, Wk)
+    cd, idd = seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=rho)
+    c, ix = cd.cpu().numpy(), idd.cpu().numpy()
+    O, lse = _run(Q, K, V, c, ix)
+    assert torch.isfinite(lse).all() and torch.isfinite(O.float()).all()
+    units = sample_units(w.B, w.Hq, w.nb, 24, seed=int(rho * 100))
+    O_ref, lse_ref = oracle.sparse_attn_units(Q, K, V, c, ix, units)
+    check_o(unit_rows(O, units, w.nb).double().numpy(), O_ref)
+    check_lse(unit_rows(lse, units, w.nb).double().numpy(), lse_ref)
+
+
+def test_all_ones_mask_equals_dense():
+    w = synth.custom("dense", 1, 8, 2, 64 * 40, 128, 128, "bf16", "layer", 12)
+    Q, K, V = synth.make_qkv(w)
+    c, ix = oracle.dense_lists(w.B, w.Hq, w.nb)
+    O, lse = _run(Q, K, V, c, ix)
+    O_ref, lse_ref = oracle.sparse_attn(Q, K, V, c, ix)
+    check_o(O.double().numpy(), O_ref)
+    check_lse(lse.double().numpy(), lse_ref)
+    # cross-check with the library SDPA of the same device
+    G = w.Hq // w.Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.cuda(), K.cuda().repeat_interleave(G, 1), V.cuda().repeat_interleave(G, 1), is_causal=True)
+    assert (ref.float().cpu() - O.float()).abs().max() < 2e-2
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,nb,d", [(2, 4, 4, 5, 128), (1, 2, 1, 1, 128), (3, 6, 2, 9, 64),
+                                            (1, 4, 1, 33, 128)])
+def test_edge_cases(B, Hq, Hkv, nb, d):
+    """Empty rows, diagonal-only rows, single-block lists, odd counts, full
+    rows, batch > 1, MHA, d = 64, a single 64-token sequence."""
+    w = synth.custom("edge", B, Hq, Hkv, 64 * nb, d, 16, "bf16", "layer", 20 + nb)
+    Q, K, V = synth.make_qkv(w)
+    rng = np.random.default_rng(nb)
+    cap = nb + 3
+    counts = np.zeros((B, Hq, nb), np.int32)
+    idx = np.full((B, Hq, nb, cap), -1, np.int32)
+    for b, h, i in np.ndindex(B, Hq, nb):
+        kind = (b + h + i) % 5
+        if kind == 0:
+            lst = []                               # empty row
+        elif kind == 1:
+            lst = [i]                              # diagonal only
+        elif kind == 2:
+            lst = list(range(i + 1))               # full causal row
+        elif kind == 3:
+            lst = [0]                              # sink only
+        else:
+            m = rng.integers(1, i + 2)
+            lst = sorted(rng.choice(i + 1, size=m, replace=False).tolist())
+        counts[b, h, i] = len(lst)
+        idx[b, h, i, :len(lst)] = lst
+    O, lse = _run(Q, K, V, counts, idx)
+    O_ref, lse_ref = oracle.sparse_attn(Q, K, V, counts, idx)
+    check_o(O.double().numpy(), O_ref)
+    check_lse(lse.double().numpy(), lse_ref)
+    empty = counts == 0
+    assert torch.all(O.view(B, Hq, nb, 64, d)[torch.as_tensor(empty)] == 0)
+
+
+def test_bad_lists_are_flagged_not_followed():
+    """Out-of-range counts and indices are clamped by the kernel and reported
+    as SEER_ERR_DEVICE_CHECK; nothing outside the tensors is read."""
+    w = synth.custom("bad", 1, 2, 1, 64 * 4, 64, 16, "bf16", "layer", 3)
+    Q, K, V = synth.make_qkv(w)
+    cap = 4
+    counts = np.array([[[1, 2, 3, 9], [1, 1, 1, 1]]], np.int32)       # 9 > cap
+    idx = np.zeros((1, 2, 4, cap), np.int32)
+    idx[0, 0, 1, :2] = [0, 1]
+    idx[0, 0, 2, :3] = [0, 2, 1]                                       # not ascending
+    idx[0, 1, 0, 0] = 3                                                # j > i
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    ws = torch.empty(seer.sparse_attn_workspace_size(1, 2, 1, 256, 64), dtype=torch.uint8,
+                     device="cuda")
+    seer.seer_sparse_attn(Qd, Kd, Vd, torch.as_tensor(counts).cuda(), torch.as_tensor(idx).cuda(),
+                          workspace=ws)
+    assert seer.seer_workspace_status(ws) == 6  # SEER_ERR_DEVICE_CHECK
+
+
+def test_repeat_runs_bitwise_identical():
+    w, Q, K, V, Wq, Wk = inputs("layer8k")
+    c, ix = _oracle_lists(w, oracle.MODE_TOPK_DENSITY, density=0.2)
+    O1, l1 = _run(Q, K, V, c, ix)
+    O2, l2 = _run(Q, K, V, c, ix)
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+
+
+def test_rejects_bad_arguments():
+    w, Q, K, V, Wq, Wk = inputs("tiny")
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    c = torch.ones(1, 2, 8, dtype=torch.int32, device="cuda")
+    ix = torch.zeros(1, 2, 8, 1, dtype=torch.int32, device="cuda")
+    with pytest.raises(seer.SeerError) as e:
+        seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, workspace=torch.empty(8, dtype=torch.uint8,
+                                                                       device="cuda"))
+    assert e.value.status in (7,)
+    with pytest.raises(seer.SeerError) as e:
+        seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, scale=-1.0)
+    assert e.value.status == 1

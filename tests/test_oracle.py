@@ -438,3 +438,19 @@ def test_synth_is_deterministic_and_shaped():
     # the sink block carries the planted shift: its mean key norm is larger
     kb = K.float().view(1, 2, 16, 64, 32).mean(3).norm(dim=-1)
     assert torch.all(kb[:, :, 0] > 2.0)
+
+
+def test_unit_subset_entry_points_agree_with_full_ones():
+    qt, kt = _gate_inputs(seed=60, B=2, Hq=4, Hkv=2, nb=11, h=8)
+    full = oracle.gate_scores(qt, kt, 64)
+    units = [0, 5, 11 + 10, 3 * 11 + 7, 8 * 11 - 1]
+    rows = oracle.gate_scores_units(qt, kt, 64, units)
+    np.testing.assert_array_equal(rows, full.reshape(-1, 11)[units])
+    row_i = np.array([u % 11 for u in units])
+    for mode, kw in ((oracle.MODE_THRESHOLD, dict(T=0.09)), (oracle.MODE_TOPK_K, dict(k=3)),
+                     (oracle.MODE_TOPK_DENSITY, dict(density=0.4))):
+        c, ix, _ = oracle.select(full, mode, **kw)
+        cr, ir = oracle.select_rows(rows, row_i, mode, **kw)
+        np.testing.assert_array_equal(cr, c.reshape(-1)[units])
+        for r, u in enumerate(units):
+            np.testing.assert_array_equal(ir[r, :cr[r]], ix.reshape(-1, 11)[u, :cr[r]])
