@@ -83,6 +83,11 @@ bool make_tmap(CUtensorMap* tm, const void* base, long long rows, int d, int box
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over [rows, 64] (128-byte rows) with a box of box_rows rows.
+bool make_tmap_rows(CUtensorMap* tm, const void* base, long long rows, int box_rows) {
+  return make_tmap(tm, base, rows, 64, box_rows);
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -121,17 +126,16 @@ GateWs gate_ws(const seer_dims* d, int h) {
 }
 
 struct AttnWs {
-  size_t q16, k16, v16, total;
+  size_t q16, kv, total;
 };
 
+// fp32 Q converted to bf16 (fp32 inputs only), then the K/V block records
+// (2 * B * Hkv * n * d bf16, K^T and V of each 64-key block together).
 AttnWs attn_ws(const seer_dims* d, seer_dtype dt) {
   seer::WsCarver c;
-  AttnWs w{0, 0, 0, 0};
-  if (dt == SEER_FP32) {
-    w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
-    w.k16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
-    w.v16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
-  }
+  AttnWs w{0, 0, 0};
+  if (dt == SEER_FP32) w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
+  w.kv = c.take(2ull * 2ull * d->B * d->Hkv * d->n * d->d);
   w.total = c.off;
   return w;
 }
@@ -330,19 +334,16 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   if (s != SEER_OK) return s;
   uint8_t* base = (uint8_t*)ws;
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
-  const void *q = Q, *k = K, *v = V;
+  const void* q = Q;
   if (dtype == SEER_FP32) {
     SEER_CUDA(to_bf16(Q, base + w.q16, (long long)B * Hq * n * d, st));
-    SEER_CUDA(to_bf16(K, base + w.k16, (long long)B * Hkv * n * d, st));
-    SEER_CUDA(to_bf16(V, base + w.v16, (long long)B * Hkv * n * d, st));
     q = base + w.q16;
-    k = base + w.k16;
-    v = base + w.v16;
   }
-  CUtensorMap tmQ, tmK, tmV;
+  const long long records = (long long)B * Hkv * (n / seer::kBlock);
+  SEER_CUDA(seer::launch_kv_tiles(K, V, dtype == SEER_FP32, base + w.kv, records, n, d, st));
+  CUtensorMap tmQ, tmKV;
   if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) ||
-      !make_tmap(&tmK, k, (long long)B * Hkv * n, d, 64) ||
-      !make_tmap(&tmV, v, (long long)B * Hkv * n, d, 64))
+      !make_tmap_rows(&tmKV, base + w.kv, records * 2 * d, 2 * d))
     return cuda_fail(cudaErrorInvalidValue);
   seer::AttnParams p;
   p.B = B;
@@ -365,7 +366,8 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.status = &hdr->status;
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
-  SEER_CUDA(seer::launch_sparse_attn(tmQ, tmK, tmV, p, num_sms(), st));
+  p.trace = reinterpret_cast<unsigned long long*>(hdr->pad + 4);  // 16 x u64 in the header
+  SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
   return SEER_OK;
 }
 

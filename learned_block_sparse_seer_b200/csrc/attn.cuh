@@ -18,11 +18,18 @@ struct AttnParams {
   uint32_t* status;          // workspace status word
   uint32_t* work_counter;    // workspace work counter (zeroed per call)
   unsigned long long timeout_ns;
+  unsigned long long* trace;  // 16 cycle counters (only with -DSEER_TRACE)
 };
 
-// Persistent launch: one CTA per SM (at most one per unit).  tmQ/tmK/tmV are
-// 2-D bf16 tensor maps over [rows, d] with 64x64 boxes and 128-byte swizzle.
-cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                               const AttnParams& p, int num_sms, cudaStream_t st);
+// Re-layout of K and V into per-block records of 2*d rows x 64 bf16 (K^T,
+// then V in 64-column panels); `records` = B * Hkv * n/64.
+cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
+                            int n, int d, cudaStream_t st);
+
+// Persistent launch: one CTA per SM (at most one per unit).  tmQ is a 2-D
+// bf16 map over Q [rows, d] with 64x64 boxes; tmKV a 2-D bf16 map over the
+// records [records * 2d, 64] with a 2d-row box; both 128-byte swizzled.
+cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
+                               int num_sms, cudaStream_t st);
 
 }  // namespace seer

@@ -58,6 +58,7 @@ struct Ctrl {
   float red[2][4][32];
 };
 constexpr uint32_t kSmemAlloc = kSmemTiles + (uint32_t)sizeof(Ctrl);
+static_assert(kSmemAlloc <= 232448, "dynamic shared memory above the per-CTA limit");
 }  // namespace bmax
 
 namespace {

@@ -39,6 +39,22 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Hardware barrier `id` over `nthreads` threads that also ORs a predicate:
+// every participating thread receives whether any of them passed true.
+// Callers must guarantee that all nthreads threads reach it (no timeout).
+__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------- mbarriers --
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -70,6 +86,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended in hardware (it issues nothing) until the phase completes or about
+// `hint_ns` nanoseconds pass, instead of re-polling shared memory.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Status word codes written by kernels (device side, read by the host).
 enum : uint32_t {
   kDevOk = 0,
@@ -78,23 +109,21 @@ enum : uint32_t {
   kDevBadSchedule = 3,  // the work list was inconsistent
 };
 
-// Bounded wait on an mbarrier phase.  Gives up after `timeout_ns` of
-// %globaltimer time, or early when *abort becomes non-zero (another warp of
-// the CTA timed out).  On giving up it records kDevTimeout in *status (if not
+// Bounded wait on an mbarrier phase.  Sleeps in try_wait between checks;
+// gives up after `timeout_ns` of %globaltimer time, or early when *abort
+// becomes non-zero (another warp of the CTA timed out).  On giving up it records kDevTimeout in *status (if not
 // null), raises *abort, and returns false.  Never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
-        if (status) atomicCAS(status, kDevOk, kDevTimeout);
-        *abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      if (status) atomicCAS(status, kDevOk, kDevTimeout);
+      *abort = 1;
+      return false;
     }
   }
 }

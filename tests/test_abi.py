@@ -66,7 +66,8 @@ def test_workspace_sizes_cover_their_buffers():
     need = 4 * (B * Hq * nb * d + B * Hkv * nb * 3 * d + B * Hq * nb * h + B * Hkv * nb * h
                 + B * Hq * nb * nb)
     assert g >= need + 256 and g % 256 == 0
-    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256
+    # bf16: header + the K/V block records (K^T and V of every 64-key block)
+    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256 + 2 * 2 * B * Hkv * n * d
     f32 = seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 1)
     assert f32 >= 256 + 2 * n * d * (Hq + 2 * Hkv)
     assert seer.blockmax_workspace_size(B, Hq, Hkv, n, d, 0) >= 256 + 4 * 128 * nb

@@ -156,14 +156,22 @@ def test_repeat_runs_bitwise_identical():
 
 
 def test_rejects_bad_arguments():
+    import ctypes
     w, Q, K, V, Wq, Wk = inputs("tiny")
     Qd, Kd, Vd = to_dev(Q, K, V)
     c = torch.ones(1, 2, 8, dtype=torch.int32, device="cuda")
     ix = torch.zeros(1, 2, 8, 1, dtype=torch.int32, device="cuda")
-    with pytest.raises(seer.SeerError) as e:
-        seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, workspace=torch.empty(8, dtype=torch.uint8,
-                                                                       device="cuda"))
-    assert e.value.status in (7,)
+    small = torch.empty(8, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, workspace=small)
+    # the C entry point itself refuses a too-small workspace before launching
+    L = seer.lib()
+    dims = seer._lib._dims(1, 2, 1, 512, 64)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    O = torch.empty_like(Qd)
+    st = L.seer_sparse_attn(ctypes.byref(dims), p(Qd), p(Kd), p(Vd), 1, p(c), p(ix), 1, 0.0, p(O),
+                            None, p(small), 8, None)
+    assert st == 7  # SEER_ERR_WORKSPACE
     with pytest.raises(seer.SeerError) as e:
         seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, scale=-1.0)
     assert e.value.status == 1
