@@ -184,6 +184,38 @@ SEER_API seer_status seer_attn_blockmax(const seer_dims *dims, const void *Q, co
 SEER_API size_t seer_blockmax_workspace_size(const seer_dims *dims, seer_dtype dtype);
 
 /* ------------------------------------------------------------------------ */
+/* seer_gate_noalloc -- seer_gate for callers that cannot allocate device
+ * memory.  (The paper has no counterpart: this is an integration variant.)
+ *
+ * seer_gate's scratch (pooled Q/K, gate vectors, block logits) normally comes
+ * from a caller-allocated workspace.  Callers that cannot allocate -- a plugin
+ * inside a host framework that owns all device memory, code running while a
+ * CUDA graph is being captured (cudaMalloc is not allowed then), or a runtime
+ * that forbids allocation after start-up -- call this instead: same inputs and
+ * outputs, no workspace argument, and no allocation of any kind.  Its scratch
+ * is a static device buffer of SEER_GATE_NOALLOC_MAX_SCRATCH bytes inside the
+ * library, which every GPU that loads the library's device code keeps until
+ * the process exits.
+ *  - Problems whose scratch (seer_gate_workspace_size) exceeds the buffer are
+ *    rejected with SEER_ERR_WORKSPACE before anything is launched (for
+ *    example the 8k-token, 32-head layer fits; 32k tokens do not).
+ *  - The first call on each device resolves the buffer's device address
+ *    (once, with that device current); make that first call before any stream
+ *    capture.  A failure there returns SEER_ERR_CUDA.
+ *  - All calls on a device share the buffer: calls whose work may overlap on
+ *    the GPU (different streams without ordering) race and must not be made.
+ *  - Device status (seer_workspace_status) is not available for this entry
+ *    point; results and errors are otherwise those of seer_gate.          */
+#define SEER_GATE_NOALLOC_MAX_SCRATCH (32u << 20) /* bytes */
+
+SEER_API seer_status seer_gate_noalloc(const seer_dims *dims, const void *Q, const void *K,
+                                       seer_dtype dtype, const float *Wq, const float *Wk,
+                                       int32_t h, float rope_theta, seer_select_mode mode, float T,
+                                       int32_t k, float density, float *scores_out,
+                                       int32_t *counts, int32_t *indices, int32_t cap,
+                                       seer_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Synchronises `stream`, reads the device status word at the start of a
  * workspace that a previous call used, and maps it: SEER_OK,
  * SEER_ERR_TIMEOUT or SEER_ERR_DEVICE_CHECK (SEER_ERR_CUDA if the read

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.seer_gate_workspace_size.restype = SZ
         L.seer_gate_required_cap.argtypes = [DP, I32, I32, F]
         L.seer_gate_required_cap.restype = I32
+        L.seer_gate_noalloc.argtypes = [DP, P, P, I32, P, P, I32, F, I32, F, I32, F, P, P, P, I32, P]
+        L.seer_gate_noalloc.restype = I32
         L.seer_gate_select.argtypes = [DP, P, I32, F, I32, F, P, P, I32, P]
         L.seer_gate_select.restype = I32
         L.seer_sparse_attn.argtypes = [DP, P, P, P, I32, P, P, I32, F, P, P, P, SZ, P]
@@ -165,6 +167,35 @@ def seer_gate(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, retur
                          _ptr(scores), _ptr(counts), _ptr(indices), int(cap), _ptr(ws),
                          ws.numel(), _stream(dev))
     _check("seer_gate", st)
+    return (counts, indices, scores) if return_scores else (counts, indices)
+
+
+def seer_gate_noalloc(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0,
+                      return_scores=False, cap=None, out=None):
+    """seer_gate without a workspace, for callers that cannot allocate device
+    memory (their scratch lives in a fixed buffer inside the library; see
+    seer_gate_noalloc in include/seer.h for its size limit and sharing rules).
+    Outputs are still passed in (`out`) or allocated here for convenience."""
+    dev = _dev(Q, K, Wq, Wk)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    h = Wq.shape[1]
+    nb = n // 64
+    mc = mode_code(mode)
+    dims = _dims(B, Hq, Hkv, n, d)
+    if cap is None:
+        cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
+    if out is None:
+        counts = torch.empty(B, Hq, nb, dtype=torch.int32, device=dev)
+        indices = torch.empty(B, Hq, nb, cap, dtype=torch.int32, device=dev)
+        scores = torch.empty(B, Hq, nb, nb, dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        counts, indices, scores = out
+    st = lib().seer_gate_noalloc(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq),
+                                 _ptr(Wk), int(h), float(rope_theta), mc, float(T), int(k),
+                                 float(density), _ptr(scores), _ptr(counts), _ptr(indices),
+                                 int(cap), _stream(dev))
+    _check("seer_gate_noalloc", st)
     return (counts, indices, scores) if return_scores else (counts, indices)
 
 

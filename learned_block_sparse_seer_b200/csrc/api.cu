@@ -167,6 +167,10 @@ seer_status begin_ws(void* ws, size_t ws_bytes, size_t need, cudaStream_t st) {
 
 }  // namespace
 
+namespace seer {
+void set_last_cuda_error(int32_t e) { g_last_cuda_error = e; }
+}  // namespace seer
+
 extern "C" {
 
 const char* seer_version(void) { return "0.1.0"; }

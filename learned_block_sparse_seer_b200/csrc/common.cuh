@@ -23,6 +23,10 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
+// Records the CUDA error reported by seer_last_cuda_error() on this host
+// thread (api.cu).
+void set_last_cuda_error(int32_t e);
+
 __host__ __device__ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Carves consecutive 256-byte-aligned regions out of a workspace.
