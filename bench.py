@@ -27,6 +27,7 @@ import subprocess
 import sys
 import threading
 import time
+import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -40,7 +41,7 @@ BMAX_WORKLOAD = "bmax32k"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="seer", choices=["seer", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
@@ -61,7 +62,13 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled during the timed region.
+
+    The sampler is started (and its first line awaited) before the region, so
+    that the process start-up of nvidia-smi falls outside it; each line is
+    stamped on arrival and only lines that arrive inside [mark_start,
+    mark_end] are used (if the region is shorter than the sampling period, the
+    first line after it, which covers its last 200 ms, is used instead)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -70,8 +77,9 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
-    def start(self):
+    def start(self, wait_s: float = 5.0):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
@@ -80,22 +88,41 @@ class ClockSampler:
             self.thread.start()
         except Exception:
             self.proc = None
+            return
+        t = time.time()
+        while not self.lines and time.time() - t < wait_s and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t = time.time()
+        while self.t1 is not None and not any(ts > self.t1 for ts, _ in self.lines) and time.time() - t < 1.0:
+            time.sleep(0.02)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        inside = [ln for ts, ln in self.lines if self.t0 is not None and self.t0 <= ts <= self.t1]
+        window = "inside the timed region"
+        if not inside:
+            after = [ln for ts, ln in self.lines if self.t1 is not None and ts > self.t1]
+            inside = after[:1]
+            window = "first sample after the timed region (region shorter than the 200 ms period)"
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -108,7 +135,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
 def attn_flops(counts, indices, d):
@@ -337,10 +364,11 @@ def main():
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    clocks.mark_start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -352,6 +380,7 @@ def main():
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark_end()
     clk = clocks.stop()
     if world > 1:
         dist.barrier()

@@ -152,12 +152,11 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int w) {
   return r;
 }
 
-// Entry m of a unit's list, checked: it must satisfy 0 <= j <= i and be larger
-// than the previous entry.  A failing entry is recorded and replaced by a safe
-// in-range block so that no load leaves the tensor.
-__device__ __forceinline__ int list_entry(const AttnParams& p, const UnitInfo& u, int m) {
-  int j = p.indices[u.u * p.cap + m];
-  int prev = m > 0 ? p.indices[u.u * p.cap + m - 1] : -1;
+// A list entry j, checked: it must satisfy 0 <= j <= i and be larger than the
+// previous entry `prev` (as read, -1 before the first).  A failing entry is
+// recorded and replaced by a safe in-range block so that no load leaves the
+// tensor.
+__device__ __forceinline__ int checked_entry(const AttnParams& p, const UnitInfo& u, int j, int prev) {
   if (j < 0 || j > u.i || j <= prev) {
     record_status(p.status, kDevBadIndex, (uint32_t)u.u);
     j = j < 0 ? 0 : (j > u.i ? u.i : j);
@@ -373,18 +372,33 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           tma_load_2d(smem + kOffQ + qs * kQBytes + pn * 8192, &tmQ, &bars.q_full[qs], pn * 64, row);
         ++qn;
         const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;
+        // The list entries of the next pair step are loaded before this
+        // step's wait for a free stage, so that their global-memory latency
+        // is hidden behind it instead of delaying the gather.
+        const int* lst = p.indices + u.u * p.cap;
+        int jn0 = lst[0];
+        int jn1 = u.count > 1 ? lst[1] : 0;
+        int prev = -1;
         for (int m = 0; m < u.count; m += 2, ++g) {
+          const int ntile = m + 1 < u.count ? 2 : 1;
+          const int ja = jn0, jb = jn1;
+          if (m + 2 < u.count) jn0 = lst[m + 2];
+          if (m + 3 < u.count) jn1 = lst[m + 3];
           const int st = g % kStages;
           if (g >= kStages && !SEER_TIMED(0, mbar_wait(&bars.st_empty[st], ((g / kStages) - 1) & 1, abort_p, p.status, tmo))) {
             ok = false;
             break;
           }
-          const int ntile = m + 1 < u.count ? 2 : 1;
           mbar_arrive_expect_tx(&bars.st_full[st], (uint32_t)ntile * rec_rows * 128u);
-          for (int h = 0; h < ntile; ++h) {
-            const int j = list_entry(p, u, m + h);
-            tma_load_2d(smem + kOffRing + st * kStageBytes + h * kRecBytes, &tmKV, &bars.st_full[st], 0,
-                        (int)((rec0 + j) * rec_rows));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (h < ntile) {
+              const int raw = h == 0 ? ja : jb;
+              const int j = checked_entry(p, u, raw, prev);
+              prev = raw;
+              tma_load_2d(smem + kOffRing + st * kStageBytes + h * kRecBytes, &tmKV, &bars.st_full[st], 0,
+                          (int)((rec0 + j) * rec_rows));
+            }
           }
         }
       }
