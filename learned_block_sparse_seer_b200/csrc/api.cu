@@ -347,7 +347,7 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   SEER_CUDA(seer::launch_kv_tiles(K, V, dtype == SEER_FP32, base + w.kv, records, n, d, st));
   CUtensorMap tmQ, tmKV;
   if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) ||
-      !make_tmap_rows(&tmKV, base + w.kv, records * 2 * d, 2 * d))
+      !make_tmap_rows(&tmKV, base + w.kv, records * 2 * d, d))
     return cuda_fail(cudaErrorInvalidValue);
   seer::AttnParams p;
   p.B = B;
@@ -371,6 +371,7 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
   p.trace = reinterpret_cast<unsigned long long*>(hdr->pad + 4);  // 16 x u64 in the header
+  SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
   return SEER_OK;
 }

@@ -15,30 +15,33 @@
 //        O^T[d x 64 queries]         += V_pair^T[d x 128] . P^T        (PV)
 //    S^T and O^T live in tensor memory (TMEM); K/V/Q/P^T are 128-byte
 //    swizzled shared-memory tiles.
-//  * TMA on B200 costs about the same per instruction for any box up to
-//    16 KB, so a gathered tile must arrive in as few instructions as
-//    possible.  A re-layout pass (kv_tile_kernel) first writes every
-//    (KV head, key block) as one contiguous record [K^T: d rows x 64 keys |
-//    V: 64 keys x d in 64-column panels]; one 2*d-row TMA box (32 KB at
-//    d = 128, no cluster multicast) then brings both K and V of a block into
-//    the ring.  The ring has 3 pair stages of two records; K^T is read by the
-//    QK MMA as an MN-major operand whose two 64-key halves are the stage's
-//    two records (leading-byte offset = one record).
+//  * A re-layout pass (kv_tile_kernel) first writes every (KV head, key
+//    block) as one contiguous record [K^T: d rows x 64 keys | V: 64 keys x d
+//    in 64-column panels]; a d-row TMA box (16 KB at d = 128, no cluster
+//    multicast) brings either part of a block into shared memory.
+//  * The tensor pipe stalls for about 200 cycles whenever the thread that
+//    issues the MMAs synchronises (an mbarrier wait, a shared-memory read, a
+//    barrier), so the MMA thread waits exactly once per pair step, on one
+//    barrier go(g) that collects everything the next MMA group needs: the
+//    softmax's P^T of step g, the V records of step g and the K^T records
+//    (and, at a unit's start, the Q tile) of step g+2.  It then issues PV(g)
+//    and QK(g+2) back to back.  QK therefore runs two steps ahead of PV, which
+//    keeps the softmax of step g+1 busy while PV(g) and QK(g+2) execute.
+//  * Separate rings keep each buffer only as long as it is needed: K^T pairs
+//    (2 slots, free once their QK is done), V pairs (3 slots, free once their
+//    PV is done), P^T tiles (2 slots), Q tiles (2 slots), S^T in TMEM (3
+//    buffers).  224 KB of shared memory in all.
 //  * Warp roles (576 threads): warps 0..15 are four softmax warpgroups, each
 //    owning 16 of the 64 query columns (its own running max, row sums, vote
 //    and epilogue), one key (TMEM lane) per thread -- a warp w reaches TMEM
-//    lanes 32*(w%4)..+31; warp 16 schedules units and issues every TMA load
-//    (Q and the gathered records); warp 17 issues all MMAs from one thread
-//    and owns the TMEM allocation.  Four warps per SMSP work on the same
-//    step, so their latency chains interleave.
+//    lanes 32*(w%4)..+31; warp 16 schedules units and issues every TMA load;
+//    warp 17 issues all MMAs from one thread and owns the TMEM allocation.
 //  * Online softmax with a lazily updated running maximum per query column:
 //    the exact column maximum is formed on a unit's first step; afterwards a
 //    warpgroup vote re-forms it only when some score exceeds the running
 //    maximum by more than 2^8 (log2 domain), rescaling the row sums and O^T.
 //    The vote is one hardware barrier-with-reduction per step, taken after
 //    the exponentials (which are recomputed in the rare rescale case).
-//  * P^T of a step is written into the K^T half of its own stage (dead once
-//    the step's QK MMA is done), so P is buffered as deeply as the ring.
 //  * Units are handed out by an atomic counter in KV-head-major order, query
 //    blocks from the last (longest lists) to the first, so the K/V of one KV
 //    head stay hot in L2 while its query heads are processed.
@@ -51,36 +54,53 @@
 #include "common.cuh"
 #include "ptx.cuh"
 
+
 namespace seer {
 
 namespace attn {
-constexpr int kThreads = 576;
-constexpr int kStages = 3;  // pair stages: two K^T+V records each
-constexpr uint32_t kRecBytes = 32768, kStageBytes = 2 * kRecBytes;
-constexpr uint32_t kQBytes = 16384;
-constexpr uint32_t kOffRing = 0;                               // 3 x 64 KB
-constexpr uint32_t kOffQ = kOffRing + kStages * kStageBytes;   // 2 x 16 KB
-constexpr uint32_t kSmemBytes = kOffQ + 2 * kQBytes;           // 224 KB of tiles
-// P^T of a pair step is written into its stage: the K^T part of record h
-// (dead once the step's QK MMA has completed) takes keys 64h .. 64h+63.
-constexpr uint32_t kTmemCols = 256;  // S^T x 2 (64 cols each) + O^T (64 cols)
-constexpr uint32_t kColS0 = 0, kColO = 128;
+constexpr int kThreads = 608;
+constexpr int kWarpLoad = 16, kWarpPV = 17, kWarpQK = 18;
+constexpr uint32_t kHalf = 16384;              // one record's K^T or V part (d = 128)
+constexpr uint32_t kPair = 2 * kHalf;          // the K^T (or V) of a pair step
+constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 2, kQSlots = 2;
+constexpr uint32_t kPBytes = 16384;            // P^T of a pair step: 2 x [64 keys x 64 queries]
+constexpr uint32_t kQBytes = 16384;            // Q tile: 64 rows x d (two 64-column panels)
+constexpr uint32_t kOffK = 0;
+constexpr uint32_t kOffV = kOffK + kKSlots * kPair;       //  64 KB
+constexpr uint32_t kOffP = kOffV + kVSlots * kPair;       // 160 KB
+constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 192 KB
+constexpr uint32_t kSmemBytes = kOffQ + kQSlots * kQBytes;  // 224 KB of tiles
+constexpr int kRing = 4;   // go / qk_done / pv_done barriers, indexed by step
+constexpr int kSBuf = 3;   // S^T buffers in TMEM (QK runs two steps ahead of PV)
+constexpr int kUnits = 8;  // unit ring entries (the loader runs ahead of the consumers)
+constexpr uint32_t kTmemCols = 256;            // S^T x 3 (64 columns each) + O^T (64)
+constexpr uint32_t kColO = kSBuf * 64;
 constexpr int kWG = 4;     // softmax warpgroups
 constexpr int kCols = 16;  // query columns per warpgroup
+constexpr int kSoftmaxWarps = 4 * kWG;
+static_assert(kSBuf < kRing, "kfull(h) takes softmax(h - kSBuf) arrivals");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
-  uint64_t unit_full[2], unit_empty[2];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t st_full[kStages], st_empty[kStages];
-  uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t o_free, fin;
+  uint64_t unit_full[kUnits], unit_empty[kUnits];
+  uint64_t kfull[kRing];    // K^T(h) [+ Q] landed and softmax(h-3) done: the QK warp's one wait per step
+  uint64_t go[kRing];       // P^T(g) and V(g) ready: the PV warp's one wait per step
+  uint64_t qk_done[kRing];  // QK(g) complete: S^T(g) readable, K slot of g free
+  uint64_t pv_done[kRing];  // PV(g) complete: V slot and P^T slot of g free
+  uint64_t q_free[kQSlots];  // the last QK of the unit that used a Q slot is complete
+  uint64_t fin_qk, fin_pv;
+};
+// What the loader publishes about each unit: the unit index (-1 ends the
+// work), its checked list length and whether its last entry is the diagonal
+// block.  Consumers read only this, never the lists in global memory.
+struct UnitEntry {
+  int w, count, diag, pad;
 };
 // Control block, placed in dynamic shared memory right after the tiles (the
 // tiles need nearly the whole 227 KB budget, so nothing is static).
 struct Ctrl {
   Bars bars;
-  int unit_w[2];
+  UnitEntry unit[kUnits];
   uint32_t tmem_base;
   int abort_flag;
   alignas(16) float red[kWG][2][4][kCols];  // read with 16-byte vector loads
@@ -133,6 +153,23 @@ struct UnitInfo {
   long long u;  // (b*Hq + hq)*nb + i
 };
 
+// Coordinates of unit w (no memory access): batch, query head, its KV head,
+// query block and flat unit index.
+__device__ __forceinline__ UnitInfo unit_coords(const AttnParams& p, int w) {
+  UnitInfo r;
+  const int per_bg = p.nb * p.G;
+  const int bg = w / per_bg, rem = w % per_bg;
+  r.b = bg / p.Hkv;
+  r.g = bg % p.Hkv;
+  r.i = p.nb - 1 - rem / p.G;
+  r.hq = r.g * p.G + rem % p.G;
+  r.u = ((long long)r.b * p.Hq + r.hq) * p.nb + r.i;
+  r.count = 0;
+  return r;
+}
+
+// unit_coords plus the unit's list length, read and checked: it must lie in
+// [0, min(cap, i + 1)].  A failing count is recorded and clamped.
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int w) {
   UnitInfo r;
   const int per_bg = p.nb * p.G;
@@ -248,39 +285,45 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[attn::kCo
   }
 }
 
-// Issues the PV MMAs of pair step g: O^T (+)= V_pair^T . P^T, 16 keys per
-// MMA (8 MMAs for two records, 4 for one).  Waits for the step's P^T and, on
-// a unit's first step after an earlier unit, for that unit's epilogue to
-// have read O^T.  Then releases the stage and signals pv_done.
-__device__ __forceinline__ bool issue_pv(attn::Ctrl& C, const AttnParams& p, uint32_t tmem,
-                                         uint32_t sbase, uint32_t vpart, int g, bool wait_o_free,
-                                         bool first, bool two, int units_done) {
-  using namespace attn;
-  Bars& bars = C.bars;
-  volatile int* abort_p = &C.abort_flag;
-  const uint64_t tmo = p.timeout_ns;
-  // p_full is double-buffered by step: the four softmax warpgroups are not
-  // synchronised with each other, so one may already arrive for step g+1
-  // while another is still on step g (never for g+2: S(g+2) needs PV(g)).
-  if (!SEER_TIMED(3, mbar_wait(&bars.p_full[g & 1], (g >> 1) & 1, abort_p, p.status, tmo))) return false;
-  if (wait_o_free && !SEER_TIMED(5, mbar_wait(&bars.o_free, (units_done - 1) & 1, abort_p, p.status, tmo)))
-    return false;
-  tc_fence_after();
-  const uint32_t idesc_pv = make_idesc_bf16(128, 64, 1, 1);  // A = V^T, B = P^T (MN-major)
-  const uint32_t stage = sbase + kOffRing + (g % kStages) * kStageBytes;
-  const int nk = two ? 8 : 4;
-  for (int kk = 0; kk < nk; ++kk) {
-    const uint32_t rec = stage + (kk >> 2) * kRecBytes;  // keys 64*(kk/4) .. of the pair
-    const uint32_t va = rec + vpart + (kk & 3) * 2048;
-    const uint32_t pa = rec + (kk & 3) * 2048;           // P^T rows in the record's K^T part
-    mma_bf16_ss(tmem + kColO, make_sw128_desc(va, 8192, 1024), make_sw128_desc(pa, 16384, 1024),
-                idesc_pv, (first && kk == 0) ? 0u : 1u);
+// A consumer's walk over the unit ring, one pair step at a time.  next()
+// returns the step's info -- bit 0: two records, bit 1: first step of its
+// unit, bit 2: last step, bit 3: the unit's Q slot -- or -1 at the end (or on
+// a timeout, which also clears ok).  A ring entry is released as soon as it
+// has been read.
+struct UnitCursor {
+  int ur = 0, qn = 0, count = 0, rem = 0, t = 0, qslot = 0;
+  bool end = false;
+  __device__ __forceinline__ int next(attn::Ctrl& C, const AttnParams& p, volatile int* abort_p, bool& ok) {
+    using namespace attn;
+    while (rem == 0) {
+      if (end) return -1;
+      const int slot = ur % kUnits;
+      if (!mbar_wait(&C.bars.unit_full[slot], (ur / kUnits) & 1, abort_p, p.status, p.timeout_ns)) {
+        ok = false;
+        end = true;
+        return -1;
+      }
+      const int w = C.unit[slot].w, cnt = C.unit[slot].count;
+      ++ur;
+      if (w < 0) {  // the end marker is never released: nothing reuses its slot
+        end = true;
+        return -1;
+      }
+      mbar_arrive(&C.bars.unit_empty[slot]);
+      count = cnt;
+      rem = (cnt + 1) / 2;
+      t = 0;
+      qslot = qn & 1;
+      ++qn;
+    }
+    const int info = (2 * t + 1 < count ? 1 : 0) | (t == 0 ? 2 : 0) | (rem == 1 ? 4 : 0) | (qslot << 3);
+    ++t;
+    --rem;
+    return info;
   }
-  mma_commit(&bars.pv_done[g & 1]);
-  mma_commit(&bars.st_empty[g % kStages]);
-  return true;
-}
+};
 
+template <int D>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                        const AttnParams p) {
@@ -298,8 +341,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   volatile int* abort_p = &C.abort_flag;
   const uint64_t tmo = p.timeout_ns;
-  const uint32_t rec_rows = 2u * p.d;            // K^T rows + V rows of a record
-  const uint32_t vpart = (uint32_t)p.d * 128u;   // byte offset of V inside a record
 
 #ifdef SEER_TRACE
   const long long t_kernel0 = clock64();
@@ -307,36 +348,36 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #endif
   if (threadIdx.x == 0) {
     C.abort_flag = 0;
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kUnits; ++s) {
       mbar_init(&bars.unit_full[s], 1);
-      mbar_init(&bars.unit_empty[s], 1 + 4 * kWG);  // MMA + softmax warps
-      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.unit_empty[s], 2 + kSoftmaxWarps);  // both MMA warps + softmax warps, on reading
+    }
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&bars.kfull[s], 1 + kSoftmaxWarps);  // loader's K^T part + softmax(h-3) done
+      mbar_init(&bars.go[s], 1 + kSoftmaxWarps);     // loader's V part + softmax's P^T(g)
+      mbar_init(&bars.qk_done[s], 1);
       mbar_init(&bars.pv_done[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.q_full[s], 1);
-      mbar_init(&bars.q_empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) mbar_init(&bars.p_full[s], 4 * kWG);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.st_full[s], 1);
-      mbar_init(&bars.st_empty[s], 1);
-    }
-    mbar_init(&bars.o_free, 4 * kWG);
-    mbar_init(&bars.fin, 1);
+    // The first kSBuf steps' S^T buffers are free from the start: their
+    // "softmax(h-3) done" arrivals are made here.
+    for (int s = 0; s < kSBuf; ++s)
+      for (int a = 0; a < kSoftmaxWarps; ++a) mbar_arrive(&bars.kfull[s]);
+    for (int s = 0; s < kQSlots; ++s) mbar_init(&bars.q_free[s], 1);
+    mbar_init(&bars.fin_qk, 1);
+    mbar_init(&bars.fin_pv, 1);
     fence_barrier_init();
   }
-  if (p.d == 64) {
-    // With d = 64 a record is [K^T 64 rows | V 64 rows]; the PV product's
-    // second 64-row panel of V^T (head dims 64..127) then reads the zeroed
-    // third quarter of the record slot, which no load ever writes.
-    for (int r = 0; r < 2 * kStages; ++r) {
-      uint4* z = reinterpret_cast<uint4*>(smem + kOffRing + r * kRecBytes + 16384);
+  if (D == 64) {
+    // With d = 64 a record part is 64 rows (8 KB); the PV product's second
+    // 64-row panel of V^T (head dims 64..127) then reads the zeroed upper
+    // half of each V record slot, which no load ever writes.
+    for (int r = 0; r < 2 * kVSlots; ++r) {
+      uint4* z = reinterpret_cast<uint4*>(smem + kOffV + r * kHalf + 8192);
       for (int e = threadIdx.x; e < 8192 / 16; e += blockDim.x) z[e] = make_uint4(0, 0, 0, 0);
     }
     fence_async_shared();
   }
-  if (warp == 17) {
+  if (warp == kWarpPV) {
     tmem_alloc(&C.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -344,130 +385,182 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
-  const int dpanels = p.d / 64;
+  constexpr int dpanels = D / 64;
 
-  if (warp == 16) {
+  if (warp == kWarpLoad) {
     // ------------------------------- scheduler, Q loads, record gathers --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmKV);
-      int u_idx = 0, qn = 0, g = 0;
+      constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a record's K^T or V part
+      constexpr int rec_rows = 2 * D;
+      int u_idx = 0, qn = 0, h = 0;
       bool ok = true;
       while (ok) {
-        const int slot = u_idx & 1;
-        if (u_idx >= 2 && !mbar_wait(&bars.unit_empty[slot], ((u_idx >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
-        int w = (int)atomicAdd(p.work_counter, 1u);
-        if (w >= p.total_units || *abort_p) w = -1;
-        C.unit_w[slot] = w;
+        const int slot = u_idx % kUnits;
+        if (u_idx >= kUnits &&
+            !mbar_wait(&bars.unit_empty[slot], ((u_idx / kUnits) - 1) & 1, abort_p, p.status, tmo))
+          break;
+        // Units with an empty list never enter the ring: their output (O = 0,
+        // LSE = -inf) is written by empty_rows_kernel before this kernel.
+        int w;
+        UnitInfo u{};
+        for (;;) {
+          w = (int)atomicAdd(p.work_counter, 1u);
+          if (w >= p.total_units || *abort_p) {
+            w = -1;
+            break;
+          }
+          u = decode_unit(p, w);
+          if (u.count > 0) break;
+        }
+        // lists are ascending, so only the last entry can be the diagonal block
+        const int diag = w >= 0 ? (p.indices[u.u * p.cap + u.count - 1] == u.i) : 0;
+        C.unit[slot].w = w;
+        C.unit[slot].count = u.count;
+        C.unit[slot].diag = diag;
         mbar_arrive(&bars.unit_full[slot]);
-        if (w < 0) break;
         ++u_idx;
-        const UnitInfo u = decode_unit(p, w);
-        if (u.count == 0) continue;
-        const int qs = qn & 1;
-        if (qn >= 2 && !mbar_wait(&bars.q_empty[qs], ((qn >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
-        mbar_arrive_expect_tx(&bars.q_full[qs], 64u * p.d * 2u);
-        const int row = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
-        for (int pn = 0; pn < dpanels; ++pn)
-          tma_load_2d(smem + kOffQ + qs * kQBytes + pn * 8192, &tmQ, &bars.q_full[qs], pn * 64, row);
+        if (w < 0) break;
+        const int qs = qn % kQSlots;
+        if (qn >= kQSlots && !mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo)) break;
         ++qn;
+        const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
         const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;
-        // The list entries of the next pair step are loaded before this
-        // step's wait for a free stage, so that their global-memory latency
-        // is hidden behind it instead of delaying the gather.
+        // The list entries of the next pair step are read one step early, so
+        // that their global-memory latency hides behind this step's waits.
         const int* lst = p.indices + u.u * p.cap;
         int jn0 = lst[0];
         int jn1 = u.count > 1 ? lst[1] : 0;
         int prev = -1;
-        for (int m = 0; m < u.count; m += 2, ++g) {
+        for (int m = 0; m < u.count; m += 2, ++h) {
           const int ntile = m + 1 < u.count ? 2 : 1;
-          const int ja = jn0, jb = jn1;
+          const int ra = jn0, rb = jn1;
           if (m + 2 < u.count) jn0 = lst[m + 2];
           if (m + 3 < u.count) jn1 = lst[m + 3];
-          const int st = g % kStages;
-          if (g >= kStages && !SEER_TIMED(0, mbar_wait(&bars.st_empty[st], ((g / kStages) - 1) & 1, abort_p, p.status, tmo))) {
+          int jj[2];
+          jj[0] = checked_entry(p, u, ra, prev);
+          prev = ra;
+          jj[1] = 0;
+          if (ntile == 2) {
+            jj[1] = checked_entry(p, u, rb, prev);
+            prev = rb;
+          }
+          // K^T part: its slot is free once QK(h-2) is complete; it (and the
+          // unit's Q tile on its first step) completes kfull(h).
+          if (h >= 2 && !SEER_TIMED(0, mbar_wait(&bars.qk_done[(h - 2) % kRing], ((h - 2) / kRing) & 1, abort_p,
+                                                 p.status, tmo))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bars.st_full[st], (uint32_t)ntile * rec_rows * 128u);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (h < ntile) {
-              const int raw = h == 0 ? ja : jb;
-              const int j = checked_entry(p, u, raw, prev);
-              prev = raw;
-              tma_load_2d(smem + kOffRing + st * kStageBytes + h * kRecBytes, &tmKV, &bars.st_full[st], 0,
-                          (int)((rec0 + j) * rec_rows));
-            }
+          uint64_t* tk = &bars.kfull[h % kRing];
+          mbar_arrive_expect_tx(tk, (uint32_t)ntile * part_bytes + (m == 0 ? 64u * D * 2u : 0u));
+          if (m == 0)
+            for (int pn = 0; pn < dpanels; ++pn)
+              tma_load_2d(smem + kOffQ + qs * kQBytes + pn * 8192, &tmQ, tk, pn * 64, qrow);
+          for (int t = 0; t < ntile; ++t)
+            tma_load_2d(smem + kOffK + (h % kKSlots) * kPair + t * kHalf, &tmKV, tk, 0,
+                        (int)((rec0 + jj[t]) * rec_rows));
+          // V part: its slot is free once PV(h-3) is complete; it completes go(h).
+          if (h >= kVSlots &&
+              !SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing], ((h - kVSlots) / kRing) & 1, abort_p,
+                                       p.status, tmo))) {
+            ok = false;
+            break;
           }
+          mbar_arrive_expect_tx(&bars.go[h % kRing], (uint32_t)ntile * part_bytes);
+          for (int t = 0; t < ntile; ++t)
+            tma_load_2d(smem + kOffV + (h % kVSlots) * kPair + t * kHalf, &tmKV, &bars.go[h % kRing], 0,
+                        (int)((rec0 + jj[t]) * rec_rows + D));
         }
       }
-      // wait for loads still in flight before the CTA may exit
-      for (int k = 0; k < 2 && k < qn; ++k) {
-        const int qq = qn - 1 - k;
-        mbar_wait(&bars.q_full[qq & 1], (qq >> 1) & 1, abort_p, nullptr, 20000000ull);
-      }
-      for (int k = 0; k < kStages && k < g; ++k) {
-        const int gg = g - 1 - k;
-        mbar_wait(&bars.st_full[gg % kStages], (gg / kStages) & 1, abort_p, nullptr, 20000000ull);
-      }
     }
-  } else if (warp == 17) {
-    // ------------------------------------------------------------ MMA ----
+  } else if (warp == kWarpQK) {
+    // ------------------------------------------------------ QK issuer ----
+    // Two warps issue the MMAs, QK and PV, each waiting once per step on its
+    // own barrier: while one waits, the other keeps the tensor pipe fed.
+    // The issue code is straight-line (fully unrolled groups, descriptors as
+    // a per-step base plus compile-time offsets, ring positions as counters):
+    // per-MMA branches or address arithmetic measurably slow the pipe's intake.
     if (lane == 0) {
-      const uint32_t idesc_qk = make_idesc_bf16(128, 64, 1, 0);  // A = K^T pair (MN-major)
+      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 64, 1, 0);  // A = K^T pair (MN-major)
       const uint32_t sbase = smem_u32(smem);
-      int u_idx = 0, qn = 0, step = 0, units_done = 0;
-      const int ksteps_qk = p.d / 16;
+      // The start address field holds (address >> 4): a byte offset b inside
+      // the 256 KB window is added as (b >> 4).
+      const uint64_t dK0 = make_sw128_desc(sbase + kOffK, kHalf, 1024);
+      const uint64_t dQ0 = make_sw128_desc(sbase + kOffQ, 16, 1024);
+      UnitCursor cur;
       bool ok = true;
-      while (ok) {
-        const int slot = u_idx & 1;
-        if (!mbar_wait(&bars.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
-        const int w = C.unit_w[slot];
-        mbar_arrive(&bars.unit_empty[slot]);
-        if (w < 0) break;
-        ++u_idx;
-        const UnitInfo u = decode_unit(p, w);
-        if (u.count == 0) continue;
-        const int T = (u.count + 1) / 2;
-        const int qs = qn & 1;
-        if (!SEER_TIMED(4, mbar_wait(&bars.q_full[qs], (qn >> 1) & 1, abort_p, p.status, tmo))) break;
-        const uint32_t qa = sbase + kOffQ + qs * kQBytes;
-        for (int t = 0; t < T && ok; ++t) {
-          const int g = step + t;
-          const int st = g % kStages;
-          if (!SEER_TIMED(2, mbar_wait(&bars.st_full[st], (g / kStages) & 1, abort_p, p.status, tmo))) { ok = false; break; }
-          SEER_TRACE_ADD(12, 1);
-          tc_fence_after();
-          const uint32_t ka = sbase + kOffRing + st * kStageBytes;
-          for (int kk = 0; kk < ksteps_qk; ++kk) {
-            const uint32_t qoff = (kk >> 2) * 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + kColS0 + (g & 1) * 64, make_sw128_desc(ka + kk * 2048, kRecBytes, 1024),
-                        make_sw128_desc(qa + qoff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars.s_full[g & 1]);
-          if (t == T - 1) mma_commit(&bars.q_empty[qs]);
-          if (t >= 1 && !issue_pv(C, p, tmem, sbase, vpart, g - 1, t - 1 == 0 && units_done > 0,
-                                  t - 1 == 0, 2 * (t - 1) + 1 < u.count, units_done)) { ok = false; break; }
-        }
-        if (!ok) break;
-        if (!issue_pv(C, p, tmem, sbase, vpart, step + T - 1, T == 1 && units_done > 0, T == 1,
-                      2 * (T - 1) + 1 < u.count, units_done)) break;
-        step += T;
-        ++qn;
-        ++units_done;
+      int h = 0, kslot = 0, sbuf = 0, ring = 0;
+      for (;;) {
+        const int info = cur.next(C, p, abort_p, ok);
+        if (info < 0) break;
+        if (!SEER_TIMED(4, mbar_wait(&bars.kfull[ring], (h / kRing) & 1, abort_p, p.status, tmo))) break;
+        tc_fence_after();
+        const uint64_t dk = dK0 + ((uint64_t)(kslot * kPair) >> 4);
+        const uint64_t dq = dQ0 + ((uint64_t)(((info >> 3) & 1) * kQBytes) >> 4);
+        const uint32_t sc = tmem + (uint32_t)sbuf * 64u;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(sc, dk + (uint64_t)(kk * 2048 / 16), dq + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) / 16),
+                      idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(&bars.qk_done[ring]);
+        if (info & 4) mma_commit(&bars.q_free[(info >> 3) & 1]);
+        ++h;
+        kslot = kslot + 1 == kKSlots ? 0 : kslot + 1;
+        sbuf = sbuf + 1 == kSBuf ? 0 : sbuf + 1;
+        ring = ring + 1 == kRing ? 0 : ring + 1;
       }
-      // all MMAs complete before TMEM is released
-      mma_commit(&bars.fin);
-      mbar_wait(&bars.fin, 0, abort_p, nullptr, 20000000ull);
+      // this thread's MMAs complete before TMEM is released
+      mma_commit(&bars.fin_qk);
+      mbar_wait(&bars.fin_qk, 0, abort_p, nullptr, 20000000ull);
     }
-  } else if (warp < 16) {
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------------------ PV issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, 64, 1, 1);  // A = V^T, B = P^T (MN-major)
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t dV0 = make_sw128_desc(sbase + kOffV, 8192, 1024);
+      const uint64_t dP0 = make_sw128_desc(sbase + kOffP, 16384, 1024);
+      UnitCursor cur;
+      bool ok = true;
+      int g = 0, vslot = 0, pslot = 0, ring = 0;
+      for (;;) {
+        const int info = cur.next(C, p, abort_p, ok);
+        if (info < 0) break;
+        if (!SEER_TIMED(3, mbar_wait(&bars.go[ring], (g / kRing) & 1, abort_p, p.status, tmo))) break;
+        SEER_TRACE_ADD(12, 1);
+        tc_fence_after();
+        const uint64_t dv = dV0 + ((uint64_t)(vslot * kPair) >> 4);
+        const uint64_t dp = dP0 + ((uint64_t)(pslot * kPBytes) >> 4);
+        const uint32_t acc0 = (info & 2) ? 0u : 1u;
+        if (info & 1) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + kColO, dv + (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 2048) / 16),
+                        dp + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 2048) / 16), idesc_pv, kk == 0 ? acc0 : 1u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + kColO, dv + (uint64_t)((kk * 2048) / 16), dp + (uint64_t)((kk * 2048) / 16), idesc_pv,
+                        kk == 0 ? acc0 : 1u);
+        }
+        mma_commit(&bars.pv_done[ring]);
+        ++g;
+        vslot = vslot + 1 == kVSlots ? 0 : vslot + 1;
+        pslot = pslot + 1 == kPSlots ? 0 : pslot + 1;
+        ring = ring + 1 == kRing ? 0 : ring + 1;
+      }
+      mma_commit(&bars.fin_pv);
+      mbar_wait(&bars.fin_pv, 0, abort_p, nullptr, 20000000ull);
+    }
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------- softmax WGs ---
     // The warpgroup synchronises with barrier.cta.red (hardware, no timeout),
     // so every one of its 128 threads must reach every barrier: a bounded wait
     // that gives up does not leave the loop on its own; its failure is ORed
     // into the next barrier and the whole warpgroup leaves together.
-    const int wgi = warp >> 2;                 // warpgroup: query columns 32*wgi..
+    const int wgi = warp >> 2;                 // warpgroup: query columns 16*wgi..
     const int ww = warp & 3;                   // TMEM sub-partition
     const int tl = ww * 32 + lane;             // TMEM lane == key in pair / dim of O^T
     const int q0 = wgi * kCols;
@@ -478,46 +571,39 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     int u_idx = 0, step = 0, red_use = 0;
     float lpart[kCols], m[kCols];
     for (;;) {
-      const int slot = u_idx & 1;
-      const bool okw = mbar_wait(&bars.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo);
-      const int w = okw ? C.unit_w[slot] : -1;
+      const int slot = u_idx % kUnits;
+      const bool okw = mbar_wait(&bars.unit_full[slot], (u_idx / kUnits) & 1, abort_p, p.status, tmo);
+      const int w = okw ? C.unit[slot].w : -1;
+      const int count = okw ? C.unit[slot].count : 0;
+      const bool last_is_diag = okw && C.unit[slot].diag != 0;
       if (bar_red_or(bar_id, 128, !okw)) break;
+      if (w < 0) break;  // the end marker is never released: nothing reuses its slot
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
-      if (w < 0) break;
       ++u_idx;
-      const UnitInfo u = decode_unit(p, w);
+      const UnitInfo u = unit_coords(p, w);
       const long long orow0 = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + q0;
-      if (u.count == 0) {
-        if (tl < p.d) {
-          for (int q = 0; q < kCols; ++q) {
-            if (p.out_fp32)
-              reinterpret_cast<float*>(p.O)[(orow0 + q) * p.d + tl] = 0.f;
-            else
-              reinterpret_cast<uint16_t*>(p.O)[(orow0 + q) * p.d + tl] = 0;
-          }
-        }
-        if (tl < kCols && p.lse) p.lse[orow0 + tl] = -INFINITY;
-        continue;
-      }
-      const int T = (u.count + 1) / 2;
-      // lists are ascending, so only the last entry can be the diagonal block
-      const bool last_is_diag = p.indices[u.u * p.cap + u.count - 1] == u.i;
+      const int T = (count + 1) / 2;
 #pragma unroll
       for (int q = 0; q < kCols; ++q) lpart[q] = 0.f;
       bool fail = false;
       for (int t = 0; t < T; ++t) {
         const int g = step + t;
         const int mi = 2 * t + half;
-        const bool valid = mi < u.count;
-        const bool diag = valid && last_is_diag && mi == u.count - 1;
-        const bool okS = SEER_TIMED_L0(6, mbar_wait(&bars.s_full[g & 1], (g >> 1) & 1, abort_p, p.status, tmo));
+        const bool valid = mi < count;
+        const bool diag = valid && last_is_diag && mi == count - 1;
+        const bool okS = SEER_TIMED_L0(6, mbar_wait(&bars.qk_done[g % kRing], (g / kRing) & 1, abort_p, p.status, tmo));
+        // P^T(g) goes to the slot of step g-2, free once PV(g-2) is complete
+        // (long done in steady state); a failed wait joins the step's first
+        // barrier below.
+        const bool okP = g < kPSlots || mbar_wait(&bars.pv_done[(g - kPSlots) % kRing], ((g - kPSlots) / kRing) & 1,
+                                                  abort_p, p.status, tmo);
 #ifdef SEER_TRACE
         const long long tstep0 = clock64();
         long long tmark = tstep0;
 #endif
         tc_fence_after();
-        const uint32_t saddr = lane_addr + kColS0 + (g & 1) * 64 + q0;
+        const uint32_t saddr = lane_addr + (uint32_t)(g % kSBuf) * 64u + q0;
         float x[kCols];
         if (okS) load_scores(saddr, x, c, valid, diag, kl, q0);
         SEER_MARK(14);
@@ -526,7 +612,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           // exact column maxima of the unit's first step
           warp_reduce_scatter16<false>(x, lane, red + ww * kCols);
           ++red_use;
-          if (bar_red_or(bar_id, 128, !okS)) { fail = true; break; }
+          if (bar_red_or(bar_id, 128, !okS || !okP)) { fail = true; break; }
           col_combine<false>(red, m);
           load_scores(saddr, x, c, valid, diag, kl, q0);
 #pragma unroll
@@ -543,7 +629,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
           SEER_MARK(16);
-          if (SEER_TIMED_L0(8, bar_red_or(bar_id, 128, !okS || dmax > kRescaleThreshold))) {
+          if (SEER_TIMED_L0(8, bar_red_or(bar_id, 128, !okS || !okP || dmax > kRescaleThreshold))) {
             if (*abort_p) { fail = true; break; }
             if (lane == 0) SEER_TRACE_ADD(13, 1);
             // exact column maxima of this step relative to the running max
@@ -563,7 +649,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             }
             // O^T columns are rescaled once the previous PV has landed
             const int gp = g - 1;
-            const bool okPV = mbar_wait(&bars.pv_done[gp & 1], (gp >> 1) & 1, abort_p, p.status, tmo);
+            const bool okPV = mbar_wait(&bars.pv_done[gp % kRing], (gp / kRing) & 1, abort_p, p.status, tmo);
             if (okPV) {
               tc_fence_after();
               uint32_t o[16];
@@ -591,8 +677,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           pk[q >> 1] = pack_bf16x2(x[q], x[q + 1]);
         }
         SEER_MARK(18);
-        // P^T row `kl` of record `half` of the step's stage (its K^T part)
-        uint8_t* prow = smem + kOffRing + (g % kStages) * kStageBytes + half * kRecBytes + kl * 128;
+        // P^T row `kl` of half `half` of the step's P^T slot
+        uint8_t* prow = smem + kOffP + (g % kPSlots) * kPBytes + half * 8192 + kl * 128;
 #pragma unroll
         for (int ch = 0; ch < kCols / 8; ++ch) {
           const int chunk = wgi * (kCols / 8) + ch;
@@ -604,7 +690,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         SEER_MARK(21);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[g & 1]);
+        if (lane == 0) {
+          mbar_arrive(&bars.go[g % kRing]);
+          mbar_arrive(&bars.kfull[(g + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
+        }
         SEER_MARK(22);
 #ifdef SEER_TRACE
         if (lane == 0) SEER_TRACE_ADD(9, clock64() - tstep0);
@@ -616,7 +705,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const long long tep0 = clock64();
 #endif
       const int gl = step + T - 1;
-      const bool okPV = mbar_wait(&bars.pv_done[gl & 1], (gl >> 1) & 1, abort_p, p.status, tmo);
+      const bool okPV = mbar_wait(&bars.pv_done[gl % kRing], (gl / kRing) & 1, abort_p, p.status, tmo);
       float* red = &C.red[wgi][red_use & 1][0][0];
       warp_reduce_scatter16<true>(lpart, lane, red + ww * kCols);
       ++red_use;
@@ -628,9 +717,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         uint32_t o[16];
         tmem_ld16(lane_addr + kColO + q0, o);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.o_free);
         if (tl < p.d) {
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
@@ -663,7 +749,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 17) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpPV) tmem_dealloc(tmem, kTmemCols);
+  // After an abort the consumers stopped waiting, so loads may still be in
+  // flight: give them time to land before the CTA's shared memory is released.
+  if (threadIdx.x == 0 && *abort_p) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
 #ifdef SEER_TRACE
   if (threadIdx.x == 0) {
     C.trace[11] = clock64() - t_kernel0;
@@ -731,6 +824,33 @@ __global__ void __launch_bounds__(256) kv_tile_kernel(const T* __restrict__ K, c
   }
 }
 
+// Units whose list is empty (count <= 0) get O = 0 and LSE = -inf here; the
+// attention kernel never schedules them.  One warp per unit.
+__global__ void __launch_bounds__(256) empty_rows_kernel(const int32_t* __restrict__ counts, void* O, float* lse,
+                                                         int out_fp32, long long units, int d) {
+  const long long u = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (u >= units || counts[u] > 0) return;
+  const long long elems = 64LL * d;  // the unit's 64 rows of O
+  if (out_fp32) {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(O) + u * elems);
+    for (long long e = lane; e < elems / 4; e += 32) o[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(O) + u * elems);
+    for (long long e = lane; e < elems / 8; e += 32) o[e] = make_uint4(0, 0, 0, 0);
+  }
+  if (lse) {
+    lse[u * 64 + lane] = -INFINITY;
+    lse[u * 64 + 32 + lane] = -INFINITY;
+  }
+}
+
+cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st) {
+  const long long blocks = (p.total_units + 7) / 8;
+  empty_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.counts, p.O, p.lse, p.out_fp32, p.total_units, p.d);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
                             int n, int d, cudaStream_t st) {
   if (fp32)
@@ -744,12 +864,12 @@ cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, 
 
 cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
                                int num_sms, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)attn::kSmemAlloc);
+  auto kern = p.d == 64 ? sparse_attn_kernel<64> : sparse_attn_kernel<128>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn::kSmemAlloc);
   if (e != cudaSuccess) return e;
   long long grid = p.total_units < num_sms ? p.total_units : num_sms;
   if (grid < 1) grid = 1;
-  sparse_attn_kernel<<<(unsigned)grid, attn::kThreads, attn::kSmemAlloc, st>>>(tmQ, tmKV, p);
+  kern<<<(unsigned)grid, attn::kThreads, attn::kSmemAlloc, st>>>(tmQ, tmKV, p);
   return cudaGetLastError();
 }
 

@@ -26,9 +26,14 @@ struct AttnParams {
 cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
                             int n, int d, cudaStream_t st);
 
+// O = 0 and LSE = -inf for every unit whose list is empty (count <= 0); the
+// attention kernel skips those units.  Launch before launch_sparse_attn.
+cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st);
+
 // Persistent launch: one CTA per SM (at most one per unit).  tmQ is a 2-D
 // bf16 map over Q [rows, d] with 64x64 boxes; tmKV a 2-D bf16 map over the
-// records [records * 2d, 64] with a 2d-row box; both 128-byte swizzled.
+// records [records * 2d, 64] with a d-row box (the K^T or the V part of one
+// record); both 128-byte swizzled.
 cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
                                int num_sms, cudaStream_t st);
 
