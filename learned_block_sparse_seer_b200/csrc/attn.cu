@@ -323,6 +323,43 @@ struct UnitCursor {
   }
 };
 
+// This thread's kCols S^T columns from TMEM as (score * c - m) in the log2
+// domain, with packed pair arithmetic (nm2 holds -m); absent or causally
+// masked keys become -inf.
+__device__ __forceinline__ void scores_minus_max(uint32_t taddr, float (&x)[attn::kCols], uint64_t c2,
+                                                 const uint64_t (&nm2)[attn::kCols / 2], bool valid, bool diag,
+                                                 int kl, int q0) {
+  uint32_t r[16];
+  tmem_ld16(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q = 0; q < attn::kCols / 2; ++q) {
+    const uint64_t v = fma_f32x2(f32x2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), c2, nm2[q]);
+    f32x2_unpack(v, x[2 * q], x[2 * q + 1]);
+  }
+  if (!valid) {
+#pragma unroll
+    for (int q = 0; q < attn::kCols; ++q) x[q] = -INFINITY;
+  } else if (diag) {
+#pragma unroll
+    for (int q = 0; q < attn::kCols; ++q) x[q] = (q0 + q < kl) ? -INFINITY : x[q];
+  }
+}
+
+// This warpgroup's 16 bf16 probabilities of key row kl into the step's P^T
+// tile (128-byte rows, 16-byte chunks swizzled by the row index).
+__device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kCols], int wgi, int kl) {
+  uint32_t pk[attn::kCols / 2];
+#pragma unroll
+  for (int q = 0; q < attn::kCols; q += 2) pk[q >> 1] = pack_bf16x2(x[q], x[q + 1]);
+#pragma unroll
+  for (int ch = 0; ch < attn::kCols / 8; ++ch) {
+    const int chunk = wgi * (attn::kCols / 8) + ch;
+    *reinterpret_cast<uint4*>(prow + ((chunk ^ (kl & 7)) << 4)) =
+        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
@@ -569,7 +606,10 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const float c = p.scale_log2;
     const int half = tl >> 6, kl = tl & 63;
     int u_idx = 0, step = 0, red_use = 0;
-    float lpart[kCols], m[kCols];
+    // Per query column of this warpgroup, as packed pairs: the negated
+    // running maximum (log2 domain) and this thread's row-sum partial.
+    uint64_t nm2[kCols / 2], lp2[kCols / 2];
+    const uint64_t c2 = f32x2_pack(c, c);
     for (;;) {
       const int slot = u_idx % kUnits;
       const bool okw = mbar_wait(&bars.unit_full[slot], (u_idx / kUnits) & 1, abort_p, p.status, tmo);
@@ -585,7 +625,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const long long orow0 = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + q0;
       const int T = (count + 1) / 2;
 #pragma unroll
-      for (int q = 0; q < kCols; ++q) lpart[q] = 0.f;
+      for (int q = 0; q < kCols / 2; ++q) lp2[q] = 0ull;
       bool fail = false;
       for (int t = 0; t < T; ++t) {
         const int g = step + t;
@@ -604,48 +644,53 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #endif
         tc_fence_after();
         const uint32_t saddr = lane_addr + (uint32_t)(g % kSBuf) * 64u + q0;
+        // P^T row `kl` of half `half` of the step's P^T slot
+        uint8_t* prow = smem + kOffP + (g % kPSlots) * kPBytes + half * 8192 + kl * 128;
         float x[kCols];
-        if (okS) load_scores(saddr, x, c, valid, diag, kl, q0);
-        SEER_MARK(14);
-        float* red = &C.red[wgi][red_use & 1][0][0];
         if (t == 0) {
           // exact column maxima of the unit's first step
+          if (okS) load_scores(saddr, x, c, valid, diag, kl, q0);
+          float* red = &C.red[wgi][red_use & 1][0][0];
           warp_reduce_scatter16<false>(x, lane, red + ww * kCols);
           ++red_use;
           if (bar_red_or(bar_id, 128, !okS || !okP)) { fail = true; break; }
-          col_combine<false>(red, m);
-          load_scores(saddr, x, c, valid, diag, kl, q0);
+          float mcol[kCols];
+          col_combine<false>(red, mcol);
 #pragma unroll
-          for (int q = 0; q < kCols; ++q) x[q] = exp2f_approx_sub(x[q], m[q]);
-        } else {
-          float dmax = -INFINITY;
-#pragma unroll
-          for (int q = 0; q < kCols; ++q) {
-            x[q] -= m[q];
-            dmax = fmaxf(dmax, x[q]);
-          }
-          // probabilities with the running max; the barrier then tells
-          // whether any score of the step exceeded it by more than 2^8
+          for (int q = 0; q < kCols / 2; ++q) nm2[q] = f32x2_pack(-mcol[2 * q], -mcol[2 * q + 1]);
+          scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
+          store_p(prow, x, wgi, kl);
+        } else {
+          if (okS) scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
+          const float dmax =
+              fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
+                    fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
+          // probabilities with the running max, stored before the vote; the
+          // barrier then tells whether any score of the step exceeded the
+          // running max by more than 2^8, in which case they are redone
+#pragma unroll
+          for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
+          store_p(prow, x, wgi, kl);
           SEER_MARK(16);
           if (SEER_TIMED_L0(8, bar_red_or(bar_id, 128, !okS || !okP || dmax > kRescaleThreshold))) {
             if (*abort_p) { fail = true; break; }
             if (lane == 0) SEER_TRACE_ADD(13, 1);
             // exact column maxima of this step relative to the running max
-            load_scores(saddr, x, c, valid, diag, kl, q0);
-#pragma unroll
-            for (int q = 0; q < kCols; ++q) x[q] -= m[q];
+            scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
+            float* red = &C.red[wgi][red_use & 1][0][0];
             warp_reduce_scatter16<false>(x, lane, red + ww * kCols);
             ++red_use;
             bar_red_or(bar_id, 128, false);
             col_combine<false>(red, x);
             float (&inc)[kCols] = x;  // increase of the running max per column
 #pragma unroll
-            for (int q = 0; q < kCols; ++q) {
-              inc[q] = fmaxf(inc[q], 0.f);
-              m[q] += inc[q];
-              lpart[q] *= ex2_approx(-inc[q]);
+            for (int q = 0; q < kCols; ++q) inc[q] = fmaxf(inc[q], 0.f);
+#pragma unroll
+            for (int q = 0; q < kCols / 2; ++q) {
+              nm2[q] = add_f32x2(nm2[q], f32x2_pack(-inc[2 * q], -inc[2 * q + 1]));
+              lp2[q] = mul_f32x2(lp2[q], f32x2_pack(ex2_approx(-inc[2 * q]), ex2_approx(-inc[2 * q + 1])));
             }
             // O^T columns are rescaled once the previous PV has landed
             const int gp = g - 1;
@@ -662,29 +707,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
               tmem_wait_st();
             }
             if (bar_red_or(bar_id, 128, !okPV)) { fail = true; break; }
-            load_scores(saddr, x, c, valid, diag, kl, q0);
+            scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
 #pragma unroll
-            for (int q = 0; q < kCols; ++q) x[q] = exp2f_approx_sub(x[q], m[q]);
+            for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
+            store_p(prow, x, wgi, kl);
           }
           SEER_MARK(17);
         }
-        // row-sum partials and this warpgroup's half of the bf16 P^T row
-        uint32_t pk[kCols / 2];
+        // row-sum partials
 #pragma unroll
-        for (int q = 0; q < kCols; q += 2) {
-          lpart[q] += x[q];
-          lpart[q + 1] += x[q + 1];
-          pk[q >> 1] = pack_bf16x2(x[q], x[q + 1]);
-        }
-        SEER_MARK(18);
-        // P^T row `kl` of half `half` of the step's P^T slot
-        uint8_t* prow = smem + kOffP + (g % kPSlots) * kPBytes + half * 8192 + kl * 128;
-#pragma unroll
-        for (int ch = 0; ch < kCols / 8; ++ch) {
-          const int chunk = wgi * (kCols / 8) + ch;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (kl & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        }
+        for (int q = 0; q < kCols / 2; ++q) lp2[q] = add_f32x2(lp2[q], f32x2_pack(x[2 * q], x[2 * q + 1]));
         SEER_MARK(20);
         fence_async_shared();
         SEER_MARK(21);
@@ -707,6 +739,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const int gl = step + T - 1;
       const bool okPV = mbar_wait(&bars.pv_done[gl % kRing], (gl / kRing) & 1, abort_p, p.status, tmo);
       float* red = &C.red[wgi][red_use & 1][0][0];
+      float lpart[kCols];
+#pragma unroll
+      for (int q = 0; q < kCols / 2; ++q) f32x2_unpack(lp2[q], lpart[2 * q], lpart[2 * q + 1]);
       warp_reduce_scatter16<true>(lpart, lane, red + ww * kCols);
       ++red_use;
       if (bar_red_or(bar_id, 128, !okPV)) break;
@@ -730,11 +765,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         }
       }
       if (tl < kCols && p.lse) {
-        float mq = m[0], lq = l[0];
+        float m[kCols];
+#pragma unroll
+        for (int q = 0; q < kCols / 2; ++q) f32x2_unpack(nm2[q], m[2 * q], m[2 * q + 1]);
+        float mq = -m[0], lq = l[0];
 #pragma unroll
         for (int q = 1; q < kCols; ++q)
           if (q == tl) {
-            mq = m[q];
+            mq = -m[q];
             lq = l[q];
           }
         p.lse[orow0 + tl] = (mq + log2f(lq)) * 0.6931471805599453f;
