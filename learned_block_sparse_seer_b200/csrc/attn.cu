@@ -62,13 +62,13 @@ constexpr int kThreads = 608;
 constexpr int kWarpLoad = 16, kWarpPV = 17, kWarpQK = 18;
 constexpr uint32_t kHalf = 16384;              // one record's K^T or V part (d = 128)
 constexpr uint32_t kPair = 2 * kHalf;          // the K^T (or V) of a pair step
-constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 2, kQSlots = 2;
+constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 3, kQSlots = 1;
 constexpr uint32_t kPBytes = 16384;            // P^T of a pair step: 2 x [64 keys x 64 queries]
 constexpr uint32_t kQBytes = 16384;            // Q tile: 64 rows x d (two 64-column panels)
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kKSlots * kPair;       //  64 KB
 constexpr uint32_t kOffP = kOffV + kVSlots * kPair;       // 160 KB
-constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 192 KB
+constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 208 KB
 constexpr uint32_t kSmemBytes = kOffQ + kQSlots * kQBytes;  // 224 KB of tiles
 constexpr int kRing = 4;   // go / qk_done / pv_done barriers, indexed by step
 constexpr int kSBuf = 3;   // S^T buffers in TMEM (QK runs two steps ahead of PV)
@@ -313,7 +313,7 @@ struct UnitCursor {
       count = cnt;
       rem = (cnt + 1) / 2;
       t = 0;
-      qslot = qn & 1;
+      qslot = qn % kQSlots;
       ++qn;
     }
     const int info = (2 * t + 1 < count ? 1 : 0) | (t == 0 ? 2 : 0) | (rem == 1 ? 4 : 0) | (qslot << 3);
