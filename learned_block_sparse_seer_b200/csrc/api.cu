@@ -126,16 +126,18 @@ GateWs gate_ws(const seer_dims* d, int h) {
 }
 
 struct AttnWs {
-  size_t q16, kv, total;
+  size_t q16, kv, redo, total;
 };
 
 // fp32 Q converted to bf16 (fp32 inputs only), then the K/V block records
 // (2 * B * Hkv * n * d bf16, K^T and V of each 64-key block together).
 AttnWs attn_ws(const seer_dims* d, seer_dtype dt) {
   seer::WsCarver c;
-  AttnWs w{0, 0, 0};
+  AttnWs w{0, 0, 0, 0};
   if (dt == SEER_FP32) w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
   w.kv = c.take(2ull * 2ull * d->B * d->Hkv * d->n * d->d);
+  // units flagged for the exact fallback (one int32 per unit at most)
+  w.redo = c.take(sizeof(int32_t) * (size_t)d->B * d->Hq * (d->n / seer::kBlock));
   w.total = c.off;
   return w;
 }
@@ -371,8 +373,12 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
   p.trace = reinterpret_cast<unsigned long long*>(hdr->pad + 4);  // 16 x u64 in the header
+  p.redo_count = &hdr->work_counter2;
+  p.redo_list = reinterpret_cast<int*>(base + w.redo);
+  p.redo_cap = (int)p.total_units;
   SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
+  SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kv, p, st));
   return SEER_OK;
 }
 

@@ -79,7 +79,10 @@ constexpr int kWG = 4;     // softmax warpgroups
 constexpr int kCols = 16;  // query columns per warpgroup
 constexpr int kSoftmaxWarps = 4 * kWG;
 static_assert(kSBuf < kRing, "kfull(h) takes softmax(h - kSBuf) arrivals");
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// A score more than 2^64 above its unit's first-step column maximum (log2
+// domain) sends the unit to the exact fallback kernel.  Below it nothing
+// overflows: P <= 2^64 in bf16, row sums <= 2^81 and O in fp32.
+constexpr float kFlagThreshold = 64.0f;
 
 struct Bars {
   uint64_t unit_full[kUnits], unit_empty[kUnits];
@@ -103,6 +106,7 @@ struct Ctrl {
   UnitEntry unit[kUnits];
   uint32_t tmem_base;
   int abort_flag;
+  int redo_unit;  // the last unit this CTA flagged for the exact fallback
   alignas(16) float red[kWG][2][4][kCols];  // read with 16-byte vector loads
 #ifdef SEER_TRACE
   unsigned long long trace[24];
@@ -385,6 +389,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #endif
   if (threadIdx.x == 0) {
     C.abort_flag = 0;
+    C.redo_unit = -1;
     for (int s = 0; s < kUnits; ++s) {
       mbar_init(&bars.unit_full[s], 1);
       mbar_init(&bars.unit_empty[s], 2 + kSoftmaxWarps);  // both MMA warps + softmax warps, on reading
@@ -667,51 +672,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           const float dmax =
               fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
                     fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
-          // probabilities with the running max, stored before the vote; the
-          // barrier then tells whether any score of the step exceeded the
-          // running max by more than 2^8, in which case they are redone
+          // The running maximum stays at the first step's: no rescale, no
+          // per-step barrier.  A score far above it flags the unit, which the
+          // fallback kernel then recomputes exactly (one list entry per unit:
+          // the first warp to flag it appends it).
+          if (__any_sync(0xffffffffu, dmax > kFlagThreshold) && lane == 0 && atomicExch(&C.redo_unit, w) != w) {
+            const uint32_t e = atomicAdd(p.redo_count, 1u);
+            if (e < (uint32_t)p.redo_cap) p.redo_list[e] = w;
+          }
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
           store_p(prow, x, wgi, kl);
-          SEER_MARK(16);
-          if (SEER_TIMED_L0(8, bar_red_or(bar_id, 128, !okS || !okP || dmax > kRescaleThreshold))) {
-            if (*abort_p) { fail = true; break; }
-            if (lane == 0) SEER_TRACE_ADD(13, 1);
-            // exact column maxima of this step relative to the running max
-            scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
-            float* red = &C.red[wgi][red_use & 1][0][0];
-            warp_reduce_scatter16<false>(x, lane, red + ww * kCols);
-            ++red_use;
-            bar_red_or(bar_id, 128, false);
-            col_combine<false>(red, x);
-            float (&inc)[kCols] = x;  // increase of the running max per column
-#pragma unroll
-            for (int q = 0; q < kCols; ++q) inc[q] = fmaxf(inc[q], 0.f);
-#pragma unroll
-            for (int q = 0; q < kCols / 2; ++q) {
-              nm2[q] = add_f32x2(nm2[q], f32x2_pack(-inc[2 * q], -inc[2 * q + 1]));
-              lp2[q] = mul_f32x2(lp2[q], f32x2_pack(ex2_approx(-inc[2 * q]), ex2_approx(-inc[2 * q + 1])));
-            }
-            // O^T columns are rescaled once the previous PV has landed
-            const int gp = g - 1;
-            const bool okPV = mbar_wait(&bars.pv_done[gp % kRing], (gp / kRing) & 1, abort_p, p.status, tmo);
-            if (okPV) {
-              tc_fence_after();
-              uint32_t o[16];
-              tmem_ld16(lane_addr + kColO + q0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 16; ++q)
-                o[q] = __float_as_uint(__uint_as_float(o[q]) * ex2_approx(-inc[q]));
-              tmem_st16(lane_addr + kColO + q0, o);
-              tmem_wait_st();
-            }
-            if (bar_red_or(bar_id, 128, !okPV)) { fail = true; break; }
-            scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
-#pragma unroll
-            for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
-            store_p(prow, x, wgi, kl);
-          }
           SEER_MARK(17);
         }
         // row-sum partials
@@ -881,6 +852,79 @@ __global__ void __launch_bounds__(256) empty_rows_kernel(const int32_t* __restri
     lse[u * 64 + lane] = -INFINITY;
     lse[u * 64 + 32 + lane] = -INFINITY;
   }
+}
+
+// Exact recomputation of the units the attention kernel flagged: plain fp32
+// online softmax that rescales at every key, one warp per query row, lanes
+// splitting the head dimension.  It reads the same bf16 Q and K/V block
+// records as the attention kernel (so fp32 inputs see the same rounding), and
+// the same checked list entries.  Slow by design: it only runs for inputs
+// whose scores rise more than 2^64 above a unit's first-step maximum.
+template <int D>
+__global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat16* __restrict__ Q16,
+                                                               const __nv_bfloat16* __restrict__ recs,
+                                                               const AttnParams p) {
+  constexpr int DL = D / 32;  // head dims per lane
+  const uint32_t nredo = min(*reinterpret_cast<volatile uint32_t*>(p.redo_count), (uint32_t)p.redo_cap);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  for (uint32_t e = blockIdx.x; e < nredo; e += gridDim.x) {
+    const int w = p.redo_list[e];
+    const UnitInfo u = decode_unit(p, w);
+    const int* lst = p.indices + u.u * p.cap;
+    const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;
+    for (int r = warp; r < 64; r += 8) {
+      const long long qrow = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + r;
+      float q[DL], o[DL];
+#pragma unroll
+      for (int k = 0; k < DL; ++k) {
+        q[k] = __bfloat162float(Q16[qrow * D + lane * DL + k]);
+        o[k] = 0.f;
+      }
+      float m = -INFINITY, l = 0.f;
+      int prev = -1;
+      for (int t = 0; t < u.count; ++t) {
+        const int raw = lst[t];
+        const int j = checked_entry(p, u, raw, prev);
+        prev = raw;
+        const __nv_bfloat16* rec = recs + (rec0 + j) * (2LL * D * 64);
+        const int kmax = j == u.i ? r : 63;  // causal inside the diagonal block
+        for (int key = 0; key <= kmax; ++key) {
+          float sdot = 0.f;
+#pragma unroll
+          for (int k = 0; k < DL; ++k) sdot += q[k] * __bfloat162float(rec[(lane * DL + k) * 64 + key]);
+          const float sc = warp_sum(sdot) * p.scale_log2;
+          const float mn = fmaxf(m, sc);
+          const float a = exp2f(m - mn), pr = exp2f(sc - mn);
+          l = l * a + pr;
+#pragma unroll
+          for (int k = 0; k < DL; ++k) {
+            const int dim = lane * DL + k;
+            const float v = __bfloat162float(rec[D * 64 + (dim / 64) * 4096 + key * 64 + (dim % 64)]);
+            o[k] = o[k] * a + pr * v;
+          }
+          m = mn;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < DL; ++k) {
+        const float v = o[k] / l;
+        const long long idx = qrow * D + lane * DL + k;
+        if (p.out_fp32)
+          reinterpret_cast<float*>(p.O)[idx] = v;
+        else
+          reinterpret_cast<__nv_bfloat16*>(p.O)[idx] = __float2bfloat16_rn(v);
+      }
+      if (lane == 0 && p.lse) p.lse[qrow] = (m + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+}
+
+cudaError_t launch_sparse_attn_redo(const void* Q16, const void* recs, const AttnParams& p, cudaStream_t st) {
+  if (p.d == 64)
+    sparse_attn_redo_kernel<64><<<148, 256, 0, st>>>((const __nv_bfloat16*)Q16, (const __nv_bfloat16*)recs, p);
+  else
+    sparse_attn_redo_kernel<128><<<148, 256, 0, st>>>((const __nv_bfloat16*)Q16, (const __nv_bfloat16*)recs, p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st) {

@@ -19,12 +19,21 @@ struct AttnParams {
   uint32_t* work_counter;    // workspace work counter (zeroed per call)
   unsigned long long timeout_ns;
   unsigned long long* trace;  // 16 cycle counters (only with -DSEER_TRACE)
+  uint32_t* redo_count;       // units flagged for the exact fallback (workspace)
+  int* redo_list;             // [redo_cap] flagged unit indices
+  int redo_cap;
 };
 
 // Re-layout of K and V into per-block records of 2*d rows x 64 bf16 (K^T,
 // then V in 64-column panels); `records` = B * Hkv * n/64.
 cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
                             int n, int d, cudaStream_t st);
+
+// Exact fp32 recomputation of the units the attention kernel flagged (a
+// score above the unit's first-step column maximum by more than 2^64);
+// returns at once when none was.  Q16 is the bf16 Q the attention kernel
+// read, recs the K/V block records.  Launch after launch_sparse_attn.
+cudaError_t launch_sparse_attn_redo(const void* Q16, const void* recs, const AttnParams& p, cudaStream_t st);
 
 // O = 0 and LSE = -inf for every unit whose list is empty (count <= 0); the
 // attention kernel skips those units.  Launch before launch_sparse_attn.

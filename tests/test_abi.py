@@ -67,7 +67,9 @@ def test_workspace_sizes_cover_their_buffers():
                 + B * Hq * nb * nb)
     assert g >= need + 256 and g % 256 == 0
     # bf16: header + the K/V block records (K^T and V of every 64-key block)
-    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256 + 2 * 2 * B * Hkv * n * d
+    # + the list of units flagged for the exact fallback (one int32 per unit)
+    redo = -(-(4 * B * Hq * nb) // 256) * 256
+    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256 + 2 * 2 * B * Hkv * n * d + redo
     f32 = seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 1)
     assert f32 >= 256 + 2 * n * d * (Hq + 2 * Hkv)
     assert seer.blockmax_workspace_size(B, Hq, Hkv, n, d, 0) >= 256 + 4 * 128 * nb

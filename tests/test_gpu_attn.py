@@ -7,7 +7,7 @@ import learned_block_sparse_seer_b200 as seer
 import oracle
 from learned_block_sparse_seer_b200 import synth
 
-from gpu_common import (LSE_TOL_FP32_INPUT, check_lse, check_o, inputs, sample_units, to_dev,
+from gpu_common import (LSE_TOL, LSE_TOL_FP32_INPUT, check_lse, check_o, inputs, sample_units, to_dev,
                         unit_rows)
 
 pytestmark = pytest.mark.gpu
@@ -126,6 +126,40 @@ def test_edge_cases(B, Hq, Hkv, nb, d):
     check_lse(lse.double().numpy(), lse_ref)
     empty = counts == 0
     assert torch.all(O.view(B, Hq, nb, 64, d)[torch.as_tensor(empty)] == 0)
+
+
+@pytest.mark.parametrize("d,dtype", [(128, torch.bfloat16), (64, torch.bfloat16), (128, torch.float32)])
+def test_score_far_above_first_step_takes_exact_fallback(d, dtype):
+    """The attention kernel keeps each unit's running maximum at its first
+    step's column maximum.  A later key whose score is far above it (here a
+    shifted query block against one large key in a later block: about 2^120
+    in probability) must still give the exact softmax: the kernel flags the
+    unit and the fallback kernel recomputes it."""
+    nb = 7
+    w = synth.custom("spike", 1, 2, 1, 64 * nb, d, 16, "bf16", "layer", 31)
+    Q, K, V = synth.make_qkv(w)
+    Q = Q.float()
+    K = K.float()
+    Q[:, :, 64 * 3:, :] += 2.0
+    K[:, :, 64 * 3 + 8, :] = 4.0
+    Q, K, V = Q.to(dtype), K.to(dtype), V.to(dtype)
+    counts, idx = oracle.dense_lists(1, 2, nb)
+    Qd, Kd, Vd = to_dev(Q, K, V)
+    ws = torch.empty(seer.sparse_attn_workspace_size(1, 2, 1, 64 * nb, d,
+                                                     0 if dtype == torch.bfloat16 else 1),
+                     dtype=torch.uint8, device="cuda")
+    O, lse = seer.seer_sparse_attn(Qd, Kd, Vd, torch.as_tensor(counts).cuda(),
+                                   torch.as_tensor(idx).cuda(), workspace=ws)
+    assert seer.seer_workspace_status(ws) == 0
+    # the header's second work counter holds the number of flagged units
+    assert int(ws[12:16].view(torch.int32).item()) > 0
+    # fp32 inputs are converted to bf16 before the tensor-core pass; with
+    # logits near 100 that rounding alone moves the LSE by up to ~0.4, so the
+    # oracle is given the same bf16 values
+    Qr, Kr, Vr = (t.to(torch.bfloat16) for t in (Q, K, V))
+    O_ref, lse_ref = oracle.sparse_attn(Qr, Kr, Vr, counts, idx)
+    check_o(O.double().cpu().numpy(), O_ref)
+    check_lse(lse.double().cpu().numpy(), lse_ref, LSE_TOL)
 
 
 def test_bad_lists_are_flagged_not_followed():
