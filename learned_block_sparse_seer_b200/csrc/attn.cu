@@ -352,16 +352,14 @@ __device__ __forceinline__ void scores_minus_max(uint32_t taddr, float (&x)[attn
 
 // This warpgroup's 16 bf16 probabilities of key row kl into the step's P^T
 // tile (128-byte rows, 16-byte chunks swizzled by the row index).
-__device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kCols], int wgi, int kl) {
+// off0/off1 are the row's two swizzled 16-byte chunk offsets.
+__device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kCols], uint32_t off0, uint32_t off1) {
+  static_assert(attn::kCols == 16, "two 16-byte chunks per row and warpgroup");
   uint32_t pk[attn::kCols / 2];
 #pragma unroll
   for (int q = 0; q < attn::kCols; q += 2) pk[q >> 1] = pack_bf16x2(x[q], x[q + 1]);
-#pragma unroll
-  for (int ch = 0; ch < attn::kCols / 8; ++ch) {
-    const int chunk = wgi * (attn::kCols / 8) + ch;
-    *reinterpret_cast<uint4*>(prow + ((chunk ^ (kl & 7)) << 4)) =
-        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-  }
+  *reinterpret_cast<uint4*>(prow + off0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  *reinterpret_cast<uint4*>(prow + off1) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
 template <int D>
@@ -615,6 +613,14 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // running maximum (log2 domain) and this thread's row-sum partial.
     uint64_t nm2[kCols / 2], lp2[kCols / 2];
     const uint64_t c2 = f32x2_pack(c, c);
+    // this thread's P^T row (key kl of half `half`) and its two swizzled
+    // 16-byte chunks (this warpgroup's 16 query columns)
+    uint8_t* const prow0 = smem + kOffP + half * 8192 + kl * 128;
+    const uint32_t poff0 = (uint32_t)(((2 * wgi) ^ (kl & 7)) << 4);
+    const uint32_t poff1 = (uint32_t)(((2 * wgi + 1) ^ (kl & 7)) << 4);
+    // ring positions of the current step g: barrier ring slot and phase,
+    // S^T buffer, P^T slot
+    int rg = 0, rph = 0, sb = 0, ps = 0;
     for (;;) {
       const int slot = u_idx % kUnits;
       const bool okw = mbar_wait(&bars.unit_full[slot], (u_idx / kUnits) & 1, abort_p, p.status, tmo);
@@ -634,23 +640,25 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       bool fail = false;
       for (int t = 0; t < T; ++t) {
         const int g = step + t;
+        (void)g;
         const int mi = 2 * t + half;
         const bool valid = mi < count;
         const bool diag = valid && last_is_diag && mi == count - 1;
-        const bool okS = SEER_TIMED_L0(6, mbar_wait(&bars.qk_done[g % kRing], (g / kRing) & 1, abort_p, p.status, tmo));
-        // P^T(g) goes to the slot of step g-2, free once PV(g-2) is complete
-        // (long done in steady state); a failed wait joins the step's first
-        // barrier below.
-        const bool okP = g < kPSlots || mbar_wait(&bars.pv_done[(g - kPSlots) % kRing], ((g - kPSlots) / kRing) & 1,
-                                                  abort_p, p.status, tmo);
+        const bool okS = SEER_TIMED_L0(6, mbar_wait(&bars.qk_done[rg], rph, abort_p, p.status, tmo));
+        // P^T(g) goes to the slot of step g-kPSlots, free once that step's PV
+        // is complete (long done in steady state); a failed wait joins the
+        // unit's next barrier.
+        static_assert(kPSlots <= kRing, "P^T slot reuse is tracked on the pv_done ring");
+        const int pr = rg >= kPSlots ? rg - kPSlots : rg - kPSlots + kRing;
+        const int pph = rg >= kPSlots ? rph : rph ^ 1;
+        const bool okP = g < kPSlots || mbar_wait(&bars.pv_done[pr], pph, abort_p, p.status, tmo);
 #ifdef SEER_TRACE
         const long long tstep0 = clock64();
         long long tmark = tstep0;
 #endif
         tc_fence_after();
-        const uint32_t saddr = lane_addr + (uint32_t)(g % kSBuf) * 64u + q0;
-        // P^T row `kl` of half `half` of the step's P^T slot
-        uint8_t* prow = smem + kOffP + (g % kPSlots) * kPBytes + half * 8192 + kl * 128;
+        const uint32_t saddr = lane_addr + (uint32_t)sb * 64u + q0;
+        uint8_t* const prow = prow0 + ps * kPBytes;
         float x[kCols];
         if (t == 0) {
           // exact column maxima of the unit's first step
@@ -666,7 +674,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
-          store_p(prow, x, wgi, kl);
+          store_p(prow, x, poff0, poff1);
         } else {
           if (okS) scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
           const float dmax =
@@ -682,7 +690,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           }
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
-          store_p(prow, x, wgi, kl);
+          store_p(prow, x, poff0, poff1);
           SEER_MARK(17);
         }
         // row-sum partials
@@ -694,9 +702,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bars.go[g % kRing]);
-          mbar_arrive(&bars.kfull[(g + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
+          mbar_arrive(&bars.go[rg]);
+          mbar_arrive(&bars.kfull[(rg + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
         }
+        if (++rg == kRing) {
+          rg = 0;
+          rph ^= 1;
+        }
+        sb = sb + 1 == kSBuf ? 0 : sb + 1;
+        ps = ps + 1 == kPSlots ? 0 : ps + 1;
         SEER_MARK(22);
 #ifdef SEER_TRACE
         if (lane == 0) SEER_TRACE_ADD(9, clock64() - tstep0);
@@ -707,8 +721,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #ifdef SEER_TRACE
       const long long tep0 = clock64();
 #endif
-      const int gl = step + T - 1;
-      const bool okPV = mbar_wait(&bars.pv_done[gl % kRing], (gl / kRing) & 1, abort_p, p.status, tmo);
+      // the unit's last step is the one before the current ring position
+      const bool okPV = mbar_wait(&bars.pv_done[rg > 0 ? rg - 1 : kRing - 1], rg > 0 ? rph : rph ^ 1, abort_p,
+                                  p.status, tmo);
       float* red = &C.red[wgi][red_use & 1][0][0];
       float lpart[kCols];
 #pragma unroll
