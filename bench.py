@@ -27,7 +27,8 @@ import subprocess
 import sys
 import threading
 import time
-import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -466,11 +467,20 @@ def main():
     sweep = None
     if args.sweep and rank == 0:
         sweep = []
-        for rho in (0.5, 0.3, 0.2, 0.1, 0.05):
-            c2 = seer.gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, "density", density=rho)
+        # top-k density sweep (50..95 % block sparsity), then threshold mode
+        cases = [("density", rho) for rho in (0.5, 0.3, 0.2, 0.1, 0.05)] + \
+                [("threshold", t) for t in (1e-4, 5e-4, 2e-3)]
+        for mode, val in cases:
+            if mode == "density":
+                c2 = seer.gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, "density", density=val)
+            else:
+                c2 = seer.gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, "threshold")
             cc = torch.empty(w.B, w.Hq, nb, dtype=torch.int32, device=dev)
             ii = torch.empty(w.B, w.Hq, nb, c2, dtype=torch.int32, device=dev)
-            seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=rho, cap=c2, workspace=gws, out=(cc, ii, None))
+            if mode == "density":
+                seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=val, cap=c2, workspace=gws, out=(cc, ii, None))
+            else:
+                seer.seer_gate(Qd, Kd, Wqd, Wkd, "threshold", T=val, cap=c2, workspace=gws, out=(cc, ii, None))
             for _ in range(2):
                 seer.seer_sparse_attn(Qd, Kd, Vd, cc, ii, workspace=aws, out=(O, lse))
             torch.cuda.synchronize(dev)
@@ -482,8 +492,18 @@ def main():
             torch.cuda.synchronize(dev)
             ms = a.elapsed_time(b) / 3
             f, nbk, _, sp = attn_flops(cc, ii, w.d)
-            sweep.append({"density": rho, "sparsity": sp, "active_blocks": nbk, "attn_ms": ms,
+            sweep.append({mode: val, "sparsity": sp, "active_blocks": nbk, "attn_ms": ms,
                           "tflops": f / (ms * 1e-3) / 1e12})
+            del cc, ii
+        # time against active tiles over the density sweep: least-squares line and R^2
+        pts = [(e["active_blocks"], e["attn_ms"]) for e in sweep if "density" in e]
+        xs = np.array([x for x, _ in pts], dtype=np.float64)
+        ys = np.array([y for _, y in pts], dtype=np.float64)
+        slope, icpt = np.polyfit(xs, ys, 1)
+        resid = ys - (slope * xs + icpt)
+        r2 = 1.0 - float((resid ** 2).sum() / max(((ys - ys.mean()) ** 2).sum(), 1e-30))
+        sweep.append({"fit": "attn_ms = a * active_blocks + b over the density sweep",
+                      "a_ms_per_block": float(slope), "b_ms": float(icpt), "r2": r2})
 
     # ------------------------------------------------------ oracle baseline --
     cpu = None
