@@ -156,7 +156,7 @@ BmaxWs bmax_ws(const seer_dims* d, seer_dtype dt, int sms) {
   }
   const long long nb = d->n / seer::kBlock;
   w.ctas = sms;
-  w.r = c.take(sizeof(float) * (size_t)sms * 128 * nb);
+  w.r = c.take(sizeof(float) * (size_t)sms * 256 * nb);  // [ctas][nb][2 column halves][128 rows]
   w.total = c.off;
   return w;
 }

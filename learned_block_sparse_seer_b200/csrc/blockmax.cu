@@ -14,18 +14,23 @@
 //  * A unit is one query head and two consecutive 64-row query blocks
 //    (i0 = 2m, i1 = 2m+1): a 128-row tile, so every tcgen05 MMA is
 //    M = 128 x N = 128 (two key blocks per step), both operands from 128-byte
-//    swizzled shared memory loaded by TMA (no multicast), S in TMEM.
-//  * Two softmax warpgroups split the 128 score columns (one key block each);
-//    each thread owns one query row, keeps its own (max, sum) with a lazily
-//    raised running max, and stores its per-key-block raw maxima to a per-CTA
-//    scratch slot (L2-resident, rewritten by every unit).
-//  * The second pass runs in the unit's epilogue: every thread reads back the
-//    maxima it stored, turns them into probabilities with the final
-//    log-sum-exp, and a shuffle reduce-scatter takes the maximum over the 64
-//    rows of each query block.
-//  * Warp roles (384 threads): warp 0 schedules units and loads Q, warp 1
-//    loads K pairs, warp 2 issues the MMAs, warps 4..7 and 8..11 are the two
-//    softmax warpgroups.  All waits are bounded.
+//    swizzled shared memory loaded by TMA (no multicast), S in TMEM (three
+//    buffers, so the MMA runs up to two steps ahead of the softmax).
+//  * The work is bound by the exponentials (one per causal pair; the MMA is
+//    half as long), so four softmax warpgroups share each step: warpgroup w
+//    takes the 32 score columns of key block 2s + (w >> 1), half (w & 1).
+//    Each thread owns one query row, keeps its own (max, sum) with a lazily
+//    raised running max, uses packed f32x2 arithmetic and 3-input max trees,
+//    and stores its per-half-block raw maximum to a per-CTA scratch slot
+//    (L2-resident, rewritten by every unit).
+//  * The second pass runs in the unit's epilogue: the four warpgroups'
+//    statistics give each row's log-sum-exp; then each warpgroup takes every
+//    fourth key block, reads both halves' kept maxima of each row, turns them
+//    into probabilities, and a shuffle reduce-scatter takes the maximum over
+//    the 64 rows of each query block.
+//  * Warp roles (608 threads): warps 0..15 are the softmax warpgroups, warp
+//    16 schedules units and loads Q, warp 17 loads K pairs, warp 18 issues
+//    the MMAs (straight-line, unrolled groups).  All waits are bounded.
 #include <cstdint>
 
 #include "blockmax.cuh"
@@ -35,27 +40,30 @@
 namespace seer {
 
 namespace bmax {
-constexpr int kThreads = 384;
-constexpr int kNK = 4;
+constexpr int kThreads = 608;
+constexpr int kWarpSched = 16, kWarpK = 17, kWarpMma = 18;
+constexpr int kWG = 4;                  // softmax warpgroups
+constexpr int kSoftmaxWarps = 4 * kWG;
+constexpr int kNK = 4;                  // K pair ring
+constexpr int kSBuf = 3;                // S buffers in TMEM (128 columns each)
 constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 dims x bf16
 constexpr uint32_t kOffQ = 0;           // 2 x 32 KB
 constexpr uint32_t kOffK = 2 * kTileBytes;
 constexpr uint32_t kSmemTiles = kOffK + kNK * kTileBytes;  // 192 KB
-constexpr uint32_t kTmemCols = 256;                        // S x 2 (128 cols each)
+constexpr uint32_t kTmemCols = 512;                        // S x 3 (128 cols each)
 constexpr float kRaise = 8.0f;
 
 struct Ctrl {
   uint64_t unit_full[2], unit_empty[2];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kNK], k_empty[kNK];
-  uint64_t s_full[2], s_free[2];
-  uint64_t wg[2], both, fin;
+  uint64_t s_full[kSBuf], s_free[kSBuf];
+  uint64_t wg[kWG], all, fin;
   int unit_w[2];
   uint32_t tmem_base;
   int abort_flag;
-  float m_part[2][128], l_part[2][128];
-  float lse2[128];
-  float red[2][4][32];
+  float m_part[kWG][128], l_part[kWG][128];
+  float red[kWG][4][32];
 };
 constexpr uint32_t kSmemAlloc = kSmemTiles + (uint32_t)sizeof(Ctrl);
 static_assert(kSmemAlloc <= 232448, "dynamic shared memory above the per-CTA limit");
@@ -63,6 +71,7 @@ static_assert(kSmemAlloc <= 232448, "dynamic shared memory above the per-CTA lim
 
 namespace {
 
+// A named group of warps meeting at an mbarrier (one arrival per warp).
 struct Sync {
   uint64_t* bar;
   volatile int* abort;
@@ -95,6 +104,7 @@ __device__ __forceinline__ BUnit decode(const BmaxParams& p, int w) {
 
 }  // namespace
 
+template <int D>
 __global__ void __launch_bounds__(bmax::kThreads, 1)
     blockmax_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const BmaxParams p) {
@@ -113,22 +123,24 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
     C.abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&C.unit_full[s], 1);
-      mbar_init(&C.unit_empty[s], 2 + 8);  // K loader, MMA, 8 softmax warps
+      mbar_init(&C.unit_empty[s], 2 + kSoftmaxWarps);  // K loader, MMA, softmax warps
       mbar_init(&C.q_full[s], 1);
       mbar_init(&C.q_empty[s], 1);
-      mbar_init(&C.s_full[s], 1);
-      mbar_init(&C.s_free[s], 8);
-      mbar_init(&C.wg[s], 4);
     }
+    for (int s = 0; s < kSBuf; ++s) {
+      mbar_init(&C.s_full[s], 1);
+      mbar_init(&C.s_free[s], kSoftmaxWarps);
+    }
+    for (int s = 0; s < kWG; ++s) mbar_init(&C.wg[s], 4);
     for (int s = 0; s < kNK; ++s) {
       mbar_init(&C.k_full[s], 1);
       mbar_init(&C.k_empty[s], 1);
     }
-    mbar_init(&C.both, 8);
+    mbar_init(&C.all, kSoftmaxWarps);
     mbar_init(&C.fin, 1);
     fence_barrier_init();
   }
-  if (warp == 2) {
+  if (warp == kWarpMma) {
     tmem_alloc(&C.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -136,10 +148,10 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
-  const int dpanels = p.d / 64;
-  const uint32_t tile_bytes = 128u * p.d * 2u;
+  constexpr int dpanels = D / 64;
+  constexpr uint32_t tile_bytes = 128u * D * 2u;
 
-  if (warp == 0) {
+  if (warp == kWarpSched) {
     // ------------------------------------------------ scheduler + Q loads --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -165,7 +177,7 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
         mbar_wait(&C.q_full[uu & 1], (uu >> 1) & 1, abort_p, nullptr, 20000000ull);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpK) {
     // --------------------------------------------------------- K loads ---
     if (lane == 0) {
       prefetch_tmap(&tmK);
@@ -197,13 +209,16 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
         mbar_wait(&C.k_full[st % kNK], (st / kNK) & 1, abort_p, nullptr, 20000000ull);
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA ----
+    // Straight-line groups: descriptors are a per-step base plus constant
+    // offsets (the start address field holds address >> 4).
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t sbase = smem_u32(smem);
-      const int ksteps = p.d / 16;
-      int u_idx = 0, step = 0;
+      const uint64_t dQ0 = make_sw128_desc(sbase + kOffQ, 16, 1024);
+      const uint64_t dK0 = make_sw128_desc(sbase + kOffK, 16, 1024);
+      int u_idx = 0, g = 0, ks = 0, kph = 0, sb = 0, sph = 0;
       bool ok = true;
       while (ok) {
         const int slot = u_idx & 1;
@@ -213,42 +228,51 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
         if (w < 0) break;
         const BUnit u = decode(p, w);
         if (!mbar_wait(&C.q_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
-        const uint32_t qa = sbase + kOffQ + slot * kTileBytes;
-        for (int s = 0; s <= u.m; ++s) {
-          const int g = step + s;
-          const int ks = g % kNK;
-          if (!mbar_wait(&C.k_full[ks], (g / kNK) & 1, abort_p, p.status, tmo)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(&C.s_free[g & 1], ((g - 2) >> 1) & 1, abort_p, p.status, tmo)) { ok = false; break; }
+        const uint64_t dq = dQ0 + ((uint64_t)(slot * kTileBytes) >> 4);
+        for (int s = 0; s <= u.m; ++s, ++g) {
+          if (!mbar_wait(&C.k_full[ks], kph, abort_p, p.status, tmo)) { ok = false; break; }
+          // S buffer sb was last read by the softmax of step g - kSBuf
+          if (g >= kSBuf && !mbar_wait(&C.s_free[sb], sph ^ 1, abort_p, p.status, tmo)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t ka = sbase + kOffK + ks * kTileBytes;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + (g & 1) * 128, make_sw128_desc(qa + off, 16, 1024),
-                        make_sw128_desc(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          const uint64_t dk = dK0 + ((uint64_t)(ks * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) / 16);
+            mma_bf16_ss(tmem + (uint32_t)sb * 128u, dq + off, dk + off, idesc, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&C.s_full[g & 1]);
+          mma_commit(&C.s_full[sb]);
           mma_commit(&C.k_empty[ks]);
+          if (++ks == kNK) {
+            ks = 0;
+            kph ^= 1;
+          }
+          if (++sb == kSBuf) {
+            sb = 0;
+            sph ^= 1;
+          }
         }
         if (!ok) break;
         mma_commit(&C.q_empty[slot]);
-        step += u.m + 1;
         ++u_idx;
       }
       mma_commit(&C.fin);
       mbar_wait(&C.fin, 0, abort_p, nullptr, 20000000ull);
     }
-  } else if (warp >= 4) {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------ softmax WGs ---
-    const int wgi = (warp - 4) / 4;   // 0: even key block of a step, 1: odd
-    const int ww = (warp - 4) % 4;    // TMEM sub-partition
-    const int row = ww * 32 + lane;   // 0..127
+    const int wgi = warp >> 2;          // warpgroup 0..3
+    const int ww = warp & 3;            // TMEM sub-partition
+    const int row = ww * 32 + lane;     // query row of the unit's tile, 0..127
     const int half = row >> 6, rloc = row & 63;
-    const uint32_t lane_addr = tmem + ((uint32_t)(ww * 32) << 16) + wgi * 64;
+    const int jo = wgi >> 1, hh = wgi & 1;  // key block of the pair, column half
+    const uint32_t lane_addr = tmem + ((uint32_t)(ww * 32) << 16) + (uint32_t)(jo * 64 + hh * 32);
     const float c = p.scale_log2;
+    const uint64_t c2 = f32x2_pack(c, c);
     Sync wgs{&C.wg[wgi], abort_p, p.status, tmo, 0};
-    Sync both{&C.both, abort_p, p.status, tmo, 0};
-    float* rslot = p.r + (long long)blockIdx.x * 128 * p.nb;
-    int u_idx = 0, step = 0;
+    Sync all{&C.all, abort_p, p.status, tmo, 0};
+    // per-CTA scratch: [key block][column half][128 rows] raw maxima (log2)
+    float* rslot = p.r + (long long)blockIdx.x * 256 * p.nb;
+    int u_idx = 0, sb = 0, sph = 0;
     for (;;) {
       const int slot = u_idx & 1;
       if (!mbar_wait(&C.unit_full[slot], (u_idx >> 1) & 1, abort_p, p.status, tmo)) break;
@@ -258,70 +282,89 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
       if (w < 0) break;
       ++u_idx;
       const BUnit u = decode(p, w);
-      const int irow = 2 * u.m + half;        // query block of this row
+      const int irow = 2 * u.m + half;  // query block of this row
       const bool row_valid = irow < p.nb;
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int s = 0; s <= u.m; ++s) {
-        const int g = step + s;
-        const int j = 2 * s + wgi;           // key block of these columns
-        if (!mbar_wait(&C.s_full[g & 1], (g >> 1) & 1, abort_p, p.status, tmo)) { ok = false; break; }
+        const int j = 2 * s + jo;  // key block of these columns
+        if (!mbar_wait(&C.s_full[sb], sph, abort_p, p.status, tmo)) { ok = false; break; }
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_addr + (g & 1) * 128, r0);
-        tmem_ld32(lane_addr + (g & 1) * 128 + 32, r1);
+        uint32_t r[32];
+        tmem_ld32(lane_addr + (uint32_t)sb * 128u, r);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&C.s_free[g & 1]);
-        if (j > irow || !row_valid) continue;  // key block entirely in the future
-        float x[64];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          x[q] = __uint_as_float(r0[q]) * c;
-          x[q + 32] = __uint_as_float(r1[q]) * c;
+        if (lane == 0) mbar_arrive(&C.s_free[sb]);
+        if (++sb == kSBuf) {
+          sb = 0;
+          sph ^= 1;
         }
+        if (j > irow || !row_valid) continue;  // key block entirely in the future
+        float x[32];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          f32x2_unpack(mul_f32x2(f32x2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), c2),
+                       x[2 * q], x[2 * q + 1]);
         if (j == irow) {
 #pragma unroll
-          for (int q = 0; q < 64; ++q) x[q] = q > rloc ? -INFINITY : x[q];
+          for (int q = 0; q < 32; ++q) x[q] = hh * 32 + q > rloc ? -INFINITY : x[q];
         }
-        float mx = x[0];
+        float t[11];
 #pragma unroll
-        for (int q = 1; q < 64; ++q) mx = fmaxf(mx, x[q]);
-        rslot[(long long)j * 128 + row] = mx;
+        for (int q = 0; q < 10; ++q) t[q] = fmax3(x[3 * q], x[3 * q + 1], x[3 * q + 2]);
+        t[10] = fmaxf(x[30], x[31]);
+        const float mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]),
+                               fmax3(fmax3(t[6], t[7], t[8]), t[9], t[10]));
+        rslot[((long long)j * 2 + hh) * 128 + row] = mx;
         if (mx > m_run + kRaise) {
           l_run *= ex2_approx(m_run - mx);
           m_run = mx;
         }
-        float sum = 0.f;
+        const uint64_t nm2 = f32x2_pack(-m_run, -m_run);
+        uint64_t acc = 0ull;
 #pragma unroll
-        for (int q = 0; q < 64; ++q) sum += ex2_approx(x[q] - m_run);
-        l_run += sum;
+        for (int q = 0; q < 16; ++q) {
+          float a, b;
+          f32x2_unpack(add_f32x2(f32x2_pack(x[2 * q], x[2 * q + 1]), nm2), a, b);
+          acc = add_f32x2(acc, f32x2_pack(ex2_approx(a), ex2_approx(b)));
+        }
+        float s0, s1;
+        f32x2_unpack(acc, s0, s1);
+        l_run += s0 + s1;
       }
       if (!ok) break;
-      // ---- combine the two warpgroups' statistics into the row's lse (log2)
+      // ---- combine the four warpgroups' statistics into the row's lse (log2)
       C.m_part[wgi][row] = m_run;
       C.l_part[wgi][row] = l_run;
-      if (!both.sync(lane)) break;
-      float lse2 = -INFINITY;
+      if (!all.sync(lane)) break;
+      float lse2;
       {
-        const float m0 = C.m_part[0][row], m1 = C.m_part[1][row];
-        const float mm = fmaxf(m0, m1);
-        const float l = (m0 > -INFINITY ? C.l_part[0][row] * ex2_approx(m0 - mm) : 0.f) +
-                        (m1 > -INFINITY ? C.l_part[1][row] * ex2_approx(m1 - mm) : 0.f);
+        float mm = C.m_part[0][row];
+#pragma unroll
+        for (int k = 1; k < kWG; ++k) mm = fmaxf(mm, C.m_part[k][row]);
+        float l = 0.f;
+#pragma unroll
+        for (int k = 0; k < kWG; ++k) {
+          const float mk = C.m_part[k][row];
+          if (mk > -INFINITY) l += C.l_part[k][row] * ex2_approx(mk - mm);
+        }
         lse2 = mm + log2f(l);
       }
       if (wgi == 0 && row_valid && p.lse)
         p.lse[((long long)u.b * p.Hq + u.hq) * p.n + (long long)irow * 64 + rloc] = lse2 * 0.6931471805599453f;
       // ---- second pass: probabilities of the kept maxima, max over rows ----
-      // this warpgroup owns the key blocks j = 2s + wgi that it stored itself
-      const int nsj = u.m + 1;
-      for (int s0 = 0; s0 < nsj && ok; s0 += 32) {
+      // warpgroup wgi takes key blocks j = wgi, wgi + 4, ... of the unit
+      const int nkb = 2 * (u.m + 1);
+      for (int t0 = 0; 4 * t0 < nkb && ok; t0 += 32) {
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const int j = 2 * (s0 + k) + wgi;
-          v[k] = (s0 + k < nsj && j <= irow && row_valid) ? ex2_approx(rslot[(long long)j * 128 + row] - lse2) : 0.f;
+          const int j = 4 * (t0 + k) + wgi;
+          v[k] = (j < nkb && j <= irow && row_valid)
+                     ? ex2_approx(fmaxf(rslot[((long long)j * 2) * 128 + row], rslot[((long long)j * 2 + 1) * 128 + row]) -
+                                  lse2)
+                     : 0.f;
         }
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -352,15 +395,14 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
           const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
           v[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
         }
-        // lane holds the max over this warp's 32 rows for s = s0 + lane
+        // lane holds the max over this warp's 32 rows for key block 4(t0 + lane) + wgi
         C.red[wgi][ww][lane] = v[0];
         if (!wgs.sync(lane)) { ok = false; break; }
         if (ww == 0 || ww == 2) {
           const int hb = ww >> 1;  // 0: block i0 (warps 0,1), 1: block i1 (warps 2,3)
           const int ib = 2 * u.m + hb;
-          const int s = s0 + lane;
-          const int j = 2 * s + wgi;
-          if (ib < p.nb && s < nsj && j <= ib) {
+          const int j = 4 * (t0 + lane) + wgi;
+          if (ib < p.nb && j < nkb && j <= ib) {
             const float val = fmaxf(C.red[wgi][ww][lane], C.red[wgi][ww + 1][lane]);
             p.map[(((long long)u.b * p.Hq + u.hq) * p.nb + ib) * p.nb + j] = val;
           }
@@ -368,29 +410,28 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
         if (!wgs.sync(lane)) { ok = false; break; }
       }
       if (!ok) break;
-      // keep the statistics area until both warpgroups have read it
-      if (!both.sync(lane)) break;
-      step += u.m + 1;
+      // keep the statistics area until every warpgroup has read it
+      if (!all.sync(lane)) break;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, bmax::kTmemCols);
+  if (warp == bmax::kWarpMma) tmem_dealloc(tmem, bmax::kTmemCols);
 }
 
 cudaError_t launch_blockmax(const CUtensorMap& tmQ, const CUtensorMap& tmK, const BmaxParams& p,
                             int ctas, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(blockmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)bmax::kSmemAlloc);
+  auto kern = p.d == 64 ? blockmax_kernel<64> : blockmax_kernel<128>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bmax::kSmemAlloc);
   if (e != cudaSuccess) return e;
   // entries above the diagonal are 0; the kernel writes j <= i only
   e = cudaMemsetAsync(p.map, 0, sizeof(float) * (size_t)p.B * p.Hq * p.nb * p.nb, st);
   if (e != cudaSuccess) return e;
   long long grid = p.total_units < ctas ? p.total_units : ctas;
   if (grid < 1) grid = 1;
-  blockmax_kernel<<<(unsigned)grid, bmax::kThreads, bmax::kSmemAlloc, st>>>(tmQ, tmK, p);
+  kern<<<(unsigned)grid, bmax::kThreads, bmax::kSmemAlloc, st>>>(tmQ, tmK, p);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@ struct BmaxParams {
   float* map;              // [B, Hq, nb, nb] fp32
   float* lse;              // [B, Hq, n] fp32 or null
   float scale_log2;        // softmax scale * log2(e)
-  float* r;                // scratch: [ctas, nb, 128] per-row block maxima (log2 units)
+  float* r;                // scratch: [ctas, nb, 2, 128] per-row half-block maxima (log2 units)
   uint32_t* status;
   uint32_t* work_counter;
   unsigned long long timeout_ns;
