@@ -300,3 +300,57 @@ def blockmax_units(Q, K, units, scale: float | None = None):
     _load().orc_blockmax_units(_p(q), _p(k), B, Hq, Hkv, n, d, BLOCK, scale, _p(u), len(u),
                                _p(gt), _p(lse))
     return gt, lse
+
+
+# ------------------------------------------------ gate distillation loss ---
+def gate_kl(scores, gt):
+    """KL(gt || score) per query-block row and its gradient with respect to
+    the gate's logits (summary page, section 3.4, "Loss function:
+    KL-divergence"; Eq. 1 for the score).
+
+    Reading: the page treats both maps as row distributions, so each gt row
+    is divided by its sum over the causal blocks j <= i before the
+    divergence; the loss is the mean over all rows (batch x query head x
+    query block).  With g the normalised row and s the score row,
+    loss_row = sum_j g_j (log g_j - log s_j), terms with g_j = 0 being 0, and
+    d loss / d z_ij = (s_ij - g_ij) / rows, since s = softmax(z) over j <= i
+    and sum_j g_j = 1.  Returns (loss, dz [B,Hq,nb,nb], 0 above the diagonal).
+    """
+    s = _f64(scores)
+    g = _f64(gt)
+    B, Hq, nb, _ = s.shape
+    causal = np.tril(np.ones((nb, nb), dtype=bool))
+    g = np.where(causal, g, 0.0)
+    gn = g / g.sum(axis=-1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        terms = np.where(gn > 0, gn * (np.log(gn) - np.log(np.where(causal, s, 1.0))), 0.0)
+    rows = B * Hq * nb
+    loss = terms.sum() / rows
+    dz = np.where(causal, (s - gn) / rows, 0.0)
+    return loss, dz
+
+
+def gate_kl_backward(Q, K, Wq, Wk, gt):
+    """The AttnGate's distillation step without RoPE: forward (pooling,
+    projection, Eq. 1), KL(gt || score) and the gradients of the loss with
+    respect to Wq [Hq,h,d] and Wk [Hkv,h,3d] (summary page, section 3.4:
+    only the gate's linear layers are trained).  Chain rule through
+    z_ij = q~_i . k~_j / sqrt(d), q~ = Wq qbar, k~ = Wk kbar:
+      dq~_i = sum_j dz_ij k~_j / sqrt(d),  dk~_j = sum_{heads of g} sum_i dz_ij q~_i / sqrt(d),
+      dWq[hq] = sum_{b,i} dq~_i qbar_i^T,  dWk[g] = sum_{b,j} dk~_j kbar_j^T.
+    Returns (loss, dWq, dWk) in fp64."""
+    d = Q.shape[-1]
+    qb, kb = pool_q(Q), pool_k(K)
+    qt, kt = project(qb, Wq), project(kb, Wk)
+    s = gate_scores(qt, kt, d)
+    loss, dz = gate_kl(s, gt)
+    B, Hq, nb, h = qt.shape
+    Hkv = kt.shape[1]
+    G = Hq // Hkv
+    kt_q = np.repeat(kt, G, axis=1)                      # KV head of each query head
+    dqt = np.matmul(dz, kt_q) / math.sqrt(d)             # [B,Hq,nb,h]
+    dkt_q = np.matmul(np.swapaxes(dz, -1, -2), qt) / math.sqrt(d)
+    dkt = dkt_q.reshape(B, Hkv, G, nb, h).sum(axis=2)    # [B,Hkv,nb,h]
+    dWq = np.einsum("bhic,bhie->hce", dqt, qb)
+    dWk = np.einsum("bgjc,bgje->gce", dkt, kb)
+    return loss, dWq, dWk

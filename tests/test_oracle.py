@@ -454,3 +454,107 @@ def test_unit_subset_entry_points_agree_with_full_ones():
         np.testing.assert_array_equal(cr, c.reshape(-1)[units])
         for r, u in enumerate(units):
             np.testing.assert_array_equal(ir[r, :cr[r]], ix.reshape(-1, 11)[u, :cr[r]])
+
+
+# ------------------------------------------- gate distillation (KL) -------
+def _gate_torch_chain(Q, K, Wq, Wk):
+    """The gate forward as torch fp64 ops (library pooling and softmax), with
+    Wq and Wk as leaf tensors for autograd."""
+    q = Q.double()
+    k = K.double()
+    B, Hq, n, d = q.shape
+    Hkv = k.shape[1]
+    nb = n // 64
+    qb = F.avg_pool1d(q.reshape(-1, n, d).transpose(1, 2), 64).transpose(1, 2).reshape(B, Hq, nb, d)
+    kt_ = k.reshape(-1, n, d).transpose(1, 2)
+    kb = torch.cat([F.max_pool1d(kt_, 64), -F.max_pool1d(-kt_, 64), F.avg_pool1d(kt_, 64)], dim=1)
+    kb = kb.transpose(1, 2).reshape(B, Hkv, nb, 3 * d)
+    wq = Wq.double().clone().requires_grad_(True)
+    wk = Wk.double().clone().requires_grad_(True)
+    qt = torch.einsum("hcd,bhid->bhic", wq, qb)
+    ktil = torch.einsum("hcd,bhid->bhic", wk, kb)
+    ktil = ktil.repeat_interleave(Hq // Hkv, dim=1)
+    z = torch.matmul(qt, ktil.transpose(-1, -2)) / math.sqrt(d)
+    mask = torch.tril(torch.ones(nb, nb, dtype=torch.bool))
+    logp = torch.log_softmax(z.masked_fill(~mask, float("-inf")), dim=-1)
+    return logp, mask, wq, wk
+
+
+def test_gate_kl_gradients_match_autograd():
+    """Hand-derived chain rule (oracle) against torch autograd through the
+    whole gate on the same inputs, in fp64."""
+    w = synth.custom("kl", 2, 4, 2, 8 * 64, 32, 16, "fp32", "layer", 11)
+    Q, K, _ = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    gt, _ = oracle.blockmax(Q, K)
+    loss, dWq, dWk = oracle.gate_kl_backward(Q, K, Wq, Wk, gt)
+    logp, mask, wq, wk = _gate_torch_chain(Q, K, Wq, Wk)
+    g = torch.from_numpy(gt).masked_fill(~mask, 0.0)
+    g = g / g.sum(dim=-1, keepdim=True)
+    terms = torch.where(g > 0, g * (torch.log(g) - logp.masked_fill(~mask, 0.0)), torch.zeros_like(g))
+    tl = terms.sum() / (g.shape[0] * g.shape[1] * g.shape[2])
+    tl.backward()
+    assert abs(tl.item() - loss) <= 1e-12 * max(1.0, abs(loss))
+    np.testing.assert_allclose(dWq, wq.grad.numpy(), rtol=1e-9, atol=1e-15)
+    np.testing.assert_allclose(dWk, wk.grad.numpy(), rtol=1e-9, atol=1e-15)
+
+
+def test_gate_kl_gradient_by_finite_differences():
+    """Central differences of the oracle's own loss on a tiny gate."""
+    w = synth.custom("klfd", 1, 2, 1, 4 * 64, 16, 8, "fp32", "layer", 13)
+    Q, K, _ = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    Wq = Wq * 20.0   # larger logits so that the loss is not flat
+    Wk = Wk * 20.0
+    gt, _ = oracle.blockmax(Q, K)
+    _, dWq, dWk = oracle.gate_kl_backward(Q, K, Wq, Wk, gt)
+    rng = np.random.default_rng(5)
+    for W, dW, which in ((Wq, dWq, "q"), (Wk, dWk, "k")):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in W.shape)
+            h = 1e-3
+            Wp, Wm = W.clone().double(), W.clone().double()
+            Wp[idx] += h
+            Wm[idx] -= h
+            if which == "q":
+                lp = oracle.gate_kl_backward(Q, K, Wp, Wk, gt)[0]
+                lm = oracle.gate_kl_backward(Q, K, Wm, Wk, gt)[0]
+            else:
+                lp = oracle.gate_kl_backward(Q, K, Wq, Wp, gt)[0]
+                lm = oracle.gate_kl_backward(Q, K, Wq, Wm, gt)[0]
+            fd = (lp - lm) / (2 * h)
+            # central differences carry an O(h^2) truncation error (~1e-5 relative here)
+            assert abs(fd - dW[idx]) <= 1e-4 * max(1e-3, abs(dW[idx])) + 1e-9, (which, idx, fd, dW[idx])
+
+
+def test_gate_kl_zero_at_match_and_nonnegative():
+    w = synth.custom("kl0", 1, 2, 1, 6 * 64, 16, 8, "fp32", "layer", 17)
+    Q, K, _ = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    s = oracle.gate(Q, K, Wq, Wk)
+    # gt equal to the score (up to a per-row factor): zero loss, zero gradient
+    loss, dz = oracle.gate_kl(s * 3.0, s)
+    loss, dz = oracle.gate_kl(s, s * 3.0)
+    assert abs(loss) < 1e-14 and np.abs(dz).max() < 1e-15
+    gt, _ = oracle.blockmax(Q, K)
+    loss, dz = oracle.gate_kl(s, gt)
+    assert loss > 0
+    # each causal row of dz sums to zero (both rows are distributions)
+    assert np.abs(dz.sum(axis=-1)).max() < 1e-15
+
+
+def test_gate_kl_two_block_closed_form():
+    """nb = 2: row 0 has one candidate (loss 0); row 1 is a two-way softmax
+    s = (sigmoid(z0 - z1), sigmoid(z1 - z0)) against g = gt / sum(gt)."""
+    s = np.zeros((1, 1, 2, 2))
+    z0, z1 = 0.3, -0.4
+    s[0, 0, 0, 0] = 1.0
+    s[0, 0, 1, 0] = 1.0 / (1.0 + math.exp(z1 - z0))
+    s[0, 0, 1, 1] = 1.0 / (1.0 + math.exp(z0 - z1))
+    gt = np.array([[[[0.7, 0.0], [0.2, 0.6]]]])
+    loss, dz = oracle.gate_kl(s, gt)
+    g0, g1 = 0.2 / 0.8, 0.6 / 0.8
+    row1 = g0 * math.log(g0 / s[0, 0, 1, 0]) + g1 * math.log(g1 / s[0, 0, 1, 1])
+    assert abs(loss - row1 / 2) < 1e-15
+    assert abs(dz[0, 0, 1, 0] - (s[0, 0, 1, 0] - g0) / 2) < 1e-16
+    assert dz[0, 0, 0, 0] == 0.0 and dz[0, 0, 0, 1] == 0.0
