@@ -461,7 +461,27 @@ def main():
                 "frac_of_peak": bflops / (bms * 1e-3) / 1e12 / pk["bf16_tflops"],
                 "exp_per_s": pairs / (bms * 1e-3),
                 "status": seer.seer_workspace_status(bws)}
-        del bQd, bKd, bws, M, bl
+        # the gate's distillation step on that map: KL(gt || score) and the
+        # gradients of Wq, Wk (the map just produced serves as gt)
+        bWq, bWk = (t.to(dev) for t in synth.make_gate_weights(bw))
+        tws = torch.empty(seer.gate_kl_backward_workspace_size(bw.B, bw.Hq, bw.Hkv, bw.n, bw.d, bw.h),
+                          dtype=torch.uint8, device=dev)
+        kout = (torch.empty(1, dtype=torch.float32, device=dev), torch.empty_like(bWq), torch.empty_like(bWk))
+        for _ in range(2):
+            seer.seer_gate_kl_backward(bQd, bKd, bWq, bWk, M, workspace=tws, out=kout)
+        torch.cuda.synchronize(dev)
+        b0.record(stream)
+        for _ in range(nrep):
+            seer.seer_gate_kl_backward(bQd, bKd, bWq, bWk, M, workspace=tws, out=kout)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        kms = b0.elapsed_time(b1) / nrep
+        # algorithmic bytes: Q and K read once (pooling), gt read, the logits
+        # written and read back as dz, the small pooled/projected tensors
+        kbytes = (bQd.numel() + bKd.numel()) * 2 + 3 * M.numel() * 4
+        bmax["gate_kl_step"] = {"ms": kms, "loss": float(kout[0].item()), "gb_s": kbytes / (kms * 1e-3) / 1e9,
+                                "algorithmic_bytes": kbytes}
+        del bQd, bKd, bws, M, bl, tws, kout
 
     # ------------------------------------------------------ density sweep ----
     sweep = None

@@ -125,6 +125,37 @@ SEER_API size_t seer_gate_workspace_size(const seer_dims *dims, int32_t h);
 SEER_API int32_t seer_gate_required_cap(const seer_dims *dims, seer_select_mode mode, int32_t k,
                                float density);
 
+/* seer_gate_kl_backward -- one distillation step of the AttnGate: its loss
+ * and the gradients of the loss with respect to the gate's two linear layers
+ * (summary page, section 3.4, "Loss function: KL-divergence": loss =
+ * D_KL(gt || score); "Training data and hyperparameters": only the gate is
+ * trained).
+ *
+ * Recomputes the gate forward exactly as seer_gate does (block RoPE off),
+ * then, per causal row (b, hq, i) with g = gt row / sum_{j<=i} gt row:
+ *   loss = mean over rows of sum_{j<=i, g_j>0} g_j (log g_j - log score_ij)
+ *   dz_ij = (score_ij - g_ij) / rows          (gradient of loss wrt the logits)
+ *   dq~_i = sum_j dz_ij k~_j / sqrt(d),   dk~_j = sum_{hq of g} sum_i dz_ij q~_i / sqrt(d)
+ *   dWq[hq] = sum_{b,i} dq~_i qbar_i^T,   dWk[g] = sum_{b,j} dk~_j kbar_j^T
+ *
+ *   Q, K, dtype, Wq, Wk, h   as seer_gate
+ *   gt        [B, Hq, nb, nb] fp32: the max-pooled map (seer_attn_blockmax's
+ *             map_out); entries j > i are ignored; every row must have a
+ *             positive causal sum
+ *   loss      one fp32 on the device: the mean KL term (fixed summation
+ *             order, deterministic)
+ *   dWq       [Hq, h, d] fp32 and dWk [Hkv, h, 3d] fp32: overwritten
+ *   ws/ws_bytes  workspace of at least seer_gate_kl_backward_workspace_size(...)
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
+SEER_API seer_status seer_gate_kl_backward(const seer_dims *dims, const void *Q, const void *K,
+                                          seer_dtype dtype, const float *Wq, const float *Wk,
+                                          int32_t h, const float *gt, float *loss, float *dWq,
+                                          float *dWk, void *ws, size_t ws_bytes,
+                                          seer_stream_t stream);
+
+SEER_API size_t seer_gate_kl_backward_workspace_size(const seer_dims *dims, int32_t h);
+
 /* seer_gate_select -- the mask-generation step alone on caller-supplied fp32
  * scores [B, Hq, nb, nb] (entries j > i are ignored).  Same selection rules
  * and outputs as seer_gate; used to check index lists bit-exactly against an

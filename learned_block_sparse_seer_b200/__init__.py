@@ -5,6 +5,7 @@ thin Python binding plus the seeded synthetic-input recipe.
 """
 from ._lib import (  # noqa: F401
     SELECT_THRESHOLD, SELECT_TOPK_DENSITY, SELECT_TOPK_K, SeerError, blockmax_workspace_size,
-    gate_required_cap, gate_workspace_size, lib, seer_attn_blockmax, seer_gate, seer_gate_noalloc, seer_gate_select,
-    seer_sparse_attn, seer_workspace_status, sparse_attn_workspace_size,
+    gate_kl_backward_workspace_size, gate_required_cap, gate_workspace_size, lib, seer_attn_blockmax, seer_gate,
+    seer_gate_kl_backward, seer_gate_noalloc, seer_gate_select, seer_sparse_attn, seer_workspace_status,
+    sparse_attn_workspace_size,
 )

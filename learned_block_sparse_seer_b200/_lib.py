@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
         L.seer_gate_noalloc.restype = I32
         L.seer_gate_select.argtypes = [DP, P, I32, F, I32, F, P, P, I32, P]
         L.seer_gate_select.restype = I32
+        L.seer_gate_kl_backward.argtypes = [DP, P, P, I32, P, P, I32, P, P, P, P, P, SZ, P]
+        L.seer_gate_kl_backward.restype = I32
+        L.seer_gate_kl_backward_workspace_size.argtypes = [DP, I32]
+        L.seer_gate_kl_backward_workspace_size.restype = SZ
         L.seer_sparse_attn.argtypes = [DP, P, P, P, I32, P, P, I32, F, P, P, P, SZ, P]
         L.seer_sparse_attn.restype = I32
         L.seer_sparse_attn_workspace_size.argtypes = [DP, I32]
@@ -168,6 +172,34 @@ def seer_gate(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, retur
                          ws.numel(), _stream(dev))
     _check("seer_gate", st)
     return (counts, indices, scores) if return_scores else (counts, indices)
+
+
+def gate_kl_backward_workspace_size(B, Hq, Hkv, n, d, h) -> int:
+    return int(lib().seer_gate_kl_backward_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)), int(h)))
+
+
+def seer_gate_kl_backward(Q, K, Wq, Wk, gt, workspace=None, out=None):
+    """One AttnGate distillation step: (loss [1] fp32, dWq [Hq,h,d], dWk
+    [Hkv,h,3d]) for KL(gt || score), gt the max-pooled map [B,Hq,nb,nb]."""
+    dev = _dev(Q, K, Wq, Wk, gt)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    if Wq.dtype != torch.float32 or Wk.dtype != torch.float32 or gt.dtype != torch.float32:
+        raise TypeError("gate weights and gt must be fp32")
+    h = Wq.shape[1]
+    if out is None:
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        dWq = torch.empty_like(Wq)
+        dWk = torch.empty_like(Wk)
+    else:
+        loss, dWq, dWk = out
+    dims = _dims(B, Hq, Hkv, n, d)
+    ws = _workspace(gate_kl_backward_workspace_size(B, Hq, Hkv, n, d, h), dev, workspace)
+    st = lib().seer_gate_kl_backward(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq), _ptr(Wk),
+                                     int(h), _ptr(gt), _ptr(loss), _ptr(dWq), _ptr(dWk), _ptr(ws), ws.numel(),
+                                     _stream(dev))
+    _check("seer_gate_kl_backward", st)
+    return loss, dWq, dWk
 
 
 def seer_gate_noalloc(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0,

@@ -13,6 +13,7 @@
 #include "../../include/seer.h"
 #include "attn.cuh"
 #include "blockmax.cuh"
+#include "gate_train.cuh"
 #include "common.cuh"
 #include "gate.cuh"
 #include "ptx.cuh"
@@ -125,6 +126,26 @@ GateWs gate_ws(const seer_dims* d, int h) {
   return w;
 }
 
+// The gate's workspace, then the KL step's: per-row loss terms and the
+// gradients of q~ and k~ (dz is written over the logits).
+struct GateTrainWs {
+  GateWs gate;
+  size_t row_loss, dqt, dkt, total;
+};
+
+GateTrainWs gate_train_ws(const seer_dims* d, int h) {
+  const long long nb = d->n / seer::kBlock;
+  GateTrainWs w;
+  w.gate = gate_ws(d, h);
+  seer::WsCarver c;
+  c.off = w.gate.total;
+  w.row_loss = c.take(sizeof(float) * d->B * d->Hq * nb);
+  w.dqt = c.take(sizeof(float) * d->B * d->Hq * nb * h);
+  w.dkt = c.take(sizeof(float) * d->B * d->Hkv * nb * h);
+  w.total = c.off;
+  return w;
+}
+
 struct AttnWs {
   size_t q16, kv, redo, total;
 };
@@ -210,6 +231,93 @@ seer_status seer_workspace_status(const void* ws, seer_stream_t stream) {
 size_t seer_gate_workspace_size(const seer_dims* dims, int32_t h) {
   if (!dims_ok(dims) || h < 1) return 0;
   return gate_ws(dims, h).total;
+}
+
+size_t seer_gate_kl_backward_workspace_size(const seer_dims* dims, int32_t h) {
+  if (!dims_ok(dims) || h < 1) return 0;
+  return gate_train_ws(dims, h).total;
+}
+
+seer_status seer_gate_kl_backward(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype,
+                                  const float* Wq, const float* Wk, int32_t h, const float* gt, float* loss,
+                                  float* dWq, float* dWk, void* ws, size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !Wq || !Wk || !gt || !loss || !dWq || !dWk) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (h < 1 || h > 256 || (h % 4) != 0) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16)) return SEER_ERR_INVALID_ARG;
+  const GateTrainWs w = gate_train_ws(dims, h);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+
+  uint8_t* base = (uint8_t*)ws;
+  float* qbar = (float*)(base + w.gate.qbar);
+  float* kbar = (float*)(base + w.gate.kbar);
+  float* qt = (float*)(base + w.gate.qt);
+  float* kt = (float*)(base + w.gate.kt);
+  float* zdz = (float*)(base + w.gate.logits);
+  float* row_loss = (float*)(base + w.row_loss);
+  float* dqt = (float*)(base + w.dqt);
+  float* dkt = (float*)(base + w.dkt);
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  const int nb = n / seer::kBlock, G = Hq / Hkv;
+  const float inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  const long long rows = (long long)B * Hq * nb;
+
+  // gate forward, as in seer_gate (no RoPE): pooling, projections, logits
+  SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st));
+  SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st));
+  SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
+                                 (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
+  SEER_CUDA(seer::launch_gemm_nt(kbar, Wk, kt, nb, h, 3 * d, (long long)nb * 3 * d,
+                                 (long long)h * 3 * d, (long long)nb * h, h, B * Hkv, Hkv, 0, 1,
+                                 1.0f, false, st));
+  SEER_CUDA(seer::launch_gemm_nt(qt, kt, zdz, nb, nb, h, (long long)nb * h, (long long)nb * h,
+                                 (long long)nb * nb, nb, B * Hq, Hq, Hkv, G, inv_sqrt_d, true, st));
+  // KL per row and dz over the logits, then the loss
+  SEER_CUDA(seer::launch_kl_rows(zdz, gt, row_loss, rows, nb, st));
+  SEER_CUDA(seer::launch_loss_sum(row_loss, rows, loss, st));
+  seer::GemmBatched g{};
+  // dq~[b,hq] = dz[b,hq] k~[b,g] / sqrt(d): (i, j) x (j, c); dz is zero for j > i
+  g = seer::GemmBatched{};
+  g.A = zdz; g.B = kt; g.C = dqt;
+  g.M = nb; g.N = h; g.K = nb; g.R = 1; g.Z1 = B; g.Z2 = Hq; g.b_div = G; g.band = 1;
+  g.a_m = nb; g.a_k = 1; g.a_z1 = (long long)Hq * nb * nb; g.a_z2 = (long long)nb * nb; g.a_r = 0;
+  g.b_k = h; g.b_n = 1; g.b_z1 = (long long)Hkv * nb * h; g.b_z2 = (long long)nb * h; g.b_r = 0;
+  g.c_m = h; g.c_n = 1; g.c_z1 = (long long)Hq * nb * h; g.c_z2 = (long long)nb * h;
+  g.alpha = inv_sqrt_d;
+  SEER_CUDA(seer::launch_gemm_batched(g, st));
+  // dk~[b,g] = sum over the G query heads of dz^T q~ / sqrt(d): (j, i) x (i, c); nonzero for i >= j
+  g = seer::GemmBatched{};
+  g.A = zdz; g.B = qt; g.C = dkt;
+  g.M = nb; g.N = h; g.K = nb; g.R = G; g.Z1 = B; g.Z2 = Hkv; g.b_div = 1; g.band = 2;
+  g.a_m = 1; g.a_k = nb; g.a_z1 = (long long)Hq * nb * nb; g.a_z2 = (long long)G * nb * nb;
+  g.a_r = (long long)nb * nb;
+  g.b_k = h; g.b_n = 1; g.b_z1 = (long long)Hq * nb * h; g.b_z2 = (long long)G * nb * h; g.b_r = (long long)nb * h;
+  g.c_m = h; g.c_n = 1; g.c_z1 = (long long)Hkv * nb * h; g.c_z2 = (long long)nb * h;
+  g.alpha = inv_sqrt_d;
+  SEER_CUDA(seer::launch_gemm_batched(g, st));
+  // dWq[hq] = sum_b dq~[b,hq]^T qbar[b,hq]: (c, i) x (i, e)
+  g = seer::GemmBatched{};
+  g.A = dqt; g.B = qbar; g.C = dWq;
+  g.M = h; g.N = d; g.K = nb; g.R = B; g.Z1 = 1; g.Z2 = Hq; g.b_div = 1; g.band = 0;
+  g.a_m = 1; g.a_k = h; g.a_z1 = 0; g.a_z2 = (long long)nb * h; g.a_r = (long long)Hq * nb * h;
+  g.b_k = d; g.b_n = 1; g.b_z1 = 0; g.b_z2 = (long long)nb * d; g.b_r = (long long)Hq * nb * d;
+  g.c_m = d; g.c_n = 1; g.c_z1 = 0; g.c_z2 = (long long)h * d;
+  g.alpha = 1.0f;
+  SEER_CUDA(seer::launch_gemm_batched(g, st));
+  // dWk[g] = sum_b dk~[b,g]^T kbar[b,g]: (c, j) x (j, e)
+  g = seer::GemmBatched{};
+  g.A = dkt; g.B = kbar; g.C = dWk;
+  g.M = h; g.N = 3 * d; g.K = nb; g.R = B; g.Z1 = 1; g.Z2 = Hkv; g.b_div = 1; g.band = 0;
+  g.a_m = 1; g.a_k = h; g.a_z1 = 0; g.a_z2 = (long long)nb * h; g.a_r = (long long)Hkv * nb * h;
+  g.b_k = 3 * d; g.b_n = 1; g.b_z1 = 0; g.b_z2 = (long long)nb * 3 * d; g.b_r = (long long)Hkv * nb * 3 * d;
+  g.c_m = 3 * d; g.c_n = 1; g.c_z1 = 0; g.c_z2 = (long long)h * 3 * d;
+  g.alpha = 1.0f;
+  SEER_CUDA(seer::launch_gemm_batched(g, st));
+  return SEER_OK;
 }
 
 int32_t seer_gate_required_cap(const seer_dims* dims, seer_select_mode mode, int32_t k,
