@@ -481,6 +481,26 @@ def main():
         kbytes = (bQd.numel() + bKd.numel()) * 2 + 3 * M.numel() * 4
         bmax["gate_kl_step"] = {"ms": kms, "loss": float(kout[0].item()), "gb_s": kbytes / (kms * 1e-3) / 1e9,
                                 "algorithmic_bytes": kbytes}
+        # the training forward (O, LSE and the map) on the same layer
+        bV = synth.make_qkv(bw)[2].to(dev)
+        fws = torch.empty(seer.attn_forward_map_workspace_size(bw.B, bw.Hq, bw.Hkv, bw.n, bw.d),
+                          dtype=torch.uint8, device=dev)
+        fout = (torch.empty_like(bQd), torch.empty(bw.B, bw.Hq, bw.n, dtype=torch.float32, device=dev),
+                torch.empty(bw.B, bw.Hq, bw.nb, bw.nb, dtype=torch.float32, device=dev))
+        for _ in range(2):
+            seer.seer_attn_forward_map(bQd, bKd, bV, workspace=fws, out=fout)
+        torch.cuda.synchronize(dev)
+        b0.record(stream)
+        for _ in range(nrep):
+            seer.seer_attn_forward_map(bQd, bKd, bV, workspace=fws, out=fout)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        fms = b0.elapsed_time(b1) / nrep
+        # map: 2 d per causal pair; attention: 4 d per causal pair
+        fflops = 6.0 * bw.d * pairs
+        bmax["forward_map"] = {"ms": fms, "tflops": fflops / (fms * 1e-3) / 1e12,
+                               "flops": fflops, "status": seer.seer_workspace_status(fws)}
+        del bV, fws, fout
         del bQd, bKd, bws, M, bl, tws, kout
 
     # ------------------------------------------------------ density sweep ----

@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
         L.seer_sparse_attn_workspace_size.restype = SZ
         L.seer_attn_blockmax.argtypes = [DP, P, P, I32, F, P, P, P, SZ, P]
         L.seer_attn_blockmax.restype = I32
+        L.seer_attn_forward_map.argtypes = [DP, P, P, P, I32, F, P, P, P, P, SZ, P]
+        L.seer_attn_forward_map.restype = I32
+        L.seer_attn_forward_map_workspace_size.argtypes = [DP, I32]
+        L.seer_attn_forward_map_workspace_size.restype = SZ
         L.seer_blockmax_workspace_size.argtypes = [DP, I32]
         L.seer_blockmax_workspace_size.restype = SZ
         L.seer_workspace_status.argtypes = [P, P]
@@ -310,3 +314,29 @@ def seer_attn_blockmax(Q, K, scale=0.0, workspace=None, out=None, return_lse=Tru
 def seer_workspace_status(workspace: torch.Tensor) -> int:
     """Synchronises the current stream and returns the device status code."""
     return int(lib().seer_workspace_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def attn_forward_map_workspace_size(B, Hq, Hkv, n, d, dtype_code=SEER_BF16) -> int:
+    return int(lib().seer_attn_forward_map_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)), int(dtype_code)))
+
+
+def seer_attn_forward_map(Q, K, V, scale=0.0, workspace=None, out=None):
+    """Training forward: (O [B,Hq,n,d], lse [B,Hq,n] fp32, map [B,Hq,nb,nb]
+    fp32) -- dense causal attention and the 2D-max-pooled probability map."""
+    dev = _dev(Q, K, V)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    nb = n // 64
+    dc = _dtype_code(Q)
+    if out is None:
+        O = torch.empty_like(Q)
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=dev)
+        M = torch.empty(B, Hq, nb, nb, dtype=torch.float32, device=dev)
+    else:
+        O, lse, M = out
+    dims = _dims(B, Hq, Hkv, n, d)
+    ws = _workspace(attn_forward_map_workspace_size(B, Hq, Hkv, n, d, dc), dev, workspace)
+    st = lib().seer_attn_forward_map(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), dc, float(scale), _ptr(O),
+                                     _ptr(lse), _ptr(M), _ptr(ws), ws.numel(), _stream(dev))
+    _check("seer_attn_forward_map", st)
+    return O, lse, M

@@ -431,11 +431,15 @@ size_t seer_sparse_attn_workspace_size(const seer_dims* dims, seer_dtype dtype) 
   return attn_ws(dims, dtype).total;
 }
 
-seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V,
-                             seer_dtype dtype, const int32_t* counts, const int32_t* indices,
-                             int32_t cap, float scale, void* O, float* lse, void* ws,
-                             size_t ws_bytes, seer_stream_t stream) {
-  if (!dims_ok(dims) || !Q || !K || !V || !counts || !indices || !O) return SEER_ERR_INVALID_ARG;
+namespace {
+// The sparse attention call; `dense` runs every causal block without lists.
+seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V, seer_dtype dtype,
+                            const int32_t* counts, const int32_t* indices, int32_t cap, float scale, void* O,
+                            float* lse, void* ws, size_t ws_bytes, seer_stream_t stream, bool dense,
+                            bool keep_status = false) {
+  if (!dims_ok(dims) || !Q || !K || !V || !O) return SEER_ERR_INVALID_ARG;
+  if (!dense && (!counts || !indices)) return SEER_ERR_INVALID_ARG;
+  if (dense) cap = dims->n / seer::kBlock;
   if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
   if (cap < 1 || !(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
   seer_status s = dims_supported(dims);
@@ -444,7 +448,15 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
     return SEER_ERR_INVALID_ARG;
   const AttnWs w = attn_ws(dims, dtype);
   cudaStream_t st = (cudaStream_t)stream;
-  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (keep_status) {
+    // a call made on behalf of another in the same workspace: reset only the
+    // work counters, so that the earlier launch's device status survives
+    if (!ws || !aligned(ws, 256) || ws_bytes < w.total) return SEER_ERR_WORKSPACE;
+    SEER_CUDA(cudaMemsetAsync((uint8_t*)ws + 8, 0, sizeof(seer::WsHeader) - 8, st));
+    s = SEER_OK;
+  } else {
+    s = begin_ws(ws, ws_bytes, w.total, st);
+  }
   if (s != SEER_OK) return s;
   uint8_t* base = (uint8_t*)ws;
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
@@ -471,6 +483,7 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.total_units = (long long)B * Hq * p.nb;
   p.counts = counts;
   p.indices = indices;
+  p.dense = dense ? 1 : 0;
   p.O = O;
   p.lse = lse;
   p.out_fp32 = dtype == SEER_FP32;
@@ -484,10 +497,18 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.redo_count = &hdr->work_counter2;
   p.redo_list = reinterpret_cast<int*>(base + w.redo);
   p.redo_cap = (int)p.total_units;
-  SEER_CUDA(seer::launch_empty_rows(p, st));
+  if (!dense) SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
   SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kv, p, st));
   return SEER_OK;
+}
+}  // namespace
+
+seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V,
+                             seer_dtype dtype, const int32_t* counts, const int32_t* indices,
+                             int32_t cap, float scale, void* O, float* lse, void* ws,
+                             size_t ws_bytes, seer_stream_t stream) {
+  return run_sparse_attn(dims, Q, K, V, dtype, counts, indices, cap, scale, O, lse, ws, ws_bytes, stream, false);
 }
 
 // -------------------------------------------------------------- blockmax --
@@ -544,6 +565,25 @@ seer_status seer_attn_blockmax(const seer_dims* dims, const void* Q, const void*
   p.timeout_ns = kTimeoutNs;
   SEER_CUDA(seer::launch_blockmax(tmQ, tmK, p, w.ctas, st));
   return SEER_OK;
+}
+
+// --------------------------------------------------- training forward ----
+size_t seer_attn_forward_map_workspace_size(const seer_dims* dims, seer_dtype dtype) {
+  if (!dims_ok(dims)) return 0;
+  const size_t a = attn_ws(dims, dtype).total, m = bmax_ws(dims, dtype, num_sms()).total;
+  return a > m ? a : m;
+}
+
+seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const void* K, const void* V,
+                                  seer_dtype dtype, float scale, void* O, float* lse, float* map_out, void* ws,
+                                  size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !V || !O || !map_out) return SEER_ERR_INVALID_ARG;
+  // the max-pooled map first (its own log-sum-exp is not kept), then the
+  // attention output over every causal block on the same workspace
+  seer_status s = seer_attn_blockmax(dims, Q, K, dtype, scale, map_out, nullptr, ws, ws_bytes, stream);
+  if (s != SEER_OK) return s;
+  return run_sparse_attn(dims, Q, K, V, dtype, nullptr, nullptr, 0, scale, O, lse, ws, ws_bytes, stream, true,
+                         true);
 }
 
 }  // extern "C"

@@ -183,6 +183,10 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int w) {
   r.i = p.nb - 1 - rem / p.G;
   r.hq = r.g * p.G + rem % p.G;
   r.u = ((long long)r.b * p.Hq + r.hq) * p.nb + r.i;
+  if (p.dense) {
+    r.count = r.i + 1;
+    return r;
+  }
   int c = p.counts[r.u];
   int lim = min(p.cap, r.i + 1);
   if (c < 0 || c > lim) {
@@ -455,7 +459,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           if (u.count > 0) break;
         }
         // lists are ascending, so only the last entry can be the diagonal block
-        const int diag = w >= 0 ? (p.indices[u.u * p.cap + u.count - 1] == u.i) : 0;
+        const int diag = w >= 0 ? (p.dense ? 1 : (p.indices[u.u * p.cap + u.count - 1] == u.i)) : 0;
         C.unit[slot].w = w;
         C.unit[slot].count = u.count;
         C.unit[slot].diag = diag;
@@ -470,14 +474,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // The list entries of the next pair step are read one step early, so
         // that their global-memory latency hides behind this step's waits.
         const int* lst = p.indices + u.u * p.cap;
-        int jn0 = lst[0];
-        int jn1 = u.count > 1 ? lst[1] : 0;
+        auto entry = [&](int t) { return p.dense ? t : lst[t]; };
+        int jn0 = entry(0);
+        int jn1 = u.count > 1 ? entry(1) : 0;
         int prev = -1;
         for (int m = 0; m < u.count; m += 2, ++h) {
           const int ntile = m + 1 < u.count ? 2 : 1;
           const int ra = jn0, rb = jn1;
-          if (m + 2 < u.count) jn0 = lst[m + 2];
-          if (m + 3 < u.count) jn1 = lst[m + 3];
+          if (m + 2 < u.count) jn0 = entry(m + 2);
+          if (m + 3 < u.count) jn1 = entry(m + 3);
           int jj[2];
           jj[0] = checked_entry(p, u, ra, prev);
           prev = ra;
@@ -898,7 +903,7 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
       float m = -INFINITY, l = 0.f;
       int prev = -1;
       for (int t = 0; t < u.count; ++t) {
-        const int raw = lst[t];
+        const int raw = p.dense ? t : lst[t];
         const int j = checked_entry(p, u, raw, prev);
         prev = raw;
         const __nv_bfloat16* rec = recs + (rec0 + j) * (2LL * D * 64);

@@ -11,6 +11,7 @@ struct AttnParams {
   long long total_units;     // B * Hq * nb
   const int32_t* counts;     // [B, Hq, nb]
   const int32_t* indices;    // [B, Hq, nb, cap]
+  int dense;                 // 1: every causal block (count = i+1, entry t = t); lists not read
   void* O;                   // [B, Hq, n, d] bf16 or fp32
   float* lse;                // [B, Hq, n] or null
   int out_fp32;              // O element type
