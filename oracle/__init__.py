@@ -354,3 +354,98 @@ def gate_kl_backward(Q, K, Wq, Wk, gt):
     dWq = np.einsum("bhic,bhie->hce", dqt, qb)
     dWk = np.einsum("bgjc,bgje->gce", dkt, kb)
     return loss, dWq, dWk
+
+
+# --------------------------------------------------------- decode stage ---
+# Rebuttal, "decode-stage evaluation": the decode gate drops the Q branch's
+# pooling and projection (each token's own Q scores the blocks) and keeps a
+# small compressed K cache (pooled after RoPE) for gating; its ground truth is
+# the 1D max-pooling of the token's attention row along the sequence.
+# Readings: the compressed cache holds k~_j = Wk [max | min | avg](K block j)
+# for the complete blocks j < c, where c = (n - 1) // 64 is the block of the
+# current token (position n - 1); the current block is always attended and is
+# not a selection candidate; no further RoPE is applied (K and Q arrive
+# rotated); h = d so that q . k~ is defined; the row softmax and the selection
+# rules are the prefill ones over the c candidates.
+
+def decode_kcache(K, Wk, nblocks: int) -> np.ndarray:
+    """k~ [B, Hkv, nblocks, h] for key blocks 0 .. nblocks-1 of K."""
+    k = _f32(K)
+    kb = pool_k(k[:, :, :nblocks * BLOCK])
+    return project(kb, Wk)
+
+
+def decode_gate(q, kt, d: int) -> np.ndarray:
+    """Scores [B, Hq, c] = softmax_j(q . k~_j / sqrt(d)) over the c candidate
+    blocks (q [B, Hq, d] is the current token's query)."""
+    qv = _f64(q)
+    kv = _f64(kt)
+    B, Hq, _ = qv.shape
+    Hkv, c = kv.shape[1], kv.shape[2]
+    out = np.zeros((B, Hq, c), np.float64)
+    for b in range(B):
+        for hq in range(Hq):
+            g = hq // (Hq // Hkv)
+            z = kv[b, g] @ qv[b, hq] / math.sqrt(d)
+            e = np.exp(z - z.max())
+            out[b, hq] = e / e.sum()
+    return out
+
+
+def decode_select(scores, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0):
+    """Per (b, hq) row, the selected candidate blocks (ascending), by the
+    prefill rules applied to a row with c candidates."""
+    s = _f64(scores)
+    B, Hq, c = s.shape
+    rows = s.reshape(B * Hq, c)
+    cnt, idx = select_rows(rows, np.full(B * Hq, c - 1, dtype=np.int64), mode, T=T, k=k, density=density)
+    return cnt.reshape(B, Hq), idx.reshape(B, Hq, -1)
+
+
+def decode_attn(q, K, V, n: int, counts, idx, scale: float | None = None):
+    """O [B, Hq, d] and LSE [B, Hq] of the current token (position n - 1)
+    over the keys of its selected complete blocks and of its own block
+    c = (n - 1) // 64 (positions 64c .. n-1)."""
+    qv, kv, vv = _f64(q), _f64(K), _f64(V)
+    B, Hq, d = qv.shape
+    Hkv = kv.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    c = (n - 1) // BLOCK
+    O = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    for b in range(B):
+        for hq in range(Hq):
+            g = hq // (Hq // Hkv)
+            keys = [np.arange(j * BLOCK, (j + 1) * BLOCK) for j in idx[b, hq, :counts[b, hq]]]
+            keys.append(np.arange(c * BLOCK, n))
+            ks = np.concatenate(keys)
+            z = kv[b, g, ks] @ qv[b, hq] * scale
+            m = z.max()
+            e = np.exp(z - m)
+            O[b, hq] = e @ vv[b, g, ks] / e.sum()
+            lse[b, hq] = m + math.log(e.sum())
+    return O, lse
+
+
+def decode_blockmax(q, K, n: int, scale: float | None = None):
+    """1D ground truth: gt [B, Hq, c + 1], the maximum of the token's causal
+    attention probabilities over each key block (the last block partial),
+    and the row's LSE [B, Hq]."""
+    qv, kv = _f64(q), _f64(K)
+    B, Hq, d = qv.shape
+    Hkv = kv.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    c = (n - 1) // BLOCK
+    gt = np.zeros((B, Hq, c + 1), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    for b in range(B):
+        for hq in range(Hq):
+            g = hq // (Hq // Hkv)
+            z = kv[b, g, :n] @ qv[b, hq] * scale
+            m = z.max()
+            l = np.exp(z - m).sum()
+            p = np.exp(z - m) / l
+            for j in range(c + 1):
+                gt[b, hq, j] = p[j * BLOCK:min((j + 1) * BLOCK, n)].max()
+            lse[b, hq] = m + math.log(l)
+    return gt, lse

@@ -558,3 +558,103 @@ def test_gate_kl_two_block_closed_form():
     assert abs(loss - row1 / 2) < 1e-15
     assert abs(dz[0, 0, 1, 0] - (s[0, 0, 1, 0] - g0) / 2) < 1e-16
     assert dz[0, 0, 0, 0] == 0.0 and dz[0, 0, 0, 1] == 0.0
+
+
+# ----------------------------------------------------------- decode stage --
+def _decode_inputs(B=2, Hq=4, Hkv=2, n=5 * 64 + 17, d=32, seed=23):
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, Hq, d, generator=g)
+    K = torch.randn(B, Hkv, n, d, generator=g)
+    V = torch.randn(B, Hkv, n, d, generator=g)
+    return q, K, V
+
+
+def test_decode_attn_all_blocks_is_last_row_of_prefill_attention():
+    """Every candidate selected: the token attends to all n keys, which is the
+    prefill oracle's causal attention at query position n - 1."""
+    B, Hq, Hkv, d, nblk = 2, 4, 2, 32, 6
+    n = nblk * 64
+    q, K, V = _decode_inputs(B, Hq, Hkv, n, d, 29)
+    c = (n - 1) // 64
+    counts = np.full((B, Hq), c, np.int32)
+    idx = np.tile(np.arange(c, dtype=np.int32), (B, Hq, 1))
+    O, lse = oracle.decode_attn(q, K, V, n, counts, idx)
+    Qf = torch.zeros(B, Hq, n, d)
+    Qf[:, :, n - 1] = q
+    cl, il = oracle.dense_lists(B, Hq, nblk)
+    Of, lf = oracle.sparse_attn(Qf, K, V, cl, il)
+    np.testing.assert_allclose(O, Of[:, :, n - 1], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, lf[:, :, n - 1], rtol=1e-12, atol=1e-12)
+
+
+def test_decode_attn_subset_matches_sdpa_with_key_mask():
+    B, Hq, Hkv, d = 2, 4, 2, 32
+    n = 7 * 64 + 9
+    q, K, V = _decode_inputs(B, Hq, Hkv, n, d, 31)
+    c = (n - 1) // 64
+    rng = np.random.default_rng(1)
+    counts = np.zeros((B, Hq), np.int32)
+    idx = np.full((B, Hq, c), -1, np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            sel = np.sort(rng.choice(c, size=int(rng.integers(0, c + 1)), replace=False))
+            counts[b, h] = len(sel)
+            idx[b, h, :len(sel)] = sel
+    O, _ = oracle.decode_attn(q, K, V, n, counts, idx)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            mask = torch.zeros(n, dtype=torch.bool)
+            for j in idx[b, h, :counts[b, h]]:
+                mask[j * 64:(j + 1) * 64] = True
+            mask[c * 64:n] = True
+            ref = F.scaled_dot_product_attention(q[b, h].double().view(1, 1, 1, d),
+                                                 K[b, h // G].double().view(1, 1, n, d),
+                                                 V[b, h // G].double().view(1, 1, n, d),
+                                                 attn_mask=mask.view(1, 1, 1, n))
+            np.testing.assert_allclose(O[b, h], ref.view(d).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_decode_blockmax_is_maxpool1d_of_softmax():
+    B, Hq, Hkv, d = 2, 4, 2, 32
+    n = 4 * 64 + 33
+    q, K, _ = _decode_inputs(B, Hq, Hkv, n, d, 37)
+    gt, lse = oracle.decode_blockmax(q, K, n)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            z = (K[b, h // G].double() @ q[b, h].double()) / math.sqrt(d)
+            p = torch.softmax(z, dim=0)
+            ref = F.max_pool1d(p.view(1, 1, n), 64, ceil_mode=True).view(-1)
+            np.testing.assert_allclose(gt[b, h], ref.numpy(), rtol=1e-12, atol=1e-15)
+            assert abs(lse[b, h] - torch.logsumexp(z, 0).item()) < 1e-12
+    # the block holding the row maximum has the largest entry; every entry <= 1
+    assert np.all(gt <= 1.0) and np.all(gt.max(-1) >= 1.0 / n)
+
+
+def test_decode_gate_is_softmax_over_compressed_cache():
+    B, Hq, Hkv, d = 2, 4, 2, 32
+    n = 6 * 64 + 5
+    q, K, _ = _decode_inputs(B, Hq, Hkv, n, d, 41)
+    g = torch.Generator("cpu").manual_seed(43)
+    Wk = torch.randn(Hkv, d, 3 * d, generator=g) * 0.05
+    c = (n - 1) // 64
+    kt = oracle.decode_kcache(K, Wk, c)
+    assert kt.shape == (B, Hkv, c, d)
+    # the compressed entry of a block is Wk applied to its [max | min | avg]
+    blk = K[1, 1, 2 * 64:3 * 64].double()
+    feat = torch.cat([blk.max(0).values, blk.min(0).values, blk.mean(0)])
+    np.testing.assert_allclose(kt[1, 1, 2], (Wk[1].double() @ feat).numpy(), rtol=1e-12, atol=1e-12)
+    s = oracle.decode_gate(q, kt, d)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            ref = torch.softmax(torch.from_numpy(kt[b, h // G]) @ q[b, h].double() / math.sqrt(d), 0)
+            np.testing.assert_allclose(s[b, h], ref.numpy(), rtol=1e-12, atol=1e-15)
+    cnt, ix = oracle.decode_select(s, oracle.MODE_TOPK_DENSITY, density=0.5)
+    assert np.all(cnt == math.ceil(0.5 * c))
+    cnt, ix = oracle.decode_select(s, oracle.MODE_TOPK_K, k=2)
+    for b in range(B):
+        for h in range(Hq):
+            top = np.argsort(-s[b, h], kind="stable")[:2]
+            assert sorted(top.tolist()) == ix[b, h, :2].tolist()
