@@ -8,6 +8,8 @@
  *   seer_sparse_attn    block-sparse causal attention over the selected blocks
  *   seer_attn_blockmax  2D max-pooled attention-probability map (the gate's
  *                       self-distillation target)
+ *   seer_decode_*       the decode stage: compressed K cache, token gate,
+ *                       block-sparse decode attention, 1D ground truth
  *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
@@ -263,6 +265,98 @@ SEER_API seer_status seer_attn_forward_map(const seer_dims *dims, const void *Q,
                                           void *ws, size_t ws_bytes, seer_stream_t stream);
 
 SEER_API size_t seer_attn_forward_map_workspace_size(const seer_dims *dims, seer_dtype dtype);
+
+/* ------------------------------------------------------------------------ */
+/* Decode stage (the authors' OpenReview rebuttal, "decode-stage
+ * evaluation"): one new token per (batch, query head) attends to a KV cache.
+ * The gate keeps no Q-branch pooling or projection -- the token's own query
+ * q scores the key blocks -- and reads only a compressed K cache, one
+ * vector k~_j per complete 64-key block; attention then loads K/V only for
+ * the selected blocks.  Readings of that passage:
+ *  - the token sits at position seq_len - 1, in block c = (seq_len - 1) / 64;
+ *    the candidates are the complete blocks j < c; block c (positions
+ *    64c .. seq_len-1) is always attended and is never a candidate;
+ *  - k~_j = Wk[g] [max | min | avg](K block j) (the prefill gate's K branch,
+ *    applied to the cached keys as stored), so h = d and
+ *    score_j = softmax_{j < c}(q . k~_j / sqrt(d));
+ *  - the distillation target is the 1D max-pooling of the token's attention
+ *    probabilities over each key block.
+ * The KV cache is [B, Hkv, n, d] (dims->n = its capacity in tokens, a
+ * multiple of 64); the query is [B, Hq, d].
+ */
+
+/* seer_decode_kcache_update -- writes k~_j for key blocks
+ * block_begin .. block_end-1 of every (batch, KV head): call it once a block
+ * of the cache is complete (or once after a prefill, for all its blocks).
+ *   Kcache    [B, Hkv, n, d] bf16 or fp32 (dtype)
+ *   Wk        [Hkv, h, 3d] fp32, input features ordered [max | min | avg]
+ *   h         must equal d (the query meets k~ directly)
+ *   kt_cache  [B, Hkv, n/64, h] fp32; only the listed blocks are written
+ * An empty range does nothing.  No workspace.
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CUDA.       */
+SEER_API seer_status seer_decode_kcache_update(const seer_dims *dims, const void *Kcache, seer_dtype dtype,
+                                              const float *Wk, int32_t h, int32_t block_begin,
+                                              int32_t block_end, float *kt_cache, seer_stream_t stream);
+
+/* seer_decode_gate -- scores of the c = (seq_len-1)/64 candidate blocks and
+ * the selected ones, by the prefill rules applied to a row of c candidates
+ * (THRESHOLD: score > T; TOPK_K: min(k, c) largest; TOPK_DENSITY:
+ * clamp(ceil(density*c), 1, c) largest, the product rounded in fp32).
+ *   q         [B, Hq, d] bf16 or fp32 (dtype): the current token's query
+ *   kt_cache  [B, Hkv, n/64, d] fp32 from seer_decode_kcache_update, valid
+ *             for blocks 0 .. c-1
+ *   seq_len   tokens in the cache including the current one, 1 .. n
+ *   scores_out  optional [B, Hq, c] fp32 (NULL to skip)
+ *   counts    [B, Hq] int32;  indices [B, Hq, cap] int32 ascending, entries
+ *             past counts[row] untouched; c == 0 gives counts 0
+ *   cap       >= seer_decode_gate_required_cap(...)
+ *   ws/ws_bytes  workspace of at least seer_decode_gate_workspace_size(...)
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_CAPACITY,
+ *         SEER_ERR_WORKSPACE, SEER_ERR_CUDA.                               */
+SEER_API seer_status seer_decode_gate(const seer_dims *dims, const void *q, seer_dtype dtype,
+                                     const float *kt_cache, int32_t seq_len, seer_select_mode mode, float T,
+                                     int32_t k, float density, float *scores_out, int32_t *counts,
+                                     int32_t *indices, int32_t cap, void *ws, size_t ws_bytes,
+                                     seer_stream_t stream);
+
+SEER_API size_t seer_decode_gate_workspace_size(const seer_dims *dims);
+
+/* Smallest `cap` for seer_decode_gate at this seq_len (0 when c == 0);
+ * -1 on invalid arguments. */
+SEER_API int32_t seer_decode_gate_required_cap(const seer_dims *dims, int32_t seq_len, seer_select_mode mode,
+                                              int32_t k, float density);
+
+/* seer_sparse_decode_attn -- the token's attention over the keys of its
+ * selected blocks and of its own block c (positions 64c .. seq_len-1):
+ *   O   = sum_s softmax_s(scale * q . k_s) v_s,  lse = ln sum_s exp(...)
+ * Split over the list (split-KV) with a log-sum-exp merge.
+ *   q [B,Hq,d], Kcache/Vcache [B,Hkv,n,d]: bf16 or fp32 (dtype)
+ *   counts [B,Hq], indices [B,Hq,cap]: lists as seer_decode_gate writes them
+ *             (every entry < c); a count outside 0..min(cap, c) or an entry
+ *             outside 0..c-1 is clamped and recorded as SEER_ERR_DEVICE_CHECK
+ *   scale     0 means 1/sqrt(d)
+ *   O [B,Hq,d] (dtype), lse [B,Hq] fp32 (may be NULL)
+ *   ws/ws_bytes  workspace of at least seer_sparse_decode_attn_workspace_size
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
+SEER_API seer_status seer_sparse_decode_attn(const seer_dims *dims, const void *q, const void *Kcache,
+                                            const void *Vcache, seer_dtype dtype, int32_t seq_len,
+                                            const int32_t *counts, const int32_t *indices, int32_t cap,
+                                            float scale, void *O, float *lse, void *ws, size_t ws_bytes,
+                                            seer_stream_t stream);
+
+SEER_API size_t seer_sparse_decode_attn_workspace_size(const seer_dims *dims);
+
+/* seer_decode_blockmax -- the decode gate's distillation target: over the
+ * token's full causal attention row (positions 0 .. seq_len-1),
+ *   gt[j] = max over the keys of block j of softmax(scale * q . K^T)
+ * for j = 0 .. c (block c partial), and the row's lse.
+ *   gt_out [B, Hq, c+1] fp32;  lse_out [B, Hq] fp32 (may be NULL)
+ * No workspace.  Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED,
+ * SEER_ERR_CUDA.                                                           */
+SEER_API seer_status seer_decode_blockmax(const seer_dims *dims, const void *q, const void *Kcache,
+                                         seer_dtype dtype, int32_t seq_len, float scale, float *gt_out,
+                                         float *lse_out, seer_stream_t stream);
 
 /* Synchronises `stream`, reads the device status word at the start of a
  * workspace that a previous call used, and maps it: SEER_OK,

@@ -79,6 +79,20 @@ def lib() -> ctypes.CDLL:
         L.seer_attn_forward_map_workspace_size.restype = SZ
         L.seer_blockmax_workspace_size.argtypes = [DP, I32]
         L.seer_blockmax_workspace_size.restype = SZ
+        L.seer_decode_kcache_update.argtypes = [DP, P, I32, P, I32, I32, I32, P, P]
+        L.seer_decode_kcache_update.restype = I32
+        L.seer_decode_gate.argtypes = [DP, P, I32, P, I32, I32, F, I32, F, P, P, P, I32, P, SZ, P]
+        L.seer_decode_gate.restype = I32
+        L.seer_decode_gate_workspace_size.argtypes = [DP]
+        L.seer_decode_gate_workspace_size.restype = SZ
+        L.seer_decode_gate_required_cap.argtypes = [DP, I32, I32, I32, F]
+        L.seer_decode_gate_required_cap.restype = I32
+        L.seer_sparse_decode_attn.argtypes = [DP, P, P, P, I32, I32, P, P, I32, F, P, P, P, SZ, P]
+        L.seer_sparse_decode_attn.restype = I32
+        L.seer_sparse_decode_attn_workspace_size.argtypes = [DP]
+        L.seer_sparse_decode_attn_workspace_size.restype = SZ
+        L.seer_decode_blockmax.argtypes = [DP, P, P, I32, I32, F, P, P, P]
+        L.seer_decode_blockmax.restype = I32
         L.seer_workspace_status.argtypes = [P, P]
         L.seer_workspace_status.restype = I32
         L.seer_status_string.argtypes = [I32]
@@ -340,3 +354,108 @@ def seer_attn_forward_map(Q, K, V, scale=0.0, workspace=None, out=None):
                                      _ptr(lse), _ptr(M), _ptr(ws), ws.numel(), _stream(dev))
     _check("seer_attn_forward_map", st)
     return O, lse, M
+
+
+# ------------------------------------------------------------------ decode --
+# The KV cache is [B, Hkv, n, d] with n its capacity in tokens; the current
+# token (query q [B, Hq, d]) sits at position seq_len - 1, in block
+# c = (seq_len - 1) // 64.  Candidates are the complete blocks j < c.
+def _cache_dims(q, Kc):
+    B, Hq, d = q.shape
+    _, Hkv, n, dk = Kc.shape
+    if dk != d:
+        raise ValueError("q and the cache disagree on d")
+    return _dims(B, Hq, Hkv, n, d)
+
+
+def seer_decode_kcache_update(Kc, Wk, block_begin, block_end, kt_cache=None):
+    """k~ of key blocks [block_begin, block_end) of the cache into kt_cache
+    [B, Hkv, n/64, d] fp32 (allocated when None); returns kt_cache."""
+    dev = _dev(Kc, Wk)
+    B, Hkv, n, d = Kc.shape
+    if Wk.dtype != torch.float32:
+        raise TypeError("gate weights must be fp32")
+    h = Wk.shape[1]
+    if kt_cache is None:
+        kt_cache = torch.zeros(B, Hkv, n // 64, h, dtype=torch.float32, device=dev)
+    dims = _dims(B, Hkv, Hkv, n, d)
+    st = lib().seer_decode_kcache_update(ctypes.byref(dims), _ptr(Kc), _dtype_code(Kc), _ptr(Wk), int(h),
+                                         int(block_begin), int(block_end), _ptr(kt_cache), _stream(dev))
+    _check("seer_decode_kcache_update", st)
+    return kt_cache
+
+
+def decode_gate_required_cap(B, Hq, Hkv, n, d, seq_len, mode, k=0, density=0.0) -> int:
+    return int(lib().seer_decode_gate_required_cap(ctypes.byref(_dims(B, Hq, Hkv, n, d)), int(seq_len),
+                                                   mode_code(mode), int(k), float(density)))
+
+
+def decode_gate_workspace_size(B, Hq, Hkv, n, d) -> int:
+    return int(lib().seer_decode_gate_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d))))
+
+
+def seer_decode_gate(q, kt_cache, n, seq_len, mode, T=0.0, k=0, density=0.0, return_scores=False, cap=None,
+                     workspace=None, out=None):
+    """Decode-stage gate: (counts [B,Hq], indices [B,Hq,cap][, scores
+    [B,Hq,c]]) for the token at seq_len - 1 of a cache of n tokens."""
+    dev = _dev(q, kt_cache)
+    B, Hq, d = q.shape
+    Hkv = kt_cache.shape[1]
+    dims = _dims(B, Hq, Hkv, n, d)
+    mc = mode_code(mode)
+    c = (int(seq_len) - 1) // 64
+    if cap is None:
+        cap = max(1, lib().seer_decode_gate_required_cap(ctypes.byref(dims), int(seq_len), mc, int(k),
+                                                         float(density)))
+    if out is None:
+        counts = torch.empty(B, Hq, dtype=torch.int32, device=dev)
+        indices = torch.empty(B, Hq, cap, dtype=torch.int32, device=dev)
+        scores = torch.empty(B, Hq, c, dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        counts, indices, scores = out
+    ws = _workspace(decode_gate_workspace_size(B, Hq, Hkv, n, d), dev, workspace)
+    st = lib().seer_decode_gate(ctypes.byref(dims), _ptr(q), _dtype_code(q), _ptr(kt_cache), int(seq_len), mc,
+                                float(T), int(k), float(density), _ptr(scores), _ptr(counts), _ptr(indices),
+                                int(cap), _ptr(ws), ws.numel(), _stream(dev))
+    _check("seer_decode_gate", st)
+    return (counts, indices, scores) if return_scores else (counts, indices)
+
+
+def sparse_decode_attn_workspace_size(B, Hq, Hkv, n, d) -> int:
+    return int(lib().seer_sparse_decode_attn_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d))))
+
+
+def seer_sparse_decode_attn(q, Kc, Vc, seq_len, counts, indices, scale=0.0, workspace=None, out=None):
+    """Block-sparse decode attention: (O [B,Hq,d], lse [B,Hq] fp32)."""
+    dev = _dev(q, Kc, Vc, counts, indices)
+    dims = _cache_dims(q, Kc)
+    B, Hq, d = q.shape
+    if out is None:
+        O = torch.empty_like(q)
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    else:
+        O, lse = out
+    ws = _workspace(sparse_decode_attn_workspace_size(B, Hq, Kc.shape[1], Kc.shape[2], d), dev, workspace)
+    st = lib().seer_sparse_decode_attn(ctypes.byref(dims), _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q),
+                                       int(seq_len), _ptr(counts), _ptr(indices), int(indices.shape[-1]),
+                                       float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev))
+    _check("seer_sparse_decode_attn", st)
+    return O, lse
+
+
+def seer_decode_blockmax(q, Kc, seq_len, scale=0.0, out=None):
+    """1D ground truth of the token's attention row: (gt [B,Hq,c+1], lse
+    [B,Hq]) fp32."""
+    dev = _dev(q, Kc)
+    dims = _cache_dims(q, Kc)
+    B, Hq, d = q.shape
+    c = (int(seq_len) - 1) // 64
+    if out is None:
+        gt = torch.empty(B, Hq, c + 1, dtype=torch.float32, device=dev)
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    else:
+        gt, lse = out
+    st = lib().seer_decode_blockmax(ctypes.byref(dims), _ptr(q), _ptr(Kc), _dtype_code(q), int(seq_len),
+                                    float(scale), _ptr(gt), _ptr(lse), _stream(dev))
+    _check("seer_decode_blockmax", st)
+    return gt, lse

@@ -14,6 +14,7 @@
 #include "attn.cuh"
 #include "blockmax.cuh"
 #include "gate_train.cuh"
+#include "decode.cuh"
 #include "common.cuh"
 #include "gate.cuh"
 #include "ptx.cuh"
@@ -564,6 +565,147 @@ seer_status seer_attn_blockmax(const seer_dims* dims, const void* Q, const void*
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
   SEER_CUDA(seer::launch_blockmax(tmQ, tmK, p, w.ctas, st));
+  return SEER_OK;
+}
+
+// ---------------------------------------------------------- decode stage --
+namespace {
+int decode_splits(long long rows) {
+  long long s = (4LL * 148 + rows - 1) / rows;
+  return (int)(s < 1 ? 1 : (s > 32 ? 32 : s));
+}
+// Largest list a decode row can need: c candidates, the prefill rules.
+int decode_required_cap(seer_select_mode mode, int32_t k, float density, int c) {
+  if (c <= 0) return 0;
+  if (mode == SEER_SELECT_TOPK_K) return k < c ? k : c;
+  if (mode == SEER_SELECT_TOPK_DENSITY) {
+    int kk = (int)std::ceil((double)(density * (float)c));
+    return kk < 1 ? 1 : (kk > c ? c : kk);
+  }
+  return c;
+}
+bool decode_len_ok(const seer_dims* d, int32_t seq_len) { return seq_len >= 1 && seq_len <= d->n; }
+}  // namespace
+
+size_t seer_decode_gate_workspace_size(const seer_dims* dims) {
+  if (!dims_ok(dims)) return 0;
+  seer::WsCarver c;
+  c.take(sizeof(float) * (size_t)dims->B * dims->Hq * (dims->n / seer::kBlock));
+  return c.off;
+}
+
+size_t seer_sparse_decode_attn_workspace_size(const seer_dims* dims) {
+  if (!dims_ok(dims)) return 0;
+  const long long rows = (long long)dims->B * dims->Hq;
+  seer::WsCarver c;
+  c.take(sizeof(float) * (size_t)rows * decode_splits(rows) * (dims->d + 2));
+  return c.off;
+}
+
+seer_status seer_decode_kcache_update(const seer_dims* dims, const void* Kcache, seer_dtype dtype, const float* Wk,
+                                      int32_t h, int32_t block_begin, int32_t block_end, float* kt_cache,
+                                      seer_stream_t stream) {
+  if (!dims_ok(dims) || !Kcache || !Wk || !kt_cache) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (h != dims->d) return SEER_ERR_INVALID_ARG;  // the token's q meets k~ directly
+  const int nb = dims->n / seer::kBlock;
+  if (block_begin < 0 || block_end < block_begin || block_end > nb) return SEER_ERR_INVALID_ARG;
+  if (block_end == block_begin) return SEER_OK;
+  SEER_CUDA(seer::launch_kcache(Kcache, dtype == SEER_FP32, Wk, kt_cache, (long long)dims->B * dims->Hkv, dims->Hkv,
+                                dims->n, dims->d, h, block_begin, block_end - block_begin, (cudaStream_t)stream));
+  return SEER_OK;
+}
+
+int32_t seer_decode_gate_required_cap(const seer_dims* dims, int32_t seq_len, seer_select_mode mode, int32_t k,
+                                      float density) {
+  if (!dims_ok(dims) || !decode_len_ok(dims, seq_len)) return -1;
+  return decode_required_cap(mode, k, density, (seq_len - 1) / seer::kBlock);
+}
+
+seer_status seer_decode_gate(const seer_dims* dims, const void* q, seer_dtype dtype, const float* kt_cache,
+                             int32_t seq_len, seer_select_mode mode, float T, int32_t k, float density,
+                             float* scores_out, int32_t* counts, int32_t* indices, int32_t cap, void* ws,
+                             size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !q || !kt_cache || !counts || !indices) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  if (mode == SEER_SELECT_THRESHOLD && !(T > 0.f)) return SEER_ERR_INVALID_ARG;
+  if (mode == SEER_SELECT_TOPK_K && k < 1) return SEER_ERR_INVALID_ARG;
+  if (mode == SEER_SELECT_TOPK_DENSITY && !(density > 0.f && density <= 1.f)) return SEER_ERR_INVALID_ARG;
+  if (mode != SEER_SELECT_THRESHOLD && mode != SEER_SELECT_TOPK_K && mode != SEER_SELECT_TOPK_DENSITY)
+    return SEER_ERR_INVALID_ARG;
+  const int c = (seq_len - 1) / seer::kBlock;
+  if (cap < decode_required_cap(mode, k, density, c) || cap < 1) return SEER_ERR_CAPACITY;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, seer_decode_gate_workspace_size(dims), st);
+  if (s != SEER_OK) return s;
+  const long long rows = (long long)dims->B * dims->Hq;
+  if (c == 0) {  // no complete block yet: nothing to select
+    SEER_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * rows, st));
+    return SEER_OK;
+  }
+  float* logits = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
+  SEER_CUDA(seer::launch_decode_logits(q, dtype == SEER_FP32, kt_cache, logits, rows, dims->Hq, dims->Hkv, dims->d,
+                                       c, dims->n / seer::kBlock, (float)(1.0 / std::sqrt((double)dims->d)), st));
+  SEER_CUDA(seer::launch_row_select(logits, scores_out, true, rows, c, (int)mode, T, k, density, counts, indices, cap,
+                                    st, c));
+  return SEER_OK;
+}
+
+seer_status seer_sparse_decode_attn(const seer_dims* dims, const void* q, const void* Kcache, const void* Vcache,
+                                    seer_dtype dtype, int32_t seq_len, const int32_t* counts, const int32_t* indices,
+                                    int32_t cap, float scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                                    seer_stream_t stream) {
+  if (!dims_ok(dims) || !q || !Kcache || !Vcache || !counts || !indices || !O) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (cap < 1 || !(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, seer_sparse_decode_attn_workspace_size(dims), st);
+  if (s != SEER_OK) return s;
+  seer::DecodeAttnArgs a{};
+  a.q = q;
+  a.K = Kcache;
+  a.V = Vcache;
+  a.fp32 = dtype == SEER_FP32;
+  a.counts = counts;
+  a.indices = indices;
+  a.cap = cap;
+  a.Hq = dims->Hq;
+  a.Hkv = dims->Hkv;
+  a.d = dims->d;
+  a.n_cap = dims->n;
+  a.seq_len = seq_len;
+  a.rows = (long long)dims->B * dims->Hq;
+  a.splits = decode_splits(a.rows);
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)dims->d);
+  a.scale_log2 = (float)(sc * 1.4426950408889634);
+  a.part = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
+  a.O = O;
+  a.lse = lse;
+  a.status = &((seer::WsHeader*)ws)->status;
+  SEER_CUDA(seer::launch_decode_attn(a, st));
+  return SEER_OK;
+}
+
+seer_status seer_decode_blockmax(const seer_dims* dims, const void* q, const void* Kcache, seer_dtype dtype,
+                                 int32_t seq_len, float scale, float* gt_out, float* lse_out, seer_stream_t stream) {
+  if (!dims_ok(dims) || !q || !Kcache || !gt_out) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)dims->d);
+  SEER_CUDA(seer::launch_decode_gt(q, Kcache, dtype == SEER_FP32, (long long)dims->B * dims->Hq, dims->Hq, dims->Hkv,
+                                   dims->d, dims->n, seq_len, (float)(sc * 1.4426950408889634), gt_out, lse_out,
+                                   (cudaStream_t)stream));
   return SEER_OK;
 }
 

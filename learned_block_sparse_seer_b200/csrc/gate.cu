@@ -263,7 +263,7 @@ __device__ __forceinline__ int topk_count(int i, int mode, int k, float density)
 template <bool FROM_LOGITS>
 __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
     const float* in, float* scores, int nb, int mode, float T, int k,
-    float density, int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap) {
+    float density, int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len) {
   extern __shared__ float sv[];  // [nb]
   __shared__ int sh_i[32];
   __shared__ float sh_f[32];
@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
   __shared__ uint32_t sel_prefix, sel_remaining;
 
   const long long row = blockIdx.x;
-  const int i = (int)(row % nb);
+  // causal prefill rows: query block i = row % nb; row_len > 0: every row
+  // has row_len candidates (the decode gate)
+  const int i = row_len > 0 ? row_len - 1 : (int)(row % nb);
   const int len = i + 1;
   const int tid = threadIdx.x;
   const float* src = in + row * (long long)nb;
@@ -447,20 +449,20 @@ cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cu
 
 cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, long long rows,
                               int nb, int mode, float T, int k, float density, int32_t* counts,
-                              int32_t* indices, int cap, cudaStream_t st) {
+                              int32_t* indices, int cap, cudaStream_t st, int row_len) {
   const size_t smem = (size_t)nb * sizeof(float);
   if (from_logits) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(row_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
     row_select_kernel<true><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, scores, nb, mode, T, k, density, counts, indices, cap);
+        in, scores, nb, mode, T, k, density, counts, indices, cap, row_len);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(row_select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
     row_select_kernel<false><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, nullptr, nb, mode, T, k, density, counts, indices, cap);
+        in, nullptr, nb, mode, T, k, density, counts, indices, cap, row_len);
   }
   return cudaGetLastError();
 }

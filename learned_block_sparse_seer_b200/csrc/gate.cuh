@@ -23,6 +23,6 @@ cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cu
 // Causal softmax of logit rows (from_logits) and/or index-list selection.
 cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, long long rows,
                               int nb, int mode, float T, int k, float density, int32_t* counts,
-                              int32_t* indices, int cap, cudaStream_t st);
+                              int32_t* indices, int cap, cudaStream_t st, int row_len = 0);
 
 }  // namespace seer

@@ -32,6 +32,14 @@ Recipe (all draws from ``torch.Generator('cpu').manual_seed(seed)``, fp32):
     values (upcast exactly to fp32).
   * Gate weights Wq [Hq, h, d] and Wk [Hkv, h, 3d] ~ N(0, 0.02), fp32, from a
     second generator seeded with seed + 100.
+  * ``decode`` structure (one new token per (batch, query head) against a KV
+    cache of capacity n holding seq_len tokens; make_decode): K, V ~ N(0, 1)
+    [B, Hkv, n, d] and q ~ N(0, 1) [B, Hq, d], drawn in that order; per KV
+    head g the layer's sink (K block 0 += 3u, q += 0.5u) and vertical stripes
+    (ceil(0.05 nb) random blocks += 3 w_g, q += 0.5 w_g), and for the token's
+    local window the key blocks c-3 .. c (c = (seq_len-1) // 64) get
+    += 2 e_g with q += 2 e_g; cache rows at positions >= seq_len are set to
+    NaN, so any read past the token shows up in the result.
 """
 from __future__ import annotations
 
@@ -74,7 +82,13 @@ WORKLOADS = {
     "layer128k": Workload("layer128k", 1, 32, 8, 131072, 128, 128, "bf16", "layer", 3),
     "bmax4k": Workload("bmax4k", 4, 32, 8, 4096, 128, 128, "bf16", "layer", 4),
     "bmax32k": Workload("bmax32k", 1, 32, 8, 32768, 128, 128, "bf16", "layer", 5),
+    # decode: the layer's heads against a 128k-token KV cache
+    "decode128k": Workload("decode128k", 1, 32, 8, 131072, 128, 128, "bf16", "decode", 6),
 }
+
+# Tokens in the decode cache by default: 37 short of capacity, so the token's
+# own block is partial.
+DECODE_TAIL = 37
 
 
 def custom(name: str, B: int, Hq: int, Hkv: int, n: int, d: int, h: int,
@@ -154,3 +168,40 @@ def make_scores_like(w: Workload, seed: int = 11, ties: bool = False):
     x = x * tri
     x = x / x.sum(-1, keepdim=True)
     return x.to(torch.float32).contiguous()
+
+
+def decode_seq_len(w: Workload) -> int:
+    return w.n - DECODE_TAIL
+
+
+def make_decode(w: Workload, seq_len: int | None = None):
+    """Return (q [B, Hq, d], Kc, Vc [B, Hkv, n, d]) CPU tensors of w.dtype for
+    a token at position seq_len - 1 (default n - 37)."""
+    seq_len = decode_seq_len(w) if seq_len is None else seq_len
+    assert 1 <= seq_len <= w.n
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    K = torch.randn(w.B, w.Hkv, w.n, w.d, generator=g)
+    V = torch.randn(w.B, w.Hkv, w.n, w.d, generator=g)
+    q = torch.randn(w.B, w.Hq, w.d, generator=g)
+    nb, G = w.nb, w.G
+    c = (seq_len - 1) // BLOCK
+    Kb = K.view(w.B, w.Hkv, nb, BLOCK, w.d)
+    u = _unit(g, w.d)
+    n_stripes = math.ceil(0.05 * nb)
+    for kv in range(w.Hkv):
+        heads = slice(kv * G, (kv + 1) * G)
+        Kb[:, kv, 0] += 3.0 * u
+        q[:, heads] += 0.5 * u
+        wv = _unit(g, w.d)
+        if nb > 1:
+            stripes = torch.randperm(nb - 1, generator=g)[:n_stripes] + 1
+            Kb[:, kv, stripes] += 3.0 * wv
+        q[:, heads] += 0.5 * wv
+        e = _unit(g, w.d)
+        Kb[:, kv, max(0, c - 3):c + 1] += 2.0 * e
+        q[:, heads] += 2.0 * e
+    K[:, :, seq_len:] = float("nan")
+    V[:, :, seq_len:] = float("nan")
+    if w.dtype == "bf16":
+        q, K, V = (t.to(torch.bfloat16) for t in (q, K, V))
+    return q.contiguous(), K.contiguous(), V.contiguous()
