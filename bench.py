@@ -37,6 +37,7 @@ METRIC = ("sparse prefill attn ms & active-block TFLOP/s (% BF16 peak) at 128k, 
 WORKLOAD = "layer128k"
 DENSITY = 0.1
 BMAX_WORKLOAD = "bmax32k"
+DECODE_WORKLOAD = "decode128k"
 
 
 def parse():
@@ -48,6 +49,7 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--density", type=float, default=DENSITY)
     ap.add_argument("--no-blockmax", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time the 50-95%% sparsity sweep")
@@ -311,6 +313,97 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def decode_bench(seer, synth, dev, stream, density, pk):
+    """The decode stage on a 128k-token cache: the compressed K cache built
+    once for every complete block, then per token the gate (top-k density)
+    and the block-sparse attention, and the 1D ground truth.  The L2 is
+    flushed (a 256 MB write) before every timed launch, so each reads HBM."""
+    import torch
+    w = synth.WORKLOADS[DECODE_WORKLOAD]
+    seq_len = synth.decode_seq_len(w)
+    c = (seq_len - 1) // 64
+    q, Kc, Vc = synth.make_decode(w, seq_len)
+    _, Wk = synth.make_gate_weights(w)
+    qd, Kd, Vd, Wkd = (t.to(dev) for t in (q, Kc, Vc, Wk))
+    del q, Kc, Vc
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    kt = torch.zeros(w.B, w.Hkv, w.nb, w.d, dtype=torch.float32, device=dev)
+    cap = max(1, seer.decode_gate_required_cap(w.B, w.Hq, w.Hkv, w.n, w.d, seq_len, "density", density=density))
+    counts = torch.empty(w.B, w.Hq, dtype=torch.int32, device=dev)
+    idx = torch.empty(w.B, w.Hq, cap, dtype=torch.int32, device=dev)
+    gws = torch.empty(seer.decode_gate_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device=dev)
+    aws = torch.empty(seer.sparse_decode_attn_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8,
+                      device=dev)
+    O = torch.empty_like(qd)
+    lse = torch.empty(w.B, w.Hq, dtype=torch.float32, device=dev)
+    gt = torch.empty(w.B, w.Hq, c + 1, dtype=torch.float32, device=dev)
+    glse = torch.empty(w.B, w.Hq, dtype=torch.float32, device=dev)
+
+    def timed(fn, reps=10, warm=3):
+        for _ in range(warm):
+            fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            tot += a.elapsed_time(b)
+        return tot / reps
+
+    kc_ms = timed(lambda: seer.seer_decode_kcache_update(Kd, Wkd, 0, c, kt))
+    gate_ms = timed(lambda: seer.seer_decode_gate(qd, kt, w.n, seq_len, "density", density=density, cap=cap,
+                                                  workspace=gws, out=(counts, idx, None)))
+    attn_ms = timed(lambda: seer.seer_sparse_decode_attn(qd, Kd, Vd, seq_len, counts, idx, workspace=aws,
+                                                         out=(O, lse)))
+    step_ms = timed(lambda: (seer.seer_decode_gate(qd, kt, w.n, seq_len, "density", density=density, cap=cap,
+                                                   workspace=gws, out=(counts, idx, None)),
+                             seer.seer_sparse_decode_attn(qd, Kd, Vd, seq_len, counts, idx, workspace=aws,
+                                                          out=(O, lse))))
+    gt_ms = timed(lambda: seer.seer_decode_blockmax(qd, Kd, seq_len, out=(gt, glse)))
+    # algorithmic bytes: each distinct (b, g, block) that some query head of
+    # the group selects, plus the token's own block, read once for K and V
+    cn = counts.cpu().numpy()
+    ix = idx.cpu().numpy()
+    G = w.G
+    uniq = 0
+    per_row = 0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            sel = set()
+            for hq in range(g * G, (g + 1) * G):
+                sel.update(int(j) for j in ix[b, hq, :cn[b, hq]])
+                per_row += int(cn[b, hq])
+            uniq += len(sel)
+    tail = seq_len - 64 * c
+    kv_row = 64 * w.d * 2 * 2
+    attn_bytes = (uniq * kv_row + w.B * w.Hkv * tail * w.d * 2 * 2 + qd.numel() * 2 * 2 + counts.numel() * 4
+                  + cn.sum() * 4)
+    gate_bytes = w.B * w.Hkv * c * w.d * 4 + qd.numel() * 2 + counts.numel() * 4 + cn.sum() * 4
+    kc_bytes = w.B * w.Hkv * c * 64 * w.d * 2 + w.B * w.Hkv * c * w.d * 4
+    gt_bytes = w.B * w.Hkv * seq_len * w.d * 2 + w.B * w.Hq * (c + 1) * 4
+    hbm = pk["hbm_gbs"]
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms * 1e-3) / 1e9
+
+    return {"workload": f"{DECODE_WORKLOAD}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} cache n={w.n} d={w.d} "
+                        f"seq_len={seq_len}, top-k density {density}",
+            "l2": "flushed (256 MB write) before every timed launch",
+            "candidates": c, "selected_per_row": float(cn.mean()), "distinct_blocks_per_kv_head":
+                uniq / (w.B * w.Hkv),
+            "kcache_build": {"ms": kc_ms, "gb_s": gbs(kc_bytes, kc_ms), "frac_hbm": gbs(kc_bytes, kc_ms) / hbm},
+            "gate": {"us": gate_ms * 1e3, "gb_s": gbs(gate_bytes, gate_ms)},
+            "attn": {"us": attn_ms * 1e3, "gb_s": gbs(attn_bytes, attn_ms),
+                     "frac_hbm": gbs(attn_bytes, attn_ms) / hbm, "algorithmic_bytes": int(attn_bytes),
+                     "status": seer.seer_workspace_status(aws)},
+            "token_step_us": step_ms * 1e3,
+            "ground_truth": {"us": gt_ms * 1e3, "gb_s": gbs(gt_bytes, gt_ms), "frac_hbm": gbs(gt_bytes, gt_ms) / hbm},
+            "hbm_peak_gbs": hbm}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -503,6 +596,11 @@ def main():
         del bV, fws, fout
         del bQd, bKd, bws, M, bl, tws, kout
 
+    # ----------------------------------------------------------- decode path --
+    dec = None
+    if not args.no_decode and rank == 0:
+        dec = decode_bench(seer, synth, dev, stream, args.density, pk)
+
     # ------------------------------------------------------ density sweep ----
     sweep = None
     if args.sweep and rank == 0:
@@ -576,7 +674,7 @@ def main():
                          "algorithmic_flops_per_launch": flops},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 7 * args.steps,
-            "blockmax": bmax, "sweep": sweep,
+            "blockmax": bmax, "decode": dec, "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -282,7 +282,8 @@ SEER_API size_t seer_attn_forward_map_workspace_size(const seer_dims *dims, seer
  *  - the distillation target is the 1D max-pooling of the token's attention
  *    probabilities over each key block.
  * The KV cache is [B, Hkv, n, d] (dims->n = its capacity in tokens, a
- * multiple of 64); the query is [B, Hq, d].
+ * multiple of 64); the query is [B, Hq, d].  Cache pointers (K, V, the
+ * compressed cache) must be 16-byte aligned.
  */
 
 /* seer_decode_kcache_update -- writes k~_j for key blocks
@@ -350,13 +351,17 @@ SEER_API size_t seer_sparse_decode_attn_workspace_size(const seer_dims *dims);
 /* seer_decode_blockmax -- the decode gate's distillation target: over the
  * token's full causal attention row (positions 0 .. seq_len-1),
  *   gt[j] = max over the keys of block j of softmax(scale * q . K^T)
- * for j = 0 .. c (block c partial), and the row's lse.
+ * for j = 0 .. c (block c partial), and the row's lse.  The query heads of a
+ * KV head are scored together, so the K cache is read once per KV head.
  *   gt_out [B, Hq, c+1] fp32;  lse_out [B, Hq] fp32 (may be NULL)
- * No workspace.  Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED,
- * SEER_ERR_CUDA.                                                           */
+ *   ws/ws_bytes  workspace of at least seer_decode_blockmax_workspace_size
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
 SEER_API seer_status seer_decode_blockmax(const seer_dims *dims, const void *q, const void *Kcache,
                                          seer_dtype dtype, int32_t seq_len, float scale, float *gt_out,
-                                         float *lse_out, seer_stream_t stream);
+                                         float *lse_out, void *ws, size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_decode_blockmax_workspace_size(const seer_dims *dims);
 
 /* Synchronises `stream`, reads the device status word at the start of a
  * workspace that a previous call used, and maps it: SEER_OK,

@@ -8,6 +8,7 @@ from ._lib import (  # noqa: F401
     blockmax_workspace_size, seer_attn_forward_map,
     gate_kl_backward_workspace_size, gate_required_cap, gate_workspace_size, lib, seer_attn_blockmax, seer_gate,
     seer_gate_kl_backward, seer_gate_noalloc, seer_gate_select, seer_sparse_attn, seer_workspace_status,
-    sparse_attn_workspace_size, decode_gate_required_cap, decode_gate_workspace_size, seer_decode_blockmax,
+    sparse_attn_workspace_size, decode_blockmax_workspace_size, decode_gate_required_cap,
+    decode_gate_workspace_size, seer_decode_blockmax,
     seer_decode_gate, seer_decode_kcache_update, seer_sparse_decode_attn, sparse_decode_attn_workspace_size,
 )

@@ -91,7 +91,9 @@ def lib() -> ctypes.CDLL:
         L.seer_sparse_decode_attn.restype = I32
         L.seer_sparse_decode_attn_workspace_size.argtypes = [DP]
         L.seer_sparse_decode_attn_workspace_size.restype = SZ
-        L.seer_decode_blockmax.argtypes = [DP, P, P, I32, I32, F, P, P, P]
+        L.seer_decode_blockmax.argtypes = [DP, P, P, I32, I32, F, P, P, P, SZ, P]
+        L.seer_decode_blockmax_workspace_size.argtypes = [DP]
+        L.seer_decode_blockmax_workspace_size.restype = SZ
         L.seer_decode_blockmax.restype = I32
         L.seer_workspace_status.argtypes = [P, P]
         L.seer_workspace_status.restype = I32
@@ -443,7 +445,11 @@ def seer_sparse_decode_attn(q, Kc, Vc, seq_len, counts, indices, scale=0.0, work
     return O, lse
 
 
-def seer_decode_blockmax(q, Kc, seq_len, scale=0.0, out=None):
+def decode_blockmax_workspace_size(B, Hq, Hkv, n, d) -> int:
+    return int(lib().seer_decode_blockmax_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d))))
+
+
+def seer_decode_blockmax(q, Kc, seq_len, scale=0.0, workspace=None, out=None):
     """1D ground truth of the token's attention row: (gt [B,Hq,c+1], lse
     [B,Hq]) fp32."""
     dev = _dev(q, Kc)
@@ -455,7 +461,8 @@ def seer_decode_blockmax(q, Kc, seq_len, scale=0.0, out=None):
         lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
     else:
         gt, lse = out
+    ws = _workspace(decode_blockmax_workspace_size(B, Hq, Kc.shape[1], Kc.shape[2], d), dev, workspace)
     st = lib().seer_decode_blockmax(ctypes.byref(dims), _ptr(q), _ptr(Kc), _dtype_code(q), int(seq_len),
-                                    float(scale), _ptr(gt), _ptr(lse), _stream(dev))
+                                    float(scale), _ptr(gt), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev))
     _check("seer_decode_blockmax", st)
     return gt, lse

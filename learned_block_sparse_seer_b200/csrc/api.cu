@@ -570,10 +570,6 @@ seer_status seer_attn_blockmax(const seer_dims* dims, const void* Q, const void*
 
 // ---------------------------------------------------------- decode stage --
 namespace {
-int decode_splits(long long rows) {
-  long long s = (4LL * 148 + rows - 1) / rows;
-  return (int)(s < 1 ? 1 : (s > 32 ? 32 : s));
-}
 // Largest list a decode row can need: c candidates, the prefill rules.
 int decode_required_cap(seer_select_mode mode, int32_t k, float density, int c) {
   if (c <= 0) return 0;
@@ -585,6 +581,34 @@ int decode_required_cap(seer_select_mode mode, int32_t k, float density, int c) 
   return c;
 }
 bool decode_len_ok(const seer_dims* d, int32_t seq_len) { return seq_len >= 1 && seq_len <= d->n; }
+
+struct DecAttnWs {
+  size_t ticket, part, total;
+  int splits;
+};
+DecAttnWs dec_attn_ws(const seer_dims* d) {
+  const long long rows = (long long)d->B * d->Hq;
+  DecAttnWs w;
+  w.splits = seer::decode_attn_splits(rows);
+  seer::WsCarver c;
+  w.ticket = c.take(sizeof(int32_t) * (size_t)rows);
+  w.part = c.take(sizeof(float) * (size_t)rows * w.splits * (d->d + 2));
+  w.total = c.off;
+  return w;
+}
+
+struct DecGtWs {
+  size_t ticket, stats, total;
+};
+DecGtWs dec_gt_ws(const seer_dims* d) {
+  const long long rows = (long long)d->B * d->Hq;
+  DecGtWs w;
+  seer::WsCarver c;
+  w.ticket = c.take(sizeof(int32_t) * (size_t)rows);
+  w.stats = c.take(sizeof(float) * 2 * (size_t)rows * seer::kGtMaxChunks);
+  w.total = c.off;
+  return w;
+}
 }  // namespace
 
 size_t seer_decode_gate_workspace_size(const seer_dims* dims) {
@@ -596,10 +620,12 @@ size_t seer_decode_gate_workspace_size(const seer_dims* dims) {
 
 size_t seer_sparse_decode_attn_workspace_size(const seer_dims* dims) {
   if (!dims_ok(dims)) return 0;
-  const long long rows = (long long)dims->B * dims->Hq;
-  seer::WsCarver c;
-  c.take(sizeof(float) * (size_t)rows * decode_splits(rows) * (dims->d + 2));
-  return c.off;
+  return dec_attn_ws(dims).total;
+}
+
+size_t seer_decode_blockmax_workspace_size(const seer_dims* dims) {
+  if (!dims_ok(dims)) return 0;
+  return dec_gt_ws(dims).total;
 }
 
 seer_status seer_decode_kcache_update(const seer_dims* dims, const void* Kcache, seer_dtype dtype, const float* Wk,
@@ -610,11 +636,12 @@ seer_status seer_decode_kcache_update(const seer_dims* dims, const void* Kcache,
   seer_status s = dims_supported(dims);
   if (s != SEER_OK) return s;
   if (h != dims->d) return SEER_ERR_INVALID_ARG;  // the token's q meets k~ directly
+  if (!aligned(Kcache, 16) || !aligned(kt_cache, 16)) return SEER_ERR_INVALID_ARG;
   const int nb = dims->n / seer::kBlock;
   if (block_begin < 0 || block_end < block_begin || block_end > nb) return SEER_ERR_INVALID_ARG;
   if (block_end == block_begin) return SEER_OK;
   SEER_CUDA(seer::launch_kcache(Kcache, dtype == SEER_FP32, Wk, kt_cache, (long long)dims->B * dims->Hkv, dims->Hkv,
-                                dims->n, dims->d, h, block_begin, block_end - block_begin, (cudaStream_t)stream));
+                                dims->n, dims->d, block_begin, block_end - block_begin, (cudaStream_t)stream));
   return SEER_OK;
 }
 
@@ -632,7 +659,7 @@ seer_status seer_decode_gate(const seer_dims* dims, const void* q, seer_dtype dt
   if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
   seer_status s = dims_supported(dims);
   if (s != SEER_OK) return s;
-  if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  if (!decode_len_ok(dims, seq_len) || !aligned(kt_cache, 16)) return SEER_ERR_INVALID_ARG;
   if (mode == SEER_SELECT_THRESHOLD && !(T > 0.f)) return SEER_ERR_INVALID_ARG;
   if (mode == SEER_SELECT_TOPK_K && k < 1) return SEER_ERR_INVALID_ARG;
   if (mode == SEER_SELECT_TOPK_DENSITY && !(density > 0.f && density <= 1.f)) return SEER_ERR_INVALID_ARG;
@@ -649,8 +676,9 @@ seer_status seer_decode_gate(const seer_dims* dims, const void* q, seer_dtype dt
     return SEER_OK;
   }
   float* logits = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
-  SEER_CUDA(seer::launch_decode_logits(q, dtype == SEER_FP32, kt_cache, logits, rows, dims->Hq, dims->Hkv, dims->d,
-                                       c, dims->n / seer::kBlock, (float)(1.0 / std::sqrt((double)dims->d)), st));
+  SEER_CUDA(seer::launch_decode_logits(q, dtype == SEER_FP32, kt_cache, logits, dims->B, dims->Hq, dims->Hkv,
+                                       dims->d, c, dims->n / seer::kBlock, (float)(1.0 / std::sqrt((double)dims->d)),
+                                       st));
   SEER_CUDA(seer::launch_row_select(logits, scores_out, true, rows, c, (int)mode, T, k, density, counts, indices, cap,
                                     st, c));
   return SEER_OK;
@@ -666,9 +694,13 @@ seer_status seer_sparse_decode_attn(const seer_dims* dims, const void* q, const 
   seer_status s = dims_supported(dims);
   if (s != SEER_OK) return s;
   if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  if (!aligned(Kcache, 16) || !aligned(Vcache, 16)) return SEER_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  s = begin_ws(ws, ws_bytes, seer_sparse_decode_attn_workspace_size(dims), st);
+  const DecAttnWs w = dec_attn_ws(dims);
+  s = begin_ws(ws, ws_bytes, w.total, st);
   if (s != SEER_OK) return s;
+  const long long rows = (long long)dims->B * dims->Hq;
+  SEER_CUDA(cudaMemsetAsync((uint8_t*)ws + w.ticket, 0, sizeof(int32_t) * rows, st));
   seer::DecodeAttnArgs a{};
   a.q = q;
   a.K = Kcache;
@@ -682,11 +714,12 @@ seer_status seer_sparse_decode_attn(const seer_dims* dims, const void* q, const 
   a.d = dims->d;
   a.n_cap = dims->n;
   a.seq_len = seq_len;
-  a.rows = (long long)dims->B * dims->Hq;
-  a.splits = decode_splits(a.rows);
+  a.rows = rows;
+  a.splits = w.splits;
   const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)dims->d);
   a.scale_log2 = (float)(sc * 1.4426950408889634);
-  a.part = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
+  a.part = (float*)((uint8_t*)ws + w.part);
+  a.ticket = (int32_t*)((uint8_t*)ws + w.ticket);
   a.O = O;
   a.lse = lse;
   a.status = &((seer::WsHeader*)ws)->status;
@@ -695,17 +728,23 @@ seer_status seer_sparse_decode_attn(const seer_dims* dims, const void* q, const 
 }
 
 seer_status seer_decode_blockmax(const seer_dims* dims, const void* q, const void* Kcache, seer_dtype dtype,
-                                 int32_t seq_len, float scale, float* gt_out, float* lse_out, seer_stream_t stream) {
+                                 int32_t seq_len, float scale, float* gt_out, float* lse_out, void* ws,
+                                 size_t ws_bytes, seer_stream_t stream) {
   if (!dims_ok(dims) || !q || !Kcache || !gt_out) return SEER_ERR_INVALID_ARG;
   if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
   if (!(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
   seer_status s = dims_supported(dims);
   if (s != SEER_OK) return s;
-  if (!decode_len_ok(dims, seq_len)) return SEER_ERR_INVALID_ARG;
+  if (!decode_len_ok(dims, seq_len) || !aligned(Kcache, 16)) return SEER_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const DecGtWs w = dec_gt_ws(dims);
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+  SEER_CUDA(cudaMemsetAsync((uint8_t*)ws + w.ticket, 0, sizeof(int32_t) * (size_t)dims->B * dims->Hq, st));
   const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)dims->d);
-  SEER_CUDA(seer::launch_decode_gt(q, Kcache, dtype == SEER_FP32, (long long)dims->B * dims->Hq, dims->Hq, dims->Hkv,
-                                   dims->d, dims->n, seq_len, (float)(sc * 1.4426950408889634), gt_out, lse_out,
-                                   (cudaStream_t)stream));
+  SEER_CUDA(seer::launch_decode_gt(q, Kcache, dtype == SEER_FP32, dims->B, dims->Hq, dims->Hkv, dims->d, dims->n,
+                                   seq_len, (float)(sc * 1.4426950408889634), gt_out, lse_out,
+                                   (float*)((uint8_t*)ws + w.stats), (int32_t*)((uint8_t*)ws + w.ticket), st));
   return SEER_OK;
 }
 

@@ -10,19 +10,33 @@
 // c = (seq_len - 1) / 64 is the current token's block; that block is always
 // attended and is not a candidate; no further RoPE; h = d.
 //
-// Kernels (memory-bound: one query row per (batch, head)):
-//   kcache_kernel       one CTA per (batch, KV head, new block): pooling over
-//                       the block's 64 keys, then k~ = Wk[g] kbar
-//   decode_logits_kernel  one CTA per (batch, query head): q . k~_j / sqrt(d)
-//                       for the c candidates (a warp per block); the softmax
-//                       and selection then reuse the prefill row kernel
-//   decode_attn_kernel  split-KV online softmax: CTA (row, split) walks every
-//                       split-th entry of the row's list (selected blocks, then
-//                       the current block); partial (m, l, o) per split
-//   decode_combine_kernel  merges the splits by log-sum-exp into O and LSE
-//   decode_gt_kernel    the 1D ground truth: a warp per key block keeps the
-//                       block's raw maximum and an online (m, l); the row's
-//                       LSE then turns the maxima into probabilities
+// Everything here is bound by HBM (one query row per (batch, head), so no
+// contraction is large enough for the tensor cores).  The common pattern is
+// the "slab": a warp reads 8 x 512 contiguous bytes with one 16-byte load per
+// lane per row chunk (lane l takes chunk l % LPR of row i * RPI + l / LPR in
+// load i), multiplies its chunk by the matching chunk of the query in
+// registers, and a butterfly reduce-scatter over the LPR lanes of a row
+// leaves every lane with the full dot product of one row (7 shuffles for 8
+// rows instead of 8 full reductions).
+//
+// Kernels:
+//   kcache_kernel       CTA per (batch, KV head, 16 blocks): pooling by slabs,
+//                       then the projection k~ = Wk[g] kbar as a shared-memory
+//                       tiled product (Wk read once per 16 blocks)
+//   decode_logits_kernel  CTA per (batch, KV head, head group, row chunk):
+//                       q . k~_j / sqrt(d) for GT query heads of the group at
+//                       once (k~ read once for them); the softmax and the
+//                       selection then reuse the prefill row kernel
+//   decode_attn_kernel  split-KV: CTA (row, split) takes a contiguous range of
+//                       the row's list (selected blocks, then the current
+//                       block); each warp runs its own online softmax over
+//                       16..64-row slabs with K and V loads issued together;
+//                       the last CTA of a row (atomic ticket) merges the splits
+//                       by log-sum-exp into O and LSE
+//   decode_gt_kernel    CTA per (batch, KV head, head group, chunk of key
+//                       blocks): scores of GT query heads per K read, each
+//                       block's raw maximum and the chunk's (m, l); the last
+//                       CTA of the group turns the maxima into probabilities
 #include <cmath>
 #include <cstdint>
 
@@ -32,279 +46,713 @@
 
 namespace seer {
 
-namespace {
+namespace dec {
+
+// 16-byte chunk conversions.
 template <typename T>
-__device__ __forceinline__ float ld(const T* p, long long i) {
-  if constexpr (sizeof(T) == 2)
-    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
-  else
-    return reinterpret_cast<const float*>(p)[i];
+struct Chunk;
+template <>
+struct Chunk<uint16_t> {  // bf16
+  static constexpr int N = 8;
+  __device__ static __forceinline__ void cvt(const uint4& u, float (&x)[8]) {
+    x[0] = __uint_as_float(u.x << 16);
+    x[1] = __uint_as_float(u.x & 0xffff0000u);
+    x[2] = __uint_as_float(u.y << 16);
+    x[3] = __uint_as_float(u.y & 0xffff0000u);
+    x[4] = __uint_as_float(u.z << 16);
+    x[5] = __uint_as_float(u.z & 0xffff0000u);
+    x[6] = __uint_as_float(u.w << 16);
+    x[7] = __uint_as_float(u.w & 0xffff0000u);
+  }
+};
+template <>
+struct Chunk<float> {
+  static constexpr int N = 4;
+  __device__ static __forceinline__ void cvt(const uint4& u, float (&x)[4]) {
+    x[0] = __uint_as_float(u.x);
+    x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z);
+    x[3] = __uint_as_float(u.w);
+  }
+};
+
+template <typename T, int D>
+struct Slab {
+  static constexpr int EPC = Chunk<T>::N;   // elements per 16-byte chunk
+  static constexpr int LPR = D / EPC;       // lanes (chunks) per row
+  static constexpr int RPI = 32 / LPR;      // rows per load instruction
+  static constexpr int ROWS = 8 * RPI;      // rows per slab
+  static_assert(LPR >= 8 && LPR <= 32, "a row must be 8..32 chunks");
+  // lane's row within the slab for load i, and its chunk
+  __device__ static __forceinline__ int row(int i, int lane) { return i * RPI + lane / LPR; }
+  __device__ static __forceinline__ int chunk(int lane) { return lane % LPR; }
+};
+
+// Streaming 16-byte read-only load (no L1 allocation).
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
 }
-}  // namespace
+
+template <typename T>
+__device__ __forceinline__ float ld1(const T* p, long long i) {
+  if constexpr (sizeof(T) == 2)
+    return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(p)[i] << 16);
+  else
+    return p[i];
+}
+
+// Butterfly reduce-scatter of 8 load-rows x GT heads over the LPR lanes that
+// hold a row's chunks.  On return v[0][h] is the full dot product, for head
+// h, of the lane's row; the function returns that row's load index (the row
+// is Slab::row(index, lane)).
+template <int LPR, int GT>
+__device__ __forceinline__ int reduce_rows(float (&v)[8][GT], int lane) {
+  constexpr int O1 = LPR / 2, O2 = LPR / 4, O3 = LPR / 8;
+  const bool a = lane & O1, b = lane & O2, c = lane & O3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+      const float send = a ? v[i][h] : v[i + 4][h];
+      const float keep = a ? v[i + 4][h] : v[i][h];
+      v[i][h] = keep + __shfl_xor_sync(0xffffffffu, send, O1);
+    }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+      const float send = b ? v[i][h] : v[i + 2][h];
+      const float keep = b ? v[i + 2][h] : v[i][h];
+      v[i][h] = keep + __shfl_xor_sync(0xffffffffu, send, O2);
+    }
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    const float send = c ? v[0][h] : v[1][h];
+    const float keep = c ? v[1][h] : v[0][h];
+    v[0][h] = keep + __shfl_xor_sync(0xffffffffu, send, O3);
+  }
+#pragma unroll
+  for (int o = O3 / 2; o > 0; o >>= 1)
+#pragma unroll
+    for (int h = 0; h < GT; ++h) v[0][h] += __shfl_xor_sync(0xffffffffu, v[0][h], o);
+  return 4 * (int)a + 2 * (int)b + (int)c;
+}
+
+// The lane of this lane's row group that holds load-row i after reduce_rows.
+template <int LPR>
+__device__ __forceinline__ int holder(int i, int lane) {
+  return (lane & ~(LPR - 1)) | (((i >> 2) & 1) * (LPR / 2)) | (((i >> 1) & 1) * (LPR / 4)) | ((i & 1) * (LPR / 8));
+}
+
+// True on exactly one lane of each row's LPR lanes after reduce_rows.
+template <int LPR>
+__device__ __forceinline__ bool row_owner(int lane) {
+  return (lane & (LPR / 8 - 1)) == 0;
+}
+
+}  // namespace dec
 
 // ---------------------------------------------------- compressed K cache --
-template <typename T>
-__global__ void __launch_bounds__(128) kcache_kernel(const T* __restrict__ K, const float* __restrict__ Wk,
-                                                     float* __restrict__ kt, int Hkv, int n_cap, int d, int h,
-                                                     int j0, int nnew) {
-  extern __shared__ float kb[];  // [3d]: max | min | avg
-  const long long bhj = blockIdx.x;
-  const int t = (int)(bhj % nnew);
-  const long long bh = bhj / nnew;
+namespace {
+constexpr int kKcBlocks = 16;  // key blocks per CTA
+constexpr int kKcThreads = 256;
+}  // namespace
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict__ K, const float* __restrict__ Wk,
+                                                            float* __restrict__ kt, int Hkv, int n_cap, int j0,
+                                                            int nnew) {
+  using S = dec::Slab<T, D>;
+  constexpr int E = S::EPC;
+  constexpr int NG = kKcThreads / D;       // output groups
+  constexpr int BPG = kKcBlocks / NG;      // blocks per output group
+  extern __shared__ float sm[];
+  float* kbar = sm;                        // [kKcBlocks][3D]
+  float* wt = sm + kKcBlocks * 3 * D;      // [D][33]
+  const int nch = (nnew + kKcBlocks - 1) / kKcBlocks;
+  const long long bh = blockIdx.x / nch;
+  const int ch = (int)(blockIdx.x % nch);
   const int g = (int)(bh % Hkv);
-  const int j = j0 + t;
+  const int jb = j0 + ch * kKcBlocks;
+  const int nblk = min(kKcBlocks, j0 + nnew - jb);
   const int nb_cap = n_cap / kBlock;
-  const long long row0 = (bh * n_cap + (long long)j * kBlock) * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float mx = -INFINITY, mn = INFINITY, s = 0.f;
-    for (int r = 0; r < kBlock; ++r) {
-      const float v = ld(K, row0 + (long long)r * d + c);
-      mx = fmaxf(mx, v);
-      mn = fminf(mn, v);
-      s += v;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- pooling: warp w takes blocks w, w + 8
+  for (int t = warp; t < nblk; t += kKcThreads / 32) {
+    const T* base = K + (bh * n_cap + (long long)(jb + t) * kBlock) * D + S::chunk(lane) * E;
+    float mx[E], mn[E], su[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      mx[e] = -INFINITY;
+      mn[e] = INFINITY;
+      su[e] = 0.f;
     }
-    kb[c] = mx;
-    kb[d + c] = mn;
-    kb[2 * d + c] = s * (1.0f / kBlock);
+#pragma unroll
+    for (int s = 0; s < kBlock / S::ROWS; ++s) {
+      uint4 u[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[i] = dec::ldg16(base + (long long)(s * S::ROWS + S::row(i, lane)) * D);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x[E];
+        dec::Chunk<T>::cvt(u[i], x);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          mx[e] = fmaxf(mx[e], x[e]);
+          mn[e] = fminf(mn[e], x[e]);
+          su[e] += x[e];
+        }
+      }
+    }
+#pragma unroll
+    for (int o = S::LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
+        mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], o));
+        su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
+      }
+    if (lane < S::LPR) {
+      float* kb = kbar + t * 3 * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        kb[e] = mx[e];
+        kb[D + e] = mn[e];
+        kb[2 * D + e] = su[e] * (1.0f / kBlock);
+      }
+    }
   }
-  __syncthreads();
-  for (int o = threadIdx.x; o < h; o += blockDim.x) {
-    const float* w = Wk + ((long long)g * h + o) * 3 * d;
-    float acc = 0.f;
-    for (int e = 0; e < 3 * d; ++e) acc = fmaf(w[e], kb[e], acc);
-    kt[(bh * nb_cap + j) * h + o] = acc;
+
+  // ---- projection: thread (o, group) accumulates BPG blocks
+  const int o = threadIdx.x % D, grp = threadIdx.x / D;
+  float acc[BPG];
+#pragma unroll
+  for (int b = 0; b < BPG; ++b) acc[b] = 0.f;
+  const float* W = Wk + (long long)g * D * 3 * D;
+  for (int e0 = 0; e0 < 3 * D; e0 += 32) {
+    __syncthreads();  // kbar complete / previous tile consumed
+    for (int x = threadIdx.x; x < D * 32; x += kKcThreads) {
+      const int r = x >> 5, cc = x & 31;
+      wt[r * 33 + cc] = W[(long long)r * 3 * D + e0 + cc];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int ee = 0; ee < 32; ++ee) {
+      const float w = wt[o * 33 + ee];
+#pragma unroll
+      for (int b = 0; b < BPG; ++b) acc[b] = fmaf(w, kbar[(grp * BPG + b) * 3 * D + e0 + ee], acc[b]);
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < BPG; ++b) {
+    const int t = grp * BPG + b;
+    if (t < nblk) kt[(bh * nb_cap + jb + t) * D + o] = acc[b];
   }
 }
 
 // ------------------------------------------------------------ gate logits --
-template <typename T>
-__global__ void __launch_bounds__(256) decode_logits_kernel(const T* __restrict__ q, const float* __restrict__ kt,
-                                                            float* __restrict__ logits, int Hq, int Hkv, int d,
-                                                            int nc, int nb_cap, float scale) {
-  __shared__ float qs[256];
-  const long long row = blockIdx.x;  // b * Hq + hq
-  const long long b = row / Hq;
-  const int hq = (int)(row % Hq), g = hq / (Hq / Hkv);
-  for (int c = threadIdx.x; c < d; c += blockDim.x) qs[c] = ld(q, row * d + c);
-  __syncthreads();
-  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const float* kg = kt + (b * Hkv + g) * (long long)nb_cap * d;
-  for (int j = warp; j < nc; j += blockDim.x / 32) {
-    float acc = 0.f;
-    for (int c = lane; c < d; c += 32) acc = fmaf(qs[c], kg[(long long)j * d + c], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) logits[row * nc + j] = acc * scale;
+template <typename T, int D, int GT>
+__global__ void __launch_bounds__(128) decode_logits_kernel(const T* __restrict__ q, const float* __restrict__ kt,
+                                                            float* __restrict__ logits, int Hq, int Hkv, int nc,
+                                                            int nb_cap, int rows_per_cta, int nch, float scale) {
+  using S = dec::Slab<float, D>;
+  constexpr int E = S::EPC;
+  const int G = Hq / Hkv, nhg = G / GT;
+  const int ch = (int)(blockIdx.x % nch);
+  const long long grp = blockIdx.x / nch;  // (b * Hkv + g) * nhg + hg
+  const int hg = (int)(grp % nhg);
+  const long long bg = grp / nhg;
+  const long long b = bg / Hkv;
+  const int g = (int)(bg % Hkv);
+  const long long row0 = b * Hq + (long long)g * G + hg * GT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float qv[GT][E];
+#pragma unroll
+  for (int h = 0; h < GT; ++h)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[h][e] = dec::ld1(q, (row0 + h) * D + S::chunk(lane) * E + e) * scale;
+  const float* kg = kt + bg * (long long)nb_cap * D + S::chunk(lane) * E;
+  const int r_begin = ch * rows_per_cta, r_end = min(nc, r_begin + rows_per_cta);
+  for (int r0 = r_begin + warp * S::ROWS; r0 < r_end; r0 += 4 * S::ROWS) {
+    uint4 u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + S::row(i, lane);
+      u[i] = r < r_end ? dec::ldg16(kg + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float v[8][GT];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x[E];
+      dec::Chunk<float>::cvt(u[i], x);
+#pragma unroll
+      for (int h = 0; h < GT; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[h][e], a);
+        v[i][h] = a;
+      }
+    }
+    const int ii = dec::reduce_rows<S::LPR, GT>(v, lane);
+    const int r = r0 + S::row(ii, lane);
+    if (dec::row_owner<S::LPR>(lane) && r < r_end) {
+#pragma unroll
+      for (int h = 0; h < GT; ++h) logits[(row0 + h) * nc + r] = v[0][h];
+    }
   }
 }
 
 // ------------------------------------------------------ decode attention --
-// 128 threads: for scores two threads per key (each half of d), for PV one
-// thread per head dimension.  part: [rows, splits, d + 2] = (o[d], m, l), m
-// in the log2 domain.
-template <typename T>
-__global__ void __launch_bounds__(128) decode_attn_kernel(const T* __restrict__ q, const T* __restrict__ K,
-                                                          const T* __restrict__ V, const int32_t* __restrict__ counts,
-                                                          const int32_t* __restrict__ indices, int cap, int Hq,
-                                                          int Hkv, int d, int n_cap, int seq_len, float scale_log2,
-                                                          int splits, float* __restrict__ part,
-                                                          uint32_t* __restrict__ status) {
-  __shared__ float qs[128];
-  __shared__ float ps[64];
-  __shared__ float sh_l;
-  const long long row = blockIdx.x;
-  const int split = blockIdx.y;
-  const long long b = row / Hq;
-  const int hq = (int)(row % Hq), g = hq / (Hq / Hkv);
-  const int tid = threadIdx.x;
-  const int c = (seq_len - 1) / kBlock;
-  int cnt = counts[row];
-  const int lim = min(cap, c);
+struct DecAttnP {
+  const void* q;
+  const void* K;
+  const void* V;
+  const int32_t* counts;
+  const int32_t* indices;
+  int cap, Hq, Hkv, n_cap, seq_len, splits;
+  float scale_log2;
+  float* part;
+  int32_t* ticket;
+  void* O;
+  float* lse;
+  uint32_t* status;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128, 4) decode_attn_kernel(const DecAttnP p) {
+  using S = dec::Slab<T, D>;
+  constexpr int E = S::EPC;
+  constexpr int LPR = S::LPR;
+  constexpr int SPB = kBlock / S::ROWS;  // slabs per key block
+  const long long row = blockIdx.x / p.splits;
+  const int split = (int)(blockIdx.x % p.splits);
+  const long long b = row / p.Hq;
+  const int hq = (int)(row % p.Hq), g = hq / (p.Hq / p.Hkv);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = (p.seq_len - 1) / kBlock;
+  int cnt = p.counts[row];
+  const int lim = min(p.cap, c);
   if (cnt < 0 || cnt > lim) {
-    if (tid == 0 && split == 0) record_status(status, kDevBadIndex, (uint32_t)row);
+    if (tid == 0 && split == 0) record_status(p.status, kDevBadIndex, (uint32_t)row);
     cnt = cnt < 0 ? 0 : lim;
   }
-  for (int e = tid; e < d; e += blockDim.x) qs[e] = ld(q, row * d + e) * scale_log2;
-  const long long head0 = (b * Hkv + g) * (long long)n_cap * d;
-  float m = -INFINITY, l = 0.f, o = 0.f;
-  const int key = tid >> 1, hp = tid & 1, half = d / 2;
-  __syncthreads();
-  for (int e = split; e <= cnt; e += splits) {
-    int j = c, nkeys = seq_len - c * kBlock;
-    if (e < cnt) {
-      j = indices[row * cap + e];
+  // this CTA's range of the row's entries (the selected blocks, then block c)
+  const int total = cnt + 1;
+  const int per = (total + p.splits - 1) / p.splits;
+  const int e0 = split * per, e1 = min(total, e0 + per);
+  const T* q = reinterpret_cast<const T*>(p.q);
+  float qv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) qv[e] = dec::ld1(q, row * D + S::chunk(lane) * E + e) * p.scale_log2;
+  const long long head0 = (b * p.Hkv + g) * (long long)p.n_cap * D + S::chunk(lane) * E;
+  const T* Kh = reinterpret_cast<const T*>(p.K) + head0;
+  const T* Vh = reinterpret_cast<const T*>(p.V) + head0;
+  float m = -INFINITY, l = 0.f, o[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o[e] = 0.f;
+  const int nslabs = e1 > e0 ? (e1 - e0) * SPB : 0;
+  for (int s = warp; s < nslabs; s += 4) {
+    const int ent = e0 + s / SPB;
+    const int rbase = (s % SPB) * S::ROWS;
+    int j = c, nk = p.seq_len - c * kBlock;
+    if (ent < cnt) {
+      j = p.indices[row * p.cap + ent];
       if (j < 0 || j >= c) {
-        if (tid == 0) record_status(status, kDevBadIndex, (uint32_t)row);
+        if (lane == 0) record_status(p.status, kDevBadIndex, (uint32_t)row);
         j = j < 0 ? 0 : c - 1;
       }
-      nkeys = kBlock;
+      nk = kBlock;
     }
-    const long long kbase = head0 + (long long)j * kBlock * d;
-    float acc = 0.f;
-    if (key < nkeys) {
-      const long long r = kbase + (long long)key * d + hp * half;
-      for (int x = 0; x < half; ++x) acc = fmaf(qs[hp * half + x], ld(K, r + x), acc);
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);  // the key's two halves
-    if (hp == 0) ps[key] = key < nkeys ? acc : -INFINITY;
-    __syncthreads();
-    float bm = fmaxf(ps[tid & 31], ps[32 + (tid & 31)]);
-    bm = warp_max(bm);
-    const float mn = fmaxf(m, bm);
-    const float alpha = exp2f(m - mn);
-    __syncthreads();
-    if (tid < kBlock) ps[tid] = exp2f(ps[tid] - mn);  // -inf for absent keys -> 0
-    __syncthreads();
-    if (tid < 32) {
-      const float s = warp_sum(ps[tid] + ps[tid + 32]);
-      if (tid == 0) sh_l = s;
-    }
-    if (tid < d) {
-      float acc = 0.f;
-      for (int k = 0; k < nkeys; ++k) acc = fmaf(ps[k], ld(V, kbase + (long long)k * d + tid), acc);
-      o = o * alpha + acc;
-    }
-    __syncthreads();
-    l = l * alpha + sh_l;
-    m = mn;
-    __syncthreads();
-  }
-  float* pp = part + (row * splits + split) * (long long)(d + 2);
-  if (tid < d) pp[tid] = o;
-  if (tid == 0) {
-    pp[d] = m;
-    pp[d + 1] = l;
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part, int splits, int d,
-                                                             T* __restrict__ O, float* __restrict__ lse) {
-  const long long row = blockIdx.x;
-  const float* pr = part + row * splits * (long long)(d + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, pr[s * (d + 2) + d]);
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = pr[s * (d + 2) + d];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - M);
-    L += pr[s * (d + 2) + d + 1] * w;
-    if ((int)threadIdx.x < d) acc += pr[s * (d + 2) + threadIdx.x] * w;
-  }
-  if ((int)threadIdx.x < d) {
-    const float v = acc / L;
-    if constexpr (sizeof(T) == 2)
-      reinterpret_cast<__nv_bfloat16*>(O)[row * d + threadIdx.x] = __float2bfloat16_rn(v);
-    else
-      reinterpret_cast<float*>(O)[row * d + threadIdx.x] = v;
-  }
-  if (threadIdx.x == 0 && lse) lse[row] = (M + log2f(L)) * 0.6931471805599453f;
-}
-
-// ------------------------------------------------------ 1D ground truth ---
-template <typename T>
-__global__ void __launch_bounds__(256) decode_gt_kernel(const T* __restrict__ q, const T* __restrict__ K, int Hq,
-                                                        int Hkv, int d, int n_cap, int seq_len, float scale_log2,
-                                                        float* __restrict__ gt, float* __restrict__ lse) {
-  __shared__ float qs[256];
-  __shared__ float wm[8], wl[8];
-  __shared__ float sh_lse;
-  const long long row = blockIdx.x;
-  const long long b = row / Hq;
-  const int hq = (int)(row % Hq), g = hq / (Hq / Hkv);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int nbc = (seq_len - 1) / kBlock + 1;  // blocks 0 .. c
-  for (int e = threadIdx.x; e < d; e += blockDim.x) qs[e] = ld(q, row * d + e) * scale_log2;
-  __syncthreads();
-  const long long head0 = (b * Hkv + g) * (long long)n_cap * d;
-  float m = -INFINITY, l = 0.f;
-  for (int j = warp; j < nbc; j += 8) {
-    float s2[2];
+    if (rbase >= nk) continue;  // past the token (warp-uniform)
+    const long long off = ((long long)j * kBlock + rbase) * D;
+    uint4 ku[8], vu[8];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int key = j * kBlock + 2 * lane + u;
-      float acc = -INFINITY;
-      if (key < seq_len) {
-        acc = 0.f;
-        const long long r = head0 + (long long)key * d;
-        for (int x = 0; x < d; ++x) acc = fmaf(qs[x], ld(K, r + x), acc);
-      }
-      s2[u] = acc;
+    for (int i = 0; i < 8; ++i) {
+      const int r = S::row(i, lane);
+      const bool ok = rbase + r < nk;
+      ku[i] = ok ? dec::ldg16(Kh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
+      vu[i] = ok ? dec::ldg16(Vh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
     }
-    const float bm = warp_max(fmaxf(s2[0], s2[1]));
-    const float mn = fmaxf(m, bm);
-    const float part = warp_sum(exp2f(s2[0] - mn) + exp2f(s2[1] - mn));
-    l = l * exp2f(m - mn) + part;
+    float v[8][1];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x[E];
+      dec::Chunk<T>::cvt(ku[i], x);
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[e], a);
+      v[i][0] = a;
+    }
+    const int ii = dec::reduce_rows<LPR, 1>(v, lane);
+    const float sc = rbase + S::row(ii, lane) < nk ? v[0][0] : -INFINITY;
+    const float mn = fmaxf(m, warp_max(sc));  // finite: row rbase is a key
+    const float alpha = exp2f(m - mn);
+    const float pr = exp2f(sc - mn);
+    l = l * alpha + (dec::row_owner<LPR>(lane) ? pr : 0.f);
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] *= alpha;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float pi = __shfl_sync(0xffffffffu, pr, dec::holder<LPR>(i, lane));
+      float x[E];
+      dec::Chunk<T>::cvt(vu[i], x);
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = fmaf(pi, x[e], o[e]);
+    }
     m = mn;
-    if (lane == 0) gt[row * nbc + j] = bm;  // raw maximum for now
+  }
+  // ---- the warp's totals, then the CTA's partial (m, l, o)
+  l = warp_sum(l);
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
+  __shared__ float wm[4], wl[4], wo[4][D];
+  __shared__ int last;
+  if (lane < LPR) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) wo[warp][lane * E + e] = o[e];
   }
   if (lane == 0) {
     wm[warp] = m;
     wl[warp] = l;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
+  float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+  float* pp = p.part + (row * p.splits + split) * (long long)(D + 2);
+  for (int t = tid; t < D; t += 128) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      if (wm[w] > -INFINITY) a += wo[w][t] * exp2f(wm[w] - M);
+    pp[t] = a;
+  }
+  if (tid == 0) {
     float L = 0.f;
-    for (int w = 0; w < 8; ++w)
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
       if (wm[w] > -INFINITY) L += wl[w] * exp2f(wm[w] - M);
-    sh_lse = M + log2f(L);
-    if (lse) lse[row] = sh_lse * 0.6931471805599453f;
+    pp[D] = M;
+    pp[D + 1] = L;
+  }
+  // ---- the row's last CTA merges the splits
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(p.ticket + row, 1) == p.splits - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* pr = p.part + row * p.splits * (long long)(D + 2);
+  M = -INFINITY;
+  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, __ldcg(pr + s * (D + 2) + D));
+  float L = 0.f;
+  for (int s = 0; s < p.splits; ++s) {
+    const float ms = __ldcg(pr + s * (D + 2) + D);
+    if (ms > -INFINITY) L += __ldcg(pr + s * (D + 2) + D + 1) * exp2f(ms - M);
+  }
+  const float invL = 1.0f / L;
+  for (int t = tid; t < D; t += 128) {
+    float a = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float ms = __ldcg(pr + s * (D + 2) + D);
+      if (ms > -INFINITY) a += __ldcg(pr + s * (D + 2) + t) * exp2f(ms - M);
+    }
+    const float v = a * invL;
+    if constexpr (sizeof(T) == 2)
+      reinterpret_cast<__nv_bfloat16*>(p.O)[row * D + t] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<float*>(p.O)[row * D + t] = v;
+  }
+  if (tid == 0) {
+    if (p.lse) p.lse[row] = (M + log2f(L)) * 0.6931471805599453f;
+    p.ticket[row] = 0;
+  }
+}
+
+// ------------------------------------------------------ 1D ground truth ---
+struct DecGtP {
+  const void* q;
+  const void* K;
+  int Hq, Hkv, n_cap, seq_len, bpc, nch;
+  float scale_log2;
+  float* gt;
+  float* lse;
+  float* stats;
+  int32_t* ticket;
+};
+
+template <typename T, int D, int GT>
+__global__ void __launch_bounds__(128, 3) decode_gt_kernel(const DecGtP p) {
+  using S = dec::Slab<T, D>;
+  constexpr int E = S::EPC;
+  constexpr int LPR = S::LPR;
+  constexpr int SPB = kBlock / S::ROWS;
+  const int G = p.Hq / p.Hkv, nhg = G / GT;
+  const int ch = (int)(blockIdx.x % p.nch);
+  const long long grp = blockIdx.x / p.nch;  // (b * Hkv + g) * nhg + hg
+  const int hg = (int)(grp % nhg);
+  const long long bg = grp / nhg;
+  const long long b = bg / p.Hkv;
+  const int g = (int)(bg % p.Hkv);
+  const long long row0 = b * p.Hq + (long long)g * G + hg * GT;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = (p.seq_len - 1) / kBlock;
+  const int nbc = c + 1;
+  const T* q = reinterpret_cast<const T*>(p.q);
+  float qv[GT][E];
+#pragma unroll
+  for (int h = 0; h < GT; ++h)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[h][e] = dec::ld1(q, (row0 + h) * D + S::chunk(lane) * E + e) * p.scale_log2;
+  const T* Kh = reinterpret_cast<const T*>(p.K) + bg * (long long)p.n_cap * D + S::chunk(lane) * E;
+  float m[GT], l[GT];
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+  }
+  const int jb = ch * p.bpc, je = min(nbc, jb + p.bpc);
+  for (int j = jb + warp; j < je; j += 4) {
+    const int nk = j < c ? kBlock : p.seq_len - c * kBlock;
+    float bm[GT];
+#pragma unroll
+    for (int h = 0; h < GT; ++h) bm[h] = -INFINITY;
+#pragma unroll
+    for (int sb = 0; sb < SPB; ++sb) {
+      const int rbase = sb * S::ROWS;
+      if (rbase >= nk) break;  // warp-uniform
+      const long long off = ((long long)j * kBlock + rbase) * D;
+      uint4 ku[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = S::row(i, lane);
+        ku[i] = rbase + r < nk ? dec::ldg16(Kh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float v[8][GT];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x[E];
+        dec::Chunk<T>::cvt(ku[i], x);
+#pragma unroll
+        for (int h = 0; h < GT; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[h][e], a);
+          v[i][h] = a;
+        }
+      }
+      const int ii = dec::reduce_rows<LPR, GT>(v, lane);
+      const bool ok = rbase + S::row(ii, lane) < nk;
+      const bool own = dec::row_owner<LPR>(lane);
+#pragma unroll
+      for (int h = 0; h < GT; ++h) {
+        const float sc = ok ? v[0][h] : -INFINITY;
+        const float mx = warp_max(sc);
+        bm[h] = fmaxf(bm[h], mx);
+        const float mn = fmaxf(m[h], mx);
+        l[h] = l[h] * exp2f(m[h] - mn) + (own ? exp2f(sc - mn) : 0.f);
+        m[h] = mn;
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < GT; ++h) p.gt[(row0 + h) * nbc + j] = bm[h];  // raw, log2 units
+    }
+  }
+  // ---- the chunk's statistics per head
+  __shared__ float wm[4][GT], wl[4][GT];
+  __shared__ float lse2[GT];
+  __shared__ int last;
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    const float lw = warp_sum(l[h]);
+    if (lane == 0) {
+      wm[warp][h] = m[h];
+      wl[warp][h] = lw;
+    }
   }
   __syncthreads();
-  const float l2 = sh_lse;
-  for (int j = threadIdx.x; j < nbc; j += blockDim.x) gt[row * nbc + j] = exp2f(gt[row * nbc + j] - l2);
+  if (tid < GT) {
+    float M = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      if (wm[w][tid] > -INFINITY) L += wl[w][tid] * exp2f(wm[w][tid] - M);
+    float* st = p.stats + ((row0 + tid) * kGtMaxChunks + ch) * 2;
+    st[0] = M;
+    st[1] = L;
+  }
+  // ---- the group's last CTA: the rows' LSE, then maxima -> probabilities
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(p.ticket + grp, 1) == p.nch - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (tid < GT) {
+    const float* st = p.stats + (row0 + tid) * kGtMaxChunks * 2;
+    float M = -INFINITY;
+    for (int k = 0; k < p.nch; ++k) M = fmaxf(M, __ldcg(st + 2 * k));
+    float L = 0.f;
+    for (int k = 0; k < p.nch; ++k) {
+      const float mk = __ldcg(st + 2 * k);
+      if (mk > -INFINITY) L += __ldcg(st + 2 * k + 1) * exp2f(mk - M);
+    }
+    lse2[tid] = M + log2f(L);
+    if (p.lse) p.lse[row0 + tid] = lse2[tid] * 0.6931471805599453f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < GT; ++h) {
+    float* gr = p.gt + (row0 + h) * nbc;
+    for (int j = tid; j < nbc; j += 128) gr[j] = exp2f(__ldcg(gr + j) - lse2[h]);
+  }
+  if (tid == 0) p.ticket[grp] = 0;
 }
 
 // ------------------------------------------------------------- launchers --
+namespace {
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n = v;
+  }
+  return n;
+}
+
+// largest of 4, 2, 1 that divides the group size
+int head_tile(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
+}  // namespace
+
 cudaError_t launch_kcache(const void* K, bool fp32, const float* Wk, float* kt, long long BHkv, int Hkv, int n_cap,
-                          int d, int h, int j0, int nnew, cudaStream_t st) {
-  const size_t smem = sizeof(float) * 3 * d;
-  const unsigned grid = (unsigned)(BHkv * nnew);
-  if (fp32)
-    kcache_kernel<float><<<grid, 128, smem, st>>>((const float*)K, Wk, kt, Hkv, n_cap, d, h, j0, nnew);
-  else
-    kcache_kernel<uint16_t><<<grid, 128, smem, st>>>((const uint16_t*)K, Wk, kt, Hkv, n_cap, d, h, j0, nnew);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_decode_logits(const void* q, bool fp32, const float* kt, float* logits, long long rows, int Hq,
-                                 int Hkv, int d, int nc, int nb_cap, float scale, cudaStream_t st) {
-  if (fp32)
-    decode_logits_kernel<float><<<(unsigned)rows, 256, 0, st>>>((const float*)q, kt, logits, Hq, Hkv, d, nc, nb_cap,
-                                                                scale);
-  else
-    decode_logits_kernel<uint16_t><<<(unsigned)rows, 256, 0, st>>>((const uint16_t*)q, kt, logits, Hq, Hkv, d, nc,
-                                                                   nb_cap, scale);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_decode_attn(const DecodeAttnArgs& a, cudaStream_t st) {
-  dim3 grid((unsigned)a.rows, (unsigned)a.splits);
-  if (a.fp32) {
-    decode_attn_kernel<float><<<grid, 128, 0, st>>>((const float*)a.q, (const float*)a.K, (const float*)a.V,
-                                                    a.counts, a.indices, a.cap, a.Hq, a.Hkv, a.d, a.n_cap, a.seq_len,
-                                                    a.scale_log2, a.splits, a.part, a.status);
-    decode_combine_kernel<float><<<(unsigned)a.rows, 128, 0, st>>>(a.part, a.splits, a.d, (float*)a.O, a.lse);
+                          int d, int j0, int nnew, cudaStream_t st) {
+  const size_t smem = sizeof(float) * ((size_t)kKcBlocks * 3 * d + (size_t)d * 33);
+  const long long grid = BHkv * ((nnew + kKcBlocks - 1) / kKcBlocks);
+  if (fp32) {
+    if (d == 64)
+      kcache_kernel<float, 64><<<(unsigned)grid, kKcThreads, smem, st>>>((const float*)K, Wk, kt, Hkv, n_cap, j0, nnew);
+    else
+      kcache_kernel<float, 128><<<(unsigned)grid, kKcThreads, smem, st>>>((const float*)K, Wk, kt, Hkv, n_cap, j0,
+                                                                          nnew);
   } else {
-    decode_attn_kernel<uint16_t><<<grid, 128, 0, st>>>((const uint16_t*)a.q, (const uint16_t*)a.K,
-                                                       (const uint16_t*)a.V, a.counts, a.indices, a.cap, a.Hq, a.Hkv,
-                                                       a.d, a.n_cap, a.seq_len, a.scale_log2, a.splits, a.part,
-                                                       a.status);
-    decode_combine_kernel<uint16_t><<<(unsigned)a.rows, 128, 0, st>>>(a.part, a.splits, a.d, (uint16_t*)a.O, a.lse);
+    if (d == 64)
+      kcache_kernel<uint16_t, 64><<<(unsigned)grid, kKcThreads, smem, st>>>((const uint16_t*)K, Wk, kt, Hkv, n_cap,
+                                                                            j0, nnew);
+    else
+      kcache_kernel<uint16_t, 128><<<(unsigned)grid, kKcThreads, smem, st>>>((const uint16_t*)K, Wk, kt, Hkv, n_cap,
+                                                                             j0, nnew);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_gt(const void* q, const void* K, bool fp32, long long rows, int Hq, int Hkv, int d,
-                             int n_cap, int seq_len, float scale_log2, float* gt, float* lse, cudaStream_t st) {
-  if (fp32)
-    decode_gt_kernel<float><<<(unsigned)rows, 256, 0, st>>>((const float*)q, (const float*)K, Hq, Hkv, d, n_cap,
-                                                            seq_len, scale_log2, gt, lse);
+template <typename T, int D>
+static void logits_dispatch_gt(int GT, unsigned grid, const T* q, const float* kt, float* logits, int Hq, int Hkv,
+                               int nc, int nb_cap, int rpc, int nch, float scale, cudaStream_t st) {
+  if (GT == 4)
+    decode_logits_kernel<T, D, 4><<<grid, 128, 0, st>>>(q, kt, logits, Hq, Hkv, nc, nb_cap, rpc, nch, scale);
+  else if (GT == 2)
+    decode_logits_kernel<T, D, 2><<<grid, 128, 0, st>>>(q, kt, logits, Hq, Hkv, nc, nb_cap, rpc, nch, scale);
   else
-    decode_gt_kernel<uint16_t><<<(unsigned)rows, 256, 0, st>>>((const uint16_t*)q, (const uint16_t*)K, Hq, Hkv, d,
-                                                               n_cap, seq_len, scale_log2, gt, lse);
+    decode_logits_kernel<T, D, 1><<<grid, 128, 0, st>>>(q, kt, logits, Hq, Hkv, nc, nb_cap, rpc, nch, scale);
+}
+
+cudaError_t launch_decode_logits(const void* q, bool fp32, const float* kt, float* logits, long long B, int Hq,
+                                 int Hkv, int d, int nc, int nb_cap, float scale, cudaStream_t st) {
+  const int GT = head_tile(Hq / Hkv);
+  const long long groups = B * (long long)Hq / GT;
+  // rows of a CTA: a multiple of the 4 warps' slabs, about 8 CTAs per SM
+  const int unit = 4 * (d == 64 ? 16 : 8);
+  long long rpc = (nc * groups + 8LL * sm_count() - 1) / (8LL * sm_count());
+  rpc = ((rpc + unit - 1) / unit) * unit;
+  if (rpc < unit) rpc = unit;
+  const int nch = (int)((nc + rpc - 1) / rpc);
+  const unsigned grid = (unsigned)(groups * nch);
+  if (fp32) {
+    if (d == 64)
+      logits_dispatch_gt<float, 64>(GT, grid, (const float*)q, kt, logits, Hq, Hkv, nc, nb_cap, (int)rpc, nch, scale,
+                                    st);
+    else
+      logits_dispatch_gt<float, 128>(GT, grid, (const float*)q, kt, logits, Hq, Hkv, nc, nb_cap, (int)rpc, nch, scale,
+                                     st);
+  } else {
+    if (d == 64)
+      logits_dispatch_gt<uint16_t, 64>(GT, grid, (const uint16_t*)q, kt, logits, Hq, Hkv, nc, nb_cap, (int)rpc, nch,
+                                       scale, st);
+    else
+      logits_dispatch_gt<uint16_t, 128>(GT, grid, (const uint16_t*)q, kt, logits, Hq, Hkv, nc, nb_cap, (int)rpc, nch,
+                                        scale, st);
+  }
+  return cudaGetLastError();
+}
+
+int decode_attn_splits(long long rows) {
+  // about four resident CTAs per SM over all rows
+  const long long target = 4LL * sm_count();
+  long long s = (target + rows - 1) / rows;
+  return (int)(s < 1 ? 1 : (s > 64 ? 64 : s));
+}
+
+cudaError_t launch_decode_attn(const DecodeAttnArgs& a, cudaStream_t st) {
+  DecAttnP p{a.q, a.K, a.V, a.counts, a.indices, a.cap, a.Hq, a.Hkv, a.n_cap, a.seq_len, a.splits, a.scale_log2,
+             a.part, a.ticket, a.O, a.lse, a.status};
+  const unsigned grid = (unsigned)(a.rows * a.splits);
+  if (a.fp32) {
+    if (a.d == 64)
+      decode_attn_kernel<float, 64><<<grid, 128, 0, st>>>(p);
+    else
+      decode_attn_kernel<float, 128><<<grid, 128, 0, st>>>(p);
+  } else {
+    if (a.d == 64)
+      decode_attn_kernel<uint16_t, 64><<<grid, 128, 0, st>>>(p);
+    else
+      decode_attn_kernel<uint16_t, 128><<<grid, 128, 0, st>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+static void gt_dispatch(int GT, unsigned grid, const DecGtP& p, cudaStream_t st) {
+  if (GT == 4)
+    decode_gt_kernel<T, D, 4><<<grid, 128, 0, st>>>(p);
+  else if (GT == 2)
+    decode_gt_kernel<T, D, 2><<<grid, 128, 0, st>>>(p);
+  else
+    decode_gt_kernel<T, D, 1><<<grid, 128, 0, st>>>(p);
+}
+
+cudaError_t launch_decode_gt(const void* q, const void* K, bool fp32, long long B, int Hq, int Hkv, int d, int n_cap,
+                             int seq_len, float scale_log2, float* gt, float* lse, float* stats, int32_t* ticket,
+                             cudaStream_t st) {
+  const int GT = head_tile(Hq / Hkv);
+  const long long groups = B * (long long)Hq / GT;
+  const int nbc = (seq_len - 1) / kBlock + 1;
+  // about two waves of three CTAs per SM, at most kGtMaxChunks chunks a row
+  long long nch = (6LL * sm_count() + groups - 1) / groups;
+  if (nch > kGtMaxChunks) nch = kGtMaxChunks;
+  if (nch > nbc) nch = nbc;
+  if (nch < 1) nch = 1;
+  const int bpc = (int)((nbc + nch - 1) / nch);
+  nch = (nbc + bpc - 1) / bpc;
+  DecGtP p{q, K, Hq, Hkv, n_cap, seq_len, bpc, (int)nch, scale_log2, gt, lse, stats, ticket};
+  const unsigned grid = (unsigned)(groups * nch);
+  if (fp32) {
+    if (d == 64)
+      gt_dispatch<float, 64>(GT, grid, p, st);
+    else
+      gt_dispatch<float, 128>(GT, grid, p, st);
+  } else {
+    if (d == 64)
+      gt_dispatch<uint16_t, 64>(GT, grid, p, st);
+    else
+      gt_dispatch<uint16_t, 128>(GT, grid, p, st);
+  }
   return cudaGetLastError();
 }
 

@@ -63,10 +63,12 @@ def test_kcache_rejects():
 
 
 @pytest.mark.parametrize("mode,kw", MODES)
-@pytest.mark.parametrize("dtype,d,nb,seq_len", [("fp32", 64, 12, 64 * 11 + 1), ("bf16", 128, 20, 64 * 20),
-                                                ("bf16", 128, 40, 64 * 33 + 17)])
-def test_gate(mode, kw, dtype, d, nb, seq_len):
-    w, q, Kc, Vc, Wk = _case(2, 8, 2, nb, d, dtype, seq_len)
+@pytest.mark.parametrize("dtype,d,nb,seq_len,Hq,Hkv", [("fp32", 64, 12, 64 * 11 + 1, 8, 2), ("bf16", 128, 20, 64 * 20, 8, 2),
+                                                        ("bf16", 128, 40, 64 * 33 + 17, 8, 2),
+                                                        ("bf16", 64, 300, 64 * 290 + 3, 6, 2),
+                                                        ("fp32", 128, 50, 64 * 45, 4, 2)])
+def test_gate(mode, kw, dtype, d, nb, seq_len, Hq, Hkv):
+    w, q, Kc, Vc, Wk = _case(2, Hq, Hkv, nb, d, dtype, seq_len)
     c = (seq_len - 1) // 64
     kt = _kt(Kc, Wk, c)
     counts, idx, scores = seer.seer_decode_gate(q.cuda(), kt, w.n, seq_len, mode, return_scores=True, **kw)
@@ -112,6 +114,24 @@ def test_attn_selected(dtype, d, nb, seq_len):
     assert np.abs(lse.cpu().double().numpy() - lse_ref).max() <= tol
 
 
+def test_attn_repeat_same_workspace():
+    """Back-to-back calls on one workspace give identical results (the
+    per-row merge tickets are left at zero)."""
+    w, q, Kc, Vc, Wk = _case(2, 8, 2, 40, 128, "bf16", 64 * 39 + 11)
+    seq_len = 64 * 39 + 11
+    kt = _kt(Kc, Wk, 39)
+    counts, idx = seer.seer_decode_gate(q.cuda(), kt, w.n, seq_len, seer.SELECT_TOPK_K, k=9)
+    ws = torch.empty(seer.sparse_decode_attn_workspace_size(2, 8, 2, w.n, 128), dtype=torch.uint8, device="cuda")
+    qd, Kd, Vd = q.cuda(), Kc.cuda(), Vc.cuda()
+    O1, l1 = seer.seer_sparse_decode_attn(qd, Kd, Vd, seq_len, counts, idx, workspace=ws)
+    O2, l2 = seer.seer_sparse_decode_attn(qd, Kd, Vd, seq_len, counts, idx, workspace=ws)
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    gws = torch.empty(seer.decode_blockmax_workspace_size(2, 8, 2, w.n, 128), dtype=torch.uint8, device="cuda")
+    g1, _ = seer.seer_decode_blockmax(qd, Kd, seq_len, workspace=gws)
+    g2, _ = seer.seer_decode_blockmax(qd, Kd, seq_len, workspace=gws)
+    assert torch.equal(g1, g2)
+
+
 def test_attn_all_candidates_is_dense():
     """Every complete block listed: the result is the token's full causal
     attention (blockmax's LSE is the same row statistic)."""
@@ -151,10 +171,11 @@ def test_attn_bad_list_recorded():
     assert seer.seer_workspace_status(ws) == 6  # SEER_ERR_DEVICE_CHECK
 
 
-@pytest.mark.parametrize("dtype,d,nb,seq_len", [("fp32", 64, 6, 64 * 5 + 7), ("bf16", 128, 20, 64 * 20),
-                                                ("bf16", 64, 9, 33)])
-def test_blockmax(dtype, d, nb, seq_len):
-    w, q, Kc, Vc, Wk = _case(2, 8, 4, nb, d, dtype, seq_len)
+@pytest.mark.parametrize("dtype,d,nb,seq_len,Hq,Hkv", [("fp32", 64, 6, 64 * 5 + 7, 8, 4), ("bf16", 128, 20, 64 * 20, 8, 2),
+                                                        ("bf16", 64, 9, 33, 8, 4), ("bf16", 128, 70, 64 * 67 + 5, 6, 2),
+                                                        ("fp32", 128, 12, 64 * 11 + 30, 3, 3)])
+def test_blockmax(dtype, d, nb, seq_len, Hq, Hkv):
+    w, q, Kc, Vc, Wk = _case(2, Hq, Hkv, nb, d, dtype, seq_len)
     gt, lse = seer.seer_decode_blockmax(q.cuda(), Kc.cuda(), seq_len)
     gt_ref, lse_ref = oracle.decode_blockmax(q, Kc, seq_len)
     assert gt.shape[-1] == (seq_len - 1) // 64 + 1
