@@ -723,6 +723,7 @@ seer_status seer_sparse_decode_attn(const seer_dims* dims, const void* q, const 
   a.O = O;
   a.lse = lse;
   a.status = &((seer::WsHeader*)ws)->status;
+  a.timeout_ns = kTimeoutNs;
   SEER_CUDA(seer::launch_decode_attn(a, st));
   return SEER_OK;
 }
@@ -744,7 +745,8 @@ seer_status seer_decode_blockmax(const seer_dims* dims, const void* q, const voi
   const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)dims->d);
   SEER_CUDA(seer::launch_decode_gt(q, Kcache, dtype == SEER_FP32, dims->B, dims->Hq, dims->Hkv, dims->d, dims->n,
                                    seq_len, (float)(sc * 1.4426950408889634), gt_out, lse_out,
-                                   (float*)((uint8_t*)ws + w.stats), (int32_t*)((uint8_t*)ws + w.ticket), st));
+                                   (float*)((uint8_t*)ws + w.stats), (int32_t*)((uint8_t*)ws + w.ticket),
+                                   &((seer::WsHeader*)ws)->status, kTimeoutNs, st));
   return SEER_OK;
 }
 

@@ -22,7 +22,8 @@
 // Kernels:
 //   kcache_kernel       CTA per (batch, KV head, 16 blocks): pooling by slabs,
 //                       then the projection k~ = Wk[g] kbar as a shared-memory
-//                       tiled product (Wk read once per 16 blocks)
+//                       tiled product in packed f32x2 FMAs (Wk read once per
+//                       16 blocks)
 //   decode_logits_kernel  CTA per (batch, KV head, head group, row chunk):
 //                       q . k~_j / sqrt(d) for GT query heads of the group at
 //                       once (k~ read once for them); the softmax and the
@@ -168,11 +169,13 @@ __global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict_
                                                             int nnew) {
   using S = dec::Slab<T, D>;
   constexpr int E = S::EPC;
-  constexpr int NG = kKcThreads / D;       // output groups
-  constexpr int BPG = kKcBlocks / NG;      // blocks per output group
-  extern __shared__ float sm[];
-  float* kbar = sm;                        // [kKcBlocks][3D]
-  float* wt = sm + kKcBlocks * 3 * D;      // [D][33]
+  constexpr int NG = kKcThreads / D;   // output groups
+  constexpr int BPG = kKcBlocks / NG;  // blocks per output group (4 or 8)
+  constexpr int SPB = kBlock / S::ROWS;
+  constexpr int WS = D + 1;            // padded row of the weight tile
+  extern __shared__ __align__(16) float sm[];
+  float* kbarT = sm;                   // [3D][kKcBlocks]: pooled features, blocks contiguous
+  float* wt = sm + 3 * D * kKcBlocks;  // [32][D + 1]: a 32-feature slice of Wk[g]^T
   const int nch = (nnew + kKcBlocks - 1) / kKcBlocks;
   const long long bh = blockIdx.x / nch;
   const int ch = (int)(blockIdx.x % nch);
@@ -182,9 +185,8 @@ __global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict_
   const int nb_cap = n_cap / kBlock;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- pooling: warp w takes blocks w, w + 8
-  for (int t = warp; t < nblk; t += kKcThreads / 32) {
-    const T* base = K + (bh * n_cap + (long long)(jb + t) * kBlock) * D + S::chunk(lane) * E;
+  // ---- pooling: warp w takes blocks w, w + 8; two slabs of loads in flight
+  for (int t = warp; t < kKcBlocks; t += kKcThreads / 32) {
     float mx[E], mn[E], su[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -192,20 +194,24 @@ __global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict_
       mn[e] = INFINITY;
       su[e] = 0.f;
     }
+    if (t < nblk) {
+      const T* base = K + (bh * n_cap + (long long)(jb + t) * kBlock) * D + S::chunk(lane) * E;
 #pragma unroll
-    for (int s = 0; s < kBlock / S::ROWS; ++s) {
-      uint4 u[8];
+      for (int s0 = 0; s0 < SPB; s0 += 2) {
+        uint4 u[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) u[i] = dec::ldg16(base + (long long)(s * S::ROWS + S::row(i, lane)) * D);
+        for (int i = 0; i < 16; ++i)
+          u[i] = dec::ldg16(base + (long long)((s0 + (i >> 3)) * S::ROWS + S::row(i & 7, lane)) * D);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float x[E];
-        dec::Chunk<T>::cvt(u[i], x);
+        for (int i = 0; i < 16; ++i) {
+          float x[E];
+          dec::Chunk<T>::cvt(u[i], x);
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          mx[e] = fmaxf(mx[e], x[e]);
-          mn[e] = fminf(mn[e], x[e]);
-          su[e] += x[e];
+          for (int e = 0; e < E; ++e) {
+            mx[e] = fmaxf(mx[e], x[e]);
+            mn[e] = fminf(mn[e], x[e]);
+            su[e] += x[e];
+          }
         }
       }
     }
@@ -218,40 +224,51 @@ __global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict_
         su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
       }
     if (lane < S::LPR) {
-      float* kb = kbar + t * 3 * D + lane * E;
+      // blocks past the range pool to 0 (finite), their outputs are dropped
+      const bool live = t < nblk;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        kb[e] = mx[e];
-        kb[D + e] = mn[e];
-        kb[2 * D + e] = su[e] * (1.0f / kBlock);
+        const int f = lane * E + e;
+        kbarT[f * kKcBlocks + t] = live ? mx[e] : 0.f;
+        kbarT[(D + f) * kKcBlocks + t] = live ? mn[e] : 0.f;
+        kbarT[(2 * D + f) * kKcBlocks + t] = live ? su[e] * (1.0f / kBlock) : 0.f;
       }
     }
   }
 
-  // ---- projection: thread (o, group) accumulates BPG blocks
+  // ---- projection: thread (o, group) accumulates BPG blocks in f32x2 pairs
   const int o = threadIdx.x % D, grp = threadIdx.x / D;
-  float acc[BPG];
+  uint64_t acc[BPG / 2];
 #pragma unroll
-  for (int b = 0; b < BPG; ++b) acc[b] = 0.f;
+  for (int b = 0; b < BPG / 2; ++b) acc[b] = 0ull;
   const float* W = Wk + (long long)g * D * 3 * D;
   for (int e0 = 0; e0 < 3 * D; e0 += 32) {
-    __syncthreads();  // kbar complete / previous tile consumed
+    __syncthreads();  // kbarT complete / previous tile consumed
     for (int x = threadIdx.x; x < D * 32; x += kKcThreads) {
       const int r = x >> 5, cc = x & 31;
-      wt[r * 33 + cc] = W[(long long)r * 3 * D + e0 + cc];
+      wt[cc * WS + r] = W[(long long)r * 3 * D + e0 + cc];
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int ee = 0; ee < 32; ++ee) {
-      const float w = wt[o * 33 + ee];
+      const float w = wt[ee * WS + o];
+      const uint64_t w2 = f32x2_pack(w, w);
+      const float4* kb = reinterpret_cast<const float4*>(kbarT + (e0 + ee) * kKcBlocks + grp * BPG);
 #pragma unroll
-      for (int b = 0; b < BPG; ++b) acc[b] = fmaf(w, kbar[(grp * BPG + b) * 3 * D + e0 + ee], acc[b]);
+      for (int b4 = 0; b4 < BPG / 4; ++b4) {
+        const float4 v = kb[b4];
+        acc[2 * b4] = fma_f32x2(w2, f32x2_pack(v.x, v.y), acc[2 * b4]);
+        acc[2 * b4 + 1] = fma_f32x2(w2, f32x2_pack(v.z, v.w), acc[2 * b4 + 1]);
+      }
     }
   }
 #pragma unroll
-  for (int b = 0; b < BPG; ++b) {
-    const int t = grp * BPG + b;
-    if (t < nblk) kt[(bh * nb_cap + jb + t) * D + o] = acc[b];
+  for (int b = 0; b < BPG / 2; ++b) {
+    float lo, hi;
+    f32x2_unpack(acc[b], lo, hi);
+    const int t = grp * BPG + 2 * b;
+    if (t < nblk) kt[(bh * nb_cap + jb + t) * D + o] = lo;
+    if (t + 1 < nblk) kt[(bh * nb_cap + jb + t + 1) * D + o] = hi;
   }
 }
 
@@ -307,6 +324,19 @@ __global__ void __launch_bounds__(128) decode_logits_kernel(const T* __restrict_
   }
 }
 
+// ------------------------------------------------ streamed key-block ring --
+// The attention and ground-truth kernels stream whole key blocks through a
+// shared-memory ring filled by 1D bulk copies (TMA, no multicast): warp NS
+// issues the copies, consumer warp w takes the CTA's blocks w, w + NS, ...
+// from stage w, so every stage has one consumer and its own full/empty
+// mbarrier pair.  About 96 KB of ring per CTA, two CTAs per SM.
+template <int BLK_BYTES>
+struct Ring {
+  static constexpr int NS = (98304 / BLK_BYTES) < 2 ? 2 : ((98304 / BLK_BYTES) > 8 ? 8 : (98304 / BLK_BYTES));
+  static constexpr int THREADS = 32 * (NS + 1);
+  static constexpr uint32_t SMEM = (uint32_t)NS * BLK_BYTES;
+};
+
 // ------------------------------------------------------ decode attention --
 struct DecAttnP {
   const void* q;
@@ -321,20 +351,33 @@ struct DecAttnP {
   void* O;
   float* lse;
   uint32_t* status;
+  unsigned long long timeout_ns;
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(128, 4) decode_attn_kernel(const DecAttnP p) {
+struct AttnRing : Ring<2 * kBlock * D * (int)sizeof(T)> {
+  static constexpr uint32_t HALF = (uint32_t)kBlock * D * sizeof(T);  // K (then V) of a block
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel(const DecAttnP p) {
   using S = dec::Slab<T, D>;
+  using R = AttnRing<T, D>;
   constexpr int E = S::EPC;
   constexpr int LPR = S::LPR;
-  constexpr int SPB = kBlock / S::ROWS;  // slabs per key block
+  constexpr int NS = R::NS;
+  constexpr int SPB = kBlock / S::ROWS;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[NS], empty[NS];
+  __shared__ int abort_flag, last;
+  __shared__ float wm[NS], wl[NS], wo[NS][D];
   const long long row = blockIdx.x / p.splits;
   const int split = (int)(blockIdx.x % p.splits);
   const long long b = row / p.Hq;
   const int hq = (int)(row % p.Hq), g = hq / (p.Hq / p.Hkv);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = (p.seq_len - 1) / kBlock;
+  const int tail = p.seq_len - c * kBlock;  // keys of the token's own block
   int cnt = p.counts[row];
   const int lim = min(p.cap, c);
   if (cnt < 0 || cnt > lim) {
@@ -345,97 +388,134 @@ __global__ void __launch_bounds__(128, 4) decode_attn_kernel(const DecAttnP p) {
   const int total = cnt + 1;
   const int per = (total + p.splits - 1) / p.splits;
   const int e0 = split * per, e1 = min(total, e0 + per);
-  const T* q = reinterpret_cast<const T*>(p.q);
-  float qv[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) qv[e] = dec::ld1(q, row * D + S::chunk(lane) * E + e) * p.scale_log2;
-  const long long head0 = (b * p.Hkv + g) * (long long)p.n_cap * D + S::chunk(lane) * E;
-  const T* Kh = reinterpret_cast<const T*>(p.K) + head0;
-  const T* Vh = reinterpret_cast<const T*>(p.V) + head0;
-  float m = -INFINITY, l = 0.f, o[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) o[e] = 0.f;
-  const int nslabs = e1 > e0 ? (e1 - e0) * SPB : 0;
-  for (int s = warp; s < nslabs; s += 4) {
-    const int ent = e0 + s / SPB;
-    const int rbase = (s % SPB) * S::ROWS;
-    int j = c, nk = p.seq_len - c * kBlock;
-    if (ent < cnt) {
-      j = p.indices[row * p.cap + ent];
-      if (j < 0 || j >= c) {
-        if (lane == 0) record_status(p.status, kDevBadIndex, (uint32_t)row);
-        j = j < 0 ? 0 : c - 1;
-      }
-      nk = kBlock;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    if (rbase >= nk) continue;  // past the token (warp-uniform)
-    const long long off = ((long long)j * kBlock + rbase) * D;
-    uint4 ku[8], vu[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = S::row(i, lane);
-      const bool ok = rbase + r < nk;
-      ku[i] = ok ? dec::ldg16(Kh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
-      vu[i] = ok ? dec::ldg16(Vh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float v[8][1];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float x[E];
-      dec::Chunk<T>::cvt(ku[i], x);
-      float a = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[e], a);
-      v[i][0] = a;
-    }
-    const int ii = dec::reduce_rows<LPR, 1>(v, lane);
-    const float sc = rbase + S::row(ii, lane) < nk ? v[0][0] : -INFINITY;
-    const float mn = fmaxf(m, warp_max(sc));  // finite: row rbase is a key
-    const float alpha = exp2f(m - mn);
-    const float pr = exp2f(sc - mn);
-    l = l * alpha + (dec::row_owner<LPR>(lane) ? pr : 0.f);
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[e] *= alpha;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float pi = __shfl_sync(0xffffffffu, pr, dec::holder<LPR>(i, lane));
-      float x[E];
-      dec::Chunk<T>::cvt(vu[i], x);
-#pragma unroll
-      for (int e = 0; e < E; ++e) o[e] = fmaf(pi, x[e], o[e]);
-    }
-    m = mn;
-  }
-  // ---- the warp's totals, then the CTA's partial (m, l, o)
-  l = warp_sum(l);
-#pragma unroll
-  for (int off = LPR; off < 32; off <<= 1)
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
-  __shared__ float wm[4], wl[4], wo[4][D];
-  __shared__ int last;
-  if (lane < LPR) {
-#pragma unroll
-    for (int e = 0; e < E; ++e) wo[warp][lane * E + e] = o[e];
-  }
-  if (lane == 0) {
-    wm[warp] = m;
-    wl[warp] = l;
+    abort_flag = 0;
+    fence_barrier_init();
   }
   __syncthreads();
-  float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+  volatile int* abort_p = &abort_flag;
+  const long long head0 = (b * p.Hkv + g) * (long long)p.n_cap * D;
+
+  if (warp == NS) {
+    // ------------------------------------------------------- producer ---
+    if (lane == 0) {
+      const T* Kh = reinterpret_cast<const T*>(p.K) + head0;
+      const T* Vh = reinterpret_cast<const T*>(p.V) + head0;
+      int it = 0;
+      for (int e = e0; e < e1; ++e, ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_p, p.status, p.timeout_ns)) break;
+        int j = c, nk = tail;
+        if (e < cnt) {
+          j = p.indices[row * p.cap + e];
+          if (j < 0 || j >= c) {
+            record_status(p.status, kDevBadIndex, (uint32_t)row);
+            j = j < 0 ? 0 : c - 1;
+          }
+          nk = kBlock;
+        }
+        const uint32_t bytes = (uint32_t)nk * D * sizeof(T);
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_load(ring + (size_t)s * 2 * R::HALF, Kh + (long long)j * kBlock * D, bytes, &full[s]);
+        bulk_load(ring + (size_t)s * 2 * R::HALF + R::HALF, Vh + (long long)j * kBlock * D, bytes, &full[s]);
+      }
+      // every issued copy has landed before the CTA may exit
+      for (int k = it > NS ? it - NS : 0; k < it; ++k)
+        mbar_wait(&full[k % NS], (k / NS) & 1, abort_p, nullptr, 20000000ull);
+    }
+  } else {
+    // ------------------------------------------------------ consumers ---
+    const T* q = reinterpret_cast<const T*>(p.q);
+    float qv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[e] = dec::ld1(q, row * D + S::chunk(lane) * E + e) * p.scale_log2;
+    float m = -INFINITY, l = 0.f, o[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = 0.f;
+    int k = 0;  // this warp's uses of its stage
+    for (int e = e0 + warp; e < e1; e += NS, ++k) {
+      if (!mbar_wait(&full[warp], k & 1, abort_p, p.status, p.timeout_ns)) break;
+      const int nk = e < cnt ? kBlock : tail;
+      const uint8_t* Ks = ring + (size_t)warp * 2 * R::HALF + S::chunk(lane) * 16;
+      const uint8_t* Vs = Ks + R::HALF;
+#pragma unroll
+      for (int sb = 0; sb < SPB; ++sb) {
+        const int rbase = sb * S::ROWS;
+        if (rbase >= nk) break;  // past the token (warp-uniform)
+        uint4 ku[8], vu[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = rbase + S::row(i, lane);
+          const bool ok = r < nk;
+          ku[i] = ok ? *reinterpret_cast<const uint4*>(Ks + (size_t)r * D * sizeof(T)) : make_uint4(0u, 0u, 0u, 0u);
+          vu[i] = ok ? *reinterpret_cast<const uint4*>(Vs + (size_t)r * D * sizeof(T)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float v[8][1];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float x[E];
+          dec::Chunk<T>::cvt(ku[i], x);
+          float a = 0.f;
+#pragma unroll
+          for (int ee = 0; ee < E; ++ee) a = fmaf(x[ee], qv[ee], a);
+          v[i][0] = a;
+        }
+        const int ii = dec::reduce_rows<LPR, 1>(v, lane);
+        const float sc = rbase + S::row(ii, lane) < nk ? v[0][0] : -INFINITY;
+        const float mn = fmaxf(m, warp_max(sc));  // finite: row rbase is a key
+        const float alpha = exp2f(m - mn);
+        const float pr = exp2f(sc - mn);
+        l = l * alpha + (dec::row_owner<LPR>(lane) ? pr : 0.f);
+#pragma unroll
+        for (int ee = 0; ee < E; ++ee) o[ee] *= alpha;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float pi = __shfl_sync(0xffffffffu, pr, dec::holder<LPR>(i, lane));
+          float x[E];
+          dec::Chunk<T>::cvt(vu[i], x);
+#pragma unroll
+          for (int ee = 0; ee < E; ++ee) o[ee] = fmaf(pi, x[ee], o[ee]);
+        }
+        m = mn;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[warp]);
+    }
+    l = warp_sum(l);
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+      for (int ee = 0; ee < E; ++ee) o[ee] += __shfl_xor_sync(0xffffffffu, o[ee], off);
+    if (lane < LPR) {
+#pragma unroll
+      for (int ee = 0; ee < E; ++ee) wo[warp][lane * E + ee] = o[ee];
+    }
+    if (lane == 0) {
+      wm[warp] = m;
+      wl[warp] = l;
+    }
+  }
+  __syncthreads();
+  // ---- the CTA's partial (m, l, o)
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NS; ++w) M = fmaxf(M, wm[w]);
   float* pp = p.part + (row * p.splits + split) * (long long)(D + 2);
-  for (int t = tid; t < D; t += 128) {
+  for (int t = tid; t < D; t += R::THREADS) {
     float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+    for (int w = 0; w < NS; ++w)
       if (wm[w] > -INFINITY) a += wo[w][t] * exp2f(wm[w] - M);
     pp[t] = a;
   }
   if (tid == 0) {
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+    for (int w = 0; w < NS; ++w)
       if (wm[w] > -INFINITY) L += wl[w] * exp2f(wm[w] - M);
     pp[D] = M;
     pp[D + 1] = L;
@@ -456,7 +536,7 @@ __global__ void __launch_bounds__(128, 4) decode_attn_kernel(const DecAttnP p) {
     if (ms > -INFINITY) L += __ldcg(pr + s * (D + 2) + D + 1) * exp2f(ms - M);
   }
   const float invL = 1.0f / L;
-  for (int t = tid; t < D; t += 128) {
+  for (int t = tid; t < D; t += R::THREADS) {
     float a = 0.f;
     for (int s = 0; s < p.splits; ++s) {
       const float ms = __ldcg(pr + s * (D + 2) + D);
@@ -484,14 +564,28 @@ struct DecGtP {
   float* lse;
   float* stats;
   int32_t* ticket;
+  uint32_t* status;
+  unsigned long long timeout_ns;
+};
+
+template <typename T, int D>
+struct GtRing : Ring<kBlock * D * (int)sizeof(T)> {
+  static constexpr uint32_t BLK = (uint32_t)kBlock * D * sizeof(T);
 };
 
 template <typename T, int D, int GT>
-__global__ void __launch_bounds__(128, 3) decode_gt_kernel(const DecGtP p) {
+__global__ void __launch_bounds__(GtRing<T, D>::THREADS, 2) decode_gt_kernel(const DecGtP p) {
   using S = dec::Slab<T, D>;
+  using R = GtRing<T, D>;
   constexpr int E = S::EPC;
   constexpr int LPR = S::LPR;
+  constexpr int NS = R::NS;
   constexpr int SPB = kBlock / S::ROWS;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[NS], empty[NS];
+  __shared__ int abort_flag, last;
+  __shared__ float wm[NS][GT], wl[NS][GT];
+  __shared__ float lse2[GT];
   const int G = p.Hq / p.Hkv, nhg = G / GT;
   const int ch = (int)(blockIdx.x % p.nch);
   const long long grp = blockIdx.x / p.nch;  // (b * Hkv + g) * nhg + hg
@@ -503,85 +597,124 @@ __global__ void __launch_bounds__(128, 3) decode_gt_kernel(const DecGtP p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = (p.seq_len - 1) / kBlock;
   const int nbc = c + 1;
-  const T* q = reinterpret_cast<const T*>(p.q);
-  float qv[GT][E];
-#pragma unroll
-  for (int h = 0; h < GT; ++h)
-#pragma unroll
-    for (int e = 0; e < E; ++e) qv[h][e] = dec::ld1(q, (row0 + h) * D + S::chunk(lane) * E + e) * p.scale_log2;
-  const T* Kh = reinterpret_cast<const T*>(p.K) + bg * (long long)p.n_cap * D + S::chunk(lane) * E;
-  float m[GT], l[GT];
-#pragma unroll
-  for (int h = 0; h < GT; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-  }
+  const int tail = p.seq_len - c * kBlock;
   const int jb = ch * p.bpc, je = min(nbc, jb + p.bpc);
-  for (int j = jb + warp; j < je; j += 4) {
-    const int nk = j < c ? kBlock : p.seq_len - c * kBlock;
-    float bm[GT];
-#pragma unroll
-    for (int h = 0; h < GT; ++h) bm[h] = -INFINITY;
-#pragma unroll
-    for (int sb = 0; sb < SPB; ++sb) {
-      const int rbase = sb * S::ROWS;
-      if (rbase >= nk) break;  // warp-uniform
-      const long long off = ((long long)j * kBlock + rbase) * D;
-      uint4 ku[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = S::row(i, lane);
-        ku[i] = rbase + r < nk ? dec::ldg16(Kh + off + (long long)r * D) : make_uint4(0u, 0u, 0u, 0u);
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* abort_p = &abort_flag;
+
+  if (warp == NS) {
+    // ------------------------------------------------------- producer ---
+    if (lane == 0) {
+      const T* Kh = reinterpret_cast<const T*>(p.K) + bg * (long long)p.n_cap * D;
+      int it = 0;
+      for (int j = jb; j < je; ++j, ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_p, p.status, p.timeout_ns)) break;
+        const uint32_t bytes = (uint32_t)(j < c ? kBlock : tail) * D * sizeof(T);
+        mbar_arrive_expect_tx(&full[s], bytes);
+        bulk_load(ring + (size_t)s * R::BLK, Kh + (long long)j * kBlock * D, bytes, &full[s]);
       }
-      float v[8][GT];
+      for (int k = it > NS ? it - NS : 0; k < it; ++k)
+        mbar_wait(&full[k % NS], (k / NS) & 1, abort_p, nullptr, 20000000ull);
+    }
+  } else {
+    // ------------------------------------------------------ consumers ---
+    const T* q = reinterpret_cast<const T*>(p.q);
+    float qv[GT][E];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float x[E];
-        dec::Chunk<T>::cvt(ku[i], x);
+    for (int h = 0; h < GT; ++h)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[h][e] = dec::ld1(q, (row0 + h) * D + S::chunk(lane) * E + e) * p.scale_log2;
+    // per-lane online statistics over the lane's own rows
+    float m[GT], l[GT];
+#pragma unroll
+    for (int h = 0; h < GT; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+    }
+    const bool own = dec::row_owner<LPR>(lane);
+    int k = 0;
+    for (int j = jb + warp; j < je; j += NS, ++k) {
+      if (!mbar_wait(&full[warp], k & 1, abort_p, p.status, p.timeout_ns)) break;
+      const int nk = j < c ? kBlock : tail;
+      const uint8_t* Ks = ring + (size_t)warp * R::BLK + S::chunk(lane) * 16;
+      float bm[GT];
+#pragma unroll
+      for (int h = 0; h < GT; ++h) bm[h] = -INFINITY;
+#pragma unroll
+      for (int sb = 0; sb < SPB; ++sb) {
+        const int rbase = sb * S::ROWS;
+        if (rbase >= nk) break;  // warp-uniform
+        uint4 ku[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = rbase + S::row(i, lane);
+          ku[i] = r < nk ? *reinterpret_cast<const uint4*>(Ks + (size_t)r * D * sizeof(T)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float v[8][GT];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float x[E];
+          dec::Chunk<T>::cvt(ku[i], x);
+#pragma unroll
+          for (int h = 0; h < GT; ++h) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[h][e], a);
+            v[i][h] = a;
+          }
+        }
+        const int ii = dec::reduce_rows<LPR, GT>(v, lane);
+        const bool ok = rbase + S::row(ii, lane) < nk;
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < E; ++e) a = fmaf(x[e], qv[h][e], a);
-          v[i][h] = a;
+          if (ok) {
+            const float sc = v[0][h];
+            bm[h] = fmaxf(bm[h], sc);
+            if (own) {
+              const float mn = fmaxf(m[h], sc);
+              l[h] = l[h] * exp2f(m[h] - mn) + exp2f(sc - mn);
+              m[h] = mn;
+            }
+          }
         }
       }
-      const int ii = dec::reduce_rows<LPR, GT>(v, lane);
-      const bool ok = rbase + S::row(ii, lane) < nk;
-      const bool own = dec::row_owner<LPR>(lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[warp]);
 #pragma unroll
-      for (int h = 0; h < GT; ++h) {
-        const float sc = ok ? v[0][h] : -INFINITY;
-        const float mx = warp_max(sc);
-        bm[h] = fmaxf(bm[h], mx);
-        const float mn = fmaxf(m[h], mx);
-        l[h] = l[h] * exp2f(m[h] - mn) + (own ? exp2f(sc - mn) : 0.f);
-        m[h] = mn;
+      for (int h = 0; h < GT; ++h) bm[h] = warp_max(bm[h]);
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < GT; ++h) p.gt[(row0 + h) * nbc + j] = bm[h];  // raw, log2 units
       }
     }
-    if (lane == 0) {
+    // the warp's statistics per head
 #pragma unroll
-      for (int h = 0; h < GT; ++h) p.gt[(row0 + h) * nbc + j] = bm[h];  // raw, log2 units
-    }
-  }
-  // ---- the chunk's statistics per head
-  __shared__ float wm[4][GT], wl[4][GT];
-  __shared__ float lse2[GT];
-  __shared__ int last;
-#pragma unroll
-  for (int h = 0; h < GT; ++h) {
-    const float lw = warp_sum(l[h]);
-    if (lane == 0) {
-      wm[warp][h] = m[h];
-      wl[warp][h] = lw;
+    for (int h = 0; h < GT; ++h) {
+      const float M = warp_max(m[h]);
+      const float lw = warp_sum(m[h] > -INFINITY ? l[h] * exp2f(m[h] - M) : 0.f);
+      if (lane == 0) {
+        wm[warp][h] = M;
+        wl[warp][h] = lw;
+      }
     }
   }
   __syncthreads();
   if (tid < GT) {
-    float M = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NS; ++w) M = fmaxf(M, wm[w][tid]);
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+    for (int w = 0; w < NS; ++w)
       if (wm[w][tid] > -INFINITY) L += wl[w][tid] * exp2f(wm[w][tid] - M);
     float* st = p.stats + ((row0 + tid) * kGtMaxChunks + ch) * 2;
     st[0] = M;
@@ -610,7 +743,7 @@ __global__ void __launch_bounds__(128, 3) decode_gt_kernel(const DecGtP p) {
 #pragma unroll
   for (int h = 0; h < GT; ++h) {
     float* gr = p.gt + (row0 + h) * nbc;
-    for (int j = tid; j < nbc; j += 128) gr[j] = exp2f(__ldcg(gr + j) - lse2[h]);
+    for (int j = tid; j < nbc; j += R::THREADS) gr[j] = exp2f(__ldcg(gr + j) - lse2[h]);
   }
   if (tid == 0) p.ticket[grp] = 0;
 }
@@ -633,7 +766,7 @@ int head_tile(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
 
 cudaError_t launch_kcache(const void* K, bool fp32, const float* Wk, float* kt, long long BHkv, int Hkv, int n_cap,
                           int d, int j0, int nnew, cudaStream_t st) {
-  const size_t smem = sizeof(float) * ((size_t)kKcBlocks * 3 * d + (size_t)d * 33);
+  const size_t smem = sizeof(float) * ((size_t)kKcBlocks * 3 * d + 32 * (size_t)(d + 1));
   const long long grid = BHkv * ((nnew + kKcBlocks - 1) / kKcBlocks);
   if (fp32) {
     if (d == 64)
@@ -693,67 +826,65 @@ cudaError_t launch_decode_logits(const void* q, bool fp32, const float* kt, floa
 }
 
 int decode_attn_splits(long long rows) {
-  // about four resident CTAs per SM over all rows
-  const long long target = 4LL * sm_count();
-  long long s = (target + rows - 1) / rows;
+  // two resident CTAs per SM over all rows
+  const long long target = 2LL * sm_count();
+  long long s = target / rows;
   return (int)(s < 1 ? 1 : (s > 64 ? 64 : s));
 }
 
+template <typename T, int D>
+static cudaError_t attn_launch(const DecAttnP& p, unsigned grid, cudaStream_t st) {
+  using R = AttnRing<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)R::SMEM);
+  if (e != cudaSuccess) return e;
+  decode_attn_kernel<T, D><<<grid, R::THREADS, R::SMEM, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, cudaStream_t st) {
-  DecAttnP p{a.q, a.K, a.V, a.counts, a.indices, a.cap, a.Hq, a.Hkv, a.n_cap, a.seq_len, a.splits, a.scale_log2,
-             a.part, a.ticket, a.O, a.lse, a.status};
+  DecAttnP p{a.q,        a.K,          a.V,      a.counts, a.indices, a.cap, a.Hq,    a.Hkv,
+             a.n_cap,    a.seq_len,    a.splits, a.scale_log2, a.part, a.ticket, a.O, a.lse,
+             a.status,   a.timeout_ns};
   const unsigned grid = (unsigned)(a.rows * a.splits);
-  if (a.fp32) {
-    if (a.d == 64)
-      decode_attn_kernel<float, 64><<<grid, 128, 0, st>>>(p);
-    else
-      decode_attn_kernel<float, 128><<<grid, 128, 0, st>>>(p);
-  } else {
-    if (a.d == 64)
-      decode_attn_kernel<uint16_t, 64><<<grid, 128, 0, st>>>(p);
-    else
-      decode_attn_kernel<uint16_t, 128><<<grid, 128, 0, st>>>(p);
-  }
+  if (a.fp32) return a.d == 64 ? attn_launch<float, 64>(p, grid, st) : attn_launch<float, 128>(p, grid, st);
+  return a.d == 64 ? attn_launch<uint16_t, 64>(p, grid, st) : attn_launch<uint16_t, 128>(p, grid, st);
+}
+
+template <typename T, int D, int GT>
+static cudaError_t gt_launch_one(const DecGtP& p, unsigned grid, cudaStream_t st) {
+  using R = GtRing<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(decode_gt_kernel<T, D, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)R::SMEM);
+  if (e != cudaSuccess) return e;
+  decode_gt_kernel<T, D, GT><<<grid, R::THREADS, R::SMEM, st>>>(p);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
-static void gt_dispatch(int GT, unsigned grid, const DecGtP& p, cudaStream_t st) {
-  if (GT == 4)
-    decode_gt_kernel<T, D, 4><<<grid, 128, 0, st>>>(p);
-  else if (GT == 2)
-    decode_gt_kernel<T, D, 2><<<grid, 128, 0, st>>>(p);
-  else
-    decode_gt_kernel<T, D, 1><<<grid, 128, 0, st>>>(p);
+static cudaError_t gt_dispatch(int GT, unsigned grid, const DecGtP& p, cudaStream_t st) {
+  if (GT == 4) return gt_launch_one<T, D, 4>(p, grid, st);
+  if (GT == 2) return gt_launch_one<T, D, 2>(p, grid, st);
+  return gt_launch_one<T, D, 1>(p, grid, st);
 }
 
 cudaError_t launch_decode_gt(const void* q, const void* K, bool fp32, long long B, int Hq, int Hkv, int d, int n_cap,
                              int seq_len, float scale_log2, float* gt, float* lse, float* stats, int32_t* ticket,
-                             cudaStream_t st) {
+                             uint32_t* status, unsigned long long timeout_ns, cudaStream_t st) {
   const int GT = head_tile(Hq / Hkv);
   const long long groups = B * (long long)Hq / GT;
   const int nbc = (seq_len - 1) / kBlock + 1;
-  // about two waves of three CTAs per SM, at most kGtMaxChunks chunks a row
-  long long nch = (6LL * sm_count() + groups - 1) / groups;
+  // one wave of two CTAs per SM, at most kGtMaxChunks chunks a row
+  long long nch = (2LL * sm_count()) / groups;
   if (nch > kGtMaxChunks) nch = kGtMaxChunks;
   if (nch > nbc) nch = nbc;
   if (nch < 1) nch = 1;
   const int bpc = (int)((nbc + nch - 1) / nch);
   nch = (nbc + bpc - 1) / bpc;
-  DecGtP p{q, K, Hq, Hkv, n_cap, seq_len, bpc, (int)nch, scale_log2, gt, lse, stats, ticket};
+  DecGtP p{q, K, Hq, Hkv, n_cap, seq_len, bpc, (int)nch, scale_log2, gt, lse, stats, ticket, status, timeout_ns};
   const unsigned grid = (unsigned)(groups * nch);
-  if (fp32) {
-    if (d == 64)
-      gt_dispatch<float, 64>(GT, grid, p, st);
-    else
-      gt_dispatch<float, 128>(GT, grid, p, st);
-  } else {
-    if (d == 64)
-      gt_dispatch<uint16_t, 64>(GT, grid, p, st);
-    else
-      gt_dispatch<uint16_t, 128>(GT, grid, p, st);
-  }
-  return cudaGetLastError();
+  if (fp32) return d == 64 ? gt_dispatch<float, 64>(GT, grid, p, st) : gt_dispatch<float, 128>(GT, grid, p, st);
+  return d == 64 ? gt_dispatch<uint16_t, 64>(GT, grid, p, st) : gt_dispatch<uint16_t, 128>(GT, grid, p, st);
 }
 
 }  // namespace seer

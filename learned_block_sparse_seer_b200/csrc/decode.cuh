@@ -35,6 +35,7 @@ struct DecodeAttnArgs {
   void* O;          // [rows, d]
   float* lse;       // [rows] or null
   uint32_t* status;
+  unsigned long long timeout_ns;  // bound of every wait
 };
 cudaError_t launch_decode_attn(const DecodeAttnArgs& a, cudaStream_t st);
 
@@ -46,6 +47,6 @@ constexpr int kGtMaxChunks = 256;
 // entry and left zero.
 cudaError_t launch_decode_gt(const void* q, const void* K, bool fp32, long long B, int Hq, int Hkv, int d, int n_cap,
                              int seq_len, float scale_log2, float* gt, float* lse, float* stats, int32_t* ticket,
-                             cudaStream_t st);
+                             uint32_t* status, unsigned long long timeout_ns, cudaStream_t st);
 
 }  // namespace seer

@@ -330,9 +330,17 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = tid; b < 256; b += kRowThreads) hist[b] = 0;
     __syncthreads();
-    for (int j = tid; j < len; j += kRowThreads) {
-      const uint32_t key = f2key(sv[j]);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 0xffu], 1u);
+    // Scores of a row share their top bits, so most keys fall into a few
+    // bins: lanes with the same bin are counted by one atomic (match_any).
+    for (int j0 = 0; j0 < len; j0 += kRowThreads) {
+      const int j = j0 + tid;
+      uint32_t bin = 0x100u;  // not counted
+      if (j < len) {
+        const uint32_t key = f2key(sv[j]);
+        if ((key & pmask) == prefix) bin = (key >> shift) & 0xffu;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0x100u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (tid < 32) {
