@@ -70,7 +70,14 @@ typedef enum {
   SEER_SELECT_TOPK_K = 1,
   /* TopK with a density rho: k_i = clamp(ceil(rho*(i+1)), 1, i+1), the product
      rounded in fp32.  Gives block sparsity ~ 1 - rho on every causal row. */
-  SEER_SELECT_TOPK_DENSITY = 2
+  SEER_SELECT_TOPK_DENSITY = 2,
+  /* Flag, OR-ed into any of the modes above: the diagonal block i always
+     joins row i's list (the list is the mode's selection plus i), so no row
+     is empty.  A top-k row may then hold k_i + 1 blocks.  (The pages do not
+     force the diagonal; the flag is an option, off unless given.)  For the
+     decode gate it changes nothing: the token's own block is always
+     attended there. */
+  SEER_SELECT_FORCE_DIAGONAL = 0x100
 } seer_select_mode;
 
 /* Problem shape.  n must be a multiple of `block`; Hq a multiple of Hkv. */
@@ -122,10 +129,44 @@ SEER_API seer_status seer_gate(const seer_dims *dims, const void *Q, const void 
 SEER_API size_t seer_gate_workspace_size(const seer_dims *dims, int32_t h);
 
 /* Smallest `cap` that can hold every row's list for this selection:
- * nb for THRESHOLD, min(k, nb) for TOPK_K, the largest k_i for TOPK_DENSITY.
+ * nb for THRESHOLD, min(k, nb) for TOPK_K, the largest k_i for TOPK_DENSITY;
+ * with SEER_SELECT_FORCE_DIAGONAL the top-k figures allow one more block
+ * (never more than the row length).  Also valid for seer_gate_varlen.
  * Returns -1 on invalid arguments. */
 SEER_API int32_t seer_gate_required_cap(const seer_dims *dims, seer_select_mode mode, int32_t k,
                                float density);
+
+/* seer_gate_varlen -- seer_gate over variable-length sequences packed along
+ * the token axis (rebuttal, batching: "variable-length inputs can be packed
+ * along the sequence dimension").  dims->B must be 1 and dims->n is the
+ * packed buffer's length (a multiple of 64).
+ *   seq_start, seq_len  DEVICE int32 arrays [nseq]: sequence s occupies tokens
+ *             seq_start[s] .. seq_start[s] + seq_len[s] - 1.  Each start is a
+ *             multiple of 64 (so a block belongs to one sequence), the
+ *             sequences ascend without overlap, and seq_len[s] >= 1.  Tokens
+ *             of no sequence are padding; the gate never reads them.
+ * Per sequence the gate is seer_gate's on that sequence alone: its last
+ * block pools only its own tokens, row i's candidates are the sequence's
+ * blocks f .. i (f its first block), k_i is taken at the local row i - f,
+ * and block RoPE (if on) rotates by block position (scores depend only on
+ * i - j, so packed and separate positions agree).  Lists hold global block
+ * indices, so seer_sparse_attn runs on the packed Q/K/V unchanged: inside a
+ * sequence's last block the causal rule already hides its padding keys from
+ * its tokens.  For that call the padding tokens of K and V must hold finite
+ * values (zero them), since a masked key still enters the PV product with
+ * weight 0.  Rows of blocks outside every sequence get count 0; rows of the
+ * padding positions of a last block are not meaningful.
+ * A malformed seq_start/seq_len entry is recorded as SEER_ERR_DEVICE_CHECK
+ * in the workspace status and its blocks are treated as padding.
+ * Other arguments, outputs and errors as seer_gate.                        */
+SEER_API seer_status seer_gate_varlen(const seer_dims *dims, const void *Q, const void *K, seer_dtype dtype,
+                                     const float *Wq, const float *Wk, int32_t h, float rope_theta,
+                                     const int32_t *seq_start, const int32_t *seq_len, int32_t nseq,
+                                     seer_select_mode mode, float T, int32_t k, float density,
+                                     float *scores_out, int32_t *counts, int32_t *indices, int32_t cap,
+                                     void *ws, size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_gate_varlen_workspace_size(const seer_dims *dims, int32_t h);
 
 /* seer_gate_kl_backward -- one distillation step of the AttnGate: its loss
  * and the gradients of the loss with respect to the gate's two linear layers

@@ -22,6 +22,7 @@ STATUS_NAMES = {
 }
 SEER_BF16, SEER_FP32 = 0, 1
 SELECT_THRESHOLD, SELECT_TOPK_K, SELECT_TOPK_DENSITY = 0, 1, 2
+SELECT_FORCE_DIAGONAL = 0x100  # flag OR-ed into a mode: the diagonal block joins every list
 
 
 class SeerError(RuntimeError):
@@ -56,6 +57,10 @@ def lib() -> ctypes.CDLL:
         L.seer_gate.argtypes = [DP, P, P, I32, P, P, I32, F, I32, F, I32, F, P, P, P, I32, P, SZ, P]
         L.seer_gate.restype = I32
         L.seer_gate_workspace_size.argtypes = [DP, I32]
+        L.seer_gate_varlen.argtypes = [DP, P, P, I32, P, P, I32, F, P, P, I32, I32, F, I32, F, P, P, P, I32, P, SZ, P]
+        L.seer_gate_varlen.restype = I32
+        L.seer_gate_varlen_workspace_size.argtypes = [DP, I32]
+        L.seer_gate_varlen_workspace_size.restype = SZ
         L.seer_gate_workspace_size.restype = SZ
         L.seer_gate_required_cap.argtypes = [DP, I32, I32, F]
         L.seer_gate_required_cap.restype = I32
@@ -148,11 +153,11 @@ def _workspace(nbytes: int, dev, ws: torch.Tensor | None) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
 
 
-def mode_code(mode) -> int:
-    if isinstance(mode, int):
-        return mode
-    return {"threshold": SELECT_THRESHOLD, "topk": SELECT_TOPK_K, "topk_k": SELECT_TOPK_K,
-            "density": SELECT_TOPK_DENSITY, "topk_density": SELECT_TOPK_DENSITY}[mode]
+def mode_code(mode, force_diagonal: bool = False) -> int:
+    if not isinstance(mode, int):
+        mode = {"threshold": SELECT_THRESHOLD, "topk": SELECT_TOPK_K, "topk_k": SELECT_TOPK_K,
+                "density": SELECT_TOPK_DENSITY, "topk_density": SELECT_TOPK_DENSITY}[mode]
+    return mode | (SELECT_FORCE_DIAGONAL if force_diagonal else 0)
 
 
 # --------------------------------------------------------------------- gate --
@@ -166,7 +171,7 @@ def gate_required_cap(B, Hq, Hkv, n, d, mode, k=0, density=0.0) -> int:
 
 
 def seer_gate(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, return_scores=False,
-              cap=None, workspace=None, out=None):
+              cap=None, workspace=None, out=None, force_diagonal=False):
     """AttnGate + mask generation.  Returns (counts, indices[, scores])."""
     dev = _dev(Q, K, Wq, Wk)
     B, Hq, n, d = Q.shape
@@ -175,7 +180,7 @@ def seer_gate(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, retur
         raise TypeError("gate weights must be fp32")
     h = Wq.shape[1]
     nb = n // 64
-    mc = mode_code(mode)
+    mc = mode_code(mode, force_diagonal)
     dims = _dims(B, Hq, Hkv, n, d)
     if cap is None:
         cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
@@ -251,13 +256,13 @@ def seer_gate_noalloc(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.
     return (counts, indices, scores) if return_scores else (counts, indices)
 
 
-def seer_gate_select(scores, mode, T=0.0, k=0, density=0.0, cap=None, out=None):
+def seer_gate_select(scores, mode, T=0.0, k=0, density=0.0, cap=None, out=None, force_diagonal=False):
     """Mask generation on supplied fp32 scores [B, Hq, nb, nb]."""
     dev = _dev(scores)
     if scores.dtype != torch.float32:
         raise TypeError("scores must be fp32")
     B, Hq, nb, _ = scores.shape
-    mc = mode_code(mode)
+    mc = mode_code(mode, force_diagonal)
     dims = _dims(B, Hq, 1, nb * 64, 64)
     if cap is None:
         cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
@@ -466,3 +471,43 @@ def seer_decode_blockmax(q, Kc, seq_len, scale=0.0, workspace=None, out=None):
                                     float(scale), _ptr(gt), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev))
     _check("seer_decode_blockmax", st)
     return gt, lse
+
+
+# ------------------------------------------------------------------ varlen --
+def gate_varlen_workspace_size(Hq, Hkv, n, d, h) -> int:
+    return int(lib().seer_gate_varlen_workspace_size(ctypes.byref(_dims(1, Hq, Hkv, n, d)), int(h)))
+
+
+def seer_gate_varlen(Q, K, Wq, Wk, seq_start, seq_len, mode, T=0.0, k=0, density=0.0, rope_theta=0.0,
+                     return_scores=False, cap=None, workspace=None, out=None, force_diagonal=False):
+    """AttnGate + mask generation over sequences packed along the token axis
+    (Q [1,Hq,n,d], K [1,Hkv,n,d]; seq_start / seq_len int32 CUDA tensors).
+    Returns (counts, indices[, scores]) with global block indices."""
+    dev = _dev(Q, K, Wq, Wk, seq_start, seq_len)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    if B != 1:
+        raise ValueError("packed sequences: B must be 1")
+    if seq_start.dtype != torch.int32 or seq_len.dtype != torch.int32:
+        raise TypeError("seq_start and seq_len must be int32")
+    if Wq.dtype != torch.float32 or Wk.dtype != torch.float32:
+        raise TypeError("gate weights must be fp32")
+    h = Wq.shape[1]
+    nb = n // 64
+    mc = mode_code(mode, force_diagonal)
+    dims = _dims(1, Hq, Hkv, n, d)
+    if cap is None:
+        cap = max(1, lib().seer_gate_required_cap(ctypes.byref(dims), mc, int(k), float(density)))
+    if out is None:
+        counts = torch.empty(1, Hq, nb, dtype=torch.int32, device=dev)
+        indices = torch.empty(1, Hq, nb, cap, dtype=torch.int32, device=dev)
+        scores = torch.empty(1, Hq, nb, nb, dtype=torch.float32, device=dev) if return_scores else None
+    else:
+        counts, indices, scores = out
+    ws = _workspace(gate_varlen_workspace_size(Hq, Hkv, n, d, h), dev, workspace)
+    st = lib().seer_gate_varlen(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq), _ptr(Wk), int(h),
+                                float(rope_theta), _ptr(seq_start), _ptr(seq_len), int(seq_start.numel()), mc,
+                                float(T), int(k), float(density), _ptr(scores), _ptr(counts), _ptr(indices),
+                                int(cap), _ptr(ws), ws.numel(), _stream(dev))
+    _check("seer_gate_varlen", st)
+    return (counts, indices, scores) if return_scores else (counts, indices)

@@ -324,16 +324,20 @@ seer_status seer_gate_kl_backward(const seer_dims* dims, const void* Q, const vo
 int32_t seer_gate_required_cap(const seer_dims* dims, seer_select_mode mode, int32_t k,
                                float density) {
   if (!dims_ok(dims)) return -1;
+  const int flags = (int)mode & ~0xff;
+  if (flags & ~(int)SEER_SELECT_FORCE_DIAGONAL) return -1;
+  const int fd = (flags & SEER_SELECT_FORCE_DIAGONAL) ? 1 : 0;
   const int nb = dims->n / seer::kBlock;
-  switch (mode) {
+  switch ((int)mode & 0xff) {
     case SEER_SELECT_THRESHOLD: return nb;
-    case SEER_SELECT_TOPK_K: return k < 1 ? -1 : (k < nb ? k : nb);
+    case SEER_SELECT_TOPK_K: return k < 1 ? -1 : (k + fd < nb ? k + fd : nb);
     case SEER_SELECT_TOPK_DENSITY: {
       if (!(density > 0.f && density <= 1.f)) return -1;
       int worst = 0;
       for (int i = 0; i < nb; ++i) {
         int ki = (int)std::ceil((double)(density * (float)(i + 1)));
         if (ki < 1) ki = 1;
+        ki += fd;
         if (ki > i + 1) ki = i + 1;
         if (ki > worst) worst = ki;
       }
@@ -345,7 +349,8 @@ int32_t seer_gate_required_cap(const seer_dims* dims, seer_select_mode mode, int
 
 static seer_status check_select(const seer_dims* dims, seer_select_mode mode, float T, int32_t k,
                                 float density, int32_t cap) {
-  switch (mode) {
+  if ((int)mode & ~0xff & ~(int)SEER_SELECT_FORCE_DIAGONAL) return SEER_ERR_INVALID_ARG;
+  switch ((int)mode & 0xff) {
     case SEER_SELECT_THRESHOLD:
       if (!(T > 0.f) || !std::isfinite(T)) return SEER_ERR_INVALID_ARG;
       break;
@@ -363,25 +368,14 @@ static seer_status check_select(const seer_dims* dims, seer_select_mode mode, fl
   return SEER_OK;
 }
 
-seer_status seer_gate(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype,
-                      const float* Wq, const float* Wk, int32_t h, float rope_theta,
-                      seer_select_mode mode, float T, int32_t k, float density, float* scores_out,
-                      int32_t* counts, int32_t* indices, int32_t cap, void* ws, size_t ws_bytes,
-                      seer_stream_t stream) {
-  if (!dims_ok(dims) || !Q || !K || !Wq || !Wk || !counts || !indices) return SEER_ERR_INVALID_ARG;
-  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
-  if (h < 1 || h > 256 || (h % 4) != 0) return SEER_ERR_INVALID_ARG;
-  if (!std::isfinite(rope_theta)) return SEER_ERR_INVALID_ARG;
-  seer_status s = dims_supported(dims);
-  if (s != SEER_OK) return s;
-  if (!aligned(Q, 16) || !aligned(K, 16)) return SEER_ERR_INVALID_ARG;
-  s = check_select(dims, mode, T, k, density, cap);
-  if (s != SEER_OK) return s;
+namespace {
+// The gate on a workspace laid out by gate_ws; `tab` is the varlen block
+// table (null for the plain batched layout).
+seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype, const float* Wq,
+                     const float* Wk, int32_t h, float rope_theta, seer_select_mode mode, float T, int32_t k,
+                     float density, float* scores_out, int32_t* counts, int32_t* indices, int32_t cap, void* ws,
+                     const int2* tab, cudaStream_t st) {
   const GateWs w = gate_ws(dims, h);
-  cudaStream_t st = (cudaStream_t)stream;
-  s = begin_ws(ws, ws_bytes, w.total, st);
-  if (s != SEER_OK) return s;
-
   uint8_t* base = (uint8_t*)ws;
   float* qbar = (float*)(base + w.qbar);
   float* kbar = (float*)(base + w.kbar);
@@ -391,8 +385,8 @@ seer_status seer_gate(const seer_dims* dims, const void* Q, const void* K, seer_
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
   const int nb = n / seer::kBlock, G = Hq / Hkv;
 
-  SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st));
-  SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st));
+  SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st, tab));
+  SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st, tab));
   // q~ = Wq[hq] qbar, k~ = Wk[g] kbar (batch z = b*H + head; weights by head)
   SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
                                  (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
@@ -408,8 +402,62 @@ seer_status seer_gate(const seer_dims* dims, const void* Q, const void* K, seer_
                                  (long long)nb * nb, nb, B * Hq, Hq, Hkv, G,
                                  (float)(1.0 / std::sqrt((double)d)), true, st));
   SEER_CUDA(seer::launch_row_select(logits, scores_out, true, (long long)B * Hq * nb, nb, (int)mode,
-                                    T, k, density, counts, indices, cap, st));
+                                    T, k, density, counts, indices, cap, st, 0, tab));
   return SEER_OK;
+}
+
+seer_status check_gate_args(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype, const float* Wq,
+                            const float* Wk, int32_t h, float rope_theta, seer_select_mode mode, float T, int32_t k,
+                            float density, int32_t* counts, int32_t* indices, int32_t cap) {
+  if (!dims_ok(dims) || !Q || !K || !Wq || !Wk || !counts || !indices) return SEER_ERR_INVALID_ARG;
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (h < 1 || h > 256 || (h % 4) != 0) return SEER_ERR_INVALID_ARG;
+  if (!std::isfinite(rope_theta)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16)) return SEER_ERR_INVALID_ARG;
+  return check_select(dims, mode, T, k, density, cap);
+}
+}  // namespace
+
+seer_status seer_gate(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype,
+                      const float* Wq, const float* Wk, int32_t h, float rope_theta,
+                      seer_select_mode mode, float T, int32_t k, float density, float* scores_out,
+                      int32_t* counts, int32_t* indices, int32_t cap, void* ws, size_t ws_bytes,
+                      seer_stream_t stream) {
+  seer_status s = check_gate_args(dims, Q, K, dtype, Wq, Wk, h, rope_theta, mode, T, k, density, counts, indices, cap);
+  if (s != SEER_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, gate_ws(dims, h).total, st);
+  if (s != SEER_OK) return s;
+  return run_gate(dims, Q, K, dtype, Wq, Wk, h, rope_theta, mode, T, k, density, scores_out, counts, indices, cap,
+                  ws, nullptr, st);
+}
+
+size_t seer_gate_varlen_workspace_size(const seer_dims* dims, int32_t h) {
+  if (!dims_ok(dims) || h < 1) return 0;
+  seer::WsCarver c;
+  c.off = gate_ws(dims, h).total;
+  c.take(sizeof(int2) * (size_t)(dims->n / seer::kBlock));
+  return c.off;
+}
+
+seer_status seer_gate_varlen(const seer_dims* dims, const void* Q, const void* K, seer_dtype dtype,
+                             const float* Wq, const float* Wk, int32_t h, float rope_theta,
+                             const int32_t* seq_start, const int32_t* seq_len, int32_t nseq,
+                             seer_select_mode mode, float T, int32_t k, float density, float* scores_out,
+                             int32_t* counts, int32_t* indices, int32_t cap, void* ws, size_t ws_bytes,
+                             seer_stream_t stream) {
+  seer_status s = check_gate_args(dims, Q, K, dtype, Wq, Wk, h, rope_theta, mode, T, k, density, counts, indices, cap);
+  if (s != SEER_OK) return s;
+  if (dims->B != 1 || !seq_start || !seq_len || nseq < 1) return SEER_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, seer_gate_varlen_workspace_size(dims, h), st);
+  if (s != SEER_OK) return s;
+  int2* tab = (int2*)((uint8_t*)ws + gate_ws(dims, h).total);
+  SEER_CUDA(seer::launch_varlen_table(seq_start, seq_len, nseq, dims->n, tab, &((seer::WsHeader*)ws)->status, st));
+  return run_gate(dims, Q, K, dtype, Wq, Wk, h, rope_theta, mode, T, k, density, scores_out, counts, indices, cap,
+                  ws, tab, st);
 }
 
 seer_status seer_gate_select(const seer_dims* dims, const float* scores, seer_select_mode mode,
@@ -648,6 +696,9 @@ seer_status seer_decode_kcache_update(const seer_dims* dims, const void* Kcache,
 int32_t seer_decode_gate_required_cap(const seer_dims* dims, int32_t seq_len, seer_select_mode mode, int32_t k,
                                       float density) {
   if (!dims_ok(dims) || !decode_len_ok(dims, seq_len)) return -1;
+  if ((int)mode & ~0xff & ~(int)SEER_SELECT_FORCE_DIAGONAL) return -1;
+  // the token's own block is always attended: the diagonal flag changes nothing
+  mode = (seer_select_mode)((int)mode & 0xff);
   return decode_required_cap(mode, k, density, (seq_len - 1) / seer::kBlock);
 }
 
@@ -660,6 +711,9 @@ seer_status seer_decode_gate(const seer_dims* dims, const void* q, seer_dtype dt
   seer_status s = dims_supported(dims);
   if (s != SEER_OK) return s;
   if (!decode_len_ok(dims, seq_len) || !aligned(kt_cache, 16)) return SEER_ERR_INVALID_ARG;
+  if ((int)mode & ~0xff & ~(int)SEER_SELECT_FORCE_DIAGONAL) return SEER_ERR_INVALID_ARG;
+  // the token's own block is always attended: the diagonal flag changes nothing
+  mode = (seer_select_mode)((int)mode & 0xff);
   if (mode == SEER_SELECT_THRESHOLD && !(T > 0.f)) return SEER_ERR_INVALID_ARG;
   if (mode == SEER_SELECT_TOPK_K && k < 1) return SEER_ERR_INVALID_ARG;
   if (mode == SEER_SELECT_TOPK_DENSITY && !(density > 0.f && density <= 1.f)) return SEER_ERR_INVALID_ARG;

@@ -21,15 +21,19 @@
 
 #include "common.cuh"
 #include "gate.cuh"
+#include "ptx.cuh"
 
 namespace seer {
 
 // ------------------------------------------------------------------ pool --
 // One warp per (head, block i).  Every lane loads 16 bytes of a row per step;
 // lanes that cover the same columns are combined with shuffles at the end.
+// With a varlen table, block i pools only its tab[i].y valid tokens (the
+// sequence's last block may be partial); a block of no sequence writes 0.
 template <typename T, bool IS_K>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long long nblocks,
-                                                   int n, int d, float* __restrict__ out) {
+                                                   int n, int d, float* __restrict__ out,
+                                                   const int2* __restrict__ tab) {
   constexpr int EPL = 16 / sizeof(T);  // elements per lane per load
   const long long warp = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (warp >= nblocks) return;
@@ -41,6 +45,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
   const int rpi = 32 / lpr;   // rows per iteration
   const int cg = lane % lpr;  // column group of this lane
   const T* base = X + ((bh * n) + (long long)i * kBlock) * d + cg * EPL;
+  const int valid = tab ? tab[i].y : kBlock;  // tokens of the block that belong to a sequence
 
   float sum[EPL], mx[EPL], mn[EPL];
 #pragma unroll
@@ -49,7 +54,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
     mx[e] = -INFINITY;
     mn[e] = INFINITY;
   }
-  for (int r = lane / lpr; r < kBlock; r += rpi) {
+  for (int r = lane / lpr; r < valid; r += rpi) {
     uint4 v = *reinterpret_cast<const uint4*>(base + (long long)r * d);
     float f[EPL];
     if constexpr (sizeof(T) == 2) {
@@ -85,17 +90,18 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
     }
   }
   if (lane < lpr) {
+    const float inv = valid > 0 ? 1.0f / (float)valid : 0.f;
     if (!IS_K) {
       float* o = out + ((bh * nb) + i) * (long long)d + cg * EPL;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) o[e] = sum[e] * (1.0f / kBlock);
+      for (int e = 0; e < EPL; ++e) o[e] = sum[e] * inv;
     } else {
       float* o = out + ((bh * nb) + i) * (long long)(3 * d) + cg * EPL;
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
-        o[e] = mx[e];
-        o[d + e] = mn[e];
-        o[2 * d + e] = sum[e] * (1.0f / kBlock);
+        o[e] = valid > 0 ? mx[e] : 0.f;
+        o[d + e] = valid > 0 ? mn[e] : 0.f;
+        o[2 * d + e] = sum[e] * inv;
       }
     }
   }
@@ -260,23 +266,40 @@ __device__ __forceinline__ int topk_count(int i, int mode, int k, float density)
 // j <= i (written to `scores` when non-null; j > i written as 0).  Otherwise
 // the row already holds scores.  Then the active blocks are written as an
 // ascending list.
+//  * mode carries SEER_SELECT_FORCE_DIAGONAL as a flag: block i joins the
+//    list whatever its score.
+//  * row_len > 0 (the decode gate): every row has row_len candidates.
+//  * tab (varlen packing): row i's candidates are its own sequence's blocks
+//    f .. i with f = tab[i].x (none when f < 0); k_i is taken at the local
+//    row i - f, and the list holds global block indices.
 template <bool FROM_LOGITS>
 __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
-    const float* in, float* scores, int nb, int mode, float T, int k,
-    float density, int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len) {
+    const float* in, float* scores, int nb, int mode_flags, float T, int k,
+    float density, int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len,
+    const int2* __restrict__ tab) {
   extern __shared__ float sv[];  // [nb]
   __shared__ int sh_i[32];
   __shared__ float sh_f[32];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sel_prefix, sel_remaining;
 
+  const int mode = mode_flags & 0xff;
+  const bool force_diag = (mode_flags & SEER_SELECT_FORCE_DIAGONAL) != 0;
   const long long row = blockIdx.x;
-  // causal prefill rows: query block i = row % nb; row_len > 0: every row
-  // has row_len candidates (the decode gate)
-  const int i = row_len > 0 ? row_len - 1 : (int)(row % nb);
-  const int len = i + 1;
+  const int ig = row_len > 0 ? row_len - 1 : (int)(row % nb);  // query block (global)
+  const int off = tab ? tab[ig].x : 0;  // first candidate block
   const int tid = threadIdx.x;
-  const float* src = in + row * (long long)nb;
+  if (off < 0) {  // a block of no sequence: no candidates
+    if (FROM_LOGITS && scores != nullptr) {
+      float* dst = scores + row * (long long)nb;
+      for (int j = tid; j < nb; j += kRowThreads) dst[j] = 0.f;
+    }
+    if (tid == 0) counts[row] = 0;
+    return;
+  }
+  const int i = ig - off;  // local query block: candidates are local 0 .. i
+  const int len = i + 1;
+  const float* src = in + row * (long long)nb + off;
 
   for (int j = tid; j < len; j += kRowThreads) sv[j] = src[j];
   __syncthreads();
@@ -296,7 +319,7 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
     __syncthreads();
     if (scores != nullptr) {
       float* dst = scores + row * (long long)nb;
-      for (int j = tid; j < nb; j += kRowThreads) dst[j] = j < len ? sv[j] : 0.f;
+      for (int j = tid; j < nb; j += kRowThreads) dst[j] = (j >= off && j - off < len) ? sv[j - off] : 0.f;
     }
   }
 
@@ -308,18 +331,18 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
 
   if (mode == SEER_SELECT_THRESHOLD) {
     int c = 0;
-    for (int j = j0; j < j1; ++j) c += sv[j] > T;
+    for (int j = j0; j < j1; ++j) c += sv[j] > T || (force_diag && j == i);
     int total;
     int pos = block_exclusive_scan(c, sh_i, &total);
     for (int j = j0; j < j1; ++j)
-      if (sv[j] > T) out[pos++] = j;
+      if (sv[j] > T || (force_diag && j == i)) out[pos++] = j + off;
     if (tid == 0) counts[row] = total;
     return;
   }
 
   const int ki = topk_count(i, mode, k, density);
   if (ki >= len) {  // every causal block is kept
-    for (int j = tid; j < len; j += kRowThreads) out[j] = j;
+    for (int j = tid; j < len; j += kRowThreads) out[j] = j + off;
     if (tid == 0) counts[row] = len;
     return;
   }
@@ -388,12 +411,14 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
     int r = eq_rank;
     for (int j = j0; j < j1; ++j) {
       const uint32_t key = f2key(sv[j]);
+      bool keep = force_diag && j == i;
       if (key > prefix) {
-        ++c;
+        keep = true;
       } else if (key == prefix) {
-        if ((uint32_t)r < remaining) ++c;
+        keep = keep || (uint32_t)r < remaining;
         ++r;
       }
+      c += keep;
     }
   }
   int total;
@@ -402,35 +427,74 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
     int r = eq_rank;
     for (int j = j0; j < j1; ++j) {
       const uint32_t key = f2key(sv[j]);
-      bool keep = false;
+      bool keep = force_diag && j == i;
       if (key > prefix) {
         keep = true;
       } else if (key == prefix) {
-        keep = (uint32_t)r < remaining;
+        keep = keep || (uint32_t)r < remaining;
         ++r;
       }
-      if (keep) out[pos++] = j;
+      if (keep) out[pos++] = j + off;
     }
   }
   if (tid == 0) counts[row] = total;
 }
 
+// ---------------------------------------------------------- varlen table --
+// Packed variable-length prefill: sequence s occupies tokens
+// start[s] .. start[s] + len[s] - 1 of the packed buffer, start[s] a multiple
+// of 64, the sequences in ascending order without overlap.  tab[i] = (first
+// block of block i's sequence, tokens of block i inside it), or (-1, 0) for a
+// block of no sequence.  Thread s also checks sequence s; a bad entry is
+// recorded in the status word and its blocks are treated as gaps.
+__global__ void varlen_table_kernel(const int32_t* __restrict__ start, const int32_t* __restrict__ len, int nseq,
+                                    int n, int2* __restrict__ tab, uint32_t* __restrict__ status) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nb = n / kBlock;
+  if (t < nseq) {
+    const int a = start[t], l = len[t];
+    const int lim = t + 1 < nseq ? start[t + 1] : n;
+    if (a < 0 || (a % kBlock) != 0 || l < 1 || a + l > lim || a + l > n) record_status(status, kDevBadIndex, (uint32_t)t);
+  }
+  if (t >= nb) return;
+  const int p = t * kBlock;  // first token of block t
+  // last sequence whose start is <= p (starts ascending)
+  int lo = 0, hi = nseq - 1, s = -1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    if (start[mid] <= p) {
+      s = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  int2 v = make_int2(-1, 0);
+  if (s >= 0) {
+    const int a = start[s], l = len[s];
+    const int lim = s + 1 < nseq ? start[s + 1] : n;
+    const bool ok = a >= 0 && (a % kBlock) == 0 && l >= 1 && a + l <= lim && a + l <= n;
+    if (ok && p < a + l) v = make_int2(a / kBlock, min(kBlock, a + l - p));
+  }
+  tab[t] = v;
+}
+
 // --------------------------------------------------------------- launchers --
 cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, int n, int d,
-                        float* out, cudaStream_t st) {
+                        float* out, cudaStream_t st, const int2* tab) {
   const long long nblocks = BH * (n / kBlock);
   const int warps = 8;
   const unsigned grid = (unsigned)((nblocks + warps - 1) / warps);
   if (dt == SEER_BF16) {
     if (is_k)
-      pool_kernel<uint16_t, true><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out);
+      pool_kernel<uint16_t, true><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab);
     else
-      pool_kernel<uint16_t, false><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out);
+      pool_kernel<uint16_t, false><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab);
   } else {
     if (is_k)
-      pool_kernel<float, true><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out);
+      pool_kernel<float, true><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab);
     else
-      pool_kernel<float, false><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out);
+      pool_kernel<float, false><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab);
   }
   return cudaGetLastError();
 }
@@ -457,22 +521,32 @@ cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cu
 
 cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, long long rows,
                               int nb, int mode, float T, int k, float density, int32_t* counts,
-                              int32_t* indices, int cap, cudaStream_t st, int row_len) {
+                              int32_t* indices, int cap, cudaStream_t st, int row_len, const int2* tab) {
   const size_t smem = (size_t)nb * sizeof(float);
   if (from_logits) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(row_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
     row_select_kernel<true><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, scores, nb, mode, T, k, density, counts, indices, cap, row_len);
+        in, scores, nb, mode, T, k, density, counts, indices, cap, row_len, tab);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(row_select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
     row_select_kernel<false><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, nullptr, nb, mode, T, k, density, counts, indices, cap, row_len);
+        in, nullptr, nb, mode, T, k, density, counts, indices, cap, row_len, tab);
   }
   return cudaGetLastError();
 }
 
+}  // namespace seer
+
+namespace seer {
+cudaError_t launch_varlen_table(const int32_t* start, const int32_t* len, int nseq, int n, int2* tab,
+                                uint32_t* status, cudaStream_t st) {
+  const int nb = n / kBlock;
+  const int m = nb > nseq ? nb : nseq;
+  varlen_table_kernel<<<(m + 255) / 256, 256, 0, st>>>(start, len, nseq, n, tab, status);
+  return cudaGetLastError();
+}
 }  // namespace seer

@@ -205,3 +205,42 @@ def make_decode(w: Workload, seq_len: int | None = None):
     if w.dtype == "bf16":
         q, K, V = (t.to(torch.bfloat16) for t in (q, K, V))
     return q.contiguous(), K.contiguous(), V.contiguous()
+
+
+def varlen_layout(lens, gap_blocks=None):
+    """Packed variable-length layout: sequence s starts at the first 64-token
+    boundary after sequence s - 1 plus gap_blocks[s] empty blocks.  Returns
+    (starts, n) with n the packed length (a multiple of 64)."""
+    gap_blocks = [0] * len(lens) if gap_blocks is None else gap_blocks
+    starts, pos = [], 0
+    for l, gb in zip(lens, gap_blocks):
+        pos += gb * BLOCK
+        starts.append(pos)
+        pos += ((l + BLOCK - 1) // BLOCK) * BLOCK
+    return starts, pos
+
+
+def make_varlen(w: Workload, starts, lens, pad: str = "zero"):
+    """(Q, K, V) [1, H, w.n, d] for a packed layout: w's recipe over the whole
+    buffer, then every token outside the sequences set by `pad`: "zero",
+    "nan", or "noise" (fresh N(0, 1) draws from seed + 200)."""
+    assert w.B == 1
+    Q, K, V = (t.float() for t in make_qkv(Workload(w.name, 1, w.Hq, w.Hkv, w.n, w.d, w.h, "fp32",
+                                                     w.structure, w.seed)))
+    inside = torch.zeros(w.n, dtype=torch.bool)
+    for a, l in zip(starts, lens):
+        inside[a:a + l] = True
+    out = []
+    g = torch.Generator("cpu").manual_seed(w.seed + 200)
+    for t in (Q, K, V):
+        t = t.clone()
+        if pad == "zero":
+            t[:, :, ~inside] = 0.0
+        elif pad == "nan":
+            t[:, :, ~inside] = float("nan")
+        elif pad == "noise":
+            t[:, :, ~inside] = torch.randn(t.shape[0], t.shape[1], int((~inside).sum()), t.shape[3], generator=g)
+        else:
+            raise ValueError(pad)
+        out.append(t.to(torch.bfloat16) if w.dtype == "bf16" else t)
+    return tuple(o.contiguous() for o in out)

@@ -54,9 +54,9 @@ def _load():
         lib.orc_project.argtypes = [P, P, I, I, I, I, I, P]
         lib.orc_block_rope.argtypes = [P, I, I, I, D, I]
         lib.orc_gate_scores.argtypes = [P, P, I, I, I, I, I, D, P]
-        lib.orc_select_threshold.argtypes = [P, I, I, F, P, P, I, P]
+        lib.orc_select_threshold.argtypes = [P, I, I, F, P, P, I, P, ctypes.c_int]
         lib.orc_select_threshold.restype = I
-        lib.orc_select_topk.argtypes = [P, I, I, ctypes.c_int, I, F, P, P, I, P]
+        lib.orc_select_topk.argtypes = [P, I, I, ctypes.c_int, I, F, P, P, I, P, ctypes.c_int]
         lib.orc_gate_scores_units.argtypes = [P, P, I, I, I, I, I, D, P, I, P]
         lib.orc_select_topk.restype = I
         lib.orc_topk_count.argtypes = [I, ctypes.c_int, I, F]
@@ -175,11 +175,13 @@ MODE_THRESHOLD, MODE_TOPK_K, MODE_TOPK_DENSITY = 0, 1, 2
 
 
 def select(scores, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
-           cap: int | None = None):
+           cap: int | None = None, force_diag: bool = False):
     """Binary block mask as ascending index lists (summary page, section 3.4,
-    "Generating the binary block mask"; rebuttal section 3.3).
-    Returns (counts [B,Hq,nb] int32, idx [B,Hq,nb,cap] int32 padded with -1,
-    worst) where worst is the largest per-row count before truncation."""
+    "Generating the binary block mask"; rebuttal section 3.3).  With
+    force_diag the diagonal block joins every row's list (an option the
+    pages do not use).  Returns (counts [B,Hq,nb] int32, idx [B,Hq,nb,cap]
+    int32 padded with -1, worst) where worst is the largest per-row count
+    before truncation."""
     s = _f64(scores)
     B, Hq, nb, _ = s.shape
     cap = nb if cap is None else cap
@@ -187,16 +189,17 @@ def select(scores, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
     counts = np.zeros((B, Hq, nb), np.int32)
     idx = np.full((B, Hq, nb, cap), -1, np.int32)
     lib = _load()
+    fd = 1 if force_diag else 0
     if mode == MODE_THRESHOLD:
-        worst = lib.orc_select_threshold(_p(s), rows, nb, float(T), _p(counts), _p(idx), cap, None)
+        worst = lib.orc_select_threshold(_p(s), rows, nb, float(T), _p(counts), _p(idx), cap, None, fd)
     else:
         worst = lib.orc_select_topk(_p(s), rows, nb, int(mode), int(k), float(density),
-                                    _p(counts), _p(idx), cap, None)
+                                    _p(counts), _p(idx), cap, None, fd)
     return counts, idx, int(worst)
 
 
 def select_rows(rows_scores, row_i, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
-                cap: int | None = None):
+                cap: int | None = None, force_diag: bool = False):
     """As select, for a stack of score rows [R, nb] whose query blocks are
     given by row_i [R].  Returns (counts [R], idx [R, cap])."""
     s = _f64(rows_scores)
@@ -206,11 +209,12 @@ def select_rows(rows_scores, row_i, mode: int, T: float = 0.0, k: int = 0, densi
     counts = np.zeros(R, np.int32)
     idx = np.full((R, cap), -1, np.int32)
     lib = _load()
+    fd = 1 if force_diag else 0
     if mode == MODE_THRESHOLD:
-        lib.orc_select_threshold(_p(s), R, nb, float(T), _p(counts), _p(idx), cap, _p(ri))
+        lib.orc_select_threshold(_p(s), R, nb, float(T), _p(counts), _p(idx), cap, _p(ri), fd)
     else:
         lib.orc_select_topk(_p(s), R, nb, int(mode), int(k), float(density), _p(counts), _p(idx),
-                            cap, _p(ri))
+                            cap, _p(ri), fd)
     return counts, idx
 
 
@@ -449,3 +453,94 @@ def decode_blockmax(q, K, n: int, scale: float | None = None):
                 gt[b, hq, j] = p[j * BLOCK:min((j + 1) * BLOCK, n)].max()
             lse[b, hq] = m + math.log(l)
     return gt, lse
+
+
+# ------------------------------------------------------- varlen packing ---
+# Rebuttal (batching): variable-length prefill inputs are packed along the
+# sequence axis.  Reading: sequence s occupies tokens start[s] .. start[s] +
+# len[s] - 1 of the packed buffer, start[s] a multiple of 64, so every block
+# belongs to one sequence.  Each sequence is then its own prefill problem; the
+# functions below run the plain definitions on each sequence alone (local
+# positions) and place the results at the sequence's blocks.
+def _seq_blocks(a: int, l: int):
+    return a // BLOCK, (l + BLOCK - 1) // BLOCK
+
+
+def pool_varlen(X, a: int, l: int, is_k: bool) -> np.ndarray:
+    """Pooling over the blocks of one packed sequence; its last block pools
+    only the sequence's own tokens.  Q: mean; K: [max | min | mean]."""
+    x = _f64(X)[:, :, a:a + l]
+    f, nbs = _seq_blocks(a, l)
+    outs = []
+    for b in range(nbs):
+        blk = x[:, :, BLOCK * b:min(BLOCK * (b + 1), l)]
+        if is_k:
+            outs.append(np.concatenate([blk.max(axis=2), blk.min(axis=2), blk.mean(axis=2)], axis=-1))
+        else:
+            outs.append(blk.mean(axis=2))
+    return np.stack(outs, axis=2)
+
+
+def gate_varlen(Q, K, Wq, Wk, starts, lens, rope_theta: float = 0.0) -> np.ndarray:
+    """The AttnGate per packed sequence: scores [1, Hq, nb, nb] with row i's
+    Eq. 1 softmax over its own sequence's blocks f .. i; 0 elsewhere (rows
+    of no sequence are all 0)."""
+    d = Q.shape[-1]
+    nb = Q.shape[2] // BLOCK
+    out = np.zeros((1, Q.shape[1], nb, nb), np.float64)
+    for a, l in zip(starts, lens):
+        f, nbs = _seq_blocks(int(a), int(l))
+        qt = project(pool_varlen(Q, int(a), int(l), False), Wq)
+        kt = project(pool_varlen(K, int(a), int(l), True), Wk)
+        if rope_theta > 0:
+            qt = block_rope(qt, rope_theta)
+            kt = block_rope(kt, rope_theta)
+        out[:, :, f:f + nbs, f:f + nbs] = gate_scores(qt, kt, d)
+    return out
+
+
+def select_varlen(scores, starts, lens, mode: int, T: float = 0.0, k: int = 0, density: float = 0.0,
+                  force_diag: bool = False, cap: int | None = None):
+    """Selection per packed sequence at local rows; lists hold global block
+    indices.  Returns (counts [1,Hq,nb], idx [1,Hq,nb,cap] padded with -1)."""
+    s = _f64(scores)
+    _, Hq, nb, _ = s.shape
+    cap = nb if cap is None else cap
+    counts = np.zeros((1, Hq, nb), np.int32)
+    idx = np.full((1, Hq, nb, cap), -1, np.int32)
+    for a, l in zip(starts, lens):
+        f, nbs = _seq_blocks(int(a), int(l))
+        c, ix, _ = select(np.ascontiguousarray(s[:, :, f:f + nbs, f:f + nbs]), mode, T=T, k=k, density=density,
+                          cap=cap, force_diag=force_diag)
+        counts[:, :, f:f + nbs] = c
+        idx[:, :, f:f + nbs] = np.where(ix >= 0, ix + f, -1)
+    return counts, idx
+
+
+def sparse_attn_varlen(Q, K, V, counts, idx, starts, lens, scale: float | None = None):
+    """Block-sparse attention per packed sequence, each on its own tokens
+    (the keys of its listed blocks, causal, none past the sequence's end).
+    Returns (O [1,Hq,n,d], lse [1,Hq,n]) fp64; positions of no sequence are
+    NaN (not defined)."""
+    q, k, v = _f64(Q), _f64(K), _f64(V)
+    _, Hq, n, d = q.shape
+    O = np.full((1, Hq, n, d), np.nan)
+    lse = np.full((1, Hq, n), np.nan)
+    cn = np.asarray(counts)
+    ix = np.asarray(idx)
+    for a, l in zip(starts, lens):
+        a, l = int(a), int(l)
+        f, nbs = _seq_blocks(a, l)
+        # the sequence alone, its last block filled out with zeros: keys past
+        # its end come after every one of its queries, so the causal rule
+        # already leaves them out
+        pad = nbs * BLOCK - l
+        def seq(x):
+            t = x[:, :, a:a + l]
+            return np.concatenate([t, np.zeros((1, x.shape[1], pad, d))], axis=2) if pad else t
+        loc = np.where(ix[:, :, f:f + nbs] >= 0, ix[:, :, f:f + nbs] - f, -1).astype(np.int32)
+        o, ls = sparse_attn(seq(q), seq(k), seq(v), np.ascontiguousarray(cn[:, :, f:f + nbs]),
+                            np.ascontiguousarray(loc), scale)
+        O[:, :, a:a + l] = o[:, :, :l]
+        lse[:, :, a:a + l] = ls[:, :, :l]
+    return O, lse

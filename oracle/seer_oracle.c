@@ -203,7 +203,7 @@ void orc_gate_scores_units(const double *qt, const double *kt, i64 B, i64 Hq,
  * so that supplied fp32 scores are compared exactly as an fp32 kernel does. */
 i64 orc_select_threshold(const double *scores, i64 rows, i64 nb, float T,
                          int32_t *counts, int32_t *idx, i64 cap,
-                         const i64 *row_i)
+                         const i64 *row_i, int force_diag)
 {
     i64 worst = 0;
 #pragma omp parallel for schedule(static) reduction(max : worst)
@@ -211,7 +211,7 @@ i64 orc_select_threshold(const double *scores, i64 rows, i64 nb, float T,
         i64 i = row_i ? row_i[r] : r % nb, c = 0;
         const double *s = scores + r * nb;
         for (i64 j = 0; j <= i; ++j)
-            if (s[j] > (double)T) {
+            if (s[j] > (double)T || (force_diag && j == i)) {
                 if (c < cap) idx[r * cap + c] = (int32_t)j;
                 ++c;
             }
@@ -259,7 +259,7 @@ static int int_cmp(const void *pa, const void *pb)
  * returned in ascending j.                                                 */
 i64 orc_select_topk(const double *scores, i64 rows, i64 nb, int mode, i64 k,
                     float density, int32_t *counts, int32_t *idx, i64 cap,
-                    const i64 *row_i)
+                    const i64 *row_i, int force_diag)
 {
     i64 worst = 0;
 #pragma omp parallel reduction(max : worst)
@@ -273,10 +273,20 @@ i64 orc_select_topk(const double *scores, i64 rows, i64 nb, int mode, i64 k,
             qsort(buf, (size_t)(i + 1), sizeof(cand_t), cand_cmp);
             i64 ki = orc_topk_count(i, mode, k, density);
             i64 c = ki < cap ? ki : cap;
-            for (i64 m = 0; m < c; ++m) idx[r * cap + m] = (int32_t)buf[m].j;
+            int has_diag = 0;
+            for (i64 m = 0; m < c; ++m) {
+                idx[r * cap + m] = (int32_t)buf[m].j;
+                if (buf[m].j == i) has_diag = 1;
+            }
+            /* the optional forced diagonal joins the list when not chosen */
+            i64 need = ki;
+            if (force_diag && !has_diag) {
+                need = ki + 1;
+                if (c < cap) idx[r * cap + c++] = (int32_t)i;
+            }
             qsort(idx + r * cap, (size_t)c, sizeof(int32_t), int_cmp);
             counts[r] = (int32_t)c;
-            if (ki > worst) worst = ki;
+            if (need > worst) worst = need;
         }
         free(buf);
     }

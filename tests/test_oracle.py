@@ -658,3 +658,105 @@ def test_decode_gate_is_softmax_over_compressed_cache():
         for h in range(Hq):
             top = np.argsort(-s[b, h], kind="stable")[:2]
             assert sorted(top.tolist()) == ix[b, h, :2].tolist()
+
+
+# ------------------------------------------------------- force diagonal ---
+def test_force_diagonal_threshold_keeps_only_diagonal_above_all_scores():
+    """T above every score: the forced lists are exactly [i]."""
+    w = synth.custom("fd", 1, 3, 1, 64 * 10, 32, 8, "fp32")
+    s = synth.make_scores_like(w, seed=31)
+    cnt, idx, _ = oracle.select(s, oracle.MODE_THRESHOLD, T=2.0, force_diag=True)
+    assert np.all(cnt == 1)
+    assert np.array_equal(idx[..., 0], np.broadcast_to(np.arange(10), (1, 3, 10)))
+    cnt0, _, _ = oracle.select(s, oracle.MODE_THRESHOLD, T=2.0)
+    assert np.all(cnt0 == 0)
+
+
+@pytest.mark.parametrize("mode,kw", [(oracle.MODE_THRESHOLD, dict(T=0.08)), (oracle.MODE_TOPK_K, dict(k=3)),
+                                     (oracle.MODE_TOPK_DENSITY, dict(density=0.3))])
+def test_force_diagonal_is_selection_plus_diagonal(mode, kw):
+    """Forced lists = the mode's own lists (an independent call) with i
+    added where it was missing; the worst count follows."""
+    w = synth.custom("fd", 2, 2, 1, 64 * 12, 32, 8, "fp32")
+    s = synth.make_scores_like(w, seed=32, ties=True)
+    c0, i0, _ = oracle.select(s, mode, **kw)
+    c1, i1, worst = oracle.select(s, mode, force_diag=True, **kw)
+    for r in np.ndindex(c0.shape):
+        base = set(i0[r][:c0[r]].tolist())
+        forced = i1[r][:c1[r]].tolist()
+        assert forced == sorted(base | {r[-1]})
+    assert worst == int(c1.max())
+
+
+# -------------------------------------------------------- varlen packing ---
+def test_varlen_single_full_sequence_is_the_plain_gate():
+    Q, K = _rand((1, 4, 64 * 7, 16), 71), _rand((1, 2, 64 * 7, 16), 72)
+    Wq, Wk = _rand((4, 8, 16), 73, 0.3), _rand((2, 8, 48), 74, 0.3)
+    ref = oracle.gate(Q, K, Wq, Wk)
+    got = oracle.gate_varlen(Q, K, Wq, Wk, [0], [64 * 7])
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-13)
+
+
+def test_varlen_partial_block_pooling_is_ceil_mode_pooling():
+    """A sequence of 150 tokens: the last block pools its 22 tokens only,
+    as avg/max pooling with ceil_mode on the unpadded sequence does."""
+    X = _rand((1, 2, 64 * 5, 8), 75)
+    a, l = 128, 150
+    x = X[:, :, a:a + l].double().reshape(2, l, 8).transpose(1, 2)
+    av = F.avg_pool1d(x, BLK, BLK, ceil_mode=True).transpose(1, 2).reshape(1, 2, 3, 8).numpy()
+    mx = F.max_pool1d(x, BLK, BLK, ceil_mode=True).transpose(1, 2).reshape(1, 2, 3, 8).numpy()
+    mn = -F.max_pool1d(-x, BLK, BLK, ceil_mode=True).transpose(1, 2).reshape(1, 2, 3, 8).numpy()
+    np.testing.assert_allclose(oracle.pool_varlen(X, a, l, False), av, rtol=0, atol=1e-14)
+    kp = oracle.pool_varlen(X, a, l, True)
+    np.testing.assert_array_equal(kp[..., :8], mx)
+    np.testing.assert_array_equal(kp[..., 8:16], mn)
+    np.testing.assert_allclose(kp[..., 16:], av, rtol=0, atol=1e-14)
+
+
+def test_varlen_packed_sequence_equals_the_gate_on_it_alone():
+    """Two sequences with a gap: the second one's block of the packed scores
+    equals the plain gate run on that sequence cut out of the buffer, and
+    nothing crosses between sequences."""
+    starts, n = synth.varlen_layout([200, 256], [0, 1])
+    Q, K = _rand((1, 4, n, 16), 76), _rand((1, 2, n, 16), 77)
+    Wq, Wk = _rand((4, 8, 16), 78, 0.3), _rand((2, 8, 48), 79, 0.3)
+    s = oracle.gate_varlen(Q, K, Wq, Wk, starts, [200, 256])
+    a = starts[1]
+    alone = oracle.gate(Q[:, :, a:a + 256].contiguous(), K[:, :, a:a + 256].contiguous(), Wq, Wk)
+    f = a // BLK
+    np.testing.assert_allclose(s[:, :, f:f + 4, f:f + 4], alone, rtol=0, atol=1e-13)
+    assert np.all(s[:, :, f:, :f] == 0) and np.all(s[:, :, :f, f:] == 0)
+    assert np.all(s[:, :, 4, :] == 0)  # the gap block
+    # the first sequence's rows sum to one over its own blocks
+    np.testing.assert_allclose(s[:, :, :4, :4].sum(-1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_varlen_rope_depends_on_block_distance_only():
+    """Block RoPE scores at packed (global) positions equal those at the
+    sequence's own positions: the rotation leaves q~_i . k~_j a function of
+    i - j.  (The CUDA gate rotates at global positions.)"""
+    h = 8
+    q = _rand((1, 1, 12, h), 80)
+    k = _rand((1, 1, 12, h), 81)
+    g_q, g_k = oracle.block_rope(q, 5000.0), oracle.block_rope(k, 5000.0)
+    l_q, l_k = oracle.block_rope(q[:, :, 5:].contiguous(), 5000.0), oracle.block_rope(k[:, :, 5:].contiguous(), 5000.0)
+    np.testing.assert_allclose(g_q[0, 0, 5:] @ g_k[0, 0, 5:].T, l_q[0, 0] @ l_k[0, 0].T, rtol=0, atol=1e-12)
+
+
+def test_varlen_attention_is_causal_sdpa_per_sequence():
+    """Every block listed: each packed sequence (lengths 150 and 64, a gap
+    between them) gets causal attention over its own tokens only."""
+    lens = [150, 64]
+    starts, n = synth.varlen_layout(lens, [0, 1])
+    Q, K, V = _attn_case(n=n, d=16, seed=82)
+    nb = n // BLK
+    s = np.zeros((1, 4, nb, nb))
+    for a, l in zip(starts, lens):
+        f, nbs = a // BLK, (l + BLK - 1) // BLK
+        s[:, :, f:f + nbs, f:f + nbs] = np.tril(np.ones((nbs, nbs)))
+    cnt, idx = oracle.select_varlen(s, starts, lens, oracle.MODE_THRESHOLD, T=0.5)
+    O, lse = oracle.sparse_attn_varlen(Q, K, V, cnt, idx, starts, lens)
+    for a, l in zip(starts, lens):
+        ref = _sdpa(Q[:, :, a:a + l], K[:, :, a:a + l], V[:, :, a:a + l], causal=True).numpy()
+        np.testing.assert_allclose(O[:, :, a:a + l], ref, rtol=0, atol=1e-12)
+    assert np.isnan(O[:, :, 150:192]).all()  # padding and gap are not defined
