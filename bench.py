@@ -38,6 +38,8 @@ WORKLOAD = "layer128k"
 DENSITY = 0.1
 BMAX_WORKLOAD = "bmax32k"
 DECODE_WORKLOAD = "decode128k"
+# packed variable-length prefill: sequence lengths inside the 128k layer buffer
+VARLEN_LENS = [61477, 30000, 16384, 9000, 8191, 4000, 1500, 129]
 
 
 def parse():
@@ -50,6 +52,7 @@ def parse():
     ap.add_argument("--density", type=float, default=DENSITY)
     ap.add_argument("--no-blockmax", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time the 50-95%% sparsity sweep")
@@ -311,6 +314,57 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def varlen_bench(seer, synth, dev, stream, w, Qd, Kd, Vd, Wqd, Wkd, density, pk):
+    """Packed variable-length prefill on the 128k layer's buffers: the
+    sequences of VARLEN_LENS placed at 64-token boundaries, gate (top-k
+    density) and sparse attention on the packed tensors.  Tokens outside the
+    sequences keep the layer's finite values (the gate skips them, attention
+    masks them).  FLOPs as attn_flops (a sequence's last, partial block is
+    counted as a full tile)."""
+    import torch
+    starts, n = synth.varlen_layout(VARLEN_LENS)
+    assert n <= w.n
+    st = torch.tensor(starts, dtype=torch.int32, device=dev)
+    ln = torch.tensor(VARLEN_LENS, dtype=torch.int32, device=dev)
+    nb = w.nb
+    cap = seer.gate_required_cap(1, w.Hq, w.Hkv, w.n, w.d, "density", density=density)
+    counts = torch.empty(1, w.Hq, nb, dtype=torch.int32, device=dev)
+    idx = torch.empty(1, w.Hq, nb, cap, dtype=torch.int32, device=dev)
+    gws = torch.empty(seer.gate_varlen_workspace_size(w.Hq, w.Hkv, w.n, w.d, w.h), dtype=torch.uint8, device=dev)
+    aws = torch.empty(seer.sparse_attn_workspace_size(1, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Qd)
+    lse = torch.empty(1, w.Hq, w.n, dtype=torch.float32, device=dev)
+
+    def gate():
+        seer.seer_gate_varlen(Qd, Kd, Wqd, Wkd, st, ln, "density", density=density, cap=cap, workspace=gws,
+                              out=(counts, idx, None))
+
+    def attn():
+        seer.seer_sparse_attn(Qd, Kd, Vd, counts, idx, workspace=aws, out=(O, lse))
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    gms = timed(gate)
+    ams = timed(attn)
+    flops, nblk, _, _ = attn_flops(counts, idx, w.d)
+    causal = sum(((l + 63) // 64) * ((l + 63) // 64 + 1) // 2 for l in VARLEN_LENS) * w.Hq
+    return {"workload": f"{len(VARLEN_LENS)} sequences {VARLEN_LENS} packed at 64-token boundaries into the "
+                        f"{w.name} buffers (Hq={w.Hq} Hkv={w.Hkv} d={w.d}), top-k density {density}",
+            "gate_ms": gms, "attn_ms": ams, "attn_tflops": flops / (ams * 1e-3) / 1e12,
+            "active_blocks": nblk, "achieved_sparsity": 1.0 - nblk / causal,
+            "gate_status": seer.seer_workspace_status(gws), "attn_status": seer.seer_workspace_status(aws)}
 
 
 def decode_bench(seer, synth, dev, stream, density, pk):
@@ -603,6 +657,11 @@ def main():
     if not args.no_decode and rank == 0:
         dec = decode_bench(seer, synth, dev, stream, args.density, pk)
 
+    # ------------------------------------------------------- varlen packing --
+    vl = None
+    if not args.no_varlen and rank == 0:
+        vl = varlen_bench(seer, synth, dev, stream, w, Qd, Kd, Vd, Wqd, Wkd, args.density, pk)
+
     # ------------------------------------------------------ density sweep ----
     sweep = None
     if args.sweep and rank == 0:
@@ -676,7 +735,7 @@ def main():
                          "algorithmic_flops_per_launch": flops},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 7 * args.steps,
-            "blockmax": bmax, "decode": dec, "sweep": sweep,
+            "blockmax": bmax, "decode": dec, "varlen": vl, "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -235,6 +235,23 @@ SEER_API seer_status seer_sparse_attn(const seer_dims *dims, const void *Q, cons
 
 SEER_API size_t seer_sparse_attn_workspace_size(const seer_dims *dims, seer_dtype dtype);
 
+/* seer_sparse_attn_tf32 -- seer_sparse_attn for fp32 Q/K/V/O on the tf32
+ * tensor cores: the operands are read as fp32 (the tensor core uses their
+ * top 19 bits, tf32) instead of being rounded to bf16 first, and P enters
+ * the PV product as fp32 (tf32) too.  About 8x smaller rounding error than
+ * the bf16 path, at half its tensor-core rate.  Same lists, scale, layouts
+ * and outputs as seer_sparse_attn; O and lse are fp32.
+ *   ws/ws_bytes  workspace of at least seer_sparse_attn_tf32_workspace_size
+ *               (the status word and V transposed per 64-key block)
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA.                                                    */
+SEER_API seer_status seer_sparse_attn_tf32(const seer_dims *dims, const float *Q, const float *K,
+                                          const float *V, const int32_t *counts, const int32_t *indices,
+                                          int32_t cap, float scale, float *O, float *lse, void *ws,
+                                          size_t ws_bytes, seer_stream_t stream);
+
+SEER_API size_t seer_sparse_attn_tf32_workspace_size(const seer_dims *dims);
+
 /* ------------------------------------------------------------------------ */
 /* seer_attn_blockmax -- the ground truth of the gate's self-distillation
  * (summary page, section 3.4, "Ground truth generation" and "The customized

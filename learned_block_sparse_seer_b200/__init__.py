@@ -5,7 +5,7 @@ thin Python binding plus the seeded synthetic-input recipe.
 """
 from ._lib import (  # noqa: F401
     SELECT_FORCE_DIAGONAL, SELECT_THRESHOLD, SELECT_TOPK_DENSITY, SELECT_TOPK_K, gate_varlen_workspace_size,
-    seer_gate_varlen, SeerError, attn_forward_map_workspace_size,
+    seer_gate_varlen, seer_sparse_attn_tf32, sparse_attn_tf32_workspace_size, SeerError, attn_forward_map_workspace_size,
     blockmax_workspace_size, seer_attn_forward_map,
     gate_kl_backward_workspace_size, gate_required_cap, gate_workspace_size, lib, seer_attn_blockmax, seer_gate,
     seer_gate_kl_backward, seer_gate_noalloc, seer_gate_select, seer_sparse_attn, seer_workspace_status,

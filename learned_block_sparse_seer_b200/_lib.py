@@ -100,6 +100,10 @@ def lib() -> ctypes.CDLL:
         L.seer_decode_blockmax_workspace_size.argtypes = [DP]
         L.seer_decode_blockmax_workspace_size.restype = SZ
         L.seer_decode_blockmax.restype = I32
+        L.seer_sparse_attn_tf32.argtypes = [DP, P, P, P, P, P, I32, F, P, P, P, SZ, P]
+        L.seer_sparse_attn_tf32.restype = I32
+        L.seer_sparse_attn_tf32_workspace_size.argtypes = [DP]
+        L.seer_sparse_attn_tf32_workspace_size.restype = SZ
         L.seer_workspace_status.argtypes = [P, P]
         L.seer_workspace_status.restype = I32
         L.seer_status_string.argtypes = [I32]
@@ -511,3 +515,31 @@ def seer_gate_varlen(Q, K, Wq, Wk, seq_start, seq_len, mode, T=0.0, k=0, density
                                 int(cap), _ptr(ws), ws.numel(), _stream(dev))
     _check("seer_gate_varlen", st)
     return (counts, indices, scores) if return_scores else (counts, indices)
+
+
+# -------------------------------------------------------------- tf32 attn --
+def sparse_attn_tf32_workspace_size(B, Hq, Hkv, n, d) -> int:
+    return int(lib().seer_sparse_attn_tf32_workspace_size(ctypes.byref(_dims(B, Hq, Hkv, n, d))))
+
+
+def seer_sparse_attn_tf32(Q, K, V, counts, indices, scale=0.0, workspace=None, out=None):
+    """Block-sparse attention for fp32 Q/K/V on the tf32 tensor cores:
+    (O [B,Hq,n,d] fp32, lse [B,Hq,n] fp32)."""
+    dev = _dev(Q, K, V, counts, indices)
+    for t in (Q, K, V):
+        if t.dtype != torch.float32:
+            raise TypeError("the tf32 path takes fp32 Q, K, V")
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        O = torch.empty_like(Q)
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=dev)
+    else:
+        O, lse = out
+    dims = _dims(B, Hq, Hkv, n, d)
+    ws = _workspace(sparse_attn_tf32_workspace_size(B, Hq, Hkv, n, d), dev, workspace)
+    st = lib().seer_sparse_attn_tf32(ctypes.byref(dims), _ptr(Q), _ptr(K), _ptr(V), _ptr(counts), _ptr(indices),
+                                     int(indices.shape[-1]), float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+                                     _stream(dev))
+    _check("seer_sparse_attn_tf32", st)
+    return O, lse

@@ -15,6 +15,7 @@
 #include "blockmax.cuh"
 #include "gate_train.cuh"
 #include "decode.cuh"
+#include "attn_tf32.cuh"
 #include "common.cuh"
 #include "gate.cuh"
 #include "ptx.cuh"
@@ -83,6 +84,20 @@ bool make_tmap(CUtensorMap* tm, const void* base, long long rows, int d, int box
   return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 map over [rows, d] with a 32 x 64 box (128 bytes by 64 rows),
+// 128-byte swizzle.
+bool make_tmap_f32(CUtensorMap* tm, const void* base, long long rows, int d, int box_rows = 64) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D bf16 map over [rows, 64] (128-byte rows) with a box of box_rows rows.
@@ -613,6 +628,53 @@ seer_status seer_attn_blockmax(const seer_dims* dims, const void* Q, const void*
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
   SEER_CUDA(seer::launch_blockmax(tmQ, tmK, p, w.ctas, st));
+  return SEER_OK;
+}
+
+// ----------------------------------------------------------- tf32 attn ---
+size_t seer_sparse_attn_tf32_workspace_size(const seer_dims* dims) {
+  if (!dims_ok(dims)) return 0;
+  seer::WsCarver c;  // V^T per key block
+  c.take(sizeof(float) * (size_t)dims->B * dims->Hkv * dims->n * dims->d);
+  return c.off;
+}
+
+seer_status seer_sparse_attn_tf32(const seer_dims* dims, const float* Q, const float* K, const float* V,
+                                  const int32_t* counts, const int32_t* indices, int32_t cap, float scale, float* O,
+                                  float* lse, void* ws, size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !V || !O || !counts || !indices) return SEER_ERR_INVALID_ARG;
+  if (cap < 1 || !(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return SEER_ERR_INVALID_ARG;
+  if ((long long)dims->B * dims->Hq * (dims->n / seer::kBlock) >= (1LL << 31)) return SEER_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, seer_sparse_attn_tf32_workspace_size(dims), st);
+  if (s != SEER_OK) return s;
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  float* Vt = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_tmap_f32(&tmQ, Q, (long long)B * Hq * n, d) || !make_tmap_f32(&tmK, K, (long long)B * Hkv * n, d) ||
+      !make_tmap_f32(&tmV, Vt, (long long)B * Hkv * n * d / 64 * 1LL, 64, d))
+    return cuda_fail(cudaErrorInvalidValue);
+  SEER_CUDA(seer::launch_vt(V, Vt, (long long)B * Hkv, n, d, st));
+  seer::Tf32AttnParams p{};
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.d = d;
+  p.nb = n / seer::kBlock;
+  p.cap = cap;
+  p.total_units = (long long)B * Hq * p.nb;
+  p.counts = counts;
+  p.indices = indices;
+  p.O = O;
+  p.lse = lse;
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+  p.scale_log2 = (float)(sc * 1.4426950408889634);
+  p.status = &((seer::WsHeader*)ws)->status;
+  p.timeout_ns = kTimeoutNs;
+  SEER_CUDA(seer::launch_attn_tf32(tmQ, tmK, tmV, p, st));
   return SEER_OK;
 }
 

@@ -1,0 +1,388 @@
+// attn_tf32.cu -- block-sparse causal attention for fp32 Q/K/V on the tf32
+// tensor cores (tcgen05 kind::tf32), for callers who want fp32 I/O without
+// the bf16 rounding of the main kernel.
+//
+// Paper: "SeerAttention: Learning Intrinsic Sparse Attention in Your LLMs";
+// paper-graph summary page, section 3.4, "Block-sparse FlashAttention kernel":
+// for query block i only the listed key blocks take part, causal inside the
+// diagonal block, online softmax, O and the row log-sum-exp.
+//
+// Design (one CTA per unit = (batch, query head, 64-row query block)):
+//  * Operands come straight from the fp32 tensors by TMA (no re-layout, no
+//    conversion): 64-row boxes of 32 floats (128 bytes), 128-byte swizzle.
+//  * S = Q K^T per key block: tcgen05 kind::tf32, M = 64 query rows, N = 64
+//    keys, K = d (8 per instruction); A and B K-major.  With M = 64 the rows
+//    sit in TMEM lanes 0-15 of each 32-lane sub-partition (row r at lane
+//    r % 16 + 32 (r / 16)), so each softmax warp owns 16 rows.
+//  * O^T += V^T P^T per block: M = d (the d rows of O^T fill the TMEM lanes at
+//    d = 128), N = 64 query columns, K = 64 keys; A = V^T, B = P^T, both
+//    K-major: V is first transposed per 64-key block into the workspace
+//    (vt_kernel: d rows of 64 keys), and P^T is the P tile the softmax writes
+//    (fp32 values, read by the tensor core as tf32).  Every operand is
+//    K-major, the layout the QK product uses too.
+//  * Two S buffers in TMEM and two K/V stages: QK of block t+1 runs while the
+//    softmax works on block t.  The running row maximum is raised lazily (by
+//    more than 8 in log2 units), and only then is O^T rescaled in TMEM.
+//  * Warp roles (192 threads): warps 0-3 softmax and epilogue (TMEM
+//    sub-partitions 0-3), warp 4 TMA producer, warp 5 MMA issuer.  Every
+//    wait is bounded; the softmax warps meet at hardware barriers that all
+//    128 threads always reach, carrying any failure with them.
+#include <cmath>
+#include <cstdint>
+
+#include "attn_tf32.cuh"
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace seer {
+
+namespace tf32a {
+constexpr int kThreads = 192;
+constexpr int kWarpLoad = 4, kWarpMma = 5;
+constexpr uint32_t kPanel = 64u * 128u;  // 64 rows x 32 floats
+constexpr uint32_t kTmemCols = 256;      // S x 2 (64 cols each), O^T (64 cols)
+constexpr uint32_t kColO = 128;
+constexpr float kRaise = 8.0f;
+
+template <int D>
+struct Layout {
+  static constexpr int P = D / 32;                  // 32-float panels per row
+  static constexpr uint32_t kTile = P * kPanel;     // a 64-row tile of d floats
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = kTile;         // 2 stages x (K tile, V tile)
+  static constexpr uint32_t kOffP = kOffKV + 4 * kTile;
+  static constexpr uint32_t kSmem = kOffP + 2 * kPanel;
+  static constexpr uint32_t kVtPanel = (uint32_t)D * 128u;  // V^T: d rows x 32 keys
+};
+
+struct Ctrl {
+  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, pv_done, fin;
+  uint32_t tmem_base;
+  int abort_flag;
+  float alpha[2][64], linv[64];  // alpha by step parity
+};
+
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::tf32: D f32, A and B tf32 (format 2).
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  uint32_t a[16], b[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    a[k] = r[k];
+    b[k] = r[16 + k];
+  }
+  tmem_st16(taddr, a);
+  tmem_st16(taddr + 16u, b);
+}
+
+// The list entry t of a unit, checked: an entry outside 0..i is recorded
+// and replaced by the diagonal block.
+__device__ __forceinline__ int entry(const Tf32AttnParams& p, long long unit, int i, int t) {
+  int j = p.indices[unit * p.cap + t];
+  if (j < 0 || j > i) {
+    record_status(p.status, kDevBadIndex, (uint32_t)unit);
+    j = i;
+  }
+  return j;
+}
+}  // namespace tf32a
+
+template <int D>
+__global__ void __launch_bounds__(tf32a::kThreads, 1)
+    attn_tf32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const Tf32AttnParams p) {
+  using namespace tf32a;
+  using L = Layout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) record_status(p.status, kDevBadSchedule, smem_u32(smem));
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long unit = blockIdx.x;  // (b * Hq + hq) * nb + i
+  const int i = (int)(unit % p.nb);
+  const long long bh = unit / p.nb;
+  const long long b = bh / p.Hq;
+  const int hq = (int)(bh % p.Hq), g = hq / (p.Hq / p.Hkv);
+  const long long qrow0 = bh * p.n + (long long)i * kBlock;
+  int cnt = p.counts[unit];
+  const int lim = min(p.cap, i + 1);
+  if (cnt < 0 || cnt > lim) {
+    if (threadIdx.x == 0) record_status(p.status, kDevBadIndex, (uint32_t)unit);
+    cnt = cnt < 0 ? 0 : lim;
+  }
+  Ctrl& C = *reinterpret_cast<Ctrl*>(smem + L::kSmem);
+  float* O = p.O;
+  if (cnt == 0) {  // no admissible key: O = 0, LSE = -inf
+    for (int x = threadIdx.x; x < kBlock * D; x += kThreads) O[qrow0 * D + x] = 0.f;
+    if (p.lse)
+      for (int x = threadIdx.x; x < kBlock; x += kThreads) p.lse[qrow0 + x] = -INFINITY;
+    return;
+  }
+  volatile int* abort_p = &C.abort_flag;
+  const uint64_t tmo = p.timeout_ns;
+  if (threadIdx.x == 0) {
+    C.abort_flag = 0;
+    mbar_init(&C.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&C.kv_full[s], 1);
+      mbar_init(&C.kv_empty[s], 1);
+      mbar_init(&C.s_full[s], 1);
+      mbar_init(&C.s_free[s], 4);
+    }
+    mbar_init(&C.p_full, 4);
+    mbar_init(&C.pv_done, 1);
+    mbar_init(&C.fin, 1);
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&C.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = C.tmem_base;
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------- producer ---
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(&C.q_full, L::kTile);
+      for (int pn = 0; pn < L::P; ++pn)
+        tma_load_2d(smem + L::kOffQ + pn * kPanel, &tmQ, &C.q_full, pn * 32, (int)qrow0);
+      const long long krow0 = (b * p.Hkv + g) * p.n;
+      int t = 0;
+      for (; t < cnt; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !mbar_wait(&C.kv_empty[s], ((t >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+        const int j = tf32a::entry(p, unit, i, t);
+        const int row = (int)(krow0 + (long long)j * kBlock);
+        // V^T block of this key block: d rows of 64 keys in the workspace
+        const int vrow = (int)(((b * p.Hkv + g) * p.nb + j) * (long long)D);
+        uint8_t* kt = smem + L::kOffKV + (uint32_t)s * 2 * L::kTile;
+        mbar_arrive_expect_tx(&C.kv_full[s], 2 * L::kTile);
+        for (int pn = 0; pn < L::P; ++pn) tma_load_2d(kt + pn * kPanel, &tmK, &C.kv_full[s], pn * 32, row);
+        for (int pn = 0; pn < 2; ++pn)
+          tma_load_2d(kt + L::kTile + pn * L::kVtPanel, &tmV, &C.kv_full[s], pn * 32, vrow);
+      }
+      // copies in flight land before the CTA exits
+      mbar_wait(&C.q_full, 0, abort_p, nullptr, 20000000ull);
+      for (int k = t > 2 ? t - 2 : 0; k < t; ++k)
+        mbar_wait(&C.kv_full[k & 1], (k >> 1) & 1, abort_p, nullptr, 20000000ull);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------ MMA issuer ---
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_tf32(64, 64, 0, 0);  // A = Q, B = K (both K-major)
+      constexpr uint32_t idesc_pv = make_idesc_tf32(D, 64, 0, 0);   // A = V^T, B = P^T (both K-major)
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t dQ = make_sw128_desc(sbase + L::kOffQ, 16, 1024);
+      const uint64_t dP = make_sw128_desc(sbase + L::kOffP, 16, 1024);
+      bool ok = mbar_wait(&C.q_full, 0, abort_p, p.status, tmo);
+      for (int t = 0; ok && t <= cnt; ++t) {
+        if (t < cnt) {
+          const int s = t & 1;
+          if (!mbar_wait(&C.kv_full[s], (t >> 1) & 1, abort_p, p.status, tmo)) break;
+          if (t >= 2 && !mbar_wait(&C.s_free[s], ((t >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+          tc_fence_after();
+          const uint64_t dK = make_sw128_desc(sbase + L::kOffKV + (uint32_t)s * 2 * L::kTile, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 8; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
+            mma_tf32_ss(tmem + (uint32_t)s * 64u, dQ + off, dK + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&C.s_full[s]);
+        }
+        if (t >= 1) {  // PV of block t - 1
+          const int u = t - 1, s = u & 1;
+          if (!mbar_wait(&C.p_full, u & 1, abort_p, p.status, tmo)) break;
+          tc_fence_after();
+          // V^T, K-major: d rows of 32 keys per panel, two panels
+          const uint64_t dV = make_sw128_desc(sbase + L::kOffKV + (uint32_t)s * 2 * L::kTile + L::kTile, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_tf32_ss(tmem + kColO, dV + (uint64_t)(((kk >> 2) * L::kVtPanel + (kk & 3) * 32) >> 4),
+                        dP + (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_pv,
+                        (u > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&C.pv_done);
+          mma_commit(&C.kv_empty[s]);
+        }
+      }
+      mma_commit(&C.fin);
+      mbar_wait(&C.fin, 0, abort_p, nullptr, 20000000ull);
+    }
+  } else {
+    // ------------------------------------------- softmax and epilogue ---
+    // Warp ww owns query rows 16 ww .. 16 ww + 15 (lanes 0-15 of its TMEM
+    // sub-partition) and, for O^T, the d rows of its sub-partition's lanes.
+    const int ww = warp;
+    const bool row_thread = lane < 16;
+    const int q = 16 * ww + (lane & 15);
+    const uint32_t lane_base = tmem + ((uint32_t)(ww * 32) << 16);
+    const float c = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < cnt; ++t) {
+      const int s = t & 1;
+      const int j = tf32a::entry(p, unit, i, t);
+      ok = ok && mbar_wait(&C.s_full[s], (t >> 1) & 1, abort_p, p.status, tmo);
+      uint32_t r0[32], r1[32];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(lane_base + (uint32_t)s * 64u, r0);
+        tmem_ld32(lane_base + (uint32_t)s * 64u + 32u, r1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&C.s_free[s]);
+      float x[64];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        x[k] = __uint_as_float(r0[k]) * c;
+        x[32 + k] = __uint_as_float(r1[k]) * c;
+      }
+      if (j == i) {  // causal rule inside the diagonal block
+#pragma unroll
+        for (int k = 0; k < 64; ++k) x[k] = k > q ? -INFINITY : x[k];
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int k = 1; k < 64; ++k) mx = fmaxf(mx, x[k]);
+      float alpha = 1.f;
+      bool raise = false;
+      if (mx > m + kRaise) {
+        if (t > 0) {
+          alpha = exp2f(m - mx);
+          raise = true;
+        }
+        l *= alpha;
+        m = mx;
+      }
+      float ps = 0.f;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        x[k] = exp2f(x[k] - m);
+        ps += x[k];
+      }
+      l += ps;
+      // P(t) overwrites P(t-1) and O^T may be rescaled: PV(t-1) must be done
+      if (t >= 1) ok = ok && mbar_wait(&C.pv_done, (t - 1) & 1, abort_p, p.status, tmo);
+      if (row_thread) C.alpha[t & 1][q] = alpha;
+      // every softmax thread reaches this barrier; a failure anywhere ends
+      // the loop for all of them together
+      const bool any_raise = bar_red_or(1, 128, row_thread && raise);
+      ok = !bar_red_or(2, 128, !ok);
+      if (!ok) break;
+      if (any_raise) {
+        tc_fence_after();
+        uint32_t o0[32], o1[32];
+        tmem_ld32(lane_base + kColO, o0);
+        tmem_ld32(lane_base + kColO + 32u, o1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          o0[k] = __float_as_uint(__uint_as_float(o0[k]) * C.alpha[t & 1][k]);
+          o1[k] = __float_as_uint(__uint_as_float(o1[k]) * C.alpha[t & 1][32 + k]);
+        }
+        tmem_st32(lane_base + kColO, o0);
+        tmem_st32(lane_base + kColO + 32u, o1);
+        tmem_wait_st();
+      }
+      if (row_thread) {
+        // P[q][0..63] as fp32 into the two 32-key panels, 128-byte swizzle
+        uint8_t* prow = smem + L::kOffP + (uint32_t)q * 128u;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int pn = cc >> 3, ch = cc & 7;
+          float4 v = make_float4(x[4 * cc], x[4 * cc + 1], x[4 * cc + 2], x[4 * cc + 3]);
+          *reinterpret_cast<float4*>(prow + pn * kPanel + ((ch ^ (q & 7)) << 4)) = v;
+        }
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&C.p_full);
+    }
+    // ---- epilogue: O = O^T columns / l, LSE
+    if (ok) ok = mbar_wait(&C.pv_done, (cnt - 1) & 1, abort_p, p.status, tmo);
+    if (row_thread) {
+      C.linv[q] = 1.0f / l;
+      if (p.lse) p.lse[qrow0 + q] = (m + log2f(l)) * 0.6931471805599453f;
+    }
+    ok = !bar_red_or(2, 128, !ok);
+    if (ok) {
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      tmem_ld32(lane_base + kColO, o0);
+      tmem_ld32(lane_base + kColO + 32u, o1);
+      tmem_wait_ld();
+      // O^T lane -> d: all 128 lanes at d = 128; lanes 0-15 of each
+      // sub-partition (d = 16 ww + lane) at d = 64
+      const bool d_thread = D == 128 || lane < 16;
+      const int dd = D == 128 ? ww * 32 + lane : 16 * ww + (lane & 15);
+      if (d_thread) {
+        float* out = O + qrow0 * D + dd;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          out[(long long)k * D] = __uint_as_float(o0[k]) * C.linv[k];
+          out[(long long)(32 + k) * D] = __uint_as_float(o1[k]) * C.linv[32 + k];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+}
+
+// V^T per 64-key block: Vt[(bh * nb + j) * d + c][k] = V[bh][64 j + k][c].
+__global__ void __launch_bounds__(256) vt_kernel(const float* __restrict__ V, float* __restrict__ Vt, int n, int d) {
+  __shared__ float tile[64][129];
+  const long long blk = blockIdx.x;  // bh * nb + j
+  const int nb = n / kBlock;
+  const long long bh = blk / nb;
+  const int j = (int)(blk % nb);
+  const float* src = V + (bh * n + (long long)j * kBlock) * d;
+  for (int x = threadIdx.x; x < kBlock * d; x += 256) tile[x / d][x % d] = src[x];
+  __syncthreads();
+  float* dst = Vt + blk * (long long)d * kBlock;
+  for (int x = threadIdx.x; x < kBlock * d; x += 256) dst[x] = tile[x % kBlock][x / kBlock];
+}
+
+cudaError_t launch_vt(const float* V, float* Vt, long long BHkv, int n, int d, cudaStream_t st) {
+  vt_kernel<<<(unsigned)(BHkv * (n / kBlock)), 256, 0, st>>>(V, Vt, n, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tf32(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                             const Tf32AttnParams& p, cudaStream_t st) {
+  auto kern = p.d == 64 ? attn_tf32_kernel<64> : attn_tf32_kernel<128>;
+  const uint32_t smem =
+      (p.d == 64 ? tf32a::Layout<64>::kSmem : tf32a::Layout<128>::kSmem) + (uint32_t)sizeof(tf32a::Ctrl);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)p.total_units, tf32a::kThreads, smem, st>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace seer
