@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--no-blockmax", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-tf32", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time the 50-95%% sparsity sweep")
@@ -314,6 +315,38 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def tf32_bench(seer, dev, stream, w, Qd, Kd, Vd, counts, indices, flops, pk):
+    """The fp32 path on the tf32 tensor cores: the 128k layer's tensors held
+    in fp32 (the bf16 values, exact), the same density lists.  Peak: the
+    measured bf16 peaks times the nominal dense tf32 / bf16 ratio (1.1 / 2.25
+    PFLOP/s)."""
+    import torch
+    Qf, Kf, Vf = Qd.float(), Kd.float(), Vd.float()
+    ws = torch.empty(seer.sparse_attn_tf32_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Qf)
+    lse = torch.empty(w.B, w.Hq, w.n, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        seer.seer_sparse_attn_tf32(Qf, Kf, Vf, counts, indices, workspace=ws, out=(O, lse))
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    a.record(stream)
+    for _ in range(reps):
+        seer.seer_sparse_attn_tf32(Qf, Kf, Vf, counts, indices, workspace=ws, out=(O, lse))
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / reps
+    ratio = 1.1 / 2.25
+    tfl = flops / (ms * 1e-3) / 1e12
+    res = {"workload": f"{w.name} in fp32, same lists", "ms": ms, "tflops": tfl,
+           "peak_tf32_tflops": {"burst": pk["bf16_tflops"] * ratio,
+                                "sustained": pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * ratio},
+           "frac_of_tf32_peak": tfl / (pk["bf16_tflops"] * ratio),
+           "status": seer.seer_workspace_status(ws)}
+    del Qf, Kf, Vf, O, lse, ws
+    return res
 
 
 def varlen_bench(seer, synth, dev, stream, w, Qd, Kd, Vd, Wqd, Wkd, density, pk):
@@ -662,6 +695,11 @@ def main():
     if not args.no_varlen and rank == 0:
         vl = varlen_bench(seer, synth, dev, stream, w, Qd, Kd, Vd, Wqd, Wkd, args.density, pk)
 
+    # ------------------------------------------------------------ tf32 path --
+    tf = None
+    if not args.no_tf32 and rank == 0:
+        tf = tf32_bench(seer, dev, stream, w, Qd, Kd, Vd, counts, indices, flops, pk)
+
     # ------------------------------------------------------ density sweep ----
     sweep = None
     if args.sweep and rank == 0:
@@ -735,7 +773,7 @@ def main():
                          "algorithmic_flops_per_launch": flops},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 7 * args.steps,
-            "blockmax": bmax, "decode": dec, "varlen": vl, "sweep": sweep,
+            "blockmax": bmax, "decode": dec, "varlen": vl, "tf32": tf, "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
