@@ -100,6 +100,23 @@ bool make_tmap_f32(CUtensorMap* tm, const void* base, long long rows, int d, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map that reads a [rows, inner] tensor as panels: x = 32 floats
+// of a row (128 bytes), y = rows, z = the row's 32-float chunks (128 bytes
+// apart).  One box {32, box_rows, inner / 32} lands in shared memory as
+// inner/32 panels of box_rows x 128 bytes, 128-byte swizzled: a whole tile
+// per copy.
+bool make_tmap_f32_panels(CUtensorMap* tm, const void* base, long long rows, int inner, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(inner / 32)};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 4, 128};
+  cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)(inner / 32)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 map over [rows, 64] (128-byte rows) with a box of box_rows rows.
 bool make_tmap_rows(CUtensorMap* tm, const void* base, long long rows, int box_rows) {
   return make_tmap(tm, base, rows, 64, box_rows);
@@ -654,8 +671,9 @@ seer_status seer_sparse_attn_tf32(const seer_dims* dims, const float* Q, const f
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
   float* Vt = (float*)((uint8_t*)ws + sizeof(seer::WsHeader));
   CUtensorMap tmQ, tmK, tmV;
-  if (!make_tmap_f32(&tmQ, Q, (long long)B * Hq * n, d) || !make_tmap_f32(&tmK, K, (long long)B * Hkv * n, d) ||
-      !make_tmap_f32(&tmV, Vt, (long long)B * Hkv * n * d / 64 * 1LL, 64, d))
+  if (!make_tmap_f32_panels(&tmQ, Q, (long long)B * Hq * n, d, 64) ||
+      !make_tmap_f32_panels(&tmK, K, (long long)B * Hkv * n, d, 64) ||
+      !make_tmap_f32_panels(&tmV, Vt, (long long)B * Hkv * n * d / 64, 64, d))
     return cuda_fail(cudaErrorInvalidValue);
   SEER_CUDA(seer::launch_vt(V, Vt, (long long)B * Hkv, n, d, st));
   seer::Tf32AttnParams p{};

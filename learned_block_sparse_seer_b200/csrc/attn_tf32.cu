@@ -8,8 +8,10 @@
 // diagonal block, online softmax, O and the row log-sum-exp.
 //
 // Design (one CTA per unit = (batch, query head, 64-row query block)):
-//  * Operands come straight from the fp32 tensors by TMA (no re-layout, no
-//    conversion): 64-row boxes of 32 floats (128 bytes), 128-byte swizzle.
+//  * Operands come straight from the fp32 tensors by TMA (no conversion): a
+//    3-D tensor map reads a [rows, d] tensor as 32-float panels, so one copy
+//    brings a whole 64-row tile (d/32 panels of 64 rows x 128 bytes, 128-byte
+//    swizzle); copies of 8 KB or less cost about as much per copy as 32 KB.
 //  * S = Q K^T per key block: tcgen05 kind::tf32, M = 64 query rows, N = 64
 //    keys, K = d (8 per instruction); A and B K-major.  With M = 64 the rows
 //    sit in TMEM lanes 0-15 of each 32-lane sub-partition (row r at lane
@@ -20,11 +22,12 @@
 //    (vt_kernel: d rows of 64 keys), and P^T is the P tile the softmax writes
 //    (fp32 values, read by the tensor core as tf32).  Every operand is
 //    K-major, the layout the QK product uses too.
-//  * Two S buffers in TMEM and two K/V stages: QK of block t+1 runs while the
-//    softmax works on block t.  The running row maximum is raised lazily (by
+//  * Two S buffers in TMEM, two P tiles: QK of block t+1 and PV of block t-1
+//    run while the softmax works on block t.  The running row maximum is raised lazily (by
 //    more than 8 in log2 units), and only then is O^T rescaled in TMEM.
-//  * Warp roles (192 threads): warps 0-3 softmax and epilogue (TMEM
-//    sub-partitions 0-3), warp 4 TMA producer, warp 5 MMA issuer.  Every
+//  * Warp roles (224 threads): warps 0-3 softmax and epilogue (TMEM
+//    sub-partitions 0-3), warp 4 loads Q and K (two K stages, freed by QK),
+//    warp 5 issues the MMAs, warp 6 loads V^T (three stages, freed by PV).  Every
 //    wait is bounded; the softmax warps meet at hardware barriers that all
 //    128 threads always reach, carrying any failure with them.
 #include <cmath>
@@ -37,8 +40,9 @@
 namespace seer {
 
 namespace tf32a {
-constexpr int kThreads = 192;
-constexpr int kWarpLoad = 4, kWarpMma = 5;
+constexpr int kThreads = 224;
+constexpr int kWarpLoad = 4, kWarpMma = 5, kWarpLoadV = 6;
+constexpr int kKS = 2, kVS = 3;  // K and V^T stages
 constexpr uint32_t kPanel = 64u * 128u;  // 64 rows x 32 floats
 constexpr uint32_t kTmemCols = 256;      // S x 2 (64 cols each), O^T (64 cols)
 constexpr uint32_t kColO = 128;
@@ -49,14 +53,16 @@ struct Layout {
   static constexpr int P = D / 32;                  // 32-float panels per row
   static constexpr uint32_t kTile = P * kPanel;     // a 64-row tile of d floats
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffKV = kTile;         // 2 stages x (K tile, V tile)
-  static constexpr uint32_t kOffP = kOffKV + 4 * kTile;
-  static constexpr uint32_t kSmem = kOffP + 2 * kPanel;
+  static constexpr uint32_t kOffK = kTile;                  // kKS K tiles
+  static constexpr uint32_t kOffV = kOffK + kKS * kTile;     // kVS V^T tiles
+  static constexpr uint32_t kOffP = kOffV + kVS * kTile;
+  static constexpr uint32_t kSmem = kOffP + 4 * kPanel;  // two P tiles
   static constexpr uint32_t kVtPanel = (uint32_t)D * 128u;  // V^T: d rows x 32 keys
 };
 
 struct Ctrl {
-  uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, pv_done, fin;
+  uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS], s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t fin;
   uint32_t tmem_base;
   int abort_flag;
   float alpha[2][64], linv[64];  // alpha by step parity
@@ -138,14 +144,22 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
   if (threadIdx.x == 0) {
     C.abort_flag = 0;
     mbar_init(&C.q_full, 1);
+    for (int s = 0; s < kKS; ++s) {
+      mbar_init(&C.k_full[s], 1);
+      mbar_init(&C.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(&C.v_full[s], 1);
+      mbar_init(&C.v_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&C.kv_full[s], 1);
-      mbar_init(&C.kv_empty[s], 1);
       mbar_init(&C.s_full[s], 1);
       mbar_init(&C.s_free[s], 4);
     }
-    mbar_init(&C.p_full, 4);
-    mbar_init(&C.pv_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&C.p_full[s], 4);
+      mbar_init(&C.pv_done[s], 1);
+    }
     mbar_init(&C.fin, 1);
     fence_barrier_init();
   }
@@ -159,33 +173,45 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
   const uint32_t tmem = C.tmem_base;
 
   if (warp == kWarpLoad) {
-    // ------------------------------------------------------- producer ---
+    // ----------------------------------------------- producer: Q, K ---
+    // K tiles free as soon as their QK is done, V^T tiles only after PV:
+    // separate rings and separate producers, so a V^T slot never holds up K.
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&C.q_full, L::kTile);
-      for (int pn = 0; pn < L::P; ++pn)
-        tma_load_2d(smem + L::kOffQ + pn * kPanel, &tmQ, &C.q_full, pn * 32, (int)qrow0);
+      tma_load_3d(smem + L::kOffQ, &tmQ, &C.q_full, 0, (int)qrow0, 0);
       const long long krow0 = (b * p.Hkv + g) * p.n;
       int t = 0;
       for (; t < cnt; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !mbar_wait(&C.kv_empty[s], ((t >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+        const int s = t % kKS;
+        if (t >= kKS && !mbar_wait(&C.k_empty[s], ((t / kKS) - 1) & 1, abort_p, p.status, tmo)) break;
         const int j = tf32a::entry(p, unit, i, t);
-        const int row = (int)(krow0 + (long long)j * kBlock);
-        // V^T block of this key block: d rows of 64 keys in the workspace
-        const int vrow = (int)(((b * p.Hkv + g) * p.nb + j) * (long long)D);
-        uint8_t* kt = smem + L::kOffKV + (uint32_t)s * 2 * L::kTile;
-        mbar_arrive_expect_tx(&C.kv_full[s], 2 * L::kTile);
-        for (int pn = 0; pn < L::P; ++pn) tma_load_2d(kt + pn * kPanel, &tmK, &C.kv_full[s], pn * 32, row);
-        for (int pn = 0; pn < 2; ++pn)
-          tma_load_2d(kt + L::kTile + pn * L::kVtPanel, &tmV, &C.kv_full[s], pn * 32, vrow);
+        mbar_arrive_expect_tx(&C.k_full[s], L::kTile);
+        tma_load_3d(smem + L::kOffK + (uint32_t)s * L::kTile, &tmK, &C.k_full[s], 0,
+                    (int)(krow0 + (long long)j * kBlock), 0);
       }
       // copies in flight land before the CTA exits
       mbar_wait(&C.q_full, 0, abort_p, nullptr, 20000000ull);
-      for (int k = t > 2 ? t - 2 : 0; k < t; ++k)
-        mbar_wait(&C.kv_full[k & 1], (k >> 1) & 1, abort_p, nullptr, 20000000ull);
+      for (int k = t > kKS ? t - kKS : 0; k < t; ++k)
+        mbar_wait(&C.k_full[k % kKS], (k / kKS) & 1, abort_p, nullptr, 20000000ull);
+    }
+  } else if (warp == kWarpLoadV) {
+    // --------------------------------------------------- producer: V^T ---
+    if (lane == 0) {
+      prefetch_tmap(&tmV);
+      int t = 0;
+      for (; t < cnt; ++t) {
+        const int s = t % kVS;
+        if (t >= kVS && !mbar_wait(&C.v_empty[s], ((t / kVS) - 1) & 1, abort_p, p.status, tmo)) break;
+        const int j = tf32a::entry(p, unit, i, t);
+        // V^T block of this key block: d rows of 64 keys in the workspace
+        mbar_arrive_expect_tx(&C.v_full[s], L::kTile);
+        tma_load_3d(smem + L::kOffV + (uint32_t)s * L::kTile, &tmV, &C.v_full[s], 0,
+                    (int)(((b * p.Hkv + g) * p.nb + j) * (long long)D), 0);
+      }
+      for (int k = t > kVS ? t - kVS : 0; k < t; ++k)
+        mbar_wait(&C.v_full[k % kVS], (k / kVS) & 1, abort_p, nullptr, 20000000ull);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------ MMA issuer ---
@@ -198,31 +224,33 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       bool ok = mbar_wait(&C.q_full, 0, abort_p, p.status, tmo);
       for (int t = 0; ok && t <= cnt; ++t) {
         if (t < cnt) {
-          const int s = t & 1;
-          if (!mbar_wait(&C.kv_full[s], (t >> 1) & 1, abort_p, p.status, tmo)) break;
+          const int s = t & 1, ks = t % kKS;
+          if (!mbar_wait(&C.k_full[ks], (t / kKS) & 1, abort_p, p.status, tmo)) break;
           if (t >= 2 && !mbar_wait(&C.s_free[s], ((t >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
           tc_fence_after();
-          const uint64_t dK = make_sw128_desc(sbase + L::kOffKV + (uint32_t)s * 2 * L::kTile, 16, 1024);
+          const uint64_t dK = make_sw128_desc(sbase + L::kOffK + (uint32_t)ks * L::kTile, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < D / 8; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
             mma_tf32_ss(tmem + (uint32_t)s * 64u, dQ + off, dK + off, idesc_qk, kk > 0 ? 1u : 0u);
           }
           mma_commit(&C.s_full[s]);
+          mma_commit(&C.k_empty[ks]);
         }
         if (t >= 1) {  // PV of block t - 1
-          const int u = t - 1, s = u & 1;
-          if (!mbar_wait(&C.p_full, u & 1, abort_p, p.status, tmo)) break;
+          const int u = t - 1, vs = u % kVS;
+          if (!mbar_wait(&C.v_full[vs], (u / kVS) & 1, abort_p, p.status, tmo)) break;
+          if (!mbar_wait(&C.p_full[u & 1], (u >> 1) & 1, abort_p, p.status, tmo)) break;
           tc_fence_after();
           // V^T, K-major: d rows of 32 keys per panel, two panels
-          const uint64_t dV = make_sw128_desc(sbase + L::kOffKV + (uint32_t)s * 2 * L::kTile + L::kTile, 16, 1024);
+          const uint64_t dV = make_sw128_desc(sbase + L::kOffV + (uint32_t)vs * L::kTile, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_tf32_ss(tmem + kColO, dV + (uint64_t)(((kk >> 2) * L::kVtPanel + (kk & 3) * 32) >> 4),
-                        dP + (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_pv,
+                        dP + (uint64_t)(((u & 1) * 2 * kPanel + (kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_pv,
                         (u > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&C.pv_done);
-          mma_commit(&C.kv_empty[s]);
+          mma_commit(&C.pv_done[u & 1]);
+          mma_commit(&C.v_empty[vs]);
         }
       }
       mma_commit(&C.fin);
@@ -237,11 +265,15 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
     const int q = 16 * ww + (lane & 15);
     const uint32_t lane_base = tmem + ((uint32_t)(ww * 32) << 16);
     const float c = p.scale_log2;
+    const uint64_t c2 = f32x2_pack(c, c);
     float m = -INFINITY, l = 0.f;
+    // lists ascend with every entry <= i, so only the last can be the
+    // diagonal block (a bad entry reads as the diagonal, as the producers do)
+    const int last_j = tf32a::entry(p, unit, i, cnt - 1);
     bool ok = true;
     for (int t = 0; t < cnt; ++t) {
       const int s = t & 1;
-      const int j = tf32a::entry(p, unit, i, t);
+      const int j = t == cnt - 1 ? last_j : -1;
       ok = ok && mbar_wait(&C.s_full[s], (t >> 1) & 1, abort_p, p.status, tmo);
       uint32_t r0[32], r1[32];
       if (ok) {
@@ -253,42 +285,67 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(&C.s_free[s]);
+      // scores in log2 units, two at a time (packed f32x2)
       float x[64];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        x[k] = __uint_as_float(r0[k]) * c;
-        x[32 + k] = __uint_as_float(r1[k]) * c;
+      for (int k = 0; k < 16; ++k) {
+        f32x2_unpack(mul_f32x2(f32x2_pack(__uint_as_float(r0[2 * k]), __uint_as_float(r0[2 * k + 1])), c2), x[2 * k],
+                     x[2 * k + 1]);
+        f32x2_unpack(mul_f32x2(f32x2_pack(__uint_as_float(r1[2 * k]), __uint_as_float(r1[2 * k + 1])), c2),
+                     x[32 + 2 * k], x[33 + 2 * k]);
       }
       if (j == i) {  // causal rule inside the diagonal block
 #pragma unroll
         for (int k = 0; k < 64; ++k) x[k] = k > q ? -INFINITY : x[k];
       }
-      float mx = x[0];
+      // row maximum by a tree of 3-input maxima (depth 4, not a 63-long chain)
+      float t1[22];
 #pragma unroll
-      for (int k = 1; k < 64; ++k) mx = fmaxf(mx, x[k]);
+      for (int k = 0; k < 21; ++k) t1[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+      t1[21] = x[63];
+      float t2[8];
+#pragma unroll
+      for (int k = 0; k < 7; ++k) t2[k] = fmax3(t1[3 * k], t1[3 * k + 1], t1[3 * k + 2]);
+      t2[7] = t1[21];
+      const float mx = fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), fmaxf(t2[6], t2[7]));
       float alpha = 1.f;
       bool raise = false;
       if (mx > m + kRaise) {
         if (t > 0) {
-          alpha = exp2f(m - mx);
+          alpha = ex2_approx(m - mx);
           raise = true;
         }
         l *= alpha;
         m = mx;
       }
-      float ps = 0.f;
+      // probabilities, and their sum by a tree of packed adds
+      const uint64_t nm2 = f32x2_pack(-m, -m);
+      uint64_t acc[16];
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        x[k] = exp2f(x[k] - m);
-        ps += x[k];
+      for (int k = 0; k < 32; ++k) {
+        float a, bb;
+        f32x2_unpack(add_f32x2(f32x2_pack(x[2 * k], x[2 * k + 1]), nm2), a, bb);
+        x[2 * k] = ex2_approx(a);
+        x[2 * k + 1] = ex2_approx(bb);
       }
-      l += ps;
-      // P(t) overwrites P(t-1) and O^T may be rescaled: PV(t-1) must be done
-      if (t >= 1) ok = ok && mbar_wait(&C.pv_done, (t - 1) & 1, abort_p, p.status, tmo);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        acc[k] = add_f32x2(f32x2_pack(x[4 * k], x[4 * k + 1]), f32x2_pack(x[4 * k + 2], x[4 * k + 3]));
+#pragma unroll
+      for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int k = 0; k < w2; ++k) acc[k] = add_f32x2(acc[k], acc[k + w2]);
+      float s0, s1;
+      f32x2_unpack(acc[0], s0, s1);
+      l += s0 + s1;
+      // P(t) goes to the tile PV(t-2) read
+      if (t >= 2) ok = ok && mbar_wait(&C.pv_done[t & 1], ((t >> 1) - 1) & 1, abort_p, p.status, tmo);
       if (row_thread) C.alpha[t & 1][q] = alpha;
-      // every softmax thread reaches this barrier; a failure anywhere ends
+      // every softmax thread reaches these barriers; a failure anywhere ends
       // the loop for all of them together
       const bool any_raise = bar_red_or(1, 128, row_thread && raise);
+      // a rescale of O^T waits for every PV so far (PV(t-1) and before)
+      if (any_raise && t >= 1) ok = ok && mbar_wait(&C.pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_p, p.status, tmo);
       ok = !bar_red_or(2, 128, !ok);
       if (!ok) break;
       if (any_raise) {
@@ -308,7 +365,7 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       }
       if (row_thread) {
         // P[q][0..63] as fp32 into the two 32-key panels, 128-byte swizzle
-        uint8_t* prow = smem + L::kOffP + (uint32_t)q * 128u;
+        uint8_t* prow = smem + L::kOffP + (uint32_t)(t & 1) * 2u * kPanel + (uint32_t)q * 128u;
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
           const int pn = cc >> 3, ch = cc & 7;
@@ -319,10 +376,10 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       fence_async_shared();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&C.p_full);
+      if (lane == 0) mbar_arrive(&C.p_full[t & 1]);
     }
     // ---- epilogue: O = O^T columns / l, LSE
-    if (ok) ok = mbar_wait(&C.pv_done, (cnt - 1) & 1, abort_p, p.status, tmo);
+    if (ok) ok = mbar_wait(&C.pv_done[(cnt - 1) & 1], ((cnt - 1) >> 1) & 1, abort_p, p.status, tmo);
     if (row_thread) {
       C.linv[q] = 1.0f / l;
       if (p.lse) p.lse[qrow0 + q] = (m + log2f(l)) * 0.6931471805599453f;

@@ -22,9 +22,9 @@ struct Tf32AttnParams {
 // V^T per 64-key block into Vt [B*Hkv*nb*d, 64] (fp32).
 cudaError_t launch_vt(const float* V, float* Vt, long long BHkv, int n, int d, cudaStream_t st);
 
-// tmQ, tmK: 2-D fp32 maps over Q [B*Hq*n, d] and K [B*Hkv*n, d] with 32 x 64
-// boxes (128 bytes by 64 rows); tmV over Vt [B*Hkv*nb*d, 64] with 32 x d
-// boxes; all 128-byte swizzled.
+// tmQ, tmK: 3-D fp32 panel maps over Q [B*Hq*n, d] and K [B*Hkv*n, d] (box
+// {32, 64, d/32}); tmV over Vt [B*Hkv*nb*d, 64] (box {32, d, 2}); all
+// 128-byte swizzled.
 cudaError_t launch_attn_tf32(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const Tf32AttnParams& p, cudaStream_t st);
 
