@@ -145,6 +145,33 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
+# ------------------------------------------------------------ multi-rank --
+# One process per GPU, each running its own independent layer (weak
+# scaling); the only cross-rank traffic is these scalar reductions.
+def rank_workload(base, rank: int):
+    """The rank's own layer: the workload's shapes with seed + 1000 * rank."""
+    from learned_block_sparse_seer_b200 import synth
+    return synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.n, base.d, base.h, base.dtype,
+                          base.structure, base.seed + 1000 * rank)
+
+
+def reduce_over_ranks(x: float, dev, op: str = "max") -> float:
+    """x reduced over all ranks ("max" or "sum"); x itself with one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_all_ranks: float, ms: float) -> float:
+    """Whole-job throughput: the FLOPs of every rank over the slowest rank's
+    time."""
+    return flops_all_ranks / (ms * 1e-3) / 1e12
+
+
 def attn_flops(counts, indices, d):
     """Algorithmic FLOPs of the active blocks: 4*d per (query, key) pair, a
     diagonal block counts its 64*65/2 causal pairs."""
@@ -515,8 +542,7 @@ def main():
     seer.lib()
 
     base = synth.WORKLOADS[args.workload]
-    w = synth.Workload(base.name, base.B, base.Hq, base.Hkv, base.n, base.d, base.h, base.dtype,
-                       base.structure, base.seed + 1000 * rank)
+    w = rank_workload(base, rank)
     Q, K, V = synth.make_qkv(w)
     Wq, Wk = synth.make_gate_weights(w)
     Qd, Kd, Vd, Wqd, Wkd = (t.to(dev) for t in (Q, K, V, Wq, Wk))
@@ -570,14 +596,12 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     gate_ms = [a.elapsed_time(b) for a, b, _ in ev]
     attn_ms = [b.elapsed_time(c) for _, b, c in ev]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_over_ranks(total_ms, dev, "max")
+    flops_all = reduce_over_ranks(flops, dev, "sum")
     ms_per_step = total_ms / args.steps
     attn_avg = sum(attn_ms) / len(attn_ms)
     gate_avg = sum(gate_ms) / len(gate_ms)
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops_all, ms_per_step)
     attn_tflops = flops / (attn_avg * 1e-3) / 1e12
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
@@ -606,11 +630,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = reduce_over_ranks(e2e_ms, dev, "max")
+        e2e = {"value": whole_job_tflops(flops_all, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * 2,
                "d2h_bytes_per_step": O.numel() * 2}
