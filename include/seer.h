@@ -310,14 +310,18 @@ SEER_API seer_status seer_gate_noalloc(const seer_dims *dims, const void *Q, con
 /* seer_attn_forward_map -- the training forward of the summary page's
  * customized kernel ("The customized training kernel", Figure 10): dense
  * causal attention output O and row log-sum-exp, plus the 2D-max-pooled
- * probability map gt, in one call.  Two launches on the stream: the map (as
- * seer_attn_blockmax), then the attention over every causal block (as
- * seer_sparse_attn with the full causal lists, which are not materialised).
+ * probability map gt, in one pass.  The attention kernel runs over every
+ * causal block and also keeps, per step, each column's score maximum over
+ * each 32-key half block; at the end of each 64-row unit those maxima become
+ * probabilities with the final row sums, and their maximum over the rows is
+ * the map entry.  Units that need the exact fallback (a score more than 2^64
+ * above the unit's first-step maximum) get their O, LSE and map row
+ * recomputed exactly.
  *   Q [B,Hq,n,d], K, V [B,Hkv,n,d] (dtype); scale 0 means 1/sqrt(d)
  *   O [B,Hq,n,d] (dtype), lse [B,Hq,n] fp32 (may be NULL),
  *   map_out [B,Hq,nb,nb] fp32 (0 above the diagonal)
  *   ws/ws_bytes  workspace of at least seer_attn_forward_map_workspace_size(...)
- * Errors: as seer_attn_blockmax and seer_sparse_attn.                      */
+ * Errors: as seer_sparse_attn.                                              */
 SEER_API seer_status seer_attn_forward_map(const seer_dims *dims, const void *Q, const void *K, const void *V,
                                           seer_dtype dtype, float scale, void *O, float *lse, float *map_out,
                                           void *ws, size_t ws_bytes, seer_stream_t stream);

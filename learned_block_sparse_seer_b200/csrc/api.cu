@@ -517,7 +517,7 @@ namespace {
 seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V, seer_dtype dtype,
                             const int32_t* counts, const int32_t* indices, int32_t cap, float scale, void* O,
                             float* lse, void* ws, size_t ws_bytes, seer_stream_t stream, bool dense,
-                            bool keep_status = false) {
+                            bool keep_status = false, float* map = nullptr, size_t map_scratch_off = 0) {
   if (!dims_ok(dims) || !Q || !K || !V || !O) return SEER_ERR_INVALID_ARG;
   if (!dense && (!counts || !indices)) return SEER_ERR_INVALID_ARG;
   if (dense) cap = dims->n / seer::kBlock;
@@ -528,15 +528,18 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
     return SEER_ERR_INVALID_ARG;
   const AttnWs w = attn_ws(dims, dtype);
+  // with a map, its per-CTA scratch follows the attention workspace
+  const size_t need = map ? map_scratch_off + sizeof(float) * (size_t)num_sms() * (dims->n / seer::kBlock) * 128
+                          : w.total;
   cudaStream_t st = (cudaStream_t)stream;
   if (keep_status) {
     // a call made on behalf of another in the same workspace: reset only the
     // work counters, so that the earlier launch's device status survives
-    if (!ws || !aligned(ws, 256) || ws_bytes < w.total) return SEER_ERR_WORKSPACE;
+    if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEER_ERR_WORKSPACE;
     SEER_CUDA(cudaMemsetAsync((uint8_t*)ws + 8, 0, sizeof(seer::WsHeader) - 8, st));
     s = SEER_OK;
   } else {
-    s = begin_ws(ws, ws_bytes, w.total, st);
+    s = begin_ws(ws, ws_bytes, need, st);
   }
   if (s != SEER_OK) return s;
   uint8_t* base = (uint8_t*)ws;
@@ -578,6 +581,9 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   p.redo_count = &hdr->work_counter2;
   p.redo_list = reinterpret_cast<int*>(base + w.redo);
   p.redo_cap = (int)p.total_units;
+  p.map = map;
+  p.map_scratch = map ? (float*)(base + map_scratch_off) : nullptr;
+  if (map) SEER_CUDA(cudaMemsetAsync(map, 0, sizeof(float) * (size_t)p.total_units * p.nb, st));
   if (!dense) SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
   SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kv, p, st));
@@ -887,20 +893,20 @@ seer_status seer_decode_blockmax(const seer_dims* dims, const void* q, const voi
 // --------------------------------------------------- training forward ----
 size_t seer_attn_forward_map_workspace_size(const seer_dims* dims, seer_dtype dtype) {
   if (!dims_ok(dims)) return 0;
-  const size_t a = attn_ws(dims, dtype).total, m = bmax_ws(dims, dtype, num_sms()).total;
-  return a > m ? a : m;
+  // the attention workspace, then the map's per-CTA scratch [nb][2][64] fp32
+  return attn_ws(dims, dtype).total + sizeof(float) * (size_t)num_sms() * (dims->n / seer::kBlock) * 128;
 }
 
 seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const void* K, const void* V,
                                   seer_dtype dtype, float scale, void* O, float* lse, float* map_out, void* ws,
                                   size_t ws_bytes, seer_stream_t stream) {
   if (!dims_ok(dims) || !Q || !K || !V || !O || !map_out) return SEER_ERR_INVALID_ARG;
-  // the max-pooled map first (its own log-sum-exp is not kept), then the
-  // attention output over every causal block on the same workspace
-  seer_status s = seer_attn_blockmax(dims, Q, K, dtype, scale, map_out, nullptr, ws, ws_bytes, stream);
-  if (s != SEER_OK) return s;
+  // one pass: the attention kernel over every causal block, keeping each
+  // (row block, key half, column) score maximum and turning them into the map
+  // at each unit's end (the exact fallback redoes the map rows of the units
+  // it recomputes)
   return run_sparse_attn(dims, Q, K, V, dtype, nullptr, nullptr, 0, scale, O, lse, ws, ws_bytes, stream, true,
-                         true);
+                         false, map_out, attn_ws(dims, dtype).total);
 }
 
 }  // extern "C"

@@ -354,6 +354,47 @@ __device__ __forceinline__ void scores_minus_max(uint32_t taddr, float (&x)[attn
   }
 }
 
+// MAP mode: this warp's per-column maxima over its 32 keys (lanes) of the
+// step's scores x (log2 units, relative to the unit's fixed maximum).  A
+// butterfly reduce-scatter (16 shuffles for 16 columns) leaves the maximum of
+// column map_col(lane) on each lane; the even lanes store it later, after the
+// step's barrier arrivals (an arrival releases the thread's earlier global
+// stores, so a store just before it would stall the step on its write).
+__device__ __forceinline__ float warp_col_max(const float (&x)[attn::kCols], int lane) {
+  static_assert(attn::kCols == 16, "16 columns per warp");
+  float v[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) v[q] = x[q];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const bool up = lane & 16;
+    const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
+    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const bool up = lane & 8;
+    const float send = up ? v[k] : v[k + 4], keep = up ? v[k + 4] : v[k];
+    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const bool up = lane & 4;
+    const float send = up ? v[k] : v[k + 2], keep = up ? v[k + 2] : v[k];
+    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+  {
+    const bool up = lane & 2;
+    const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+    v[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+  }
+  return fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+}
+
+__device__ __forceinline__ int map_col(int lane) {
+  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
+
 // This warpgroup's 16 bf16 probabilities of key row kl into the step's P^T
 // tile (128-byte rows, 16-byte chunks swizzled by the row index).
 // off0/off1 are the row's two swizzled 16-byte chunk offsets.
@@ -366,7 +407,14 @@ __device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kC
   *reinterpret_cast<uint4*>(prow + off1) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
-template <int D>
+// MAP (the training forward): also the 2D-max-pooled probability map.  Each
+// step every warp takes, per query column, the maximum of its 32 keys'
+// scores (redux.sync over the lanes = keys) and keeps it in the CTA's scratch
+// slot [key block][key half][64 columns]; the unit's epilogue turns the
+// kept maxima into probabilities with the final row sums and max-combines
+// them over the 64 rows into the map (atomicMax on the non-negative bit
+// patterns; one partial per warpgroup of 16 columns).
+template <int D, bool MAP>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                        const AttnParams p) {
@@ -618,6 +666,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // running maximum (log2 domain) and this thread's row-sum partial.
     uint64_t nm2[kCols / 2], lp2[kCols / 2];
     const uint64_t c2 = f32x2_pack(c, c);
+    // MAP mode: this CTA's scratch of per-(key block, key half, column) maxima
+    float* const mscr = MAP ? p.map_scratch + (long long)blockIdx.x * p.nb * 128 : nullptr;
     // this thread's P^T row (key kl of half `half`) and its two swizzled
     // 16-byte chunks (this warpgroup's 16 query columns)
     uint8_t* const prow0 = smem + kOffP + half * 8192 + kl * 128;
@@ -665,6 +715,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const uint32_t saddr = lane_addr + (uint32_t)sb * 64u + q0;
         uint8_t* const prow = prow0 + ps * kPBytes;
         float x[kCols];
+        float mval = 0.f;  // MAP mode: this lane's column maximum of the step
+        (void)mval;
         if (t == 0) {
           // exact column maxima of the unit's first step
           if (okS) load_scores(saddr, x, c, valid, diag, kl, q0);
@@ -677,11 +729,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kCols / 2; ++q) nm2[q] = f32x2_pack(-mcol[2 * q], -mcol[2 * q + 1]);
           scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
+          if constexpr (MAP) mval = warp_col_max(x, lane);
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
           store_p(prow, x, poff0, poff1);
         } else {
           if (okS) scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
+          if constexpr (MAP) mval = warp_col_max(x, lane);
           const float dmax =
               fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
                     fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
@@ -709,6 +763,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (lane == 0) {
           mbar_arrive(&bars.go[rg]);
           mbar_arrive(&bars.kfull[(rg + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
+        }
+        if constexpr (MAP) {
+          if (valid && (lane & 1) == 0) mscr[((long long)mi * 2 + (ww & 1)) * 64 + q0 + map_col(lane)] = mval;
         }
         if (++rg == kRing) {
           rg = 0;
@@ -767,6 +824,34 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             lq = l[q];
           }
         p.lse[orow0 + tl] = (mq + log2f(lq)) * 0.6931471805599453f;
+      }
+      if constexpr (MAP) {
+        // the kept maxima become probabilities with the row sums: x - log2(l)
+        // (x is relative to the fixed maximum); max over this warpgroup's 16
+        // columns, then over the 4 warpgroups by atomicMax into the map row
+        float ll[kCols];
+#pragma unroll
+        for (int q = 0; q < kCols; ++q) ll[q] = log2f(l[q]);
+        const int* lst = p.indices + u.u * p.cap;
+        for (int mi2 = tl; mi2 < count; mi2 += 128) {
+          const float4* s0 = reinterpret_cast<const float4*>(mscr + (long long)mi2 * 128 + q0);
+          float4 a[4], b2[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            a[k] = s0[k];
+            b2[k] = s0[16 + k];  // the other key half, 64 floats on
+          }
+          float v = 0.f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            v = fmaxf(v, ex2_approx(fmaxf(a[k].x, b2[k].x) - ll[4 * k]));
+            v = fmaxf(v, ex2_approx(fmaxf(a[k].y, b2[k].y) - ll[4 * k + 1]));
+            v = fmaxf(v, ex2_approx(fmaxf(a[k].z, b2[k].z) - ll[4 * k + 2]));
+            v = fmaxf(v, ex2_approx(fmaxf(a[k].w, b2[k].w) - ll[4 * k + 3]));
+          }
+          const int j = p.dense ? mi2 : lst[mi2];
+          atomicMax(reinterpret_cast<int*>(p.map + u.u * p.nb + j), __float_as_int(v));
+        }
       }
 #ifdef SEER_TRACE
       if (lane == 0) SEER_TRACE_ADD(10, clock64() - tep0);
@@ -885,6 +970,7 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
                                                                const __nv_bfloat16* __restrict__ recs,
                                                                const AttnParams p) {
   constexpr int DL = D / 32;  // head dims per lane
+  __shared__ float lse2s[64];  // the unit's row LSEs (log2), for the map
   const uint32_t nredo = min(*reinterpret_cast<volatile uint32_t*>(p.redo_count), (uint32_t)p.redo_cap);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   for (uint32_t e = blockIdx.x; e < nredo; e += gridDim.x) {
@@ -935,6 +1021,33 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
           reinterpret_cast<__nv_bfloat16*>(p.O)[idx] = __float2bfloat16_rn(v);
       }
       if (lane == 0 && p.lse) p.lse[qrow] = (m + log2f(l)) * 0.6931471805599453f;
+      if (lane == 0) lse2s[r] = m + log2f(l);
+    }
+    if (p.map) {
+      // the unit's map row, exactly: for each listed key block, the largest
+      // probability exp2(score - lse2) over the 64 rows and the block's keys
+      __syncthreads();
+      for (int t = warp; t < u.count; t += 8) {
+        int j = p.dense ? t : lst[t];
+        j = j < 0 ? 0 : (j > u.i ? u.i : j);
+        const __nv_bfloat16* rec = recs + (rec0 + j) * (2LL * D * 64);
+        float best = 0.f;
+        for (int r = 0; r < 64; ++r) {
+          const long long qrow = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + r;
+          float q[DL];
+#pragma unroll
+          for (int k = 0; k < DL; ++k) q[k] = __bfloat162float(Q16[qrow * D + lane * DL + k]);
+          const int kmax = j == u.i ? r : 63;
+          for (int key = 0; key <= kmax; ++key) {
+            float sdot = 0.f;
+#pragma unroll
+            for (int k = 0; k < DL; ++k) sdot += q[k] * __bfloat162float(rec[(lane * DL + k) * 64 + key]);
+            best = fmaxf(best, exp2f(warp_sum(sdot) * p.scale_log2 - lse2s[r]));
+          }
+        }
+        if (lane == 0) p.map[u.u * p.nb + j] = best;
+      }
+      __syncthreads();
     }
   }
 }
@@ -966,7 +1079,8 @@ cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, 
 
 cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
                                int num_sms, cudaStream_t st) {
-  auto kern = p.d == 64 ? sparse_attn_kernel<64> : sparse_attn_kernel<128>;
+  auto kern = p.map ? (p.d == 64 ? sparse_attn_kernel<64, true> : sparse_attn_kernel<128, true>)
+                    : (p.d == 64 ? sparse_attn_kernel<64, false> : sparse_attn_kernel<128, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn::kSmemAlloc);
   if (e != cudaSuccess) return e;
   long long grid = p.total_units < num_sms ? p.total_units : num_sms;

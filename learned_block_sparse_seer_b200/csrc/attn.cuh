@@ -23,6 +23,8 @@ struct AttnParams {
   uint32_t* redo_count;       // units flagged for the exact fallback (workspace)
   int* redo_list;             // [redo_cap] flagged unit indices
   int redo_cap;
+  float* map;          // training forward: [B*Hq*nb, nb] max-pooled map (zeroed first), or null
+  float* map_scratch;  // with map: per CTA [nb][2][64] fp32
 };
 
 // Re-layout of K and V into per-block records of 2*d rows x 64 bf16 (K^T,

@@ -67,3 +67,21 @@ def test_layer8k_sampled():
     assert np.abs(M.reshape(-1, nb)[units] - gt_ref).max() <= BMAX_TOL
     iu = np.triu_indices(nb, 1)
     assert np.all(M[..., iu[0], iu[1]] == 0)
+
+
+def test_fallback_units_keep_an_exact_map():
+    """A key block far above the first step's maximum (scores more than 2^64
+    above it) sends its units to the exact fallback, which also rewrites their
+    map rows."""
+    wl = synth.custom("fm", 1, 2, 1, 64 * 6, 64, 16, "bf16", "layer", 43)
+    Q, K, V = synth.make_qkv(wl)
+    K = K.float()
+    K[:, :, 64 * 4:64 * 5] *= 40.0
+    K = K.to(torch.bfloat16).contiguous()
+    O, lse, M = _run(Q, K, V)
+    counts, idx = oracle.dense_lists(1, 2, 6)
+    O_ref, lse_ref = oracle.sparse_attn(Q, K, V, counts, idx)
+    check_o(O.double().numpy(), O_ref)
+    check_lse(lse, lse_ref, LSE_TOL)
+    gt_ref, _ = oracle.blockmax(Q, K)
+    assert np.abs(M - gt_ref).max() <= BMAX_TOL
