@@ -699,8 +699,8 @@ def main():
         b1.record(stream)
         torch.cuda.synchronize(dev)
         fms = b0.elapsed_time(b1) / nrep
-        # map: 2 d per causal pair; attention: 4 d per causal pair
-        fflops = 6.0 * bw.d * pairs
+        # one pass: QK^T (shared by the map) and PV, 4 d per causal pair
+        fflops = 4.0 * bw.d * pairs
         bmax["forward_map"] = {"ms": fms, "tflops": fflops / (fms * 1e-3) / 1e12,
                                "flops": fflops, "status": seer.seer_workspace_status(fws)}
         del bV, fws, fout
