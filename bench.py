@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-tf32", action="store_true")
+    ap.add_argument("--no-context", action="store_true", help="skip the dense-attention comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="also time the 50-95%% sparsity sweep")
@@ -342,6 +343,40 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def context_bench(seer, dev, stream, w, Qd, Kd, Vd, O, lse, gate_ms, attn_ms):
+    """Context for the sparse step: dense causal attention of the same layer
+    by torch's scaled_dot_product_attention (its fastest backend on this GPU,
+    GQA native) and by this library's kernel with every causal block listed
+    (the all-ones mask), and the sparse step's speedup over the dense one."""
+    import torch
+    import torch.nn.functional as F
+
+    def timed(fn, reps=2):
+        fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    sdpa_ms = timed(lambda: F.scaled_dot_product_attention(Qd, Kd, Vd, is_causal=True, enable_gqa=True))
+    nb = w.nb
+    counts = (torch.arange(nb, device=dev, dtype=torch.int32) + 1).repeat(w.B, w.Hq, 1).contiguous()
+    idx = torch.arange(nb, device=dev, dtype=torch.int32).repeat(w.B, w.Hq, nb, 1).contiguous()
+    ws = torch.empty(seer.sparse_attn_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device=dev)
+    ones_ms = timed(lambda: seer.seer_sparse_attn(Qd, Kd, Vd, counts, idx, workspace=ws, out=(O, lse)))
+    del idx, counts, ws
+    dense_flops = 4.0 * w.d * w.B * w.Hq * (w.n * (w.n + 1) / 2)
+    return {"workload": f"{w.name}: dense causal attention, same shapes",
+            "sdpa_dense_ms": sdpa_ms, "sdpa_tflops": dense_flops / (sdpa_ms * 1e-3) / 1e12,
+            "all_ones_mask_ms": ones_ms, "all_ones_tflops": dense_flops / (ones_ms * 1e-3) / 1e12,
+            "speedup_sparse_attn_vs_sdpa": sdpa_ms / attn_ms,
+            "speedup_gate_plus_sparse_attn_vs_sdpa": sdpa_ms / (gate_ms + attn_ms)}
 
 
 def tf32_bench(seer, dev, stream, w, Qd, Kd, Vd, counts, indices, flops, pk):
@@ -721,6 +756,11 @@ def main():
     if not args.no_tf32 and rank == 0:
         tf = tf32_bench(seer, dev, stream, w, Qd, Kd, Vd, counts, indices, flops, pk)
 
+    # ------------------------------------------------- dense-attention context --
+    ctx = None
+    if not args.no_context and rank == 0:
+        ctx = context_bench(seer, dev, stream, w, Qd, Kd, Vd, O, lse, gate_avg, attn_avg)
+
     # ------------------------------------------------------ density sweep ----
     sweep = None
     if args.sweep and rank == 0:
@@ -794,7 +834,7 @@ def main():
                          "algorithmic_flops_per_launch": flops},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 7 * args.steps,
-            "blockmax": bmax, "decode": dec, "varlen": vl, "tf32": tf, "sweep": sweep,
+            "blockmax": bmax, "decode": dec, "varlen": vl, "tf32": tf, "dense_context": ctx, "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
