@@ -20,31 +20,34 @@
 //    in 64-column panels]; a d-row TMA box (16 KB at d = 128, no cluster
 //    multicast) brings either part of a block into shared memory.
 //  * The tensor pipe stalls for about 200 cycles whenever the thread that
-//    issues the MMAs synchronises (an mbarrier wait, a shared-memory read, a
-//    barrier), so the MMA thread waits exactly once per pair step, on one
-//    barrier go(g) that collects everything the next MMA group needs: the
-//    softmax's P^T of step g, the V records of step g and the K^T records
-//    (and, at a unit's start, the Q tile) of step g+2.  It then issues PV(g)
-//    and QK(g+2) back to back.  QK therefore runs two steps ahead of PV, which
-//    keeps the softmax of step g+1 busy while PV(g) and QK(g+2) execute.
+//    issues MMAs synchronises (an mbarrier wait, a shared-memory read, a
+//    barrier), so two warps issue them, each waiting once per pair step on
+//    its own barrier: the QK warp on kfull(h) (K^T of step h landed, plus the
+//    unit's Q tile on its first step, and the softmax has released the S^T
+//    buffer of step h-3), the PV warp on go(g) (P^T and V of step g ready).
+//    While one waits the other keeps the pipe fed.  The MMA groups are
+//    straight-line code: fully unrolled, descriptors as a base plus constant
+//    offsets, ring positions as counters.
 //  * Separate rings keep each buffer only as long as it is needed: K^T pairs
 //    (2 slots, free once their QK is done), V pairs (3 slots, free once their
-//    PV is done), P^T tiles (2 slots), Q tiles (2 slots), S^T in TMEM (3
-//    buffers).  224 KB of shared memory in all.
-//  * Warp roles (576 threads): warps 0..15 are four softmax warpgroups, each
-//    owning 16 of the 64 query columns (its own running max, row sums, vote
-//    and epilogue), one key (TMEM lane) per thread -- a warp w reaches TMEM
-//    lanes 32*(w%4)..+31; warp 16 schedules units and issues every TMA load;
-//    warp 17 issues all MMAs from one thread and owns the TMEM allocation.
-//  * Online softmax with a lazily updated running maximum per query column:
-//    the exact column maximum is formed on a unit's first step; afterwards a
-//    warpgroup vote re-forms it only when some score exceeds the running
-//    maximum by more than 2^8 (log2 domain), rescaling the row sums and O^T.
-//    The vote is one hardware barrier-with-reduction per step, taken after
-//    the exponentials (which are recomputed in the rare rescale case).
+//    PV is done), P^T tiles (3 slots), one Q tile, S^T in TMEM (3 buffers).
+//    224 KB of shared memory in all.
+//  * Warp roles (608 threads): warps 0..15 are four softmax warpgroups, each
+//    owning 16 of the 64 query columns, one key (TMEM lane) per thread -- a
+//    warp w reaches TMEM lanes 32*(w%4)..+31; warp 16 schedules units and
+//    issues every TMA load; warp 17 issues the PV MMAs and owns the TMEM
+//    allocation; warp 18 issues the QK MMAs.
+//  * Softmax without a per-step barrier: each unit's column maxima are formed
+//    exactly on its first step and then kept; later steps compute
+//    exp2(score * scale - max) with packed f32x2 arithmetic.  A score more
+//    than 2^64 above its column's kept maximum flags the unit (a warp vote),
+//    and sparse_attn_redo_kernel recomputes flagged units exactly afterwards.
 //  * Units are handed out by an atomic counter in KV-head-major order, query
 //    blocks from the last (longest lists) to the first, so the K/V of one KV
-//    head stay hot in L2 while its query heads are processed.
+//    head stay hot in L2 while its query heads are processed.  Units with an
+//    empty list never enter the ring (empty_rows_kernel writes their rows).
+//  * MAP mode (the training forward) also forms the 2D-max-pooled map in the
+//    same pass (see the kernel's comment).
 //  * Every mbarrier wait is bounded (%globaltimer); on expiry the kernel
 //    records a timeout in the workspace status word and unwinds.
 #include <cstddef>
@@ -409,11 +412,11 @@ __device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kC
 
 // MAP (the training forward): also the 2D-max-pooled probability map.  Each
 // step every warp takes, per query column, the maximum of its 32 keys'
-// scores (redux.sync over the lanes = keys) and keeps it in the CTA's scratch
-// slot [key block][key half][64 columns]; the unit's epilogue turns the
-// kept maxima into probabilities with the final row sums and max-combines
-// them over the 64 rows into the map (atomicMax on the non-negative bit
-// patterns; one partial per warpgroup of 16 columns).
+// scores (a shuffle reduce-scatter over the lanes = keys) and keeps it in the
+// CTA's scratch slot [key block][key half][64 columns]; the unit's epilogue
+// turns the kept maxima into probabilities with the final row sums and
+// max-combines them over the 64 rows into the map (atomicMax on the
+// non-negative bit patterns; one partial per warpgroup of 16 columns).
 template <int D, bool MAP>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
