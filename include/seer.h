@@ -8,6 +8,15 @@
  *   seer_sparse_attn    block-sparse causal attention over the selected blocks
  *   seer_attn_blockmax  2D max-pooled attention-probability map (the gate's
  *                       self-distillation target)
+ *   seer_attn_forward_map  the training forward: dense causal O, LSE and the
+ *                       max-pooled map in one pass
+ *   seer_gate_kl_backward  one distillation step: KL(gt || score) and the
+ *                       gradients of the gate's two linear layers
+ *   seer_gate_varlen    the gate over variable-length sequences packed along
+ *                       the token axis (then seer_sparse_attn as usual)
+ *   seer_sparse_attn_tf32  the attention for fp32 inputs on the tf32 tensor
+ *                       cores
+ *   seer_gate_noalloc   seer_gate without a workspace
  *   seer_decode_*       the decode stage: compressed K cache, token gate,
  *                       block-sparse decode attention, 1D ground truth
  *
