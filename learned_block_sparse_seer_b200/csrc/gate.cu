@@ -272,8 +272,8 @@ __device__ __forceinline__ int topk_count(int i, int mode, int k, float density)
 //  * tab (varlen packing): row i's candidates are its own sequence's blocks
 //    f .. i with f = tab[i].x (none when f < 0); k_i is taken at the local
 //    row i - f, and the list holds global block indices.
-template <bool FROM_LOGITS>
-__global__ void __launch_bounds__(kRowThreads) row_select_kernel(
+template <bool FROM_LOGITS, int NT>
+__global__ void __launch_bounds__(NT) row_select_kernel(
     const float* in, float* scores, int nb, int mode_flags, float T, int k,
     float density, int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len,
     const int2* __restrict__ tab) {
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
   if (off < 0) {  // a block of no sequence: no candidates
     if (FROM_LOGITS && scores != nullptr) {
       float* dst = scores + row * (long long)nb;
-      for (int j = tid; j < nb; j += kRowThreads) dst[j] = 0.f;
+      for (int j = tid; j < nb; j += NT) dst[j] = 0.f;
     }
     if (tid == 0) counts[row] = 0;
     return;
@@ -301,30 +301,30 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
   const int len = i + 1;
   const float* src = in + row * (long long)nb + off;
 
-  for (int j = tid; j < len; j += kRowThreads) sv[j] = src[j];
+  for (int j = tid; j < len; j += NT) sv[j] = src[j];
   __syncthreads();
 
   if (FROM_LOGITS) {
     float m = -INFINITY;
-    for (int j = tid; j < len; j += kRowThreads) m = fmaxf(m, sv[j]);
+    for (int j = tid; j < len; j += NT) m = fmaxf(m, sv[j]);
     m = block_reduce_max(m, sh_f);
     float s = 0.f;
-    for (int j = tid; j < len; j += kRowThreads) {
+    for (int j = tid; j < len; j += NT) {
       const float e = expf(sv[j] - m);
       sv[j] = e;
       s += e;
     }
     s = block_reduce_sum(s, sh_f);
-    for (int j = tid; j < len; j += kRowThreads) sv[j] = sv[j] / s;
+    for (int j = tid; j < len; j += NT) sv[j] = sv[j] / s;
     __syncthreads();
     if (scores != nullptr) {
       float* dst = scores + row * (long long)nb;
-      for (int j = tid; j < nb; j += kRowThreads) dst[j] = (j >= off && j - off < len) ? sv[j - off] : 0.f;
+      for (int j = tid; j < nb; j += NT) dst[j] = (j >= off && j - off < len) ? sv[j - off] : 0.f;
     }
   }
 
   // Each thread owns a contiguous chunk so that compaction keeps ascending j.
-  const int chunk = (len + kRowThreads - 1) / kRowThreads;
+  const int chunk = (len + NT - 1) / NT;
   const int j0 = tid * chunk;
   const int j1 = min(j0 + chunk, len);
   int32_t* out = indices + row * (long long)cap;
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
 
   const int ki = topk_count(i, mode, k, density);
   if (ki >= len) {  // every causal block is kept
-    for (int j = tid; j < len; j += kRowThreads) out[j] = j + off;
+    for (int j = tid; j < len; j += NT) out[j] = j + off;
     if (tid == 0) counts[row] = len;
     return;
   }
@@ -351,11 +351,11 @@ __global__ void __launch_bounds__(kRowThreads) row_select_kernel(
   uint32_t prefix = 0, pmask = 0;
   uint32_t remaining = (uint32_t)ki;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 256; b += kRowThreads) hist[b] = 0;
+    for (int b = tid; b < 256; b += NT) hist[b] = 0;
     __syncthreads();
     // Scores of a row share their top bits, so most keys fall into a few
     // bins: lanes with the same bin are counted by one atomic (match_any).
-    for (int j0 = 0; j0 < len; j0 += kRowThreads) {
+    for (int j0 = 0; j0 < len; j0 += NT) {
       const int j = j0 + tid;
       uint32_t bin = 0x100u;  // not counted
       if (j < len) {
@@ -519,24 +519,39 @@ cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cu
   return cudaGetLastError();
 }
 
+namespace {
+template <bool FROM_LOGITS, int NT>
+cudaError_t row_select_launch(const float* in, float* scores, long long rows, int nb, int mode, float T, int k,
+                              float density, int32_t* counts, int32_t* indices, int cap, cudaStream_t st,
+                              int row_len, const int2* tab) {
+  const size_t smem = (size_t)nb * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(row_select_kernel<FROM_LOGITS, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  row_select_kernel<FROM_LOGITS, NT><<<(unsigned)rows, NT, smem, st>>>(in, FROM_LOGITS ? scores : nullptr, nb, mode,
+                                                                       T, k, density, counts, indices, cap, row_len,
+                                                                       tab);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, long long rows,
                               int nb, int mode, float T, int k, float density, int32_t* counts,
                               int32_t* indices, int cap, cudaStream_t st, int row_len, const int2* tab) {
-  const size_t smem = (size_t)nb * sizeof(float);
-  if (from_logits) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(row_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    row_select_kernel<true><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, scores, nb, mode, T, k, density, counts, indices, cap, row_len, tab);
-  } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(row_select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    row_select_kernel<false><<<(unsigned)rows, kRowThreads, smem, st>>>(
-        in, nullptr, nb, mode, T, k, density, counts, indices, cap, row_len, tab);
-  }
-  return cudaGetLastError();
+  // Few rows (the decode gate, small batches) leave most SMs idle and each
+  // row's latency exposed: then 1024 threads share a row's work.
+  const bool wide = rows < 2LL * 148;
+  if (from_logits)
+    return wide ? row_select_launch<true, 1024>(in, scores, rows, nb, mode, T, k, density, counts, indices, cap, st,
+                                                row_len, tab)
+                : row_select_launch<true, kRowThreads>(in, scores, rows, nb, mode, T, k, density, counts, indices,
+                                                       cap, st, row_len, tab);
+  return wide ? row_select_launch<false, 1024>(in, scores, rows, nb, mode, T, k, density, counts, indices, cap, st,
+                                               row_len, tab)
+              : row_select_launch<false, kRowThreads>(in, scores, rows, nb, mode, T, k, density, counts, indices, cap,
+                                                      st, row_len, tab);
 }
 
 }  // namespace seer
