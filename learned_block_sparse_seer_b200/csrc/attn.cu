@@ -96,11 +96,13 @@ struct Bars {
   uint64_t q_free[kQSlots];  // the last QK of the unit that used a Q slot is complete
   uint64_t fin_qk, fin_pv;
 };
-// What the loader publishes about each unit: the unit index (-1 ends the
-// work), its checked list length and whether its last entry is the diagonal
-// block.  Consumers read only this, never the lists in global memory.
+// What the loader publishes about each unit: the work index (-1 ends the
+// work), its checked list length, whether its last entry is the diagonal
+// block, and the flat unit index u = (b*Hq + hq)*nb + i (its 64 query rows
+// start at row 64*u of Q and O).  Consumers read only this, never the lists
+// in global memory.
 struct UnitEntry {
-  int w, count, diag, pad;
+  int w, count, diag, u;
 };
 // Control block, placed in dynamic shared memory right after the tiles (the
 // tiles need nearly the whole 227 KB budget, so nothing is static).
@@ -178,14 +180,7 @@ __device__ __forceinline__ UnitInfo unit_coords(const AttnParams& p, int w) {
 // unit_coords plus the unit's list length, read and checked: it must lie in
 // [0, min(cap, i + 1)].  A failing count is recorded and clamped.
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int w) {
-  UnitInfo r;
-  const int per_bg = p.nb * p.G;
-  const int bg = w / per_bg, rem = w % per_bg;
-  r.b = bg / p.Hkv;
-  r.g = bg % p.Hkv;
-  r.i = p.nb - 1 - rem / p.G;
-  r.hq = r.g * p.G + rem % p.G;
-  r.u = ((long long)r.b * p.Hq + r.hq) * p.nb + r.i;
+  UnitInfo r = unit_coords(p, w);
   if (p.dense) {
     r.count = r.i + 1;
     return r;
@@ -514,6 +509,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         C.unit[slot].w = w;
         C.unit[slot].count = u.count;
         C.unit[slot].diag = diag;
+        C.unit[slot].u = w >= 0 ? (int)u.u : 0;
         mbar_arrive(&bars.unit_full[slot]);
         ++u_idx;
         if (w < 0) break;
@@ -685,13 +681,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const int w = okw ? C.unit[slot].w : -1;
       const int count = okw ? C.unit[slot].count : 0;
       const bool last_is_diag = okw && C.unit[slot].diag != 0;
+      const int uu = okw ? C.unit[slot].u : 0;
       if (bar_red_or(bar_id, 128, !okw)) break;
       if (w < 0) break;  // the end marker is never released: nothing reuses its slot
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       ++u_idx;
-      const UnitInfo u = unit_coords(p, w);
-      const long long orow0 = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + q0;
+      const long long orow0 = (long long)uu * 64 + q0;
       const int T = (count + 1) / 2;
 #pragma unroll
       for (int q = 0; q < kCols / 2; ++q) lp2[q] = 0ull;
@@ -806,7 +802,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (tl < p.d) {
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
-            const float v = __uint_as_float(o[q]) * (1.0f / l[q]);
+            // l >= 1: the column's maximum contributes exp2(0)
+            const float v = __uint_as_float(o[q]) * rcp_approx(l[q]);
             const long long idx = (orow0 + q) * p.d + tl;
             if (p.out_fp32)
               reinterpret_cast<float*>(p.O)[idx] = v;
@@ -826,7 +823,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             mq = -m[q];
             lq = l[q];
           }
-        p.lse[orow0 + tl] = (mq + log2f(lq)) * 0.6931471805599453f;
+        p.lse[orow0 + tl] = (mq + lg2_approx(lq)) * 0.6931471805599453f;
       }
       if constexpr (MAP) {
         // the kept maxima become probabilities with the row sums: x - log2(l)
@@ -834,8 +831,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         // columns, then over the 4 warpgroups by atomicMax into the map row
         float ll[kCols];
 #pragma unroll
-        for (int q = 0; q < kCols; ++q) ll[q] = log2f(l[q]);
-        const int* lst = p.indices + u.u * p.cap;
+        for (int q = 0; q < kCols; ++q) ll[q] = lg2_approx(l[q]);
+        const int* lst = p.indices + (long long)uu * p.cap;
         for (int mi2 = tl; mi2 < count; mi2 += 128) {
           const float4* s0 = reinterpret_cast<const float4*>(mscr + (long long)mi2 * 128 + q0);
           float4 a[4], b2[4];
@@ -853,7 +850,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             v = fmaxf(v, ex2_approx(fmaxf(a[k].w, b2[k].w) - ll[4 * k + 3]));
           }
           const int j = p.dense ? mi2 : lst[mi2];
-          atomicMax(reinterpret_cast<int*>(p.map + u.u * p.nb + j), __float_as_int(v));
+          atomicMax(reinterpret_cast<int*>(p.map + (long long)uu * p.nb + j), __float_as_int(v));
         }
       }
 #ifdef SEER_TRACE
