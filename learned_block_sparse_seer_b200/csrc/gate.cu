@@ -12,7 +12,8 @@
 //   pool_kernel      Q avg-pool / K [max|min|avg]-pool, one warp per block,
 //                    16-byte vector loads, shuffle reductions
 //   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections and the causal
-//                    block logits q~ k~^T / sqrt(d) (upper tiles skipped)
+//                    block logits q~ k~^T / sqrt(d) (upper tiles skipped);
+//                    gemm_nt128_kernel is its 128 x 128-tile form for K % 16 == 0
 //   rope_kernel      optional block-level RoPE on q~ / k~
 //   row_select_kernel  one CTA per score row: causal softmax (Eq. 1), optional
 //                    score write-out, then threshold compaction or exact top-k
@@ -165,6 +166,107 @@ __global__ void __launch_bounds__(256) gemm_nt_kernel(const float* __restrict__ 
     for (int q = 0; q < 4; ++q) {
       const int gn = tn * 64 + tx * 4 + q;
       if (gn < N) Cb[(long long)gm * ldc + gn] = alpha * acc[p][q];
+    }
+  }
+}
+
+// The same product with 128 x 128 tiles, for K % 16 == 0 and 16-byte aligned
+// A/B rows: 256 threads, each owning an 8 x 8 block of outputs (rows
+// 4*ty + {0..3} and 64 + 4*ty + {0..3}, columns likewise with tx), so every
+// k step takes four 16-byte shared loads for 64 FMAs.  k slices of 16 are
+// staged transposed ([k][m]) in two shared buffers; the next slice's global
+// loads are in flight while the current one is multiplied.
+template <bool CAUSAL>
+__global__ void __launch_bounds__(256, 1) gemm_nt128_kernel(const float* __restrict__ A,
+                                                            const float* __restrict__ B,
+                                                            float* __restrict__ C, int M, int N, int K,
+                                                            long long a_bs, long long b_bs,
+                                                            long long c_bs, int ldc, int zh, int zmul,
+                                                            int zg, float alpha) {
+  const int tm = blockIdx.x, tn = blockIdx.y, z = blockIdx.z;
+  if (CAUSAL && tn > tm) return;
+  const float* Ab = A + z * a_bs;
+  const int bz = (z / zh) * zmul + (z % zh) / zg;
+  const float* Bb = B + bz * b_bs;
+  float* Cb = C + z * c_bs;
+  __shared__ __align__(16) float As[2][16][132];
+  __shared__ __align__(16) float Bs[2][16][132];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // this thread's two 16-byte global loads per operand and slice: float4
+  // f = tid + 256 s covers row f / 4, k offset 4 * (f % 4)
+  float4 ra[2], rb[2];
+  auto gload = [&](int k0) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int f = tid + 256 * s, r = f >> 2, kq = (f & 3) * 4;
+      const int gm = tm * 128 + r, gn = tn * 128 + r;
+      ra[s] = gm < M ? *reinterpret_cast<const float4*>(Ab + (long long)gm * K + k0 + kq)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      rb[s] = gn < N ? *reinterpret_cast<const float4*>(Bb + (long long)gn * K + k0 + kq)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto sstore = [&](int buf) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int f = tid + 256 * s, r = f >> 2, kq = (f & 3) * 4;
+      As[buf][kq][r] = ra[s].x;
+      As[buf][kq + 1][r] = ra[s].y;
+      As[buf][kq + 2][r] = ra[s].z;
+      As[buf][kq + 3][r] = ra[s].w;
+      Bs[buf][kq][r] = rb[s].x;
+      Bs[buf][kq + 1][r] = rb[s].y;
+      Bs[buf][kq + 2][r] = rb[s].z;
+      Bs[buf][kq + 3][r] = rb[s].w;
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  gload(0);
+  sstore(0);
+  __syncthreads();
+  const int nk = K / 16;
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) gload((kt + 1) * 16);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
+    }
+    // the other buffer was last read in the previous slice, before the
+    // barrier that ended it
+    if (kt + 1 < nk) sstore(buf ^ 1);
+    __syncthreads();
+  }
+  const bool vec = (ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(Cb) & 15) == 0;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int gm = tm * 128 + (p >> 2) * 64 + ty * 4 + (p & 3);
+    if (gm >= M) continue;
+    float* crow = Cb + (long long)gm * ldc;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int gn = tn * 128 + h * 64 + tx * 4;
+      if (vec && gn + 3 < N) {
+        *reinterpret_cast<float4*>(crow + gn) = make_float4(alpha * acc[p][4 * h], alpha * acc[p][4 * h + 1],
+                                                            alpha * acc[p][4 * h + 2], alpha * acc[p][4 * h + 3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (gn + q < N) crow[gn + q] = alpha * acc[p][4 * h + q];
+      }
     }
   }
 }
@@ -502,6 +604,16 @@ cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, i
 cudaError_t launch_gemm_nt(const float* A, const float* B, float* C, int M, int N, int K,
                            long long a_bs, long long b_bs, long long c_bs, int ldc, int batch,
                            int zh, int zmul, int zg, float alpha, bool causal, cudaStream_t st) {
+  const bool big = K % 16 == 0 && a_bs % 4 == 0 && b_bs % 4 == 0 && (reinterpret_cast<uintptr_t>(A) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(B) & 15) == 0;
+  if (big) {
+    dim3 grid((M + 127) / 128, (N + 127) / 128, batch);
+    if (causal)
+      gemm_nt128_kernel<true><<<grid, 256, 0, st>>>(A, B, C, M, N, K, a_bs, b_bs, c_bs, ldc, zh, zmul, zg, alpha);
+    else
+      gemm_nt128_kernel<false><<<grid, 256, 0, st>>>(A, B, C, M, N, K, a_bs, b_bs, c_bs, ldc, zh, zmul, zg, alpha);
+    return cudaGetLastError();
+  }
   dim3 grid((M + 63) / 64, (N + 63) / 64, batch);
   if (causal)
     gemm_nt_kernel<true><<<grid, 256, 0, st>>>(A, B, C, M, N, K, a_bs, b_bs, c_bs, ldc, zh, zmul,
