@@ -542,6 +542,191 @@ __global__ void __launch_bounds__(NT) row_select_kernel(
   if (tid == 0) counts[row] = total;
 }
 
+// The same selection with one warp per row, for rows of at most 32 * NPL
+// candidates and many rows (the prefill gate): a row's values stay in the
+// lanes' registers (local candidate j = 32 t + lane in v[t]), reductions are
+// warp shuffles, the radix histogram is the warp's own 256 shared bins, and
+// the ascending lists are compacted with ballots, so no CTA barrier is
+// taken.  The softmax multiplies by the reciprocal of the row sum; the key
+// order, ties to the lower j, the forced diagonal and varlen windows follow
+// row_select_kernel.
+constexpr int kSelWarps = 8;
+constexpr int kSelNPL = 64;  // rows of up to 2048 candidates
+template <bool FROM_LOGITS>
+__global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
+    const float* in, float* scores, long long rows, int nb, int mode_flags, float T, int k, float density,
+    int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len, const int2* __restrict__ tab) {
+  constexpr int NPL = kSelNPL;
+  __shared__ uint32_t hist_all[kSelWarps][256];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSelWarps + wid;
+  if (row >= rows) return;  // whole warps only: no CTA barrier follows
+  uint32_t* const hist = hist_all[wid];
+  const unsigned lt = (1u << lane) - 1u;
+
+  const int mode = mode_flags & 0xff;
+  const bool force_diag = (mode_flags & SEER_SELECT_FORCE_DIAGONAL) != 0;
+  const int ig = row_len > 0 ? row_len - 1 : (int)(row % nb);
+  const int off = tab ? tab[ig].x : 0;
+  float* const dst = (FROM_LOGITS && scores != nullptr) ? scores + row * (long long)nb : nullptr;
+  if (off < 0) {
+    if (dst)
+      for (int j = lane; j < nb; j += 32) dst[j] = 0.f;
+    if (lane == 0) counts[row] = 0;
+    return;
+  }
+  const int i = ig - off;
+  const int len = i + 1;
+  const int nt = (len + 31) >> 5;  // register slots in use
+  const float* src = in + row * (long long)nb + off;
+  // Every loop over the register slots stops at the row's last slot (a
+  // warp-uniform exit), so short rows cost little.
+  float v[NPL];
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    if (t >= nt) break;
+    const int j = 32 * t + lane;
+    v[t] = j < len ? src[j] : -INFINITY;
+  }
+  if (FROM_LOGITS) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      if (t >= nt) break;
+      m = fmaxf(m, v[t]);
+    }
+    m = warp_max(m);
+    float sum = 0.f;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      if (t >= nt) break;
+      v[t] = expf(v[t] - m);  // exp(-inf) = 0 past the row's end
+      sum += v[t];
+    }
+    const float inv = 1.0f / warp_sum(sum);
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      if (t >= nt) break;
+      v[t] *= inv;
+    }
+    if (dst) {
+      // the window off .. off + len - 1 from the registers, zeros elsewhere
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) {
+        if (t >= nt) break;
+        const int j = 32 * t + lane;
+        if (j < len) dst[off + j] = v[t];
+      }
+      for (int j = lane; j < nb; j += 32)
+        if (j < off || j >= off + len) dst[j] = 0.f;
+    }
+  }
+  int32_t* out = indices + row * (long long)cap;
+
+  if (mode == SEER_SELECT_THRESHOLD) {
+    int base = 0;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      if (t >= nt) break;
+      const int j = 32 * t + lane;
+      const bool keep = j < len && (v[t] > T || (force_diag && j == i));
+      const unsigned km = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[base + __popc(km & lt)] = j + off;
+      base += __popc(km);
+    }
+    if (lane == 0) counts[row] = base;
+    return;
+  }
+
+  const int ki = topk_count(i, mode, k, density);
+  if (ki >= len) {
+    for (int j = lane; j < len; j += 32) out[j] = j + off;
+    if (lane == 0) counts[row] = len;
+    return;
+  }
+
+  // The order-preserving keys replace the values (as bit patterns; slots
+  // past the row hold 0 and are never counted).
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    if (t >= nt) break;
+    v[t] = __uint_as_float(32 * t + lane < len ? f2key(v[t]) : 0u);
+  }
+  // Radix select of the ki-th largest key, 8 bits at a time from the top.
+  uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)ki;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
+    __syncwarp();
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) {
+      if (t >= nt) break;
+      const uint32_t kt = __float_as_uint(v[t]);
+      // not counted: past the row, or outside the prefix chosen so far
+      const uint32_t bin = (32 * t + lane < len && (kt & pmask) == prefix) ? (kt >> shift) & 0xffu : 0x100u;
+      // scores of a row share their top bits: lanes with the same bin are
+      // counted by one atomic
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0x100u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+    __syncwarp();
+    // lane l owns bins 255-8l .. 248-8l (descending)
+    uint32_t cnt[8], part = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cnt[q] = hist[255 - 8 * lane - q];
+      part += cnt[q];
+    }
+    uint32_t incl = part;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - part;
+    uint32_t sel_bin = 0, sel_rem = 0;
+    const bool mine = excl < remaining && remaining <= incl;
+    if (mine) {
+      uint32_t before = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (before < remaining && remaining <= before + cnt[q]) {
+          sel_bin = (uint32_t)(255 - 8 * lane - q);
+          sel_rem = remaining - before;
+        }
+        before += cnt[q];
+      }
+    }
+    const int owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    sel_bin = __shfl_sync(0xffffffffu, sel_bin, owner);
+    sel_rem = __shfl_sync(0xffffffffu, sel_rem, owner);
+    prefix |= sel_bin << shift;
+    remaining = sel_rem;
+    pmask |= 0xffu << shift;
+    __syncwarp();  // the bins are cleared again only after every lane read them
+  }
+  // keys > prefix are all kept; of the keys == prefix the `remaining` ones
+  // with the lowest j; the diagonal joins when forced
+  int base = 0;
+  uint32_t eq_before = 0;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    if (t >= nt) break;
+    const int j = 32 * t + lane;
+    const uint32_t kt = __float_as_uint(v[t]);
+    const bool eq = j < len && kt == prefix;
+    const unsigned em = __ballot_sync(0xffffffffu, eq);
+    const uint32_t rank = eq_before + __popc(em & lt);
+    eq_before += __popc(em);
+    const bool keep = j < len && (kt > prefix || (eq && rank < remaining) || (force_diag && j == i));
+    const unsigned km = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[base + __popc(km & lt)] = j + off;
+    base += __popc(km);
+  }
+  if (lane == 0) counts[row] = base;
+}
+
 // ---------------------------------------------------------- varlen table --
 // Packed variable-length prefill: sequence s occupies tokens
 // start[s] .. start[s] + len[s] - 1 of the packed buffer, start[s] a multiple
@@ -655,6 +840,14 @@ cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, 
   // Few rows (the decode gate, small batches) leave most SMs idle and each
   // row's latency exposed: then 1024 threads share a row's work.
   const bool wide = rows < 2LL * 148;
+  // Many rows of at most 2048 candidates: one warp per row
+  if (!wide && rows >= 8LL * 148 && nb <= 32 * kSelNPL && (row_len > 0 ? row_len : nb) <= 32 * kSelNPL) {
+    const unsigned grid = (unsigned)((rows + kSelWarps - 1) / kSelWarps);
+    auto kern = from_logits ? row_select_warp_kernel<true> : row_select_warp_kernel<false>;
+    kern<<<grid, 32 * kSelWarps, 0, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density, counts,
+                                             indices, cap, row_len, tab);
+    return cudaGetLastError();
+  }
   if (from_logits)
     return wide ? row_select_launch<true, 1024>(in, scores, rows, nb, mode, T, k, density, counts, indices, cap, st,
                                                 row_len, tab)

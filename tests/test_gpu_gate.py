@@ -109,6 +109,41 @@ def test_gate_select_bitexact(nb, ties):
         lists_equal(c.cpu().numpy(), ix.cpu().numpy(), c_ref, i_ref)
 
 
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("B,Hq,nb", [(2, 16, 40), (1, 12, 130), (1, 1, 2048), (1, 1, 2049)])
+def test_gate_select_bitexact_many_rows(B, Hq, nb, ties):
+    """Enough rows for the warp-per-row selection (rows of up to 2048
+    candidates), and a row length one past it (the CTA-per-row kernel), with
+    and without the forced diagonal."""
+    w = synth.custom("sel", B, Hq, 1, 64 * nb, 64, 16, "fp32")
+    s = synth.make_scores_like(w, seed=nb + 7, ties=ties)
+    sd = s.cuda()
+    for fd in (False, True):
+        for mode, kw in (("threshold", dict(T=1.0 / (nb + 1))), ("topk", dict(k=5)),
+                         ("density", dict(density=0.3)), ("density", dict(density=1.0))):
+            c, ix = seer.seer_gate_select(sd, mode, force_diagonal=fd, **kw)
+            torch.cuda.synchronize()
+            mc = seer._lib.mode_code(mode)
+            c_ref, i_ref, _ = oracle.select(s, mc, T=kw.get("T", 0.0), k=kw.get("k", 0),
+                                            density=kw.get("density", 0.0), cap=ix.shape[-1], force_diag=fd)
+            lists_equal(c.cpu().numpy(), ix.cpu().numpy(), c_ref, i_ref)
+
+
+def test_gate_force_diagonal_layer8k():
+    """The whole gate (softmax of the logits, then selection) on 4096 rows with
+    the forced diagonal: bit-exact against the oracle's selection of the GPU's
+    scores, every row holding its diagonal block."""
+    for mode, kw in (("threshold", dict(T=0.02)), ("density", dict(density=0.05))):
+        w, Q, K, Wq, Wk, c, ix, sc = _gate_case("layer8k", mode, force_diagonal=True, **kw)
+        mc = seer._lib.mode_code(mode)
+        c_ref, i_ref, _ = oracle.select(sc, mc, T=kw.get("T", 0.0), density=kw.get("density", 0.0),
+                                        cap=ix.shape[-1], force_diag=True)
+        lists_equal(c, ix, c_ref, i_ref)
+        # ascending lists: the diagonal block is each row's last entry
+        last = np.take_along_axis(ix[0], (c[0] - 1)[..., None].astype(np.int64), axis=-1)[..., 0]
+        assert np.array_equal(last, np.broadcast_to(np.arange(w.nb), last.shape))
+
+
 def test_gate_select_threshold_empty_rows():
     w = synth.custom("sel", 1, 2, 1, 64 * 600, 64, 16, "fp32")
     # uniform rows: 1/(i+1) > 2e-3 only for rows shorter than 500 blocks

@@ -83,6 +83,26 @@ def test_gate_varlen(lens, gaps, mode, kw, fd):
     _lists_equal(c.cpu().numpy(), ix.cpu().numpy(), c_ref, i_ref)
 
 
+@pytest.mark.parametrize("mode,kw", MODES)
+@pytest.mark.parametrize("fd", [False, True])
+def test_gate_varlen_many_rows(mode, kw, fd):
+    """32 query heads over about 40 blocks: enough rows for the warp-per-row
+    selection, with its varlen windows."""
+    lens, gaps = [1000, 700, 65, 300], [0, 2, 1, 0]
+    w, starts, n, Q, K, V, Wq, Wk = _varlen_case(lens, gaps, pad="nan", Hq=32, Hkv=8, d=64)
+    st = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    ln = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    c, ix, sc = seer.seer_gate_varlen(Q.cuda(), K.cuda(), Wq.cuda(), Wk.cuda(), st, ln, mode, return_scores=True,
+                                      force_diagonal=fd, **kw)
+    assert 32 * w.nb >= 8 * 148
+    s = sc.cpu().double().numpy()
+    s_ref = oracle.gate_varlen(Q, K, Wq, Wk, starts, lens)
+    rowmax = np.maximum(s_ref.max(-1, keepdims=True), 1e-30)
+    assert (np.abs(s - s_ref) / rowmax).max() <= SCORE_RTOL
+    c_ref, i_ref = oracle.select_varlen(sc.cpu(), starts, lens, mode, force_diag=fd, cap=ix.shape[-1], **kw)
+    _lists_equal(c.cpu().numpy(), ix.cpu().numpy(), c_ref, i_ref)
+
+
 @pytest.mark.parametrize("dtype,d", [("fp32", 64), ("bf16", 64)])
 def test_gate_varlen_rope_and_dtypes(dtype, d):
     """Block RoPE at packed positions equals the per-sequence oracle's local
