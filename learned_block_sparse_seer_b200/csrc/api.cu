@@ -117,6 +117,21 @@ bool make_tmap_f32_panels(CUtensorMap* tm, const void* base, long long rows, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over a row-major [rows, inner] matrix seen as (64 columns,
+// rows, inner/64 panels): a box of 64 x box_rows x inner/64 lands as
+// inner/64 consecutive 128-byte-swizzled panels of box_rows rows.
+bool make_tmap_bf16_panels(CUtensorMap* tm, const void* base, long long rows, int inner, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(inner / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(inner / 64)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 map over [rows, 64] (128-byte rows) with a box of box_rows rows.
 bool make_tmap_rows(CUtensorMap* tm, const void* base, long long rows, int box_rows) {
   return make_tmap(tm, base, rows, 64, box_rows);
@@ -180,16 +195,20 @@ GateTrainWs gate_train_ws(const seer_dims* d, int h) {
 }
 
 struct AttnWs {
-  size_t q16, kv, redo, total;
+  size_t q16, v16, kt, redo, total;
 };
 
-// fp32 Q converted to bf16 (fp32 inputs only), then the K/V block records
-// (2 * B * Hkv * n * d bf16, K^T and V of each 64-key block together).
+// fp32 Q and V converted to bf16 (fp32 inputs only; bf16 V is read in
+// place), then the K^T block records (B * Hkv * n * d bf16: d rows x 64 keys
+// per 64-key block).
 AttnWs attn_ws(const seer_dims* d, seer_dtype dt) {
   seer::WsCarver c;
-  AttnWs w{0, 0, 0, 0};
-  if (dt == SEER_FP32) w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
-  w.kv = c.take(2ull * 2ull * d->B * d->Hkv * d->n * d->d);
+  AttnWs w{0, 0, 0, 0, 0};
+  if (dt == SEER_FP32) {
+    w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
+    w.v16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+  }
+  w.kt = c.take(2ull * d->B * d->Hkv * d->n * d->d);
   // units flagged for the exact fallback (one int32 per unit at most)
   w.redo = c.take(sizeof(int32_t) * (size_t)d->B * d->Hq * (d->n / seer::kBlock));
   w.total = c.off;
@@ -544,16 +563,18 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   if (s != SEER_OK) return s;
   uint8_t* base = (uint8_t*)ws;
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
-  const void* q = Q;
+  const void *q = Q, *v16 = V;
   if (dtype == SEER_FP32) {
     SEER_CUDA(to_bf16(Q, base + w.q16, (long long)B * Hq * n * d, st));
+    SEER_CUDA(to_bf16(V, base + w.v16, (long long)B * Hkv * n * d, st));
     q = base + w.q16;
+    v16 = base + w.v16;
   }
   const long long records = (long long)B * Hkv * (n / seer::kBlock);
-  SEER_CUDA(seer::launch_kv_tiles(K, V, dtype == SEER_FP32, base + w.kv, records, n, d, st));
-  CUtensorMap tmQ, tmKV;
-  if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) ||
-      !make_tmap_rows(&tmKV, base + w.kv, records * 2 * d, d))
+  SEER_CUDA(seer::launch_kt_tiles(K, dtype == SEER_FP32, base + w.kt, records, n, d, st));
+  CUtensorMap tmQ, tmKt, tmV;
+  if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) || !make_tmap_rows(&tmKt, base + w.kt, records * d, d) ||
+      !make_tmap_bf16_panels(&tmV, v16, (long long)B * Hkv * n, d, 64))
     return cuda_fail(cudaErrorInvalidValue);
   seer::AttnParams p;
   p.B = B;
@@ -585,8 +606,8 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   p.map_scratch = map ? (float*)(base + map_scratch_off) : nullptr;
   if (map) SEER_CUDA(cudaMemsetAsync(map, 0, sizeof(float) * (size_t)p.total_units * p.nb, st));
   if (!dense) SEER_CUDA(seer::launch_empty_rows(p, st));
-  SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKV, p, num_sms(), st));
-  SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kv, p, st));
+  SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKt, tmV, p, num_sms(), st));
+  SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kt, v16, p, st));
   return SEER_OK;
 }
 }  // namespace

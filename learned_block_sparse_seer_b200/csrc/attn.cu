@@ -15,10 +15,12 @@
 //        O^T[d x 64 queries]         += V_pair^T[d x 128] . P^T        (PV)
 //    S^T and O^T live in tensor memory (TMEM); K/V/Q/P^T are 128-byte
 //    swizzled shared-memory tiles.
-//  * A re-layout pass (kv_tile_kernel) first writes every (KV head, key
-//    block) as one contiguous record [K^T: d rows x 64 keys | V: 64 keys x d
-//    in 64-column panels]; a d-row TMA box (16 KB at d = 128, no cluster
-//    multicast) brings either part of a block into shared memory.
+//  * A re-layout pass (kt_tile_kernel) first writes K^T of every (KV head,
+//    key block) as one contiguous record (d rows x 64 keys); one d-row TMA
+//    box (16 KB at d = 128, no cluster multicast) brings it into shared
+//    memory as the MN-major A operand of QK.  V is read in place through a
+//    3-D map (64 dims x 64 keys x d/64 panels): one 16 KB box per block,
+//    landing as 64-dim panels, the MN-major A operand of PV.
 //  * The tensor pipe stalls for about 200 cycles whenever the thread that
 //    issues MMAs synchronises (an mbarrier wait, a shared-memory read, a
 //    barrier), so two warps issue them, each waiting once per pair step on
@@ -292,7 +294,7 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[attn::kCo
 }
 
 // A consumer's walk over the unit ring, one pair step at a time.  next()
-// returns the step's info -- bit 0: two records, bit 1: first step of its
+// returns the step's info -- bit 0: two key blocks, bit 1: first step of its
 // unit, bit 2: last step, bit 3: the unit's Q slot -- or -1 at the end (or on
 // a timeout, which also clears ok).  A ring entry is released as soon as it
 // has been read.
@@ -414,7 +416,8 @@ __device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kC
 // non-negative bit patterns; one partial per warpgroup of 16 columns).
 template <int D, bool MAP>
 __global__ void __launch_bounds__(attn::kThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKt,
+                       const __grid_constant__ CUtensorMap tmV,
                        const AttnParams p) {
   using namespace attn;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -458,9 +461,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     fence_barrier_init();
   }
   if (D == 64) {
-    // With d = 64 a record part is 64 rows (8 KB); the PV product's second
+    // With d = 64 a key block's V is one 8 KB panel; the PV product's second
     // 64-row panel of V^T (head dims 64..127) then reads the zeroed upper
-    // half of each V record slot, which no load ever writes.
+    // half of each block's V slot, which no load ever writes.
     for (int r = 0; r < 2 * kVSlots; ++r) {
       uint4* z = reinterpret_cast<uint4*>(smem + kOffV + r * kHalf + 8192);
       for (int e = threadIdx.x; e < 8192 / 16; e += blockDim.x) z[e] = make_uint4(0, 0, 0, 0);
@@ -481,9 +484,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // ------------------------------- scheduler, Q loads, record gathers --
     if (lane == 0) {
       prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmKV);
-      constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a record's K^T or V part
-      constexpr int rec_rows = 2 * D;
+      prefetch_tmap(&tmKt);
+      prefetch_tmap(&tmV);
+      constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a key block's K^T record, or its V
       int u_idx = 0, qn = 0, h = 0;
       bool ok = true;
       while (ok) {
@@ -517,7 +520,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         if (qn >= kQSlots && !mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo)) break;
         ++qn;
         const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
-        const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;
+        const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;  // this KV head's first K^T record
         // The list entries of the next pair step are read one step early, so
         // that their global-memory latency hides behind this step's waits.
         const int* lst = p.indices + u.u * p.cap;
@@ -551,8 +554,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             for (int pn = 0; pn < dpanels; ++pn)
               tma_load_2d(smem + kOffQ + qs * kQBytes + pn * 8192, &tmQ, tk, pn * 64, qrow);
           for (int t = 0; t < ntile; ++t)
-            tma_load_2d(smem + kOffK + (h % kKSlots) * kPair + t * kHalf, &tmKV, tk, 0,
-                        (int)((rec0 + jj[t]) * rec_rows));
+            tma_load_2d(smem + kOffK + (h % kKSlots) * kPair + t * kHalf, &tmKt, tk, 0, (int)((rec0 + jj[t]) * D));
           // V part: its slot is free once PV(h-3) is complete; it completes go(h).
           if (h >= kVSlots &&
               !SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing], ((h - kVSlots) / kRing) & 1, abort_p,
@@ -562,8 +564,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           }
           mbar_arrive_expect_tx(&bars.go[h % kRing], (uint32_t)ntile * part_bytes);
           for (int t = 0; t < ntile; ++t)
-            tma_load_2d(smem + kOffV + (h % kVSlots) * kPair + t * kHalf, &tmKV, &bars.go[h % kRing], 0,
-                        (int)((rec0 + jj[t]) * rec_rows + D));
+            tma_load_3d(smem + kOffV + (h % kVSlots) * kPair + t * kHalf, &tmV, &bars.go[h % kRing], 0,
+                        (int)((rec0 + jj[t]) * 64), 0);
         }
       }
     }
@@ -880,61 +882,46 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- re-layout --
-// Writes every (batch, KV head, key block j) as one contiguous record of
-// 2*d rows x 64 bf16 (128-byte rows):
-//   rows 0 .. d-1        K^T: row c holds K[64j + 0 .. 63][c]
-//   rows d .. 2d-1       V in 64-column panels: row d + 64p + r holds
-//                        V[64j + r][64p .. 64p + 63]
-// so that one TMA box of 2*d rows gathers K and V of a block at once.
-// fp32 inputs are rounded to bf16 here (round to nearest even).
+// Writes K^T of every (batch, KV head, key block j) as one contiguous record
+// of d rows x 64 bf16 (128-byte rows): row c holds K[64j + 0 .. 63][c].  The
+// block is read with 16-byte loads into a padded shared tile, then written 8
+// keys (16 bytes) per store.  fp32 inputs are rounded to bf16 here (round to
+// nearest even).
 template <typename T>
-__global__ void __launch_bounds__(256) kv_tile_kernel(const T* __restrict__ K, const T* __restrict__ V,
-                                                      __nv_bfloat16* __restrict__ out, int n, int d) {
-  __shared__ __nv_bfloat16 sk[64][128 + 2];
+__global__ void __launch_bounds__(256) kt_tile_kernel(const T* __restrict__ K, __nv_bfloat16* __restrict__ out,
+                                                      int n, int d) {
+  __shared__ uint16_t sk[64][128 + 2];  // [key][dim]; 260-byte rows keep the column reads spread over banks
   const int nb = n / kBlock;
   const long long rec = blockIdx.x;  // (b*Hkv + g)*nb + j
   const long long bg = rec / nb;
   const int j = (int)(rec % nb);
   const T* Kt = K + (bg * n + (long long)j * kBlock) * d;
-  const T* Vt = V + (bg * n + (long long)j * kBlock) * d;
-  __nv_bfloat16* o = out + rec * (2LL * d) * 64;
-  for (int e = threadIdx.x; e < 64 * d; e += blockDim.x) {
-    const int r = e / d, c = e % d;
-    if constexpr (sizeof(T) == 2)
-      sk[r][c] = reinterpret_cast<const __nv_bfloat16*>(Kt)[e];
-    else
-      sk[r][c] = __float2bfloat16_rn(reinterpret_cast<const float*>(Kt)[e]);
+  __nv_bfloat16* o = out + rec * (long long)d * 64;
+  constexpr int EPL = 16 / sizeof(T);  // elements per 16-byte load
+  for (int e = threadIdx.x; e < 64 * d / EPL; e += blockDim.x) {
+    const int r = e / (d / EPL), c = (e % (d / EPL)) * EPL;
+    const uint4 v = *reinterpret_cast<const uint4*>(Kt + (long long)r * d + c);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&sk[r][c]);  // c even: 4-byte aligned
+    if constexpr (sizeof(T) == 2) {
+      dst[0] = v.x;
+      dst[1] = v.y;
+      dst[2] = v.z;
+      dst[3] = v.w;
+    } else {
+      const float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w)};
+      dst[0] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[0])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[1])) << 16);
+      dst[1] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[3])) << 16);
+    }
   }
   __syncthreads();
-  // K^T: 8 keys (16 bytes) per store
   for (int e = threadIdx.x; e < d * 8; e += blockDim.x) {
     const int c = e / 8, k0 = (e % 8) * 8;
     uint32_t w[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t lo = __bfloat16_as_ushort(sk[k0 + 2 * q][c]);
-      const uint32_t hi = __bfloat16_as_ushort(sk[k0 + 2 * q + 1][c]);
-      w[q] = lo | (hi << 16);
-    }
+    for (int q = 0; q < 4; ++q) w[q] = (uint32_t)sk[k0 + 2 * q][c] | ((uint32_t)sk[k0 + 2 * q + 1][c] << 16);
     *reinterpret_cast<uint4*>(o + (long long)c * 64 + k0) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  // V panels: 8 elements (16 bytes) per move
-  for (int e = threadIdx.x; e < 64 * d / 8; e += blockDim.x) {
-    const int r = e / (d / 8), c8 = (e % (d / 8)) * 8;
-    const int pnl = c8 / 64, cc = c8 % 64;
-    uint4 v;
-    if constexpr (sizeof(T) == 2) {
-      v = *reinterpret_cast<const uint4*>(Vt + (long long)r * d + c8);
-    } else {
-      const float* f = reinterpret_cast<const float*>(Vt) + (long long)r * d + c8;
-      uint32_t w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        w[q] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * q])) |
-               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * q + 1])) << 16);
-      v = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    *reinterpret_cast<uint4*>(o + (long long)(d + pnl * 64 + r) * 64 + cc) = v;
   }
 }
 
@@ -961,13 +948,14 @@ __global__ void __launch_bounds__(256) empty_rows_kernel(const int32_t* __restri
 
 // Exact recomputation of the units the attention kernel flagged: plain fp32
 // online softmax that rescales at every key, one warp per query row, lanes
-// splitting the head dimension.  It reads the same bf16 Q and K/V block
-// records as the attention kernel (so fp32 inputs see the same rounding), and
-// the same checked list entries.  Slow by design: it only runs for inputs
+// splitting the head dimension.  It reads the same bf16 Q, K^T records and
+// V as the attention kernel (so fp32 inputs see the same rounding), and the
+// same checked list entries.  Slow by design: it only runs for inputs
 // whose scores rise more than 2^64 above a unit's first-step maximum.
 template <int D>
 __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat16* __restrict__ Q16,
-                                                               const __nv_bfloat16* __restrict__ recs,
+                                                               const __nv_bfloat16* __restrict__ Kt16,
+                                                               const __nv_bfloat16* __restrict__ V16,
                                                                const AttnParams p) {
   constexpr int DL = D / 32;  // head dims per lane
   __shared__ float lse2s[64];  // the unit's row LSEs (log2), for the map
@@ -992,7 +980,8 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
         const int raw = p.dense ? t : lst[t];
         const int j = checked_entry(p, u, raw, prev);
         prev = raw;
-        const __nv_bfloat16* rec = recs + (rec0 + j) * (2LL * D * 64);
+        const __nv_bfloat16* rec = Kt16 + (rec0 + j) * (D * 64LL);  // K^T: [dim][key]
+        const __nv_bfloat16* vb = V16 + (rec0 + j) * (64LL * D);    // V: [key][dim]
         const int kmax = j == u.i ? r : 63;  // causal inside the diagonal block
         for (int key = 0; key <= kmax; ++key) {
           float sdot = 0.f;
@@ -1005,7 +994,7 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
 #pragma unroll
           for (int k = 0; k < DL; ++k) {
             const int dim = lane * DL + k;
-            const float v = __bfloat162float(rec[D * 64 + (dim / 64) * 4096 + key * 64 + (dim % 64)]);
+            const float v = __bfloat162float(vb[key * D + dim]);
             o[k] = o[k] * a + pr * v;
           }
           m = mn;
@@ -1030,7 +1019,7 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
       for (int t = warp; t < u.count; t += 8) {
         int j = p.dense ? t : lst[t];
         j = j < 0 ? 0 : (j > u.i ? u.i : j);
-        const __nv_bfloat16* rec = recs + (rec0 + j) * (2LL * D * 64);
+        const __nv_bfloat16* rec = Kt16 + (rec0 + j) * (D * 64LL);
         float best = 0.f;
         for (int r = 0; r < 64; ++r) {
           const long long qrow = ((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64 + r;
@@ -1052,11 +1041,15 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
   }
 }
 
-cudaError_t launch_sparse_attn_redo(const void* Q16, const void* recs, const AttnParams& p, cudaStream_t st) {
+cudaError_t launch_sparse_attn_redo(const void* Q16, const void* Kt16, const void* V16, const AttnParams& p,
+                                    cudaStream_t st) {
+  const auto q = (const __nv_bfloat16*)Q16;
+  const auto kt = (const __nv_bfloat16*)Kt16;
+  const auto v = (const __nv_bfloat16*)V16;
   if (p.d == 64)
-    sparse_attn_redo_kernel<64><<<148, 256, 0, st>>>((const __nv_bfloat16*)Q16, (const __nv_bfloat16*)recs, p);
+    sparse_attn_redo_kernel<64><<<148, 256, 0, st>>>(q, kt, v, p);
   else
-    sparse_attn_redo_kernel<128><<<148, 256, 0, st>>>((const __nv_bfloat16*)Q16, (const __nv_bfloat16*)recs, p);
+    sparse_attn_redo_kernel<128><<<148, 256, 0, st>>>(q, kt, v, p);
   return cudaGetLastError();
 }
 
@@ -1066,18 +1059,15 @@ cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
-                            int n, int d, cudaStream_t st) {
+cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st) {
   if (fp32)
-    kv_tile_kernel<float><<<(unsigned)records, 256, 0, st>>>((const float*)K, (const float*)V,
-                                                             (__nv_bfloat16*)out, n, d);
+    kt_tile_kernel<float><<<(unsigned)records, 256, 0, st>>>((const float*)K, (__nv_bfloat16*)out, n, d);
   else
-    kv_tile_kernel<uint16_t><<<(unsigned)records, 256, 0, st>>>((const uint16_t*)K, (const uint16_t*)V,
-                                                                (__nv_bfloat16*)out, n, d);
+    kt_tile_kernel<uint16_t><<<(unsigned)records, 256, 0, st>>>((const uint16_t*)K, (__nv_bfloat16*)out, n, d);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
+cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKt, const CUtensorMap& tmV, const AttnParams& p,
                                int num_sms, cudaStream_t st) {
   auto kern = p.map ? (p.d == 64 ? sparse_attn_kernel<64, true> : sparse_attn_kernel<128, true>)
                     : (p.d == 64 ? sparse_attn_kernel<64, false> : sparse_attn_kernel<128, false>);
@@ -1085,7 +1075,7 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, 
   if (e != cudaSuccess) return e;
   long long grid = p.total_units < num_sms ? p.total_units : num_sms;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, attn::kThreads, attn::kSmemAlloc, st>>>(tmQ, tmKV, p);
+  kern<<<(unsigned)grid, attn::kThreads, attn::kSmemAlloc, st>>>(tmQ, tmKt, tmV, p);
   return cudaGetLastError();
 }
 

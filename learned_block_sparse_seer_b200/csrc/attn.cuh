@@ -27,26 +27,28 @@ struct AttnParams {
   float* map_scratch;  // with map: per CTA [nb][2][64] fp32
 };
 
-// Re-layout of K and V into per-block records of 2*d rows x 64 bf16 (K^T,
-// then V in 64-column panels); `records` = B * Hkv * n/64.
-cudaError_t launch_kv_tiles(const void* K, const void* V, bool fp32, void* out, long long records,
-                            int n, int d, cudaStream_t st);
+// Re-layout of K into per-block K^T records of d rows x 64 bf16;
+// `records` = B * Hkv * n/64.
+cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st);
 
 // Exact fp32 recomputation of the units the attention kernel flagged (a
 // score above the unit's first-step column maximum by more than 2^64);
 // returns at once when none was.  Q16 is the bf16 Q the attention kernel
-// read, recs the K/V block records.  Launch after launch_sparse_attn.
-cudaError_t launch_sparse_attn_redo(const void* Q16, const void* recs, const AttnParams& p, cudaStream_t st);
+// read, Kt16 the K^T records and V16 the bf16 V [B*Hkv*n, d].  Launch after
+// launch_sparse_attn.
+cudaError_t launch_sparse_attn_redo(const void* Q16, const void* Kt16, const void* V16, const AttnParams& p,
+                                    cudaStream_t st);
 
 // O = 0 and LSE = -inf for every unit whose list is empty (count <= 0); the
 // attention kernel skips those units.  Launch before launch_sparse_attn.
 cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st);
 
 // Persistent launch: one CTA per SM (at most one per unit).  tmQ is a 2-D
-// bf16 map over Q [rows, d] with 64x64 boxes; tmKV a 2-D bf16 map over the
-// records [records * 2d, 64] with a d-row box (the K^T or the V part of one
-// record); both 128-byte swizzled.
-cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKV, const AttnParams& p,
-                               int num_sms, cudaStream_t st);
+// bf16 map over Q [rows, d] with 64x64 boxes; tmKt a 2-D bf16 map over the
+// K^T records [records * d, 64] with a d-row box; tmV a 3-D bf16 map over V
+// (64 dims, B*Hkv*n rows, d/64 panels) with a 64 x 64 x d/64 box; all
+// 128-byte swizzled.
+cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKt, const CUtensorMap& tmV,
+                               const AttnParams& p, int num_sms, cudaStream_t st);
 
 }  // namespace seer

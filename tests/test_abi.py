@@ -66,10 +66,12 @@ def test_workspace_sizes_cover_their_buffers():
     need = 4 * (B * Hq * nb * d + B * Hkv * nb * 3 * d + B * Hq * nb * h + B * Hkv * nb * h
                 + B * Hq * nb * nb)
     assert g >= need + 256 and g % 256 == 0
-    # bf16: header + the K/V block records (K^T and V of every 64-key block)
-    # + the list of units flagged for the exact fallback (one int32 per unit)
+    # bf16: header + the K^T block records (d rows x 64 keys per 64-key block;
+    # V is read in place) + the list of units flagged for the exact fallback
+    # (one int32 per unit)
     redo = -(-(4 * B * Hq * nb) // 256) * 256
-    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256 + 2 * 2 * B * Hkv * n * d + redo
+    assert seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 0) == 256 + 2 * B * Hkv * n * d + redo
+    # fp32: also bf16 copies of Q and V
     f32 = seer.sparse_attn_workspace_size(B, Hq, Hkv, n, d, 1)
     assert f32 >= 256 + 2 * n * d * (Hq + 2 * Hkv)
     assert seer.blockmax_workspace_size(B, Hq, Hkv, n, d, 0) >= 256 + 4 * 128 * nb
