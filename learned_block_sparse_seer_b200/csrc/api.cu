@@ -158,8 +158,12 @@ cudaError_t to_bf16(const void* x, void* y, long long n, cudaStream_t st) {
 }
 
 struct GateWs {
-  size_t qbar, kbar, qt, kt, logits, total;
+  size_t qbar, kbar, qt, kt, logits, qlo, klo, total;
 };
+
+// The causal logits run on the tensor cores (three tf32 products) when the
+// gate hidden size is a multiple of 32; otherwise on the fp32 SIMT GEMM.
+bool gate_tf32x3(int h) { return h % 32 == 0; }
 
 GateWs gate_ws(const seer_dims* d, int h) {
   const long long nb = d->n / seer::kBlock;
@@ -170,6 +174,9 @@ GateWs gate_ws(const seer_dims* d, int h) {
   w.qt = c.take(sizeof(float) * d->B * d->Hq * nb * h);
   w.kt = c.take(sizeof(float) * d->B * d->Hkv * nb * h);
   w.logits = c.take(sizeof(float) * d->B * d->Hq * nb * nb);
+  // tf32 remainders of q~ and k~ (the tensor-core logits only)
+  w.qlo = gate_tf32x3(h) ? c.take(sizeof(float) * d->B * d->Hq * nb * h) : 0;
+  w.klo = gate_tf32x3(h) ? c.take(sizeof(float) * d->B * d->Hkv * nb * h) : 0;
   w.total = c.off;
   return w;
 }
@@ -449,9 +456,36 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     SEER_CUDA(seer::launch_rope(kt, (long long)B * Hkv * nb, nb, h, rope_theta, st));
   }
   // causal block logits q~_i . k~_j / sqrt(d), KV head of query head z%Hq
-  SEER_CUDA(seer::launch_gemm_nt(qt, kt, logits, nb, nb, h, (long long)nb * h, (long long)nb * h,
-                                 (long long)nb * nb, nb, B * Hq, Hq, Hkv, G,
-                                 (float)(1.0 / std::sqrt((double)d)), true, st));
+  const float alpha = (float)(1.0 / std::sqrt((double)d));
+  if (gate_tf32x3(h)) {
+    float* qlo = (float*)(base + w.qlo);
+    float* klo = (float*)(base + w.klo);
+    SEER_CUDA(seer::launch_split_tf32(qt, qlo, (long long)B * Hq * nb * h, st));
+    SEER_CUDA(seer::launch_split_tf32(kt, klo, (long long)B * Hkv * nb * h, st));
+    CUtensorMap tmAh, tmAl, tmBh, tmBl;
+    if (!make_tmap_f32(&tmAh, qt, (long long)B * Hq * nb, h, 128) ||
+        !make_tmap_f32(&tmAl, qlo, (long long)B * Hq * nb, h, 128) ||
+        !make_tmap_f32(&tmBh, kt, (long long)B * Hkv * nb, h, 128) ||
+        !make_tmap_f32(&tmBl, klo, (long long)B * Hkv * nb, h, 128))
+      return cuda_fail(cudaErrorInvalidValue);
+    seer::Tf32x3Params tp;
+    tp.M = nb;
+    tp.N = nb;
+    tp.K = h;
+    tp.ldc = nb;
+    tp.zh = Hq;
+    tp.zmul = Hkv;
+    tp.zg = G;
+    tp.c_bs = (long long)nb * nb;
+    tp.alpha = alpha;
+    tp.C = logits;
+    tp.status = &((seer::WsHeader*)ws)->status;
+    tp.timeout_ns = kTimeoutNs;
+    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hq, st));
+  } else {
+    SEER_CUDA(seer::launch_gemm_nt(qt, kt, logits, nb, nb, h, (long long)nb * h, (long long)nb * h,
+                                   (long long)nb * nb, nb, B * Hq, Hq, Hkv, G, alpha, true, st));
+  }
   SEER_CUDA(seer::launch_row_select(logits, scores_out, true, (long long)B * Hq * nb, nb, (int)mode,
                                     T, k, density, counts, indices, cap, st, 0, tab));
   return SEER_OK;

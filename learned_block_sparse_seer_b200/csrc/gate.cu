@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "gate.cuh"
 #include "ptx.cuh"
+#include "tf32mma.cuh"
 
 namespace seer {
 
@@ -269,6 +270,166 @@ __global__ void __launch_bounds__(256, 1) gemm_nt128_kernel(const float* __restr
       }
     }
   }
+}
+
+// ------------------------------------------------------ tf32x3 logits --
+// The causal block logits on the tensor cores with fp32-level accuracy: each
+// fp32 operand is split into a tf32 part and its remainder (hi = x rounded
+// to tf32, lo = x - hi, both exact in fp32) and C = alpha (Ah Bh^T + Ah Bl^T
+// + Al Bh^T); the dropped Al Bl^T term and lo's own tf32 rounding leave a
+// relative error near 2^-21 per product.  One CTA per 128 x 128 tile of C
+// (tiles strictly above the diagonal skipped): warp 0 loads 32-column
+// k slices of the four operands by TMA (no cluster multicast) into a
+// 3-stage ring, warp 1 issues the tcgen05 MMAs into a 128-column TMEM
+// accumulator, then all four warps read it back (TMEM lane = tile row).
+void split_tf32_launch(float* x, float* lo, long long n, cudaStream_t st);
+
+__global__ void split_tf32_kernel(float* __restrict__ x, float* __restrict__ lo, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    uint32_t h;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
+    const float hi = __uint_as_float(h);
+    x[i] = hi;
+    lo[i] = v - hi;
+  }
+}
+
+namespace gt3 {
+constexpr int kStages = 3;
+constexpr uint32_t kOp = 128u * 128u;                 // one operand slice: 128 rows x 32 floats
+constexpr uint32_t kStage = 4u * kOp;                 // Ah, Al, Bh, Bl
+constexpr uint32_t kSmem = kStages * kStage + 1024u;  // + slack to align the ring to 1024 bytes
+}  // namespace gt3
+
+__global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmAh,
+                                                             const __grid_constant__ CUtensorMap tmAl,
+                                                             const __grid_constant__ CUtensorMap tmBh,
+                                                             const __grid_constant__ CUtensorMap tmBl,
+                                                             const Tf32x3Params p) {
+  using namespace gt3;
+  const int tm = blockIdx.x, tn = blockIdx.y, z = blockIdx.z;
+  if (tn > tm) return;  // causal: tiles strictly above the diagonal are never read
+  extern __shared__ uint8_t gt3_raw[];
+  uint8_t* const ring = gt3_raw + ((1024u - (smem_u32(gt3_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t full[kStages], empty[kStages], done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_p = &abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int nk = p.K / 32;
+  const int arow = z * p.M + tm * 128;
+  const int bz = (z / p.zh) * p.zmul + (z % p.zh) / p.zg;
+  const int brow = bz * p.N + tn * 128;
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmAh);
+    prefetch_tmap(&tmAl);
+    prefetch_tmap(&tmBh);
+    prefetch_tmap(&tmBl);
+    for (int c = 0; c < nk; ++c) {
+      const int s = c % kStages;
+      if (c >= kStages && !mbar_wait(&empty[s], ((c / kStages) - 1) & 1, abort_p, p.status, p.timeout_ns)) break;
+      mbar_arrive_expect_tx(&full[s], kStage);
+      uint8_t* const st = ring + s * kStage;
+      tma_load_2d(st, &tmAh, &full[s], c * 32, arow);
+      tma_load_2d(st + kOp, &tmAl, &full[s], c * 32, arow);
+      tma_load_2d(st + 2 * kOp, &tmBh, &full[s], c * 32, brow);
+      tma_load_2d(st + 3 * kOp, &tmBl, &full[s], c * 32, brow);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = make_idesc_tf32(128, 128, 0, 0);  // A and B K-major
+    const uint32_t rbase = smem_u32(ring);
+    for (int c = 0; c < nk; ++c) {
+      const int s = c % kStages;
+      if (!mbar_wait(&full[s], (c / kStages) & 1, abort_p, p.status, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint64_t dAh = make_sw128_desc(rbase + s * kStage, 16, 1024);
+      const uint64_t dAl = dAh + (kOp >> 4), dBh = dAh + ((2 * kOp) >> 4), dBl = dAh + ((3 * kOp) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t off = (uint64_t)((kk * 32) >> 4);  // 8 floats = 32 bytes per k step
+        mma_tf32_ss(tmem, dAh + off, dBh + off, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        mma_tf32_ss(tmem, dAh + off, dBl + off, idesc, 1u);
+        mma_tf32_ss(tmem, dAl + off, dBh + off, idesc, 1u);
+      }
+      mma_commit(&empty[s]);
+    }
+    // issued even after a failed wait: it arrives once this thread's MMAs are done
+    mma_commit(&done);
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&done, 0, abort_p, p.status, p.timeout_ns) && *abort_p == 0;
+  tc_fence_after();
+  const int r = warp * 32 + lane;  // TMEM lane = tile row
+  const int gm = tm * 128 + r;
+  float* const crow = p.C + (long long)z * p.c_bs + (long long)gm * p.ldc;
+  const bool vec = (p.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(p.C + (long long)z * p.c_bs) & 15) == 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < 128; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+    tmem_wait_ld();
+    const int gn = tn * 128 + c0;
+    if (ok && gm < p.M && gn < p.N) {
+      if (vec && gn + 32 <= p.N) {
+#pragma unroll
+        for (int q = 0; q < 32; q += 4)
+          *reinterpret_cast<float4*>(crow + gn + q) =
+              make_float4(p.alpha * __uint_as_float(v[q]), p.alpha * __uint_as_float(v[q + 1]),
+                          p.alpha * __uint_as_float(v[q + 2]), p.alpha * __uint_as_float(v[q + 3]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (gn + q < p.N) crow[gn + q] = p.alpha * __uint_as_float(v[q]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 128);
+  // after an abort, loads may still be in flight: let them land before the
+  // shared memory is released
+  if (threadIdx.x == 0 && *abort_p) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+}
+
+void split_tf32_launch(float* x, float* lo, long long n, cudaStream_t st) {
+  split_tf32_kernel<<<1184, 256, 0, st>>>(x, lo, n);
+}
+
+cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
+                                      const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gt3::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.M + 127) / 128, (p.N + 127) / 128, batch);
+  gemm_tf32x3_kernel<<<grid, 128, gt3::kSmem, st>>>(tmAh, tmAl, tmBh, tmBl, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st) {
+  split_tf32_launch(x, lo, n, st);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ rope --

@@ -1,6 +1,7 @@
 // gate.cuh -- host-side launchers of the AttnGate kernels (gate.cu).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/seer.h"
@@ -17,6 +18,23 @@ cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, i
 cudaError_t launch_gemm_nt(const float* A, const float* B, float* C, int M, int N, int K,
                            long long a_bs, long long b_bs, long long c_bs, int ldc, int batch,
                            int zh, int zmul, int zg, float alpha, bool causal, cudaStream_t st);
+
+// The causal logits C[z] = alpha * A[z] B[bz]^T on the tensor cores in three
+// tf32 products (fp32-level accuracy).  A, B are split first: launch_split_tf32
+// rounds x to tf32 in place and writes the remainder to lo.  tmAh/tmAl are
+// fp32 maps over A's hi/lo [batch * M rows, K], tmBh/tmBl over B's
+// [(max bz + 1) * N rows, K], 32 x 128 boxes, 128-byte swizzle.  K % 32 == 0.
+struct Tf32x3Params {
+  int M, N, K, ldc, zh, zmul, zg;
+  long long c_bs;
+  float alpha;
+  float* C;
+  uint32_t* status;
+  unsigned long long timeout_ns;
+};
+cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st);
+cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
+                                      const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st);
 
 // Block-level RoPE with base theta / 64 on x [rows, h] (row position = row % nb).
 cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cudaStream_t st);

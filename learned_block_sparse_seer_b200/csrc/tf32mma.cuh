@@ -1,0 +1,27 @@
+// tf32mma.cuh -- tcgen05 kind::tf32 helpers shared by the tf32 attention and
+// the gate's tensor-core logits product.
+#pragma once
+#include <cstdint>
+
+namespace seer {
+
+// Instruction descriptor for kind::tf32: D f32, A and B tf32 (format 2).
+// a_mn / b_mn select MN-major (1) or K-major (0) operand layouts.
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (+)= A . B^T on tf32 operands read from shared memory (fp32 bit
+// patterns; the tensor core uses their top 19 bits).
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+}  // namespace seer
