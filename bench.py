@@ -189,6 +189,22 @@ def attn_flops(counts, indices, d):
     return 4.0 * d * pairs, total_blocks, diag, 1.0 - total_blocks / causal
 
 
+def launches_per_step(w) -> int:
+    """This library's kernel launches in one timed step (gate, then sparse
+    attention), as the host code issues them for workload w (no RoPE).
+
+    Gate: Q and K pooling (2), the two projections (2), the causal logits
+    (split of q~ and k~ into tf32 parts + the tensor-core product when the
+    gate hidden size is a multiple of 32, else one SIMT GEMM), the softmax
+    and selection (1).  Attention: fp32 inputs first convert Q and V (2); the
+    K^T re-layout (1), the empty-row writer (1), the attention kernel (1)
+    and the exact fallback (1).
+    """
+    gate = 2 + 2 + (3 if w.h % 32 == 0 else 1) + 1
+    attn = (2 if w.dtype == "fp32" else 0) + 4
+    return gate + attn
+
+
 def source_hash(names):
     h = hashlib.sha256()
     for n in names:
@@ -833,7 +849,7 @@ def main():
                          "kernel": "sparse_attn_kernel", "peak_kind": f"bf16 sustained ({pk_kind})",
                          "algorithmic_flops_per_launch": flops},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "gpu_launches": 7 * args.steps,
+            "gpu_launches": launches_per_step(w) * args.steps,
             "blockmax": bmax, "decode": dec, "varlen": vl, "tf32": tf, "dense_context": ctx, "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
