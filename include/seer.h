@@ -17,11 +17,14 @@
  *   seer_sparse_attn_tf32  the attention for fp32 inputs on the tf32 tensor
  *                       cores
  *   seer_gate_noalloc   seer_gate without a workspace
+ *   seer_prefill_host   gate + attention for inputs and outputs in host
+ *                       memory, the copies overlapped with the compute
  *   seer_decode_*       the decode stage: compressed K cache, token gate,
  *                       block-sparse decode attention, 1D ground truth
  *
  * Conventions shared by every call
- *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *  - All tensor pointers are DEVICE pointers owned by the caller (except the
+ *    host tensors of seer_prefill_host, named hQ, hK, hV, hO, hLSE).  The library
  *    allocates no device memory; scratch comes from the caller's workspace,
  *    whose size the matching *_workspace_size() call returns.  Workspace
  *    pointers must be 256-byte aligned.
@@ -433,6 +436,42 @@ SEER_API seer_status seer_decode_blockmax(const seer_dims *dims, const void *q, 
                                          float *lse_out, void *ws, size_t ws_bytes, seer_stream_t stream);
 
 SEER_API size_t seer_decode_blockmax_workspace_size(const seer_dims *dims);
+
+/* ------------------------------------------------------------------------ */
+/* seer_prefill_host -- the whole prefill hot path (seer_gate, then
+ * seer_sparse_attn) for inputs and outputs in host memory, with the
+ * host-device copies overlapped with the compute.
+ *
+ * The layer is processed one KV head's group of query heads (b, g) at a
+ * time: the group's Q, K, V are copied in on a copy stream, its gate and
+ * attention run on `stream`, its O (and LSE) are copied out on a second copy
+ * stream, through two device buffer slots, so that the copy in of group
+ * i + 1 and the copy out of group i - 1 overlap the compute of group i.  The
+ * results are those of seer_gate + seer_sparse_attn on the whole layer
+ * (every step is per head and per query block).
+ *
+ *   hQ [B,Hq,n,d], hK/hV [B,Hkv,n,d]  host memory, dtype (page-locked memory
+ *             gives the overlap; pageable memory works but serialises)
+ *   Wq, Wk    device pointers, as for seer_gate;  h, rope_theta, mode, T, k,
+ *             density as for seer_gate;  scale as for seer_sparse_attn
+ *   hO [B,Hq,n,d] host, dtype;  hLSE [B,Hq,n] host fp32, or NULL
+ *   dbuf      device buffer of at least seer_prefill_host_buffer_size(...)
+ *             bytes, 256-byte aligned (two slots of one group's Q, K, V, O,
+ *             LSE and lists, one gate and one attention workspace)
+ * The call returns when the outputs are in host memory.  It checks every
+ * group's device status words and returns SEER_ERR_TIMEOUT or
+ * SEER_ERR_DEVICE_CHECK if one was set.
+ * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
+ *         SEER_ERR_CUDA, SEER_ERR_TIMEOUT, SEER_ERR_DEVICE_CHECK.            */
+SEER_API seer_status seer_prefill_host(const seer_dims *dims, const void *hQ, const void *hK, const void *hV,
+                                       seer_dtype dtype, const float *Wq, const float *Wk, int32_t h,
+                                       float rope_theta, seer_select_mode mode, float T, int32_t k, float density,
+                                       float scale, void *hO, float *hLSE, void *dbuf, size_t dbuf_bytes,
+                                       seer_stream_t stream);
+
+/* Device buffer bytes seer_prefill_host needs; 0 for invalid arguments. */
+SEER_API size_t seer_prefill_host_buffer_size(const seer_dims *dims, seer_dtype dtype, int32_t h,
+                                              seer_select_mode mode, int32_t k, float density);
 
 /* Synchronises `stream`, reads the device status word at the start of a
  * workspace that a previous call used, and maps it: SEER_OK,

@@ -12,4 +12,5 @@ from ._lib import (  # noqa: F401
     sparse_attn_workspace_size, decode_blockmax_workspace_size, decode_gate_required_cap,
     decode_gate_workspace_size, seer_decode_blockmax,
     seer_decode_gate, seer_decode_kcache_update, seer_sparse_decode_attn, sparse_decode_attn_workspace_size,
+    prefill_host_buffer_size, seer_prefill_host,
 )

@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
         L.seer_gate_kl_backward_workspace_size.restype = SZ
         L.seer_sparse_attn.argtypes = [DP, P, P, P, I32, P, P, I32, F, P, P, P, SZ, P]
         L.seer_sparse_attn.restype = I32
+        L.seer_prefill_host.argtypes = [DP, P, P, P, I32, P, P, I32, F, I32, F, I32, F, F, P, P, P, SZ, P]
+        L.seer_prefill_host.restype = I32
+        L.seer_prefill_host_buffer_size.argtypes = [DP, I32, I32, I32, I32, F]
+        L.seer_prefill_host_buffer_size.restype = SZ
         L.seer_sparse_attn_workspace_size.argtypes = [DP, I32]
         L.seer_sparse_attn_workspace_size.restype = SZ
         L.seer_attn_blockmax.argtypes = [DP, P, P, I32, F, P, P, P, SZ, P]
@@ -308,6 +312,42 @@ def seer_sparse_attn(Q, K, V, counts, indices, scale=0.0, workspace=None, out=No
                                 dt, _ptr(counts), _ptr(indices), int(cap), float(scale), _ptr(O),
                                 _ptr(lse), _ptr(ws), ws.numel(), _stream(dev))
     _check("seer_sparse_attn", st)
+    return O, lse
+
+
+def prefill_host_buffer_size(B, Hq, Hkv, n, d, h, mode, T=0.0, k=0, density=0.0, dtype_code=SEER_BF16,
+                             force_diagonal=False) -> int:
+    return int(lib().seer_prefill_host_buffer_size(ctypes.byref(_dims(B, Hq, Hkv, n, d)), int(dtype_code), int(h),
+                                                   mode_code(mode, force_diagonal), int(k), float(density)))
+
+
+def seer_prefill_host(Q, K, V, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.0, scale=0.0, out=None,
+                      return_lse=True, buffer=None, force_diagonal=False):
+    """seer_gate + seer_sparse_attn for Q/K/V in host memory (page-locked
+    for the copy/compute overlap), the weights on the device.  Returns
+    (O, lse) in host memory once they are there."""
+    for t in (Q, K, V):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("Q, K, V must be contiguous host tensors")
+    dev = _dev(Wq, Wk)
+    B, Hq, n, d = Q.shape
+    Hkv = K.shape[1]
+    h = Wq.shape[1]
+    dt = _dtype_code(Q)
+    mc = mode_code(mode, force_diagonal)
+    if out is None:
+        O = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, pin_memory=True) if return_lse else None
+    else:
+        O, lse = out
+    nbytes = prefill_host_buffer_size(B, Hq, Hkv, n, d, h, mode, T, k, density, dt, force_diagonal)
+    if nbytes == 0:
+        raise ValueError("invalid arguments for seer_prefill_host")
+    buf = _workspace(nbytes, dev, buffer)
+    st = lib().seer_prefill_host(ctypes.byref(_dims(B, Hq, Hkv, n, d)), _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(Wq),
+                                 _ptr(Wk), int(h), float(rope_theta), mc, float(T), int(k), float(density),
+                                 float(scale), _ptr(O), _ptr(lse), _ptr(buf), buf.numel(), _stream(dev))
+    _check("seer_prefill_host", st)
     return O, lse
 
 

@@ -4,6 +4,7 @@
 // memory.
 #include <cmath>
 #include <cstdint>
+#include <vector>
 #include <cstring>
 #include <mutex>
 
@@ -962,6 +963,183 @@ seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const vo
   // it recomputes)
   return run_sparse_attn(dims, Q, K, V, dtype, nullptr, nullptr, 0, scale, O, lse, ws, ws_bytes, stream, true,
                          false, map_out, attn_ws(dims, dtype).total);
+}
+
+// ------------------------------------------------ prefill from host memory --
+// One KV head's group of query heads (b, g) at a time: its Q/K/V are copied
+// in on one stream, its gate and attention run on the caller's stream, its
+// O (and LSE) are copied out on a third, through two buffer slots, so the
+// copies of one group overlap the compute of its neighbours.
+namespace {
+constexpr int kHostSlots = 2;
+
+struct HostPlan {
+  seer_dims g;  // one group: B = 1, Hq = G, Hkv = 1
+  int G = 0, cap = 0, groups = 0;
+  size_t q = 0, kv = 0, o = 0, lse = 0, cnt = 0, idx = 0;       // bytes per slot buffer
+  size_t s_q = 0, s_k = 0, s_v = 0, s_o = 0, s_lse = 0, s_cnt = 0, s_idx = 0, slot = 0;  // offsets in a slot
+  size_t gate_ws = 0, gate_ws_bytes = 0, attn_ws = 0, attn_ws_bytes = 0, status = 0, total = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_mode mode, int32_t k, float density,
+               HostPlan* P) {
+  if (!dims_ok(dims) || (dtype != SEER_BF16 && dtype != SEER_FP32) || h < 1) return false;
+  HostPlan p;
+  p.G = dims->Hq / dims->Hkv;
+  p.groups = dims->B * dims->Hkv;
+  p.g = *dims;
+  p.g.B = 1;
+  p.g.Hq = p.G;
+  p.g.Hkv = 1;
+  p.cap = seer_gate_required_cap(&p.g, mode, k, density);
+  if (p.cap < 1) return false;
+  const size_t es = dtype == SEER_FP32 ? 4 : 2;
+  const size_t n = (size_t)dims->n, d = (size_t)dims->d, nb = n / seer::kBlock;
+  p.q = (size_t)p.G * n * d * es;
+  p.kv = n * d * es;
+  p.o = p.q;
+  p.lse = (size_t)p.G * n * sizeof(float);
+  p.cnt = (size_t)p.G * nb * sizeof(int32_t);
+  p.idx = (size_t)p.G * nb * p.cap * sizeof(int32_t);
+  size_t off = 0;
+  p.s_q = off;
+  off += align256(p.q);
+  p.s_k = off;
+  off += align256(p.kv);
+  p.s_v = off;
+  off += align256(p.kv);
+  p.s_o = off;
+  off += align256(p.o);
+  p.s_lse = off;
+  off += align256(p.lse);
+  p.s_cnt = off;
+  off += align256(p.cnt);
+  p.s_idx = off;
+  off += align256(p.idx);
+  p.slot = off;
+  off = kHostSlots * p.slot;
+  p.gate_ws_bytes = seer_gate_workspace_size(&p.g, h);
+  p.attn_ws_bytes = seer_sparse_attn_workspace_size(&p.g, dtype);
+  if (p.gate_ws_bytes == 0 || p.attn_ws_bytes == 0) return false;
+  p.gate_ws = off;
+  off += align256(p.gate_ws_bytes);
+  p.attn_ws = off;
+  off += align256(p.attn_ws_bytes);
+  p.status = off;  // two device status words per group (gate, attention)
+  off += align256(sizeof(uint32_t) * 2 * (size_t)p.groups);
+  p.total = off;
+  *P = p;
+  return true;
+}
+
+// The streams and events of one call; released however the call ends.
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, copied_in[kHostSlots] = {}, computed[kHostSlots] = {}, copied_out[kHostSlots] = {};
+  ~HostPipe() {
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+    if (start) cudaEventDestroy(start);
+    for (int s = 0; s < kHostSlots; ++s) {
+      if (copied_in[s]) cudaEventDestroy(copied_in[s]);
+      if (computed[s]) cudaEventDestroy(computed[s]);
+      if (copied_out[s]) cudaEventDestroy(copied_out[s]);
+    }
+  }
+  cudaError_t create() {
+    cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+    for (int s = 0; s < kHostSlots && e == cudaSuccess; ++s) {
+      e = cudaEventCreateWithFlags(&copied_in[s], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[s], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&copied_out[s], cudaEventDisableTiming);
+    }
+    return e;
+  }
+};
+}  // namespace
+
+size_t seer_prefill_host_buffer_size(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_mode mode,
+                                     int32_t k, float density) {
+  HostPlan p;
+  return host_plan(dims, dtype, h, mode, k, density, &p) ? p.total : 0;
+}
+
+seer_status seer_prefill_host(const seer_dims* dims, const void* hQ, const void* hK, const void* hV,
+                              seer_dtype dtype, const float* Wq, const float* Wk, int32_t h, float rope_theta,
+                              seer_select_mode mode, float T, int32_t k, float density, float scale, void* hO,
+                              float* hLSE, void* dbuf, size_t dbuf_bytes, seer_stream_t stream) {
+  if (!hQ || !hK || !hV || !hO || !Wq || !Wk) return SEER_ERR_INVALID_ARG;
+  HostPlan P;
+  if (!host_plan(dims, dtype, h, mode, k, density, &P)) return SEER_ERR_INVALID_ARG;
+  if (!dbuf || !aligned(dbuf, 256) || dbuf_bytes < P.total) return SEER_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  HostPipe pipe;
+  SEER_CUDA(pipe.create());
+  // the copy streams start after the work already queued on the caller's stream
+  SEER_CUDA(cudaEventRecord(pipe.start, st));
+  SEER_CUDA(cudaStreamWaitEvent(pipe.in, pipe.start, 0));
+  SEER_CUDA(cudaStreamWaitEvent(pipe.out, pipe.start, 0));
+  uint8_t* const base = (uint8_t*)dbuf;
+  uint32_t* const status = (uint32_t*)(base + P.status);
+  SEER_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t) * 2 * (size_t)P.groups, st));
+  const size_t n = (size_t)dims->n, d = (size_t)dims->d, es = dtype == SEER_FP32 ? 4 : 2;
+  const int Hq = dims->Hq, Hkv = dims->Hkv, G = P.G;
+  seer_status err = SEER_OK;
+  for (int i = 0; i < P.groups && err == SEER_OK; ++i) {
+    const int b = i / Hkv, g = i % Hkv, s = i % kHostSlots;
+    uint8_t* const slot = base + (size_t)s * P.slot;
+    const size_t q_off = ((size_t)b * Hq + (size_t)g * G) * n * d * es;  // this group's first query head
+    const size_t kv_off = ((size_t)b * Hkv + g) * n * d * es;
+    // in: the slot's Q/K/V are free once the compute two groups back is done
+    if (i >= kHostSlots) SEER_CUDA(cudaStreamWaitEvent(pipe.in, pipe.computed[s], 0));
+    SEER_CUDA(cudaMemcpyAsync(slot + P.s_q, (const uint8_t*)hQ + q_off, P.q, cudaMemcpyHostToDevice, pipe.in));
+    SEER_CUDA(cudaMemcpyAsync(slot + P.s_k, (const uint8_t*)hK + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
+    SEER_CUDA(cudaMemcpyAsync(slot + P.s_v, (const uint8_t*)hV + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
+    SEER_CUDA(cudaEventRecord(pipe.copied_in[s], pipe.in));
+    // compute: after the copy in, and once the copy out two groups back has
+    // released the slot's O, LSE and lists
+    SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_in[s], 0));
+    if (i >= kHostSlots) SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_out[s], 0));
+    int32_t* const cnt = (int32_t*)(slot + P.s_cnt);
+    int32_t* const idx = (int32_t*)(slot + P.s_idx);
+    err = seer_gate(&P.g, slot + P.s_q, slot + P.s_k, dtype, Wq + (size_t)g * G * h * d, Wk + (size_t)g * h * 3 * d,
+                    h, rope_theta, mode, T, k, density, nullptr, cnt, idx, P.cap, base + P.gate_ws,
+                    P.gate_ws_bytes, stream);
+    if (err != SEER_OK) break;
+    SEER_CUDA(cudaMemcpyAsync(status + 2 * i, base + P.gate_ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
+    err = seer_sparse_attn(&P.g, slot + P.s_q, slot + P.s_k, slot + P.s_v, dtype, cnt, idx, P.cap, scale,
+                           slot + P.s_o, hLSE ? (float*)(slot + P.s_lse) : nullptr, base + P.attn_ws,
+                           P.attn_ws_bytes, stream);
+    if (err != SEER_OK) break;
+    SEER_CUDA(cudaMemcpyAsync(status + 2 * i + 1, base + P.attn_ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
+    SEER_CUDA(cudaEventRecord(pipe.computed[s], st));
+    // out
+    SEER_CUDA(cudaStreamWaitEvent(pipe.out, pipe.computed[s], 0));
+    SEER_CUDA(cudaMemcpyAsync((uint8_t*)hO + q_off, slot + P.s_o, P.o, cudaMemcpyDeviceToHost, pipe.out));
+    if (hLSE)
+      SEER_CUDA(cudaMemcpyAsync(hLSE + ((size_t)b * Hq + (size_t)g * G) * n, slot + P.s_lse, P.lse,
+                                cudaMemcpyDeviceToHost, pipe.out));
+    SEER_CUDA(cudaEventRecord(pipe.copied_out[s], pipe.out));
+  }
+  // the caller's stream ends after the last copy out (the copy-out stream is in order)
+  const int last = (P.groups - 1) % kHostSlots;
+  SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_out[last], 0));
+  if (err != SEER_OK) {
+    cudaStreamSynchronize(st);
+    return err;
+  }
+  std::vector<uint32_t> words(2 * (size_t)P.groups);
+  SEER_CUDA(cudaMemcpyAsync(words.data(), status, sizeof(uint32_t) * words.size(), cudaMemcpyDeviceToHost, st));
+  SEER_CUDA(cudaStreamSynchronize(st));
+  for (uint32_t w : words)
+    if (w == seer::kDevTimeout) return SEER_ERR_TIMEOUT;
+  for (uint32_t w : words)
+    if (w != seer::kDevOk) return SEER_ERR_DEVICE_CHECK;
+  return SEER_OK;
 }
 
 }  // extern "C"
