@@ -966,18 +966,22 @@ seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const vo
 }
 
 // ------------------------------------------------ prefill from host memory --
-// One KV head's group of query heads (b, g) at a time: its Q/K/V are copied
-// in on one stream, its gate and attention run on the caller's stream, its
-// O (and LSE) are copied out on a third, through two buffer slots, so the
-// copies of one group overlap the compute of its neighbours.
+// The layer is processed in chunks of query heads that share a KV head: each
+// KV head's K and V are copied in once (with its first chunk), each chunk's Q
+// in on a copy stream, its gate and attention run on the caller's stream,
+// its O (and LSE) go out on a third stream.  Two slots for chunks and two
+// for KV heads let the copies of one chunk overlap the compute of its
+// neighbours; small chunks keep the unoverlapped start (first copy in) and
+// end (last compute and copy out) short.
 namespace {
 constexpr int kHostSlots = 2;
 
 struct HostPlan {
-  seer_dims g;  // one group: B = 1, Hq = G, Hkv = 1
-  int G = 0, cap = 0, groups = 0;
-  size_t q = 0, kv = 0, o = 0, lse = 0, cnt = 0, idx = 0;       // bytes per slot buffer
-  size_t s_q = 0, s_k = 0, s_v = 0, s_o = 0, s_lse = 0, s_cnt = 0, s_idx = 0, slot = 0;  // offsets in a slot
+  seer_dims g;  // one chunk: B = 1, Hq = C query heads, Hkv = 1
+  int G = 0, C = 0, cap = 0, chunks = 0, per_kv = 0;
+  size_t q = 0, kv = 0, o = 0, lse = 0, cnt = 0, idx = 0;                        // bytes
+  size_t s_q = 0, s_o = 0, s_lse = 0, s_cnt = 0, s_idx = 0, slot = 0;            // chunk slot layout
+  size_t s_k = 0, s_v = 0, kvslot = 0, kv_base = 0;                              // KV-head slot layout
   size_t gate_ws = 0, gate_ws_bytes = 0, attn_ws = 0, attn_ws_bytes = 0, status = 0, total = 0;
 };
 
@@ -988,28 +992,26 @@ bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_m
   if (!dims_ok(dims) || (dtype != SEER_BF16 && dtype != SEER_FP32) || h < 1) return false;
   HostPlan p;
   p.G = dims->Hq / dims->Hkv;
-  p.groups = dims->B * dims->Hkv;
+  p.C = p.G % 2 == 0 ? p.G / 2 : p.G;  // two chunks per KV head when the group splits evenly
+  p.per_kv = p.G / p.C;
+  p.chunks = dims->B * dims->Hkv * p.per_kv;
   p.g = *dims;
   p.g.B = 1;
-  p.g.Hq = p.G;
+  p.g.Hq = p.C;
   p.g.Hkv = 1;
   p.cap = seer_gate_required_cap(&p.g, mode, k, density);
   if (p.cap < 1) return false;
   const size_t es = dtype == SEER_FP32 ? 4 : 2;
   const size_t n = (size_t)dims->n, d = (size_t)dims->d, nb = n / seer::kBlock;
-  p.q = (size_t)p.G * n * d * es;
+  p.q = (size_t)p.C * n * d * es;
   p.kv = n * d * es;
   p.o = p.q;
-  p.lse = (size_t)p.G * n * sizeof(float);
-  p.cnt = (size_t)p.G * nb * sizeof(int32_t);
-  p.idx = (size_t)p.G * nb * p.cap * sizeof(int32_t);
+  p.lse = (size_t)p.C * n * sizeof(float);
+  p.cnt = (size_t)p.C * nb * sizeof(int32_t);
+  p.idx = (size_t)p.C * nb * p.cap * sizeof(int32_t);
   size_t off = 0;
   p.s_q = off;
   off += align256(p.q);
-  p.s_k = off;
-  off += align256(p.kv);
-  p.s_v = off;
-  off += align256(p.kv);
   p.s_o = off;
   off += align256(p.o);
   p.s_lse = off;
@@ -1019,7 +1021,11 @@ bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_m
   p.s_idx = off;
   off += align256(p.idx);
   p.slot = off;
-  off = kHostSlots * p.slot;
+  p.kv_base = kHostSlots * p.slot;
+  p.s_k = 0;
+  p.s_v = align256(p.kv);
+  p.kvslot = 2 * align256(p.kv);
+  off = p.kv_base + kHostSlots * p.kvslot;
   p.gate_ws_bytes = seer_gate_workspace_size(&p.g, h);
   p.attn_ws_bytes = seer_sparse_attn_workspace_size(&p.g, dtype);
   if (p.gate_ws_bytes == 0 || p.attn_ws_bytes == 0) return false;
@@ -1027,8 +1033,8 @@ bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_m
   off += align256(p.gate_ws_bytes);
   p.attn_ws = off;
   off += align256(p.attn_ws_bytes);
-  p.status = off;  // two device status words per group (gate, attention)
-  off += align256(sizeof(uint32_t) * 2 * (size_t)p.groups);
+  p.status = off;  // two device status words per chunk (gate, attention)
+  off += align256(sizeof(uint32_t) * 2 * (size_t)p.chunks);
   p.total = off;
   *P = p;
   return true;
@@ -1037,26 +1043,26 @@ bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_m
 // The streams and events of one call; released however the call ends.
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
-  cudaEvent_t start = nullptr, copied_in[kHostSlots] = {}, computed[kHostSlots] = {}, copied_out[kHostSlots] = {};
+  cudaEvent_t start = nullptr;
+  cudaEvent_t copied_in[kHostSlots] = {}, computed[kHostSlots] = {}, copied_out[kHostSlots] = {};
+  cudaEvent_t kv_in[kHostSlots] = {}, kv_done[kHostSlots] = {};
   ~HostPipe() {
     if (in) cudaStreamDestroy(in);
     if (out) cudaStreamDestroy(out);
-    if (start) cudaEventDestroy(start);
-    for (int s = 0; s < kHostSlots; ++s) {
-      if (copied_in[s]) cudaEventDestroy(copied_in[s]);
-      if (computed[s]) cudaEventDestroy(computed[s]);
-      if (copied_out[s]) cudaEventDestroy(copied_out[s]);
-    }
+    cudaEvent_t* all[] = {&start};
+    for (cudaEvent_t* e : all)
+      if (*e) cudaEventDestroy(*e);
+    for (int s = 0; s < kHostSlots; ++s)
+      for (cudaEvent_t e : {copied_in[s], computed[s], copied_out[s], kv_in[s], kv_done[s]})
+        if (e) cudaEventDestroy(e);
   }
   cudaError_t create() {
     cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
-    for (int s = 0; s < kHostSlots && e == cudaSuccess; ++s) {
-      e = cudaEventCreateWithFlags(&copied_in[s], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[s], cudaEventDisableTiming);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&copied_out[s], cudaEventDisableTiming);
-    }
+    for (int s = 0; s < kHostSlots && e == cudaSuccess; ++s)
+      for (cudaEvent_t* ev : {&copied_in[s], &computed[s], &copied_out[s], &kv_in[s], &kv_done[s]})
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
     return e;
   }
 };
@@ -1085,54 +1091,67 @@ seer_status seer_prefill_host(const seer_dims* dims, const void* hQ, const void*
   SEER_CUDA(cudaStreamWaitEvent(pipe.out, pipe.start, 0));
   uint8_t* const base = (uint8_t*)dbuf;
   uint32_t* const status = (uint32_t*)(base + P.status);
-  SEER_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t) * 2 * (size_t)P.groups, st));
+  SEER_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t) * 2 * (size_t)P.chunks, st));
   const size_t n = (size_t)dims->n, d = (size_t)dims->d, es = dtype == SEER_FP32 ? 4 : 2;
-  const int Hq = dims->Hq, Hkv = dims->Hkv, G = P.G;
+  const int Hq = dims->Hq, Hkv = dims->Hkv, G = P.G, C = P.C;
   seer_status err = SEER_OK;
-  for (int i = 0; i < P.groups && err == SEER_OK; ++i) {
-    const int b = i / Hkv, g = i % Hkv, s = i % kHostSlots;
+  for (int i = 0; i < P.chunks && err == SEER_OK; ++i) {
+    const int kvi = i / P.per_kv, part = i % P.per_kv;  // KV head (b*Hkv + g) and chunk within it
+    const int b = kvi / Hkv, g = kvi % Hkv, s = i % kHostSlots, t = kvi % kHostSlots;
+    const int hq0 = g * G + part * C;  // first query head of the chunk
     uint8_t* const slot = base + (size_t)s * P.slot;
-    const size_t q_off = ((size_t)b * Hq + (size_t)g * G) * n * d * es;  // this group's first query head
+    uint8_t* const kvs = base + P.kv_base + (size_t)t * P.kvslot;
+    const size_t q_off = ((size_t)b * Hq + hq0) * n * d * es;
     const size_t kv_off = ((size_t)b * Hkv + g) * n * d * es;
-    // in: the slot's Q/K/V are free once the compute two groups back is done
+    if (part == 0) {
+      // K and V of this KV head, once its slot's previous KV head is done
+      if (kvi >= kHostSlots) SEER_CUDA(cudaStreamWaitEvent(pipe.in, pipe.kv_done[t], 0));
+      SEER_CUDA(cudaMemcpyAsync(kvs + P.s_k, (const uint8_t*)hK + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
+      SEER_CUDA(cudaMemcpyAsync(kvs + P.s_v, (const uint8_t*)hV + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
+      SEER_CUDA(cudaEventRecord(pipe.kv_in[t], pipe.in));
+    }
+    // the chunk slot's Q is free once the compute two chunks back is done
     if (i >= kHostSlots) SEER_CUDA(cudaStreamWaitEvent(pipe.in, pipe.computed[s], 0));
     SEER_CUDA(cudaMemcpyAsync(slot + P.s_q, (const uint8_t*)hQ + q_off, P.q, cudaMemcpyHostToDevice, pipe.in));
-    SEER_CUDA(cudaMemcpyAsync(slot + P.s_k, (const uint8_t*)hK + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
-    SEER_CUDA(cudaMemcpyAsync(slot + P.s_v, (const uint8_t*)hV + kv_off, P.kv, cudaMemcpyHostToDevice, pipe.in));
     SEER_CUDA(cudaEventRecord(pipe.copied_in[s], pipe.in));
-    // compute: after the copy in, and once the copy out two groups back has
-    // released the slot's O, LSE and lists
+    // compute: after the copies in, and once the copy out two chunks back
+    // has released the slot's O, LSE and lists
     SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_in[s], 0));
+    SEER_CUDA(cudaStreamWaitEvent(st, pipe.kv_in[t], 0));
     if (i >= kHostSlots) SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_out[s], 0));
     int32_t* const cnt = (int32_t*)(slot + P.s_cnt);
     int32_t* const idx = (int32_t*)(slot + P.s_idx);
-    err = seer_gate(&P.g, slot + P.s_q, slot + P.s_k, dtype, Wq + (size_t)g * G * h * d, Wk + (size_t)g * h * 3 * d,
+    err = seer_gate(&P.g, slot + P.s_q, kvs + P.s_k, dtype, Wq + (size_t)hq0 * h * d, Wk + (size_t)g * h * 3 * d,
                     h, rope_theta, mode, T, k, density, nullptr, cnt, idx, P.cap, base + P.gate_ws,
                     P.gate_ws_bytes, stream);
     if (err != SEER_OK) break;
     SEER_CUDA(cudaMemcpyAsync(status + 2 * i, base + P.gate_ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
-    err = seer_sparse_attn(&P.g, slot + P.s_q, slot + P.s_k, slot + P.s_v, dtype, cnt, idx, P.cap, scale,
+    err = seer_sparse_attn(&P.g, slot + P.s_q, kvs + P.s_k, kvs + P.s_v, dtype, cnt, idx, P.cap, scale,
                            slot + P.s_o, hLSE ? (float*)(slot + P.s_lse) : nullptr, base + P.attn_ws,
                            P.attn_ws_bytes, stream);
     if (err != SEER_OK) break;
     SEER_CUDA(cudaMemcpyAsync(status + 2 * i + 1, base + P.attn_ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st));
     SEER_CUDA(cudaEventRecord(pipe.computed[s], st));
+    if (part == P.per_kv - 1) SEER_CUDA(cudaEventRecord(pipe.kv_done[t], st));
     // out
     SEER_CUDA(cudaStreamWaitEvent(pipe.out, pipe.computed[s], 0));
     SEER_CUDA(cudaMemcpyAsync((uint8_t*)hO + q_off, slot + P.s_o, P.o, cudaMemcpyDeviceToHost, pipe.out));
     if (hLSE)
-      SEER_CUDA(cudaMemcpyAsync(hLSE + ((size_t)b * Hq + (size_t)g * G) * n, slot + P.s_lse, P.lse,
-                                cudaMemcpyDeviceToHost, pipe.out));
+      SEER_CUDA(cudaMemcpyAsync(hLSE + ((size_t)b * Hq + hq0) * n, slot + P.s_lse, P.lse, cudaMemcpyDeviceToHost,
+                                pipe.out));
     SEER_CUDA(cudaEventRecord(pipe.copied_out[s], pipe.out));
   }
-  // the caller's stream ends after the last copy out (the copy-out stream is in order)
-  const int last = (P.groups - 1) % kHostSlots;
-  SEER_CUDA(cudaStreamWaitEvent(st, pipe.copied_out[last], 0));
+  // the caller's stream ends after the last copy out (the copy-out stream is
+  // in order) and after every copy in
+  SEER_CUDA(cudaEventRecord(pipe.start, pipe.out));
+  SEER_CUDA(cudaStreamWaitEvent(st, pipe.start, 0));
+  SEER_CUDA(cudaEventRecord(pipe.start, pipe.in));
+  SEER_CUDA(cudaStreamWaitEvent(st, pipe.start, 0));
   if (err != SEER_OK) {
     cudaStreamSynchronize(st);
     return err;
   }
-  std::vector<uint32_t> words(2 * (size_t)P.groups);
+  std::vector<uint32_t> words(2 * (size_t)P.chunks);
   SEER_CUDA(cudaMemcpyAsync(words.data(), status, sizeof(uint32_t) * words.size(), cudaMemcpyDeviceToHost, st));
   SEER_CUDA(cudaStreamSynchronize(st));
   for (uint32_t w : words)
