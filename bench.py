@@ -689,7 +689,7 @@ def main():
         e2e_ms = reduce_over_ranks(e2e_ms, dev, "max")
         assert torch.equal(hO, O.cpu()), "host-memory path differs from the device path"
         e2e = {"value": whole_job_tflops(flops_all, e2e_ms), "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "call": "seer_prefill_host (copies overlapped with the compute per KV-head group)",
+               "ms_per_step": e2e_ms, "call": "seer_prefill_host (copies overlapped with the compute, per chunk of query heads sharing a KV head)",
                "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * Q.element_size(),
                "d2h_bytes_per_step": O.numel() * O.element_size() + lse.numel() * lse.element_size()}
 
