@@ -77,6 +77,31 @@ def test_workspace_sizes_cover_their_buffers():
     assert seer.blockmax_workspace_size(B, Hq, Hkv, n, d, 0) >= 256 + 4 * 128 * nb
 
 
+def test_prefill_host_buffer_size():
+    """The host-memory call's device buffer: two chunk slots (half a KV-head
+    group of Q, O, LSE and lists each), two KV slots, a gate and an attention
+    workspace for one chunk; 0 for invalid arguments."""
+    B, Hq, Hkv, n, d, h = 1, 32, 8, 8192, 128, 128
+    nb, C = n // 64, 2  # chunk: half of the 4 query heads of a KV head
+    size = seer.prefill_host_buffer_size(B, Hq, Hkv, n, d, h, "density", density=0.1)
+    cap = seer.gate_required_cap(1, C, 1, n, d, "density", density=0.1)
+    slot = 2 * C * n * d * 2 + C * n * 4 + C * nb * 4 + C * nb * cap * 4
+    kv = 2 * n * d * 2
+    ws = seer.gate_workspace_size(1, C, 1, n, d, h) + seer.sparse_attn_workspace_size(1, C, 1, n, d)
+    assert size >= 2 * slot + 2 * kv + ws
+    assert size <= 2 * slot + 2 * kv + ws + 64 * 256 + 4 * B * Hkv * 2 * 2
+    # fp32 inputs need more; the size does not depend on the batch
+    assert seer.prefill_host_buffer_size(B, Hq, Hkv, n, d, h, "density", density=0.1, dtype_code=1) > size
+    assert seer.prefill_host_buffer_size(4, Hq, Hkv, n, d, h, "density", density=0.1) >= size
+    # odd groups are not split
+    odd = seer.prefill_host_buffer_size(1, 3, 1, n, d, h, "topk", k=4)
+    assert odd >= 2 * (2 * 3 * n * d * 2)
+    # invalid: Hq not a multiple of Hkv, a density above 1, a non-positive h
+    assert seer.prefill_host_buffer_size(1, 3, 2, n, d, h, "topk", k=4) == 0
+    assert seer.prefill_host_buffer_size(1, 4, 2, n, d, h, "density", density=1.5) == 0
+    assert seer.prefill_host_buffer_size(1, 4, 2, n, d, 0, "topk", k=4) == 0
+
+
 def test_invalid_arguments_rejected_before_any_launch(L):
     bad = _lib.Dims(1, 3, 2, 512, 128, 64)        # Hq not a multiple of Hkv
     st = L.seer_sparse_attn(ctypes.byref(bad), None, None, None, 0, None, None, 1, 0.0, None,
