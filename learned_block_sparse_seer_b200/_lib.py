@@ -325,7 +325,9 @@ def seer_prefill_host(Q, K, V, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta
                       return_lse=True, buffer=None, force_diagonal=False):
     """seer_gate + seer_sparse_attn for Q/K/V in host memory (page-locked
     for the copy/compute overlap), the weights on the device.  Returns
-    (O, lse) in host memory once they are there."""
+    (O, lse) in host memory once they are there.  Without `out`, page-locked
+    outputs are allocated per call (pinning is slow for large tensors: pass
+    `out` and `buffer` when calling repeatedly)."""
     for t in (Q, K, V):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError("Q, K, V must be contiguous host tensors")
