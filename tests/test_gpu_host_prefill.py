@@ -36,7 +36,8 @@ def _host_path(Q, K, V, Wq, Wk, mode, kw, fd=False, pinned=True, return_lse=True
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,nb,d,dtype", [(2, 8, 2, 40, 128, "bf16"), (1, 4, 4, 37, 64, "bf16"),
-                                                 (1, 6, 2, 24, 128, "fp32"), (3, 2, 1, 9, 64, "bf16")])
+                                                 (1, 6, 2, 24, 128, "fp32"), (3, 2, 1, 9, 64, "bf16"),
+                                                 (2, 1, 1, 1, 64, "bf16"), (1, 3, 1, 130, 128, "bf16")])
 @pytest.mark.parametrize("mode,kw", [("density", dict(density=0.2)), ("threshold", dict(T=0.02)),
                                      ("topk", dict(k=3))])
 def test_matches_device_path_bit_exact(B, Hq, Hkv, nb, d, dtype, mode, kw):
