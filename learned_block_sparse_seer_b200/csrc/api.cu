@@ -1049,9 +1049,7 @@ struct HostPipe {
   ~HostPipe() {
     if (in) cudaStreamDestroy(in);
     if (out) cudaStreamDestroy(out);
-    cudaEvent_t* all[] = {&start};
-    for (cudaEvent_t* e : all)
-      if (*e) cudaEventDestroy(*e);
+    if (start) cudaEventDestroy(start);
     for (int s = 0; s < kHostSlots; ++s)
       for (cudaEvent_t e : {copied_in[s], computed[s], copied_out[s], kv_in[s], kv_done[s]})
         if (e) cudaEventDestroy(e);

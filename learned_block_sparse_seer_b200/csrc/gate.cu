@@ -282,8 +282,6 @@ __global__ void __launch_bounds__(256, 1) gemm_nt128_kernel(const float* __restr
 // k slices of the four operands by TMA (no cluster multicast) into a
 // 3-stage ring, warp 1 issues the tcgen05 MMAs into a 128-column TMEM
 // accumulator, then all four warps read it back (TMEM lane = tile row).
-void split_tf32_launch(float* x, float* lo, long long n, cudaStream_t st);
-
 __global__ void split_tf32_kernel(float* __restrict__ x, float* __restrict__ lo, long long n) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const float v = x[i];
@@ -413,10 +411,6 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
   }
 }
 
-void split_tf32_launch(float* x, float* lo, long long n, cudaStream_t st) {
-  split_tf32_kernel<<<1184, 256, 0, st>>>(x, lo, n);
-}
-
 cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
                                       const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -428,7 +422,7 @@ cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap
 }
 
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st) {
-  split_tf32_launch(x, lo, n, st);
+  split_tf32_kernel<<<1184, 256, 0, st>>>(x, lo, n);
   return cudaGetLastError();
 }
 
