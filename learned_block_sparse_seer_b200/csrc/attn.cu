@@ -65,7 +65,7 @@ namespace seer {
 namespace attn {
 constexpr int kThreads = 608;
 constexpr int kWarpLoad = 16, kWarpPV = 17, kWarpQK = 18;
-constexpr uint32_t kHalf = 16384;              // one record's K^T or V part (d = 128)
+constexpr uint32_t kHalf = 16384;              // one key block's K^T record or V (d = 128)
 constexpr uint32_t kPair = 2 * kHalf;          // the K^T (or V) of a pair step
 constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 3, kQSlots = 1;
 constexpr uint32_t kPBytes = 16384;            // P^T of a pair step: 2 x [64 keys x 64 queries]
