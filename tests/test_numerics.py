@@ -1,0 +1,44 @@
+"""CPU check of the numerical claim behind the gate's tensor-core logits:
+splitting each fp32 operand into a tf32 part (rounded to nearest, 10
+mantissa bits) and its fp32 remainder, and forming hi*hi + hi*lo + lo*hi on
+a tf32 multiplier (which reads the top 19 bits of each operand, truncated or
+rounded), keeps the dot products within about 2^-20 of sum|a b| -- the
+fp32-level accuracy the gate's 1e-4 score tolerance needs.  Plain numpy, no
+GPU; it checks the arithmetic, not the kernel (the GPU tests do that)."""
+import numpy as np
+import pytest
+
+
+def _tf32_round(x):
+    """Round fp32 to the nearest tf32 value (ties away from zero)."""
+    b = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x1000) & 0xFFFFE000
+    return b.astype(np.uint32).view(np.float32)
+
+
+def _tf32_trunc(x):
+    b = x.astype(np.float32).view(np.uint32) & np.uint32(0xFFFFE000)
+    return b.view(np.float32)
+
+
+@pytest.mark.parametrize("read", [_tf32_trunc, _tf32_round])
+def test_three_product_split_keeps_fp32_accuracy(read):
+    rng = np.random.default_rng(0)
+    a = rng.standard_normal((512, 128)).astype(np.float32) * rng.uniform(0.01, 10, (512, 1)).astype(np.float32)
+    b = rng.standard_normal((512, 128)).astype(np.float32)
+    ah = _tf32_round(a)
+    al = (a - ah).astype(np.float32)
+    bh = _tf32_round(b)
+    bl = (b - bh).astype(np.float32)
+    # the remainders are exact in fp32 and small
+    assert np.all(np.abs(al) <= np.abs(a) * 2.0 ** -11 + 1e-45)
+    A, Al, B, Bl = (read(x).astype(np.float64) for x in (ah, al, bh, bl))
+    assert np.array_equal(A, ah.astype(np.float64))  # the tf32 parts pass unchanged
+    approx = A @ B.T + A @ Bl.T + Al @ B.T  # products exact in fp64; accumulation order aside
+    exact = a.astype(np.float64) @ b.astype(np.float64).T
+    scale = np.abs(a).astype(np.float64) @ np.abs(b).astype(np.float64).T
+    rel = np.abs(approx - exact) / scale
+    assert rel.max() <= 2.0 ** -20
+    # one tf32 product alone is about three orders of magnitude worse
+    one = A @ B.T
+    assert (np.abs(one - exact) / scale).max() > 2.0 ** -14
