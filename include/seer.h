@@ -292,23 +292,27 @@ SEER_API size_t seer_blockmax_workspace_size(const seer_dims *dims, seer_dtype d
  *
  * seer_gate's scratch (pooled Q/K, gate vectors, block logits) normally comes
  * from a caller-allocated workspace.  Callers that cannot allocate -- a plugin
- * inside a host framework that owns all device memory, code running while a
- * CUDA graph is being captured (cudaMalloc is not allowed then), or a runtime
- * that forbids allocation after start-up -- call this instead: same inputs and
- * outputs, no workspace argument, and no allocation of any kind.  Its scratch
- * is a static device buffer of SEER_GATE_NOALLOC_MAX_SCRATCH bytes inside the
- * library, which every GPU that loads the library's device code keeps until
- * the process exits.
+ * inside a host framework that owns all device memory and hands out only its
+ * own tensors, or a runtime that forbids device allocation after start-up --
+ * call this instead: same inputs and outputs, no workspace argument, and no
+ * allocation of any kind.  Its scratch is a static device buffer of
+ * SEER_GATE_NOALLOC_MAX_SCRATCH bytes inside the library, which every GPU that
+ * loads the library's device code keeps until the process exits.
  *  - Problems whose scratch (seer_gate_workspace_size) exceeds the buffer are
  *    rejected with SEER_ERR_WORKSPACE before anything is launched (for
  *    example the 8k-token, 32-head layer fits; 32k tokens do not).
+ *  - The device that holds the tensors and the stream must be the current
+ *    device when the call is made: the buffer used is the current device's.
  *  - The first call on each device resolves the buffer's device address
- *    (once, with that device current); make that first call before any stream
- *    capture.  A failure there returns SEER_ERR_CUDA.
+ *    (once, with that device current; again after a device reset); make that
+ *    first call before any stream capture.  A failure there returns
+ *    SEER_ERR_CUDA.
  *  - All calls on a device share the buffer: calls whose work may overlap on
  *    the GPU (different streams without ordering) race and must not be made.
- *  - Device status (seer_workspace_status) is not available for this entry
- *    point; results and errors are otherwise those of seer_gate.          */
+ *  - Device status (seer_workspace_status) cannot be read for this entry
+ *    point.  Instead, if a bounded wait inside the gate gives up, every count
+ *    is set to -1 after the gate has run (indices and scores are then
+ *    unspecified).  Results and errors are otherwise those of seer_gate.   */
 #define SEER_GATE_NOALLOC_MAX_SCRATCH (32u << 20) /* bytes */
 
 SEER_API seer_status seer_gate_noalloc(const seer_dims *dims, const void *Q, const void *K,

@@ -240,7 +240,8 @@ def seer_gate_noalloc(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.
     """seer_gate without a workspace, for callers that cannot allocate device
     memory (their scratch lives in a fixed buffer inside the library; see
     seer_gate_noalloc in include/seer.h for its size limit and sharing rules).
-    Outputs are still passed in (`out`) or allocated here for convenience."""
+    Outputs are still passed in (`out`) or allocated here for convenience.
+    Every count is -1 if a bounded wait on the device gave up."""
     dev = _dev(Q, K, Wq, Wk)
     B, Hq, n, d = Q.shape
     Hkv = K.shape[1]
@@ -256,10 +257,12 @@ def seer_gate_noalloc(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, rope_theta=0.
         scores = torch.empty(B, Hq, nb, nb, dtype=torch.float32, device=dev) if return_scores else None
     else:
         counts, indices, scores = out
-    st = lib().seer_gate_noalloc(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq),
-                                 _ptr(Wk), int(h), float(rope_theta), mc, float(T), int(k),
-                                 float(density), _ptr(scores), _ptr(counts), _ptr(indices),
-                                 int(cap), _stream(dev))
+    # the library's buffer is the current device's: make the tensors' device current
+    with torch.cuda.device(dev):
+        st = lib().seer_gate_noalloc(ctypes.byref(dims), _ptr(Q), _ptr(K), _dtype_code(Q), _ptr(Wq),
+                                     _ptr(Wk), int(h), float(rope_theta), mc, float(T), int(k),
+                                     float(density), _ptr(scores), _ptr(counts), _ptr(indices),
+                                     int(cap), _stream(dev))
     _check("seer_gate_noalloc", st)
     return (counts, indices, scores) if return_scores else (counts, indices)
 

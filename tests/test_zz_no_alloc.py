@@ -1,7 +1,7 @@
 """seer_gate_noalloc: the gate for callers that cannot allocate device memory
-(a plugin inside a framework that owns all device allocations, code running
-during CUDA-graph capture where cudaMalloc is not allowed, runtimes that forbid
-allocation after start-up).  Its scratch is a fixed buffer inside the library.
+(a plugin inside a framework that owns all device allocations and hands out
+only its own tensors, or a runtime that forbids device allocation after
+start-up).  Its scratch is a fixed buffer inside the library.
 
 This file is collected last on purpose.  The test calls the entry point
 through the C ABI and checks it against seer_gate (which uses a caller
@@ -22,7 +22,7 @@ from gpu_common import SCORE_RTOL, inputs
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc_c_abi(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0):
+def _noalloc_c_abi(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0, with_scores=True):
     L = _lib.lib()
     B, Hq, n, d = Q.shape
     Hkv, h, nb = K.shape[1], Wq.shape[1], n // 64
@@ -33,8 +33,10 @@ def _noalloc_c_abi(Q, K, Wq, Wk, mode, T=0.0, k=0, density=0.0):
     idx = torch.full((B, Hq, nb, cap), -7, dtype=torch.int32, device="cuda")
     scores = torch.full((B, Hq, nb, nb), float("nan"), dtype=torch.float32, device="cuda")
     p = lambda t: ctypes.c_void_p(t.data_ptr())
+    # without scores_out the block logits stay in the library's own buffer
+    sp = p(scores) if with_scores else None
     st = L.seer_gate_noalloc(ctypes.byref(dims), p(Q), p(K), _lib._dtype_code(Q), p(Wq), p(Wk), h,
-                             0.0, mc, T, k, density, p(scores), p(counts), p(idx), cap,
+                             0.0, mc, T, k, density, sp, p(counts), p(idx), cap,
                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     torch.cuda.synchronize()
     return st, counts.cpu().numpy(), idx.cpu().numpy(), scores.cpu().double().numpy()
@@ -48,14 +50,19 @@ def test_noalloc_matches_workspace_gate_on_two_calls(name, mode, kw):
     c_ref, i_ref, s_ref = seer.seer_gate(Qd, Kd, Wqd, Wkd, mode, return_scores=True, **kw)
     c_ref, i_ref = c_ref.cpu().numpy(), i_ref.cpu().numpy()
     s_ref = s_ref.cpu().double().numpy()
-    for _ in range(2):
-        st, c, ix, sc = _noalloc_c_abi(Qd, Kd, Wqd, Wkd, mode, **kw)
+    # two calls in a row with the logits going to the caller's tensor, then two
+    # that keep them in the library's buffer (scores_out = NULL)
+    for with_scores in (True, True, False, False):
+        st, c, ix, sc = _noalloc_c_abi(Qd, Kd, Wqd, Wkd, mode, with_scores=with_scores, **kw)
         assert st == 0, _lib.STATUS_NAMES.get(st, st)
         np.testing.assert_array_equal(c, c_ref)
         for r in zip(*np.nonzero(c_ref)):
             np.testing.assert_array_equal(ix[r][:c_ref[r]], i_ref[r][:c_ref[r]])
-        rowmax = np.maximum(s_ref.max(-1, keepdims=True), 1e-300)
-        assert np.max(np.abs(sc - s_ref) / rowmax) <= SCORE_RTOL
+        if with_scores:
+            rowmax = np.maximum(s_ref.max(-1, keepdims=True), 1e-300)
+            assert np.max(np.abs(sc - s_ref) / rowmax) <= SCORE_RTOL
+        else:
+            assert np.isnan(sc).all()  # nothing was written to the unused tensor
 
 
 def test_noalloc_rejects_problems_above_its_buffer():
