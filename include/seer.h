@@ -36,8 +36,11 @@
  *  - Device-side failures (a bounded wait that gave up, an index that failed a
  *    bounds check) are recorded in a status word at the start of the
  *    workspace.  seer_workspace_status() synchronises `stream` and reads it.
- *  - The library keeps no global state and is safe to call from several host
- *    threads on different streams (each call with its own workspace).
+ *  - The library keeps no global state (except the per-thread copy streams of
+ *    seer_prefill_host, the fixed buffer of seer_gate_noalloc and the
+ *    per-thread test hook seer_testing_attn_wait_fault) and is safe to call
+ *    from several host threads on different streams (each call with its own
+ *    workspace).
  *  - The block size is fixed at 64 tokens (the pages fix B = 64 in all
  *    experiments: summary page, section 3.4, "Key Configuration Summary").
  */
@@ -464,7 +467,10 @@ SEER_API size_t seer_decode_blockmax_workspace_size(const seer_dims *dims);
  *             LSE and lists, one gate and one attention workspace)
  * The call returns when the outputs are in host memory.  It checks every
  * group's device status words and returns SEER_ERR_TIMEOUT or
- * SEER_ERR_DEVICE_CHECK if one was set.
+ * SEER_ERR_DEVICE_CHECK if one was set.  The two copy streams and their
+ * events are made on the first call of each host thread on each device and
+ * kept until the thread exits (this is the one piece of state the library
+ * keeps between calls).
  * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,
  *         SEER_ERR_CUDA, SEER_ERR_TIMEOUT, SEER_ERR_DEVICE_CHECK.            */
 SEER_API seer_status seer_prefill_host(const seer_dims *dims, const void *hQ, const void *hK, const void *hV,
@@ -491,6 +497,19 @@ SEER_API int32_t seer_last_cuda_error(void);
 
 /* Library version, e.g. "0.1.0". */
 SEER_API const char *seer_version(void);
+
+/* seer_testing_attn_wait_fault -- a test hook for the failure path of the
+ * attention kernels' bounded waits (no counterpart in the pages: it exists so
+ * that the timeout path can be exercised without faulting or hanging a GPU).
+ * After this call, seer_sparse_attn calls made on the same host thread leave
+ * out the completion signal of QK step `step` (counted from 0 in every CTA of
+ * the persistent kernel) and bound each of their waits by `wait_limit_ns`
+ * (0 keeps the default of 2 s).  The waits that depend on the missing signal
+ * then give up: the kernel unwinds (every bulk copy it issued lands before
+ * it exits), SEER_ERR_TIMEOUT is recorded in the workspace status word, and
+ * the device stays usable.  `step` < 0 turns the hook off (the default).
+ * Outputs of a call made with the hook on are unspecified.               */
+SEER_API void seer_testing_attn_wait_fault(int32_t step, uint64_t wait_limit_ns);
 
 #ifdef __cplusplus
 }

@@ -114,6 +114,8 @@ def lib() -> ctypes.CDLL:
         L.seer_status_string.restype = ctypes.c_char_p
         L.seer_last_cuda_error.restype = I32
         L.seer_version.restype = ctypes.c_char_p
+        L.seer_testing_attn_wait_fault.argtypes = [I32, ctypes.c_uint64]
+        L.seer_testing_attn_wait_fault.restype = None
         _lib = L
     return _lib
 

@@ -7,6 +7,7 @@
 #include <vector>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -14,6 +15,7 @@
 #include "../../include/seer.h"
 #include "attn.cuh"
 #include "blockmax.cuh"
+#include "fwd.cuh"
 #include "gate_train.cuh"
 #include "decode.cuh"
 #include "attn_tf32.cuh"
@@ -24,6 +26,9 @@
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
+// seer_testing_attn_wait_fault's settings for this host thread
+thread_local int32_t g_test_skip_qk_commit = -1;
+thread_local unsigned long long g_test_wait_limit_ns = 0;
 
 seer_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int32_t)e;
@@ -259,6 +264,11 @@ extern "C" {
 const char* seer_version(void) { return "0.1.0"; }
 
 int32_t seer_last_cuda_error(void) { return g_last_cuda_error; }
+
+void seer_testing_attn_wait_fault(int32_t step, uint64_t wait_limit_ns) {
+  g_test_skip_qk_commit = step < 0 ? -1 : step;
+  g_test_wait_limit_ns = wait_limit_ns;
+}
 
 const char* seer_status_string(seer_status s) {
   switch (s) {
@@ -608,7 +618,8 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   const long long records = (long long)B * Hkv * (n / seer::kBlock);
   SEER_CUDA(seer::launch_kt_tiles(K, dtype == SEER_FP32, base + w.kt, records, n, d, st));
   CUtensorMap tmQ, tmKt, tmV;
-  if (!make_tmap(&tmQ, q, (long long)B * Hq * n, d, 64) || !make_tmap_rows(&tmKt, base + w.kt, records * d, d) ||
+  if (!make_tmap_bf16_panels(&tmQ, q, (long long)B * Hq * n, d, 64) ||
+      !make_tmap_rows(&tmKt, base + w.kt, records * d, d) ||
       !make_tmap_bf16_panels(&tmV, v16, (long long)B * Hkv * n, d, 64))
     return cuda_fail(cudaErrorInvalidValue);
   seer::AttnParams p;
@@ -639,6 +650,9 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   p.redo_cap = (int)p.total_units;
   p.map = map;
   p.map_scratch = map ? (float*)(base + map_scratch_off) : nullptr;
+  p.test_skip_qk_commit = g_test_skip_qk_commit;
+  p.k_rows = 0;
+  if (g_test_wait_limit_ns) p.timeout_ns = g_test_wait_limit_ns;
   if (map) SEER_CUDA(cudaMemsetAsync(map, 0, sizeof(float) * (size_t)p.total_units * p.nb, st));
   if (!dense) SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKt, tmV, p, num_sms(), st));
@@ -947,22 +961,119 @@ seer_status seer_decode_blockmax(const seer_dims* dims, const void* q, const voi
 }
 
 // --------------------------------------------------- training forward ----
+namespace {
+// The training forward's workspace: bf16 copies of fp32 inputs, the exact
+// fallback's unit list, then the map scratch of every CTA ([nb][2][128] fp32).
+struct FwdWs {
+  size_t q16, k16, v16, redo, r, total;
+  int ctas;
+};
+
+FwdWs fwd_ws(const seer_dims* d, seer_dtype dt, int sms) {
+  seer::WsCarver c;
+  FwdWs w{0, 0, 0, 0, 0, 0, sms};
+  if (dt == SEER_FP32) {
+    w.q16 = c.take(2ull * d->B * d->Hq * d->n * d->d);
+    w.k16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+    w.v16 = c.take(2ull * d->B * d->Hkv * d->n * d->d);
+  }
+  w.redo = c.take(sizeof(int32_t) * (size_t)d->B * d->Hq * (d->n / seer::kBlock));
+  w.r = c.take(sizeof(float) * (size_t)sms * (d->n / seer::kBlock) * 256);
+  w.total = c.off;
+  return w;
+}
+}  // namespace
+
 size_t seer_attn_forward_map_workspace_size(const seer_dims* dims, seer_dtype dtype) {
   if (!dims_ok(dims)) return 0;
-  // the attention workspace, then the map's per-CTA scratch [nb][2][64] fp32
-  return attn_ws(dims, dtype).total + sizeof(float) * (size_t)num_sms() * (dims->n / seer::kBlock) * 128;
+  return fwd_ws(dims, dtype, num_sms()).total;
 }
 
 seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const void* K, const void* V,
                                   seer_dtype dtype, float scale, void* O, float* lse, float* map_out, void* ws,
                                   size_t ws_bytes, seer_stream_t stream) {
   if (!dims_ok(dims) || !Q || !K || !V || !O || !map_out) return SEER_ERR_INVALID_ARG;
-  // one pass: the attention kernel over every causal block, keeping each
-  // (row block, key half, column) score maximum and turning them into the map
-  // at each unit's end (the exact fallback redoes the map rows of the units
-  // it recomputes)
-  return run_sparse_attn(dims, Q, K, V, dtype, nullptr, nullptr, 0, scale, O, lse, ws, ws_bytes, stream, true,
-                         false, map_out, attn_ws(dims, dtype).total);
+  if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
+  seer_status s = dims_supported(dims);
+  if (s != SEER_OK) return s;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16)) return SEER_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  const FwdWs w = fwd_ws(dims, dtype, sms);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = begin_ws(ws, ws_bytes, w.total, st);
+  if (s != SEER_OK) return s;
+  uint8_t* base = (uint8_t*)ws;
+  const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
+  const void *q = Q, *k = K, *v = V;
+  if (dtype == SEER_FP32) {
+    SEER_CUDA(to_bf16(Q, base + w.q16, (long long)B * Hq * n * d, st));
+    SEER_CUDA(to_bf16(K, base + w.k16, (long long)B * Hkv * n * d, st));
+    SEER_CUDA(to_bf16(V, base + w.v16, (long long)B * Hkv * n * d, st));
+    q = base + w.q16;
+    k = base + w.k16;
+    v = base + w.v16;
+  }
+  // one pass over 128-row query tiles: O, LSE and the map (the map's entries
+  // above the diagonal stay 0)
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_tmap_bf16_panels(&tmQ, q, (long long)B * Hq * n, d, 128) ||
+      !make_tmap_bf16_panels(&tmK, k, (long long)B * Hkv * n, d, 128) ||
+      !make_tmap_bf16_panels(&tmV, v, (long long)B * Hkv * n, d, 128))
+    return cuda_fail(cudaErrorInvalidValue);
+  seer::WsHeader* hdr = (seer::WsHeader*)ws;
+  seer::FwdParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n = n;
+  p.d = d;
+  p.nb = n / seer::kBlock;
+  p.G = Hq / Hkv;
+  p.npairs = (p.nb + 1) / 2;
+  p.total_units = (long long)B * Hq * p.npairs;
+  p.O = O;
+  p.out_fp32 = dtype == SEER_FP32;
+  p.lse = lse;
+  p.map = map_out;
+  const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+  p.scale_log2 = (float)(sc * 1.4426950408889634);
+  p.r = (float*)(base + w.r);
+  p.status = &hdr->status;
+  p.work_counter = &hdr->work_counter;
+  p.timeout_ns = kTimeoutNs;
+  p.redo_count = &hdr->work_counter2;
+  p.redo_list = reinterpret_cast<int*>(base + w.redo);
+  p.redo_cap = (int)((long long)B * Hq * p.nb);
+  SEER_CUDA(cudaMemsetAsync(map_out, 0, sizeof(float) * (size_t)B * Hq * p.nb * p.nb, st));
+  SEER_CUDA(seer::launch_fwd(tmQ, tmK, tmV, p, w.ctas, st));
+  // the exact fallback for units whose scores rose far above their first
+  // step's maximum (returns at once when there are none)
+  seer::AttnParams a{};
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n = n;
+  a.d = d;
+  a.nb = p.nb;
+  a.G = p.G;
+  a.cap = p.nb;
+  a.total_units = (long long)B * Hq * p.nb;
+  a.dense = 1;
+  a.O = O;
+  a.lse = lse;
+  a.out_fp32 = p.out_fp32;
+  a.scale_log2 = p.scale_log2;
+  a.status = p.status;
+  a.timeout_ns = kTimeoutNs;
+  a.redo_count = p.redo_count;
+  a.redo_list = p.redo_list;
+  a.redo_cap = p.redo_cap;
+  a.map = map_out;
+  a.test_skip_qk_commit = -1;
+  a.k_rows = 1;
+  SEER_CUDA(seer::launch_sparse_attn_redo(q, k, v, a, st));
+  return SEER_OK;
 }
 
 // ------------------------------------------------ prefill from host memory --
@@ -1040,7 +1151,10 @@ bool host_plan(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_m
   return true;
 }
 
-// The streams and events of one call; released however the call ends.
+// The streams and events of the host-memory pipeline, made once per device
+// and host thread on first use (a call synchronises before it returns, so
+// the calls of one thread never share them concurrently) and released when
+// the thread exits.
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr;
@@ -1064,6 +1178,30 @@ struct HostPipe {
     return e;
   }
 };
+
+constexpr int kMaxPipeDevices = 64;
+
+// This host thread's pipeline on the current device, or null (with *err set).
+HostPipe* host_pipe(cudaError_t* err) {
+  thread_local HostPipe pipes[kMaxPipeDevices];
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxPipeDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  HostPipe& p = pipes[dev];
+  if (!p.in) {
+    *err = p.create();
+    if (*err != cudaSuccess) {
+      p.~HostPipe();
+      new (&p) HostPipe();
+      return nullptr;
+    }
+  }
+  return &p;
+}
 }  // namespace
 
 size_t seer_prefill_host_buffer_size(const seer_dims* dims, seer_dtype dtype, int32_t h, seer_select_mode mode,
@@ -1081,8 +1219,10 @@ seer_status seer_prefill_host(const seer_dims* dims, const void* hQ, const void*
   if (!host_plan(dims, dtype, h, mode, k, density, &P)) return SEER_ERR_INVALID_ARG;
   if (!dbuf || !aligned(dbuf, 256) || dbuf_bytes < P.total) return SEER_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
-  HostPipe pipe;
-  SEER_CUDA(pipe.create());
+  cudaError_t perr = cudaSuccess;
+  HostPipe* pp = host_pipe(&perr);
+  if (!pp) return cuda_fail(perr);
+  HostPipe& pipe = *pp;
   // the copy streams start after the work already queued on the caller's stream
   SEER_CUDA(cudaEventRecord(pipe.start, st));
   SEER_CUDA(cudaStreamWaitEvent(pipe.in, pipe.start, 0));

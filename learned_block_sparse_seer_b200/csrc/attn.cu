@@ -63,27 +63,30 @@
 namespace seer {
 
 namespace attn {
-constexpr int kThreads = 608;
-constexpr int kWarpLoad = 16, kWarpPV = 17, kWarpQK = 18;
+constexpr int kThreads = 640;
+constexpr int kWarpLoadK = 16, kWarpPV = 17, kWarpQK = 18, kWarpLoadV = 19;
 constexpr uint32_t kHalf = 16384;              // one key block's K^T record or V (d = 128)
 constexpr uint32_t kPair = 2 * kHalf;          // the K^T (or V) of a pair step
-constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 3, kQSlots = 1;
+constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 2, kQSlots = 2;
 constexpr uint32_t kPBytes = 16384;            // P^T of a pair step: 2 x [64 keys x 64 queries]
 constexpr uint32_t kQBytes = 16384;            // Q tile: 64 rows x d (two 64-column panels)
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kKSlots * kPair;       //  64 KB
 constexpr uint32_t kOffP = kOffV + kVSlots * kPair;       // 160 KB
-constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 208 KB
+constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 192 KB
 constexpr uint32_t kSmemBytes = kOffQ + kQSlots * kQBytes;  // 224 KB of tiles
-constexpr int kRing = 4;   // go / qk_done / pv_done barriers, indexed by step
+constexpr int kRing = 4;   // kfull / go / qk_done / pv_done barriers, indexed by step
 constexpr int kSBuf = 3;   // S^T buffers in TMEM (QK runs two steps ahead of PV)
-constexpr int kUnits = 8;  // unit ring entries (the loader runs ahead of the consumers)
+constexpr int kUnits = 8;  // unit ring entries (the scheduler runs ahead of the consumers)
 constexpr uint32_t kTmemCols = 256;            // S^T x 3 (64 columns each) + O^T (64)
 constexpr uint32_t kColO = kSBuf * 64;
 constexpr int kWG = 4;     // softmax warpgroups
 constexpr int kCols = 16;  // query columns per warpgroup
 constexpr int kSoftmaxWarps = 4 * kWG;
+// readers of a unit ring entry: both loaders, both MMA warps, every softmax warp
+constexpr int kUnitReaders = 4 + kSoftmaxWarps;
 static_assert(kSBuf < kRing, "kfull(h) takes softmax(h - kSBuf) arrivals");
+static_assert(kVSlots < kRing && kPSlots < kRing && kKSlots < kRing, "slot reuse is tracked on the step rings");
 // A score more than 2^64 above its unit's first-step column maximum (log2
 // domain) sends the unit to the exact fallback kernel.  Below it nothing
 // overflows: P <= 2^64 in bf16, row sums <= 2^81 and O in fp32.
@@ -98,11 +101,10 @@ struct Bars {
   uint64_t q_free[kQSlots];  // the last QK of the unit that used a Q slot is complete
   uint64_t fin_qk, fin_pv;
 };
-// What the loader publishes about each unit: the work index (-1 ends the
+// What the scheduler publishes about each unit: the work index (-1 ends the
 // work), its checked list length, whether its last entry is the diagonal
 // block, and the flat unit index u = (b*Hq + hq)*nb + i (its 64 query rows
-// start at row 64*u of Q and O).  Consumers read only this, never the lists
-// in global memory.
+// start at row 64*u of Q and O).
 struct UnitEntry {
   int w, count, diag, u;
 };
@@ -114,6 +116,10 @@ struct Ctrl {
   uint32_t tmem_base;
   int abort_flag;
   int redo_unit;  // the last unit this CTA flagged for the exact fallback
+  // Teardown accounting after an abort: the steps each loader armed, and the
+  // steps for which each softmax warp made its go / kfull arrivals.
+  int armed_k, armed_v;
+  int sm_steps[kSoftmaxWarps];
   alignas(16) float red[kWG][2][4][kCols];  // read with 16-byte vector loads
 #ifdef SEER_TRACE
   unsigned long long trace[24];
@@ -407,6 +413,32 @@ __device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kC
   *reinterpret_cast<uint4*>(prow + off1) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
+// One unit's list entries, read warp-wide 32 at a time: lane l holds entry
+// base + l (0 past the count).  Dense mode needs no list: entry t is t.
+__device__ __forceinline__ int list_raw(const AttnParams& p, const int* lst, int t, int count) {
+  return t < count ? (p.dense ? t : lst[t]) : 0;
+}
+
+// Checks the lanes' raw entries of one chunk (entry t = base + lane) against
+// their predecessors as read (lane 0's is the previous chunk's last, carried
+// in last_raw); returns this lane's checked entry.
+__device__ __forceinline__ int check_chunk(const AttnParams& p, const UnitInfo& u, int raw, int t, int count,
+                                           int& last_raw, int lane) {
+  int prev = __shfl_up_sync(0xffffffffu, raw, 1);
+  if (lane == 0) prev = last_raw;
+  last_raw = __shfl_sync(0xffffffffu, raw, 31);
+  return t < count ? checked_entry(p, u, raw, prev) : 0;
+}
+
+// Waits (bounded) until the phase of `bar` with the given parity has
+// completed; used only at teardown, so it does not look at the abort flag.
+__device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  return true;
+}
+
 // MAP (the training forward): also the 2D-max-pooled probability map.  Each
 // step every warp takes, per query column, the maximum of its 32 keys'
 // scores (a shuffle reduce-scatter over the lanes = keys) and keeps it in the
@@ -441,13 +473,15 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   if (threadIdx.x == 0) {
     C.abort_flag = 0;
     C.redo_unit = -1;
+    C.armed_k = 0;
+    C.armed_v = 0;
     for (int s = 0; s < kUnits; ++s) {
       mbar_init(&bars.unit_full[s], 1);
-      mbar_init(&bars.unit_empty[s], 2 + kSoftmaxWarps);  // both MMA warps + softmax warps, on reading
+      mbar_init(&bars.unit_empty[s], kUnitReaders);  // released by every reader on reading
     }
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(&bars.kfull[s], 1 + kSoftmaxWarps);  // loader's K^T part + softmax(h-3) done
-      mbar_init(&bars.go[s], 1 + kSoftmaxWarps);     // loader's V part + softmax's P^T(g)
+      mbar_init(&bars.kfull[s], 1 + kSoftmaxWarps);  // K loader's K^T (+Q) part + softmax(h-3) done
+      mbar_init(&bars.go[s], 1 + kSoftmaxWarps);     // V loader's V part + softmax's P^T(g)
       mbar_init(&bars.qk_done[s], 1);
       mbar_init(&bars.pv_done[s], 1);
     }
@@ -460,6 +494,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     mbar_init(&bars.fin_pv, 1);
     fence_barrier_init();
   }
+  if (threadIdx.x < kSoftmaxWarps) C.sm_steps[threadIdx.x] = 0;
   if (D == 64) {
     // With d = 64 a key block's V is one 8 KB panel; the PV product's second
     // 64-row panel of V^T (head dims 64..127) then reads the zeroed upper
@@ -478,96 +513,139 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
-  constexpr int dpanels = D / 64;
+  constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a key block's K^T record, or its V
 
-  if (warp == kWarpLoad) {
-    // ------------------------------- scheduler, Q loads, record gathers --
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmKt);
-      prefetch_tmap(&tmV);
-      constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a key block's K^T record, or its V
-      int u_idx = 0, qn = 0, h = 0;
-      bool ok = true;
-      while (ok) {
-        const int slot = u_idx % kUnits;
-        if (u_idx >= kUnits &&
-            !mbar_wait(&bars.unit_empty[slot], ((u_idx / kUnits) - 1) & 1, abort_p, p.status, tmo))
-          break;
-        // Units with an empty list never enter the ring: their output (O = 0,
-        // LSE = -inf) is written by empty_rows_kernel before this kernel.
-        int w;
-        UnitInfo u{};
-        for (;;) {
-          w = (int)atomicAdd(p.work_counter, 1u);
-          if (w >= p.total_units || *abort_p) {
-            w = -1;
-            break;
-          }
-          u = decode_unit(p, w);
-          if (u.count > 0) break;
-        }
-        // lists are ascending, so only the last entry can be the diagonal block
-        const int diag = w >= 0 ? (p.dense ? 1 : (p.indices[u.u * p.cap + u.count - 1] == u.i)) : 0;
-        C.unit[slot].w = w;
-        C.unit[slot].count = u.count;
-        C.unit[slot].diag = diag;
-        C.unit[slot].u = w >= 0 ? (int)u.u : 0;
-        mbar_arrive(&bars.unit_full[slot]);
-        ++u_idx;
-        if (w < 0) break;
-        const int qs = qn % kQSlots;
-        if (qn >= kQSlots && !mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo)) break;
-        ++qn;
-        const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
-        const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;  // this KV head's first K^T record
-        // The list entries of the next pair step are read one step early, so
-        // that their global-memory latency hides behind this step's waits.
-        const int* lst = p.indices + u.u * p.cap;
-        auto entry = [&](int t) { return p.dense ? t : lst[t]; };
-        int jn0 = entry(0);
-        int jn1 = u.count > 1 ? entry(1) : 0;
-        int prev = -1;
-        for (int m = 0; m < u.count; m += 2, ++h) {
-          const int ntile = m + 1 < u.count ? 2 : 1;
-          const int ra = jn0, rb = jn1;
-          if (m + 2 < u.count) jn0 = entry(m + 2);
-          if (m + 3 < u.count) jn1 = entry(m + 3);
-          int jj[2];
-          jj[0] = checked_entry(p, u, ra, prev);
-          prev = ra;
-          jj[1] = 0;
-          if (ntile == 2) {
-            jj[1] = checked_entry(p, u, rb, prev);
-            prev = rb;
-          }
-          // K^T part: its slot is free once QK(h-2) is complete; it (and the
-          // unit's Q tile on its first step) completes kfull(h).
-          if (h >= 2 && !SEER_TIMED(0, mbar_wait(&bars.qk_done[(h - 2) % kRing], ((h - 2) / kRing) & 1, abort_p,
-                                                 p.status, tmo))) {
-            ok = false;
-            break;
-          }
-          uint64_t* tk = &bars.kfull[h % kRing];
-          mbar_arrive_expect_tx(tk, (uint32_t)ntile * part_bytes + (m == 0 ? 64u * D * 2u : 0u));
-          if (m == 0)
-            for (int pn = 0; pn < dpanels; ++pn)
-              tma_load_2d(smem + kOffQ + qs * kQBytes + pn * 8192, &tmQ, tk, pn * 64, qrow);
-          for (int t = 0; t < ntile; ++t)
-            tma_load_2d(smem + kOffK + (h % kKSlots) * kPair + t * kHalf, &tmKt, tk, 0, (int)((rec0 + jj[t]) * D));
-          // V part: its slot is free once PV(h-3) is complete; it completes go(h).
-          if (h >= kVSlots &&
-              !SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing], ((h - kVSlots) / kRing) & 1, abort_p,
-                                       p.status, tmo))) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&bars.go[h % kRing], (uint32_t)ntile * part_bytes);
-          for (int t = 0; t < ntile; ++t)
-            tma_load_3d(smem + kOffV + (h % kVSlots) * kPair + t * kHalf, &tmV, &bars.go[h % kRing], 0,
-                        (int)((rec0 + jj[t]) * 64), 0);
-        }
+  if (warp == kWarpLoadK || warp == kWarpLoadV) {
+    // ------------------------- loaders: Q + K^T, and V with the scheduler ---
+    // Two warps issue the bulk copies (one instruction per 16 KB box): the
+    // K loader the unit's Q tile and the step's K^T records, the V loader the
+    // step's V blocks.  Each walks the unit ring itself and reads the list
+    // warp-wide, 32 checked entries at a time, the next chunk in flight while
+    // the current one is used.  Lane 0 waits and issues.
+    //
+    // The V loader also schedules: it hands out units by an atomic counter
+    // and publishes them in the unit ring, one unit ahead of its own walk (V
+    // is needed last, so its ring absorbs the scheduling latency).  Units
+    // with an empty list never enter the ring: their output (O = 0, LSE =
+    // -inf) is written by empty_rows_kernel before this kernel.
+    const bool isK = warp == kWarpLoadK;
+    int pub = 0;           // units published (V loader)
+    bool sched_end = isK;  // the end marker is out (or this warp does not schedule)
+    auto publish_one = [&]() {
+      const int slot = pub % kUnits;
+      if (pub >= kUnits &&
+          !mbar_wait(&bars.unit_empty[slot], ((pub / kUnits) - 1) & 1, abort_p, p.status, tmo)) {
+        sched_end = true;
+        return;
       }
+      int w;
+      UnitInfo u{};
+      for (;;) {
+        w = (int)atomicAdd(p.work_counter, 1u);
+        if (w >= p.total_units || *abort_p) {
+          w = -1;
+          break;
+        }
+        u = decode_unit(p, w);
+        if (u.count > 0) break;
+      }
+      // lists are ascending, so only the last entry can be the diagonal block
+      const int diag = w >= 0 ? (p.dense ? 1 : (p.indices[u.u * p.cap + u.count - 1] == u.i)) : 0;
+      C.unit[slot].w = w;
+      C.unit[slot].count = u.count;
+      C.unit[slot].diag = diag;
+      C.unit[slot].u = w >= 0 ? (int)u.u : 0;
+      mbar_arrive(&bars.unit_full[slot]);
+      ++pub;
+      if (w < 0) sched_end = true;  // the end marker is never released: nothing reuses its slot
+    };
+    if (lane == 0) {
+      if (isK) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmKt);
+      } else {
+        prefetch_tmap(&tmV);
+        publish_one();
+        if (!sched_end) publish_one();
+      }
+    }
+    int ur = 0, qn = 0, h = 0;
+    for (;;) {
+      const int slot = ur % kUnits;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(&bars.unit_full[slot], (ur / kUnits) & 1, abort_p, p.status, tmo);
+      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+      const int w = C.unit[slot].w, count = C.unit[slot].count;
+      ++ur;
+      if (w < 0) break;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars.unit_empty[slot]);
+        if (!sched_end) publish_one();
+      }
+      const UnitInfo u = unit_coords(p, w);
+      const int qs = qn % kQSlots;
+      if (isK && qn >= kQSlots) {
+        bool okq = true;
+        if (lane == 0) okq = mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo);
+        if (!__shfl_sync(0xffffffffu, okq, 0)) break;
+      }
+      ++qn;
+      const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
+      const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;  // this KV head's first block
+      const int* lst = p.indices + u.u * p.cap;
+      int raw = list_raw(p, lst, lane, count);
+      int raw_next = list_raw(p, lst, 32 + lane, count);
+      int last_raw = -1, chk = 0;
+      bool ok = true;
+      for (int m = 0; m < count; m += 2, ++h) {
+        const int c = m & 31;
+        if (c == 0) {
+          if (m > 0) {
+            raw = raw_next;
+            raw_next = list_raw(p, lst, m + 32 + lane, count);
+          }
+          chk = check_chunk(p, u, raw, m + lane, count, last_raw, lane);
+        }
+        const int ntile = m + 1 < count ? 2 : 1;
+        const int j0 = __shfl_sync(0xffffffffu, chk, c), j1 = __shfl_sync(0xffffffffu, chk, c + 1);
+        if (lane == 0) {
+          if (isK) {
+            // K^T slot free once QK(h-2) is complete; its copies (and the
+            // unit's Q tile on its first step) complete kfull(h)
+            ok = h < kKSlots || SEER_TIMED(0, mbar_wait(&bars.qk_done[(h - kKSlots) % kRing],
+                                                          ((h - kKSlots) / kRing) & 1, abort_p, p.status, tmo));
+            if (ok) {
+              uint64_t* tk = &bars.kfull[h % kRing];
+              mbar_arrive_expect_tx(tk, (uint32_t)ntile * part_bytes + (m == 0 ? 64u * D * 2u : 0u));
+              if (m == 0) tma_load_3d(smem + kOffQ + qs * kQBytes, &tmQ, tk, 0, qrow, 0);
+              uint8_t* dst = smem + kOffK + (h % kKSlots) * kPair;
+              tma_load_2d(dst, &tmKt, tk, 0, (int)((rec0 + j0) * D));
+              if (ntile == 2) tma_load_2d(dst + kHalf, &tmKt, tk, 0, (int)((rec0 + j1) * D));
+            }
+          } else {
+            // V slot free once PV(h-3) is complete; its copies complete go(h)
+            ok = h < kVSlots || SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing],
+                                                          ((h - kVSlots) / kRing) & 1, abort_p, p.status, tmo));
+            if (ok) {
+              uint64_t* tv = &bars.go[h % kRing];
+              mbar_arrive_expect_tx(tv, (uint32_t)ntile * part_bytes);
+              uint8_t* dst = smem + kOffV + (h % kVSlots) * kPair;
+              tma_load_3d(dst, &tmV, tv, 0, (int)((rec0 + j0) * 64), 0);
+              if (ntile == 2) tma_load_3d(dst + kHalf, &tmV, tv, 0, (int)((rec0 + j1) * 64), 0);
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+    // steps whose copies were issued: the teardown drains them after an abort
+    if (lane == 0) {
+      if (isK)
+        C.armed_k = h;
+      else
+        C.armed_v = h;
     }
   } else if (warp == kWarpQK) {
     // ------------------------------------------------------ QK issuer ----
@@ -598,7 +676,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           mma_bf16_ss(sc, dk + (uint64_t)(kk * 2048 / 16), dq + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) / 16),
                       idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(&bars.qk_done[ring]);
+        // (a test hook can leave out one step's completion signal, so that
+        // the waits on it run into their limit)
+        if (h != p.test_skip_qk_commit) mma_commit(&bars.qk_done[ring]);
         if (info & 4) mma_commit(&bars.q_free[(info >> 3) & 1]);
         ++h;
         kslot = kslot + 1 == kKSlots ? 0 : kslot + 1;
@@ -607,7 +687,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       // this thread's MMAs complete before TMEM is released
       mma_commit(&bars.fin_qk);
-      mbar_wait(&bars.fin_qk, 0, abort_p, nullptr, 20000000ull);
+      mbar_wait_teardown(&bars.fin_qk, 0, 20000000ull);
     }
   } else if (warp == kWarpPV) {
     // ------------------------------------------------------ PV issuer ----
@@ -646,7 +726,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         ring = ring + 1 == kRing ? 0 : ring + 1;
       }
       mma_commit(&bars.fin_pv);
-      mbar_wait(&bars.fin_pv, 0, abort_p, nullptr, 20000000ull);
+      mbar_wait_teardown(&bars.fin_pv, 0, 20000000ull);
     }
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------- softmax WGs ---
@@ -663,6 +743,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     const float c = p.scale_log2;
     const int half = tl >> 6, kl = tl & 63;
     int u_idx = 0, step = 0, red_use = 0;
+    int arrived = 0;  // steps whose go / kfull arrivals this warp has made
+    // Set (warp-uniformly, for good) by the warp's first failed wait: from
+    // then on it makes no barrier arrivals, so that every barrier phase is
+    // only ever completed by real work and the teardown can account for the
+    // arrivals that are missing.
+    bool dead = false;
     // Per query column of this warpgroup, as packed pairs: the negated
     // running maximum (log2 domain) and this thread's row-sum partial.
     uint64_t nm2[kCols / 2], lp2[kCols / 2];
@@ -684,7 +770,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       const int count = okw ? C.unit[slot].count : 0;
       const bool last_is_diag = okw && C.unit[slot].diag != 0;
       const int uu = okw ? C.unit[slot].u : 0;
-      if (bar_red_or(bar_id, 128, !okw)) break;
+      if (bar_red_or(bar_id, 128, !okw || dead)) break;
       if (w < 0) break;  // the end marker is never released: nothing reuses its slot
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
@@ -708,6 +794,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const int pr = rg >= kPSlots ? rg - kPSlots : rg - kPSlots + kRing;
         const int pph = rg >= kPSlots ? rph : rph ^ 1;
         const bool okP = g < kPSlots || mbar_wait(&bars.pv_done[pr], pph, abort_p, p.status, tmo);
+        dead = dead || __any_sync(0xffffffffu, !okS || !okP);
 #ifdef SEER_TRACE
         const long long tstep0 = clock64();
         long long tmark = tstep0;
@@ -724,7 +811,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           float* red = &C.red[wgi][red_use & 1][0][0];
           warp_reduce_scatter16<false>(x, lane, red + ww * kCols);
           ++red_use;
-          if (bar_red_or(bar_id, 128, !okS || !okP)) { fail = true; break; }
+          if (bar_red_or(bar_id, 128, dead)) { fail = true; break; }
           float mcol[kCols];
           col_combine<false>(red, mcol);
 #pragma unroll
@@ -744,7 +831,8 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           // per-step barrier.  A score far above it flags the unit, which the
           // fallback kernel then recomputes exactly (one list entry per unit:
           // the first warp to flag it appends it).
-          if (__any_sync(0xffffffffu, dmax > kFlagThreshold) && lane == 0 && atomicExch(&C.redo_unit, w) != w) {
+          if (__any_sync(0xffffffffu, dmax > kFlagThreshold) && !dead && lane == 0 &&
+              atomicExch(&C.redo_unit, w) != w) {
             const uint32_t e = atomicAdd(p.redo_count, 1u);
             if (e < (uint32_t)p.redo_cap) p.redo_list[e] = w;
           }
@@ -760,10 +848,13 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         fence_async_shared();
         SEER_MARK(21);
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars.go[rg]);
-          mbar_arrive(&bars.kfull[(rg + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
+        if (!dead) {
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars.go[rg]);
+            mbar_arrive(&bars.kfull[(rg + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
+          }
+          ++arrived;
         }
         if constexpr (MAP) {
           if (valid && (lane & 1) == 0) mscr[((long long)mi * 2 + (ww & 1)) * 64 + q0 + map_col(lane)] = mval;
@@ -793,7 +884,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       for (int q = 0; q < kCols / 2; ++q) f32x2_unpack(lp2[q], lpart[2 * q], lpart[2 * q + 1]);
       warp_reduce_scatter16<true>(lpart, lane, red + ww * kCols);
       ++red_use;
-      if (bar_red_or(bar_id, 128, !okPV)) break;
+      if (bar_red_or(bar_id, 128, !okPV || dead)) break;
       float l[kCols];
       col_combine<true>(red, l);
       tc_fence_after();
@@ -860,17 +951,33 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #endif
       step += T;
     }
+    if (lane == 0) C.sm_steps[warp] = arrived;
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kWarpPV) tmem_dealloc(tmem, kTmemCols);
-  // After an abort the consumers stopped waiting, so loads may still be in
-  // flight: give them time to land before the CTA's shared memory is released.
+  // After an abort, bulk copies may still be in flight into shared memory.
+  // Every warp has left its loop, so the arrivals each barrier still lacks
+  // are known exactly: kfull(h) waits for the softmax warps' release of step
+  // h-3, go(h) for their P^T of step h.  Make those arrivals here; each
+  // phase the loaders armed then completes exactly when its copies have
+  // landed, which the teardown waits for (bounded) before the CTA exits.
+  // A loader arms kfull(h) only after QK(h-2) and go(h) only after PV(h-3),
+  // so only the last two kfull and last three go phases can be open.
   if (threadIdx.x == 0 && *abort_p) {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 200000ull) {
+    const int hk = C.armed_k, hv = C.armed_v;
+    for (int h = hk - kKSlots > 0 ? hk - kKSlots : 0; h < hk; ++h) {
+      if (h >= kSBuf)
+        for (int w2 = 0; w2 < kSoftmaxWarps; ++w2)
+          if (C.sm_steps[w2] <= h - kSBuf) mbar_arrive(&bars.kfull[h % kRing]);
+      mbar_wait_teardown(&bars.kfull[h % kRing], (h / kRing) & 1, 20000000ull);
+    }
+    for (int h = hv - kVSlots > 0 ? hv - kVSlots : 0; h < hv; ++h) {
+      for (int w2 = 0; w2 < kSoftmaxWarps; ++w2)
+        if (C.sm_steps[w2] <= h) mbar_arrive(&bars.go[h % kRing]);
+      mbar_wait_teardown(&bars.go[h % kRing], (h / kRing) & 1, 20000000ull);
     }
   }
 #ifdef SEER_TRACE
@@ -880,6 +987,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   }
 #endif
 }
+
 
 // ---------------------------------------------------------------- re-layout --
 // Writes K^T of every (batch, KV head, key block j) as one contiguous record
@@ -952,7 +1060,7 @@ __global__ void __launch_bounds__(256) empty_rows_kernel(const int32_t* __restri
 // V as the attention kernel (so fp32 inputs see the same rounding), and the
 // same checked list entries.  Slow by design: it only runs for inputs
 // whose scores rise more than 2^64 above a unit's first-step maximum.
-template <int D>
+template <int D, bool KT>
 __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat16* __restrict__ Q16,
                                                                const __nv_bfloat16* __restrict__ Kt16,
                                                                const __nv_bfloat16* __restrict__ V16,
@@ -980,13 +1088,14 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
         const int raw = p.dense ? t : lst[t];
         const int j = checked_entry(p, u, raw, prev);
         prev = raw;
-        const __nv_bfloat16* rec = Kt16 + (rec0 + j) * (D * 64LL);  // K^T: [dim][key]
+        const __nv_bfloat16* rec = Kt16 + (rec0 + j) * (D * 64LL);  // K^T: [dim][key], or K: [key][dim]
         const __nv_bfloat16* vb = V16 + (rec0 + j) * (64LL * D);    // V: [key][dim]
         const int kmax = j == u.i ? r : 63;  // causal inside the diagonal block
         for (int key = 0; key <= kmax; ++key) {
           float sdot = 0.f;
 #pragma unroll
-          for (int k = 0; k < DL; ++k) sdot += q[k] * __bfloat162float(rec[(lane * DL + k) * 64 + key]);
+          for (int k = 0; k < DL; ++k)
+            sdot += q[k] * __bfloat162float(KT ? rec[(lane * DL + k) * 64 + key] : rec[key * D + lane * DL + k]);
           const float sc = warp_sum(sdot) * p.scale_log2;
           const float mn = fmaxf(m, sc);
           const float a = exp2f(m - mn), pr = exp2f(sc - mn);
@@ -1030,7 +1139,8 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
           for (int key = 0; key <= kmax; ++key) {
             float sdot = 0.f;
 #pragma unroll
-            for (int k = 0; k < DL; ++k) sdot += q[k] * __bfloat162float(rec[(lane * DL + k) * 64 + key]);
+            for (int k = 0; k < DL; ++k)
+              sdot += q[k] * __bfloat162float(KT ? rec[(lane * DL + k) * 64 + key] : rec[key * D + lane * DL + k]);
             best = fmaxf(best, exp2f(warp_sum(sdot) * p.scale_log2 - lse2s[r]));
           }
         }
@@ -1046,10 +1156,17 @@ cudaError_t launch_sparse_attn_redo(const void* Q16, const void* Kt16, const voi
   const auto q = (const __nv_bfloat16*)Q16;
   const auto kt = (const __nv_bfloat16*)Kt16;
   const auto v = (const __nv_bfloat16*)V16;
-  if (p.d == 64)
-    sparse_attn_redo_kernel<64><<<148, 256, 0, st>>>(q, kt, v, p);
-  else
-    sparse_attn_redo_kernel<128><<<148, 256, 0, st>>>(q, kt, v, p);
+  if (p.k_rows) {
+    if (p.d == 64)
+      sparse_attn_redo_kernel<64, false><<<148, 256, 0, st>>>(q, kt, v, p);
+    else
+      sparse_attn_redo_kernel<128, false><<<148, 256, 0, st>>>(q, kt, v, p);
+  } else {
+    if (p.d == 64)
+      sparse_attn_redo_kernel<64, true><<<148, 256, 0, st>>>(q, kt, v, p);
+    else
+      sparse_attn_redo_kernel<128, true><<<148, 256, 0, st>>>(q, kt, v, p);
+  }
   return cudaGetLastError();
 }
 

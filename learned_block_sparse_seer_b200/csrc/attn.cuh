@@ -25,6 +25,8 @@ struct AttnParams {
   int redo_cap;
   float* map;          // training forward: [B*Hq*nb, nb] max-pooled map (zeroed first), or null
   float* map_scratch;  // with map: per CTA [nb][2][64] fp32
+  int test_skip_qk_commit;  // test hook: step whose QK completion is never signalled (-1: none)
+  int k_rows;               // exact fallback only: K given as rows [B*Hkv*n, d] instead of K^T records
 };
 
 // Re-layout of K into per-block K^T records of d rows x 64 bf16;
@@ -34,8 +36,8 @@ cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long recor
 // Exact fp32 recomputation of the units the attention kernel flagged (a
 // score above the unit's first-step column maximum by more than 2^64);
 // returns at once when none was.  Q16 is the bf16 Q the attention kernel
-// read, Kt16 the K^T records and V16 the bf16 V [B*Hkv*n, d].  Launch after
-// launch_sparse_attn.
+// read, Kt16 the K^T records (or, with p.k_rows, the bf16 K rows) and V16 the
+// bf16 V [B*Hkv*n, d].  Launch after launch_sparse_attn (or launch_fwd).
 cudaError_t launch_sparse_attn_redo(const void* Q16, const void* Kt16, const void* V16, const AttnParams& p,
                                     cudaStream_t st);
 
@@ -43,8 +45,9 @@ cudaError_t launch_sparse_attn_redo(const void* Q16, const void* Kt16, const voi
 // attention kernel skips those units.  Launch before launch_sparse_attn.
 cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st);
 
-// Persistent launch: one CTA per SM (at most one per unit).  tmQ is a 2-D
-// bf16 map over Q [rows, d] with 64x64 boxes; tmKt a 2-D bf16 map over the
+// Persistent launch: one CTA per SM (at most one per unit).  tmQ is a 3-D
+// bf16 map over Q (64 dims, B*Hq*n rows, d/64 panels) with a 64 x 64 x d/64
+// box; tmKt a 2-D bf16 map over the
 // K^T records [records * d, 64] with a d-row box; tmV a 3-D bf16 map over V
 // (64 dims, B*Hkv*n rows, d/64 panels) with a 64 x 64 x d/64 box; all
 // 128-byte swizzled.

@@ -209,3 +209,33 @@ def test_rejects_bad_arguments():
     with pytest.raises(seer.SeerError) as e:
         seer.seer_sparse_attn(Qd, Kd, Vd, c, ix, scale=-1.0)
     assert e.value.status == 1
+
+
+def test_bounded_wait_gives_up_and_the_device_stays_usable():
+    """The failure path of the kernel's bounded waits, without faulting the GPU:
+    the library's test hook leaves out the completion signal of every CTA's
+    first QK step, so the waits that depend on it give up after 20 ms.  The
+    call must report SEER_ERR_TIMEOUT through the workspace status word (its
+    kernel unwinds, draining its bulk copies), and the next call on the same
+    device and workspace must match the oracle."""
+    from learned_block_sparse_seer_b200 import _lib
+    L = _lib.lib()
+    w, Q, K, V, Wq, Wk = inputs("tiny")
+    Qb, Kb, Vb = (t.to(torch.bfloat16) for t in (Q, K, V))
+    c, ix, _ = oracle.select(oracle.gate(Qb, Kb, Wq, Wk), oracle.MODE_TOPK_K, k=8)
+    Qd, Kd, Vd = to_dev(Qb, Kb, Vb)
+    cd = torch.as_tensor(c, dtype=torch.int32).cuda()
+    idd = torch.as_tensor(ix, dtype=torch.int32).cuda()
+    ws = torch.empty(seer.sparse_attn_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8, device="cuda")
+    try:
+        L.seer_testing_attn_wait_fault(0, 20_000_000)
+        seer.seer_sparse_attn(Qd, Kd, Vd, cd, idd, workspace=ws)
+        assert seer.seer_workspace_status(ws) == 5  # SEER_ERR_TIMEOUT
+    finally:
+        L.seer_testing_attn_wait_fault(-1, 0)
+    for _ in range(2):
+        O, lse = seer.seer_sparse_attn(Qd, Kd, Vd, cd, idd, workspace=ws)
+        assert seer.seer_workspace_status(ws) == 0
+        O_ref, lse_ref = oracle.sparse_attn(Qb, Kb, Vb, c, ix)
+        check_o(O.cpu().double().numpy(), O_ref)
+        check_lse(lse.cpu().double().numpy(), lse_ref)
