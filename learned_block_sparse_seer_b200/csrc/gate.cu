@@ -7,16 +7,23 @@
 // and the OpenReview rebuttal, section 3.3 (top-k indices [S/B, k];
 // threshold mask o > threshold).
 //
-// Kernels (all HBM- or latency-bound; none is a dense contraction worth the
-// tensor cores -- the gate is ~1/4096 of the attention map):
+// Kernels (the gate is ~1/4096 of the attention map; pooling is HBM-bound,
+// the rest small):
 //   pool_kernel      Q avg-pool / K [max|min|avg]-pool, one warp per block,
 //                    16-byte vector loads, shuffle reductions
-//   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections and the causal
-//                    block logits q~ k~^T / sqrt(d) (upper tiles skipped);
-//                    gemm_nt128_kernel is its 128 x 128-tile form for K % 16 == 0
+//   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections, and the causal
+//                    block logits q~ k~^T / sqrt(d) (upper tiles skipped) when
+//                    h is not a multiple of 32; gemm_nt128_kernel is its
+//                    128 x 128-tile form for K % 16 == 0
+//   split_tf32_kernel + gemm_tf32x3_kernel
+//                    the causal block logits on the tf32 tensor cores (tcgen05)
+//                    when h % 32 == 0: three products of tf32 parts (hi*hi +
+//                    hi*lo + lo*hi) keep fp32-level accuracy
 //   rope_kernel      optional block-level RoPE on q~ / k~
-//   row_select_kernel  one CTA per score row: causal softmax (Eq. 1), optional
-//                    score write-out, then threshold compaction or exact top-k
+//   row_select_warp_kernel / row_select_kernel
+//                    one warp (many rows of <= 2048 candidates) or one CTA per
+//                    score row: causal softmax (Eq. 1), optional score
+//                    write-out, then threshold compaction or exact top-k
 //                    (radix select on the fp32 bit patterns, ties to lower j)
 #include <cstdint>
 
@@ -807,10 +814,33 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
     if (t >= nt) break;
     v[t] = __uint_as_float(32 * t + lane < len ? f2key(v[t]) : 0u);
   }
-  // Radix select of the ki-th largest key, 8 bits at a time from the top.
-  uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)ki;
+  // Radix select of the ki-th largest key, 8 bits at a time.  Bits that all
+  // of the row's keys share are fixed at once (a warp AND / OR of the keys):
+  // a softmax row's values lie close together, so its keys agree on the
+  // sign, the exponent and the top of the mantissa, and the first digit
+  // starts at the highest bit where they differ.  The search also stops as
+  // soon as the bin holding the ki-th key is taken whole.
+  uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    if (t >= nt) break;
+    if (32 * t + lane < len) {
+      kand &= __float_as_uint(v[t]);
+      kor |= __float_as_uint(v[t]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+  }
+  const uint32_t kdiff = kand ^ kor;
+  const int hb = kdiff ? 31 - __clz(kdiff) : -1;  // highest bit where keys differ
+  // bits above hb are fixed (all of them when every key is equal)
+  uint32_t pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
+  uint32_t prefix = kand & pmask, remaining = (uint32_t)ki;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int shift = hb >= 7 ? hb - 7 : 0; hb >= 0;) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
     __syncwarp();
@@ -855,20 +885,26 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
     const int owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
     sel_bin = __shfl_sync(0xffffffffu, sel_bin, owner);
     sel_rem = __shfl_sync(0xffffffffu, sel_rem, owner);
+    const uint32_t sel_cnt = __shfl_sync(0xffffffffu, hist[sel_bin], 0);
     prefix |= sel_bin << shift;
     remaining = sel_rem;
     pmask |= 0xffu << shift;
     __syncwarp();  // the bins are cleared again only after every lane read them
+    // (when the digit overlaps bits fixed earlier, those bits of sel_bin equal
+    // the prefix's: every counted key shares them)
+    if (sel_cnt == sel_rem || shift == 0) break;  // the bin is taken whole, or every bit is fixed
+    shift = shift >= 8 ? shift - 8 : 0;
   }
-  // keys > prefix are all kept; of the keys == prefix the `remaining` ones
-  // with the lowest j; the diagonal joins when forced
+  // keys above the prefix (on the bits fixed so far) are all kept; of the
+  // keys equal to it the `remaining` ones with the lowest j; the diagonal
+  // joins when forced
   int base = 0;
   uint32_t eq_before = 0;
 #pragma unroll
   for (int t = 0; t < NPL; ++t) {
     if (t >= nt) break;
     const int j = 32 * t + lane;
-    const uint32_t kt = __float_as_uint(v[t]);
+    const uint32_t kt = __float_as_uint(v[t]) & pmask;
     const bool eq = j < len && kt == prefix;
     const unsigned em = __ballot_sync(0xffffffffu, eq);
     const uint32_t rank = eq_before + __popc(em & lt);
