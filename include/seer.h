@@ -329,13 +329,13 @@ SEER_API seer_status seer_gate_noalloc(const seer_dims *dims, const void *Q, con
 /* seer_attn_forward_map -- the training forward of the summary page's
  * customized kernel ("The customized training kernel", Figure 10): dense
  * causal attention output O and row log-sum-exp, plus the 2D-max-pooled
- * probability map gt, in one pass.  The attention kernel runs over every
- * causal block and also keeps, per step, each column's score maximum over
- * each 32-key half block; at the end of each 64-row unit those maxima become
- * probabilities with the final row sums, and their maximum over the rows is
- * the map entry.  Units that need the exact fallback (a score more than 2^64
- * above the unit's first-step maximum) get their O, LSE and map row
- * recomputed exactly.
+ * probability map gt, in one pass.  A dense kernel walks 128-row query
+ * tiles (two query blocks) over every causal key pair and also keeps each
+ * row's score maximum over each 32-key half block; at the end of each tile
+ * those maxima become probabilities with the row's log-sum-exp, and their
+ * maximum over the 64 rows of a query block is the map entry.  Tiles that
+ * need the exact fallback (a score more than 2^64 above the row's
+ * first-step maximum) get their O, LSE and map rows recomputed exactly.
  *   Q [B,Hq,n,d], K, V [B,Hkv,n,d] (dtype); scale 0 means 1/sqrt(d)
  *   O [B,Hq,n,d] (dtype), lse [B,Hq,n] fp32 (may be NULL),
  *   map_out [B,Hq,nb,nb] fp32 (0 above the diagonal)

@@ -576,15 +576,11 @@ size_t seer_sparse_attn_workspace_size(const seer_dims* dims, seer_dtype dtype) 
   return attn_ws(dims, dtype).total;
 }
 
-namespace {
-// The sparse attention call; `dense` runs every causal block without lists.
-seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V, seer_dtype dtype,
-                            const int32_t* counts, const int32_t* indices, int32_t cap, float scale, void* O,
-                            float* lse, void* ws, size_t ws_bytes, seer_stream_t stream, bool dense,
-                            bool keep_status = false, float* map = nullptr, size_t map_scratch_off = 0) {
-  if (!dims_ok(dims) || !Q || !K || !V || !O) return SEER_ERR_INVALID_ARG;
-  if (!dense && (!counts || !indices)) return SEER_ERR_INVALID_ARG;
-  if (dense) cap = dims->n / seer::kBlock;
+seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V,
+                             seer_dtype dtype, const int32_t* counts, const int32_t* indices,
+                             int32_t cap, float scale, void* O, float* lse, void* ws,
+                             size_t ws_bytes, seer_stream_t stream) {
+  if (!dims_ok(dims) || !Q || !K || !V || !O || !counts || !indices) return SEER_ERR_INVALID_ARG;
   if (dtype != SEER_BF16 && dtype != SEER_FP32) return SEER_ERR_INVALID_ARG;
   if (cap < 1 || !(scale >= 0.f) || !std::isfinite(scale)) return SEER_ERR_INVALID_ARG;
   seer_status s = dims_supported(dims);
@@ -592,19 +588,8 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
     return SEER_ERR_INVALID_ARG;
   const AttnWs w = attn_ws(dims, dtype);
-  // with a map, its per-CTA scratch follows the attention workspace
-  const size_t need = map ? map_scratch_off + sizeof(float) * (size_t)num_sms() * (dims->n / seer::kBlock) * 128
-                          : w.total;
   cudaStream_t st = (cudaStream_t)stream;
-  if (keep_status) {
-    // a call made on behalf of another in the same workspace: reset only the
-    // work counters, so that the earlier launch's device status survives
-    if (!ws || !aligned(ws, 256) || ws_bytes < need) return SEER_ERR_WORKSPACE;
-    SEER_CUDA(cudaMemsetAsync((uint8_t*)ws + 8, 0, sizeof(seer::WsHeader) - 8, st));
-    s = SEER_OK;
-  } else {
-    s = begin_ws(ws, ws_bytes, need, st);
-  }
+  s = begin_ws(ws, ws_bytes, w.total, st);
   if (s != SEER_OK) return s;
   uint8_t* base = (uint8_t*)ws;
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
@@ -634,7 +619,7 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   p.total_units = (long long)B * Hq * p.nb;
   p.counts = counts;
   p.indices = indices;
-  p.dense = dense ? 1 : 0;
+  p.dense = 0;
   p.O = O;
   p.lse = lse;
   p.out_fp32 = dtype == SEER_FP32;
@@ -648,24 +633,14 @@ seer_status run_sparse_attn(const seer_dims* dims, const void* Q, const void* K,
   p.redo_count = &hdr->work_counter2;
   p.redo_list = reinterpret_cast<int*>(base + w.redo);
   p.redo_cap = (int)p.total_units;
-  p.map = map;
-  p.map_scratch = map ? (float*)(base + map_scratch_off) : nullptr;
+  p.map = nullptr;
   p.test_skip_qk_commit = g_test_skip_qk_commit;
   p.k_rows = 0;
   if (g_test_wait_limit_ns) p.timeout_ns = g_test_wait_limit_ns;
-  if (map) SEER_CUDA(cudaMemsetAsync(map, 0, sizeof(float) * (size_t)p.total_units * p.nb, st));
-  if (!dense) SEER_CUDA(seer::launch_empty_rows(p, st));
+  SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKt, tmV, p, num_sms(), st));
   SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kt, v16, p, st));
   return SEER_OK;
-}
-}  // namespace
-
-seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K, const void* V,
-                             seer_dtype dtype, const int32_t* counts, const int32_t* indices,
-                             int32_t cap, float scale, void* O, float* lse, void* ws,
-                             size_t ws_bytes, seer_stream_t stream) {
-  return run_sparse_attn(dims, Q, K, V, dtype, counts, indices, cap, scale, O, lse, ws, ws_bytes, stream, false);
 }
 
 // -------------------------------------------------------------- blockmax --

@@ -41,17 +41,19 @@
 //    allocation; warp 18 issues the QK MMAs.
 //  * Softmax without a per-step barrier: each unit's column maxima are formed
 //    exactly on its first step and then kept; later steps compute
-//    exp2(score * scale - max) with packed f32x2 arithmetic.  A score more
-//    than 2^64 above its column's kept maximum flags the unit (a warp vote),
-//    and sparse_attn_redo_kernel recomputes flagged units exactly afterwards.
+//    exp2(score * scale - max) with packed f32x2 arithmetic.  Scores above
+//    the kept maximum are harmless until P, a column sum or O would overflow
+//    fp32 / bf16 (about 2^128); the unit's epilogue checks for that, flags
+//    the unit, and sparse_attn_redo_kernel recomputes flagged units exactly.
 //  * Units are handed out by an atomic counter in KV-head-major order, query
 //    blocks from the last (longest lists) to the first, so the K/V of one KV
 //    head stay hot in L2 while its query heads are processed.  Units with an
 //    empty list never enter the ring (empty_rows_kernel writes their rows).
-//  * MAP mode (the training forward) also forms the 2D-max-pooled map in the
-//    same pass (see the kernel's comment).
 //  * Every mbarrier wait is bounded (%globaltimer); on expiry the kernel
-//    records a timeout in the workspace status word and unwinds.
+//    records a timeout in the workspace status word and unwinds: the warps
+//    stop making barrier arrivals, and before the CTA exits the teardown
+//    completes each barrier phase the loader armed with exactly the
+//    arrivals it lacks and waits until its bulk copies have landed.
 #include <cstddef>
 #include <cstdint>
 
@@ -63,17 +65,17 @@
 namespace seer {
 
 namespace attn {
-constexpr int kThreads = 640;
-constexpr int kWarpLoadK = 16, kWarpPV = 17, kWarpQK = 18, kWarpLoadV = 19;
+constexpr int kThreads = 608;
+constexpr int kWarpLoad = 16, kWarpPV = 17, kWarpQK = 18;
 constexpr uint32_t kHalf = 16384;              // one key block's K^T record or V (d = 128)
 constexpr uint32_t kPair = 2 * kHalf;          // the K^T (or V) of a pair step
-constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 2, kQSlots = 2;
+constexpr int kKSlots = 2, kVSlots = 3, kPSlots = 3, kQSlots = 1;
 constexpr uint32_t kPBytes = 16384;            // P^T of a pair step: 2 x [64 keys x 64 queries]
 constexpr uint32_t kQBytes = 16384;            // Q tile: 64 rows x d (two 64-column panels)
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kKSlots * kPair;       //  64 KB
 constexpr uint32_t kOffP = kOffV + kVSlots * kPair;       // 160 KB
-constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 192 KB
+constexpr uint32_t kOffQ = kOffP + kPSlots * kPBytes;     // 208 KB
 constexpr uint32_t kSmemBytes = kOffQ + kQSlots * kQBytes;  // 224 KB of tiles
 constexpr int kRing = 4;   // kfull / go / qk_done / pv_done barriers, indexed by step
 constexpr int kSBuf = 3;   // S^T buffers in TMEM (QK runs two steps ahead of PV)
@@ -83,14 +85,10 @@ constexpr uint32_t kColO = kSBuf * 64;
 constexpr int kWG = 4;     // softmax warpgroups
 constexpr int kCols = 16;  // query columns per warpgroup
 constexpr int kSoftmaxWarps = 4 * kWG;
-// readers of a unit ring entry: both loaders, both MMA warps, every softmax warp
-constexpr int kUnitReaders = 4 + kSoftmaxWarps;
+// readers of a unit ring entry: both MMA warps and every softmax warp
+constexpr int kUnitReaders = 2 + kSoftmaxWarps;
 static_assert(kSBuf < kRing, "kfull(h) takes softmax(h - kSBuf) arrivals");
 static_assert(kVSlots < kRing && kPSlots < kRing && kKSlots < kRing, "slot reuse is tracked on the step rings");
-// A score more than 2^64 above its unit's first-step column maximum (log2
-// domain) sends the unit to the exact fallback kernel.  Below it nothing
-// overflows: P <= 2^64 in bf16, row sums <= 2^81 and O in fp32.
-constexpr float kFlagThreshold = 64.0f;
 
 struct Bars {
   uint64_t unit_full[kUnits], unit_empty[kUnits];
@@ -116,8 +114,9 @@ struct Ctrl {
   uint32_t tmem_base;
   int abort_flag;
   int redo_unit;  // the last unit this CTA flagged for the exact fallback
-  // Teardown accounting after an abort: the steps each loader armed, and the
-  // steps for which each softmax warp made its go / kfull arrivals.
+  // Teardown accounting after an abort: the steps whose K^T (and Q) and V
+  // copies the loader issued, and the steps for which each softmax warp made
+  // its go / kfull arrivals.
   int armed_k, armed_v;
   int sm_steps[kSoftmaxWarps];
   alignas(16) float red[kWG][2][4][kCols];  // read with 16-byte vector loads
@@ -360,47 +359,6 @@ __device__ __forceinline__ void scores_minus_max(uint32_t taddr, float (&x)[attn
   }
 }
 
-// MAP mode: this warp's per-column maxima over its 32 keys (lanes) of the
-// step's scores x (log2 units, relative to the unit's fixed maximum).  A
-// butterfly reduce-scatter (16 shuffles for 16 columns) leaves the maximum of
-// column map_col(lane) on each lane; the even lanes store it later, after the
-// step's barrier arrivals (an arrival releases the thread's earlier global
-// stores, so a store just before it would stall the step on its write).
-__device__ __forceinline__ float warp_col_max(const float (&x)[attn::kCols], int lane) {
-  static_assert(attn::kCols == 16, "16 columns per warp");
-  float v[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) v[q] = x[q];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const bool up = lane & 16;
-    const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
-    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const bool up = lane & 8;
-    const float send = up ? v[k] : v[k + 4], keep = up ? v[k + 4] : v[k];
-    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const bool up = lane & 4;
-    const float send = up ? v[k] : v[k + 2], keep = up ? v[k + 2] : v[k];
-    v[k] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-  }
-  {
-    const bool up = lane & 2;
-    const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
-    v[0] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-  }
-  return fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
-}
-
-__device__ __forceinline__ int map_col(int lane) {
-  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-}
-
 // This warpgroup's 16 bf16 probabilities of key row kl into the step's P^T
 // tile (128-byte rows, 16-byte chunks swizzled by the row index).
 // off0/off1 are the row's two swizzled 16-byte chunk offsets.
@@ -413,23 +371,6 @@ __device__ __forceinline__ void store_p(uint8_t* prow, const float (&x)[attn::kC
   *reinterpret_cast<uint4*>(prow + off1) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
-// One unit's list entries, read warp-wide 32 at a time: lane l holds entry
-// base + l (0 past the count).  Dense mode needs no list: entry t is t.
-__device__ __forceinline__ int list_raw(const AttnParams& p, const int* lst, int t, int count) {
-  return t < count ? (p.dense ? t : lst[t]) : 0;
-}
-
-// Checks the lanes' raw entries of one chunk (entry t = base + lane) against
-// their predecessors as read (lane 0's is the previous chunk's last, carried
-// in last_raw); returns this lane's checked entry.
-__device__ __forceinline__ int check_chunk(const AttnParams& p, const UnitInfo& u, int raw, int t, int count,
-                                           int& last_raw, int lane) {
-  int prev = __shfl_up_sync(0xffffffffu, raw, 1);
-  if (lane == 0) prev = last_raw;
-  last_raw = __shfl_sync(0xffffffffu, raw, 31);
-  return t < count ? checked_entry(p, u, raw, prev) : 0;
-}
-
 // Waits (bounded) until the phase of `bar` with the given parity has
 // completed; used only at teardown, so it does not look at the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
@@ -439,14 +380,7 @@ __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parit
   return true;
 }
 
-// MAP (the training forward): also the 2D-max-pooled probability map.  Each
-// step every warp takes, per query column, the maximum of its 32 keys'
-// scores (a shuffle reduce-scatter over the lanes = keys) and keeps it in the
-// CTA's scratch slot [key block][key half][64 columns]; the unit's epilogue
-// turns the kept maxima into probabilities with the final row sums and
-// max-combines them over the 64 rows into the map (atomicMax on the
-// non-negative bit patterns; one partial per warpgroup of 16 columns).
-template <int D, bool MAP>
+template <int D>
 __global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKt,
                        const __grid_constant__ CUtensorMap tmV,
@@ -515,137 +449,98 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   const uint32_t tmem = C.tmem_base;
   constexpr uint32_t part_bytes = (uint32_t)D * 128u;  // a key block's K^T record, or its V
 
-  if (warp == kWarpLoadK || warp == kWarpLoadV) {
-    // ------------------------- loaders: Q + K^T, and V with the scheduler ---
-    // Two warps issue the bulk copies (one instruction per 16 KB box): the
-    // K loader the unit's Q tile and the step's K^T records, the V loader the
-    // step's V blocks.  Each walks the unit ring itself and reads the list
-    // warp-wide, 32 checked entries at a time, the next chunk in flight while
-    // the current one is used.  Lane 0 waits and issues.
-    //
-    // The V loader also schedules: it hands out units by an atomic counter
-    // and publishes them in the unit ring, one unit ahead of its own walk (V
-    // is needed last, so its ring absorbs the scheduling latency).  Units
-    // with an empty list never enter the ring: their output (O = 0, LSE =
-    // -inf) is written by empty_rows_kernel before this kernel.
-    const bool isK = warp == kWarpLoadK;
-    int pub = 0;           // units published (V loader)
-    bool sched_end = isK;  // the end marker is out (or this warp does not schedule)
-    auto publish_one = [&]() {
-      const int slot = pub % kUnits;
-      if (pub >= kUnits &&
-          !mbar_wait(&bars.unit_empty[slot], ((pub / kUnits) - 1) & 1, abort_p, p.status, tmo)) {
-        sched_end = true;
-        return;
-      }
-      int w;
-      UnitInfo u{};
-      for (;;) {
-        w = (int)atomicAdd(p.work_counter, 1u);
-        if (w >= p.total_units || *abort_p) {
-          w = -1;
-          break;
-        }
-        u = decode_unit(p, w);
-        if (u.count > 0) break;
-      }
-      // lists are ascending, so only the last entry can be the diagonal block
-      const int diag = w >= 0 ? (p.dense ? 1 : (p.indices[u.u * p.cap + u.count - 1] == u.i)) : 0;
-      C.unit[slot].w = w;
-      C.unit[slot].count = u.count;
-      C.unit[slot].diag = diag;
-      C.unit[slot].u = w >= 0 ? (int)u.u : 0;
-      mbar_arrive(&bars.unit_full[slot]);
-      ++pub;
-      if (w < 0) sched_end = true;  // the end marker is never released: nothing reuses its slot
-    };
+  if (warp == kWarpLoad) {
+    // ------------------------------- scheduler, Q loads, record gathers --
+    // Units are handed out by an atomic counter and published in the unit
+    // ring.  Units with an empty list never enter the ring: their output
+    // (O = 0, LSE = -inf) is written by empty_rows_kernel before this kernel.
     if (lane == 0) {
-      if (isK) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmKt);
-      } else {
-        prefetch_tmap(&tmV);
-        publish_one();
-        if (!sched_end) publish_one();
-      }
-    }
-    int ur = 0, qn = 0, h = 0;
-    for (;;) {
-      const int slot = ur % kUnits;
-      bool okw = true;
-      if (lane == 0) okw = mbar_wait(&bars.unit_full[slot], (ur / kUnits) & 1, abort_p, p.status, tmo);
-      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
-      const int w = C.unit[slot].w, count = C.unit[slot].count;
-      ++ur;
-      if (w < 0) break;
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars.unit_empty[slot]);
-        if (!sched_end) publish_one();
-      }
-      const UnitInfo u = unit_coords(p, w);
-      const int qs = qn % kQSlots;
-      if (isK && qn >= kQSlots) {
-        bool okq = true;
-        if (lane == 0) okq = mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo);
-        if (!__shfl_sync(0xffffffffu, okq, 0)) break;
-      }
-      ++qn;
-      const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
-      const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;  // this KV head's first block
-      const int* lst = p.indices + u.u * p.cap;
-      int raw = list_raw(p, lst, lane, count);
-      int raw_next = list_raw(p, lst, 32 + lane, count);
-      int last_raw = -1, chk = 0;
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKt);
+      prefetch_tmap(&tmV);
+      int u_idx = 0, qn = 0, hk = 0, hv = 0;  // units published, Q tiles, steps whose K^T / V copies are out
       bool ok = true;
-      for (int m = 0; m < count; m += 2, ++h) {
-        const int c = m & 31;
-        if (c == 0) {
-          if (m > 0) {
-            raw = raw_next;
-            raw_next = list_raw(p, lst, m + 32 + lane, count);
+      while (ok) {
+        const int slot = u_idx % kUnits;
+        if (u_idx >= kUnits &&
+            !mbar_wait(&bars.unit_empty[slot], ((u_idx / kUnits) - 1) & 1, abort_p, p.status, tmo))
+          break;
+        int w;
+        UnitInfo u{};
+        for (;;) {
+          w = (int)atomicAdd(p.work_counter, 1u);
+          if (w >= p.total_units || *abort_p) {
+            w = -1;
+            break;
           }
-          chk = check_chunk(p, u, raw, m + lane, count, last_raw, lane);
+          u = decode_unit(p, w);
+          if (u.count > 0) break;
         }
-        const int ntile = m + 1 < count ? 2 : 1;
-        const int j0 = __shfl_sync(0xffffffffu, chk, c), j1 = __shfl_sync(0xffffffffu, chk, c + 1);
-        if (lane == 0) {
-          if (isK) {
-            // K^T slot free once QK(h-2) is complete; its copies (and the
-            // unit's Q tile on its first step) complete kfull(h)
-            ok = h < kKSlots || SEER_TIMED(0, mbar_wait(&bars.qk_done[(h - kKSlots) % kRing],
-                                                          ((h - kKSlots) / kRing) & 1, abort_p, p.status, tmo));
-            if (ok) {
-              uint64_t* tk = &bars.kfull[h % kRing];
-              mbar_arrive_expect_tx(tk, (uint32_t)ntile * part_bytes + (m == 0 ? 64u * D * 2u : 0u));
-              if (m == 0) tma_load_3d(smem + kOffQ + qs * kQBytes, &tmQ, tk, 0, qrow, 0);
-              uint8_t* dst = smem + kOffK + (h % kKSlots) * kPair;
-              tma_load_2d(dst, &tmKt, tk, 0, (int)((rec0 + j0) * D));
-              if (ntile == 2) tma_load_2d(dst + kHalf, &tmKt, tk, 0, (int)((rec0 + j1) * D));
-            }
-          } else {
-            // V slot free once PV(h-3) is complete; its copies complete go(h)
-            ok = h < kVSlots || SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing],
-                                                          ((h - kVSlots) / kRing) & 1, abort_p, p.status, tmo));
-            if (ok) {
-              uint64_t* tv = &bars.go[h % kRing];
-              mbar_arrive_expect_tx(tv, (uint32_t)ntile * part_bytes);
-              uint8_t* dst = smem + kOffV + (h % kVSlots) * kPair;
-              tma_load_3d(dst, &tmV, tv, 0, (int)((rec0 + j0) * 64), 0);
-              if (ntile == 2) tma_load_3d(dst + kHalf, &tmV, tv, 0, (int)((rec0 + j1) * 64), 0);
-            }
+        // lists are ascending, so only the last entry can be the diagonal block
+        const int diag = w >= 0 ? (p.dense ? 1 : (p.indices[u.u * p.cap + u.count - 1] == u.i)) : 0;
+        C.unit[slot].w = w;
+        C.unit[slot].count = u.count;
+        C.unit[slot].diag = diag;
+        C.unit[slot].u = w >= 0 ? (int)u.u : 0;
+        mbar_arrive(&bars.unit_full[slot]);
+        ++u_idx;
+        if (w < 0) break;  // the end marker is never released: nothing reuses its slot
+        const int qs = qn % kQSlots;
+        if (qn >= kQSlots && !mbar_wait(&bars.q_free[qs], ((qn / kQSlots) - 1) & 1, abort_p, p.status, tmo)) break;
+        ++qn;
+        const int qrow = (int)(((long long)u.b * p.Hq + u.hq) * p.n + (long long)u.i * 64);
+        const long long rec0 = ((long long)u.b * p.Hkv + u.g) * p.nb;  // this KV head's first block
+        // The list entries of the next pair step are read one step early, so
+        // that their global-memory latency hides behind this step's waits.
+        const int* lst = p.indices + u.u * p.cap;
+        auto entry = [&](int t) { return p.dense ? t : lst[t]; };
+        int jn0 = entry(0);
+        int jn1 = u.count > 1 ? entry(1) : 0;
+        int prev = -1;
+        for (int m = 0; m < u.count; m += 2) {
+          const int h = hk;
+          const int ntile = m + 1 < u.count ? 2 : 1;
+          const int ra = jn0, rb = jn1;
+          if (m + 2 < u.count) jn0 = entry(m + 2);
+          if (m + 3 < u.count) jn1 = entry(m + 3);
+          int jj[2];
+          jj[0] = checked_entry(p, u, ra, prev);
+          prev = ra;
+          jj[1] = 0;
+          if (ntile == 2) {
+            jj[1] = checked_entry(p, u, rb, prev);
+            prev = rb;
           }
+          // K^T part: its slot is free once QK(h-2) is complete; it (and the
+          // unit's Q tile on its first step) completes kfull(h).
+          if (h >= kKSlots && !SEER_TIMED(0, mbar_wait(&bars.qk_done[(h - kKSlots) % kRing],
+                                                        ((h - kKSlots) / kRing) & 1, abort_p, p.status, tmo))) {
+            ok = false;
+            break;
+          }
+          uint64_t* tk = &bars.kfull[h % kRing];
+          mbar_arrive_expect_tx(tk, (uint32_t)ntile * part_bytes + (m == 0 ? 64u * D * 2u : 0u));
+          if (m == 0) tma_load_3d(smem + kOffQ + qs * kQBytes, &tmQ, tk, 0, qrow, 0);
+          for (int t = 0; t < ntile; ++t)
+            tma_load_2d(smem + kOffK + (h % kKSlots) * kPair + t * kHalf, &tmKt, tk, 0, (int)((rec0 + jj[t]) * D));
+          ++hk;
+          // V part: its slot is free once PV(h-3) is complete; it completes go(h).
+          if (h >= kVSlots &&
+              !SEER_TIMED(1, mbar_wait(&bars.pv_done[(h - kVSlots) % kRing], ((h - kVSlots) / kRing) & 1, abort_p,
+                                       p.status, tmo))) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars.go[h % kRing], (uint32_t)ntile * part_bytes);
+          for (int t = 0; t < ntile; ++t)
+            tma_load_3d(smem + kOffV + (h % kVSlots) * kPair + t * kHalf, &tmV, &bars.go[h % kRing], 0,
+                        (int)((rec0 + jj[t]) * 64), 0);
+          ++hv;
         }
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-    }
-    // steps whose copies were issued: the teardown drains them after an abort
-    if (lane == 0) {
-      if (isK)
-        C.armed_k = h;
-      else
-        C.armed_v = h;
+      // steps whose copies were issued: the teardown drains them after an abort
+      C.armed_k = hk;
+      C.armed_v = hv;
     }
   } else if (warp == kWarpQK) {
     // ------------------------------------------------------ QK issuer ----
@@ -753,8 +648,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // running maximum (log2 domain) and this thread's row-sum partial.
     uint64_t nm2[kCols / 2], lp2[kCols / 2];
     const uint64_t c2 = f32x2_pack(c, c);
-    // MAP mode: this CTA's scratch of per-(key block, key half, column) maxima
-    float* const mscr = MAP ? p.map_scratch + (long long)blockIdx.x * p.nb * 128 : nullptr;
     // this thread's P^T row (key kl of half `half`) and its two swizzled
     // 16-byte chunks (this warpgroup's 16 query columns)
     uint8_t* const prow0 = smem + kOffP + half * 8192 + kl * 128;
@@ -803,8 +696,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         const uint32_t saddr = lane_addr + (uint32_t)sb * 64u + q0;
         uint8_t* const prow = prow0 + ps * kPBytes;
         float x[kCols];
-        float mval = 0.f;  // MAP mode: this lane's column maximum of the step
-        (void)mval;
         if (t == 0) {
           // exact column maxima of the unit's first step
           if (okS) load_scores(saddr, x, c, valid, diag, kl, q0);
@@ -817,25 +708,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < kCols / 2; ++q) nm2[q] = f32x2_pack(-mcol[2 * q], -mcol[2 * q + 1]);
           scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
-          if constexpr (MAP) mval = warp_col_max(x, lane);
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
           store_p(prow, x, poff0, poff1);
         } else {
           if (okS) scores_minus_max(saddr, x, c2, nm2, valid, diag, kl, q0);
-          if constexpr (MAP) mval = warp_col_max(x, lane);
-          const float dmax =
-              fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
-                    fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
-          // The running maximum stays at the first step's: no rescale, no
-          // per-step barrier.  A score far above it flags the unit, which the
-          // fallback kernel then recomputes exactly (one list entry per unit:
-          // the first warp to flag it appends it).
-          if (__any_sync(0xffffffffu, dmax > kFlagThreshold) && !dead && lane == 0 &&
-              atomicExch(&C.redo_unit, w) != w) {
-            const uint32_t e = atomicAdd(p.redo_count, 1u);
-            if (e < (uint32_t)p.redo_cap) p.redo_list[e] = w;
-          }
 #pragma unroll
           for (int q = 0; q < kCols; ++q) x[q] = ex2_approx(x[q]);
           store_p(prow, x, poff0, poff1);
@@ -855,9 +732,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             mbar_arrive(&bars.kfull[(rg + kSBuf) % kRing]);  // S^T(g)'s buffer is free for QK(g+3)
           }
           ++arrived;
-        }
-        if constexpr (MAP) {
-          if (valid && (lane & 1) == 0) mscr[((long long)mi * 2 + (ww & 1)) * 64 + q0 + map_col(lane)] = mval;
         }
         if (++rg == kRing) {
           rg = 0;
@@ -892,6 +766,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         uint32_t o[16];
         tmem_ld16(lane_addr + kColO + q0, o);
         tmem_wait_ld();
+        // The column maximum stays at the unit's first step's: no rescale, no
+        // per-step barrier.  Scores far above it can overflow P, the column
+        // sums or O; such a unit is recomputed exactly by the fallback kernel
+        // (one list entry per unit: the first warp to see it appends it).
+        bool bad = false;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) bad = bad || !(fabsf(__uint_as_float(o[q])) <= 3.0e38f) || !(l[q] <= 3.0e38f);
+        if (__any_sync(0xffffffffu, bad) && !dead && lane == 0 && atomicExch(&C.redo_unit, w) != w) {
+          const uint32_t e = atomicAdd(p.redo_count, 1u);
+          if (e < (uint32_t)p.redo_cap) p.redo_list[e] = w;
+        }
         if (tl < p.d) {
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
@@ -917,34 +802,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
             lq = l[q];
           }
         p.lse[orow0 + tl] = (mq + lg2_approx(lq)) * 0.6931471805599453f;
-      }
-      if constexpr (MAP) {
-        // the kept maxima become probabilities with the row sums: x - log2(l)
-        // (x is relative to the fixed maximum); max over this warpgroup's 16
-        // columns, then over the 4 warpgroups by atomicMax into the map row
-        float ll[kCols];
-#pragma unroll
-        for (int q = 0; q < kCols; ++q) ll[q] = lg2_approx(l[q]);
-        const int* lst = p.indices + (long long)uu * p.cap;
-        for (int mi2 = tl; mi2 < count; mi2 += 128) {
-          const float4* s0 = reinterpret_cast<const float4*>(mscr + (long long)mi2 * 128 + q0);
-          float4 a[4], b2[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            a[k] = s0[k];
-            b2[k] = s0[16 + k];  // the other key half, 64 floats on
-          }
-          float v = 0.f;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            v = fmaxf(v, ex2_approx(fmaxf(a[k].x, b2[k].x) - ll[4 * k]));
-            v = fmaxf(v, ex2_approx(fmaxf(a[k].y, b2[k].y) - ll[4 * k + 1]));
-            v = fmaxf(v, ex2_approx(fmaxf(a[k].z, b2[k].z) - ll[4 * k + 2]));
-            v = fmaxf(v, ex2_approx(fmaxf(a[k].w, b2[k].w) - ll[4 * k + 3]));
-          }
-          const int j = p.dense ? mi2 : lst[mi2];
-          atomicMax(reinterpret_cast<int*>(p.map + (long long)uu * p.nb + j), __float_as_int(v));
-        }
       }
 #ifdef SEER_TRACE
       if (lane == 0) SEER_TRACE_ADD(10, clock64() - tep0);
@@ -1058,8 +915,10 @@ __global__ void __launch_bounds__(256) empty_rows_kernel(const int32_t* __restri
 // online softmax that rescales at every key, one warp per query row, lanes
 // splitting the head dimension.  It reads the same bf16 Q, K^T records and
 // V as the attention kernel (so fp32 inputs see the same rounding), and the
-// same checked list entries.  Slow by design: it only runs for inputs
-// whose scores rise more than 2^64 above a unit's first-step maximum.
+// same checked list entries.  Slow by design: it only runs for units whose
+// scores rise so far above the unit's first-step maximum that the attention
+// kernel's fp32 / bf16 values overflowed (or, in the training forward,
+// rose more than 2^64 above the row's first-step maximum).
 template <int D, bool KT>
 __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat16* __restrict__ Q16,
                                                                const __nv_bfloat16* __restrict__ Kt16,
@@ -1186,8 +1045,7 @@ cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long recor
 
 cudaError_t launch_sparse_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKt, const CUtensorMap& tmV, const AttnParams& p,
                                int num_sms, cudaStream_t st) {
-  auto kern = p.map ? (p.d == 64 ? sparse_attn_kernel<64, true> : sparse_attn_kernel<128, true>)
-                    : (p.d == 64 ? sparse_attn_kernel<64, false> : sparse_attn_kernel<128, false>);
+  auto kern = p.d == 64 ? sparse_attn_kernel<64> : sparse_attn_kernel<128>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn::kSmemAlloc);
   if (e != cudaSuccess) return e;
   long long grid = p.total_units < num_sms ? p.total_units : num_sms;

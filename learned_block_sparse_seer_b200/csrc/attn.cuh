@@ -11,7 +11,7 @@ struct AttnParams {
   long long total_units;     // B * Hq * nb
   const int32_t* counts;     // [B, Hq, nb]
   const int32_t* indices;    // [B, Hq, nb, cap]
-  int dense;                 // 1: every causal block (count = i+1, entry t = t); lists not read
+  int dense;                 // exact fallback of the training forward: every causal block (count = i+1, entry t = t); lists not read
   void* O;                   // [B, Hq, n, d] bf16 or fp32
   float* lse;                // [B, Hq, n] or null
   int out_fp32;              // O element type
@@ -23,8 +23,7 @@ struct AttnParams {
   uint32_t* redo_count;       // units flagged for the exact fallback (workspace)
   int* redo_list;             // [redo_cap] flagged unit indices
   int redo_cap;
-  float* map;          // training forward: [B*Hq*nb, nb] max-pooled map (zeroed first), or null
-  float* map_scratch;  // with map: per CTA [nb][2][64] fp32
+  float* map;          // exact fallback of the training forward: [B*Hq*nb, nb] map rows to rewrite, or null
   int test_skip_qk_commit;  // test hook: step whose QK completion is never signalled (-1: none)
   int k_rows;               // exact fallback only: K given as rows [B*Hkv*n, d] instead of K^T records
 };
@@ -33,8 +32,9 @@ struct AttnParams {
 // `records` = B * Hkv * n/64.
 cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st);
 
-// Exact fp32 recomputation of the units the attention kernel flagged (a
-// score above the unit's first-step column maximum by more than 2^64);
+// Exact fp32 recomputation of the units the attention kernel flagged (scores
+// so far above the unit's first-step column maximum that its values
+// overflowed; in the training forward, more than 2^64 above the row's);
 // returns at once when none was.  Q16 is the bf16 Q the attention kernel
 // read, Kt16 the K^T records (or, with p.k_rows, the bf16 K rows) and V16 the
 // bf16 V [B*Hkv*n, d].  Launch after launch_sparse_attn (or launch_fwd).
