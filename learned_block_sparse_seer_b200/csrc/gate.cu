@@ -301,7 +301,10 @@ __global__ void split_tf32_kernel(float* __restrict__ x, float* __restrict__ lo,
 }
 
 namespace gt3 {
-constexpr int kStages = 3;
+// One stage of 64 KB per CTA: three CTAs share an SM, so one tile's loads,
+// products and epilogue overlap the others' (a tile is only four 32-float
+// slices deep, too short to pipeline within one CTA).
+constexpr int kStages = 1;
 constexpr uint32_t kOp = 128u * 128u;                 // one operand slice: 128 rows x 32 floats
 constexpr uint32_t kStage = 4u * kOp;                 // Ah, Al, Bh, Bl
 constexpr uint32_t kSmem = kStages * kStage + 1024u;  // + slack to align the ring to 1024 bytes
@@ -320,10 +323,12 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
   __shared__ uint64_t full[kStages], empty[kStages], done;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int issued, consumed;  // slices whose copies went out / whose products were issued
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_p = &abort_flag;
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    issued = consumed = 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -357,6 +362,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
       tma_load_2d(st + kOp, &tmAl, &full[s], c * 32, arow);
       tma_load_2d(st + 2 * kOp, &tmBh, &full[s], c * 32, brow);
       tma_load_2d(st + 3 * kOp, &tmBl, &full[s], c * 32, brow);
+      issued = c + 1;
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = make_idesc_tf32(128, 128, 0, 0);  // A and B K-major
@@ -375,6 +381,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
         mma_tf32_ss(tmem, dAl + off, dBh + off, idesc, 1u);
       }
       mma_commit(&empty[s]);
+      consumed = c + 1;
     }
     // issued even after a failed wait: it arrives once this thread's MMAs are done
     mma_commit(&done);
@@ -409,11 +416,15 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, 128);
-  // after an abort, loads may still be in flight: let them land before the
-  // shared memory is released
+  // After an abort, the copies of slices that were issued but never consumed
+  // may still be in flight: each completes its stage's full phase (armed by
+  // the loader alone), so wait (bounded) for those phases before the shared
+  // memory is released.
   if (threadIdx.x == 0 && *abort_p) {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 200000ull) {
+    for (int c = consumed > issued - kStages ? consumed : issued - kStages; c < issued; ++c) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait_sleep(&full[c % kStages], (c / kStages) & 1, 20000u))
+        if (globaltimer_ns() - t0 > 20000000ull) break;
     }
   }
 }
@@ -704,26 +715,29 @@ __global__ void __launch_bounds__(NT) row_select_kernel(
   if (tid == 0) counts[row] = total;
 }
 
-// The same selection with one warp per row, for rows of at most 32 * NPL
-// candidates and many rows (the prefill gate): a row's values stay in the
-// lanes' registers (local candidate j = 32 t + lane in v[t]), reductions are
+// The same selection with one warp per row, for many rows of at most
+// kSelMaxWidth candidates (the prefill gate): the row lives in shared memory
+// (one buffer per warp; lane l owns candidates j = 32 t + l), reductions are
 // warp shuffles, the radix histogram is the warp's own 256 shared bins, and
-// the ascending lists are compacted with ballots, so no CTA barrier is
-// taken.  The softmax multiplies by the reciprocal of the row sum; the key
-// order, ties to the lower j, the forced diagonal and varlen windows follow
-// row_select_kernel.
+// the ascending lists are compacted with ballots, so no CTA barrier is taken.
+// Every loop over the row is a short rolled loop: fully unrolled register
+// copies of the row made the kernel wait on instruction fetch.  The softmax
+// multiplies by the reciprocal of the row sum; the key order, ties to the
+// lower j, the forced diagonal and varlen windows follow row_select_kernel.
 constexpr int kSelWarps = 8;
-constexpr int kSelNPL = 64;  // rows of up to 2048 candidates
+constexpr int kSelMaxWidth = 4096;
 template <bool FROM_LOGITS>
-__global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
+__global__ void __launch_bounds__(32 * kSelWarps) row_select_warp_kernel(
     const float* in, float* scores, long long rows, int nb, int mode_flags, float T, int k, float density,
     int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, int row_len, const int2* __restrict__ tab) {
-  constexpr int NPL = kSelNPL;
-  __shared__ uint32_t hist_all[kSelWarps][256];
+  extern __shared__ uint32_t sel_smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kSelWarps + wid;
   if (row >= rows) return;  // whole warps only: no CTA barrier follows
-  uint32_t* const hist = hist_all[wid];
+  const int width = row_len > 0 ? row_len : nb;  // candidates of a row, at most
+  uint32_t* const hist = sel_smem + wid * 256;
+  float* const buf = reinterpret_cast<float*>(sel_smem + kSelWarps * 256) + (size_t)wid * width;
+  uint32_t* const key = reinterpret_cast<uint32_t*>(buf);
   const unsigned lt = (1u << lane) - 1u;
 
   const int mode = mode_flags & 0xff;
@@ -739,59 +753,44 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
   }
   const int i = ig - off;
   const int len = i + 1;
-  const int nt = (len + 31) >> 5;  // register slots in use
+  const int nt = (len + 31) >> 5;  // 32-candidate chunks
   const float* src = in + row * (long long)nb + off;
-  // Every loop over the register slots stops at the row's last slot (a
-  // warp-uniform exit), so short rows cost little.
-  float v[NPL];
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    if (t >= nt) break;
-    const int j = 32 * t + lane;
-    v[t] = j < len ? src[j] : -INFINITY;
+  // The row into shared memory.  Lane sums run in the same candidate order
+  // as the per-row kernels' (j = lane, lane + 32, ...), then one butterfly.
+  float m = -INFINITY;
+#pragma unroll 4
+  for (int j = lane; j < len; j += 32) {
+    const float x = src[j];
+    buf[j] = x;
+    m = fmaxf(m, x);
   }
   if (FROM_LOGITS) {
-    float m = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) {
-      if (t >= nt) break;
-      m = fmaxf(m, v[t]);
-    }
     m = warp_max(m);
     float sum = 0.f;
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) {
-      if (t >= nt) break;
-      v[t] = expf(v[t] - m);  // exp(-inf) = 0 past the row's end
-      sum += v[t];
+#pragma unroll 4
+    for (int j = lane; j < len; j += 32) {
+      const float e = expf(buf[j] - m);
+      buf[j] = e;
+      sum += e;
     }
     const float inv = 1.0f / warp_sum(sum);
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) {
-      if (t >= nt) break;
-      v[t] *= inv;
+#pragma unroll 4
+    for (int j = lane; j < len; j += 32) {
+      const float v = buf[j] * inv;
+      buf[j] = v;
+      if (dst) dst[off + j] = v;
     }
-    if (dst) {
-      // the window off .. off + len - 1 from the registers, zeros elsewhere
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) {
-        if (t >= nt) break;
-        const int j = 32 * t + lane;
-        if (j < len) dst[off + j] = v[t];
-      }
+    if (dst)
       for (int j = lane; j < nb; j += 32)
         if (j < off || j >= off + len) dst[j] = 0.f;
-    }
   }
   int32_t* out = indices + row * (long long)cap;
 
   if (mode == SEER_SELECT_THRESHOLD) {
     int base = 0;
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) {
-      if (t >= nt) break;
+    for (int t = 0; t < nt; ++t) {
       const int j = 32 * t + lane;
-      const bool keep = j < len && (v[t] > T || (force_diag && j == i));
+      const bool keep = j < len && (buf[j] > T || (force_diag && j == i));
       const unsigned km = __ballot_sync(0xffffffffu, keep);
       if (keep) out[base + __popc(km & lt)] = j + off;
       base += __popc(km);
@@ -807,27 +806,20 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
     return;
   }
 
-  // The order-preserving keys replace the values (as bit patterns; slots
-  // past the row hold 0 and are never counted).
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    if (t >= nt) break;
-    v[t] = __uint_as_float(32 * t + lane < len ? f2key(v[t]) : 0u);
-  }
-  // Radix select of the ki-th largest key, 8 bits at a time.  Bits that all
-  // of the row's keys share are fixed at once (a warp AND / OR of the keys):
-  // a softmax row's values lie close together, so its keys agree on the
-  // sign, the exponent and the top of the mantissa, and the first digit
-  // starts at the highest bit where they differ.  The search also stops as
-  // soon as the bin holding the ki-th key is taken whole.
+  // Order-preserving keys replace the values.  Radix select of the ki-th
+  // largest key, 8 bits at a time.  Bits that all of the row's keys share
+  // are fixed at once (a warp AND / OR of the keys): a softmax row's values
+  // lie close together, so its keys agree on the sign, the exponent and the
+  // top of the mantissa, and the first digit starts at the highest bit where
+  // they differ.  The search also stops as soon as the bin holding the ki-th
+  // key is taken whole.
   uint32_t kand = 0xffffffffu, kor = 0u;
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    if (t >= nt) break;
-    if (32 * t + lane < len) {
-      kand &= __float_as_uint(v[t]);
-      kor |= __float_as_uint(v[t]);
-    }
+#pragma unroll 4
+  for (int j = lane; j < len; j += 32) {
+    const uint32_t kk = f2key(buf[j]);
+    key[j] = kk;
+    kand &= kk;
+    kor |= kk;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -844,15 +836,12 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
 #pragma unroll
     for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
     __syncwarp();
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) {
-      if (t >= nt) break;
-      const uint32_t kt = __float_as_uint(v[t]);
-      // not counted: past the row, or outside the prefix chosen so far
-      const uint32_t bin = (32 * t + lane < len && (kt & pmask) == prefix) ? (kt >> shift) & 0xffu : 0x100u;
+#pragma unroll 4
+    for (int j = lane; j < len; j += 32) {
+      const uint32_t kt = key[j];
       // plain shared atomics: measured faster here than first aggregating
-      // the lanes of equal bins with a warp match (563 against 786 us at 128k)
-      if (bin != 0x100u) atomicAdd(&hist[bin], 1u);
+      // the lanes of equal bins with a warp match
+      if ((kt & pmask) == prefix) atomicAdd(&hist[(kt >> shift) & 0xffu], 1u);
     }
     __syncwarp();
     // lane l owns bins 255-8l .. 248-8l (descending)
@@ -869,7 +858,7 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
       if (lane >= o) incl += y;
     }
     const uint32_t excl = incl - part;
-    uint32_t sel_bin = 0, sel_rem = 0;
+    uint32_t sel_bin = 0, sel_rem = 0, sel_cnt = 0;
     const bool mine = excl < remaining && remaining <= incl;
     if (mine) {
       uint32_t before = excl;
@@ -878,6 +867,7 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
         if (before < remaining && remaining <= before + cnt[q]) {
           sel_bin = (uint32_t)(255 - 8 * lane - q);
           sel_rem = remaining - before;
+          sel_cnt = cnt[q];
         }
         before += cnt[q];
       }
@@ -885,7 +875,7 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
     const int owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
     sel_bin = __shfl_sync(0xffffffffu, sel_bin, owner);
     sel_rem = __shfl_sync(0xffffffffu, sel_rem, owner);
-    const uint32_t sel_cnt = __shfl_sync(0xffffffffu, hist[sel_bin], 0);
+    sel_cnt = __shfl_sync(0xffffffffu, sel_cnt, owner);
     prefix |= sel_bin << shift;
     remaining = sel_rem;
     pmask |= 0xffu << shift;
@@ -900,11 +890,9 @@ __global__ void __launch_bounds__(32 * kSelWarps, 2) row_select_warp_kernel(
   // joins when forced
   int base = 0;
   uint32_t eq_before = 0;
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    if (t >= nt) break;
+  for (int t = 0; t < nt; ++t) {
     const int j = 32 * t + lane;
-    const uint32_t kt = __float_as_uint(v[t]) & pmask;
+    const uint32_t kt = j < len ? key[j] & pmask : 0u;
     const bool eq = j < len && kt == prefix;
     const unsigned em = __ballot_sync(0xffffffffu, eq);
     const uint32_t rank = eq_before + __popc(em & lt);
@@ -1030,12 +1018,17 @@ cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, 
   // Few rows (the decode gate, small batches) leave most SMs idle and each
   // row's latency exposed: then 1024 threads share a row's work.
   const bool wide = rows < 2LL * 148;
-  // Many rows of at most 2048 candidates: one warp per row
-  if (!wide && rows >= 8LL * 148 && nb <= 32 * kSelNPL && (row_len > 0 ? row_len : nb) <= 32 * kSelNPL) {
+  // Many rows of at most kSelMaxWidth candidates: one warp per row, the row
+  // in shared memory
+  const int width = row_len > 0 ? row_len : nb;
+  if (!wide && rows >= 8LL * 148 && width <= kSelMaxWidth) {
     const unsigned grid = (unsigned)((rows + kSelWarps - 1) / kSelWarps);
+    const size_t smem = sizeof(uint32_t) * (size_t)kSelWarps * (256 + width);
     auto kern = from_logits ? row_select_warp_kernel<true> : row_select_warp_kernel<false>;
-    kern<<<grid, 32 * kSelWarps, 0, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density, counts,
-                                             indices, cap, row_len, tab);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 32 * kSelWarps, smem, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density,
+                                             counts, indices, cap, row_len, tab);
     return cudaGetLastError();
   }
   if (from_logits)
