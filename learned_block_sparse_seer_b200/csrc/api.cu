@@ -164,12 +164,14 @@ cudaError_t to_bf16(const void* x, void* y, long long n, cudaStream_t st) {
 }
 
 struct GateWs {
-  size_t qbar, kbar, qt, kt, logits, qlo, klo, total;
+  size_t qbar, kbar, qt, kt, logits, qlo, klo, qbar_hi, qbar_lo, kbar_hi, kbar_lo, wq_hi, wq_lo, wk_hi, wk_lo, total;
 };
 
 // The causal logits run on the tensor cores (three tf32 products) when the
 // gate hidden size is a multiple of 32; otherwise on the fp32 SIMT GEMM.
 bool gate_tf32x3(int h) { return h % 32 == 0; }
+// The projections too, when the head dimension is a multiple of 32 as well.
+bool gate_proj_tf32x3(int h, int d) { return h % 32 == 0 && d % 32 == 0; }
 
 GateWs gate_ws(const seer_dims* d, int h) {
   const long long nb = d->n / seer::kBlock;
@@ -183,6 +185,17 @@ GateWs gate_ws(const seer_dims* d, int h) {
   // tf32 remainders of q~ and k~ (the tensor-core logits only)
   w.qlo = gate_tf32x3(h) ? c.take(sizeof(float) * d->B * d->Hq * nb * h) : 0;
   w.klo = gate_tf32x3(h) ? c.take(sizeof(float) * d->B * d->Hkv * nb * h) : 0;
+  // tf32 parts of the pooled Q / K and of the weights, for the projections
+  // (the pooled fp32 values stay as they are: the distillation step reads them)
+  const bool pj = gate_proj_tf32x3(h, d->d);
+  w.qbar_hi = pj ? c.take(sizeof(float) * d->B * d->Hq * nb * d->d) : 0;
+  w.qbar_lo = pj ? c.take(sizeof(float) * d->B * d->Hq * nb * d->d) : 0;
+  w.kbar_hi = pj ? c.take(sizeof(float) * d->B * d->Hkv * nb * 3 * d->d) : 0;
+  w.kbar_lo = pj ? c.take(sizeof(float) * d->B * d->Hkv * nb * 3 * d->d) : 0;
+  w.wq_hi = pj ? c.take(sizeof(float) * d->Hq * h * d->d) : 0;
+  w.wq_lo = pj ? c.take(sizeof(float) * d->Hq * h * d->d) : 0;
+  w.wk_hi = pj ? c.take(sizeof(float) * d->Hkv * h * 3 * d->d) : 0;
+  w.wk_lo = pj ? c.take(sizeof(float) * d->Hkv * h * 3 * d->d) : 0;
   w.total = c.off;
   return w;
 }
@@ -457,11 +470,56 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
   SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st, tab));
   SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st, tab));
   // q~ = Wq[hq] qbar, k~ = Wk[g] kbar (batch z = b*H + head; weights by head)
-  SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
-                                 (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
-  SEER_CUDA(seer::launch_gemm_nt(kbar, Wk, kt, nb, h, 3 * d, (long long)nb * 3 * d,
-                                 (long long)h * 3 * d, (long long)nb * h, h, B * Hkv, Hkv, 0, 1,
-                                 1.0f, false, st));
+  if (gate_proj_tf32x3(h, d)) {
+    // on the tensor cores, three tf32 products as for the logits
+    float* qbhi = (float*)(base + w.qbar_hi);
+    float* qblo = (float*)(base + w.qbar_lo);
+    float* kbhi = (float*)(base + w.kbar_hi);
+    float* kblo = (float*)(base + w.kbar_lo);
+    float* wqh = (float*)(base + w.wq_hi);
+    float* wql = (float*)(base + w.wq_lo);
+    float* wkh = (float*)(base + w.wk_hi);
+    float* wkl = (float*)(base + w.wk_lo);
+    SEER_CUDA(seer::launch_split_tf32_copy(qbar, qbhi, qblo, (long long)B * Hq * nb * d, st));
+    SEER_CUDA(seer::launch_split_tf32_copy(kbar, kbhi, kblo, (long long)B * Hkv * nb * 3 * d, st));
+    SEER_CUDA(seer::launch_split_tf32_copy(Wq, wqh, wql, (long long)Hq * h * d, st));
+    SEER_CUDA(seer::launch_split_tf32_copy(Wk, wkh, wkl, (long long)Hkv * h * 3 * d, st));
+    CUtensorMap tmAh, tmAl, tmBh, tmBl;
+    seer::Tf32x3Params tp;
+    tp.M = nb;
+    tp.N = h;
+    tp.ldc = h;
+    tp.zmul = 0;
+    tp.zg = 1;
+    tp.causal = 0;
+    tp.c_bs = (long long)nb * h;
+    tp.alpha = 1.0f;
+    tp.status = &((seer::WsHeader*)ws)->status;
+    tp.timeout_ns = kTimeoutNs;
+    if (!make_tmap_f32(&tmAh, qbhi, (long long)B * Hq * nb, d, 128) ||
+        !make_tmap_f32(&tmAl, qblo, (long long)B * Hq * nb, d, 128) ||
+        !make_tmap_f32(&tmBh, wqh, (long long)Hq * h, d, 128) || !make_tmap_f32(&tmBl, wql, (long long)Hq * h, d, 128))
+      return cuda_fail(cudaErrorInvalidValue);
+    tp.K = d;
+    tp.zh = Hq;
+    tp.C = qt;
+    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hq, st));
+    if (!make_tmap_f32(&tmAh, kbhi, (long long)B * Hkv * nb, 3 * d, 128) ||
+        !make_tmap_f32(&tmAl, kblo, (long long)B * Hkv * nb, 3 * d, 128) ||
+        !make_tmap_f32(&tmBh, wkh, (long long)Hkv * h, 3 * d, 128) ||
+        !make_tmap_f32(&tmBl, wkl, (long long)Hkv * h, 3 * d, 128))
+      return cuda_fail(cudaErrorInvalidValue);
+    tp.K = 3 * d;
+    tp.zh = Hkv;
+    tp.C = kt;
+    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hkv, st));
+  } else {
+    SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
+                                   (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
+    SEER_CUDA(seer::launch_gemm_nt(kbar, Wk, kt, nb, h, 3 * d, (long long)nb * 3 * d,
+                                   (long long)h * 3 * d, (long long)nb * h, h, B * Hkv, Hkv, 0, 1,
+                                   1.0f, false, st));
+  }
   if (rope_theta > 0.f) {
     SEER_CUDA(seer::launch_rope(qt, (long long)B * Hq * nb, nb, h, rope_theta, st));
     SEER_CUDA(seer::launch_rope(kt, (long long)B * Hkv * nb, nb, h, rope_theta, st));
@@ -487,6 +545,7 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     tp.zh = Hq;
     tp.zmul = Hkv;
     tp.zg = G;
+    tp.causal = 1;
     tp.c_bs = (long long)nb * nb;
     tp.alpha = alpha;
     tp.C = logits;

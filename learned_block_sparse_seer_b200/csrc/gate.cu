@@ -300,6 +300,18 @@ __global__ void split_tf32_kernel(float* __restrict__ x, float* __restrict__ lo,
   }
 }
 
+__global__ void split_tf32_copy_kernel(const float* __restrict__ x, float* __restrict__ hi_out,
+                                       float* __restrict__ lo, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    uint32_t h;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
+    const float hi = __uint_as_float(h);
+    hi_out[i] = hi;
+    lo[i] = v - hi;
+  }
+}
+
 namespace gt3 {
 // One stage of 64 KB per CTA: three CTAs share an SM, so one tile's loads,
 // products and epilogue overlap the others' (a tile is only four 32-float
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
                                                              const Tf32x3Params p) {
   using namespace gt3;
   const int tm = blockIdx.x, tn = blockIdx.y, z = blockIdx.z;
-  if (tn > tm) return;  // causal: tiles strictly above the diagonal are never read
+  if (p.causal && tn > tm) return;  // causal: tiles strictly above the diagonal are never read
   extern __shared__ uint8_t gt3_raw[];
   uint8_t* const ring = gt3_raw + ((1024u - (smem_u32(gt3_raw) & 1023u)) & 1023u);
   __shared__ uint64_t full[kStages], empty[kStages], done;
@@ -441,6 +453,11 @@ cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap
 
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st) {
   split_tf32_kernel<<<1184, 256, 0, st>>>(x, lo, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_tf32_copy(const float* x, float* hi, float* lo, long long n, cudaStream_t st) {
+  split_tf32_copy_kernel<<<592, 256, 0, st>>>(x, hi, lo, n);
   return cudaGetLastError();
 }
 

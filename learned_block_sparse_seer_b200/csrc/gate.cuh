@@ -19,13 +19,16 @@ cudaError_t launch_gemm_nt(const float* A, const float* B, float* C, int M, int 
                            long long a_bs, long long b_bs, long long c_bs, int ldc, int batch,
                            int zh, int zmul, int zg, float alpha, bool causal, cudaStream_t st);
 
-// The causal logits C[z] = alpha * A[z] B[bz]^T on the tensor cores in three
-// tf32 products (fp32-level accuracy).  A, B are split first: launch_split_tf32
-// rounds x to tf32 in place and writes the remainder to lo.  tmAh/tmAl are
-// fp32 maps over A's hi/lo [batch * M rows, K], tmBh/tmBl over B's
-// [(max bz + 1) * N rows, K], 32 x 128 boxes, 128-byte swizzle.  K % 32 == 0.
+// C[z] = alpha * A[z] B[bz]^T on the tensor cores in three tf32 products
+// (fp32-level accuracy): the gate's causal logits (causal = 1: tiles above
+// the diagonal are skipped) and its projections (causal = 0).  A, B are split
+// first: launch_split_tf32 rounds x to tf32 in place and writes the remainder
+// to lo; launch_split_tf32_copy writes both parts to separate buffers (for
+// inputs the caller owns).  tmAh/tmAl are fp32 maps over A's hi/lo
+// [batch * M rows, K], tmBh/tmBl over B's [(max bz + 1) * N rows, K],
+// 32 x 128 boxes, 128-byte swizzle.  K % 32 == 0.
 struct Tf32x3Params {
-  int M, N, K, ldc, zh, zmul, zg;
+  int M, N, K, ldc, zh, zmul, zg, causal;
   long long c_bs;
   float alpha;
   float* C;
@@ -33,6 +36,7 @@ struct Tf32x3Params {
   unsigned long long timeout_ns;
 };
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st);
+cudaError_t launch_split_tf32_copy(const float* x, float* hi, float* lo, long long n, cudaStream_t st);
 cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
                                       const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st);
 
