@@ -123,6 +123,22 @@ bool make_tmap_f32_panels(CUtensorMap* tm, const void* base, long long rows, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over a batch of row-major matrices C[z][rows][cols] with row
+// stride ld and batch stride bs (in elements): a box of 32 columns x 128 rows
+// x 1 matrix, 128-byte swizzle (the TMA-store staging layout).
+bool make_tmap_f32_batched(CUtensorMap* tm, const void* base, int cols, int rows, int batch, long long ld,
+                           long long bs) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 4, (cuuint64_t)bs * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 map over a row-major [rows, inner] matrix seen as (64 columns,
 // rows, inner/64 panels): a box of 64 x box_rows x inner/64 lands as
 // inner/64 consecutive 128-byte-swizzled panels of box_rows rows.
@@ -467,11 +483,13 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
   const int B = dims->B, Hq = dims->Hq, Hkv = dims->Hkv, n = dims->n, d = dims->d;
   const int nb = n / seer::kBlock, G = Hq / Hkv;
 
-  SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st, tab));
-  SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st, tab));
   // q~ = Wq[hq] qbar, k~ = Wk[g] kbar (batch z = b*H + head; weights by head)
-  if (gate_proj_tf32x3(h, d)) {
-    // on the tensor cores, three tf32 products as for the logits
+  const bool proj_tc = gate_proj_tf32x3(h, d);
+  // without RoPE the projections write q~ and k~ already split for the logits
+  const bool split_in_proj = proj_tc && gate_tf32x3(h) && !(rope_theta > 0.f);
+  if (proj_tc) {
+    // on the tensor cores, three tf32 products as for the logits; the pooling
+    // writes qbar and kbar already split into their tf32 parts and remainders
     float* qbhi = (float*)(base + w.qbar_hi);
     float* qblo = (float*)(base + w.qbar_lo);
     float* kbhi = (float*)(base + w.kbar_hi);
@@ -480,8 +498,8 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     float* wql = (float*)(base + w.wq_lo);
     float* wkh = (float*)(base + w.wk_hi);
     float* wkl = (float*)(base + w.wk_lo);
-    SEER_CUDA(seer::launch_split_tf32_copy(qbar, qbhi, qblo, (long long)B * Hq * nb * d, st));
-    SEER_CUDA(seer::launch_split_tf32_copy(kbar, kbhi, kblo, (long long)B * Hkv * nb * 3 * d, st));
+    SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbhi, st, tab, qblo));
+    SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbhi, st, tab, kblo));
     SEER_CUDA(seer::launch_split_tf32_copy(Wq, wqh, wql, (long long)Hq * h * d, st));
     SEER_CUDA(seer::launch_split_tf32_copy(Wk, wkh, wkl, (long long)Hkv * h * 3 * d, st));
     CUtensorMap tmAh, tmAl, tmBh, tmBl;
@@ -494,6 +512,8 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     tp.causal = 0;
     tp.c_bs = (long long)nb * h;
     tp.alpha = 1.0f;
+    tp.C_lo = nullptr;
+    tp.tma_out = 1;
     tp.status = &((seer::WsHeader*)ws)->status;
     tp.timeout_ns = kTimeoutNs;
     if (!make_tmap_f32(&tmAh, qbhi, (long long)B * Hq * nb, d, 128) ||
@@ -503,7 +523,12 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     tp.K = d;
     tp.zh = Hq;
     tp.C = qt;
-    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hq, st));
+    tp.C_lo = split_in_proj ? (float*)(base + w.qlo) : nullptr;
+    CUtensorMap tmC, tmClo;
+    if (!make_tmap_f32_batched(&tmC, qt, h, nb, B * Hq, h, (long long)nb * h) ||
+        !make_tmap_f32_batched(&tmClo, tp.C_lo ? tp.C_lo : qt, h, nb, B * Hq, h, (long long)nb * h))
+      return cuda_fail(cudaErrorInvalidValue);
+    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tmC, tmClo, tp, B * Hq, st));
     if (!make_tmap_f32(&tmAh, kbhi, (long long)B * Hkv * nb, 3 * d, 128) ||
         !make_tmap_f32(&tmAl, kblo, (long long)B * Hkv * nb, 3 * d, 128) ||
         !make_tmap_f32(&tmBh, wkh, (long long)Hkv * h, 3 * d, 128) ||
@@ -512,8 +537,14 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     tp.K = 3 * d;
     tp.zh = Hkv;
     tp.C = kt;
-    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hkv, st));
+    tp.C_lo = split_in_proj ? (float*)(base + w.klo) : nullptr;
+    if (!make_tmap_f32_batched(&tmC, kt, h, nb, B * Hkv, h, (long long)nb * h) ||
+        !make_tmap_f32_batched(&tmClo, tp.C_lo ? tp.C_lo : kt, h, nb, B * Hkv, h, (long long)nb * h))
+      return cuda_fail(cudaErrorInvalidValue);
+    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tmC, tmClo, tp, B * Hkv, st));
   } else {
+    SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbar, st, tab));
+    SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbar, st, tab));
     SEER_CUDA(seer::launch_gemm_nt(qbar, Wq, qt, nb, h, d, (long long)nb * d, (long long)h * d,
                                    (long long)nb * h, h, B * Hq, Hq, 0, 1, 1.0f, false, st));
     SEER_CUDA(seer::launch_gemm_nt(kbar, Wk, kt, nb, h, 3 * d, (long long)nb * 3 * d,
@@ -529,8 +560,10 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
   if (gate_tf32x3(h)) {
     float* qlo = (float*)(base + w.qlo);
     float* klo = (float*)(base + w.klo);
-    SEER_CUDA(seer::launch_split_tf32(qt, qlo, (long long)B * Hq * nb * h, st));
-    SEER_CUDA(seer::launch_split_tf32(kt, klo, (long long)B * Hkv * nb * h, st));
+    if (!split_in_proj) {
+      SEER_CUDA(seer::launch_split_tf32(qt, qlo, (long long)B * Hq * nb * h, st));
+      SEER_CUDA(seer::launch_split_tf32(kt, klo, (long long)B * Hkv * nb * h, st));
+    }
     CUtensorMap tmAh, tmAl, tmBh, tmBl;
     if (!make_tmap_f32(&tmAh, qt, (long long)B * Hq * nb, h, 128) ||
         !make_tmap_f32(&tmAl, qlo, (long long)B * Hq * nb, h, 128) ||
@@ -549,9 +582,21 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     tp.c_bs = (long long)nb * nb;
     tp.alpha = alpha;
     tp.C = logits;
+    tp.C_lo = nullptr;
+    tp.tma_out = 0;
     tp.status = &((seer::WsHeader*)ws)->status;
     tp.timeout_ns = kTimeoutNs;
-    SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tp, B * Hq, st));
+    // each q~ row block held on chip while its key tiles stream past (h <= 128)
+    if (seer::gemm_tf32x3_rows_fits(h, nb, tp.c_bs, logits)) {
+      CUtensorMap tmAph, tmApl, tmC;
+      if (!make_tmap_f32_panels(&tmAph, qt, (long long)B * Hq * nb, h, 128) ||
+          !make_tmap_f32_panels(&tmApl, qlo, (long long)B * Hq * nb, h, 128) ||
+          !make_tmap_f32_batched(&tmC, logits, nb, nb, B * Hq, nb, tp.c_bs))
+        return cuda_fail(cudaErrorInvalidValue);
+      SEER_CUDA(seer::launch_gemm_tf32x3_rows(tmAph, tmApl, tmBh, tmBl, tmC, tp, B * Hq, num_sms(), st));
+    } else {
+      SEER_CUDA(seer::launch_gemm_tf32x3_causal(tmAh, tmAl, tmBh, tmBl, tmAh, tmAh, tp, B * Hq, st));
+    }
   } else {
     SEER_CUDA(seer::launch_gemm_nt(qt, kt, logits, nb, nb, h, (long long)nb * h, (long long)nb * h,
                                    (long long)nb * nb, nb, B * Hq, Hq, Hkv, G, alpha, true, st));

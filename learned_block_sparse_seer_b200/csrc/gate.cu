@@ -39,10 +39,18 @@ namespace seer {
 // lanes that cover the same columns are combined with shuffles at the end.
 // With a varlen table, block i pools only its tab[i].y valid tokens (the
 // sequence's last block may be partial); a block of no sequence writes 0.
+// With lo non-null the result is written split for the tf32x3 products: the
+// value rounded to tf32 into out, the exact remainder into lo.
+__device__ __forceinline__ float tf32_hi(float v) {
+  uint32_t h;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
+  return __uint_as_float(h);
+}
+
 template <typename T, bool IS_K>
 __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long long nblocks,
                                                    int n, int d, float* __restrict__ out,
-                                                   const int2* __restrict__ tab) {
+                                                   const int2* __restrict__ tab, float* __restrict__ lo) {
   constexpr int EPL = 16 / sizeof(T);  // elements per lane per load
   const long long warp = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (warp >= nblocks) return;
@@ -100,18 +108,36 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
   }
   if (lane < lpr) {
     const float inv = valid > 0 ? 1.0f / (float)valid : 0.f;
-    if (!IS_K) {
-      float* o = out + ((bh * nb) + i) * (long long)d + cg * EPL;
+    const int w = IS_K ? 3 * d : d;
+    const long long at = ((bh * nb) + i) * (long long)w + cg * EPL;
+    // EPL consecutive floats per part, 16-byte aligned: float4 stores
+    auto put = [&](int c, const float (&v)[EPL]) {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) o[e] = sum[e] * inv;
-    } else {
-      float* o = out + ((bh * nb) + i) * (long long)(3 * d) + cg * EPL;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        o[e] = valid > 0 ? mx[e] : 0.f;
-        o[d + e] = valid > 0 ? mn[e] : 0.f;
-        o[2 * d + e] = sum[e] * inv;
+      for (int e = 0; e < EPL; e += 4) {
+        float4 x = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        if (lo) {
+          const float4 hv = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+          *reinterpret_cast<float4*>(lo + at + c + e) = make_float4(x.x - hv.x, x.y - hv.y, x.z - hv.z, x.w - hv.w);
+          x = hv;
+        }
+        *reinterpret_cast<float4*>(out + at + c + e) = x;
       }
+    };
+    float v[EPL];
+    if (!IS_K) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) v[e] = sum[e] * inv;
+      put(0, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) v[e] = valid > 0 ? mx[e] : 0.f;
+      put(0, v);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) v[e] = valid > 0 ? mn[e] : 0.f;
+      put(d, v);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) v[e] = sum[e] * inv;
+      put(2 * d, v);
     }
   }
 }
@@ -313,19 +339,22 @@ __global__ void split_tf32_copy_kernel(const float* __restrict__ x, float* __res
 }
 
 namespace gt3 {
-// One stage of 64 KB per CTA: three CTAs share an SM, so one tile's loads,
-// products and epilogue overlap the others' (a tile is only four 32-float
-// slices deep, too short to pipeline within one CTA).
-constexpr int kStages = 1;
+// With one stage of 64 KB per CTA, three CTAs share an SM, so one tile's
+// loads, products and epilogue overlap the others' (for many shallow tiles).
+// Few deep tiles (a projection with K = 3d) take three stages instead, so
+// that one CTA's slices stream while it multiplies.
 constexpr uint32_t kOp = 128u * 128u;                 // one operand slice: 128 rows x 32 floats
 constexpr uint32_t kStage = 4u * kOp;                 // Ah, Al, Bh, Bl
-constexpr uint32_t kSmem = kStages * kStage + 1024u;  // + slack to align the ring to 1024 bytes
+constexpr uint32_t smem_bytes(int stages) { return (uint32_t)stages * kStage + 1024u; }  // + alignment slack
 }  // namespace gt3
 
+template <int kStages>
 __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmAh,
                                                              const __grid_constant__ CUtensorMap tmAl,
                                                              const __grid_constant__ CUtensorMap tmBh,
                                                              const __grid_constant__ CUtensorMap tmBl,
+                                                             const __grid_constant__ CUtensorMap tmC,
+                                                             const __grid_constant__ CUtensorMap tmClo,
                                                              const Tf32x3Params p) {
   using namespace gt3;
   const int tm = blockIdx.x, tn = blockIdx.y, z = blockIdx.z;
@@ -405,14 +434,71 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
   const int gm = tm * 128 + r;
   float* const crow = p.C + (long long)z * p.c_bs + (long long)gm * p.ldc;
   const bool vec = (p.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(p.C + (long long)z * p.c_bs) & 15) == 0;
+  if (p.tma_out) {
+    // Every product is done, so the ring is free: 32-column chunks go through
+    // 128-byte-swizzled staging tiles there (two per output, alternating)
+    // and leave by TMA stores, clipped at the matrix's edges.
+    const bool all_ok = __syncthreads_and(ok) != 0;
 #pragma unroll 1
-  for (int c0 = 0; c0 < 128; c0 += 32) {
+    for (int c = 0; c < 4 && all_ok; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(32 * c), v);
+      tmem_wait_ld();
+      uint8_t* const sh = ring + (c & 1) * 16384;
+      uint8_t* const sl = ring + 32768 + (c & 1) * 16384;
+      if (threadIdx.x == 0 && c >= 2) bulk_wait_group_read<1>();  // the slot's previous store has read it
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float4 x = make_float4(p.alpha * __uint_as_float(v[4 * k]), p.alpha * __uint_as_float(v[4 * k + 1]),
+                               p.alpha * __uint_as_float(v[4 * k + 2]), p.alpha * __uint_as_float(v[4 * k + 3]));
+        const uint32_t at = (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
+        if (p.C_lo) {
+          const float4 hv = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+          *reinterpret_cast<float4*>(sl + at) = make_float4(x.x - hv.x, x.y - hv.y, x.z - hv.z, x.w - hv.w);
+          x = hv;
+        }
+        *reinterpret_cast<float4*>(sh + at) = x;
+      }
+      fence_async_shared();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        tma_store_3d(&tmC, sh, tn * 128 + 32 * c, tm * 128, z);
+        if (p.C_lo) tma_store_3d(&tmClo, sl, tn * 128 + 32 * c, tm * 128, z);
+        bulk_commit_group();
+      }
+    }
+    if (threadIdx.x == 0) bulk_wait_group<0>();
+  }
+#pragma unroll 1
+  for (int c0 = 0; c0 < 128 && !p.tma_out; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
     tmem_wait_ld();
     const int gn = tn * 128 + c0;
     if (ok && gm < p.M && gn < p.N) {
-      if (vec && gn + 32 <= p.N) {
+      if (p.C_lo && vec && gn + 32 <= p.N) {
+        // split output: tf32 part into C, exact remainder into C_lo
+        float* const lrow = p.C_lo + (long long)z * p.c_bs + (long long)gm * p.ldc;
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const float4 x = make_float4(p.alpha * __uint_as_float(v[q]), p.alpha * __uint_as_float(v[q + 1]),
+                                       p.alpha * __uint_as_float(v[q + 2]), p.alpha * __uint_as_float(v[q + 3]));
+          const float4 hv = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+          *reinterpret_cast<float4*>(crow + gn + q) = hv;
+          *reinterpret_cast<float4*>(lrow + gn + q) = make_float4(x.x - hv.x, x.y - hv.y, x.z - hv.z, x.w - hv.w);
+        }
+      } else if (p.C_lo) {
+        float* const lrow = p.C_lo + (long long)z * p.c_bs + (long long)gm * p.ldc;
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (gn + q < p.N) {
+            const float x = p.alpha * __uint_as_float(v[q]);
+            const float hv = tf32_hi(x);
+            crow[gn + q] = hv;
+            lrow[gn + q] = x - hv;
+          }
+      } else if (vec && gn + 32 <= p.N) {
 #pragma unroll
         for (int q = 0; q < 32; q += 4)
           *reinterpret_cast<float4*>(crow + gn + q) =
@@ -442,12 +528,307 @@ __global__ void __launch_bounds__(128, 1) gemm_tf32x3_kernel(const __grid_consta
 }
 
 cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
-                                      const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gt3::kSmem);
-  if (e != cudaSuccess) return e;
+                                      const CUtensorMap& tmBl, const CUtensorMap& tmC, const CUtensorMap& tmClo,
+                                      const Tf32x3Params& p, int batch, cudaStream_t st) {
   dim3 grid((p.M + 127) / 128, (p.N + 127) / 128, batch);
-  gemm_tf32x3_kernel<<<grid, 128, gt3::kSmem, st>>>(tmAh, tmAl, tmBh, tmBl, p);
+  // deep tiles (more than four slices) stream through three stages
+  const bool deep = p.K > 128;
+  auto kern = deep ? gemm_tf32x3_kernel<3> : gemm_tf32x3_kernel<1>;
+  const uint32_t smem = gt3::smem_bytes(deep ? 3 : 1);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 128, smem, st>>>(tmAh, tmAl, tmBh, tmBl, tmC, tmClo, p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------- tf32x3 causal logits, by rows --
+// The causal logits with the query side held on chip: a CTA takes one
+// 128-row block of q~ at a time, copies its tf32 parts and remainders into
+// tensor memory (tcgen05.cp; A of TS-form MMAs), and sweeps the key tiles
+// tn = 0..tm up to the diagonal, so each q~ row block crosses L2 once and
+// the MMAs read only the key slices from shared memory.  Warp 0 loads by
+// TMA (no cluster multicast), warp 1 issues the copies and MMAs into one of
+// two TMEM accumulators while warps 2..5 drain the other: each 32-column
+// chunk goes through a 128-byte-swizzled staging tile in shared memory and
+// leaves by a TMA store (clipped at the matrix's edges).  Work items
+// (z, tm), tm + 1 tiles each, are dealt out statically: largest first, in
+// snake order across the CTAs so that each CTA's total is close to the mean.
+namespace gtr {
+constexpr int kBStages = 4;
+constexpr uint32_t kSlice = 128u * 128u;            // 128 rows x 32 floats
+constexpr int kMaxSlices = 4;                       // h <= 128
+constexpr uint32_t kAStage = kMaxSlices * kSlice;   // one part of the q~ block: 64 KB
+constexpr uint32_t kBStage = 2u * kSlice;           // one 32-column slice of a k~ tile, both parts: 32 KB
+constexpr uint32_t kOut = kSlice;                   // one 128 x 32 output chunk: 16 KB
+constexpr uint32_t kSmem = kAStage + kBStages * kBStage + 2u * kOut + 1024u;
+constexpr int kThreads = 192;
+constexpr uint32_t kColAh = 256, kColAl = 384;      // TMEM: accumulators at 0 and 128
+}  // namespace gtr
+
+// Item w of this CTA's r-th round (snake order), or -1 past the end.
+__device__ __forceinline__ int gtr_item(int r, int items) {
+  const int G = (int)gridDim.x, b = (int)blockIdx.x;
+  const int w = r * G + ((r & 1) ? G - 1 - b : b);
+  return w < items ? w : -1;
+}
+
+__global__ void __launch_bounds__(gtr::kThreads, 1)
+    gemm_tf32x3_rows_kernel(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
+                            const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmBl,
+                            const __grid_constant__ CUtensorMap tmC, const Tf32x3Params p, int batch) {
+  using namespace gtr;
+  extern __shared__ uint8_t gtr_raw[];
+  uint8_t* const sA = gtr_raw + ((1024u - (smem_u32(gtr_raw) & 1023u)) & 1023u);
+  uint8_t* const sB = sA + kAStage;
+  uint8_t* const sO = sB + kBStages * kBStage;
+  __shared__ uint64_t a_full, a_free, atm_free, b_full[kBStages], b_empty[kBStages], acc_full[2], acc_empty[2], done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  // teardown accounting: q~ parts and key slices whose copies went out / were consumed
+  __shared__ int a_issued, a_used, b_issued, b_used;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_p = &abort_flag;
+  const uint64_t tmo = p.timeout_ns;
+  const int nk = p.K / 32;  // 32-column slices, at most kMaxSlices
+  const int T = (p.M + 127) / 128;
+  const int items = T * batch;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    a_issued = a_used = b_issued = b_used = 0;
+    mbar_init(&a_full, 1);
+    mbar_init(&a_free, 1);
+    mbar_init(&atm_free, 1);
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);
+    }
+    mbar_init(&done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads --
+    if (lane == 0) {
+      prefetch_tmap(&tmAh);
+      prefetch_tmap(&tmAl);
+      prefetch_tmap(&tmBh);
+      prefetch_tmap(&tmBl);
+      const uint32_t a_bytes = (uint32_t)nk * kSlice;
+      int su = 0, cs = 0;  // staging uses of the q~ buffer, key slices
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = gtr_item(r, items);
+        if (w < 0) break;
+        const int tm = T - 1 - w / batch, z = w % batch;
+        const int arow = z * p.M + tm * 128;
+        // the q~ parts, one at a time through the staging buffer (free once
+        // the previous part was copied into TMEM)
+        for (int part = 0; part < 2 && ok; ++part) {
+          if (su > 0 && !mbar_wait(&a_free, (su - 1) & 1, abort_p, p.status, tmo)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&a_full, a_bytes);
+          tma_load_3d(sA, part ? &tmAl : &tmAh, &a_full, 0, arow, 0);
+          a_issued = ++su;
+        }
+        const int bz = (z / p.zh) * p.zmul + (z % p.zh) / p.zg;
+        for (int tn = 0; tn <= tm && ok; ++tn) {
+          const int brow = bz * p.N + tn * 128;
+          for (int c = 0; c < nk; ++c) {
+            const int s = cs % kBStages;
+            if (cs >= kBStages && !mbar_wait(&b_empty[s], ((cs / kBStages) - 1) & 1, abort_p, p.status, tmo)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&b_full[s], kBStage);
+            tma_load_2d(sB + s * kBStage, &tmBh, &b_full[s], c * 32, brow);
+            tma_load_2d(sB + s * kBStage + kSlice, &tmBl, &b_full[s], c * 32, brow);
+            b_issued = ++cs;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- copies and MMAs ---
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_tf32(128, 128, 0, 0);  // A (TMEM) and B K-major
+      const uint64_t dA0 = make_sw128_desc(smem_u32(sA), 16, 1024);
+      const uint64_t dB0 = make_sw128_desc(smem_u32(sB), 16, 1024);
+      int it = 0, su = 0, cs = 0, tile = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = gtr_item(r, items);
+        if (w < 0) break;
+        const int tm = T - 1 - w / batch;
+        // the previous item's products must be done before its q~ is overwritten
+        if (it > 0 && !mbar_wait(&atm_free, (it - 1) & 1, abort_p, p.status, tmo)) break;
+        for (int part = 0; part < 2 && ok; ++part) {
+          if (!mbar_wait(&a_full, su & 1, abort_p, p.status, tmo)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ta = tmem + (part ? kColAl : kColAh);
+          for (int c = 0; c < nk; ++c)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tmem_cp_128x256b(ta + (uint32_t)(c * 32 + kk * 8),
+                               dA0 + (uint64_t)((c * kSlice + kk * 32) >> 4));
+          mma_commit(&a_free);  // the staging buffer is free once these copies are done
+          a_used = ++su;
+        }
+        if (!ok) break;
+        for (int tn = 0; tn <= tm && ok; ++tn, ++tile) {
+          const int buf = tile & 1;
+          if (tile >= 2 && !mbar_wait(&acc_empty[buf], ((tile >> 1) - 1) & 1, abort_p, p.status, tmo)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t acc = tmem + (uint32_t)buf * 128u;
+          for (int c = 0; c < nk; ++c) {
+            const int s = cs % kBStages;
+            if (!mbar_wait(&b_full[s], (cs / kBStages) & 1, abort_p, p.status, tmo)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dBh = dB0 + (uint64_t)((s * kBStage) >> 4);
+            const uint64_t dBl = dBh + (uint64_t)(kSlice >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = (uint64_t)((kk * 32) >> 4);  // 8 floats = 32 bytes per k step
+              const uint32_t col = (uint32_t)(c * 32 + kk * 8);
+              mma_tf32_ts(acc, tmem + kColAh + col, dBh + off, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+              mma_tf32_ts(acc, tmem + kColAh + col, dBl + off, idesc, 1u);
+              mma_tf32_ts(acc, tmem + kColAl + col, dBh + off, idesc, 1u);
+            }
+            mma_commit(&b_empty[s]);
+            b_used = ++cs;
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[buf]);
+        }
+        if (!ok) break;
+        mma_commit(&atm_free);
+        ++it;
+      }
+      // arrives once every copy and MMA this thread issued is done (even after a failed wait)
+      mma_commit(&done);
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int q = warp & 3;        // TMEM sub-partition: rows 32q .. 32q+31
+    const int rr = q * 32 + lane;  // tile row
+    const bool storer = warp == 2 && lane == 0;
+    int tile = 0, chunk = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int w = gtr_item(r, items);
+      if (w < 0) break;
+      const int tm = T - 1 - w / batch, z = w % batch;
+      for (int tn = 0; tn <= tm; ++tn, ++tile) {
+        const int buf = tile & 1;
+        ok = mbar_wait(&acc_full[buf], (tile >> 1) & 1, abort_p, p.status, tmo);
+        // every epilogue thread leaves together: the named barriers below have no timeout
+        if (bar_red_or(1, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32, ++chunk) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 128 + c0), v);
+          tmem_wait_ld();
+          if (c0 == 96) {
+            // the accumulator is read: the MMA warp may reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          }
+          uint8_t* const so = sO + (chunk & 1) * kOut;
+          // the staging tile's previous store has finished reading it
+          if (storer) bulk_wait_group_read<1>();
+          named_barrier_sync(2, 128);
+          // row rr, 16-byte piece k at (k ^ (rr & 7)) (128-byte swizzle)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(so + rr * 128 + ((k ^ (rr & 7)) << 4)) =
+                make_float4(p.alpha * __uint_as_float(v[4 * k]), p.alpha * __uint_as_float(v[4 * k + 1]),
+                            p.alpha * __uint_as_float(v[4 * k + 2]), p.alpha * __uint_as_float(v[4 * k + 3]));
+          fence_async_shared();
+          named_barrier_sync(2, 128);
+          if (storer) {
+            tma_store_3d(&tmC, so, tn * 128 + c0, tm * 128, z);
+            bulk_commit_group();
+          }
+        }
+      }
+    }
+    if (storer) bulk_wait_group<0>();  // every store complete before the CTA exits
+  }
+
+  // every copy and MMA done before TMEM is released (bounded; the MMA warp always commits)
+  __syncwarp();
+  {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(&done, 0, 20000u))
+      if (globaltimer_ns() - t0 > 20000000ull) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+  // After an abort, copies that were issued but never consumed may still be
+  // in flight: each completes its stage's full phase (armed by the loader
+  // alone), so wait (bounded) for those phases before shared memory is
+  // released.  A loader arms slice c only after slice c - kBStages was
+  // consumed, so only the last kBStages can be open; likewise the staging
+  // buffer holds at most one part.
+  if (threadIdx.x == 0 && *abort_p) {
+    for (int c = b_used > b_issued - kBStages ? b_used : b_issued - kBStages; c < b_issued; ++c) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait_sleep(&b_full[c % kBStages], (c / kBStages) & 1, 20000u))
+        if (globaltimer_ns() - t0 > 20000000ull) break;
+    }
+    if (a_used < a_issued) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait_sleep(&a_full, (a_issued - 1) & 1, 20000u))
+        if (globaltimer_ns() - t0 > 20000000ull) break;
+    }
+  }
+}
+
+bool gemm_tf32x3_rows_fits(int K, int N, long long c_bs, const void* C) {
+  return K % 32 == 0 && K / 32 <= gtr::kMaxSlices && N % 4 == 0 && c_bs % 4 == 0 &&
+         (reinterpret_cast<uintptr_t>(C) & 15) == 0;
+}
+
+cudaError_t launch_gemm_tf32x3_rows(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
+                                    const CUtensorMap& tmBl, const CUtensorMap& tmC, const Tf32x3Params& p,
+                                    int batch, int num_sms, cudaStream_t st) {
+  if (!gemm_tf32x3_rows_fits(p.K, p.N, p.c_bs, p.C)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gtr::kSmem);
+  if (e != cudaSuccess) return e;
+  const long long items = (long long)((p.M + 127) / 128) * batch;
+  const int grid = (int)(items < num_sms ? items : num_sms);
+  gemm_tf32x3_rows_kernel<<<grid < 1 ? 1 : grid, gtr::kThreads, gtr::kSmem, st>>>(tmAh, tmAl, tmBh, tmBl, tmC, p,
+                                                                                  batch);
   return cudaGetLastError();
 }
 
@@ -739,10 +1120,57 @@ __global__ void __launch_bounds__(NT) row_select_kernel(
 // the ascending lists are compacted with ballots, so no CTA barrier is taken.
 // Every loop over the row is a short rolled loop: fully unrolled register
 // copies of the row made the kernel wait on instruction fetch.  The softmax
+// is exp2-based (one FMA and one MUFU exponential per candidate) and
 // multiplies by the reciprocal of the row sum; the key order, ties to the
 // lower j, the forced diagonal and varlen windows follow row_select_kernel.
+//
+// Three passes over the row before the radix select: (A) load, maximum and
+// minimum; (B) exponentials and their sum; (C) probabilities, their
+// order-preserving keys and the first radix histogram.  The first digit's
+// position is predicted from the keys of the two extreme candidates (the
+// keys of a row share every bit above the highest bit where its largest and
+// smallest keys differ); the true AND / OR of all keys, formed in the same
+// pass, confirms the prediction, and otherwise the first histogram is built
+// again in a pass of its own.
 constexpr int kSelWarps = 8;
 constexpr int kSelMaxWidth = 4096;
+
+// Shared-memory counter increment with the condition as a predicate (no
+// branch around the atomic).
+__device__ __forceinline__ void red_shared_add1_if(uint32_t* addr, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(smem_u32(addr)),
+      "r"((uint32_t)pred)
+      : "memory");
+}
+
+// Global int32 store with the condition as a predicate.
+__device__ __forceinline__ void st_global_if(int32_t* addr, int32_t v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %2, 0;\n\t"
+      "@p st.global.b32 [%0], %1;\n\t}" ::"l"(addr),
+      "r"(v), "r"((uint32_t)pred)
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2_approx_full(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));  // keeps subnormal results
+  return y;
+}
+
+// Bits above the highest bit where the keys differ (kd = AND ^ OR of the
+// keys, or of the two extreme keys): the mask of fixed bits and the shift of
+// the first 8-bit digit below them.
+__device__ __forceinline__ void fixed_bits(uint32_t kd, int& hb, uint32_t& pmask, int& shift) {
+  hb = kd ? 31 - __clz(kd) : -1;
+  pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
+  shift = hb >= 7 ? hb - 7 : 0;
+}
+
 template <bool FROM_LOGITS>
 __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp_kernel(
     const float* in, float* scores, long long rows, int nb, int mode_flags, float T, int k, float density,
@@ -772,38 +1200,78 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp_kernel(
   const int len = i + 1;
   const int nt = (len + 31) >> 5;  // 32-candidate chunks
   const float* src = in + row * (long long)nb + off;
-  // The row into shared memory.  Lane sums run in the same candidate order
-  // as the per-row kernels' (j = lane, lane + 32, ...), then one butterfly.
-  float m = -INFINITY;
+  int32_t* out = indices + row * (long long)cap;
+  const bool threshold = mode == SEER_SELECT_THRESHOLD;
+  const int ki = threshold ? 0 : topk_count(i, mode, k, density);
+  if (!threshold && ki >= len && !dst) {
+    for (int j = lane; j < len; j += 32) out[j] = j + off;
+    if (lane == 0) counts[row] = len;
+    return;
+  }
+
+  // (A) the row into shared memory, its maximum and minimum
+  float m = -INFINITY, mn = INFINITY;
 #pragma unroll 4
   for (int j = lane; j < len; j += 32) {
     const float x = src[j];
     buf[j] = x;
     m = fmaxf(m, x);
+    mn = fminf(mn, x);
   }
+  m = warp_max(m);
+  mn = -warp_max(-mn);
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float mc = m * kLog2e;
+  float inv = 1.f;
   if (FROM_LOGITS) {
-    m = warp_max(m);
+    // (B) exponentials 2^(x log2(e) - m log2(e)) and their sum, summed in
+    // the same candidate order as the per-row kernel (j = lane, lane + 32,
+    // ...), then one butterfly
     float sum = 0.f;
 #pragma unroll 4
     for (int j = lane; j < len; j += 32) {
-      const float e = expf(buf[j] - m);
+      const float e = ex2_approx_full(fmaf(buf[j], kLog2e, -mc));
       buf[j] = e;
       sum += e;
     }
-    const float inv = 1.0f / warp_sum(sum);
-#pragma unroll 4
-    for (int j = lane; j < len; j += 32) {
-      const float v = buf[j] * inv;
-      buf[j] = v;
-      if (dst) dst[off + j] = v;
-    }
-    if (dst)
-      for (int j = lane; j < nb; j += 32)
-        if (j < off || j >= off + len) dst[j] = 0.f;
+    inv = 1.0f / warp_sum(sum);
   }
-  int32_t* out = indices + row * (long long)cap;
+  const bool radix = !threshold && ki < len;
+  // predicted fixed bits and first digit, from the extreme candidates' keys
+  // (formed exactly as every candidate's below)
+  const float vhi = FROM_LOGITS ? ex2_approx_full(fmaf(m, kLog2e, -mc)) * inv : m;
+  const float vlo = FROM_LOGITS ? ex2_approx_full(fmaf(mn, kLog2e, -mc)) * inv : mn;
+  int hb_p, shift_p;
+  uint32_t pmask_p;
+  fixed_bits(f2key(vhi) ^ f2key(vlo), hb_p, pmask_p, shift_p);
+  const bool first_hist = radix && hb_p >= 0;
+  if (first_hist) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
+    __syncwarp();
+  }
+  // (C) probabilities (written out when asked for), keys, their AND / OR and
+  // the first histogram on the predicted digit
+  uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll 4
+  for (int j = lane; j < len; j += 32) {
+    const float v = FROM_LOGITS ? buf[j] * inv : buf[j];
+    if (dst) dst[off + j] = v;
+    if (threshold) {
+      buf[j] = v;
+    } else {
+      const uint32_t kk = f2key(v);
+      key[j] = kk;
+      kand &= kk;
+      kor |= kk;
+      red_shared_add1_if(&hist[(kk >> shift_p) & 0xffu], first_hist);
+    }
+  }
+  if (dst)
+    for (int j = lane; j < nb; j += 32)
+      if (j < off || j >= off + len) dst[j] = 0.f;
 
-  if (mode == SEER_SELECT_THRESHOLD) {
+  if (threshold) {
     int base = 0;
     for (int t = 0; t < nt; ++t) {
       const int j = 32 * t + lane;
@@ -815,52 +1283,44 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp_kernel(
     if (lane == 0) counts[row] = base;
     return;
   }
-
-  const int ki = topk_count(i, mode, k, density);
-  if (ki >= len) {
+  if (!radix) {
     for (int j = lane; j < len; j += 32) out[j] = j + off;
     if (lane == 0) counts[row] = len;
     return;
   }
 
-  // Order-preserving keys replace the values.  Radix select of the ki-th
-  // largest key, 8 bits at a time.  Bits that all of the row's keys share
-  // are fixed at once (a warp AND / OR of the keys): a softmax row's values
-  // lie close together, so its keys agree on the sign, the exponent and the
-  // top of the mantissa, and the first digit starts at the highest bit where
-  // they differ.  The search also stops as soon as the bin holding the ki-th
-  // key is taken whole.
-  uint32_t kand = 0xffffffffu, kor = 0u;
-#pragma unroll 4
-  for (int j = lane; j < len; j += 32) {
-    const uint32_t kk = f2key(buf[j]);
-    key[j] = kk;
-    kand &= kk;
-    kor |= kk;
-  }
+  // Radix select of the ki-th largest key, 8 bits at a time.  Bits that all
+  // of the row's keys share are fixed at once (a warp AND / OR of the keys):
+  // a softmax row's values lie close together, so its keys agree on the
+  // sign, the exponent and the top of the mantissa, and the first digit
+  // starts at the highest bit where they differ.  The search also stops as
+  // soon as the bin holding the ki-th key is taken whole.
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kand &= __shfl_xor_sync(0xffffffffu, kand, o);
     kor |= __shfl_xor_sync(0xffffffffu, kor, o);
   }
-  const uint32_t kdiff = kand ^ kor;
-  const int hb = kdiff ? 31 - __clz(kdiff) : -1;  // highest bit where keys differ
-  // bits above hb are fixed (all of them when every key is equal)
-  uint32_t pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
+  int hb, shift;
+  uint32_t pmask;
+  fixed_bits(kand ^ kor, hb, pmask, shift);
   uint32_t prefix = kand & pmask, remaining = (uint32_t)ki;
+  // the histogram of pass C is the first pass's when the prediction held
+  bool have = first_hist && hb == hb_p && prefix == (f2key(vhi) & pmask_p);
+  __syncwarp();
 #pragma unroll 1
-  for (int shift = hb >= 7 ? hb - 7 : 0; hb >= 0;) {
+  for (; hb >= 0;) {
+    if (!have) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
-    __syncwarp();
+      for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
+      __syncwarp();
 #pragma unroll 4
-    for (int j = lane; j < len; j += 32) {
-      const uint32_t kt = key[j];
-      // plain shared atomics: measured faster here than first aggregating
-      // the lanes of equal bins with a warp match
-      if ((kt & pmask) == prefix) atomicAdd(&hist[(kt >> shift) & 0xffu], 1u);
+      for (int j = lane; j < len; j += 32) {
+        const uint32_t kt = key[j];
+        red_shared_add1_if(&hist[(kt >> shift) & 0xffu], (kt & pmask) == prefix);
+      }
+      __syncwarp();
     }
-    __syncwarp();
+    have = false;
     // lane l owns bins 255-8l .. 248-8l (descending)
     uint32_t cnt[8], part = 0;
 #pragma unroll
@@ -916,8 +1376,302 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp_kernel(
     eq_before += __popc(em);
     const bool keep = j < len && (kt > prefix || (eq && rank < remaining) || (force_diag && j == i));
     const unsigned km = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[base + __popc(km & lt)] = j + off;
+    st_global_if(out + base + __popc(km & lt), j + off, keep);
     base += __popc(km);
+  }
+  if (lane == 0) counts[row] = base;
+}
+
+// The same selection with 16-byte vectors: lane l owns candidates
+// 128 t + 4 l .. 128 t + 4 l + 3, so every pass over the row moves four
+// candidates per shared-memory access and per loop step.  For rows that
+// start 16-byte aligned (nb a multiple of 4, no varlen table).  The passes
+// are those of row_select_warp_kernel; the final compaction ranks a lane's
+// four candidates with a warp prefix sum, and skips the tie ranking when the
+// radix search ended on a bin taken whole (the usual case).
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, int lane, uint32_t& total) {
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - v;
+}
+
+template <bool FROM_LOGITS>
+__global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
+    const float* in, float* scores, long long rows, int nb, int mode_flags, float T, int k, float density,
+    int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap) {
+  extern __shared__ uint32_t sel_smem[];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSelWarps + wid;
+  if (row >= rows) return;  // whole warps only: no CTA barrier follows
+  uint32_t* const hist = sel_smem + wid * 256;
+  float4* const buf = reinterpret_cast<float4*>(sel_smem + kSelWarps * 256) + (size_t)wid * (nb / 4);
+  uint4* const key = reinterpret_cast<uint4*>(buf);
+
+  const int mode = mode_flags & 0xff;
+  const bool force_diag = (mode_flags & SEER_SELECT_FORCE_DIAGONAL) != 0;
+  const int i = (int)(row % nb);
+  const int len = i + 1;
+  const int nc = (len + 127) >> 7;  // 128-candidate chunks
+  const float4* src = reinterpret_cast<const float4*>(in + row * (long long)nb);
+  float* const dst = (FROM_LOGITS && scores != nullptr) ? scores + row * (long long)nb : nullptr;
+  int32_t* out = indices + row * (long long)cap;
+  const bool threshold = mode == SEER_SELECT_THRESHOLD;
+  const int ki = threshold ? 0 : topk_count(i, mode, k, density);
+  if (!threshold && ki >= len && !dst) {
+    for (int j = lane; j < len; j += 32) out[j] = j;
+    if (lane == 0) counts[row] = len;
+    return;
+  }
+  // lane's vector v = 32 t + lane holds candidates 4v .. 4v + 3; those at or
+  // past len are read (the row has nb >= 4v + 4 entries) but never counted
+  auto nvalid = [&](int v) { return min(4, len - 4 * v); };
+
+  // (A) the row into shared memory, its maximum and minimum
+  float m = -INFINITY, mn = INFINITY;
+#pragma unroll 2
+  for (int v = lane; 4 * v < len; v += 32) {
+    float4 x = src[v];
+    buf[v] = x;
+    const int nv = nvalid(v);
+    if (nv < 4) {  // the row's last vector: repeat its first candidate
+      if (nv < 2) x.y = x.x;
+      if (nv < 3) x.z = x.x;
+      x.w = x.x;
+    }
+    m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+    mn = fminf(mn, fminf(fminf(x.x, x.y), fminf(x.z, x.w)));
+  }
+  m = warp_max(m);
+  mn = -warp_max(-mn);
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float mc = m * kLog2e;
+  float inv = 1.f;
+  if (FROM_LOGITS) {
+    // (B) exponentials and their sum
+    float sum = 0.f;
+#pragma unroll 2
+    for (int v = lane; 4 * v < len; v += 32) {
+      const float4 x = buf[v];
+      const int nv = nvalid(v);
+      float4 e;
+      e.x = ex2_approx_full(fmaf(x.x, kLog2e, -mc));
+      e.y = nv > 1 ? ex2_approx_full(fmaf(x.y, kLog2e, -mc)) : 0.f;
+      e.z = nv > 2 ? ex2_approx_full(fmaf(x.z, kLog2e, -mc)) : 0.f;
+      e.w = nv > 3 ? ex2_approx_full(fmaf(x.w, kLog2e, -mc)) : 0.f;
+      buf[v] = e;
+      sum += (e.x + e.y) + (e.z + e.w);
+    }
+    inv = 1.0f / warp_sum(sum);
+  }
+  const bool radix = !threshold && ki < len;
+  const float vhi = FROM_LOGITS ? ex2_approx_full(fmaf(m, kLog2e, -mc)) * inv : m;
+  const float vlo = FROM_LOGITS ? ex2_approx_full(fmaf(mn, kLog2e, -mc)) * inv : mn;
+  int hb_p, shift_p;
+  uint32_t pmask_p;
+  fixed_bits(f2key(vhi) ^ f2key(vlo), hb_p, pmask_p, shift_p);
+  const bool first_hist = radix && hb_p >= 0;
+  if (first_hist) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
+    __syncwarp();
+  }
+  // (C) probabilities, keys, AND / OR, the first histogram on the predicted digit
+  uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll 2
+  for (int v = lane; 4 * v < len; v += 32) {
+    const float4 e = buf[v];
+    const int nv = nvalid(v);
+    float4 pv;
+    pv.x = FROM_LOGITS ? e.x * inv : e.x;
+    pv.y = FROM_LOGITS ? e.y * inv : e.y;
+    pv.z = FROM_LOGITS ? e.z * inv : e.z;
+    pv.w = FROM_LOGITS ? e.w * inv : e.w;
+    if (dst) {
+      if (nv == 4) {
+        *reinterpret_cast<float4*>(dst + 4 * v) = pv;
+      } else {
+        dst[4 * v] = pv.x;
+        if (nv > 1) dst[4 * v + 1] = pv.y;
+        if (nv > 2) dst[4 * v + 2] = pv.z;
+      }
+    }
+    if (threshold) {
+      buf[v] = pv;
+    } else {
+      uint4 kk = make_uint4(f2key(pv.x), f2key(pv.y), f2key(pv.z), f2key(pv.w));
+      key[v] = kk;
+      kand &= kk.x;
+      kor |= kk.x;
+      if (nv > 1) { kand &= kk.y; kor |= kk.y; }
+      if (nv > 2) { kand &= kk.z; kor |= kk.z; }
+      if (nv > 3) { kand &= kk.w; kor |= kk.w; }
+      red_shared_add1_if(&hist[(kk.x >> shift_p) & 0xffu], first_hist);
+      red_shared_add1_if(&hist[(kk.y >> shift_p) & 0xffu], first_hist && nv > 1);
+      red_shared_add1_if(&hist[(kk.z >> shift_p) & 0xffu], first_hist && nv > 2);
+      red_shared_add1_if(&hist[(kk.w >> shift_p) & 0xffu], first_hist && nv > 3);
+    }
+  }
+  if (dst)
+    for (int j = len + lane; j < nb; j += 32) dst[j] = 0.f;
+
+  if (threshold) {
+    int base = 0;
+    for (int t = 0; t < nc; ++t) {
+      const int v = 32 * t + lane;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int nv = 4 * v < len ? nvalid(v) : 0;
+      if (nv > 0) x = buf[v];
+      const int j0 = 4 * v;
+      const bool k0 = nv > 0 && (x.x > T || (force_diag && j0 == i));
+      const bool k1 = nv > 1 && (x.y > T || (force_diag && j0 + 1 == i));
+      const bool k2 = nv > 2 && (x.z > T || (force_diag && j0 + 2 == i));
+      const bool k3 = nv > 3 && (x.w > T || (force_diag && j0 + 3 == i));
+      uint32_t tot;
+      const uint32_t pos = base + warp_excl_scan((uint32_t)k0 + k1 + k2 + k3, lane, tot);
+      uint32_t q = pos;
+      st_global_if(out + q, j0, k0);
+      q += k0;
+      st_global_if(out + q, j0 + 1, k1);
+      q += k1;
+      st_global_if(out + q, j0 + 2, k2);
+      q += k2;
+      st_global_if(out + q, j0 + 3, k3);
+      base += (int)tot;
+    }
+    if (lane == 0) counts[row] = base;
+    return;
+  }
+  if (!radix) {
+    for (int j = lane; j < len; j += 32) out[j] = j;
+    if (lane == 0) counts[row] = len;
+    return;
+  }
+
+  // radix select of the ki-th largest key (as in row_select_warp_kernel)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+  }
+  int hb, shift;
+  uint32_t pmask;
+  fixed_bits(kand ^ kor, hb, pmask, shift);
+  uint32_t prefix = kand & pmask, remaining = (uint32_t)ki;
+  bool whole = hb < 0;  // the keys equal to the final prefix are all kept
+  if (hb < 0) whole = remaining >= (uint32_t)len;
+  bool have = first_hist && hb == hb_p && prefix == (f2key(vhi) & pmask_p);
+  __syncwarp();
+#pragma unroll 1
+  for (; hb >= 0;) {
+    if (!have) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
+      __syncwarp();
+#pragma unroll 2
+      for (int v = lane; 4 * v < len; v += 32) {
+        const uint4 kk = key[v];
+        const int nv = nvalid(v);
+        red_shared_add1_if(&hist[(kk.x >> shift) & 0xffu], (kk.x & pmask) == prefix);
+        red_shared_add1_if(&hist[(kk.y >> shift) & 0xffu], nv > 1 && (kk.y & pmask) == prefix);
+        red_shared_add1_if(&hist[(kk.z >> shift) & 0xffu], nv > 2 && (kk.z & pmask) == prefix);
+        red_shared_add1_if(&hist[(kk.w >> shift) & 0xffu], nv > 3 && (kk.w & pmask) == prefix);
+      }
+      __syncwarp();
+    }
+    have = false;
+    uint32_t cnt[8], part = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cnt[q] = hist[255 - 8 * lane - q];
+      part += cnt[q];
+    }
+    uint32_t incl = part;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - part;
+    uint32_t sel_bin = 0, sel_rem = 0, sel_cnt = 0;
+    const bool mine = excl < remaining && remaining <= incl;
+    if (mine) {
+      uint32_t before = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (before < remaining && remaining <= before + cnt[q]) {
+          sel_bin = (uint32_t)(255 - 8 * lane - q);
+          sel_rem = remaining - before;
+          sel_cnt = cnt[q];
+        }
+        before += cnt[q];
+      }
+    }
+    const int owner = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    sel_bin = __shfl_sync(0xffffffffu, sel_bin, owner);
+    sel_rem = __shfl_sync(0xffffffffu, sel_rem, owner);
+    sel_cnt = __shfl_sync(0xffffffffu, sel_cnt, owner);
+    prefix |= sel_bin << shift;
+    remaining = sel_rem;
+    pmask |= 0xffu << shift;
+    __syncwarp();
+    if (sel_cnt == sel_rem) {
+      whole = true;
+      break;
+    }
+    if (shift == 0) break;
+    shift = shift >= 8 ? shift - 8 : 0;
+  }
+  // keys above the prefix are kept; of those equal to it, the `remaining`
+  // with the lowest j (all of them when the bin was taken whole); the
+  // diagonal joins when forced
+  int base = 0;
+  uint32_t eq_before = 0;
+  for (int t = 0; t < nc; ++t) {
+    const int v = 32 * t + lane;
+    const int nv = 4 * v < len ? nvalid(v) : 0;
+    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
+    if (nv > 0) kk = key[v];
+    const uint32_t a0 = kk.x & pmask, a1 = kk.y & pmask, a2 = kk.z & pmask, a3 = kk.w & pmask;
+    const int j0 = 4 * v;
+    bool k0, k1, k2, k3;
+    if (whole) {
+      k0 = nv > 0 && a0 >= prefix;
+      k1 = nv > 1 && a1 >= prefix;
+      k2 = nv > 2 && a2 >= prefix;
+      k3 = nv > 3 && a3 >= prefix;
+    } else {
+      const bool e0 = nv > 0 && a0 == prefix, e1 = nv > 1 && a1 == prefix;
+      const bool e2 = nv > 2 && a2 == prefix, e3 = nv > 3 && a3 == prefix;
+      uint32_t etot;
+      const uint32_t r0 = eq_before + warp_excl_scan((uint32_t)e0 + e1 + e2 + e3, lane, etot);
+      const uint32_t r1 = r0 + e0, r2 = r1 + e1, r3 = r2 + e2;
+      eq_before += etot;
+      k0 = nv > 0 && (a0 > prefix || (e0 && r0 < remaining));
+      k1 = nv > 1 && (a1 > prefix || (e1 && r1 < remaining));
+      k2 = nv > 2 && (a2 > prefix || (e2 && r2 < remaining));
+      k3 = nv > 3 && (a3 > prefix || (e3 && r3 < remaining));
+    }
+    if (force_diag) {
+      k0 = k0 || (nv > 0 && j0 == i);
+      k1 = k1 || (nv > 1 && j0 + 1 == i);
+      k2 = k2 || (nv > 2 && j0 + 2 == i);
+      k3 = k3 || (nv > 3 && j0 + 3 == i);
+    }
+    uint32_t tot;
+    uint32_t q = base + warp_excl_scan((uint32_t)k0 + k1 + k2 + k3, lane, tot);
+    st_global_if(out + q, j0, k0);
+    q += k0;
+    st_global_if(out + q, j0 + 1, k1);
+    q += k1;
+    st_global_if(out + q, j0 + 2, k2);
+    q += k2;
+    st_global_if(out + q, j0 + 3, k3);
+    base += (int)tot;
   }
   if (lane == 0) counts[row] = base;
 }
@@ -963,20 +1717,20 @@ __global__ void varlen_table_kernel(const int32_t* __restrict__ start, const int
 
 // --------------------------------------------------------------- launchers --
 cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, int n, int d,
-                        float* out, cudaStream_t st, const int2* tab) {
+                        float* out, cudaStream_t st, const int2* tab, float* lo) {
   const long long nblocks = BH * (n / kBlock);
   const int warps = 8;
   const unsigned grid = (unsigned)((nblocks + warps - 1) / warps);
   if (dt == SEER_BF16) {
     if (is_k)
-      pool_kernel<uint16_t, true><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab);
+      pool_kernel<uint16_t, true><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab, lo);
     else
-      pool_kernel<uint16_t, false><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab);
+      pool_kernel<uint16_t, false><<<grid, warps * 32, 0, st>>>((const uint16_t*)X, nblocks, n, d, out, tab, lo);
   } else {
     if (is_k)
-      pool_kernel<float, true><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab);
+      pool_kernel<float, true><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab, lo);
     else
-      pool_kernel<float, false><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab);
+      pool_kernel<float, false><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab, lo);
   }
   return cudaGetLastError();
 }
@@ -1041,6 +1795,16 @@ cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, 
   if (!wide && rows >= 8LL * 148 && width <= kSelMaxWidth) {
     const unsigned grid = (unsigned)((rows + kSelWarps - 1) / kSelWarps);
     const size_t smem = sizeof(uint32_t) * (size_t)kSelWarps * (256 + width);
+    if (!tab && row_len <= 0 && nb % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0 &&
+        (!scores || (reinterpret_cast<uintptr_t>(scores) & 15) == 0)) {
+      // rows start 16-byte aligned: four candidates per lane and access
+      auto kern4 = from_logits ? row_select_warp4_kernel<true> : row_select_warp4_kernel<false>;
+      cudaError_t e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      kern4<<<grid, 32 * kSelWarps, smem, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density,
+                                                counts, indices, cap);
+      return cudaGetLastError();
+    }
     auto kern = from_logits ? row_select_warp_kernel<true> : row_select_warp_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

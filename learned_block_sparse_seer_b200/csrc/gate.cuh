@@ -11,8 +11,10 @@ namespace seer {
 // Q average-pool (is_k = false) or K [max|min|avg]-pool (is_k = true) of X
 // [BH, n, d] into out [BH, n/64, d] or [BH, n/64, 3d] (fp32).  tab: optional
 // varlen block table (valid tokens per block).
+// lo non-null: out receives each pooled value rounded to tf32 and lo the exact
+// remainder (the tf32x3 operand split), instead of the fp32 value.
 cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, int n, int d,
-                        float* out, cudaStream_t st, const int2* tab = nullptr);
+                        float* out, cudaStream_t st, const int2* tab = nullptr, float* lo = nullptr);
 
 // Batched C = alpha * A B^T (fp32); see gemm_nt_kernel for the batch mapping.
 cudaError_t launch_gemm_nt(const float* A, const float* B, float* C, int M, int N, int K,
@@ -32,13 +34,30 @@ struct Tf32x3Params {
   long long c_bs;
   float alpha;
   float* C;
+  float* C_lo;  // non-null: C receives the result rounded to tf32 and C_lo the exact remainder
+  int tma_out;  // launch_gemm_tf32x3_causal: write C (and C_lo) by TMA stores through tmC (tmClo)
   uint32_t* status;
   unsigned long long timeout_ns;
 };
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st);
 cudaError_t launch_split_tf32_copy(const float* x, float* hi, float* lo, long long n, cudaStream_t st);
+// tmC / tmClo (used when p.tma_out): 3-D maps over C / C_lo (N columns, M rows,
+// batch; box 32 x 128 x 1, 128-byte swizzle).
 cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
-                                      const CUtensorMap& tmBl, const Tf32x3Params& p, int batch, cudaStream_t st);
+                                      const CUtensorMap& tmBl, const CUtensorMap& tmC, const CUtensorMap& tmClo,
+                                      const Tf32x3Params& p, int batch, cudaStream_t st);
+
+// The causal logits with each 128-row block of A held in tensor memory while
+// the B tiles up to the diagonal stream past it (p.causal ignored: always
+// causal); persistent, at most num_sms CTAs.  tmAh / tmAl are 3-D panel maps
+// over the A parts (box 32 x 128 x K/32), tmBh / tmBl 2-D maps over the B
+// parts (box 32 x 128), tmC a 3-D map over C (N columns, M rows, batch; box
+// 32 x 128 x 1).  Needs K a multiple of 32 and at most 128, N and c_bs
+// multiples of 4 and C 16-byte aligned (gemm_tf32x3_rows_fits).
+bool gemm_tf32x3_rows_fits(int K, int N, long long c_bs, const void* C);
+cudaError_t launch_gemm_tf32x3_rows(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
+                                    const CUtensorMap& tmBl, const CUtensorMap& tmC, const Tf32x3Params& p,
+                                    int batch, int num_sms, cudaStream_t st);
 
 // Block-level RoPE with base theta / 64 on x [rows, h] (row position = row % nb).
 cudaError_t launch_rope(float* x, long long rows, int nb, int h, float theta, cudaStream_t st);
