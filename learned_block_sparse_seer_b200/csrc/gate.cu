@@ -10,21 +10,29 @@
 // Kernels (the gate is ~1/4096 of the attention map; pooling is HBM-bound,
 // the rest small):
 //   pool_kernel      Q avg-pool / K [max|min|avg]-pool, one warp per block,
-//                    16-byte vector loads, shuffle reductions
-//   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections, and the causal
-//                    block logits q~ k~^T / sqrt(d) (upper tiles skipped) when
-//                    h is not a multiple of 32; gemm_nt128_kernel is its
-//                    128 x 128-tile form for K % 16 == 0
-//   split_tf32_kernel + gemm_tf32x3_kernel
-//                    the causal block logits on the tf32 tensor cores (tcgen05)
-//                    when h % 32 == 0: three products of tf32 parts (hi*hi +
-//                    hi*lo + lo*hi) keep fp32-level accuracy
+//                    16-byte vector loads, shuffle reductions; optionally
+//                    writes its result split into tf32 part and remainder
+//   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections and the causal
+//                    block logits when h or d is not a multiple of 32;
+//                    gemm_nt128_kernel is its 128 x 128-tile form
+//   gemm_tf32x3_kernel
+//                    the gate projections on the tf32 tensor cores (tcgen05):
+//                    three products of tf32 parts (hi*hi + hi*lo + lo*hi)
+//                    keep fp32-level accuracy; the epilogue writes q~ / k~
+//                    already split for the logits, by TMA stores
+//   gemm_tf32x3_rows_kernel
+//                    the causal block logits q~ k~^T / sqrt(d) the same way,
+//                    persistent: each q~ row block is copied into TMEM once
+//                    and the key tiles up to the diagonal stream past it
+//   split_tf32_kernel / split_tf32_copy_kernel
+//                    the tf32 split of the weights (and of q~ / k~ after RoPE)
 //   rope_kernel      optional block-level RoPE on q~ / k~
-//   row_select_warp_kernel / row_select_kernel
-//                    one warp (many rows of <= 2048 candidates) or one CTA per
-//                    score row: causal softmax (Eq. 1), optional score
-//                    write-out, then threshold compaction or exact top-k
-//                    (radix select on the fp32 bit patterns, ties to lower j)
+//   row_select_warp4_kernel / row_select_warp_kernel / row_select_kernel
+//                    one warp (many rows of <= 4096 candidates; 16-byte
+//                    vectors when rows are aligned) or one CTA per score row:
+//                    causal softmax (Eq. 1), optional score write-out, then
+//                    threshold compaction or exact top-k (radix select on
+//                    the fp32 bit patterns, ties to lower j)
 #include <cstdint>
 
 #include "common.cuh"
@@ -71,6 +79,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
     mx[e] = -INFINITY;
     mn[e] = INFINITY;
   }
+#pragma unroll 8
   for (int r = lane / lpr; r < valid; r += rpi) {
     uint4 v = *reinterpret_cast<const uint4*>(base + (long long)r * d);
     float f[EPL];
@@ -749,17 +758,17 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32, ++chunk) {
-          uint32_t v[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 128 + c0), v);
-          tmem_wait_ld();
-          if (c0 == 96) {
-            // the accumulator is read: the MMA warp may reuse it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          }
+        // the whole 128-column row in registers with one wait, then the
+        // accumulator is free for the MMA warp
+        uint32_t v[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 128 + 32 * c), v[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c, ++chunk) {
           uint8_t* const so = sO + (chunk & 1) * kOut;
           // the staging tile's previous store has finished reading it
           if (storer) bulk_wait_group_read<1>();
@@ -768,12 +777,12 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             *reinterpret_cast<float4*>(so + rr * 128 + ((k ^ (rr & 7)) << 4)) =
-                make_float4(p.alpha * __uint_as_float(v[4 * k]), p.alpha * __uint_as_float(v[4 * k + 1]),
-                            p.alpha * __uint_as_float(v[4 * k + 2]), p.alpha * __uint_as_float(v[4 * k + 3]));
+                make_float4(p.alpha * __uint_as_float(v[c][4 * k]), p.alpha * __uint_as_float(v[c][4 * k + 1]),
+                            p.alpha * __uint_as_float(v[c][4 * k + 2]), p.alpha * __uint_as_float(v[c][4 * k + 3]));
           fence_async_shared();
           named_barrier_sync(2, 128);
           if (storer) {
-            tma_store_3d(&tmC, so, tn * 128 + c0, tm * 128, z);
+            tma_store_3d(&tmC, so, tn * 128 + 32 * c, tm * 128, z);
             bulk_commit_group();
           }
         }
@@ -1406,8 +1415,13 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
     int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap) {
   extern __shared__ uint32_t sel_smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kSelWarps + wid;
-  if (row >= rows) return;  // whole warps only: no CTA barrier follows
+  // Rows are taken query block by query block across all heads (the
+  // warps of a CTA get rows of equal length; the first rows taken are the
+  // shortest, whose logits the logits kernel wrote last and L2 still holds).
+  const long long vrow = (long long)blockIdx.x * kSelWarps + wid;
+  if (vrow >= rows) return;  // whole warps only: no CTA barrier follows
+  const long long heads = rows / nb;
+  const long long row = (vrow % heads) * nb + vrow / heads;
   uint32_t* const hist = sel_smem + wid * 256;
   float4* const buf = reinterpret_cast<float4*>(sel_smem + kSelWarps * 256) + (size_t)wid * (nb / 4);
   uint4* const key = reinterpret_cast<uint4*>(buf);
@@ -1427,24 +1441,38 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
     if (lane == 0) counts[row] = len;
     return;
   }
-  // lane's vector v = 32 t + lane holds candidates 4v .. 4v + 3; those at or
-  // past len are read (the row has nb >= 4v + 4 entries) but never counted
-  auto nvalid = [&](int v) { return min(4, len - 4 * v); };
+  // Lane l owns the vectors v = 32 t + l, i.e. candidates 4v .. 4v + 3.  The
+  // nfull vectors below len are whole; at most one more (vector nfull, of
+  // lane nfull % 32) holds the row's last rem < 4 candidates.  Every pass
+  // runs its whole vectors unmasked and the partial one separately.
+  const int nfull = len >> 2, rem = len & 3;
+  const bool tail = rem != 0 && lane == (nfull & 31);
+  // order-preserving key; probabilities are never negative
+  auto key_of = [](float x) { return FROM_LOGITS ? (__float_as_uint(x) | 0x80000000u) : f2key(x); };
 
-  // (A) the row into shared memory, its maximum and minimum
+  // (A) the row into shared memory, its maximum and minimum; four vectors
+  // per lane in flight at a time
   float m = -INFINITY, mn = INFINITY;
-#pragma unroll 2
-  for (int v = lane; 4 * v < len; v += 32) {
-    float4 x = src[v];
-    buf[v] = x;
-    const int nv = nvalid(v);
-    if (nv < 4) {  // the row's last vector: repeat its first candidate
-      if (nv < 2) x.y = x.x;
-      if (nv < 3) x.z = x.x;
-      x.w = x.x;
-    }
-    m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
-    mn = fminf(mn, fminf(fminf(x.x, x.y), fminf(x.z, x.w)));
+  for (int v0 = lane; v0 < nfull; v0 += 128) {
+    float4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (v0 + 32 * u < nfull) x[u] = src[v0 + 32 * u];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (v0 + 32 * u < nfull) {
+        buf[v0 + 32 * u] = x[u];
+        m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+        mn = fminf(mn, fminf(fminf(x[u].x, x[u].y), fminf(x[u].z, x[u].w)));
+      }
+  }
+  if (tail) {  // the row has nb >= 4 nfull + 4 entries: the whole vector is readable
+    const float4 x = src[nfull];
+    buf[nfull] = x;
+    m = fmaxf(m, x.x);
+    mn = fminf(mn, x.x);
+    if (rem > 1) m = fmaxf(m, x.y), mn = fminf(mn, x.y);
+    if (rem > 2) m = fmaxf(m, x.z), mn = fminf(mn, x.z);
   }
   m = warp_max(m);
   mn = -warp_max(-mn);
@@ -1452,12 +1480,10 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   const float mc = m * kLog2e;
   float inv = 1.f;
   if (FROM_LOGITS) {
-    // (B) exponentials and their sum
+    // (B) exponentials and their sum (candidates past len get 0)
     float sum = 0.f;
-#pragma unroll 2
-    for (int v = lane; 4 * v < len; v += 32) {
+    auto expv = [&](int v, int nv) {
       const float4 x = buf[v];
-      const int nv = nvalid(v);
       float4 e;
       e.x = ex2_approx_full(fmaf(x.x, kLog2e, -mc));
       e.y = nv > 1 ? ex2_approx_full(fmaf(x.y, kLog2e, -mc)) : 0.f;
@@ -1465,7 +1491,10 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
       e.w = nv > 3 ? ex2_approx_full(fmaf(x.w, kLog2e, -mc)) : 0.f;
       buf[v] = e;
       sum += (e.x + e.y) + (e.z + e.w);
-    }
+    };
+#pragma unroll 2
+    for (int v = lane; v < nfull; v += 32) expv(v, 4);
+    if (tail) expv(nfull, rem);
     inv = 1.0f / warp_sum(sum);
   }
   const bool radix = !threshold && ki < len;
@@ -1473,7 +1502,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   const float vlo = FROM_LOGITS ? ex2_approx_full(fmaf(mn, kLog2e, -mc)) * inv : mn;
   int hb_p, shift_p;
   uint32_t pmask_p;
-  fixed_bits(f2key(vhi) ^ f2key(vlo), hb_p, pmask_p, shift_p);
+  fixed_bits(key_of(vhi) ^ key_of(vlo), hb_p, pmask_p, shift_p);
   const bool first_hist = radix && hb_p >= 0;
   if (first_hist) {
 #pragma unroll
@@ -1482,10 +1511,8 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   }
   // (C) probabilities, keys, AND / OR, the first histogram on the predicted digit
   uint32_t kand = 0xffffffffu, kor = 0u;
-#pragma unroll 2
-  for (int v = lane; 4 * v < len; v += 32) {
+  auto probv = [&](int v, int nv) {
     const float4 e = buf[v];
-    const int nv = nvalid(v);
     float4 pv;
     pv.x = FROM_LOGITS ? e.x * inv : e.x;
     pv.y = FROM_LOGITS ? e.y * inv : e.y;
@@ -1502,29 +1529,36 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
     }
     if (threshold) {
       buf[v] = pv;
-    } else {
-      uint4 kk = make_uint4(f2key(pv.x), f2key(pv.y), f2key(pv.z), f2key(pv.w));
-      key[v] = kk;
-      kand &= kk.x;
-      kor |= kk.x;
-      if (nv > 1) { kand &= kk.y; kor |= kk.y; }
-      if (nv > 2) { kand &= kk.z; kor |= kk.z; }
-      if (nv > 3) { kand &= kk.w; kor |= kk.w; }
-      red_shared_add1_if(&hist[(kk.x >> shift_p) & 0xffu], first_hist);
-      red_shared_add1_if(&hist[(kk.y >> shift_p) & 0xffu], first_hist && nv > 1);
-      red_shared_add1_if(&hist[(kk.z >> shift_p) & 0xffu], first_hist && nv > 2);
-      red_shared_add1_if(&hist[(kk.w >> shift_p) & 0xffu], first_hist && nv > 3);
+      return;
     }
-  }
+    const uint4 kk = make_uint4(key_of(pv.x), key_of(pv.y), key_of(pv.z), key_of(pv.w));
+    key[v] = kk;
+    kand &= kk.x;
+    kor |= kk.x;
+    if (nv > 1) kand &= kk.y, kor |= kk.y;
+    if (nv > 2) kand &= kk.z, kor |= kk.z;
+    if (nv > 3) kand &= kk.w, kor |= kk.w;
+    if (first_hist) {
+      atomicAdd(&hist[(kk.x >> shift_p) & 0xffu], 1u);
+      if (nv > 1) atomicAdd(&hist[(kk.y >> shift_p) & 0xffu], 1u);
+      if (nv > 2) atomicAdd(&hist[(kk.z >> shift_p) & 0xffu], 1u);
+      if (nv > 3) atomicAdd(&hist[(kk.w >> shift_p) & 0xffu], 1u);
+    }
+  };
+#pragma unroll 2
+  for (int v = lane; v < nfull; v += 32) probv(v, 4);
+  if (tail) probv(nfull, rem);
   if (dst)
     for (int j = len + lane; j < nb; j += 32) dst[j] = 0.f;
+  // candidates of this lane's vector in chunk t (0 past the row)
+  auto nvalid = [&](int v) { return v < nfull ? 4 : (v == nfull ? rem : 0); };
 
   if (threshold) {
     int base = 0;
     for (int t = 0; t < nc; ++t) {
       const int v = 32 * t + lane;
       float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      const int nv = 4 * v < len ? nvalid(v) : 0;
+      const int nv = nvalid(v);
       if (nv > 0) x = buf[v];
       const int j0 = 4 * v;
       const bool k0 = nv > 0 && (x.x > T || (force_diag && j0 == i));
@@ -1564,7 +1598,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   uint32_t prefix = kand & pmask, remaining = (uint32_t)ki;
   bool whole = hb < 0;  // the keys equal to the final prefix are all kept
   if (hb < 0) whole = remaining >= (uint32_t)len;
-  bool have = first_hist && hb == hb_p && prefix == (f2key(vhi) & pmask_p);
+  bool have = first_hist && hb == hb_p && prefix == (key_of(vhi) & pmask_p);
   __syncwarp();
 #pragma unroll 1
   for (; hb >= 0;) {
@@ -1572,15 +1606,16 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
 #pragma unroll
       for (int q = 0; q < 8; ++q) hist[8 * lane + q] = 0;
       __syncwarp();
-#pragma unroll 2
-      for (int v = lane; 4 * v < len; v += 32) {
+      auto countv = [&](int v, int nv) {
         const uint4 kk = key[v];
-        const int nv = nvalid(v);
         red_shared_add1_if(&hist[(kk.x >> shift) & 0xffu], (kk.x & pmask) == prefix);
         red_shared_add1_if(&hist[(kk.y >> shift) & 0xffu], nv > 1 && (kk.y & pmask) == prefix);
         red_shared_add1_if(&hist[(kk.z >> shift) & 0xffu], nv > 2 && (kk.z & pmask) == prefix);
         red_shared_add1_if(&hist[(kk.w >> shift) & 0xffu], nv > 3 && (kk.w & pmask) == prefix);
-      }
+      };
+#pragma unroll 2
+      for (int v = lane; v < nfull; v += 32) countv(v, 4);
+      if (tail) countv(nfull, rem);
       __syncwarp();
     }
     have = false;
@@ -1633,7 +1668,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   uint32_t eq_before = 0;
   for (int t = 0; t < nc; ++t) {
     const int v = 32 * t + lane;
-    const int nv = 4 * v < len ? nvalid(v) : 0;
+    const int nv = nvalid(v);
     uint4 kk = make_uint4(0u, 0u, 0u, 0u);
     if (nv > 0) kk = key[v];
     const uint32_t a0 = kk.x & pmask, a1 = kk.y & pmask, a2 = kk.z & pmask, a3 = kk.w & pmask;
