@@ -570,7 +570,7 @@ constexpr uint32_t kAStage = kMaxSlices * kSlice;   // one part of the q~ block:
 constexpr uint32_t kBStage = 2u * kSlice;           // one 32-column slice of a k~ tile, both parts: 32 KB
 constexpr uint32_t kOut = kSlice;                   // one 128 x 32 output chunk: 16 KB
 constexpr uint32_t kSmem = kAStage + kBStages * kBStage + 2u * kOut + 1024u;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;                        // warps: 0 key loads, 1 MMA, 2..5 epilogue, 6 q~ loads
 constexpr uint32_t kColAh = 256, kColAl = 384;      // TMEM: accumulators at 0 and 128
 }  // namespace gtr
 
@@ -627,22 +627,20 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ loads --
+  if (warp == 6) {
+    // ------------------------------------------------------- q~ loads ----
     if (lane == 0) {
       prefetch_tmap(&tmAh);
       prefetch_tmap(&tmAl);
-      prefetch_tmap(&tmBh);
-      prefetch_tmap(&tmBl);
       const uint32_t a_bytes = (uint32_t)nk * kSlice;
-      int su = 0, cs = 0;  // staging uses of the q~ buffer, key slices
+      int su = 0;  // staging uses of the q~ buffer
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int w = gtr_item(r, items);
         if (w < 0) break;
         const int tm = T - 1 - w / batch, z = w % batch;
         const int arow = z * p.M + tm * 128;
-        // the q~ parts, one at a time through the staging buffer (free once
+        // the two parts, one at a time through the staging buffer (free once
         // the previous part was copied into TMEM)
         for (int part = 0; part < 2 && ok; ++part) {
           if (su > 0 && !mbar_wait(&a_free, (su - 1) & 1, abort_p, p.status, tmo)) {
@@ -653,6 +651,19 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
           tma_load_3d(sA, part ? &tmAl : &tmAh, &a_full, 0, arow, 0);
           a_issued = ++su;
         }
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------- key loads ---
+    if (lane == 0) {
+      prefetch_tmap(&tmBh);
+      prefetch_tmap(&tmBl);
+      int cs = 0;  // key slices
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = gtr_item(r, items);
+        if (w < 0) break;
+        const int tm = T - 1 - w / batch, z = w % batch;
         const int bz = (z / p.zh) * p.zmul + (z % p.zh) / p.zg;
         for (int tn = 0; tn <= tm && ok; ++tn) {
           const int brow = bz * p.N + tn * 128;
@@ -738,7 +749,7 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
       // arrives once every copy and MMA this thread issued is done (even after a failed wait)
       mma_commit(&done);
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // --------------------------------------------------------- epilogue --
     const int q = warp & 3;        // TMEM sub-partition: rows 32q .. 32q+31
     const int rr = q * 32 + lane;  // tile row
@@ -1412,18 +1423,20 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, int lane, uint32_
 template <bool FROM_LOGITS>
 __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
     const float* in, float* scores, long long rows, int nb, int mode_flags, float T, int k, float density,
-    int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap) {
+    int32_t* __restrict__ counts, int32_t* __restrict__ indices, int cap, long long v0, long long v1, int width) {
   extern __shared__ uint32_t sel_smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Rows are taken query block by query block across all heads (the
   // warps of a CTA get rows of equal length; the first rows taken are the
   // shortest, whose logits the logits kernel wrote last and L2 still holds).
-  const long long vrow = (long long)blockIdx.x * kSelWarps + wid;
-  if (vrow >= rows) return;  // whole warps only: no CTA barrier follows
+  // This launch takes rows v0 .. v1 - 1 of that order, none longer than
+  // width (a multiple of 4: each warp's row buffer).
+  const long long vrow = v0 + (long long)blockIdx.x * kSelWarps + wid;
+  if (vrow >= v1) return;  // whole warps only: no CTA barrier follows
   const long long heads = rows / nb;
   const long long row = (vrow % heads) * nb + vrow / heads;
   uint32_t* const hist = sel_smem + wid * 256;
-  float4* const buf = reinterpret_cast<float4*>(sel_smem + kSelWarps * 256) + (size_t)wid * (nb / 4);
+  float4* const buf = reinterpret_cast<float4*>(sel_smem + kSelWarps * 256) + (size_t)wid * (width / 4);
   uint4* const key = reinterpret_cast<uint4*>(buf);
 
   const int mode = mode_flags & 0xff;
@@ -1450,9 +1463,34 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   // order-preserving key; probabilities are never negative
   auto key_of = [](float x) { return FROM_LOGITS ? (__float_as_uint(x) | 0x80000000u) : f2key(x); };
 
-  // (A) the row into shared memory, its maximum and minimum; four vectors
-  // per lane in flight at a time
-  float m = -INFINITY, mn = INFINITY;
+  // (A) the row into shared memory, its maximum and minimum; from logits
+  // also each lane's running softmax sum (relative to its running maximum,
+  // rescaled when that grows).  Four vectors per lane in flight at a time.
+  constexpr float kLog2e = 1.4426950408889634f;
+  float m = -INFINITY, mn = INFINITY, sl = 0.f;
+  auto fold = [&](float4 x, int nv) {
+    if (nv < 4) {  // the row's partial vector: repeat its first candidate for the extremes
+      if (nv < 2) x.y = x.x;
+      if (nv < 3) x.z = x.x;
+      x.w = x.x;
+    }
+    const float vm = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
+    mn = fminf(mn, fminf(fminf(x.x, x.y), fminf(x.z, x.w)));
+    if (FROM_LOGITS) {
+      if (vm > m) {
+        sl *= ex2_approx((m - vm) * kLog2e);
+        m = vm;
+      }
+      const float mcl = m * kLog2e;
+      float e = ex2_approx(fmaf(x.x, kLog2e, -mcl));
+      if (nv > 1) e += ex2_approx(fmaf(x.y, kLog2e, -mcl));
+      if (nv > 2) e += ex2_approx(fmaf(x.z, kLog2e, -mcl));
+      if (nv > 3) e += ex2_approx(fmaf(x.w, kLog2e, -mcl));
+      sl += e;
+    } else {
+      m = fmaxf(m, vm);
+    }
+  };
   for (int v0 = lane; v0 < nfull; v0 += 128) {
     float4 x[4];
 #pragma unroll
@@ -1462,44 +1500,26 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
     for (int u = 0; u < 4; ++u)
       if (v0 + 32 * u < nfull) {
         buf[v0 + 32 * u] = x[u];
-        m = fmaxf(m, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
-        mn = fminf(mn, fminf(fminf(x[u].x, x[u].y), fminf(x[u].z, x[u].w)));
+        fold(x[u], 4);
       }
   }
   if (tail) {  // the row has nb >= 4 nfull + 4 entries: the whole vector is readable
     const float4 x = src[nfull];
     buf[nfull] = x;
-    m = fmaxf(m, x.x);
-    mn = fminf(mn, x.x);
-    if (rem > 1) m = fmaxf(m, x.y), mn = fminf(mn, x.y);
-    if (rem > 2) m = fmaxf(m, x.z), mn = fminf(mn, x.z);
+    fold(x, rem);
   }
+  const float m_lane = m;
   m = warp_max(m);
   mn = -warp_max(-mn);
-  constexpr float kLog2e = 1.4426950408889634f;
   const float mc = m * kLog2e;
   float inv = 1.f;
   if (FROM_LOGITS) {
-    // (B) exponentials and their sum (candidates past len get 0)
-    float sum = 0.f;
-    auto expv = [&](int v, int nv) {
-      const float4 x = buf[v];
-      float4 e;
-      e.x = ex2_approx_full(fmaf(x.x, kLog2e, -mc));
-      e.y = nv > 1 ? ex2_approx_full(fmaf(x.y, kLog2e, -mc)) : 0.f;
-      e.z = nv > 2 ? ex2_approx_full(fmaf(x.z, kLog2e, -mc)) : 0.f;
-      e.w = nv > 3 ? ex2_approx_full(fmaf(x.w, kLog2e, -mc)) : 0.f;
-      buf[v] = e;
-      sum += (e.x + e.y) + (e.z + e.w);
-    };
-#pragma unroll 2
-    for (int v = lane; v < nfull; v += 32) expv(v, 4);
-    if (tail) expv(nfull, rem);
-    inv = 1.0f / warp_sum(sum);
+    // lanes' sums onto the row maximum (a lane with no candidate adds 0)
+    inv = 1.0f / warp_sum(sl * ex2_approx((m_lane - m) * kLog2e));
   }
   const bool radix = !threshold && ki < len;
-  const float vhi = FROM_LOGITS ? ex2_approx_full(fmaf(m, kLog2e, -mc)) * inv : m;
-  const float vlo = FROM_LOGITS ? ex2_approx_full(fmaf(mn, kLog2e, -mc)) * inv : mn;
+  const float vhi = FROM_LOGITS ? ex2_approx(fmaf(m, kLog2e, -mc)) * inv : m;
+  const float vlo = FROM_LOGITS ? ex2_approx(fmaf(mn, kLog2e, -mc)) * inv : mn;
   int hb_p, shift_p;
   uint32_t pmask_p;
   fixed_bits(key_of(vhi) ^ key_of(vlo), hb_p, pmask_p, shift_p);
@@ -1512,12 +1532,12 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   // (C) probabilities, keys, AND / OR, the first histogram on the predicted digit
   uint32_t kand = 0xffffffffu, kor = 0u;
   auto probv = [&](int v, int nv) {
-    const float4 e = buf[v];
+    const float4 x = buf[v];
     float4 pv;
-    pv.x = FROM_LOGITS ? e.x * inv : e.x;
-    pv.y = FROM_LOGITS ? e.y * inv : e.y;
-    pv.z = FROM_LOGITS ? e.z * inv : e.z;
-    pv.w = FROM_LOGITS ? e.w * inv : e.w;
+    pv.x = FROM_LOGITS ? ex2_approx(fmaf(x.x, kLog2e, -mc)) * inv : x.x;
+    pv.y = FROM_LOGITS ? ex2_approx(fmaf(x.y, kLog2e, -mc)) * inv : x.y;
+    pv.z = FROM_LOGITS ? ex2_approx(fmaf(x.z, kLog2e, -mc)) * inv : x.z;
+    pv.w = FROM_LOGITS ? ex2_approx(fmaf(x.w, kLog2e, -mc)) * inv : x.w;
     if (dst) {
       if (nv == 4) {
         *reinterpret_cast<float4*>(dst + 4 * v) = pv;
@@ -1832,13 +1852,27 @@ cudaError_t launch_row_select(const float* in, float* scores, bool from_logits, 
     const size_t smem = sizeof(uint32_t) * (size_t)kSelWarps * (256 + width);
     if (!tab && row_len <= 0 && nb % 4 == 0 && (reinterpret_cast<uintptr_t>(in) & 15) == 0 &&
         (!scores || (reinterpret_cast<uintptr_t>(scores) & 15) == 0)) {
-      // rows start 16-byte aligned: four candidates per lane and access
+      // rows start 16-byte aligned: four candidates per lane and access.  Two
+      // launches: the shorter half of the rows (query blocks below nb / 2)
+      // with half-size row buffers, so more warps share an SM, then the rest.
       auto kern4 = from_logits ? row_select_warp4_kernel<true> : row_select_warp4_kernel<false>;
-      cudaError_t e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      kern4<<<grid, 32 * kSelWarps, smem, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density,
-                                                counts, indices, cap);
-      return cudaGetLastError();
+      const long long heads = rows / nb;
+      const int half_w = ((nb / 2 + 3) / 4) * 4;
+      const long long split = heads * (long long)(nb / 2);
+      const long long lo[2] = {0, split}, hi[2] = {split, rows};
+      const int wd[2] = {half_w, nb};
+      for (int c = 0; c < 2; ++c) {
+        if (hi[c] <= lo[c]) continue;
+        const size_t sm = sizeof(uint32_t) * (size_t)kSelWarps * (256 + wd[c]);
+        cudaError_t e = cudaFuncSetAttribute(kern4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        const unsigned g = (unsigned)((hi[c] - lo[c] + kSelWarps - 1) / kSelWarps);
+        kern4<<<g, 32 * kSelWarps, sm, st>>>(in, from_logits ? scores : nullptr, rows, nb, mode, T, k, density,
+                                            counts, indices, cap, lo[c], hi[c], wd[c]);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+      }
+      return cudaSuccess;
     }
     auto kern = from_logits ? row_select_warp_kernel<true> : row_select_warp_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
