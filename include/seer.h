@@ -239,6 +239,10 @@ SEER_API seer_status seer_gate_select(const seer_dims *dims, const float *scores
  *             count (0 <= c <= min(cap, i+1)) and entry (in range, strictly
  *             ascending) before loading; a failing one is clamped into range
  *             and recorded as SEER_ERR_DEVICE_CHECK in the workspace status.
+ *             With bf16 inputs, when every count is i + 1 (the all-ones
+ *             causal mask: valid lists are then exactly 0..i) a device-side
+ *             check hands the call to the dense 128-row-tile kernel and the
+ *             entries are not read (nor checked).
  *   scale     softmax scale; 0 means 1/sqrt(d)
  *   O         [B,Hq,n,d] same dtype as Q;  lse [B,Hq,n] fp32 (may be NULL)
  * Errors: SEER_ERR_INVALID_ARG, SEER_ERR_UNSUPPORTED, SEER_ERR_WORKSPACE,

@@ -166,6 +166,8 @@ int num_sms() {
 }
 
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+// header word of seer_sparse_attn's dense / sparse choice (1: not the all-ones mask)
+constexpr int kWsNotDenseWord = 40;
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
                                    long long n) {
@@ -704,14 +706,21 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
     q = base + w.q16;
     v16 = base + w.v16;
   }
+  seer::WsHeader* hdr = (seer::WsHeader*)ws;
+  // bf16 inputs: a device-side check picks the 128-row dense kernel when the
+  // lists are the all-ones causal mask (every count is i + 1); the sparse
+  // kernels then return at once, and the other way round
+  const bool dual = dtype == SEER_BF16;
+  uint32_t* not_dense = &hdr->pad[kWsNotDenseWord];
+  if (dual) SEER_CUDA(seer::launch_dense_check(counts, (long long)B * Hq * (n / seer::kBlock), n / seer::kBlock, not_dense, st));
   const long long records = (long long)B * Hkv * (n / seer::kBlock);
-  SEER_CUDA(seer::launch_kt_tiles(K, dtype == SEER_FP32, base + w.kt, records, n, d, st));
+  SEER_CUDA(seer::launch_kt_tiles(K, dtype == SEER_FP32, base + w.kt, records, n, d, st, dual ? not_dense : nullptr));
   CUtensorMap tmQ, tmKt, tmV;
   if (!make_tmap_bf16_panels(&tmQ, q, (long long)B * Hq * n, d, 64) ||
       !make_tmap_rows(&tmKt, base + w.kt, records * d, d) ||
       !make_tmap_bf16_panels(&tmV, v16, (long long)B * Hkv * n, d, 64))
     return cuda_fail(cudaErrorInvalidValue);
-  seer::AttnParams p;
+  seer::AttnParams p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -729,7 +738,6 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.out_fp32 = dtype == SEER_FP32;
   const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
   p.scale_log2 = (float)(sc * 1.4426950408889634);
-  seer::WsHeader* hdr = (seer::WsHeader*)ws;
   p.status = &hdr->status;
   p.work_counter = &hdr->work_counter;
   p.timeout_ns = kTimeoutNs;
@@ -741,9 +749,51 @@ seer_status seer_sparse_attn(const seer_dims* dims, const void* Q, const void* K
   p.test_skip_qk_commit = g_test_skip_qk_commit;
   p.k_rows = 0;
   if (g_test_wait_limit_ns) p.timeout_ns = g_test_wait_limit_ns;
+  p.run_if = dual ? not_dense : nullptr;
+  p.run_if_value = 1;
   SEER_CUDA(seer::launch_empty_rows(p, st));
   SEER_CUDA(seer::launch_sparse_attn(tmQ, tmKt, tmV, p, num_sms(), st));
   SEER_CUDA(seer::launch_sparse_attn_redo(q, base + w.kt, v16, p, st));
+  if (dual) {
+    // the dense path: 128-row query tiles over every causal key block, P in
+    // TMEM (the training forward's kernel without the map)
+    CUtensorMap tmQ2, tmK2, tmV2;
+    if (!make_tmap_bf16_panels(&tmQ2, q, (long long)B * Hq * n, d, 128) ||
+        !make_tmap_bf16_panels(&tmK2, K, (long long)B * Hkv * n, d, 128) ||
+        !make_tmap_bf16_panels(&tmV2, v16, (long long)B * Hkv * n, d, 128))
+      return cuda_fail(cudaErrorInvalidValue);
+    seer::FwdParams f{};
+    f.B = B;
+    f.Hq = Hq;
+    f.Hkv = Hkv;
+    f.n = n;
+    f.d = d;
+    f.nb = p.nb;
+    f.G = p.G;
+    f.npairs = (p.nb + 1) / 2;
+    f.total_units = (long long)B * Hq * f.npairs;
+    f.O = O;
+    f.out_fp32 = 0;
+    f.lse = lse;
+    f.map = nullptr;
+    f.scale_log2 = p.scale_log2;
+    f.r = nullptr;
+    f.status = p.status;
+    f.work_counter = p.work_counter;
+    f.timeout_ns = p.timeout_ns;
+    f.redo_count = p.redo_count;
+    f.redo_list = p.redo_list;
+    f.redo_cap = p.redo_cap;
+    f.run_if = not_dense;
+    f.run_if_value = 0;
+    SEER_CUDA(seer::launch_fwd(tmQ2, tmK2, tmV2, f, num_sms(), st));
+    // its exact fallback reads K as rows
+    seer::AttnParams a = p;
+    a.dense = 1;
+    a.k_rows = 1;
+    a.run_if_value = 0;
+    SEER_CUDA(seer::launch_sparse_attn_redo(q, K, v16, a, st));
+  }
   return SEER_OK;
 }
 
@@ -1101,7 +1151,8 @@ seer_status seer_attn_forward_map(const seer_dims* dims, const void* Q, const vo
       !make_tmap_bf16_panels(&tmV, v, (long long)B * Hkv * n, d, 128))
     return cuda_fail(cudaErrorInvalidValue);
   seer::WsHeader* hdr = (seer::WsHeader*)ws;
-  seer::FwdParams p;
+  seer::FwdParams p{};
+  p.run_if = nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;

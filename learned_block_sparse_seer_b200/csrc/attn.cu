@@ -387,6 +387,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
                        const AttnParams p) {
   using namespace attn;
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (p.run_if && ((*p.run_if != 0u) != (p.run_if_value != 0u))) return;  // the dense kernel takes this call
   // The 128-byte-swizzled tiles need a 1024-byte aligned base.  The dynamic
   // window starts after the reserved per-CTA area, which keeps it aligned;
   // if it ever were not, refuse to run rather than compute garbage.
@@ -854,8 +855,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 // nearest even).
 template <typename T>
 __global__ void __launch_bounds__(256) kt_tile_kernel(const T* __restrict__ K, __nv_bfloat16* __restrict__ out,
-                                                      int n, int d) {
+                                                      int n, int d, const uint32_t* __restrict__ run_if) {
   __shared__ uint16_t sk[64][128 + 2];  // [key][dim]; 260-byte rows keep the column reads spread over banks
+  if (run_if && *run_if == 0u) return;  // the dense kernel takes this call
   const int nb = n / kBlock;
   const long long rec = blockIdx.x;  // (b*Hkv + g)*nb + j
   const long long bg = rec / nb;
@@ -926,6 +928,7 @@ __global__ void __launch_bounds__(256) sparse_attn_redo_kernel(const __nv_bfloat
                                                                const AttnParams p) {
   constexpr int DL = D / 32;  // head dims per lane
   __shared__ float lse2s[64];  // the unit's row LSEs (log2), for the map
+  if (p.run_if && ((*p.run_if != 0u) != (p.run_if_value != 0u))) return;  // the other path's fallback
   const uint32_t nredo = min(*reinterpret_cast<volatile uint32_t*>(p.redo_count), (uint32_t)p.redo_cap);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   for (uint32_t e = blockIdx.x; e < nredo; e += gridDim.x) {
@@ -1035,11 +1038,27 @@ cudaError_t launch_empty_rows(const AttnParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st) {
+__global__ void dense_check_kernel(const int32_t* __restrict__ counts, long long units, int nb,
+                                   uint32_t* __restrict__ not_dense) {
+  bool bad = false;
+  for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (long long)gridDim.x * blockDim.x)
+    bad = bad || counts[u] != (int)(u % nb) + 1;
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) *not_dense = 1u;
+}
+
+cudaError_t launch_dense_check(const int32_t* counts, long long units, int nb, uint32_t* not_dense, cudaStream_t st) {
+  long long blocks = (units + 255) / 256;
+  if (blocks > 592) blocks = 592;
+  dense_check_kernel<<<(unsigned)(blocks < 1 ? 1 : blocks), 256, 0, st>>>(counts, units, nb, not_dense);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st,
+                            const uint32_t* run_if) {
   if (fp32)
-    kt_tile_kernel<float><<<(unsigned)records, 256, 0, st>>>((const float*)K, (__nv_bfloat16*)out, n, d);
+    kt_tile_kernel<float><<<(unsigned)records, 256, 0, st>>>((const float*)K, (__nv_bfloat16*)out, n, d, run_if);
   else
-    kt_tile_kernel<uint16_t><<<(unsigned)records, 256, 0, st>>>((const uint16_t*)K, (__nv_bfloat16*)out, n, d);
+    kt_tile_kernel<uint16_t><<<(unsigned)records, 256, 0, st>>>((const uint16_t*)K, (__nv_bfloat16*)out, n, d, run_if);
   return cudaGetLastError();
 }
 

@@ -26,11 +26,24 @@ struct AttnParams {
   float* map;          // exact fallback of the training forward: [B*Hq*nb, nb] map rows to rewrite, or null
   int test_skip_qk_commit;  // test hook: step whose QK completion is never signalled (-1: none)
   int k_rows;               // exact fallback only: K given as rows [B*Hkv*n, d] instead of K^T records
+  // Device-side choice between this kernel and the 128-row dense kernel: when
+  // run_if is non-null the launch does nothing unless (*run_if != 0) equals
+  // run_if_value (the word is set by launch_dense_check).
+  const uint32_t* run_if;
+  uint32_t run_if_value;
 };
+
+// *not_dense = 1 unless every unit's count is i + 1 (with ascending entries
+// in [0, i], a list of i + 1 entries is then exactly 0..i: the all-ones
+// causal mask).  The word must be 0 before the launch.
+cudaError_t launch_dense_check(const int32_t* counts, long long units, int nb, uint32_t* not_dense, cudaStream_t st);
 
 // Re-layout of K into per-block K^T records of d rows x 64 bf16;
 // `records` = B * Hkv * n/64.
-cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st);
+// With run_if non-null the pass is skipped when *run_if == 0 (the dense path
+// of launch_dense_check's choice needs no records).
+cudaError_t launch_kt_tiles(const void* K, bool fp32, void* out, long long records, int n, int d, cudaStream_t st,
+                            const uint32_t* run_if = nullptr);
 
 // Exact fp32 recomputation of the units the attention kernel flagged (scores
 // so far above the unit's first-step column maximum that its values

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using namespace fwd;
   extern __shared__ __align__(1024) uint8_t smem[];
+  if (p.run_if && ((*p.run_if != 0u) != (p.run_if_value != 0u))) return;  // the sparse kernel takes this call
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) record_status(p.status, kDevBadSchedule, smem_u32(smem));
     return;

@@ -25,6 +25,9 @@ struct FwdParams {
   uint32_t* redo_count;
   int* redo_list;
   int redo_cap;
+  // non-null: the launch does nothing unless (*run_if != 0) == run_if_value
+  const uint32_t* run_if;
+  uint32_t run_if_value;
 };
 
 // Persistent launch of at most `ctas` CTAs (the map scratch holds that many

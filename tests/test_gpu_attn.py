@@ -228,7 +228,9 @@ def test_bounded_wait_gives_up_and_the_device_stays_usable():
     L = _lib.lib()
     w, Q, K, V, Wq, Wk = inputs("tiny")
     Qb, Kb, Vb = (t.to(torch.bfloat16) for t in (Q, K, V))
-    c, ix, _ = oracle.select(oracle.gate(Qb, Kb, Wq, Wk), oracle.MODE_TOPK_K, k=8)
+    # k = 4 of 8 blocks: not the all-ones mask, which seer_sparse_attn hands
+    # to the dense 128-row kernel instead of the sparse one
+    c, ix, _ = oracle.select(oracle.gate(Qb, Kb, Wq, Wk), oracle.MODE_TOPK_K, k=4)
     Qd, Kd, Vd = to_dev(Qb, Kb, Vb)
     cd = torch.as_tensor(c, dtype=torch.int32).cuda()
     idd = torch.as_tensor(ix, dtype=torch.int32).cuda()
