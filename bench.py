@@ -194,15 +194,29 @@ def launches_per_step(w) -> int:
     """This library's kernel launches in one timed step (gate, then sparse
     attention), as the host code issues them for workload w (no RoPE).
 
-    Gate: Q and K pooling (2), the two projections (2), the causal logits
-    (split of q~ and k~ into tf32 parts + the tensor-core product when the
-    gate hidden size is a multiple of 32, else one SIMT GEMM), the softmax
-    and selection (1).  Attention: fp32 inputs first convert Q and V (2); the
-    K^T re-layout (1), the empty-row writer (1), the attention kernel (1)
-    and the exact fallback (1).
+    Gate with h and d multiples of 32: Q and K pooling, already split into
+    tf32 parts (2); the tf32 split of Wq and Wk (2); the two projections,
+    whose epilogues write q~ and k~ split (2); the causal logits (1 when
+    h <= 128 and nb % 4 == 0: the row-resident kernel; else the split of q~
+    and k~ and the tile kernel, 3); the softmax and selection (2 launches,
+    short and long rows, when nb % 4 == 0 and there are at least 8 rows per
+    SM; else 1).  Otherwise the SIMT path: pooling (2), projections (2),
+    logits (1), selection (1).
+    Attention, bf16: the all-ones check (1), the K^T re-layout (1), the
+    empty-row writer (1), the sparse kernel and its exact fallback (2), the
+    dense kernel and its fallback (2; the pair not chosen returns at once).
+    fp32: the conversion of Q and V (2), re-layout, empty rows, kernel and
+    fallback (4).
     """
-    gate = 2 + 2 + (3 if w.h % 32 == 0 else 1) + 1
-    attn = (2 if w.dtype == "fp32" else 0) + 4
+    nb = w.n // 64
+    rows = w.B * w.Hq * nb
+    if w.h % 32 == 0 and w.d % 32 == 0:
+        logits = 1 if (w.h <= 128 and nb % 4 == 0) else 3
+        select = 2 if (nb % 4 == 0 and rows >= 8 * 148) else 1
+        gate = 2 + 2 + 2 + logits + select
+    else:
+        gate = 2 + 2 + 1 + 1
+    attn = 7 if w.dtype == "bf16" else 6
     return gate + attn
 
 

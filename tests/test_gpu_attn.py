@@ -79,6 +79,31 @@ def test_full_size_density_sampled(name, rho):
     check_lse(unit_rows(lse, units, w.nb).double().numpy(), lse_ref)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,nb,d", [(2, 4, 2, 9, 64), (1, 2, 1, 1, 128), (1, 4, 4, 3, 128)])
+def test_all_ones_mask_dense_path_shapes(B, Hq, Hkv, nb, d):
+    """All-ones lists take the dense 128-row kernel (bf16 inputs): odd block
+    counts (a last tile with one valid query block), a single block, MHA,
+    d = 64 and B > 1 against the oracle; one row off the all-ones mask sends
+    the same call to the sparse kernel, with the same result."""
+    w = synth.custom("dense_shapes", B, Hq, Hkv, 64 * nb, d, 16, "bf16", "layer", 40 + nb)
+    Q, K, V = synth.make_qkv(w)
+    c, ix = oracle.dense_lists(B, Hq, nb)
+    O, lse = _run(Q, K, V, c, ix)
+    O_ref, lse_ref = oracle.sparse_attn(Q, K, V, c, ix)
+    check_o(O.double().numpy(), O_ref)
+    check_lse(lse.double().numpy(), lse_ref)
+    if nb > 1:
+        # drop block 0 from the last row of the last head: no longer all-ones
+        c2, ix2 = c.copy(), ix.copy()
+        c2[B - 1, Hq - 1, nb - 1] = nb - 1
+        ix2[B - 1, Hq - 1, nb - 1, :nb - 1] = np.arange(1, nb)
+        ix2[B - 1, Hq - 1, nb - 1, nb - 1:] = -1
+        O2, lse2 = _run(Q, K, V, c2, ix2)
+        O2_ref, lse2_ref = oracle.sparse_attn(Q, K, V, c2, ix2)
+        check_o(O2.double().numpy(), O2_ref)
+        check_lse(lse2.double().numpy(), lse2_ref)
+
+
 def test_all_ones_mask_equals_dense():
     w = synth.custom("dense", 1, 8, 2, 64 * 40, 128, 128, "bf16", "layer", 12)
     Q, K, V = synth.make_qkv(w)
