@@ -1686,7 +1686,27 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   // diagonal joins when forced
   int base = 0;
   uint32_t eq_before = 0;
-  for (int t = 0; t < nc; ++t) {
+  // chunks whose 32 vectors are all whole: with the bin taken whole (and no
+  // forced diagonal) a key is kept iff it is at least the prefix, whose bits
+  // below the fixed ones are zero
+  const int nfc = whole && !force_diag ? nfull >> 5 : 0;
+  for (int t = 0; t < nfc; ++t) {
+    const int v = 32 * t + lane;
+    const uint4 kk = key[v];
+    const bool k0 = kk.x >= prefix, k1 = kk.y >= prefix, k2 = kk.z >= prefix, k3 = kk.w >= prefix;
+    uint32_t tot;
+    uint32_t q = base + warp_excl_scan((uint32_t)k0 + k1 + k2 + k3, lane, tot);
+    const int j0 = 4 * v;
+    st_global_if(out + q, j0, k0);
+    q += k0;
+    st_global_if(out + q, j0 + 1, k1);
+    q += k1;
+    st_global_if(out + q, j0 + 2, k2);
+    q += k2;
+    st_global_if(out + q, j0 + 3, k3);
+    base += (int)tot;
+  }
+  for (int t = nfc; t < nc; ++t) {
     const int v = 32 * t + lane;
     const int nv = nvalid(v);
     uint4 kk = make_uint4(0u, 0u, 0u, 0u);
