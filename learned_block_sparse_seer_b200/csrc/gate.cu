@@ -1433,15 +1433,25 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   // width (a multiple of 4: each warp's row buffer).
   const long long vrow = v0 + (long long)blockIdx.x * kSelWarps + wid;
   if (vrow >= v1) return;  // whole warps only: no CTA barrier follows
+  // 32-bit division when the row count allows it (always, in practice)
   const long long heads = rows / nb;
-  const long long row = (vrow % heads) * nb + vrow / heads;
+  long long hq, ib;
+  if (rows <= 0x7fffffffLL) {
+    const uint32_t vr = (uint32_t)vrow, hd = (uint32_t)heads;
+    ib = vr / hd;
+    hq = vr - (uint32_t)ib * hd;
+  } else {
+    ib = vrow / heads;
+    hq = vrow - ib * heads;
+  }
+  const long long row = hq * nb + ib;
   uint32_t* const hist = sel_smem + wid * 256;
   float4* const buf = reinterpret_cast<float4*>(sel_smem + kSelWarps * 256) + (size_t)wid * (width / 4);
   uint4* const key = reinterpret_cast<uint4*>(buf);
 
   const int mode = mode_flags & 0xff;
   const bool force_diag = (mode_flags & SEER_SELECT_FORCE_DIAGONAL) != 0;
-  const int i = (int)(row % nb);
+  const int i = (int)ib;  // the row's query block
   const int len = i + 1;
   const int nc = (len + 127) >> 7;  // 128-candidate chunks
   const float4* src = reinterpret_cast<const float4*>(in + row * (long long)nb);
@@ -1467,7 +1477,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
   // also each lane's running softmax sum (relative to its running maximum,
   // rescaled when that grows).  Four vectors per lane in flight at a time.
   constexpr float kLog2e = 1.4426950408889634f;
-  float m = -INFINITY, mn = INFINITY, sl = 0.f;
+  float m = -INFINITY, mn = INFINITY, sl = 0.f, mcl = -INFINITY;  // mcl = m log2(e)
   auto fold = [&](float4 x, int nv) {
     if (nv < 4) {  // the row's partial vector: repeat its first candidate for the extremes
       if (nv < 2) x.y = x.x;
@@ -1480,8 +1490,8 @@ __global__ void __launch_bounds__(32 * kSelWarps) row_select_warp4_kernel(
       if (vm > m) {
         sl *= ex2_approx((m - vm) * kLog2e);
         m = vm;
+        mcl = m * kLog2e;
       }
-      const float mcl = m * kLog2e;
       float e = ex2_approx(fmaf(x.x, kLog2e, -mcl));
       if (nv > 1) e += ex2_approx(fmaf(x.y, kLog2e, -mcl));
       if (nv > 2) e += ex2_approx(fmaf(x.z, kLog2e, -mcl));
