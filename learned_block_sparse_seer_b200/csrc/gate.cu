@@ -695,11 +695,9 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
         const int tm = T - 1 - w / batch;
         // the previous item's products must be done before its q~ is overwritten
         if (it > 0 && !mbar_wait(&atm_free, (it - 1) & 1, abort_p, p.status, tmo)) break;
-        for (int part = 0; part < 2 && ok; ++part) {
-          if (!mbar_wait(&a_full, su & 1, abort_p, p.status, tmo)) {
-            ok = false;
-            break;
-          }
+        // one part of the q~ block from the staging buffer into TMEM
+        auto copy_part = [&](int part) -> bool {
+          if (!mbar_wait(&a_full, su & 1, abort_p, p.status, tmo)) return false;
           tc_fence_after();
           const uint32_t ta = tmem + (part ? kColAl : kColAh);
           for (int c = 0; c < nk; ++c)
@@ -709,9 +707,49 @@ __global__ void __launch_bounds__(gtr::kThreads, 1)
                                dA0 + (uint64_t)((c * kSlice + kk * 32) >> 4));
           mma_commit(&a_free);  // the staging buffer is free once these copies are done
           a_used = ++su;
+          return true;
+        };
+        if (!copy_part(0)) break;
+        // The item's first tile takes its tf32-part products while the
+        // remainder part is still loading (its nk <= kBStages slices all stay
+        // resident), then the remainder's products.
+        {
+          const int buf = tile & 1;
+          if (tile >= 2 && !mbar_wait(&acc_empty[buf], ((tile >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
+          tc_fence_after();
+          const uint32_t acc = tmem + (uint32_t)buf * 128u;
+          for (int c = 0; c < nk && ok; ++c) {
+            const int s = (cs + c) % kBStages;
+            if (!mbar_wait(&b_full[s], ((cs + c) / kBStages) & 1, abort_p, p.status, tmo)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dBh = dB0 + (uint64_t)((s * kBStage) >> 4);
+            const uint64_t dBl = dBh + (uint64_t)(kSlice >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = (uint64_t)((kk * 32) >> 4);
+              const uint32_t col = (uint32_t)(c * 32 + kk * 8);
+              mma_tf32_ts(acc, tmem + kColAh + col, dBh + off, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+              mma_tf32_ts(acc, tmem + kColAh + col, dBl + off, idesc, 1u);
+            }
+          }
+          if (!ok || !copy_part(1)) break;
+          for (int c = 0; c < nk; ++c) {
+            const int s = cs % kBStages;
+            const uint64_t dBh = dB0 + (uint64_t)((s * kBStage) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_tf32_ts(acc, tmem + kColAl + (uint32_t)(c * 32 + kk * 8), dBh + (uint64_t)((kk * 32) >> 4), idesc,
+                          1u);
+            mma_commit(&b_empty[s]);
+            b_used = ++cs;
+          }
+          mma_commit(&acc_full[buf]);
+          ++tile;
         }
-        if (!ok) break;
-        for (int tn = 0; tn <= tm && ok; ++tn, ++tile) {
+        for (int tn = 1; tn <= tm && ok; ++tn, ++tile) {
           const int buf = tile & 1;
           if (tile >= 2 && !mbar_wait(&acc_empty[buf], ((tile >> 1) - 1) & 1, abort_p, p.status, tmo)) {
             ok = false;
