@@ -354,9 +354,14 @@ struct DecAttnP {
   unsigned long long timeout_ns;
 };
 
+// The attention ring: NS stages of one key block (K then V); NC consumer
+// warps share every block, warp w taking slabs w, w + NC, ... of it, so a
+// stage is released after a quarter of a block's work instead of a whole one.
 template <typename T, int D>
 struct AttnRing : Ring<2 * kBlock * D * (int)sizeof(T)> {
   static constexpr uint32_t HALF = (uint32_t)kBlock * D * sizeof(T);  // K (then V) of a block
+  static constexpr int NC = 4;                                          // consumer warps
+  static constexpr int THREADS = 32 * (NC + 1);                         // + the copy warp
 };
 
 template <typename T, int D>
@@ -366,11 +371,12 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
   constexpr int E = S::EPC;
   constexpr int LPR = S::LPR;
   constexpr int NS = R::NS;
+  constexpr int NC = R::NC;
   constexpr int SPB = kBlock / S::ROWS;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[NS], empty[NS];
   __shared__ int abort_flag, last;
-  __shared__ float wm[NS], wl[NS], wo[NS][D];
+  __shared__ float wm[NC], wl[NC], wo[NC][D];
   const long long row = blockIdx.x / p.splits;
   const int split = (int)(blockIdx.x % p.splits);
   const long long b = row / p.Hq;
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], NC);
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -400,7 +406,7 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
   volatile int* abort_p = &abort_flag;
   const long long head0 = (b * p.Hkv + g) * (long long)p.n_cap * D;
 
-  if (warp == NS) {
+  if (warp == NC) {
     // ------------------------------------------------------- producer ---
     if (lane == 0) {
       const T* Kh = reinterpret_cast<const T*>(p.K) + head0;
@@ -436,14 +442,15 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
     float m = -INFINITY, l = 0.f, o[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] = 0.f;
-    int k = 0;  // this warp's uses of its stage
-    for (int e = e0 + warp; e < e1; e += NS, ++k) {
-      if (!mbar_wait(&full[warp], k & 1, abort_p, p.status, p.timeout_ns)) break;
+    int k = 0;  // blocks taken so far (every consumer takes every block)
+    for (int e = e0; e < e1; ++e, ++k) {
+      const int st = k % NS;
+      if (!mbar_wait(&full[st], (k / NS) & 1, abort_p, p.status, p.timeout_ns)) break;
       const int nk = e < cnt ? kBlock : tail;
-      const uint8_t* Ks = ring + (size_t)warp * 2 * R::HALF + S::chunk(lane) * 16;
+      const uint8_t* Ks = ring + (size_t)st * 2 * R::HALF + S::chunk(lane) * 16;
       const uint8_t* Vs = Ks + R::HALF;
 #pragma unroll
-      for (int sb = 0; sb < SPB; ++sb) {
+      for (int sb = warp; sb < SPB; sb += NC) {
         const int rbase = sb * S::ROWS;
         if (rbase >= nk) break;  // past the token (warp-uniform)
         uint4 ku[8], vu[8];
@@ -483,7 +490,7 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
         m = mn;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[warp]);
+      if (lane == 0) mbar_arrive(&empty[st]);
     }
     l = warp_sum(l);
 #pragma unroll
@@ -503,19 +510,19 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
   // ---- the CTA's partial (m, l, o)
   float M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < NS; ++w) M = fmaxf(M, wm[w]);
+  for (int w = 0; w < NC; ++w) M = fmaxf(M, wm[w]);
   float* pp = p.part + (row * p.splits + split) * (long long)(D + 2);
   for (int t = tid; t < D; t += R::THREADS) {
     float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < NS; ++w)
+    for (int w = 0; w < NC; ++w)
       if (wm[w] > -INFINITY) a += wo[w][t] * exp2f(wm[w] - M);
     pp[t] = a;
   }
   if (tid == 0) {
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < NS; ++w)
+    for (int w = 0; w < NC; ++w)
       if (wm[w] > -INFINITY) L += wl[w] * exp2f(wm[w] - M);
     pp[D] = M;
     pp[D + 1] = L;
