@@ -15,21 +15,26 @@
 //  * S = Q K^T per key block: tcgen05 kind::tf32, M = 64 query rows, N = 64
 //    keys, K = d (8 per instruction); A and B K-major.  With M = 64 the rows
 //    sit in TMEM lanes 0-15 of each 32-lane sub-partition (row r at lane
-//    r % 16 + 32 (r / 16)), so each softmax warp owns 16 rows.
-//  * O^T += V^T P^T per block: M = d (the d rows of O^T fill the TMEM lanes at
-//    d = 128), N = 64 query columns, K = 64 keys; A = V^T, B = P^T, both
-//    K-major: V is first transposed per 64-key block into the workspace
-//    (vt_kernel: d rows of 64 keys), and P^T is the P tile the softmax writes
-//    (fp32 values, read by the tensor core as tf32).  Every operand is
-//    K-major, the layout the QK product uses too.
-//  * Two S buffers in TMEM, two P tiles: QK of block t+1 and PV of block t-1
-//    run while the softmax works on block t.  The running row maximum is raised lazily (by
-//    more than 8 in log2 units), and only then is O^T rescaled in TMEM.
-//  * Warp roles (224 threads): warps 0-3 softmax and epilogue (TMEM
-//    sub-partitions 0-3), warp 4 loads Q and K (two K stages, freed by QK),
-//    warp 5 issues the MMAs, warp 6 loads V^T (three stages, freed by PV).  Every
-//    wait is bounded; the softmax warps meet at hardware barriers that all
-//    128 threads always reach, carrying any failure with them.
+//    r % 16 + 32 (r / 16)), so each softmax warp owns 16 rows, two threads
+//    per row: the .16x32bx2 TMEM load gives each half-warp 32 of the 64 keys.
+//  * P stays on chip: the softmax writes it (fp32 values, read by the tensor
+//    core as tf32) over S in TMEM, and O += P V runs with A = P from TMEM
+//    (M = 64, the layout of S) and B = V^T from shared memory (N = d, K = 64
+//    keys, K-major: V is first transposed per 64-key block into the
+//    workspace by vt_kernel, since kind::tf32 reads K-major operands only).
+//  * O is a 64 x d accumulator in TMEM in the same row layout, so a row's
+//    rescale (its running maximum is raised lazily, by more than 8 in log2
+//    units) is done by the two threads that own the row, and the softmax
+//    warps never wait for one another.
+//  * Three S / P buffers in TMEM: QK of block t+1 and t+2 and PV of block t-1
+//    can run while the softmax works on block t.
+//  * Warp roles (256 threads): warps 0-3 softmax and epilogue (TMEM
+//    sub-partitions 0-3), warp 4 loads Q and K (three K stages, freed by
+//    QK), warp 5 issues the QK products, warp 6 loads V^T (three stages,
+//    freed by PV), warp 7 issues the PV products.  With one issuer per
+//    product, QK runs ahead into free S buffers while PV waits for the
+//    softmax.  Every wait is bounded; a wait that gives up raises the CTA's abort
+//    flag, so every other wait of the CTA gives up too.
 #include <cmath>
 #include <cstdint>
 
@@ -41,12 +46,13 @@
 namespace seer {
 
 namespace tf32a {
-constexpr int kThreads = 224;
-constexpr int kWarpLoad = 4, kWarpMma = 5, kWarpLoadV = 6;
-constexpr int kKS = 2, kVS = 3;  // K and V^T stages
+constexpr int kThreads = 256;
+constexpr int kWarpLoad = 4, kWarpQK = 5, kWarpLoadV = 6, kWarpPV = 7;
+constexpr int kKS = 3, kVS = 3;  // K and V^T stages
+constexpr int kSB = 3;           // S / P buffers in TMEM
 constexpr uint32_t kPanel = 64u * 128u;  // 64 rows x 32 floats
-constexpr uint32_t kTmemCols = 256;      // S x 2 (64 cols each), O^T (64 cols)
-constexpr uint32_t kColO = 128;
+constexpr uint32_t kTmemCols = 512;      // S / P x 3 (64 cols each), O (d cols from kColO)
+constexpr uint32_t kColO = 256;
 constexpr float kRaise = 8.0f;
 
 template <int D>
@@ -56,28 +62,37 @@ struct Layout {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kTile;                  // kKS K tiles
   static constexpr uint32_t kOffV = kOffK + kKS * kTile;     // kVS V^T tiles
-  static constexpr uint32_t kOffP = kOffV + kVS * kTile;
-  static constexpr uint32_t kSmem = kOffP + 4 * kPanel;  // two P tiles
+  static constexpr uint32_t kSmem = kOffV + kVS * kTile;
   static constexpr uint32_t kVtPanel = (uint32_t)D * 128u;  // V^T: d rows x 32 keys
 };
 
 struct Ctrl {
-  uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS], s_full[2], s_free[2], p_full[2], pv_done[2];
-  uint64_t fin;
+  uint64_t q_full, k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS], s_full[kSB], p_full[kSB], pv_done[kSB];
+  uint64_t fin_qk, fin_pv;
   uint32_t tmem_base;
   int abort_flag;
-  float alpha[2][64], linv[64];  // alpha by step parity
 };
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  uint32_t a[16], b[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    a[k] = r[k];
-    b[k] = r[16 + k];
+// The thread's half of its O row in TMEM (row 16 w + l % 16 of warp w, lane
+// l): columns (l / 16) d/2 .. + d/2, in two (d = 128) or one (d = 64)
+// 32-column pieces.
+template <int D>
+__device__ __forceinline__ void o_load(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
+  if constexpr (D == 128) {
+    tmem_ld32_halves<64>(taddr, a);
+    tmem_ld32_halves<64>(taddr + 32u, b);
+  } else {
+    tmem_ld32_halves<32>(taddr, a);
   }
-  tmem_st16(taddr, a);
-  tmem_st16(taddr + 16u, b);
+}
+template <int D>
+__device__ __forceinline__ void o_store(uint32_t taddr, const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+  if constexpr (D == 128) {
+    tmem_st32_halves<64>(taddr, a);
+    tmem_st32_halves<64>(taddr + 32u, b);
+  } else {
+    tmem_st32_halves<32>(taddr, a);
+  }
 }
 
 // The list entry t of a unit, checked: an entry outside 0..i is recorded
@@ -137,18 +152,16 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       mbar_init(&C.v_full[s], 1);
       mbar_init(&C.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSB; ++s) {
       mbar_init(&C.s_full[s], 1);
-      mbar_init(&C.s_free[s], 4);
-    }
-    for (int s = 0; s < 2; ++s) {
       mbar_init(&C.p_full[s], 4);
       mbar_init(&C.pv_done[s], 1);
     }
-    mbar_init(&C.fin, 1);
+    mbar_init(&C.fin_qk, 1);
+    mbar_init(&C.fin_pv, 1);
     fence_barrier_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpQK) {
     tmem_alloc(&C.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -198,101 +211,104 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       for (int k = t > kVS ? t - kVS : 0; k < t; ++k)
         mbar_wait(&C.v_full[k % kVS], (k / kVS) & 1, abort_p, nullptr, 20000000ull);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------ MMA issuer ---
+  } else if (warp == kWarpQK) {
+    // ----------------------------------------------------- QK issuer ---
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc_tf32(64, 64, 0, 0);  // A = Q, B = K (both K-major)
-      constexpr uint32_t idesc_pv = make_idesc_tf32(D, 64, 0, 0);   // A = V^T, B = P^T (both K-major)
       const uint32_t sbase = smem_u32(smem);
       const uint64_t dQ = make_sw128_desc(sbase + L::kOffQ, 16, 1024);
-      const uint64_t dP = make_sw128_desc(sbase + L::kOffP, 16, 1024);
       bool ok = mbar_wait(&C.q_full, 0, abort_p, p.status, tmo);
-      for (int t = 0; ok && t <= cnt; ++t) {
-        if (t < cnt) {
-          const int s = t & 1, ks = t % kKS;
-          if (!mbar_wait(&C.k_full[ks], (t / kKS) & 1, abort_p, p.status, tmo)) break;
-          if (t >= 2 && !mbar_wait(&C.s_free[s], ((t >> 1) - 1) & 1, abort_p, p.status, tmo)) break;
-          tc_fence_after();
-          const uint64_t dK = make_sw128_desc(sbase + L::kOffK + (uint32_t)ks * L::kTile, 16, 1024);
+      for (int t = 0; ok && t < cnt; ++t) {
+        const int sb = t % kSB, ks = t % kKS;
+        if (!mbar_wait(&C.k_full[ks], (t / kKS) & 1, abort_p, p.status, tmo)) break;
+        // S / P buffer sb held P(t - kSB): free once that block's PV is done
+        if (t >= kSB && !mbar_wait(&C.pv_done[sb], ((t / kSB) - 1) & 1, abort_p, p.status, tmo)) break;
+        tc_fence_after();
+        const uint64_t dK = make_sw128_desc(sbase + L::kOffK + (uint32_t)ks * L::kTile, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < D / 8; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
-            mma_tf32_ss(tmem + (uint32_t)s * 64u, dQ + off, dK + off, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&C.s_full[s]);
-          mma_commit(&C.k_empty[ks]);
+        for (int kk = 0; kk < D / 8; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
+          mma_tf32_ss(tmem + (uint32_t)sb * 64u, dQ + off, dK + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        if (t >= 1) {  // PV of block t - 1
-          const int u = t - 1, vs = u % kVS;
-          if (!mbar_wait(&C.v_full[vs], (u / kVS) & 1, abort_p, p.status, tmo)) break;
-          if (!mbar_wait(&C.p_full[u & 1], (u >> 1) & 1, abort_p, p.status, tmo)) break;
-          tc_fence_after();
-          // V^T, K-major: d rows of 32 keys per panel, two panels
-          const uint64_t dV = make_sw128_desc(sbase + L::kOffV + (uint32_t)vs * L::kTile, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ss(tmem + kColO, dV + (uint64_t)(((kk >> 2) * L::kVtPanel + (kk & 3) * 32) >> 4),
-                        dP + (uint64_t)(((u & 1) * 2 * kPanel + (kk >> 2) * kPanel + (kk & 3) * 32) >> 4), idesc_pv,
-                        (u > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&C.pv_done[u & 1]);
-          mma_commit(&C.v_empty[vs]);
-        }
+        mma_commit(&C.s_full[sb]);
+        mma_commit(&C.k_empty[ks]);
       }
-      mma_commit(&C.fin);
-      mbar_wait(&C.fin, 0, abort_p, nullptr, 20000000ull);
+      mma_commit(&C.fin_qk);
+      mbar_wait(&C.fin_qk, 0, abort_p, nullptr, 20000000ull);
+    }
+  } else if (warp == kWarpPV) {
+    // ----------------------------------------------------- PV issuer ---
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = make_idesc_tf32(64, D, 0, 0);  // A = P (TMEM), B = V^T (K-major)
+      const uint32_t sbase = smem_u32(smem);
+      for (int u = 0; u < cnt; ++u) {
+        const int vs = u % kVS, ub = u % kSB;
+        if (!mbar_wait(&C.v_full[vs], (u / kVS) & 1, abort_p, p.status, tmo)) break;
+        if (!mbar_wait(&C.p_full[ub], (u / kSB) & 1, abort_p, p.status, tmo)) break;
+        tc_fence_after();
+        // V^T, K-major: d rows of 32 keys per panel, two panels; P: one
+        // TMEM column per key
+        const uint64_t dV = make_sw128_desc(sbase + L::kOffV + (uint32_t)vs * L::kTile, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_tf32_ts(tmem + kColO, tmem + (uint32_t)ub * 64u + (uint32_t)(8 * kk),
+                      dV + (uint64_t)(((kk >> 2) * L::kVtPanel + (kk & 3) * 32) >> 4), idesc_pv,
+                      (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&C.pv_done[ub]);
+        mma_commit(&C.v_empty[vs]);
+      }
+      mma_commit(&C.fin_pv);
+      mbar_wait(&C.fin_pv, 0, abort_p, nullptr, 20000000ull);
     }
   } else {
     // ------------------------------------------- softmax and epilogue ---
     // Warp ww owns query rows 16 ww .. 16 ww + 15 (lanes 0-15 of its TMEM
-    // sub-partition) and, for O^T, the d rows of its sub-partition's lanes.
+    // sub-partition), two threads per row: thread l takes row 16 ww + l % 16
+    // and keys 32 hf .. 32 hf + 31 of each block, hf = l / 16, and the
+    // same half of the row's d columns of O.
     const int ww = warp;
     const bool row_thread = lane < 16;
+    const int hf = lane >> 4;
     const int q = 16 * ww + (lane & 15);
     const uint32_t lane_base = tmem + ((uint32_t)(ww * 32) << 16);
     const float c = p.scale_log2;
     const uint64_t c2 = f32x2_pack(c, c);
+    // m: the row's running maximum (the same in both threads of a row);
+    // l: this thread's half of the row sum, scaled as m rises
     float m = -INFINITY, l = 0.f;
     // lists ascend with every entry <= i, so only the last can be the
     // diagonal block (a bad entry reads as the diagonal, as the producers do)
     const int last_j = tf32a::entry(p, unit, i, cnt - 1);
     bool ok = true;
     for (int t = 0; t < cnt; ++t) {
-      const int s = t & 1;
+      const int s = t % kSB;
       const int j = t == cnt - 1 ? last_j : -1;
-      ok = ok && mbar_wait(&C.s_full[s], (t >> 1) & 1, abort_p, p.status, tmo);
-      uint32_t r0[32], r1[32];
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&C.s_full[s], (t / kSB) & 1, abort_p, p.status, tmo));
+      uint32_t r0[32];
       if (ok) {
         tc_fence_after();
-        tmem_ld32(lane_base + (uint32_t)s * 64u, r0);
-        tmem_ld32(lane_base + (uint32_t)s * 64u + 32u, r1);
+        tmem_ld32_halves<32>(lane_base + (uint32_t)s * 64u, r0);
         tmem_wait_ld();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(&C.s_free[s]);
       // scores in log2 units, two at a time (packed f32x2)
-      float x[64];
+      float x[32];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 16; ++k)
         f32x2_unpack(mul_f32x2(f32x2_pack(__uint_as_float(r0[2 * k]), __uint_as_float(r0[2 * k + 1])), c2), x[2 * k],
                      x[2 * k + 1]);
-        f32x2_unpack(mul_f32x2(f32x2_pack(__uint_as_float(r1[2 * k]), __uint_as_float(r1[2 * k + 1])), c2),
-                     x[32 + 2 * k], x[33 + 2 * k]);
-      }
       if (j == i) {  // causal rule inside the diagonal block
 #pragma unroll
-        for (int k = 0; k < 64; ++k) x[k] = k > q ? -INFINITY : x[k];
+        for (int k = 0; k < 32; ++k) x[k] = 32 * hf + k > q ? -INFINITY : x[k];
       }
-      // row maximum by a tree of 3-input maxima (depth 4, not a 63-long chain)
-      float t1[22];
+      // row maximum: a tree of 3-input maxima over this thread's 32 keys,
+      // then the other half of the row
+      float t1[11];
 #pragma unroll
-      for (int k = 0; k < 21; ++k) t1[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
-      t1[21] = x[63];
-      float t2[8];
-#pragma unroll
-      for (int k = 0; k < 7; ++k) t2[k] = fmax3(t1[3 * k], t1[3 * k + 1], t1[3 * k + 2]);
-      t2[7] = t1[21];
-      const float mx = fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), fmaxf(t2[6], t2[7]));
+      for (int k = 0; k < 10; ++k) t1[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+      t1[10] = fmaxf(x[30], x[31]);
+      const float mh = fmaxf(fmax3(fmax3(t1[0], t1[1], t1[2]), fmax3(t1[3], t1[4], t1[5]), fmax3(t1[6], t1[7], t1[8])),
+                             fmaxf(t1[9], t1[10]));
+      const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
       float alpha = 1.f;
       bool raise = false;
       if (mx > m + kRaise) {
@@ -305,88 +321,78 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
       }
       // probabilities, and their sum by a tree of packed adds
       const uint64_t nm2 = f32x2_pack(-m, -m);
-      uint64_t acc[16];
+      uint64_t acc[8];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
+      for (int k = 0; k < 16; ++k) {
         float a, bb;
         f32x2_unpack(add_f32x2(f32x2_pack(x[2 * k], x[2 * k + 1]), nm2), a, bb);
         x[2 * k] = ex2_approx(a);
         x[2 * k + 1] = ex2_approx(bb);
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
+      for (int k = 0; k < 8; ++k)
         acc[k] = add_f32x2(f32x2_pack(x[4 * k], x[4 * k + 1]), f32x2_pack(x[4 * k + 2], x[4 * k + 3]));
 #pragma unroll
-      for (int w2 = 8; w2 > 0; w2 >>= 1)
+      for (int w2 = 4; w2 > 0; w2 >>= 1)
 #pragma unroll
         for (int k = 0; k < w2; ++k) acc[k] = add_f32x2(acc[k], acc[k + w2]);
       float s0, s1;
       f32x2_unpack(acc[0], s0, s1);
       l += s0 + s1;
-      // P(t) goes to the tile PV(t-2) read
-      if (t >= 2) ok = ok && mbar_wait(&C.pv_done[t & 1], ((t >> 1) - 1) & 1, abort_p, p.status, tmo);
-      if (row_thread) C.alpha[t & 1][q] = alpha;
-      // every softmax thread reaches these barriers; a failure anywhere ends
-      // the loop for all of them together
-      const bool any_raise = bar_red_or(1, 128, row_thread && raise);
-      // a rescale of O^T waits for every PV so far (PV(t-1) and before)
-      if (any_raise && t >= 1) ok = ok && mbar_wait(&C.pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_p, p.status, tmo);
-      ok = !bar_red_or(2, 128, !ok);
-      if (!ok) break;
-      if (any_raise) {
-        tc_fence_after();
-        uint32_t o0[32], o1[32];
-        tmem_ld32(lane_base + kColO, o0);
-        tmem_ld32(lane_base + kColO + 32u, o1);
-        tmem_wait_ld();
+      // a raised row rescales its O row, after every PV so far (PV(t-1) and
+      // before) has landed; the warp's rows share the TMEM access
+      if (__any_sync(0xffffffffu, raise)) {
+        const int u = t - 1;  // raise implies t > 0
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(&C.pv_done[u % kSB], (u / kSB) & 1, abort_p, p.status, tmo));
+        if (ok) {
+          tc_fence_after();
+          uint32_t oa[32], ob[32];
+          o_load<D>(lane_base + kColO, oa, ob);
+          tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          o0[k] = __float_as_uint(__uint_as_float(o0[k]) * C.alpha[t & 1][k]);
-          o1[k] = __float_as_uint(__uint_as_float(o1[k]) * C.alpha[t & 1][32 + k]);
+          for (int k = 0; k < 32; ++k) {
+            oa[k] = __float_as_uint(__uint_as_float(oa[k]) * alpha);
+            if (D == 128) ob[k] = __float_as_uint(__uint_as_float(ob[k]) * alpha);
+          }
+          o_store<D>(lane_base + kColO, oa, ob);
         }
-        tmem_st32(lane_base + kColO, o0);
-        tmem_st32(lane_base + kColO + 32u, o1);
+      }
+      // P(t) over S(t): the A operand of PV(t)
+      if (ok) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pk[k] = __float_as_uint(x[k]);
+        tmem_st32_halves<32>(lane_base + (uint32_t)s * 64u, pk);
         tmem_wait_st();
       }
-      if (row_thread) {
-        // P[q][0..63] as fp32 into the two 32-key panels, 128-byte swizzle
-        uint8_t* prow = smem + L::kOffP + (uint32_t)(t & 1) * 2u * kPanel + (uint32_t)q * 128u;
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          const int pn = cc >> 3, ch = cc & 7;
-          float4 v = make_float4(x[4 * cc], x[4 * cc + 1], x[4 * cc + 2], x[4 * cc + 3]);
-          *reinterpret_cast<float4*>(prow + pn * kPanel + ((ch ^ (q & 7)) << 4)) = v;
-        }
-      }
-      fence_async_shared();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&C.p_full[t & 1]);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive(&C.p_full[s]);
     }
-    // ---- epilogue: O = O^T columns / l, LSE
-    if (ok) ok = mbar_wait(&C.pv_done[(cnt - 1) & 1], ((cnt - 1) >> 1) & 1, abort_p, p.status, tmo);
-    if (row_thread) {
-      C.linv[q] = 1.0f / l;
-      if (p.lse) p.lse[qrow0 + q] = (m + log2f(l)) * 0.6931471805599453f;
+    // ---- epilogue: O / l, LSE
+    if (ok) {
+      const int u = cnt - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&C.pv_done[u % kSB], (u / kSB) & 1, abort_p, p.status, tmo));
     }
-    ok = !bar_red_or(2, 128, !ok);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);  // the row's two halves
+    if (row_thread && p.lse) p.lse[qrow0 + q] = (m + log2f(l)) * 0.6931471805599453f;
     if (ok) {
       tc_fence_after();
-      uint32_t o0[32], o1[32];
-      tmem_ld32(lane_base + kColO, o0);
-      tmem_ld32(lane_base + kColO + 32u, o1);
+      uint32_t oa[32], ob[32];
+      o_load<D>(lane_base + kColO, oa, ob);
       tmem_wait_ld();
-      // O^T lane -> d: all 128 lanes at d = 128; lanes 0-15 of each
-      // sub-partition (d = 16 ww + lane) at d = 64
-      const bool d_thread = D == 128 || lane < 16;
-      const int dd = D == 128 ? ww * 32 + lane : 16 * ww + (lane & 15);
-      if (d_thread) {
-        float* out = O + qrow0 * D + dd;
+      const float linv = 1.0f / l;
+      float* out = O + (qrow0 + q) * D + hf * (D / 2);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          out[(long long)k * D] = __uint_as_float(o0[k]) * C.linv[k];
-          out[(long long)(32 + k) * D] = __uint_as_float(o1[k]) * C.linv[32 + k];
-        }
+      for (int k = 0; k < 8; ++k) {
+        reinterpret_cast<float4*>(out)[k] =
+            make_float4(__uint_as_float(oa[4 * k]) * linv, __uint_as_float(oa[4 * k + 1]) * linv,
+                        __uint_as_float(oa[4 * k + 2]) * linv, __uint_as_float(oa[4 * k + 3]) * linv);
+        if (D == 128)
+          reinterpret_cast<float4*>(out + 32)[k] =
+              make_float4(__uint_as_float(ob[4 * k]) * linv, __uint_as_float(ob[4 * k + 1]) * linv,
+                          __uint_as_float(ob[4 * k + 2]) * linv, __uint_as_float(ob[4 * k + 3]) * linv);
       }
     }
   }
@@ -394,7 +400,7 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpQK) tmem_dealloc(tmem, kTmemCols);
 }
 
 // V^T per 64-key block: Vt[(bh * nb + j) * d + c][k] = V[bh][64 j + k][c].
