@@ -23,7 +23,8 @@
 //   kcache_kernel       CTA per (batch, KV head, 16 blocks): pooling by slabs,
 //                       then the projection k~ = Wk[g] kbar as a shared-memory
 //                       tiled product in packed f32x2 FMAs (Wk read once per
-//                       16 blocks)
+//                       16 blocks, each 32-feature slice loaded one slice
+//                       ahead)
 //   decode_logits_kernel  CTA per (batch, KV head, head group, row chunk):
 //                       q . k~_j / sqrt(d) for GT query heads of the group at
 //                       once (k~ read once for them); the softmax and the
@@ -164,7 +165,7 @@ constexpr int kKcThreads = 256;
 }  // namespace
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict__ K, const float* __restrict__ Wk,
+__global__ void __launch_bounds__(kKcThreads, 4) kcache_kernel(const T* __restrict__ K, const float* __restrict__ Wk,
                                                             float* __restrict__ kt, int Hkv, int n_cap, int j0,
                                                             int nnew) {
   using S = dec::Slab<T, D>;
@@ -242,13 +243,27 @@ __global__ void __launch_bounds__(kKcThreads) kcache_kernel(const T* __restrict_
 #pragma unroll
   for (int b = 0; b < BPG / 2; ++b) acc[b] = 0ull;
   const float* W = Wk + (long long)g * D * 3 * D;
+  // The 32-feature slices of Wk[g] go through registers one slice ahead, so
+  // that a slice's loads are in flight while the previous one is multiplied.
+  constexpr int PER = D * 32 / kKcThreads;  // elements of a slice per thread
+  float wr[PER];
+  auto load_slice = [&](int e0) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int x = threadIdx.x + i * kKcThreads, r = x >> 5, cc = x & 31;
+      wr[i] = W[(long long)r * 3 * D + e0 + cc];
+    }
+  };
+  load_slice(0);
   for (int e0 = 0; e0 < 3 * D; e0 += 32) {
     __syncthreads();  // kbarT complete / previous tile consumed
-    for (int x = threadIdx.x; x < D * 32; x += kKcThreads) {
-      const int r = x >> 5, cc = x & 31;
-      wt[cc * WS + r] = W[(long long)r * 3 * D + e0 + cc];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int x = threadIdx.x + i * kKcThreads, r = x >> 5, cc = x & 31;
+      wt[cc * WS + r] = wr[i];
     }
     __syncthreads();
+    if (e0 + 32 < 3 * D) load_slice(e0 + 32);
 #pragma unroll 4
     for (int ee = 0; ee < 32; ++ee) {
       const float w = wt[ee * WS + o];
