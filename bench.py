@@ -195,7 +195,7 @@ def launches_per_step(w) -> int:
     attention), as the host code issues them for workload w (no RoPE).
 
     Gate with h and d multiples of 32: Q and K pooling, already split into
-    tf32 parts (2); the tf32 split of Wq and Wk (2); the two projections,
+    tf32 parts, and the tf32 split of Wq and Wk, in one launch (1); the two projections,
     whose epilogues write q~ and k~ split (2); the causal logits (1 when
     h <= 128 and nb % 4 == 0: the row-resident kernel; else the split of q~
     and k~ and the tile kernel, 3); the softmax and selection (2 launches,
@@ -213,7 +213,7 @@ def launches_per_step(w) -> int:
     if w.h % 32 == 0 and w.d % 32 == 0:
         logits = 1 if (w.h <= 128 and nb % 4 == 0) else 3
         select = 2 if (nb % 4 == 0 and rows >= 8 * 148) else 1
-        gate = 2 + 2 + 2 + logits + select
+        gate = 1 + 2 + logits + select
     else:
         gate = 2 + 2 + 1 + 1
     attn = 7 if w.dtype == "bf16" else 6

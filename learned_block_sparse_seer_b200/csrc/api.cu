@@ -500,10 +500,29 @@ seer_status run_gate(const seer_dims* dims, const void* Q, const void* K, seer_d
     float* wql = (float*)(base + w.wq_lo);
     float* wkh = (float*)(base + w.wk_hi);
     float* wkl = (float*)(base + w.wk_lo);
-    SEER_CUDA(seer::launch_pool(Q, dtype, false, (long long)B * Hq, n, d, qbhi, st, tab, qblo));
-    SEER_CUDA(seer::launch_pool(K, dtype, true, (long long)B * Hkv, n, d, kbhi, st, tab, kblo));
-    SEER_CUDA(seer::launch_split_tf32_copy(Wq, wqh, wql, (long long)Hq * h * d, st));
-    SEER_CUDA(seer::launch_split_tf32_copy(Wk, wkh, wkl, (long long)Hkv * h * 3 * d, st));
+    seer::GateInputs gi;
+    gi.Q = Q;
+    gi.K = K;
+    gi.nq = (long long)B * Hq * nb;
+    gi.nk = (long long)B * Hkv * nb;
+    gi.cq = (gi.nq + 7) / 8;
+    gi.ck = (gi.nk + 7) / 8;
+    gi.n = n;
+    gi.d = d;
+    gi.qhi = qbhi;
+    gi.qlo = qblo;
+    gi.khi = kbhi;
+    gi.klo = kblo;
+    gi.tab = tab;
+    gi.Wq = Wq;
+    gi.Wk = Wk;
+    gi.nwq = (long long)Hq * h * d;
+    gi.nwk = (long long)Hkv * h * 3 * d;
+    gi.wqh = wqh;
+    gi.wql = wql;
+    gi.wkh = wkh;
+    gi.wkl = wkl;
+    SEER_CUDA(seer::launch_gate_inputs(gi, dtype, st));
     CUtensorMap tmAh, tmAl, tmBh, tmBl;
     seer::Tf32x3Params tp;
     tp.M = nb;

@@ -55,13 +55,12 @@ __device__ __forceinline__ float tf32_hi(float v) {
   return __uint_as_float(h);
 }
 
+// One warp pools block `warp` (the warp-uniform index over B*H*nb blocks).
 template <typename T, bool IS_K>
-__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long long nblocks,
-                                                   int n, int d, float* __restrict__ out,
-                                                   const int2* __restrict__ tab, float* __restrict__ lo) {
+__device__ __forceinline__ void pool_block(const T* __restrict__ X, long long warp, int n, int d,
+                                           float* __restrict__ out, const int2* __restrict__ tab,
+                                           float* __restrict__ lo) {
   constexpr int EPL = 16 / sizeof(T);  // elements per lane per load
-  const long long warp = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  if (warp >= nblocks) return;
   const int lane = threadIdx.x & 31;
   const int nb = n / kBlock;
   const long long bh = warp / nb;
@@ -147,6 +146,42 @@ __global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long
 #pragma unroll
       for (int e = 0; e < EPL; ++e) v[e] = sum[e] * inv;
       put(2 * d, v);
+    }
+  }
+}
+
+template <typename T, bool IS_K>
+__global__ void __launch_bounds__(256) pool_kernel(const T* __restrict__ X, long long nblocks,
+                                                   int n, int d, float* __restrict__ out,
+                                                   const int2* __restrict__ tab, float* __restrict__ lo) {
+  const long long warp = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (warp >= nblocks) return;
+  pool_block<T, IS_K>(X, warp, n, d, out, tab, lo);
+}
+
+// The gate's inputs in one launch, for the tensor-core projections: CTAs
+// [0, cq) pool Q (warp per block), [cq, cq + ck) pool K, and the rest split
+// Wq and Wk into their tf32 parts and remainders.  All three read HBM only,
+// so they share the launch's bandwidth instead of running one after another.
+template <typename T>
+__global__ void __launch_bounds__(256, 4) gate_inputs_kernel(GateInputs g) {
+  const long long cta = blockIdx.x;
+  if (cta < g.cq) {
+    const long long warp = cta * 8 + threadIdx.x / 32;
+    if (warp < g.nq) pool_block<T, false>((const T*)g.Q, warp, g.n, g.d, g.qhi, g.tab, g.qlo);
+  } else if (cta < g.cq + g.ck) {
+    const long long warp = (cta - g.cq) * 8 + threadIdx.x / 32;
+    if (warp < g.nk) pool_block<T, true>((const T*)g.K, warp, g.n, g.d, g.khi, g.tab, g.klo);
+  } else {
+    const long long t0 = (cta - g.cq - g.ck) * 256 + threadIdx.x;
+    const long long stride = (gridDim.x - g.cq - g.ck) * 256ll;
+    for (long long i = t0; i < g.nwq + g.nwk; i += stride) {
+      const bool isq = i < g.nwq;
+      const long long j = isq ? i : i - g.nwq;
+      const float v = isq ? g.Wq[j] : g.Wk[j];
+      const float hi = tf32_hi(v);
+      (isq ? g.wqh : g.wkh)[j] = hi;
+      (isq ? g.wql : g.wkl)[j] = v - hi;
     }
   }
 }
@@ -1855,6 +1890,16 @@ cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, i
     else
       pool_kernel<float, false><<<grid, warps * 32, 0, st>>>((const float*)X, nblocks, n, d, out, tab, lo);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_inputs(const GateInputs& g, seer_dtype dt, cudaStream_t st) {
+  const long long wsplit = 148;  // CTAs that split the weights (grid-stride)
+  const long long grid = g.cq + g.ck + wsplit;
+  if (dt == SEER_BF16)
+    gate_inputs_kernel<uint16_t><<<(unsigned)grid, 256, 0, st>>>(g);
+  else
+    gate_inputs_kernel<float><<<(unsigned)grid, 256, 0, st>>>(g);
   return cudaGetLastError();
 }
 

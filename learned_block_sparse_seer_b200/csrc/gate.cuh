@@ -13,6 +13,25 @@ namespace seer {
 // varlen block table (valid tokens per block).
 // lo non-null: out receives each pooled value rounded to tf32 and lo the exact
 // remainder (the tf32x3 operand split), instead of the fp32 value.
+// Inputs of the tensor-core gate, pooled and split in one launch: Q blocks
+// (average, [B*Hq*nb, d]) and K blocks ([max | min | avg], [B*Hkv*nb, 3d]),
+// each written as tf32 part (qhi, khi) and remainder (qlo, klo), and the
+// weights Wq (nwq floats) and Wk (nwk floats) split the same way.  cq and ck
+// are the CTAs (8 warps, a block per warp) of the two poolings.
+struct GateInputs {
+  const void* Q;
+  const void* K;
+  long long nq, nk, cq, ck;
+  int n, d;
+  float *qhi, *qlo, *khi, *klo;
+  const int2* tab;
+  const float* Wq;
+  const float* Wk;
+  long long nwq, nwk;
+  float *wqh, *wql, *wkh, *wkl;
+};
+cudaError_t launch_gate_inputs(const GateInputs& g, seer_dtype dt, cudaStream_t st);
+
 cudaError_t launch_pool(const void* X, seer_dtype dt, bool is_k, long long BH, int n, int d,
                         float* out, cudaStream_t st, const int2* tab = nullptr, float* lo = nullptr);
 

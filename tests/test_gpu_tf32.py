@@ -142,3 +142,47 @@ def test_layer8k_sampled():
         O_MAX, _, LSE_MAX = _bounds(Q[:, hq:hq + 1, 64 * i:64 * (i + 1)], K[:, g:g + 1], V[:, g:g + 1])
         assert np.abs(Of[u] - O_u[k]).max() <= O_MAX
         assert np.abs(lf[u] - lse_u[k]).max() <= LSE_MAX
+
+
+def _unit_bounds(Q, K, V, b, hq, g, i, keys):
+    """Per-unit tolerances over the keys the unit attends (the bound of
+    _bounds restricted to those keys)."""
+    q = Q[b, hq, 64 * i:64 * (i + 1)].double()
+    k = K[b, g, keys].double()
+    v = V[b, g, keys].double()
+    worst = (q.abs() @ k.abs().T).max().item()
+    delta = 2.0 ** -9 * worst / np.sqrt(q.shape[-1])
+    o_max = (2 * delta + 2.0 ** -9) * v.abs().max().item()
+    return o_max, delta * 1.01 + 1e-6
+
+
+def test_layer128k_sampled_bench_config():
+    """The 128k layer as the bench times it: the gate's density-0.1 lists of
+    the bf16 layer, the layer's values held in fp32, one full-size launch;
+    sampled units (first and last query blocks of the first and last heads,
+    plus seeded random ones) against the oracle."""
+    from gpu_common import inputs, sample_units, to_dev
+    w, Q, K, V, Wq, Wk = inputs("layer128k")
+    Qd, Kd, Wqd, Wkd = to_dev(Q, K, Wq, Wk)
+    cd, idd = seer.seer_gate(Qd, Kd, Wqd, Wkd, "density", density=0.1)
+    del Qd, Kd
+    c, ix = cd.cpu().numpy(), idd.cpu().numpy()
+    Qf, Kf, Vf = Q.float(), K.float(), V.float()
+    ws = torch.empty(seer.sparse_attn_tf32_workspace_size(w.B, w.Hq, w.Hkv, w.n, w.d), dtype=torch.uint8,
+                     device="cuda")
+    O, lse = seer.seer_sparse_attn_tf32(Qf.cuda(), Kf.cuda(), Vf.cuda(), cd, idd, workspace=ws)
+    assert seer.seer_workspace_status(ws) == 0
+    units = sample_units(w.B, w.Hq, w.nb, 12, seed=128)
+    O_u, lse_u = oracle.sparse_attn_units(Qf, Kf, Vf, c, ix, units)
+    Of = O.cpu().double().numpy().reshape(-1, 64, w.d)
+    lf = lse.cpu().double().numpy().reshape(-1, 64)
+    cf = c.reshape(-1)
+    ixf = ix.reshape(-1, ix.shape[-1])
+    for k, u in enumerate(units):
+        bh, i = divmod(int(u), w.nb)
+        b, hq = divmod(bh, w.Hq)
+        blocks = ixf[u, :cf[u]]
+        keys = torch.from_numpy((blocks[:, None] * 64 + np.arange(64)[None, :]).reshape(-1))
+        O_MAX, LSE_MAX = _unit_bounds(Qf, Kf, Vf, b, hq, hq // w.G, i, keys)
+        assert np.abs(Of[u] - O_u[k]).max() <= O_MAX, (u, np.abs(Of[u] - O_u[k]).max(), O_MAX)
+        assert np.abs(lf[u] - lse_u[k]).max() <= LSE_MAX, (u, np.abs(lf[u] - lse_u[k]).max(), LSE_MAX)
