@@ -12,6 +12,9 @@
 //   pool_kernel      Q avg-pool / K [max|min|avg]-pool, one warp per block,
 //                    16-byte vector loads, shuffle reductions; optionally
 //                    writes its result split into tf32 part and remainder
+//   gate_inputs_kernel
+//                    for the tensor-core gate: the Q and K pooling (split)
+//                    and the tf32 split of Wq and Wk in one launch
 //   gemm_nt_kernel   fp32 SIMT tile GEMM: gate projections and the causal
 //                    block logits when h or d is not a multiple of 32;
 //                    gemm_nt128_kernel is its 128 x 128-tile form
@@ -24,8 +27,8 @@
 //                    the causal block logits q~ k~^T / sqrt(d) the same way,
 //                    persistent: each q~ row block is copied into TMEM once
 //                    and the key tiles up to the diagonal stream past it
-//   split_tf32_kernel / split_tf32_copy_kernel
-//                    the tf32 split of the weights (and of q~ / k~ after RoPE)
+//   split_tf32_kernel
+//                    the tf32 split of q~ / k~ after RoPE, in place
 //   rope_kernel      optional block-level RoPE on q~ / k~
 //   row_select_warp4_kernel / row_select_warp_kernel / row_select_kernel
 //                    one warp (many rows of <= 4096 candidates; 16-byte
@@ -366,18 +369,6 @@ __global__ void split_tf32_kernel(float* __restrict__ x, float* __restrict__ lo,
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
     const float hi = __uint_as_float(h);
     x[i] = hi;
-    lo[i] = v - hi;
-  }
-}
-
-__global__ void split_tf32_copy_kernel(const float* __restrict__ x, float* __restrict__ hi_out,
-                                       float* __restrict__ lo, long long n) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const float v = x[i];
-    uint32_t h;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
-    const float hi = __uint_as_float(h);
-    hi_out[i] = hi;
     lo[i] = v - hi;
   }
 }
@@ -927,11 +918,6 @@ cudaError_t launch_gemm_tf32x3_rows(const CUtensorMap& tmAh, const CUtensorMap& 
 
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st) {
   split_tf32_kernel<<<1184, 256, 0, st>>>(x, lo, n);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_split_tf32_copy(const float* x, float* hi, float* lo, long long n, cudaStream_t st) {
-  split_tf32_copy_kernel<<<592, 256, 0, st>>>(x, hi, lo, n);
   return cudaGetLastError();
 }
 

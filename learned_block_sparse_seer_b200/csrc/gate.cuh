@@ -44,8 +44,8 @@ cudaError_t launch_gemm_nt(const float* A, const float* B, float* C, int M, int 
 // (fp32-level accuracy): the gate's causal logits (causal = 1: tiles above
 // the diagonal are skipped) and its projections (causal = 0).  A, B are split
 // first: launch_split_tf32 rounds x to tf32 in place and writes the remainder
-// to lo; launch_split_tf32_copy writes both parts to separate buffers (for
-// inputs the caller owns).  tmAh/tmAl are fp32 maps over A's hi/lo
+// to lo (launch_gate_inputs splits the caller's weights into workspace
+// buffers).  tmAh/tmAl are fp32 maps over A's hi/lo
 // [batch * M rows, K], tmBh/tmBl over B's [(max bz + 1) * N rows, K],
 // 32 x 128 boxes, 128-byte swizzle.  K % 32 == 0.
 struct Tf32x3Params {
@@ -59,7 +59,6 @@ struct Tf32x3Params {
   unsigned long long timeout_ns;
 };
 cudaError_t launch_split_tf32(float* x, float* lo, long long n, cudaStream_t st);
-cudaError_t launch_split_tf32_copy(const float* x, float* hi, float* lo, long long n, cudaStream_t st);
 // tmC / tmClo (used when p.tma_out): 3-D maps over C / C_lo (N columns, M rows,
 // batch; box 32 x 128 x 1, 128-byte swizzle).
 cudaError_t launch_gemm_tf32x3_causal(const CUtensorMap& tmAh, const CUtensorMap& tmAl, const CUtensorMap& tmBh,
