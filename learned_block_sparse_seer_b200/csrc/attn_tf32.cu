@@ -224,9 +224,9 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
                     (int)(krow0 + (long long)j * kBlock), 0);
       }
       // copies in flight land before the CTA exits
-      mbar_wait(&C.q_full, 0, abort_p, nullptr, 20000000ull);
+      wait_landed(&C.q_full, 0);
       for (int k = t > kKS ? t - kKS : 0; k < t; ++k)
-        mbar_wait(&C.k_full[k % kKS], (k / kKS) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&C.k_full[k % kKS], (k / kKS) & 1);
     }
   } else if (warp == kWarpLoadV) {
     // --------------------------------------------------- producer: V^T ---
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
                     (int)(((b * p.Hkv + g) * p.nb + j) * (long long)D), 0);
       }
       for (int k = t > kVS ? t - kVS : 0; k < t; ++k)
-        mbar_wait(&C.v_full[k % kVS], (k / kVS) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&C.v_full[k % kVS], (k / kVS) & 1);
     }
   } else if (warp == kWarpQK) {
     // ----------------------------------------------------- QK issuer ---
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
         mma_commit(&C.k_empty[ks]);
       }
       mma_commit(&C.fin_qk);
-      mbar_wait(&C.fin_qk, 0, abort_p, nullptr, 20000000ull);
+      wait_landed(&C.fin_qk, 0);
     }
   } else if (warp == kWarpPV) {
     // ----------------------------------------------------- PV issuer ---
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(tf32a::kThreads, 1)
         mma_commit(&C.v_empty[vs]);
       }
       mma_commit(&C.fin_pv);
-      mbar_wait(&C.fin_pv, 0, abort_p, nullptr, 20000000ull);
+      wait_landed(&C.fin_pv, 0);
     }
   } else {
     // ------------------------------------------- softmax and epilogue ---

@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
       }
       for (int k = 0; k < 2 && k < u_idx; ++k) {
         const int uu = u_idx - 1 - k;
-        mbar_wait(&C.q_full[uu & 1], (uu >> 1) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&C.q_full[uu & 1], (uu >> 1) & 1);
       }
     }
   } else if (warp == kWarpK) {
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
       }
       for (int k = 0; k < kNK && k < step; ++k) {
         const int st = step - 1 - k;
-        mbar_wait(&C.k_full[st % kNK], (st / kNK) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&C.k_full[st % kNK], (st / kNK) & 1);
       }
     }
   } else if (warp == kWarpMma) {
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(bmax::kThreads, 1)
         ++u_idx;
       }
       mma_commit(&C.fin);
-      mbar_wait(&C.fin, 0, abort_p, nullptr, 20000000ull);
+      wait_landed(&C.fin, 0);
     }
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------ softmax WGs ---

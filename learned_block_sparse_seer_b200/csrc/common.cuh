@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/seer.h"
+#include "ptx.cuh"
 
 namespace seer {
 
@@ -52,6 +53,18 @@ __device__ __forceinline__ T warp_sum(T v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// Bounded wait (timeout_ns of %globaltimer) for a phase whose completion
+// depends on no other warp of the CTA: a bulk copy this thread issued, or
+// the commit of MMAs it issued.  Used before a CTA exits, so it does not give
+// up when the CTA's abort flag is raised: copies and products in flight
+// finish before their shared or tensor memory is released.
+__device__ __forceinline__ bool wait_landed(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = 20000000ull) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  return true;
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(AttnRing<T, D>::THREADS, 2) decode_attn_kernel
       }
       // every issued copy has landed before the CTA may exit
       for (int k = it > NS ? it - NS : 0; k < it; ++k)
-        mbar_wait(&full[k % NS], (k / NS) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&full[k % NS], (k / NS) & 1);
     }
   } else {
     // ------------------------------------------------------ consumers ---
@@ -645,7 +645,7 @@ __global__ void __launch_bounds__(GtRing<T, D>::THREADS, 2) decode_gt_kernel(con
         bulk_load(ring + (size_t)s * R::BLK, Kh + (long long)j * kBlock * D, bytes, &full[s]);
       }
       for (int k = it > NS ? it - NS : 0; k < it; ++k)
-        mbar_wait(&full[k % NS], (k / NS) & 1, abort_p, nullptr, 20000000ull);
+        wait_landed(&full[k % NS], (k / NS) & 1);
     }
   } else {
     // ------------------------------------------------------ consumers ---
