@@ -42,3 +42,44 @@ def test_three_product_split_keeps_fp32_accuracy(read):
     # one tf32 product alone is about three orders of magnitude worse
     one = A @ B.T
     assert (np.abs(one - exact) / scale).max() > 2.0 ** -14
+
+
+def test_tf32_attention_tolerance_covers_tf32_arithmetic():
+    """The tolerances of the tf32 attention parity tests (tests/test_gpu_tf32.py,
+    _bounds) against the arithmetic they describe: Q, K, V and the
+    probabilities P read as tf32 (truncated to 10 mantissa bits), every
+    product and sum exact (fp64), compared with exact fp64 causal attention.
+    The row sums use P before the tensor core reads it, as the kernel's
+    softmax threads do."""
+    import torch
+    from test_gpu_tf32 import _bounds
+
+    rng = np.random.default_rng(3)
+    B, H, n, d = 1, 2, 256, 128
+    Q = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    K = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    V = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    K[:, :, 64:72] *= 3.0  # a few keys well above the rest: peaked rows
+    scale = 1.0 / np.sqrt(d)
+    causal = np.tril(np.ones((n, n), dtype=bool))
+
+    def attn(q, k, v, read_p):
+        s = np.where(causal, (q @ np.swapaxes(k, -1, -2)) * scale, -np.inf)
+        m = s.max(-1, keepdims=True)
+        p = np.exp(s - m)
+        lsum = p.sum(-1, keepdims=True)
+        o = (read_p(p) @ v) / lsum
+        return o, (m + np.log(lsum))[..., 0]
+
+    def t(x):
+        return _tf32_trunc(x.astype(np.float32)).astype(np.float64)
+
+    f64 = [x.astype(np.float64) for x in (Q, K, V)]
+    O_ex, L_ex = attn(*f64, lambda p: p)
+    O_tf, L_tf = attn(t(Q), t(K), t(V), t)
+    O_MAX, O_MEAN, LSE_MAX = _bounds(torch.from_numpy(Q), torch.from_numpy(K), torch.from_numpy(V))
+    eo, el = np.abs(O_tf - O_ex), np.abs(L_tf - L_ex)
+    assert eo.max() <= O_MAX and eo.mean() <= O_MEAN, (eo.max(), eo.mean(), O_MAX)
+    assert el.max() <= LSE_MAX, (el.max(), LSE_MAX)
+    # and the arithmetic does move the result: the bound is not vacuous
+    assert eo.max() > O_MAX / 1000
