@@ -83,3 +83,38 @@ def test_tf32_attention_tolerance_covers_tf32_arithmetic():
     assert el.max() <= LSE_MAX, (el.max(), LSE_MAX)
     # and the arithmetic does move the result: the bound is not vacuous
     assert eo.max() > O_MAX / 1000
+
+
+def test_bf16_attention_tolerance_covers_bf16_rounding():
+    """The fixed O tolerances of the bf16 attention parity tests
+    (tests/gpu_common.py) against the rounding the path adds on bf16 inputs:
+    P rounded to bf16 for the PV product, the row sums taken before that
+    rounding, O rounded to bf16 on output; a layer-structured bf16 case with
+    the oracle gate's density-0.3 lists, against the fp64 oracle."""
+    import torch
+    import oracle
+    from gpu_common import O_MAX, O_MEAN
+    from learned_block_sparse_seer_b200 import synth
+
+    w = synth.Workload("t", 1, 4, 1, 2048, 128, 128, "bf16", "layer", 7)
+    Q, K, V = synth.make_qkv(w)
+    Wq, Wk = synth.make_gate_weights(w)
+    c, ix, _ = oracle.select(oracle.gate(Q, K, Wq, Wk), oracle.MODE_TOPK_DENSITY, density=0.3)
+    O_ref, _ = oracle.sparse_attn(Q, K, V, c, ix)
+
+    def bf16(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).float().to(torch.bfloat16).double().numpy()
+
+    q, k, v = (t.double().numpy() for t in (Q, K, V))
+    O = np.empty_like(O_ref)
+    for h in range(w.Hq):
+        g = h // w.G
+        for i in range(w.nb):
+            keys = (ix[0, h, i, :c[0, h, i]][:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+            s = (q[0, h, 64 * i:64 * i + 64] @ k[0, g, keys].T) / np.sqrt(w.d)
+            s = np.where(keys[None, :] <= 64 * i + np.arange(64)[:, None], s, -np.inf)
+            p = np.exp(s - s.max(-1, keepdims=True))
+            O[0, h, 64 * i:64 * i + 64] = bf16((bf16(p) @ v[0, g, keys]) / p.sum(-1, keepdims=True))
+    e = np.abs(O - O_ref)
+    assert e.max() <= O_MAX and e.mean() <= O_MEAN, (e.max(), e.mean())
+    assert e.max() > O_MAX / 100  # the rounding is visible against the bound
